@@ -1,0 +1,119 @@
+"""Seeded synthetic inputs for the CGTP convolution.
+
+This module is the one piece shared by the CUDA path and the FP64 oracle.  It
+holds none of the method's arithmetic: it builds atom positions and draws
+random arrays of the shapes the caller asks for, nothing else.
+
+Recipe (the workloads of the LunaTP pages, arXiv 2610.18393):
+  * structure: silicon in the diamond structure, lattice constant 5.43 A
+    (Fig. 6, MD on Si), 8 atoms per conventional cell -- the fcc points
+    {0, (0,1/2,1/2), (1/2,0,1/2), (1/2,1/2,0)} and the same shifted by
+    (1/4,1/4,1/4) -- replicated nx x ny x nz, orthorhombic periodic box;
+  * isotropic Gaussian jitter sigma per coordinate, FP64, then wrapped into
+    [0, box);
+  * irreps per workload from Table 1 (Cases 1-3), the 768-atom, Lmax = 6,
+    64-channels-per-degree shape of Fig. 1, and a tiny Lmax = 1 case;
+  * x ~ N(0,1), g ~ N(0,1), W ~ N(0, var) with var = 1 / (number of paths
+    feeding the output irrep of the column), all drawn in FP64 and rounded
+    to FP32 so that both sides read identical FP32 values;
+  * random streams: numpy default_rng([seed, stream]) with stream 0 for the
+    jitter, 1 for x, 2 for W, 3 for g.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+SI_A = 5.43
+
+_DIAMOND_BASIS = np.array(
+    [[0.0, 0.0, 0.0], [0.0, 0.5, 0.5], [0.5, 0.0, 0.5], [0.5, 0.5, 0.0],
+     [0.25, 0.25, 0.25], [0.25, 0.75, 0.75], [0.75, 0.25, 0.75], [0.75, 0.75, 0.25]])
+
+_L6_IN = "+".join(f"64x{l}{'e' if l % 2 == 0 else 'o'}" for l in range(7))
+_L6_EDGE = "+".join(f"1x{l}{'e' if l % 2 == 0 else 'o'}" for l in range(7))
+
+# name -> workload.  ``metric_config`` marks the one the headline number is
+# quoted on; the others are parity cases and secondary bench lines.
+CONFIGS = {
+    "tiny": dict(
+        desc="64 Si atoms, 2x2x2 cells, rc 5.0, Lmax 1",
+        cells=(2, 2, 2), sigma=0.05, rc=5.0,
+        irreps_in="16x0e+16x1o", irreps_edge="1x0e+1x1o", irreps_out="32x0e+32x1o"),
+    "lmax2": dict(
+        desc="768 Si atoms, 4x4x6 cells, rc 5.0, Lmax 2 (Table 1 Case 1)",
+        cells=(4, 4, 6), sigma=0.05, rc=5.0,
+        irreps_in="128x0e+64x1e+32x2e", irreps_edge="1x0e+1x1e+1x2e",
+        irreps_out="224x0e+384x1e+352x2e", metric_config=True),
+    "lmax2_wide": dict(
+        desc="768 Si atoms, 4x4x6 cells, rc 6.0, Lmax 2 wide (Table 1 Case 2)",
+        cells=(4, 4, 6), sigma=0.05, rc=6.0,
+        irreps_in="128x0e+128x1o+128x2e", irreps_edge="1x0e+1x1o+1x2e+1x3o",
+        irreps_out="384x0e+640x1o+640x2e+512x3o"),
+    "lmax3": dict(
+        desc="6144 Si atoms, 8x8x12 cells, sigma 0.1, rc 5.0, Lmax 3 (Table 1 Case 3)",
+        cells=(8, 8, 12), sigma=0.1, rc=5.0,
+        irreps_in="128x0e+64x1o+32x2e+32x3o", irreps_edge="1x0e+1x1o+1x2e+1x3o",
+        irreps_out="256x0e+352x1o+384x2e+320x3o"),
+    "lmax6": dict(
+        desc="768 Si atoms, 4x4x6 cells, rc 5.0, Lmax 6, 64 channels per degree (Fig. 1)",
+        cells=(4, 4, 6), sigma=0.05, rc=5.0,
+        irreps_in=_L6_IN, irreps_edge=_L6_EDGE,
+        irreps_out="448x0e+768x1o+1024x2e+1152x3o+1216x4e+1152x5o+1024x6e"),
+}
+
+
+def rng(seed: int, stream: int) -> np.random.Generator:
+    return np.random.default_rng([int(seed), int(stream)])
+
+
+def si_diamond(cells, sigma: float, seed: int = 0, a: float = SI_A):
+    """Jittered periodic Si diamond supercell.
+
+    Returns (pos float64 [N,3] in [0, box), box float64 [3])."""
+    nx, ny, nz = (int(c) for c in cells)
+    idx = np.stack(np.meshgrid(np.arange(nx), np.arange(ny), np.arange(nz), indexing="ij"),
+                   axis=-1).reshape(-1, 3).astype(np.float64)
+    frac = (idx[:, None, :] + _DIAMOND_BASIS[None, :, :]).reshape(-1, 3)
+    pos = frac * a
+    box = np.array([nx * a, ny * a, nz * a], dtype=np.float64)
+    if sigma > 0:
+        pos = pos + rng(seed, 0).normal(0.0, sigma, size=pos.shape)
+    pos = np.mod(pos, box)
+    pos = np.where(pos >= box, pos - box, pos)
+    return np.ascontiguousarray(pos), box
+
+
+def normal_f32(shape, seed: int, stream: int, std=None, chunk_rows: int = 4096) -> np.ndarray:
+    """N(0, std^2) in FP64, rounded to FP32, drawn row-chunk by row-chunk.
+
+    ``std`` is a scalar or a per-column vector (broadcast over rows)."""
+    shape = tuple(int(s) for s in shape)
+    out = np.empty(shape, dtype=np.float32)
+    g = rng(seed, stream)
+    rows = shape[0] if shape else 1
+    std = None if std is None else np.asarray(std, dtype=np.float64)
+    for r0 in range(0, rows, chunk_rows):
+        r1 = min(rows, r0 + chunk_rows)
+        v = g.standard_normal((r1 - r0,) + shape[1:])
+        if std is not None:
+            v = v * std
+        out[r0:r1] = v
+    return out
+
+
+def column_std(out_muls, fan_in) -> np.ndarray:
+    """Per-column std of W from per-output-block fan-ins: 1/sqrt(fan_in)."""
+    cols = [np.full(int(m), 1.0 / np.sqrt(max(int(f), 1))) for m, f in zip(out_muls, fan_in)]
+    return np.concatenate(cols) if cols else np.zeros(0)
+
+
+def draw_x(n: int, d_in: int, seed: int = 0) -> np.ndarray:
+    return normal_f32((n, d_in), seed, 1)
+
+
+def draw_W(E: int, U: int, col_std, seed: int = 0) -> np.ndarray:
+    return normal_f32((E, U), seed, 2, std=col_std)
+
+
+def draw_g(n: int, d_out: int, seed: int = 0) -> np.ndarray:
+    return normal_f32((n, d_out), seed, 3)
