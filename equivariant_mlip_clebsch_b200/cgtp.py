@@ -1,0 +1,243 @@
+"""Python binding of libcgtp (include/cgtp.h): argument marshalling only.
+
+Every step of the convolution runs in the library's CUDA kernels; torch is used
+for device memory and the current stream.  There is no fallback: if the
+library is missing this module raises on import.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+if os.environ.setdefault("CGTP_JIT_CACHE", os.path.join(_PKG, "_jit_cache")):
+    os.makedirs(os.environ["CGTP_JIT_CACHE"], exist_ok=True)
+
+if not os.path.exists(_build.LIB):
+    raise ImportError(f"{_build.LIB} is not built; run equivariant_mlip_clebsch_b200.build.build()")
+
+_lib = ctypes.CDLL(_build.LIB)
+
+_P, _i, _i64, _d, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_size_t
+_pi64 = ctypes.POINTER(ctypes.c_int64)
+
+_SIGS = {
+    "cgtp_status_string": (ctypes.c_char_p, [_i]),
+    "cgtp_last_error": (ctypes.c_char_p, []),
+    "cgtp_plan_create": (_i, [ctypes.c_char_p, ctypes.c_char_p, ctypes.c_char_p, _i,
+                              ctypes.POINTER(_P)]),
+    "cgtp_plan_destroy": (_i, [_P]),
+    "cgtp_plan_info": (_i, [_P, _pi64, _pi64, _pi64, _pi64, _pi64]),
+    "cgtp_plan_paths": (_i, [_P, _P]),
+    "cgtp_plan_coefficients": (_i, [_P, _P, _pi64]),
+    "cgtp_plan_describe": (_i, [_P, ctypes.c_char_p, _sz, ctypes.POINTER(_sz)]),
+    "cgtp_real_cg": (_i, [_i, _i, _i, _P]),
+    "cgtp_sph_harm": (_i, [_P, _i64, _P, _P, _P]),
+    "cgtp_forward": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P, _P, _P]),
+    "cgtp_backward_workspace_size": (_i, [_P, _i64, _i64, _i64, ctypes.POINTER(_sz)]),
+    "cgtp_backward": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                           _P, _sz, _P]),
+    "cgtp_plan_check_device_error": (_i, [_P, ctypes.POINTER(_i)]),
+    "cgtp_plan_set_timing": (_i, [_P, _i]),
+    "cgtp_plan_kernel_times": (_i, [_P, _i, ctypes.c_char_p, _P, _P, ctypes.POINTER(_i)]),
+    "cgtp_neighbor_list": (_i, [_i64, _P, _P, _d, _P, _P, _P, _P, _pi64]),
+    "cgtp_csr_transpose": (_i, [_i64, _i64, _i64, _P, _P, _P, _P]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTS = tuple(_SIGS)
+
+
+class CgtpError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+
+
+def _check(st: int) -> None:
+    if st != 0:
+        raise CgtpError(st, _lib.cgtp_last_error().decode())
+
+
+def _np_ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _tptr(t):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("expected a contiguous CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def real_cg(l1: int, l2: int, l3: int) -> np.ndarray:
+    C = np.zeros((2 * l1 + 1, 2 * l2 + 1, 2 * l3 + 1), dtype=np.float64)
+    _check(_lib.cgtp_real_cg(l1, l2, l3, _np_ptr(C)))
+    return C
+
+
+def neighbor_list(pos, box, rc: float):
+    """Cell-list neighbour list (host).  Returns rowptr, col, shift (int32)
+    and the FP32 edge vectors r = pos_j + n*box - pos_i."""
+    pos = np.ascontiguousarray(pos, dtype=np.float64)
+    box = np.ascontiguousarray(box, dtype=np.float64)
+    N = pos.shape[0]
+    rowptr = np.zeros(N + 1, dtype=np.int32)
+    E = ctypes.c_int64(0)
+    _check(_lib.cgtp_neighbor_list(N, _np_ptr(pos), _np_ptr(box), float(rc), _np_ptr(rowptr),
+                                   None, None, None, ctypes.byref(E)))
+    col = np.zeros(E.value, dtype=np.int32)
+    shift = np.zeros((E.value, 3), dtype=np.int32)
+    r = np.zeros((E.value, 3), dtype=np.float32)
+    _check(_lib.cgtp_neighbor_list(N, _np_ptr(pos), _np_ptr(box), float(rc), _np_ptr(rowptr),
+                                   _np_ptr(col), _np_ptr(shift), _np_ptr(r), ctypes.byref(E)))
+    return rowptr, col, shift, r
+
+
+def csr_transpose(rowptr, col, n_send: int):
+    rowptr = np.ascontiguousarray(rowptr, dtype=np.int32)
+    col = np.ascontiguousarray(col, dtype=np.int32)
+    n_recv, E = rowptr.shape[0] - 1, col.shape[0]
+    rowptr_T = np.zeros(n_send + 1, dtype=np.int32)
+    perm_T = np.zeros(max(E, 1), dtype=np.int32)
+    _check(_lib.cgtp_csr_transpose(n_recv, n_send, E, _np_ptr(rowptr), _np_ptr(col),
+                                   _np_ptr(rowptr_T), _np_ptr(perm_T)))
+    return rowptr_T, perm_T[:E]
+
+
+class Plan:
+    """A CGTP plan: irreps, paths, CG tables and the compiled kernels."""
+
+    def __init__(self, irreps_in: str, irreps_edge: str, irreps_out: str, lmax: int | None = None):
+        if lmax is None:
+            lmax = 6
+        h = ctypes.c_void_p()
+        _check(_lib.cgtp_plan_create(irreps_in.encode(), irreps_edge.encode(), irreps_out.encode(),
+                                     int(lmax), ctypes.byref(h)))
+        self._h = h
+        self.irreps_in, self.irreps_edge, self.irreps_out = irreps_in, irreps_edge, irreps_out
+        v = [ctypes.c_int64() for _ in range(5)]
+        _check(_lib.cgtp_plan_info(h, *[ctypes.byref(t) for t in v]))
+        self.d_in, self.d_edge, self.d_out, self.n_weights, self.n_paths = (t.value for t in v)
+        self.L = int(round(self.d_edge ** 0.5)) - 1
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib.cgtp_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ---- host introspection
+    def paths(self) -> np.ndarray:
+        t = np.zeros((self.n_paths, 8), dtype=np.int32)
+        if self.n_paths:
+            _check(_lib.cgtp_plan_paths(self._h, _np_ptr(t)))
+        return t
+
+    def coefficients(self) -> np.ndarray:
+        n = ctypes.c_int64()
+        _check(_lib.cgtp_plan_coefficients(self._h, None, ctypes.byref(n)))
+        c = np.zeros(n.value, dtype=np.float64)
+        _check(_lib.cgtp_plan_coefficients(self._h, _np_ptr(c), ctypes.byref(n)))
+        return c
+
+    def describe(self) -> str:
+        need = ctypes.c_size_t()
+        _check(_lib.cgtp_plan_describe(self._h, None, 0, ctypes.byref(need)))
+        buf = ctypes.create_string_buffer(need.value)
+        _check(_lib.cgtp_plan_describe(self._h, buf, need.value, ctypes.byref(need)))
+        return buf.value.decode()
+
+    def out_fan_in(self) -> list:
+        """Number of paths feeding each output irrep block (in order)."""
+        muls = [int(tok.split("x")[0]) for tok in self.irreps_out.split("+")]
+        base = np.concatenate([[0], np.cumsum(muls)])
+        fan = [0] * len(muls)
+        for k0 in self.paths()[:, 5]:
+            fan[int(np.searchsorted(base, k0, side="right")) - 1] += 1
+        return fan
+
+    def check_device_error(self) -> None:
+        code = ctypes.c_int()
+        _check(_lib.cgtp_plan_check_device_error(self._h, ctypes.byref(code)))
+
+    def set_timing(self, enable: bool) -> None:
+        _check(_lib.cgtp_plan_set_timing(self._h, int(bool(enable))))
+
+    def kernel_times(self) -> dict:
+        """{kernel name: (total ms, launches)} since the previous call."""
+        mx = 16
+        names = ctypes.create_string_buffer(32 * mx)
+        ms = np.zeros(mx, dtype=np.float64)
+        cnt = np.zeros(mx, dtype=np.int64)
+        n = ctypes.c_int()
+        _check(_lib.cgtp_plan_kernel_times(self._h, mx, names, _np_ptr(ms), _np_ptr(cnt), ctypes.byref(n)))
+        out = {}
+        for k in range(min(n.value, mx)):
+            nm = names.raw[32 * k:32 * (k + 1)].split(b"\0", 1)[0].decode()
+            out[nm] = (float(ms[k]), int(cnt[k]))
+        return out
+
+    # ---- device calls
+    def sph_harm(self, r, Y=None, stream=None):
+        import torch
+        E = r.shape[0]
+        if Y is None:
+            Y = torch.empty((E, self.d_edge), dtype=torch.float32, device=r.device)
+        _check(_lib.cgtp_sph_harm(self._h, E, _tptr(r), _tptr(Y), _stream(stream)))
+        return Y
+
+    def forward(self, rowptr, col, x, Y, W, out=None, stream=None):
+        import torch
+        n_recv = rowptr.shape[0] - 1
+        if out is None:
+            out = torch.empty((n_recv, self.d_out), dtype=torch.float32, device=x.device)
+        _check(_lib.cgtp_forward(self._h, n_recv, x.shape[0], col.shape[0], _tptr(rowptr),
+                                 _tptr(col), _tptr(x), _tptr(Y), _tptr(W), _tptr(out),
+                                 _stream(stream)))
+        return out
+
+    def workspace_size(self, n_recv: int, n_send: int, E: int) -> int:
+        b = ctypes.c_size_t()
+        _check(_lib.cgtp_backward_workspace_size(self._h, n_recv, n_send, E, ctypes.byref(b)))
+        return b.value
+
+    def backward(self, rowptr, col, rowptr_T, perm_T, x, Y, W, grad_out, want=("x", "W", "Y"),
+                 grads=None, workspace=None, stream=None):
+        import torch
+        n_recv, n_send, E = rowptr.shape[0] - 1, x.shape[0], col.shape[0]
+        dev = x.device
+        if grads is None:
+            dx = torch.empty((n_send, self.d_in), dtype=torch.float32, device=dev) if "x" in want else None
+            dW = torch.empty((E, self.n_weights), dtype=torch.float32, device=dev) if "W" in want else None
+            dY = torch.empty((E, self.d_edge), dtype=torch.float32, device=dev) if "Y" in want else None
+        else:
+            dx, dW, dY = grads
+        nbytes = self.workspace_size(n_recv, n_send, E)
+        if workspace is None:
+            workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        _check(_lib.cgtp_backward(self._h, n_recv, n_send, E, _tptr(rowptr), _tptr(col),
+                                  _tptr(rowptr_T), _tptr(perm_T), _tptr(x), _tptr(Y), _tptr(W),
+                                  _tptr(grad_out), _tptr(dx), _tptr(dW), _tptr(dY),
+                                  _tptr(workspace), workspace.numel(), _stream(stream)))
+        return dx, dW, dY

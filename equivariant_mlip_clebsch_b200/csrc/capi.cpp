@@ -1,0 +1,460 @@
+// capi.cpp -- the extern "C" surface of libcgtp (declared in include/cgtp.h).
+// Argument marshalling and validation only; the work runs in the kernels.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "internal.hpp"
+
+namespace cgtp {
+
+static thread_local std::string t_err = "no error";
+
+void set_error(const std::string& msg) { t_err = msg; }
+
+cgtp_status fail(cgtp_status s, const std::string& msg) {
+  t_err = std::string(cgtp_status_string(s)) + ": " + msg;
+  return s;
+}
+
+cgtp_status neighbor_list_impl(int64_t, const double*, const double*, double, int32_t*, int32_t*,
+                               int32_t*, float*, int64_t*);
+cgtp_status csr_transpose_impl(int64_t, int64_t, int64_t, const int32_t*, const int32_t*, int32_t*,
+                               int32_t*);
+
+void destroy_plan_device(Plan& P) {
+  for (auto& t : P.tlog) {
+    cudaEventDestroy(t.a);
+    cudaEventDestroy(t.b);
+  }
+  for (auto e : P.tpool) cudaEventDestroy(e);
+  P.tlog.clear();
+  P.tpool.clear();
+  jit_unload(P.fwd);
+  jit_unload(P.bwd);
+  for (void** p : {&P.d_fwd_ent, &P.d_fwd_term, &P.d_bwd_ent, &P.d_bwd_term}) {
+    if (*p) cudaFree(*p);
+    *p = nullptr;
+  }
+  if (P.d_err) cudaFree(P.d_err);
+  P.d_err = nullptr;
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+static cgtp_status check_device(const Plan& P) {
+  int dev = -1;
+  CGTP_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev != P.device)
+    return fail(CGTP_ERR_CUDA, "plan was created on device " + std::to_string(P.device) +
+                                   " but device " + std::to_string(dev) + " is current");
+  if (P.host_only) return fail(CGTP_ERR_CUDA, "plan was built without a device (compile-only)");
+  return CGTP_OK;
+}
+
+static const char* kKindName[] = {"sph_harm", "cgtp_fwd", "cgtp_bwd", "bwd_dx_rows", "bwd_dy_slices",
+                                   "zero_fill"};
+
+// Brackets one internal launch with events when timing is on.
+struct TimedScope {
+  Plan& P;
+  int kind;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr, b = nullptr;
+  static cudaEvent_t take(Plan& P) {
+    if (!P.tpool.empty()) {
+      cudaEvent_t e = P.tpool.back();
+      P.tpool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+  TimedScope(Plan& P_, int k, cudaStream_t st) : P(P_), kind(k), s(st) {
+    if (!P.timing) return;
+    std::lock_guard<std::mutex> g(P.tmu);
+    a = take(P);
+    b = take(P);
+    if (a) cudaEventRecord(a, s);
+  }
+  ~TimedScope() {
+    if (!a || !b) return;
+    cudaEventRecord(b, s);
+    std::lock_guard<std::mutex> g(P.tmu);
+    P.tlog.push_back({kind, a, b});
+  }
+};
+
+}  // namespace cgtp
+
+using namespace cgtp;
+
+extern "C" {
+
+const char* cgtp_status_string(cgtp_status s) {
+  switch (s) {
+    case CGTP_OK: return "CGTP_OK";
+    case CGTP_ERR_NULL: return "CGTP_ERR_NULL";
+    case CGTP_ERR_ALIGN: return "CGTP_ERR_ALIGN";
+    case CGTP_ERR_IRREPS_PARSE: return "CGTP_ERR_IRREPS_PARSE";
+    case CGTP_ERR_IRREPS_MISMATCH: return "CGTP_ERR_IRREPS_MISMATCH";
+    case CGTP_ERR_LMAX: return "CGTP_ERR_LMAX";
+    case CGTP_ERR_SIZE: return "CGTP_ERR_SIZE";
+    case CGTP_ERR_INVALID_CSR: return "CGTP_ERR_INVALID_CSR";
+    case CGTP_ERR_CUDA: return "CGTP_ERR_CUDA";
+    case CGTP_ERR_OOM: return "CGTP_ERR_OOM";
+    case CGTP_ERR_TIMEOUT: return "CGTP_ERR_TIMEOUT";
+    case CGTP_ERR_JIT: return "CGTP_ERR_JIT";
+    case CGTP_ERR_WORKSPACE: return "CGTP_ERR_WORKSPACE";
+  }
+  return "CGTP_ERR_UNKNOWN";
+}
+
+const char* cgtp_last_error(void) { return t_err.c_str(); }
+
+cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge, const char* irreps_out,
+                             int lmax, cgtp_plan* out) {
+  if (!out) return fail(CGTP_ERR_NULL, "out is NULL");
+  *out = nullptr;
+  if (!irreps_in || !irreps_edge || !irreps_out) return fail(CGTP_ERR_NULL, "irreps string is NULL");
+  std::unique_ptr<Plan> P;
+  try {
+    P.reset(new Plan());
+  } catch (...) {
+    return fail(CGTP_ERR_OOM, "host allocation failed");
+  }
+  P->irreps_in_s = irreps_in;
+  P->irreps_edge_s = irreps_edge;
+  P->irreps_out_s = irreps_out;
+  P->lmax = lmax;
+  cgtp_status st;
+  try {
+    st = build_paths(*P);
+    if (st != CGTP_OK) return st;
+    P->host_only = std::getenv("CGTP_JIT_COMPILE_ONLY") != nullptr;
+    if (!P->host_only) {
+      CGTP_CUDA_TRY(cudaGetDevice(&P->device));
+      CGTP_CUDA_TRY(cudaFree(0));  // make the primary context current
+      if (cudaMalloc(&P->d_err, sizeof(int)) != cudaSuccess) return fail(CGTP_ERR_OOM, "cudaMalloc");
+      CGTP_CUDA_TRY(cudaMemset(P->d_err, 0, sizeof(int)));
+    }
+    st = build_forward(*P);
+    if (st == CGTP_OK) st = build_backward(*P);
+  } catch (const std::exception& e) {
+    destroy_plan_device(*P);
+    return fail(CGTP_ERR_OOM, std::string("exception in plan create: ") + e.what());
+  }
+  if (st != CGTP_OK) {
+    destroy_plan_device(*P);
+    return st;
+  }
+  *out = reinterpret_cast<cgtp_plan>(P.release());
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_destroy(cgtp_plan plan) {
+  if (!plan) return CGTP_OK;
+  Plan* P = reinterpret_cast<Plan*>(plan);
+  destroy_plan_device(*P);
+  delete P;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_info(cgtp_plan plan, int64_t* d_in, int64_t* d_edge, int64_t* d_out,
+                           int64_t* n_weights, int64_t* n_paths) {
+  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
+  const Plan* P = reinterpret_cast<const Plan*>(plan);
+  if (d_in) *d_in = P->D_in;
+  if (d_edge) *d_edge = P->D_e;
+  if (d_out) *d_out = P->D_out;
+  if (n_weights) *n_weights = P->U;
+  if (n_paths) *n_paths = (int64_t)P->paths.size();
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_paths(cgtp_plan plan, int32_t* table) {
+  if (!plan || !table) return fail(CGTP_ERR_NULL, "null argument");
+  const Plan* P = reinterpret_cast<const Plan*>(plan);
+  for (size_t k = 0; k < P->paths.size(); ++k) {
+    const Path& p = P->paths[k];
+    const int32_t row[8] = {p.l1, p.l2, p.l3, p.mul, p.x_off, p.k0, p.o_off, p.c_off};
+    std::memcpy(table + 8 * k, row, sizeof row);
+  }
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_coefficients(cgtp_plan plan, double* coeff, int64_t* n_coeff) {
+  if (!plan || !n_coeff) return fail(CGTP_ERR_NULL, "null argument");
+  const Plan* P = reinterpret_cast<const Plan*>(plan);
+  *n_coeff = (int64_t)P->coeff.size();
+  if (coeff) std::memcpy(coeff, P->coeff.data(), P->coeff.size() * sizeof(double));
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_real_cg(int l1, int l2, int l3, double* C) {
+  if (!C) return fail(CGTP_ERR_NULL, "C is NULL");
+  if (l1 < 0 || l2 < 0 || l1 > 12 || l2 > 12) return fail(CGTP_ERR_LMAX, "degrees must be in 0..12");
+  std::vector<double> v;
+  if (!real_cg_block(l1, l2, l3, v)) return fail(CGTP_ERR_SIZE, "triangle rule violated");
+  std::memcpy(C, v.data(), v.size() * sizeof(double));
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_sph_harm(cgtp_plan plan, int64_t E, const float* r, float* Y, cgtp_stream stream) {
+  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
+  const Plan* P = reinterpret_cast<const Plan*>(plan);
+  if (E < 0 || E >= (int64_t(1) << 31)) return fail(CGTP_ERR_SIZE, "E out of range");
+  if (E == 0) return CGTP_OK;
+  if (!r || !Y) return fail(CGTP_ERR_NULL, "r or Y is NULL");
+  if (!aligned16(r) || !aligned16(Y)) return fail(CGTP_ERR_ALIGN, "r and Y must be 16-byte aligned");
+  cgtp_status st = check_device(*P);
+  if (st != CGTP_OK) return st;
+  {
+    TimedScope ts(*const_cast<Plan*>(P), 0, (cudaStream_t)stream);
+    CGTP_CUDA_TRY(launch_sph_harm(P->L, E, r, Y, (cudaStream_t)stream));
+  }
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_forward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                         const int32_t* rowptr, const int32_t* col, const float* x, const float* Y,
+                         const float* W, float* out, cgtp_stream stream) {
+  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
+  Plan* P = reinterpret_cast<Plan*>(plan);
+  if (n_recv < 0 || n_send < 0 || E < 0 || n_recv >= (int64_t(1) << 31) ||
+      n_send >= (int64_t(1) << 31) || E >= (int64_t(1) << 31) - 1)
+    return fail(CGTP_ERR_SIZE, "sizes out of range");
+  if (n_recv == 0) return CGTP_OK;
+  if (!rowptr || !out) return fail(CGTP_ERR_NULL, "rowptr or out is NULL");
+  if (E > 0 && (!col || !Y || !W || !x)) return fail(CGTP_ERR_NULL, "col, x, Y or W is NULL");
+  if (E > 0 && n_send == 0) return fail(CGTP_ERR_SIZE, "edges without senders");
+  for (const void* p : {(const void*)x, (const void*)Y, (const void*)W, (const void*)out})
+    if (p && !aligned16(p)) return fail(CGTP_ERR_ALIGN, "float arrays must be 16-byte aligned");
+  cgtp_status st = check_device(*P);
+  if (st != CGTP_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (P->fwd_roles.empty()) {
+    CGTP_CUDA_TRY(cudaMemsetAsync(out, 0, (size_t)n_recv * P->D_out * sizeof(float), s));
+    return CGTP_OK;
+  }
+  void* args[] = {&rowptr, &col, &x, &Y, &W, &out, &P->d_fwd_ent, &P->d_fwd_term, &P->d_err};
+  TimedScope ts(*P, 1, s);
+  return jit_launch(P->fwd, dim3((unsigned)n_recv, (unsigned)P->fcfg.S), args, s);
+}
+
+cgtp_status cgtp_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                                         size_t* bytes) {
+  if (!plan || !bytes) return fail(CGTP_ERR_NULL, "null argument");
+  const Plan* P = reinterpret_cast<const Plan*>(plan);
+  if (n_recv < 0 || n_send < 0 || E < 0) return fail(CGTP_ERR_SIZE, "negative size");
+  auto r256 = [](size_t v) { return (v + 255) & ~size_t(255); };
+  size_t b = r256((size_t)E * P->D_in * sizeof(float));
+  if (P->bcfg.S > 1) b += r256((size_t)P->bcfg.S * E * P->D_e * sizeof(float));
+  *bytes = b;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                          const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
+                          const int32_t* perm_T, const float* x, const float* Y, const float* W,
+                          const float* grad_out, float* grad_x, float* grad_W, float* grad_Y,
+                          void* workspace, size_t workspace_bytes, cgtp_stream stream) {
+  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
+  Plan* P = reinterpret_cast<Plan*>(plan);
+  if (n_recv < 0 || n_send < 0 || E < 0 || n_recv >= (int64_t(1) << 31) ||
+      n_send >= (int64_t(1) << 31) || E >= (int64_t(1) << 31) - 1)
+    return fail(CGTP_ERR_SIZE, "sizes out of range");
+  cudaStream_t s = (cudaStream_t)stream;
+  cgtp_status st = check_device(*P);
+  if (st != CGTP_OK) return st;
+  for (const void* p : {(const void*)x, (const void*)Y, (const void*)W, (const void*)grad_out,
+                        (const void*)grad_x, (const void*)grad_W, (const void*)grad_Y})
+    if (p && !aligned16(p)) return fail(CGTP_ERR_ALIGN, "float arrays must be 16-byte aligned");
+  if (grad_x && n_send > 0 && (E == 0 || P->bwd_roles.empty()))
+    CGTP_CUDA_TRY(cudaMemsetAsync(grad_x, 0, (size_t)n_send * P->D_in * sizeof(float), s));
+  if (E == 0) return CGTP_OK;
+  if (!rowptr || !col || !x || !Y || !W || !grad_out)
+    return fail(CGTP_ERR_NULL, "rowptr, col, x, Y, W or grad_out is NULL");
+  if (grad_x && (!rowptr_T || !perm_T)) return fail(CGTP_ERR_NULL, "grad_x needs rowptr_T and perm_T");
+  if (P->bwd_roles.empty()) {
+    if (grad_W) CGTP_CUDA_TRY(cudaMemsetAsync(grad_W, 0, (size_t)E * P->U * sizeof(float), s));
+    if (grad_Y) CGTP_CUDA_TRY(cudaMemsetAsync(grad_Y, 0, (size_t)E * P->D_e * sizeof(float), s));
+    return CGTP_OK;
+  }
+  size_t need = 0;
+  cgtp_backward_workspace_size(plan, n_recv, n_send, E, &need);
+  const bool need_ws = grad_x || (grad_Y && P->bcfg.S > 1);
+  if (need_ws && (!workspace || workspace_bytes < need))
+    return fail(CGTP_ERR_WORKSPACE, "workspace of " + std::to_string(need) + " bytes required");
+  if (need_ws && ((uintptr_t)workspace & 255))
+    return fail(CGTP_ERR_ALIGN, "workspace must be 256-byte aligned");
+  auto r256 = [](size_t v) { return (v + 255) & ~size_t(255); };
+  float* m = grad_x ? reinterpret_cast<float*>(workspace) : nullptr;
+  float* dyp = nullptr;
+  if (grad_Y) {
+    dyp = P->bcfg.S > 1 ? reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
+                                                   r256((size_t)E * P->D_in * sizeof(float)))
+                        : grad_Y;
+  }
+  if (m && P->bwd_irrep_gap) {  // hidden irreps without paths receive zero gradient
+    TimedScope ts(*P, 5, s);
+    CGTP_CUDA_TRY(cudaMemsetAsync(m, 0, (size_t)E * P->D_in * sizeof(float), s));
+  }
+  if (n_recv > 0) {
+    void* args[] = {&rowptr, &col,   &x, &Y, &W, &grad_out, &grad_W, &dyp, &m,
+                    &P->d_bwd_ent, &P->d_bwd_term, &P->d_err};
+    TimedScope ts(*P, 2, s);
+    st = jit_launch(P->bwd, dim3((unsigned)n_recv, (unsigned)P->bcfg.S), args, s);
+    if (st != CGTP_OK) return st;
+  }
+  if (grad_Y && P->bcfg.S > 1) {
+    TimedScope ts(*P, 4, s);
+    CGTP_CUDA_TRY(launch_sum_slices(P->bcfg.S, E * P->D_e, dyp, grad_Y, s));
+  }
+  if (grad_x) {
+    TimedScope ts(*P, 3, s);
+    CGTP_CUDA_TRY(launch_segment_rows(n_send, P->D_in, rowptr_T, perm_T, m, grad_x, s));
+  }
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* needed) {
+  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
+  const Plan* P = reinterpret_cast<const Plan*>(plan);
+  std::string t;
+  t += "irreps_in=" + P->irreps_in_s + " irreps_edge=" + P->irreps_edge_s + " irreps_out=" +
+       P->irreps_out_s + "\n";
+  t += "D_in=" + std::to_string(P->D_in) + " D_e=" + std::to_string(P->D_e) + " D_out=" +
+       std::to_string(P->D_out) + " U=" + std::to_string(P->U) + " paths=" +
+       std::to_string(P->paths.size()) + "\n";
+  auto cfg = [&](const char* nm, const FwdConfig& F, const JitKernel& k, size_t nroles) {
+    t += std::string(nm) + ": roles=" + std::to_string(nroles) + " slices=" + std::to_string(F.S) +
+         " warps=" + std::to_string(F.nw) + "+1 chunk=" + std::to_string(F.B) + " stages=" +
+         std::to_string(F.stages) + " w_smem=" + std::to_string((int)F.w_smem) + " x_smem=" +
+         std::to_string((int)F.x_smem) + " nacc=" + std::to_string(F.nacc) + " smem=" +
+         std::to_string(k.smem) + " threads=" + std::to_string(k.threads);
+    char hx[40];
+    std::snprintf(hx, sizeof hx, " hash=%016llx\n", k.hash);
+    t += hx;
+    for (size_t s = 0; s < F.slice_roles.size(); ++s) {
+      t += "  slice " + std::to_string(s) + ":";
+      for (int r : F.slice_roles[s]) t += " " + std::to_string(r);
+      t += "\n";
+    }
+    t += k.log;
+    if (!k.log.empty() && k.log.back() != '\n') t += "\n";
+  };
+  cfg("forward", P->fcfg, P->fwd, P->fwd_roles.size());
+  for (size_t r = 0; r < P->fwd_roles.size(); ++r) {
+    const FwdRole& q = P->fwd_roles[r];
+    t += "  frole " + std::to_string(r) + ": irrep " + std::to_string(q.irrep) + " u0=" +
+         std::to_string(q.u0) + " R=" + std::to_string(q.R) + " paths=" +
+         std::to_string(q.paths.size()) + " cost=" + std::to_string((int)q.cost) + "\n";
+  }
+  cfg("backward", P->bcfg, P->bwd, P->bwd_roles.size());
+  for (size_t r = 0; r < P->bwd_roles.size(); ++r) {
+    const BwdRole& q = P->bwd_roles[r];
+    t += "  brole " + std::to_string(r) + ": irrep " + std::to_string(q.irrep) + " u0=" +
+         std::to_string(q.u0) + " R=" + std::to_string(q.R) + " ph=" + std::to_string(q.ph) + "/" +
+         std::to_string(q.nph) + " cost=" + std::to_string((int)q.cost) + "\n";
+  }
+  if (needed) *needed = t.size() + 1;
+  if (buf && n > 0) {
+    const size_t k = std::min(n - 1, t.size());
+    std::memcpy(buf, t.data(), k);
+    buf[k] = '\0';
+  }
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_set_timing(cgtp_plan plan, int enable) {
+  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
+  Plan* P = reinterpret_cast<Plan*>(plan);
+  std::lock_guard<std::mutex> g(P->tmu);
+  P->timing = enable != 0;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_kernel_times(cgtp_plan plan, int max, char* names, double* ms,
+                                   int64_t* launches, int* n) {
+  if (!plan || !n) return fail(CGTP_ERR_NULL, "null argument");
+  Plan* P = reinterpret_cast<Plan*>(plan);
+  const int K = (int)(sizeof(kKindName) / sizeof(kKindName[0]));
+  std::vector<double> tot(K, 0.0);
+  std::vector<int64_t> cnt(K, 0);
+  std::vector<Plan::TimedLaunch> log;
+  {
+    std::lock_guard<std::mutex> g(P->tmu);
+    log.swap(P->tlog);
+  }
+  cgtp_status st = CGTP_OK;
+  for (auto& t : log) {
+    float v = 0.f;
+    if (st == CGTP_OK) {
+      cudaError_t e = cudaEventSynchronize(t.b);
+      if (e == cudaSuccess) e = cudaEventElapsedTime(&v, t.a, t.b);
+      if (e != cudaSuccess) st = fail(CGTP_ERR_CUDA, std::string("event timing: ") + cudaGetErrorString(e));
+    }
+    tot[t.kind] += v;
+    cnt[t.kind] += 1;
+  }
+  {
+    std::lock_guard<std::mutex> g(P->tmu);
+    for (auto& t : log) {
+      P->tpool.push_back(t.a);
+      P->tpool.push_back(t.b);
+    }
+  }
+  int k = 0;
+  for (int q = 0; q < K; ++q) {
+    if (cnt[q] == 0) continue;
+    if (k < max) {
+      if (names) std::snprintf(names + 32 * k, 32, "%s", kKindName[q]);
+      if (ms) ms[k] = tot[q];
+      if (launches) launches[k] = cnt[q];
+    }
+    ++k;
+  }
+  *n = k;
+  return st;
+}
+
+cgtp_status cgtp_plan_check_device_error(cgtp_plan plan, int* code) {
+  if (!plan || !code) return fail(CGTP_ERR_NULL, "null argument");
+  Plan* P = reinterpret_cast<Plan*>(plan);
+  cgtp_status st = check_device(*P);
+  if (st != CGTP_OK) return st;
+  CGTP_CUDA_TRY(cudaDeviceSynchronize());
+  int v = 0;
+  CGTP_CUDA_TRY(cudaMemcpy(&v, P->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+  CGTP_CUDA_TRY(cudaMemset(P->d_err, 0, sizeof(int)));
+  *code = v;
+  if (v != 0) return fail(CGTP_ERR_TIMEOUT, "a bounded wait inside a kernel expired");
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_neighbor_list(int64_t N, const double* pos, const double* box, double rc,
+                               int32_t* rowptr, int32_t* col, int32_t* shift, float* r,
+                               int64_t* n_edges) {
+  try {
+    return neighbor_list_impl(N, pos, box, rc, rowptr, col, shift, r, n_edges);
+  } catch (const std::exception& e) {
+    return fail(CGTP_ERR_OOM, e.what());
+  }
+}
+
+cgtp_status cgtp_csr_transpose(int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
+                               const int32_t* col, int32_t* rowptr_T, int32_t* perm_T) {
+  try {
+    return csr_transpose_impl(n_recv, n_send, E, rowptr, col, rowptr_T, perm_T);
+  } catch (const std::exception& e) {
+    return fail(CGTP_ERR_OOM, e.what());
+  }
+}
+
+}  // extern "C"

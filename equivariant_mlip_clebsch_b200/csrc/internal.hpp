@@ -1,0 +1,154 @@
+// internal.hpp -- shared declarations of the libcgtp host code.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <memory>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "cgtp.h"
+
+namespace cgtp {
+
+// ---------------------------------------------------------------- errors
+void set_error(const std::string& msg);
+cgtp_status fail(cgtp_status s, const std::string& msg);
+
+#define CGTP_CUDA_TRY(expr)                                                          \
+  do {                                                                               \
+    cudaError_t _e = (expr);                                                         \
+    if (_e != cudaSuccess)                                                           \
+      return ::cgtp::fail(CGTP_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(_e)); \
+  } while (0)
+
+// ---------------------------------------------------------------- irreps
+struct Irrep {
+  int mul;
+  int l;
+  int parity;  // +1 even, -1 odd
+};
+bool parse_irreps(const char* s, std::vector<Irrep>& out, std::string& err);
+
+// ---------------------------------------------------------------- CG
+// Real CG block [2l1+1][2l2+1][2l3+1] in FP64 (see cgtp.h for conventions).
+bool real_cg_block(int l1, int l2, int l3, std::vector<double>& C);
+
+// ---------------------------------------------------------------- paths
+struct Path {
+  int l1, l2, l3;
+  int irrep;  // index of the hidden irrep
+  int mul;
+  int x_off;  // hidden block offset in a row of x
+  int k0;     // W column of channel 0
+  int o_off;  // out offset of channel 0
+  int c_off;  // offset into the FP64 coefficient array
+  int out_irrep;
+};
+
+// One warp's share of the forward: channels [u0, u0 + 32*R) of one hidden
+// irrep for a group of its paths (accumulators live in registers).
+struct FwdRole {
+  int irrep;
+  int u0;
+  int R;
+  std::vector<int> paths;  // indices into Plan::paths
+  double cost;
+};
+
+// One warp's share of the backward: channels [u0, u0 + 32*R) of one hidden
+// irrep, every path of that irrep, the edges of a chunk with b % nph == ph.
+struct BwdRole {
+  int irrep;
+  int u0;
+  int R;
+  int ph, nph;
+  double cost;
+};
+
+struct JitKernel {
+  void* module = nullptr;    // CUmodule
+  void* function = nullptr;  // CUfunction
+  int threads = 0;
+  int smem = 0;
+  std::string name;
+  std::string log;
+  unsigned long long hash = 0;  // of the generated source and compile options
+};
+
+struct FwdConfig {
+  int S = 1;             // slices (CTAs per receiver)
+  int nw = 0;            // consumer warps per CTA
+  int B = 4;             // edges per chunk
+  int stages = 3;        // ring depth
+  bool w_smem = true;    // W rows staged by bulk copy (needs S == 1)
+  bool x_smem = true;    // x blocks staged by bulk copy
+  int nacc = 0;          // accumulator registers per thread
+  std::vector<std::vector<int>> slice_roles;  // role ids per slice
+};
+
+struct Plan {
+  std::string irreps_in_s, irreps_edge_s, irreps_out_s;
+  std::vector<Irrep> in, edge, out;
+  int lmax = 0, L = 0;
+  int64_t D_in = 0, D_e = 0, D_out = 0, U = 0;
+  std::vector<int> x_off, out_off, chan_base;
+  std::vector<Path> paths;
+  std::vector<double> coeff;  // concatenated real CG blocks (FP64)
+  int device = -1;
+
+  // forward
+  std::vector<FwdRole> fwd_roles;
+  FwdConfig fcfg;
+  JitKernel fwd;
+  // Chat build tables per slice (device): entry -> (dst offset, term begin, term count)
+  void* d_fwd_ent = nullptr;   // int4 [n]
+  void* d_fwd_term = nullptr;  // int2 [n] (y index, coeff bits)
+  std::vector<int> fwd_ent_begin;  // per slice, into d_fwd_ent (size S+1)
+  std::vector<int> fwd_chs;        // Chat floats per edge per slice
+
+  // backward
+  std::vector<BwdRole> bwd_roles;
+  FwdConfig bcfg;
+  JitKernel bwd;
+  void* d_bwd_ent = nullptr;
+  void* d_bwd_term = nullptr;
+  std::vector<int> bwd_ent_begin;
+  std::vector<int> bwd_chs;
+  bool bwd_irrep_gap = false;  // some hidden irrep has no path
+
+  int* d_err = nullptr;  // device error word
+  // kernel timing (cgtp_plan_set_timing)
+  bool timing = false;
+  std::mutex tmu;
+  struct TimedLaunch {
+    int kind;
+    cudaEvent_t a, b;
+  };
+  std::vector<TimedLaunch> tlog;
+  std::vector<cudaEvent_t> tpool;
+  bool host_only = false;  // built for compile checks only: no device state
+  int L_sh = 0;
+};
+
+// construction steps
+cgtp_status build_paths(Plan& P);
+cgtp_status build_forward(Plan& P);
+cgtp_status build_backward(Plan& P);
+void destroy_plan_device(Plan& P);
+
+// JIT
+cgtp_status jit_compile(const std::string& src, const std::string& name, JitKernel& k);
+cgtp_status jit_launch(const JitKernel& k, dim3 grid, void** args, cudaStream_t stream);
+void jit_unload(JitKernel& k);
+
+// generic CUDA kernels (kernels.cu)
+cudaError_t launch_sph_harm(int L, int64_t E, const float* r, float* Y, cudaStream_t s);
+cudaError_t launch_segment_rows(int64_t n_send, int64_t width, const int32_t* rowptr_T,
+                                const int32_t* perm_T, const float* m, float* dx,
+                                cudaStream_t s);
+cudaError_t launch_sum_slices(int S, int64_t n, const float* parts, float* dst, cudaStream_t s);
+
+}  // namespace cgtp

@@ -1,0 +1,206 @@
+/*
+ * cgtp.h -- C ABI of the B200 Clebsch-Gordan tensor-product (CGTP)
+ * convolution library (libcgtp.so).
+ *
+ * The operation is the CGTP convolution that the LunaTP page (arXiv
+ * 2610.18393, Abstract) names as the core cost of equivariant interatomic
+ * potentials, with the irreps configurations of its Table 1 and the outputs
+ * of its Table 11 (forward x'; backward x-bar, y-bar, w-bar).  The pages give
+ * no formula; this library computes, for a receiver-sorted edge list i <- j,
+ *
+ *   out[i, o_off(p) + u (2l3+1) + m3] =
+ *       sum_{e in row i} W[e, k0(p) + u]
+ *         sum_{m1,m2} C_p[m1,m2,m3] x[col e, x_off(p) + u (2l1+1) + m1] Y[e, l2^2 + m2]
+ *
+ * over every path p = (hidden irrep l1, edge irrep l2 -> l3) allowed by the
+ * triangle rule and parity, with channelwise ("uvu") weights W per edge.
+ *
+ * Conventions
+ *   - Real spherical harmonics, component normalisation (sum_m Y_lm^2 = 2l+1),
+ *     m = -l..l, no Condon-Shortley phase: Y_1(r) = sqrt(3) (y, z, x)/|r|.
+ *   - Real CG blocks in that basis, sum C^2 = 2 l3 + 1, first non-zero entry
+ *     (lexicographic m1, m2, m3) positive.
+ *   - Paths: for each hidden irrep in order, each edge irrep in order, each l3
+ *     from |l1-l2| to l1+l2 ascending, kept when (l3, p1 p2) is an output
+ *     irrep.  Its channels are appended to that output block in this order;
+ *     every output block must receive exactly its declared multiplicity.
+ *   - W column k is the global output channel (output irreps in order).
+ *
+ * Layouts (all row-major, FP32 unless stated, device memory unless stated)
+ *   x    [n_send, d_in]    hidden irrep blocks in order, each [mul, 2l+1]
+ *   Y    [E, d_edge]       d_edge = (L+1)^2, degree l at columns l^2..l^2+2l
+ *   W    [E, n_weights]
+ *   out  [n_recv, d_out]   output irrep blocks in order, each [mul, 2l+1]
+ *   rowptr [n_recv+1] int32 (receiver CSR), col [E] int32 sender per edge
+ *   rowptr_T [n_send+1], perm_T [E] int32: edge ids grouped by sender,
+ *   ascending inside each sender (see cgtp_csr_transpose).
+ *
+ * Ownership: the caller owns every buffer.  A plan owns its own host tables,
+ * device tables and compiled kernels from cgtp_plan_create to
+ * cgtp_plan_destroy.  Forward and backward allocate nothing; the backward's
+ * scratch is a caller-provided workspace (cgtp_backward_workspace_size).
+ *
+ * Errors: every entry point returns a cgtp_status.  Arguments are validated
+ * on the host before any launch (null pointers, 16-byte alignment of float
+ * arrays, sizes, irreps, lmax).  No exception crosses the ABI.
+ * cgtp_last_error() returns a message for the calling thread's last failure.
+ * Calls are ordered on the given stream; a plan may be used from several
+ * threads for concurrent launches.
+ */
+#ifndef CGTP_H_
+#define CGTP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct cgtp_plan_s* cgtp_plan;
+typedef void* cgtp_stream; /* a cudaStream_t; NULL means the legacy default stream */
+
+typedef enum {
+  CGTP_OK = 0,
+  CGTP_ERR_NULL = 1,            /* a required pointer is NULL */
+  CGTP_ERR_ALIGN = 2,           /* a float array is not 16-byte aligned */
+  CGTP_ERR_IRREPS_PARSE = 3,    /* an irreps string does not parse */
+  CGTP_ERR_IRREPS_MISMATCH = 4, /* output multiplicities disagree with the paths */
+  CGTP_ERR_LMAX = 5,            /* some l exceeds lmax, or lmax > 6 */
+  CGTP_ERR_SIZE = 6,            /* a size is negative, too large, or inconsistent */
+  CGTP_ERR_INVALID_CSR = 7,     /* rowptr/col/perm inconsistent (host checks) */
+  CGTP_ERR_CUDA = 8,            /* a CUDA runtime or driver call failed */
+  CGTP_ERR_OOM = 9,             /* host or device allocation failed in plan create */
+  CGTP_ERR_TIMEOUT = 10,        /* a bounded wait inside a kernel gave up */
+  CGTP_ERR_JIT = 11,            /* runtime compilation of a kernel failed */
+  CGTP_ERR_WORKSPACE = 12       /* backward workspace missing or too small */
+} cgtp_status;
+
+/* Human-readable name of a status.  Never NULL. */
+const char* cgtp_status_string(cgtp_status s);
+
+/* Detail of the calling thread's most recent non-OK status.  Never NULL. */
+const char* cgtp_last_error(void);
+
+/* Build a plan on the CURRENT CUDA device.
+ *   irreps_in   hidden irreps, e.g. "128x0e+64x1o"  (LunaTP Table 1 "Hidden irreps")
+ *   irreps_edge exactly "1x0?+1x1?+...+1xL?" (Table 1 "Edge irreps"); the parity
+ *               letters only select paths, the harmonics are the true Y_l
+ *   irreps_out  output irreps (Table 1 "Output irreps"), each (l, parity) once
+ *   lmax        upper bound on every l in the three strings, 0 <= lmax <= 6
+ * Parses and checks the irreps, enumerates the paths, builds the real CG
+ * tables in FP64 (rounded to FP32 for the device), generates and compiles the
+ * path-specialised forward and backward kernels for sm_100a, and uploads the
+ * tables.  On failure *out is set to NULL. */
+cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge,
+                             const char* irreps_out, int lmax, cgtp_plan* out);
+
+/* Release every resource of the plan.  NULL is accepted.  The caller must
+ * ensure no launch using the plan is still running. */
+cgtp_status cgtp_plan_destroy(cgtp_plan plan);
+
+/* Sizes of the plan: row widths of x (d_in), Y (d_edge), out (d_out), the
+ * number of W columns (n_weights = total output channels) and of paths.
+ * Any output pointer may be NULL. */
+cgtp_status cgtp_plan_info(cgtp_plan plan, int64_t* d_in, int64_t* d_edge, int64_t* d_out,
+                           int64_t* n_weights, int64_t* n_paths);
+
+/* Host copy of the path table: n_paths rows of 8 int32
+ *   l1, l2, l3, mul, x_off, k0, o_off, c_off
+ * (c_off = offset of the path's [2l1+1][2l2+1][2l3+1] block in the
+ * coefficient array that cgtp_plan_coefficients returns). */
+cgtp_status cgtp_plan_paths(cgtp_plan plan, int32_t* table);
+
+/* Host copy of the plan's real CG blocks in FP64, concatenated in path order;
+ * n_coeff receives the total length (call with coeff == NULL to size it). */
+cgtp_status cgtp_plan_coefficients(cgtp_plan plan, double* coeff, int64_t* n_coeff);
+
+/* Host-only: the library's real CG block C[2l1+1][2l2+1][2l3+1] in FP64 for
+ * one coupling l1 (x) l2 -> l3 (each l <= 12).  Needs no GPU. */
+cgtp_status cgtp_real_cg(int l1, int l2, int l3, double* C);
+
+/* Real spherical harmonics of the edge vectors (L = the plan's edge degree).
+ *   r [E,3] FP32 device, Y [E, d_edge] FP32 device (overwritten).
+ * r need not be normalised; r = 0 gives Y_00 = 1 and zeros elsewhere.
+ * Source: Table 1 edge irreps and Fig. 1 (Lmax = 6) of the LunaTP page. */
+cgtp_status cgtp_sph_harm(cgtp_plan plan, int64_t E, const float* r, float* Y,
+                          cgtp_stream stream);
+
+/* Forward CGTP convolution (the x' of LunaTP Table 11), formula above.
+ *   n_recv receivers, n_send senders, E edges (0 <= E < 2^31)
+ *   rowptr [n_recv+1], col [E] (int32, device); x [n_send, d_in];
+ *   Y [E, d_edge]; W [E, n_weights]; out [n_recv, d_out] (overwritten;
+ *   receivers without edges get zeros).
+ * Each receiver's row is accumulated on chip and stored once: no atomics, and
+ * the result is bitwise reproducible run to run. */
+cgtp_status cgtp_forward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                         const int32_t* rowptr, const int32_t* col, const float* x,
+                         const float* Y, const float* W, float* out, cgtp_stream stream);
+
+/* Bytes of device workspace cgtp_backward needs for these sizes. */
+cgtp_status cgtp_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t n_send,
+                                         int64_t E, size_t* bytes);
+
+/* Backward of the forward above given grad_out = dL/dout [n_recv, d_out]
+ * (the x-bar, w-bar, y-bar of LunaTP Table 11):
+ *   grad_x [n_send, d_in], grad_W [E, n_weights], grad_Y [E, d_edge]
+ * each overwritten; any of the three may be NULL to skip it.  The sender-major
+ * sum for grad_x goes through the transpose edge list (rowptr_T, perm_T,
+ * needed only when grad_x != NULL) and the workspace; no atomics, bitwise
+ * reproducible.  workspace must hold cgtp_backward_workspace_size bytes and be
+ * 256-byte aligned. */
+cgtp_status cgtp_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                          const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
+                          const int32_t* perm_T, const float* x, const float* Y,
+                          const float* W, const float* grad_out, float* grad_x, float* grad_W,
+                          float* grad_Y, void* workspace, size_t workspace_bytes,
+                          cgtp_stream stream);
+
+/* Text report of the plan: paths, warp roles, slices, chunk and ring sizes,
+ * shared memory, threads and the kernel assembler's register/spill lines.
+ * Writes at most n bytes (NUL-terminated); *needed receives the full length
+ * including the NUL.  buf may be NULL to query the length. */
+cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* needed);
+
+/* Per-kernel timing.  While enabled, every launch made through the plan
+ * (harmonics, forward, backward and its reduction kernels) is bracketed by a
+ * pair of CUDA events recorded on the caller's stream.  cgtp_plan_kernel_times
+ * waits for those events and returns, per kernel name, the summed device time
+ * in milliseconds and the launch count since the previous call (which resets
+ * them).  names receives up to max entries of 32 bytes each. */
+cgtp_status cgtp_plan_set_timing(cgtp_plan plan, int enable);
+cgtp_status cgtp_plan_kernel_times(cgtp_plan plan, int max, char* names, double* ms,
+                                   int64_t* launches, int* n);
+
+/* Reads and clears the plan's device error word on the current device
+ * (synchronises the device).  *code is 0 when every bounded wait of the
+ * kernels launched since the last call completed; CGTP_ERR_TIMEOUT is
+ * returned otherwise. */
+cgtp_status cgtp_plan_check_device_error(cgtp_plan plan, int* code);
+
+/* ---- graph utilities (host, no GPU needed) ----------------------------- */
+
+/* Periodic neighbour list by cell list, FP64.  Host pointers.
+ * Edge i <- j with image n (integers, |n_a| <= ceil(rc / box_a)) exists iff
+ * (i,j,n) != (i,i,0) and |(pos_j + n*box) - pos_i|^2 < rc^2, each component
+ * formed as (pos_j[a] + n_a*box[a]) - pos_i[a] and the square summed x, y, z
+ * in that order, all in FP64 (so every decision is exactly reproducible).
+ * Edges are ordered by (receiver i, sender j, n_x, n_y, n_z).  Positions must
+ * lie in [0, box).  Call with col == NULL to get *n_edges (and rowptr); then
+ * with col/shift/r sized for it.  r [E,3] FP32 = the rounded edge vectors,
+ * shift [E,3] int32 = n.  rowptr has N+1 entries. */
+cgtp_status cgtp_neighbor_list(int64_t N, const double* pos, const double* box, double rc,
+                               int32_t* rowptr, int32_t* col, int32_t* shift, float* r,
+                               int64_t* n_edges);
+
+/* Transpose of a receiver CSR: rowptr_T [n_send+1] and perm_T [E] listing, for
+ * every sender, the ids of its edges in ascending order.  Host pointers. */
+cgtp_status cgtp_csr_transpose(int64_t n_recv, int64_t n_send, int64_t E,
+                               const int32_t* rowptr, const int32_t* col, int32_t* rowptr_T,
+                               int32_t* perm_T);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CGTP_H_ */

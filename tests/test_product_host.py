@@ -1,0 +1,126 @@
+"""Host-side checks of libcgtp that need no GPU.
+
+  * the library loads and exports every entry point include/cgtp.h declares;
+  * its real CG blocks (ladder-operator construction) equal the oracle's
+    (Racah closed form) -- two independent routes to the same table;
+  * its cell-list neighbour list equals the oracle's brute force bit for bit,
+    edge vectors included;
+  * the CSR transpose and the host argument checks;
+  * every workload's plan builds and its kernels compile for sm_100a (the
+    compile-only mode skips all device work), with the oracle's path table.
+"""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+from equivariant_mlip_clebsch_b200 import workloads as WL
+from equivariant_mlip_clebsch_b200 import cgtp as C
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "cgtp.h")
+
+
+def test_every_declared_symbol_is_exported():
+    decl = set(re.findall(r"^\s*(?:const char\*|cgtp_status)\s+(cgtp_\w+)\s*\(", open(HEADER).read(), re.M))
+    assert len(decl) >= 15
+    for name in decl:
+        assert hasattr(C._lib, name), name
+    assert decl == set(C.EXPORTS)
+
+
+def test_real_cg_matches_oracle_all_triples():
+    for l1 in range(7):
+        for l2 in range(7):
+            for l3 in range(abs(l1 - l2), l1 + l2 + 1):
+                a = C.real_cg(l1, l2, l3)
+                b = O.real_cg(l1, l2, l3)
+                assert np.allclose(a, b, atol=1e-12), (l1, l2, l3)
+                assert np.array_equal(a == 0, b == 0), (l1, l2, l3)
+
+
+def test_real_cg_rejects_bad_triples():
+    with pytest.raises(C.CgtpError) as e:
+        C.real_cg(1, 1, 3)
+    assert e.value.status == 6
+
+
+@pytest.mark.parametrize("name", ["tiny", "lmax2", "lmax2_wide", "lmax3"])
+def test_neighbor_list_bit_exact(name):
+    c = WL.CONFIGS[name]
+    pos, box = WL.si_diamond(c["cells"], c["sigma"], 0)
+    rp_o, col_o, sh_o, vec_o = O.neighbor_list(pos, box, c["rc"])
+    rp, col, sh, r = C.neighbor_list(pos, box, c["rc"])
+    assert np.array_equal(rp.astype(np.int64), rp_o)
+    assert np.array_equal(col, col_o)
+    assert np.array_equal(sh, sh_o)
+    assert np.array_equal(r, vec_o.astype(np.float32))
+
+
+@pytest.mark.parametrize("cells,rc", [((1, 1, 1), 5.0), ((1, 1, 2), 6.0), ((2, 1, 1), 11.0)])
+def test_neighbor_list_small_boxes_many_images(cells, rc):
+    pos, box = WL.si_diamond(cells, 0.07, 3)
+    rp_o, col_o, sh_o, vec_o = O.neighbor_list(pos, box, rc)
+    rp, col, sh, r = C.neighbor_list(pos, box, rc)
+    assert np.array_equal(rp.astype(np.int64), rp_o) and np.array_equal(col, col_o)
+    assert np.array_equal(sh, sh_o) and np.array_equal(r, vec_o.astype(np.float32))
+
+
+def test_neighbor_list_rejects_unwrapped_positions():
+    with pytest.raises(C.CgtpError):
+        C.neighbor_list(np.array([[0.0, 0.0, 5.0]]), np.array([4.0, 4.0, 4.0]), 3.0)
+
+
+def test_csr_transpose():
+    rng = np.random.default_rng(1)
+    deg = rng.integers(0, 6, size=40)
+    rowptr = np.concatenate([[0], np.cumsum(deg)]).astype(np.int32)
+    col = rng.integers(0, 25, size=rowptr[-1]).astype(np.int32)
+    rpt, perm = C.csr_transpose(rowptr, col, 25)
+    assert rpt[0] == 0 and rpt[-1] == len(col)
+    for j in range(25):
+        ids = perm[rpt[j]:rpt[j + 1]]
+        assert np.all(col[ids] == j) and np.all(np.diff(ids) > 0)
+    assert np.array_equal(np.sort(perm), np.arange(len(col)))
+    with pytest.raises(C.CgtpError):
+        C.csr_transpose(rowptr, np.full_like(col, 30), 25)
+
+
+@pytest.fixture
+def compile_only(monkeypatch):
+    monkeypatch.setenv("CGTP_JIT_COMPILE_ONLY", "1")
+
+
+@pytest.mark.parametrize("name", ["tiny", "lmax2", "lmax2_wide", "lmax3", "lmax6"])
+def test_plan_builds_and_compiles(name, compile_only):
+    c = WL.CONFIGS[name]
+    plan = C.Plan(c["irreps_in"], c["irreps_edge"], c["irreps_out"], 6)
+    P = O.enumerate_paths(c["irreps_in"], c["irreps_edge"], c["irreps_out"])
+    assert (plan.d_in, plan.d_edge, plan.d_out, plan.n_weights, plan.n_paths) == \
+        (P.D_in, P.D_e, P.D_out, P.U, P.npaths)
+    assert np.array_equal(plan.paths(), P.table)
+    assert np.allclose(plan.coefficients(), P.cg, atol=1e-12)
+    text = plan.describe()
+    assert "cgtp_fwd" in text and "cgtp_bwd" in text
+    # a compile-only plan refuses to launch
+    with pytest.raises(C.CgtpError):
+        plan.check_device_error()
+
+
+@pytest.mark.parametrize("args,status", [
+    (("16x0e+", "1x0e", "16x0e"), 3),
+    (("16x0e", "1x0e+1x2e", "16x0e"), 3),
+    (("16x0e+16x1o", "1x0e+1x1o", "32x0e+16x1o"), 4),
+    (("16x7e", "1x0e", "16x7e"), 5),
+])
+def test_plan_argument_errors(args, status, compile_only):
+    with pytest.raises(C.CgtpError) as e:
+        C.Plan(*args, 6)
+    assert e.value.status == status
+
+
+def test_lmax_bound(compile_only):
+    with pytest.raises(C.CgtpError) as e:
+        C.Plan("4x3e", "1x0e+1x1o", "4x3e+4x2o+4x4o", 2)
+    assert e.value.status == 5
