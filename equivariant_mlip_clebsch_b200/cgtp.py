@@ -41,6 +41,8 @@ _SIGS = {
     "cgtp_backward_workspace_size": (_i, [_P, _i64, _i64, _i64, ctypes.POINTER(_sz)]),
     "cgtp_backward": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                            _P, _sz, _P]),
+    "cgtp_backward_static_scratch": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                          _P, _P, _P]),
     "cgtp_plan_check_device_error": (_i, [_P, ctypes.POINTER(_i)]),
     "cgtp_plan_set_timing": (_i, [_P, _i]),
     "cgtp_plan_kernel_times": (_i, [_P, _i, ctypes.c_char_p, _P, _P, ctypes.POINTER(_i)]),
@@ -53,6 +55,7 @@ for _name, (_res, _args) in _SIGS.items():
     _f.argtypes = _args
 
 EXPORTS = tuple(_SIGS)
+STATIC_SCRATCH_BYTES = 64 << 20  # CGTP_STATIC_SCRATCH_BYTES of include/cgtp.h
 
 
 class CgtpError(RuntimeError):
@@ -240,4 +243,24 @@ class Plan:
                                   _tptr(rowptr_T), _tptr(perm_T), _tptr(x), _tptr(Y), _tptr(W),
                                   _tptr(grad_out), _tptr(dx), _tptr(dW), _tptr(dY),
                                   _tptr(workspace), workspace.numel(), _stream(stream)))
+        return dx, dW, dY
+
+    def backward_static_scratch(self, rowptr, col, rowptr_T, perm_T, x, Y, W, grad_out,
+                                want=("x", "W", "Y"), grads=None, stream=None):
+        """cgtp_backward_static_scratch: the backward with the library's fixed
+        device scratch instead of a workspace (no device allocation in the call
+        when ``grads`` are given)."""
+        import torch
+        n_recv, n_send, E = rowptr.shape[0] - 1, x.shape[0], col.shape[0]
+        dev = x.device
+        if grads is None:
+            dx = torch.empty((n_send, self.d_in), dtype=torch.float32, device=dev) if "x" in want else None
+            dW = torch.empty((E, self.n_weights), dtype=torch.float32, device=dev) if "W" in want else None
+            dY = torch.empty((E, self.d_edge), dtype=torch.float32, device=dev) if "Y" in want else None
+        else:
+            dx, dW, dY = grads
+        _check(_lib.cgtp_backward_static_scratch(self._h, n_recv, n_send, E, _tptr(rowptr), _tptr(col),
+                                                 _tptr(rowptr_T), _tptr(perm_T), _tptr(x), _tptr(Y),
+                                                 _tptr(W), _tptr(grad_out), _tptr(dx), _tptr(dW),
+                                                 _tptr(dY), _stream(stream)))
         return dx, dW, dY

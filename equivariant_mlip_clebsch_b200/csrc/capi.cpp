@@ -75,8 +75,8 @@ struct TimedScope {
     if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
     return e;
   }
-  TimedScope(Plan& P_, int k, cudaStream_t st) : P(P_), kind(k), s(st) {
-    if (!P.timing) return;
+  TimedScope(Plan& P_, int k, cudaStream_t st, bool allowed = true) : P(P_), kind(k), s(st) {
+    if (!allowed || !P.timing) return;
     std::lock_guard<std::mutex> g(P.tmu);
     a = take(P);
     b = take(P);
@@ -264,6 +264,21 @@ cgtp_status cgtp_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
                           const int32_t* perm_T, const float* x, const float* Y, const float* W,
                           const float* grad_out, float* grad_x, float* grad_W, float* grad_Y,
                           void* workspace, size_t workspace_bytes, cgtp_stream stream) {
+  return cgtp::backward_impl(plan, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, x, Y, W,
+                             grad_out, grad_x, grad_W, grad_Y, workspace, workspace_bytes, stream,
+                             true);
+}
+
+}  // extern "C"
+
+namespace cgtp {
+
+cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                          const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
+                          const int32_t* perm_T, const float* x, const float* Y, const float* W,
+                          const float* grad_out, float* grad_x, float* grad_W, float* grad_Y,
+                          void* workspace, size_t workspace_bytes, cgtp_stream stream,
+                          bool allow_timing) {
   if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
   Plan* P = reinterpret_cast<Plan*>(plan);
   if (n_recv < 0 || n_send < 0 || E < 0 || n_recv >= (int64_t(1) << 31) ||
@@ -302,26 +317,31 @@ cgtp_status cgtp_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
                         : grad_Y;
   }
   if (m && P->bwd_irrep_gap) {  // hidden irreps without paths receive zero gradient
-    TimedScope ts(*P, 5, s);
+    TimedScope ts(*P, 5, s, allow_timing);
     CGTP_CUDA_TRY(cudaMemsetAsync(m, 0, (size_t)E * P->D_in * sizeof(float), s));
   }
   if (n_recv > 0) {
     void* args[] = {&rowptr, &col,   &x, &Y, &W, &grad_out, &grad_W, &dyp, &m,
                     &P->d_bwd_ent, &P->d_bwd_term, &P->d_err};
-    TimedScope ts(*P, 2, s);
+    TimedScope ts(*P, 2, s, allow_timing);
     st = jit_launch(P->bwd, dim3((unsigned)n_recv, (unsigned)P->bcfg.S), args, s);
     if (st != CGTP_OK) return st;
   }
   if (grad_Y && P->bcfg.S > 1) {
-    TimedScope ts(*P, 4, s);
+    TimedScope ts(*P, 4, s, allow_timing);
     CGTP_CUDA_TRY(launch_sum_slices(P->bcfg.S, E * P->D_e, dyp, grad_Y, s));
   }
   if (grad_x) {
-    TimedScope ts(*P, 3, s);
+    TimedScope ts(*P, 3, s, allow_timing);
     CGTP_CUDA_TRY(launch_segment_rows(n_send, P->D_in, rowptr_T, perm_T, m, grad_x, s));
   }
   return CGTP_OK;
 }
+
+
+}  // namespace cgtp
+
+extern "C" {
 
 cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* needed) {
   if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");

@@ -133,6 +133,13 @@ struct Plan {
   int L_sh = 0;
 };
 
+cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                          const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
+                          const int32_t* perm_T, const float* x, const float* Y, const float* W,
+                          const float* grad_out, float* grad_x, float* grad_W, float* grad_Y,
+                          void* workspace, size_t workspace_bytes, cgtp_stream stream,
+                          bool allow_timing);
+
 // construction steps
 cgtp_status build_paths(Plan& P);
 cgtp_status build_forward(Plan& P);

@@ -172,6 +172,36 @@ cgtp_status cgtp_plan_set_timing(cgtp_plan plan, int enable);
 cgtp_status cgtp_plan_kernel_times(cgtp_plan plan, int max, char* names, double* ms,
                                    int64_t* launches, int* n);
 
+/* Size of the fixed device scratch of cgtp_backward_static_scratch: 64 MiB. */
+#define CGTP_STATIC_SCRATCH_BYTES (64u << 20)
+
+/* cgtp_backward without a caller workspace, for callers that cannot allocate
+ * device memory when they call it: e.g. a simulation engine that sizes all of
+ * its device memory once at start-up and forbids later allocation, or an
+ * embedding runtime that owns no device allocator.  (The pages have no
+ * counterpart; this is an interface convenience.)
+ *
+ * Same arguments, outputs and errors as cgtp_backward, minus the workspace.
+ * The scratch is a fixed array of CGTP_STATIC_SCRATCH_BYTES inside the
+ * library's device code: every GPU that loads the library holds it until the
+ * process exits.  The call allocates nothing (no cudaMalloc/cudaFree, no
+ * library allocator).  Sizes whose cgtp_backward_workspace_size exceeds the
+ * array are rejected with CGTP_ERR_WORKSPACE before any launch.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current (cudaGetSymbolAddress) and caches it; make that
+ *     first call before any stream capture on the device.
+ *   - All calls share the one array and it keeps the last call's contents
+ *     (nothing in it has to start at zero).  Calls whose launches overlap on
+ *     the GPU (different streams, or different threads without ordering)
+ *     race on it; order them on one stream.
+ *   - Kernel timing (cgtp_plan_set_timing) does not record these launches. */
+cgtp_status cgtp_backward_static_scratch(cgtp_plan plan, int64_t n_recv, int64_t n_send,
+                                         int64_t E, const int32_t* rowptr, const int32_t* col,
+                                         const int32_t* rowptr_T, const int32_t* perm_T,
+                                         const float* x, const float* Y, const float* W,
+                                         const float* grad_out, float* grad_x, float* grad_W,
+                                         float* grad_Y, cgtp_stream stream);
+
 /* Reads and clears the plan's device error word on the current device
  * (synchronises the device).  *code is 0 when every bounded wait of the
  * kernels launched since the last call completed; CGTP_ERR_TIMEOUT is
