@@ -188,6 +188,13 @@ def run_cgtp(args, rank, world, local_rank):
         step(T["r"], T["x"], T["W"], T["g"])
     torch.cuda.synchronize()
     plan.check_device_error()
+    if args.profile:  # for ncu: warm-up plus K plain steps, nothing else
+        for _ in range(args.steps):
+            flush.zero_()
+            step(T["r"], T["x"], T["W"], T["g"])
+        torch.cuda.synchronize()
+        plan.check_device_error()
+        return {"profile": name, "steps": args.steps, "warmup": args.warmup, "N": N, "E": E}
 
     # keep the GPU busy ~1 s while the clock sampler warms up, then time K steps
     sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ
@@ -435,6 +442,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(WL.CONFIGS))
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline field (0 to skip)")
+    ap.add_argument("--profile", action="store_true",
+                    help="warm-up + K steps only (no clock loop, e2e or CPU baseline), for ncu")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -453,7 +462,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     res = run_cgtp(args, rank, world, local_rank)
-    if rank == 0 and args.cpu_budget > 0:
+    if rank == 0 and args.cpu_budget > 0 and not args.profile:
         s = oracle_sample(args.config, args.cpu_budget)
         res["cpu_baseline"] = {"value": s["edges_per_s"], "unit": "edges/s", "cores": s["cores"],
                                "kind": "oracle",
