@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -90,6 +91,24 @@ struct TimedScope {
   }
 };
 
+// Persistent grid: T resident CTAs shared among the slices in proportion to
+// their work; CTAs [start[s], start[s+1]) serve slice s.
+static std::vector<int> slice_partition(const FwdConfig& F, int blocks_per_sm, int num_sms,
+                                        int64_t n_recv) {
+  const int S = F.S;
+  const long T = std::max<long>(S, (long)blocks_per_sm * num_sms);
+  double W = 0.0;
+  for (int s = 0; s < S; ++s) W += (s < (int)F.weight.size() ? F.weight[s] : 1.0);
+  std::vector<int> start(S + 1, 0);
+  for (int s = 0; s < S; ++s) {
+    const double w = s < (int)F.weight.size() ? F.weight[s] : 1.0;
+    long g = (long)std::floor(T * w / std::max(W, 1e-30));
+    g = std::max<long>(1, std::min<long>(g, std::max<int64_t>(1, n_recv)));
+    start[s + 1] = start[s] + (int)g;
+  }
+  return start;
+}
+
 }  // namespace cgtp
 
 using namespace cgtp;
@@ -139,6 +158,7 @@ cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge, con
     P->host_only = std::getenv("CGTP_JIT_COMPILE_ONLY") != nullptr;
     if (!P->host_only) {
       CGTP_CUDA_TRY(cudaGetDevice(&P->device));
+      CGTP_CUDA_TRY(cudaDeviceGetAttribute(&P->num_sms, cudaDevAttrMultiProcessorCount, P->device));
       CGTP_CUDA_TRY(cudaFree(0));  // make the primary context current
       if (cudaMalloc(&P->d_err, sizeof(int)) != cudaSuccess) return fail(CGTP_ERR_OOM, "cudaMalloc");
       CGTP_CUDA_TRY(cudaMemset(P->d_err, 0, sizeof(int)));
@@ -242,9 +262,13 @@ cgtp_status cgtp_forward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t
     CGTP_CUDA_TRY(cudaMemsetAsync(out, 0, (size_t)n_recv * P->D_out * sizeof(float), s));
     return CGTP_OK;
   }
-  void* args[] = {&rowptr, &col, &x, &Y, &W, &out, &P->d_fwd_ent, &P->d_fwd_term, &P->d_err};
+  int nr = (int)n_recv;
+  // persistent CTAs: about one wave of resident CTAs, each walking its slice's
+  // receivers first, first + stride, ...
+  std::vector<int> part = slice_partition(P->fcfg, P->fwd.blocks_per_sm, P->num_sms, n_recv);
+  void* args[] = {&rowptr, &col, &x, &Y, &W, &out, &P->d_fwd_ent, &nr, &P->d_err, part.data()};
   TimedScope ts(*P, 1, s);
-  return jit_launch(P->fwd, dim3((unsigned)n_recv, (unsigned)P->fcfg.S), args, s);
+  return jit_launch(P->fwd, dim3((unsigned)part.back(), 1), args, s);
 }
 
 cgtp_status cgtp_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
@@ -321,10 +345,12 @@ cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
     CGTP_CUDA_TRY(cudaMemsetAsync(m, 0, (size_t)E * P->D_in * sizeof(float), s));
   }
   if (n_recv > 0) {
-    void* args[] = {&rowptr, &col,   &x, &Y, &W, &grad_out, &grad_W, &dyp, &m,
-                    &P->d_bwd_ent, &P->d_bwd_term, &P->d_err};
+    int nr = (int)n_recv;
+    std::vector<int> part = slice_partition(P->bcfg, P->bwd.blocks_per_sm, P->num_sms, n_recv);
+    void* args[] = {&rowptr, &col, &x, &Y, &W, &grad_out, &grad_W, &dyp, &m, &P->d_bwd_ent, &nr,
+                    &P->d_err, part.data()};
     TimedScope ts(*P, 2, s, allow_timing);
-    st = jit_launch(P->bwd, dim3((unsigned)n_recv, (unsigned)P->bcfg.S), args, s);
+    st = jit_launch(P->bwd, dim3((unsigned)part.back(), 1), args, s);
     if (st != CGTP_OK) return st;
   }
   if (grad_Y && P->bcfg.S > 1) {
@@ -354,7 +380,7 @@ cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* need
        std::to_string(P->paths.size()) + "\n";
   auto cfg = [&](const char* nm, const FwdConfig& F, const JitKernel& k, size_t nroles) {
     t += std::string(nm) + ": roles=" + std::to_string(nroles) + " slices=" + std::to_string(F.S) +
-         " warps=" + std::to_string(F.nw) + "+1 chunk=" + std::to_string(F.B) + " stages=" +
+         " warps=" + std::to_string(F.nw) + "+2 chunk=" + std::to_string(F.B) + " stages=" +
          std::to_string(F.stages) + " w_smem=" + std::to_string((int)F.w_smem) + " x_smem=" +
          std::to_string((int)F.x_smem) + " nacc=" + std::to_string(F.nacc) + " smem=" +
          std::to_string(k.smem) + " threads=" + std::to_string(k.threads);

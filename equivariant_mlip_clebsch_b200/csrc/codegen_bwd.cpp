@@ -1,25 +1,25 @@
 // codegen_bwd.cpp -- the backward CGTP convolution kernel, generated per plan.
 //
 // Given g = dL/dout (LunaTP, arXiv 2610.18393, Table 11 lists the backward
-// outputs x-bar, y-bar, w-bar), per edge e = (i <- j) and path p, channel u:
+// outputs x-bar, y-bar, w-bar), per edge e = (i <- j), path p, channel u:
 //   t[m3]  = sum_m1 Chat[m3][m1] x[j][u][m1]            (as in the forward)
 //   dW[e][k0+u]      = sum_m3 g[i][u][m3] t[m3]
 //   h[m3]  = W[e][k0+u] g[i][u][m3]
-//   msg[e][u][m1]   += sum_m3 Chat[m3][m1] h[m3]        (summed over the paths of the irrep)
+//   msg[e][u][m1]   += sum_m3 Chat[m3][m1] h[m3]        (over the paths of the irrep)
 //   dY[e][l2^2+m2]  += sum_{u,m1,m3} C[m1][m2][m3] x[j][u][m1] h[m3]
 // and dx[j] = sum over the edges leaving j of msg[e] (a second, sender-major
-// pass over the transpose edge list, in kernels.cu).
+// pass over the transpose edge list, kernels.cu).
 //
-// Execution: grid (n_recv, S), receiver-major like the forward.  The
-// receiver's g row (its slice) is staged in shared memory once; W, x and Y of
-// the edges stream through the same bulk-copy ring as the forward.  A warp
-// role owns R channels per lane of one hidden irrep, ALL paths of that irrep
-// (so msg is complete in registers) and the edges b of each chunk with
-// b % nph == ph.  dW and msg are written straight to global memory; the dY
-// partial of each role is reduced across the warp by shuffles and across the
-// roles of the CTA in a fixed order through shared memory, so the result is
-// bitwise reproducible.  With S > 1 slices the per-slice dY parts go to the
-// workspace and are summed by a small kernel.
+// Execution: grid (n_recv, S) with one slice per hidden irrep, so that every
+// consumer warp of a CTA runs the same role function (instruction-cache
+// friendly, and CTAs of one slice are scheduled together).  The TMA warp
+// stages the receiver's grad_out pieces once and then, per chunk, the W and x
+// pieces of the irrep; the helper warp stages Y, builds Chat and sums the dY
+// partials of released stages.  A consumer owns R channels of the irrep, ALL
+// its paths (so msg is complete in registers) and the edges b of each chunk
+// with b % nph == ph.  dW and msg go straight to global memory; dY partials
+// are reduced over lanes by shuffles, over the CTA's warps by the helper in a
+// fixed order, and over slices by a small kernel: bitwise reproducible.
 #include <algorithm>
 #include <array>
 #include <cmath>
@@ -50,70 +50,18 @@ std::string flt(double v) {
 
 }  // namespace
 
-static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>& SL,
-                                  const std::string& kname, int& smem_bytes) {
+static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>& SL, const KernelShape& K,
+                                  const std::string& kname) {
   const FwdConfig& F = P.bcfg;
-  const int S = F.S, NW = F.nw, B = F.B;
-  int GS = 0;
-  for (const auto& sl : SL) GS = std::max(GS, sl.gs);
-  auto r128 = [](int v) { return (v + 127) & ~127; };
-  const int extra = r128(GS * 4) + r128(NW * B * (int)P.D_e * 4);
-  int off_g = 0;
+  const int S = K.S, NW = K.nw;
   std::ostringstream o;
   o << kPrelude;
-  o << gen_layout(P, F, SL, extra, off_g, smem_bytes);
-  o << "#define OFF_G " << off_g << "\n#define OFF_DY " << off_g + r128(GS * 4) << "\n";
-  o << gen_slice_helpers(P, F, SL);
-  o << gen_producer(P, F);
+  o << gen_common_device(P, SL, K, true);
 
-  // g staging per slice (by the consumer threads)
-  o << "__device__ __forceinline__ void stage_g(int s, const float* __restrict__ grow, float* sg, int tid) {\n"
-       "  switch (s) {\n";
-  for (int s = 0; s < S; ++s) {
-    o << "  case " << s << ":\n";
-    std::vector<std::array<int, 3>> cp;
-    for (int pi : SL[s].paths) {
-      const Path& p = P.paths[pi];
-      const int src = p.o_off, dst = SL[s].g_st.at(pi), n = p.mul * (2 * p.l3 + 1);
-      if (!cp.empty() && cp.back()[0] + cp.back()[2] == src && cp.back()[1] + cp.back()[2] == dst)
-        cp.back()[2] += n;
-      else
-        cp.push_back({src, dst, n});
-    }
-    for (auto& c : cp)
-      o << "    for (int t = tid; t < " << c[2] << "; t += NW * 32) sg[" << c[1] << " + t] = grow[" << c[0]
-        << " + t];\n";
-    o << "    break;\n";
-  }
-  o << "  }\n}\n";
-  // per-slot phase tables and the fixed-order dY reduction over the roles
-  o << "__device__ const int kPh[" << S * NW << "] = {";
-  for (int s = 0; s < S; ++s)
-    for (int w = 0; w < NW; ++w)
-      o << (w < (int)F.slice_roles[s].size() ? P.bwd_roles[F.slice_roles[s][w]].ph : -1) << ",";
-  o << "};\n__device__ const int kNph[" << S * NW << "] = {";
-  for (int s = 0; s < S; ++s)
-    for (int w = 0; w < NW; ++w)
-      o << (w < (int)F.slice_roles[s].size() ? P.bwd_roles[F.slice_roles[s][w]].nph : 1) << ",";
-  o << "};\n";
-  o << "__device__ __forceinline__ void dy_reduce(const float* __restrict__ sdyall, float* __restrict__ dys,\n"
-       "    int slice, int eb, int nb) {\n"
-       "  for (int t = threadIdx.x; t < nb * DE; t += NW * 32) {\n"
-       "    const int b = t / DE, k = t - b * DE;\n"
-       "    float v = 0.f;\n"
-       "    for (int w = 0; w < NW; ++w) {\n"
-       "      const int ph = kPh[slice * NW + w];\n"
-       "      if (ph >= 0 && b % kNph[slice * NW + w] == ph) v += sdyall[(w * NB + b) * DE + k];\n"
-       "    }\n"
-       "    dys[(size_t)(eb + b) * DE + k] = v;\n"
-       "  }\n"
-       "}\n";
-
-  // one consumer function per (irrep, R); channel block and phase at run time
-  std::vector<int> shape_of(P.bwd_roles.size(), -1), shape_rep;
   std::vector<int> slice_of(P.bwd_roles.size(), -1);
   for (int s = 0; s < S; ++s)
     for (int v : F.slice_roles[s]) slice_of[v] = s;
+  std::vector<int> shape_of(P.bwd_roles.size(), -1), shape_rep;
   for (size_t ri = 0; ri < P.bwd_roles.size(); ++ri) {
     const BwdRole& r = P.bwd_roles[ri];
     for (size_t k = 0; k < shape_rep.size(); ++k) {
@@ -128,92 +76,88 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       shape_rep.push_back((int)ri);
     }
   }
-  const std::string loop_head =
-      "  const int lane = threadIdx.x & 31;\n"
-      "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
-      "  const int nchunk = (e1 - e0 + NB - 1) / NB;\n"
-      "  float* sdyall = reinterpret_cast<float*>(smem + OFF_DY);\n"
-      "  bool dead = false;\n"
-      "  for (int c = 0; c < nchunk; ++c) {\n"
-      "    const int s = c % NSTAGE;\n"
-      "    if (!dead && !mbar_wait(full0 + 8 * s, (c / NSTAGE) & 1)) { dead = true; if (lane == 0) atomicOr(err, 10); }\n"
-      "    const int eb = e0 + c * NB;\n"
-      "    const int nb = min(NB, e1 - eb);\n"
-      "    unsigned char* st = smem + OFF_STAGE + s * STAGE_BYTES;\n"
-      "    const float* sY = reinterpret_cast<const float*>(st + W_BYTES + X_BYTES);\n"
-      "    float* ch = reinterpret_cast<float*>(smem + OFF_CH) + (c & 1) * NB * CHS;\n"
-      "    if (!dead) chat_build(sent, nent, term, sY, ch, chs, nb, threadIdx.x);\n"
-      "    consumer_bar(NW * 32);\n";
-  const std::string loop_tail =
-      "    consumer_bar(NW * 32);\n"
-      "    if (!dead && dys) dy_reduce(sdyall, dys, slice, eb, nb);\n"
-      "    __syncwarp();\n"
-      "    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n"
-      "  }\n";
   const std::string params =
-      "(const int* __restrict__ col, const float* __restrict__ x, const float* __restrict__ W,\n"
-      "    float* __restrict__ dW, float* __restrict__ msg, float* __restrict__ dys,\n"
-      "    const int4* __restrict__ sent, int nent, const int2* __restrict__ term, int* __restrict__ err,\n"
-      "    unsigned char* smem, const float* __restrict__ sg, int slice, int e0, int e1, int u0, int ph,\n"
-      "    int nph, int chs)";
+      "(const int* __restrict__ rowptr, int n_recv, float* __restrict__ dW, float* __restrict__ msg,\n"
+      "    int* __restrict__ err, unsigned char* smem, int u0, int ph, int nph, int chs, bool want_dy)";
   for (size_t k = 0; k < shape_rep.size(); ++k) {
     const BwdRole& r = P.bwd_roles[shape_rep[k]];
     const SliceLayout& sl = SL[slice_of[shape_rep[k]]];
     const Irrep& h = P.in[r.irrep];
     const int N1 = 2 * h.l + 1, R = r.R, MUL = h.mul;
-    const int xoff = F.x_smem ? sl.x_st.at(r.irrep) : P.x_off[r.irrep];
     std::vector<int> ps;
     for (size_t q = 0; q < P.paths.size(); ++q)
       if (P.paths[q].irrep == r.irrep) ps.push_back((int)q);
     o << "// shape " << k << ": irrep " << r.irrep << " (" << h.mul << "x" << h.l << "), R=" << R << ", "
       << ps.size() << " paths\n";
-    o << "__device__ __noinline__ void bcons_" << k << params << " {\n" << loop_head;
-    o << "    bool ok[" << R << "];\n"
-      << "#pragma unroll\n    for (int r = 0; r < " << R << "; ++r) ok[r] = u0 + r * 32 + lane < " << MUL << ";\n"
-      << "    if (!dead) {\n"
-      << "      for (int b = ph; b < nb; b += nph) {\n"
-      << "        const int e = eb + b;\n";
-    if (F.w_smem)
-      o << "        const float* wr = reinterpret_cast<const float*>(st) + b * NU;\n";
-    else
-      o << "        const float* wr = W + (size_t)e * NU;\n";
-    if (F.x_smem)
-      o << "        const float* xr = reinterpret_cast<const float*>(st + W_BYTES) + b * XS + " << xoff << ";\n";
-    else
-      o << "        const float* xr = x + (size_t)col[e] * DIN + " << xoff << ";\n";
-    o << "        const float* chb = ch + b * chs;\n"
-      << "        float* dWrow = dW ? dW + (size_t)e * NU : nullptr;\n"
-      << "        float* sdy = dys ? sdyall + ((threadIdx.x >> 5) * NB + b) * DE : nullptr;\n"
-      << "        float xv[" << R << "][" << N1 << "], mx[" << R << "][" << N1 << "];\n"
-      << "#pragma unroll\n        for (int r = 0; r < " << R << "; ++r) {\n"
-      << "          const int u = u0 + r * 32 + lane;\n"
-      << "#pragma unroll\n          for (int m1 = 0; m1 < " << N1
-      << "; ++m1) { mx[r][m1] = 0.f; xv[r][m1] = ok[r] ? LDX(xr + u * " << N1 << " + m1) : 0.f; }\n"
-      << "        }\n";
+    o << "__device__ __noinline__ void bcons_" << k << params << " {\n"
+      << "  const int lane = threadIdx.x & 31;\n"
+      << "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
+      << "  const u32 gfull0 = full0 + 2 * NSTAGE * 8, gempty0 = gfull0 + 16;\n"
+      << "  bool ok[" << R << "];\n"
+      << "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) ok[r] = u0 + r * 32 + lane < " << MUL << ";\n"
+      << "  int q = 0, kr = 0;\n"
+      << "#pragma unroll 1\n  for (int i = cta_first(smem); i < n_recv; i += cta_stride(smem)) {\n"
+      << "  const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
+      << "  if (e1 == e0) continue;\n"
+      << "  const int gb = kr & 1;\n"
+      << "  if (!mbar_wait(gfull0 + 8 * gb, (kr >> 1) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
+      << "  const float* sg = reinterpret_cast<const float*>(smem + OFF_G) + gb * GS;\n"
+      << "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
+      << "    const int s = q % NSTAGE;\n"
+      << "    if (!mbar_wait(full0 + 8 * s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
+      << "    const int nb = min(NB, e1 - eb);\n"
+      << "    unsigned char* st = stage_ptr(smem, s);\n"
+      << "    const float* sW = reinterpret_cast<const float*>(st + OFF_W);\n"
+      << "    const float* sX = reinterpret_cast<const float*>(st + OFF_X) + " << sl.x_st.at(r.irrep) << ";\n"
+      << "    const float* sC = reinterpret_cast<const float*>(st + OFF_CH);\n"
+      << "    float* sdyw = reinterpret_cast<float*>(st + OFF_DY) + (threadIdx.x >> 5) * NB * DE;\n"
+      << "#pragma unroll 1\n    for (int b = ph; b < nb; b += nph) {\n"
+      << "      const int e = eb + b;\n"
+      << "      const float* wr = sW + b * WS;\n"
+      << "      const float* xr = sX + b * XS;\n"
+      << "      const float* chb = sC + b * chs;\n"
+      << "      float* dWrow = dW ? dW + (size_t)e * NU : nullptr;\n"
+      << "      float* sdy = want_dy ? sdyw + b * DE : nullptr;\n"
+      << "      float xv[" << R << "][" << N1 << "], mx[" << R << "][" << N1 << "];\n"
+      << "#pragma unroll\n      for (int r = 0; r < " << R << "; ++r) {\n"
+      << "        const int u = u0 + r * 32 + lane;\n"
+      << "#pragma unroll\n        for (int m1 = 0; m1 < " << N1
+      << "; ++m1) { mx[r][m1] = 0.f; xv[r][m1] = ok[r] ? xr[u * " << N1 << " + m1] : 0.f; }\n"
+      << "      }\n";
+    // dY partials: one vector over every edge degree (reduced once) when
+    // (L+1)^2 <= 32, else one vector per edge degree
+    auto pow2 = [](int n) { int v = 1; while (v < n) v <<= 1; return v; };
+    const bool combined = P.D_e <= 32;
+    const int VZ = pow2((int)P.D_e);
+    if (combined)
+      o << "      float z[" << VZ << "];\n#pragma unroll\n      for (int t = 0; t < " << VZ << "; ++t) z[t] = 0.f;\n";
     std::vector<char> l2seen(P.L + 1, 0);
     size_t q = 0;
     while (q < ps.size()) {
       const int l2 = P.paths[ps[q]].l2;
       const int N2 = 2 * l2 + 1;
+      const int zo = combined ? l2 * l2 : 0;  // offset of degree l2 inside z
       l2seen[l2] = 1;
-      o << "        {\n          float z[" << N2 << "];\n#pragma unroll\n          for (int t = 0; t < " << N2
-        << "; ++t) z[t] = 0.f;\n";
+      o << "      {\n";
+      if (!combined)
+        o << "        float z[" << pow2(N2) << "];\n#pragma unroll\n        for (int t = 0; t < " << pow2(N2)
+          << "; ++t) z[t] = 0.f;\n";
       for (; q < ps.size() && P.paths[ps[q]].l2 == l2; ++q) {
         const int pi = ps[q];
         const Path& p = P.paths[pi];
         const int N3 = 2 * p.l3 + 1, n2 = 2 * p.l2 + 1;
-        o << "          {\n            float w[" << R << "], gv[" << R << "][" << N3 << "], hh[" << R << "][" << N3
+        o << "        {\n          float w[" << R << "], gv[" << R << "][" << N3 << "], hh[" << R << "][" << N3
           << "], dw[" << R << "];\n"
-          << "#pragma unroll\n            for (int r = 0; r < " << R << "; ++r) {\n"
-          << "              const int u = u0 + r * 32 + lane;\n"
-          << "              w[r] = ok[r] ? LDW(wr + " << p.k0 << " + u) : 0.f;\n"
-          << "#pragma unroll\n              for (int m3 = 0; m3 < " << N3 << "; ++m3) gv[r][m3] = ok[r] ? sg["
-          << sl.g_st.at(pi) << " + u * " << N3 << " + m3] : 0.f;\n            }\n"
-          << "            bpath<" << N1 << "," << N3 << "," << R << ">(chb + " << sl.ch_off.at(pi)
+          << "#pragma unroll\n          for (int r = 0; r < " << R << "; ++r) {\n"
+          << "            const int u = u0 + r * 32 + lane;\n"
+          << "            w[r] = ok[r] ? wr[" << sl.w_st.at(pi) << " + u] : 0.f;\n"
+          << "#pragma unroll\n            for (int m3 = 0; m3 < " << N3 << "; ++m3) gv[r][m3] = ok[r] ? sg["
+          << sl.g_st.at(pi) << " + u * " << N3 << " + m3] : 0.f;\n          }\n"
+          << "          bpath<" << N1 << "," << N3 << "," << R << ">(chb + " << sl.ch_off.at(pi)
           << ", xv, w, gv, hh, mx, dw);\n"
-          << "            if (dWrow) {\n#pragma unroll\n              for (int r = 0; r < " << R
-          << "; ++r) if (ok[r]) dWrow[" << p.k0 << " + u0 + r * 32 + lane] = dw[r];\n            }\n"
-          << "            if (sdy) {\n#pragma unroll\n              for (int r = 0; r < " << R << "; ++r) {\n";
+          << "          if (dWrow) {\n#pragma unroll\n            for (int r = 0; r < " << R
+          << "; ++r) if (ok[r]) dWrow[" << p.k0 << " + u0 + r * 32 + lane] = dw[r];\n          }\n"
+          << "          if (sdy) {\n#pragma unroll\n            for (int r = 0; r < " << R << "; ++r) {\n";
         const double* C = P.coeff.data() + p.c_off;
         for (int m1 = 0; m1 < N1; ++m1)
           for (int m3 = 0; m3 < N3; ++m3) {
@@ -223,72 +167,113 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
               if (c != 0.0) t.push_back({m2, c});
             }
             if (t.empty()) continue;
-            o << "                { const float pr = xv[r][" << m1 << "] * hh[r][" << m3 << "];";
+            o << "              { const float pr = xv[r][" << m1 << "] * hh[r][" << m3 << "];";
             for (auto& tc : t)
-              o << " z[" << tc.first << "] = fmaf(" << flt(tc.second) << ", pr, z[" << tc.first << "]);";
+              o << " z[" << zo + tc.first << "] = fmaf(" << flt(tc.second) << ", pr, z[" << zo + tc.first << "]);";
             o << " }\n";
           }
-        o << "              }\n            }\n          }\n";
+        o << "            }\n          }\n        }\n";
       }
-      o << "          if (sdy) {\n#pragma unroll\n            for (int t = 0; t < " << N2
-        << "; ++t) { const float v = warp_sum(z[t]); if (lane == 0) sdy[" << l2 * l2 << " + t] = v; }\n"
-        << "          }\n        }\n";
+      if (!combined) {
+        const int V = pow2(N2), LV = __builtin_ctz(V), sh = 5 - LV;
+        o << "        if (sdy) {\n          const float v = warp_sum_many<" << V << ">(z, lane);\n"
+          << "          const int k = lane >> " << sh << ";\n"
+          << "          if ((lane & " << ((1 << sh) - 1) << ") == 0 && k < " << N2 << ") sdy[" << l2 * l2
+          << " + k] = v;\n        }\n";
+      }
+      o << "      }\n";
     }
-    for (int l2 = 0; l2 <= P.L; ++l2)
-      if (!l2seen[l2])
-        o << "        if (sdy && lane == 0) {\n#pragma unroll\n          for (int t = 0; t < " << 2 * l2 + 1
-          << "; ++t) sdy[" << l2 * l2 << " + t] = 0.f;\n        }\n";
-    o << "        if (msg) {\n#pragma unroll\n          for (int r = 0; r < " << R
-      << "; ++r) if (ok[r]) {\n            const int u = u0 + r * 32 + lane;\n"
-      << "#pragma unroll\n            for (int m1 = 0; m1 < " << N1 << "; ++m1) msg[(size_t)e * DIN + "
-      << P.x_off[r.irrep] << " + u * " << N1 << " + m1] = mx[r][m1];\n          }\n        }\n";
-    o << "      }\n    }\n" << loop_tail << "}\n";
+    if (combined) {
+      const int LV = __builtin_ctz(VZ), sh = 5 - LV;
+      o << "      if (sdy) {\n        const float v = warp_sum_many<" << VZ << ">(z, lane);\n"
+        << "        const int k = lane >> " << sh << ";\n"
+        << "        if ((lane & " << ((1 << sh) - 1) << ") == 0 && k < DE) sdy[k] = v;\n      }\n";
+    } else {
+      for (int l2 = 0; l2 <= P.L; ++l2)
+        if (!l2seen[l2])
+          o << "      if (sdy && lane == 0) {\n#pragma unroll\n        for (int t = 0; t < " << 2 * l2 + 1
+            << "; ++t) sdy[" << l2 * l2 << " + t] = 0.f;\n      }\n";
+    }
+    // the message row segment of this role, through the warp's buffer
+    o << "      if (msg) {\n"
+      << "        float* wbuf = reinterpret_cast<float*>(smem + OFF_WB) + (threadIdx.x >> 5) * WB;\n"
+      << "#pragma unroll\n        for (int r = 0; r < " << R << "; ++r) {\n"
+      << "#pragma unroll\n          for (int m1 = 0; m1 < " << N1 << "; ++m1) wbuf[(r * 32 + lane) * " << N1
+      << " + m1] = mx[r][m1];\n        }\n"
+      << "        __syncwarp();\n"
+      << "        warp_copy_out(msg + (size_t)e * DIN + " << P.x_off[r.irrep] << " + u0 * " << N1
+      << ", wbuf, min(" << 32 * R << ", " << MUL << " - u0) * " << N1 << ", lane);\n"
+      << "        __syncwarp();\n      }\n";
+    o << "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n"
+      << "  __syncwarp();\n  if (lane == 0) mbar_arrive(gempty0 + 8 * gb);\n  ++kr;\n  }\n}\n";
   }
-  o << "__device__ __noinline__ void bcons_idle" << params << " {\n" << loop_head << loop_tail << "}\n";
-
-  o << "__device__ const int kShape[" << S * NW << "] = {";
+  o << "__device__ __noinline__ void bcons_idle" << params << " {\n"
+       "  const int lane = threadIdx.x & 31;\n"
+       "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
+       "  const u32 gempty0 = full0 + 2 * NSTAGE * 8 + 16;\n"
+       "  int q = 0, kr = 0;\n"
+       "#pragma unroll 1\n  for (int i = cta_first(smem); i < n_recv; i += cta_stride(smem)) {\n"
+       "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
+       "    if (e1 == e0) continue;\n"
+       "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
+       "      const int s = q % NSTAGE;\n"
+       "      if (!mbar_wait(full0 + 8 * s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
+       "      __syncwarp();\n"
+       "      if (lane == 0) mbar_arrive(empty0 + 8 * s);\n"
+       "    }\n"
+       "    if (lane == 0) mbar_arrive(gempty0 + 8 * (kr & 1));\n"
+       "    ++kr;\n"
+       "  }\n"
+       "}\n";
+  o << "__constant__ int kShape[" << S * NW << "] = {";
   for (int s = 0; s < S; ++s)
     for (int w = 0; w < NW; ++w)
       o << (w < (int)F.slice_roles[s].size() ? shape_of[F.slice_roles[s][w]] : -1) << ",";
-  o << "};\n__device__ const int kU0[" << S * NW << "] = {";
+  o << "};\n__constant__ int kU0[" << S * NW << "] = {";
   for (int s = 0; s < S; ++s)
     for (int w = 0; w < NW; ++w)
       o << (w < (int)F.slice_roles[s].size() ? P.bwd_roles[F.slice_roles[s][w]].u0 : 0) << ",";
-  o << "};\n__device__ const int kEntBegin[" << S + 1 << "] = {";
+  o << "};\n__constant__ int kEntBegin[" << S + 1 << "] = {";
   for (int v : P.bwd_ent_begin) o << v << ",";
   o << "};\n";
-  o << "extern \"C\" __global__ void __launch_bounds__((NW + 1) * 32) " << kname
+  // resident CTAs to plan registers for: as many as shared memory allows (at
+  // most 3), or CGTP_MIN_BLOCKS when set (1 leaves registers uncapped)
+  int min_blocks = std::max(1, std::min(3, (228 * 1024) / (K.smem + 1024)));
+  if (const char* mb = std::getenv("CGTP_MIN_BLOCKS")) min_blocks = std::max(1, std::atoi(mb));
+  o << "extern \"C\" __global__ void __launch_bounds__((NW + 2) * 32, " << min_blocks << ") " << kname
     << "(const int* __restrict__ rowptr, const int* __restrict__ col, const float* __restrict__ x,\n"
        "    const float* __restrict__ Y, const float* __restrict__ W, const float* __restrict__ g,\n"
        "    float* __restrict__ dW, float* __restrict__ dyp, float* __restrict__ msg,\n"
-       "    const int4* __restrict__ ent, const int2* __restrict__ term, int* __restrict__ err) {\n"
+       "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err, const SliceGrid sgrid) {\n"
        "  extern __shared__ __align__(128) unsigned char smem[];\n"
-       "  const int i = blockIdx.x, slice = blockIdx.y;\n"
+       "  (void)0;\n"
        "  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;\n"
-       "  const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
+       "  const u32 gfull0 = full0 + 2 * NSTAGE * 8, gempty0 = gfull0 + 16;\n"
        "  if (threadIdx.x == 0) {\n"
-       "    for (int s = 0; s < NSTAGE; ++s) { mbar_init(full0 + 8 * s, 32); mbar_init(empty0 + 8 * s, NW); }\n"
+       "    for (int s = 0; s < NSTAGE; ++s) { mbar_init(full0 + 8 * s, FULL_COUNT); mbar_init(empty0 + 8 * s, NW); }\n"
+       "    for (int b = 0; b < 2; ++b) { mbar_init(gfull0 + 8 * b, 32); mbar_init(gempty0 + 8 * b, NW); }\n"
        "    fence_mbar_init();\n"
+       "    cta_place(smem, sgrid);\n"
        "  }\n"
        "  __syncthreads();\n"
-       "  if (e1 == e0) return;\n"
-       "  if (warp == NW) { producer(col, x, Y, W, err, smem, slice, e0, e1, lane); return; }\n"
-       "  float* sg = reinterpret_cast<float*>(smem + OFF_G);\n"
-       "  stage_g(slice, g + (size_t)i * DOUT, sg, threadIdx.x);\n"
-       "  const int E = rowptr[gridDim.x];\n"
-       "  float* dys = dyp ? dyp + (size_t)slice * E * DE : nullptr;\n"
-       "  const int4* sent = ent + kEntBegin[slice];\n"
-       "  const int nent = kEntBegin[slice + 1] - kEntBegin[slice];\n"
+       "  const int slice = reinterpret_cast<const int*>(smem + 240)[2];\n"
        "  const int chs = slice_chs(slice);\n"
+       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, g, err, smem, slice, lane); return; }\n"
+       "  if (warp == NW + 1) {\n"
+       "    const int E = rowptr[n_recv];\n"
+       "    float* dys = dyp ? dyp + (size_t)slice * E * DE : nullptr;\n"
+       "    helper_warp(rowptr, n_recv, Y, ent + kEntBegin[slice], kEntBegin[slice + 1] - kEntBegin[slice],\n"
+       "                dys, err, smem, slice, chs, lane);\n"
+       "    return;\n"
+       "  }\n"
        "  const int slot = slice * NW + warp;\n"
        "  const int u0 = kU0[slot], ph = kPh[slot], nph = kNph[slot];\n"
        "  switch (kShape[slot]) {\n";
   for (size_t k = 0; k < shape_rep.size(); ++k)
     o << "  case " << k << ": bcons_" << k
-      << "(col, x, W, dW, msg, dys, sent, nent, term, err, smem, sg, slice, e0, e1, u0, ph, nph, chs); break;\n";
-  o << "  default: bcons_idle(col, x, W, dW, msg, dys, sent, nent, term, err, smem, sg, slice, e0, e1, u0, ph, nph, chs); break;\n"
-       "  }\n}\n";
+      << "(rowptr, n_recv, dW, msg, err, smem, u0, ph, nph, chs, dyp != nullptr); break;\n";
+  o << "  default: bcons_idle(rowptr, n_recv, dW, msg, err, smem, u0, ph, nph, chs, dyp != nullptr); break;\n  }\n}\n";
   return o.str();
 }
 
@@ -297,13 +282,12 @@ cgtp_status build_backward(Plan& P) {
   FwdConfig& F = P.bcfg;
   F = FwdConfig();
   if (P.paths.empty()) return CGTP_OK;
-  // cost of one channel block of each irrep per edge
+  // one slice per hidden irrep with paths; roles = channel blocks x edge phases
   struct IrrepWork {
     int a, R, nblk;
     double cost;
   };
   std::vector<IrrepWork> iw;
-  double total = 0.0;
   for (size_t a = 0; a < P.in.size(); ++a) {
     const Irrep& h = P.in[a];
     const int n1 = 2 * h.l + 1;
@@ -322,20 +306,17 @@ cgtp_status build_backward(Plan& P) {
     const int R = (h.mul >= 64 && h.l <= 3) ? 2 : 1;
     const int nblk = (h.mul + 32 * R - 1) / (32 * R);
     iw.push_back({(int)a, R, nblk, c * R});
-    total += nblk * c * R;
   }
-  const int kMaxWarps = 16;
-  int maxnph = 4;
   std::vector<SliceLayout> SL;
+  KernelShape K;
+  int maxnph = 4;
   for (int attempt = 0; attempt < 3; ++attempt) {
     P.bwd_roles.clear();
-    const double tau = total / kMaxWarps;
-    const bool fits_one = (long)P.D_out * 4 <= 64 * 1024;
+    F.slice_roles.clear();
     for (auto& w : iw) {
-      int nph = fits_one ? (int)std::lround(w.cost / std::max(tau, 1e-9))
-                         : std::max(1, 8 / w.nblk);
-      nph = std::max(1, std::min(maxnph, nph));
+      int nph = std::max(1, std::min(maxnph, 8 / std::max(1, w.nblk)));
       while (nph & (nph - 1)) --nph;  // 1, 2 or 4
+      F.slice_roles.push_back({});
       for (int blk = 0; blk < w.nblk; ++blk)
         for (int ph = 0; ph < nph; ++ph) {
           BwdRole r;
@@ -345,95 +326,43 @@ cgtp_status build_backward(Plan& P) {
           r.ph = ph;
           r.nph = nph;
           r.cost = w.cost / nph;
+          F.slice_roles.back().push_back((int)P.bwd_roles.size());
           P.bwd_roles.push_back(r);
         }
     }
-    const int NR = (int)P.bwd_roles.size();
-    // one slice holding every role when it fits in a CTA (the receiver's
-    // whole g row staged once), otherwise one slice per hidden irrep
-    const bool one = NR <= kMaxWarps && (long)P.D_out * 4 <= 64 * 1024;
-    F.slice_roles.clear();
-    if (one) {
-      F.slice_roles.assign(1, {});
-      for (int ri = 0; ri < NR; ++ri) F.slice_roles[0].push_back(ri);
-    } else {
-      for (auto& w : iw) {
-        F.slice_roles.push_back({});
-        for (int ri = 0; ri < NR; ++ri)
-          if (P.bwd_roles[ri].irrep == w.a) F.slice_roles.back().push_back(ri);
-      }
-    }
     F.S = (int)F.slice_roles.size();
-    for (auto& v : F.slice_roles) std::sort(v.begin(), v.end());
+    F.weight.clear();
+    for (auto& w : iw) F.weight.push_back(w.cost * w.nblk);
     F.nw = 0;
     for (auto& v : F.slice_roles) F.nw = std::max<int>(F.nw, (int)v.size());
-    // layouts
     SL.assign(F.S, SliceLayout());
     for (int s = 0; s < F.S; ++s) {
-      SliceLayout& sl = SL[s];
-      std::vector<char> iseen(P.in.size(), 0);
-      for (int ri : F.slice_roles[s]) iseen[P.bwd_roles[ri].irrep] = 1;
+      const int a = iw[s].a;
+      SL[s].irreps.push_back(a);
       for (size_t k = 0; k < P.paths.size(); ++k)
-        if (iseen[P.paths[k].irrep]) {
-          sl.paths.push_back((int)k);
-          sl.ch_off[(int)k] = sl.chs;
-          sl.chs += chat_size(P.paths[k].l1, P.paths[k].l3);
-        }
-      for (size_t a = 0; a < P.in.size(); ++a)
-        if (iseen[a]) {
-          sl.irreps.push_back((int)a);
-          sl.x_st[(int)a] = sl.xs;
-          sl.xs += pad4(P.in[a].mul * (2 * P.in[a].l + 1));
-        }
-      // g blocks: with every path of the plan in the slice, the row is copied
-      // as is; otherwise the slice's path blocks are packed
-      if (sl.paths.size() == P.paths.size()) {
-        for (int pi : sl.paths) sl.g_st[pi] = P.paths[pi].o_off;
-        sl.gs = (int)P.D_out;
-      } else {
-        for (int pi : sl.paths) {
-          sl.g_st[pi] = sl.gs;
-          sl.gs += P.paths[pi].mul * (2 * P.paths[pi].l3 + 1);
-        }
-      }
+        if (P.paths[k].irrep == a) SL[s].paths.push_back((int)k);
+      layout_slice(P, SL[s], true);
     }
-    F.w_smem = (F.S == 1) && (P.U % 4 == 0);
-    F.x_smem = (P.D_in % 4 == 0);
-    for (int s = 0; s < F.S && F.x_smem; ++s)
-      for (int a : SL[s].irreps)
-        if (P.x_off[a] % 4 != 0 || (P.in[a].mul * (2 * P.in[a].l + 1)) % 4 != 0) F.x_smem = false;
-    if (!F.x_smem)
-      for (auto& sl : SL) {
-        sl.xs = 0;
-        for (int a : sl.irreps) sl.x_st[a] = P.x_off[a];
-      }
-    int CHS = 0, XS = 0, GS = 0;
-    for (auto& sl : SL) {
-      CHS = std::max(CHS, sl.chs);
-      XS = std::max(XS, sl.xs);
-      GS = std::max(GS, sl.gs);
-    }
-    const long pe = (F.w_smem ? P.U * 4 : 0) + (F.x_smem ? XS * 4 : 0) + P.D_e * 4 + 64;
-    const long fixed = (long)GS * 4 + 1024;
-    const long budget = std::max<long>(100 * 1024, fixed + 40 * 1024);
-    F.B = 4;
-    auto per_b = [&](int b) { return 2L * b * CHS * 4 + (long)F.nw * b * P.D_e * 4 + 2L * b * pe; };
-    while (F.B > 1 && fixed + per_b(F.B) > budget) F.B /= 2;
-    F.stages = (int)std::min<long>(
-        8, std::max<long>(2, (budget - fixed - 2L * F.B * CHS * 4 - (long)F.nw * F.B * P.D_e * 4) /
-                                 (F.B * pe)));
-    if (F.B >= maxnph) break;
-    maxnph = F.B;
+    K = KernelShape();
+    K.S = F.S;
+    K.nw = F.nw;
+    for (auto& r : P.bwd_roles) K.WB = std::max(K.WB, 32 * r.R * (2 * P.in[r.irrep].l + 1));
+    plan_layout(P, SL, K, true);
+    if (K.B >= maxnph) break;
+    maxnph = K.B;
   }
+  F.B = K.B;
+  F.stages = K.stages;
+  F.w_smem = K.w_bulk;
+  F.x_smem = K.x_bulk;
 
   cgtp_status st = upload_chat_tables(P, SL, &P.d_bwd_ent, &P.d_bwd_term, P.bwd_ent_begin);
   if (st != CGTP_OK) return st;
-  int smem = 0;
   const std::string name = "cgtp_bwd";
-  std::string src = gen_bwd_source(P, SL, name, smem);
-  if (smem > 227 * 1024) return fail(CGTP_ERR_SIZE, "backward kernel needs too much shared memory");
-  P.bwd.threads = (F.nw + 1) * 32;
-  P.bwd.smem = smem;
+  std::string src = gen_bwd_source(P, SL, K, name);
+  if (K.smem > 227 * 1024) return fail(CGTP_ERR_SIZE, "backward kernel needs too much shared memory");
+  P.bwd.threads = (F.nw + 2) * 32;
+  P.bwd.smem = K.smem;
   if (const char* d = std::getenv("CGTP_DUMP_SOURCE")) {
     FILE* f = std::fopen((std::string(d) + "/bwd.cu").c_str(), "w");
     if (f) {

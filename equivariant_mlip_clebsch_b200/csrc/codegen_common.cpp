@@ -1,7 +1,25 @@
-// codegen_common.cpp -- device prelude text and the Chat build tables.
+// codegen_common.cpp -- staging layouts, the Chat tables and the two service
+// warps shared by the generated forward and backward kernels.
+//
+// Warp organisation of both kernels (one CTA = one receiver x one slice of
+// the warp roles):
+//   warps 0..NW-1  consumers: pure compute on staged data
+//   warp NW        TMA warp: per chunk of NB edges, bulk copies (cp.async.bulk,
+//                  completion counted in bytes on the stage's "full" mbarrier)
+//                  of the W and x row pieces the slice needs; pieces that are
+//                  not 16-byte aligned are copied with plain loads instead.
+//                  The backward's grad_out row pieces are staged once per CTA.
+//   warp NW+1      helper warp: loads the chunk's Y rows and builds
+//                  Chat_{e,p} = sum_m2 C_p[m1][m2][m3] Y[e][m2] into the stage;
+//                  in the backward it also sums the consumers' dY partials of
+//                  each released stage in a fixed order and stores them.
+// A stage is released ("empty" mbarrier, one arrival per consumer warp)
+// after the consumers finish it.  All waits are bounded.
 #include "codegen_common.hpp"
 
+#include <algorithm>
 #include <cstring>
+#include <sstream>
 
 namespace cgtp {
 
@@ -9,12 +27,350 @@ const char* kPrelude =
 #include "device_prelude.inc"
     ;
 
-// One entry per Chat element that some role reads: (dst offset inside the
-// edge's Chat block, first term, number of terms); one term per non-zero
-// C_p[m1][m2][m3]: (column l2^2+m2 of Y, coefficient as FP32 bits).
+static void merge_segment(std::vector<Segment>& v, Segment s) {
+  if (!v.empty() && v.back().src + v.back().len == s.src && v.back().dst + v.back().len == s.dst)
+    v.back().len += s.len;
+  else
+    v.push_back(s);
+}
+
+bool segments_aligned(const std::vector<Segment>& segs, long row_len) {
+  if (row_len % 4) return false;
+  for (const auto& s : segs)
+    if (s.src % 4 || s.dst % 4 || s.len % 4) return false;
+  return true;
+}
+
+void layout_slice(const Plan& P, SliceLayout& sl, bool with_g) {
+  sl.ch_off.clear();
+  sl.chs = 0;
+  for (int pi : sl.paths) {
+    sl.ch_off[pi] = sl.chs;
+    sl.chs += chat_size(P.paths[pi].l1, P.paths[pi].l3);
+  }
+  sl.x_st.clear();
+  sl.xseg.clear();
+  sl.xs = 0;
+  for (int a : sl.irreps) {
+    const int n = P.in[a].mul * (2 * P.in[a].l + 1);
+    sl.x_st[a] = sl.xs;
+    merge_segment(sl.xseg, {P.x_off[a], sl.xs, n});
+    sl.xs += pad4(n);
+  }
+  // W pieces: every channel of every path of the slice, in column order
+  std::vector<int> byk = sl.paths;
+  std::sort(byk.begin(), byk.end(), [&](int a, int b) { return P.paths[a].k0 < P.paths[b].k0; });
+  sl.w_st.clear();
+  sl.wseg.clear();
+  sl.ws = 0;
+  for (int pi : byk) {
+    const Path& p = P.paths[pi];
+    sl.w_st[pi] = sl.ws;
+    merge_segment(sl.wseg, {p.k0, sl.ws, p.mul});
+    sl.ws += pad4(p.mul);
+  }
+  sl.g_st.clear();
+  sl.gseg.clear();
+  sl.gs = 0;
+  if (with_g) {
+    std::vector<int> byo = sl.paths;
+    std::sort(byo.begin(), byo.end(), [&](int a, int b) { return P.paths[a].o_off < P.paths[b].o_off; });
+    for (int pi : byo) {
+      const Path& p = P.paths[pi];
+      const int n = p.mul * (2 * p.l3 + 1);
+      sl.g_st[pi] = sl.gs;
+      merge_segment(sl.gseg, {p.o_off, sl.gs, n});
+      sl.gs += pad4(n);
+    }
+  }
+}
+
+void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape& K, bool backward) {
+  K.WS = K.XS = K.CHS = K.GS = 0;
+  K.w_bulk = K.x_bulk = K.g_bulk = true;
+  for (const auto& sl : SL) {
+    K.WS = std::max(K.WS, sl.ws);
+    K.XS = std::max(K.XS, sl.xs);
+    K.CHS = std::max(K.CHS, sl.chs);
+    K.GS = std::max(K.GS, sl.gs);
+    K.w_bulk = K.w_bulk && segments_aligned(sl.wseg, P.U);
+    K.x_bulk = K.x_bulk && segments_aligned(sl.xseg, P.D_in);
+    K.g_bulk = K.g_bulk && segments_aligned(sl.gseg, P.D_out);
+  }
+  auto r128 = [](long v) { return (int)((v + 127) & ~127L); };
+  auto stage_of = [&](int B) {
+    long b = r128(4L * B * K.WS) + r128(4L * B * K.XS) + r128(4L * B * P.D_e) + r128(4L * B * K.CHS);
+    if (backward) b += r128(4L * K.nw * B * P.D_e);
+    return b;
+  };
+  const long fixed = 256 + (backward ? 2L * r128(4L * K.GS) : 0)  // two grad_out buffers
+                     + r128(4L * K.nw * K.WB);                      // store staging
+  // two or three CTAs per SM when it fits, at least two stages in flight
+  // wide rows (Lmax 6) may take up to half an SM to keep two edges per chunk
+  const long budget =
+      std::max<long>(72 * 1024, std::min<long>(112 * 1024, fixed + 2 * stage_of(2)));
+  K.B = 4;
+  while (K.B > 1 && fixed + 2 * stage_of(K.B) > budget) K.B /= 2;
+  K.stages = (int)std::min<long>(6, std::max<long>(2, (budget - fixed) / stage_of(K.B)));
+  K.sdy_floats = backward ? K.nw * K.B * (int)P.D_e : 0;
+  K.off_stage = 256;  // mbarriers first
+  K.off_w = 0;
+  K.off_x = r128(4L * K.B * K.WS);
+  K.off_y = K.off_x + r128(4L * K.B * K.XS);
+  K.off_ch = K.off_y + r128(4L * K.B * P.D_e);
+  K.off_dy = K.off_ch + r128(4L * K.B * K.CHS);
+  K.stage_bytes = K.off_dy + (backward ? r128(4L * K.sdy_floats) : 0);
+  K.off_g = K.off_stage + K.stages * K.stage_bytes;
+  K.off_wb = K.off_g + (backward ? 2 * r128(4L * K.GS) : 0);
+  K.smem = K.off_wb + r128(4L * K.nw * K.WB);
+}
+
+// bulk-or-plain copy of row pieces for the edges of a chunk.  Bulk copies are
+// issued by lane b for edge b; plain copies are spread over the warp.
+static void gen_copy_pieces(std::ostringstream& o, const std::vector<Segment>& segs, bool bulk,
+                            const std::string& dst_row /* float* of edge 0 */, int stride,
+                            const std::string& src_row /* expression of b */, const std::string& bar,
+                            bool one_block, long row_len) {
+  if (bulk && one_block) {
+    // staged rows identical to the global rows: one copy for the chunk
+    o << "      if (lane == 0) bulk_g2s_stream(smem_u32(" << dst_row << "), " << src_row
+      << "(0), (u32)nb * " << row_len * 4 << ", " << bar << ", pol);\n";
+    return;
+  }
+  if (bulk) {
+    o << "      if (lane < nb) {\n        const int b = lane;\n";
+    for (const auto& s : segs)
+      o << "        bulk_g2s(smem_u32(" << dst_row << " + b * " << stride << " + " << s.dst << "), " << src_row
+        << "(b) + " << s.src << ", " << s.len * 4 << ", " << bar << ");\n";
+    o << "      }\n";
+    return;
+  }
+  for (const auto& s : segs)
+    o << "      for (int t = lane; t < nb * " << s.len << "; t += 32) { const int b = t / " << s.len
+      << ", q = t - b * " << s.len << "; " << dst_row << "[b * " << stride << " + " << s.dst << " + q] = "
+      << src_row << "(b)[" << s.src << " + q]; }\n";
+}
+
+std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL, const KernelShape& K,
+                              bool backward) {
+  std::ostringstream o;
+  const int S = K.S;
+  o << "#define NW " << K.nw << "\n#define NB " << K.B << "\n#define NSTAGE " << K.stages
+    << "\n#define DIN " << P.D_in << "\n#define DE " << P.D_e << "\n#define DOUT " << P.D_out
+    << "\n#define NU " << P.U << "\n#define WS " << K.WS << "\n#define XS " << K.XS << "\n#define CHS "
+    << K.CHS << "\n#define STAGE_BYTES " << K.stage_bytes << "\n#define OFF_STAGE " << K.off_stage
+    << "\n#define OFF_W " << K.off_w << "\n#define OFF_X " << K.off_x << "\n#define OFF_Y " << K.off_y
+    << "\n#define OFF_CH " << K.off_ch << "\n#define OFF_DY " << K.off_dy << "\n#define OFF_G " << K.off_g
+    << "\n#define GS " << K.GS << "\n#define WB " << K.WB << "\n#define OFF_WB " << K.off_wb
+    << "\n#define FULL_COUNT 64\n";
+  if (backward) {
+    o << "__constant__ int kPh[" << S * K.nw << "] = {";
+    for (int s = 0; s < S; ++s)
+      for (int w = 0; w < K.nw; ++w) {
+        const auto& v = P.bcfg.slice_roles[s];
+        o << (w < (int)v.size() ? P.bwd_roles[v[w]].ph : -1) << ",";
+      }
+    o << "};\n__constant__ int kNph[" << S * K.nw << "] = {";
+    for (int s = 0; s < S; ++s)
+      for (int w = 0; w < K.nw; ++w) {
+        const auto& v = P.bcfg.slice_roles[s];
+        o << (w < (int)v.size() ? P.bwd_roles[v[w]].nph : 1) << ",";
+      }
+    o << "};\n";
+  }
+  // CTA -> (slice, first receiver, receiver stride): CTAs [start[s], start[s+1])
+  // of the one-dimensional persistent grid serve slice s
+  o << "struct SliceGrid { int start[" << S + 1 << "]; };\n"
+       "#define NSLICE " << S << "\n"
+       "__device__ __forceinline__ int cta_first(const unsigned char* smem) {\n"
+       "  return reinterpret_cast<const int*>(smem + 240)[0];\n}\n"
+       "__device__ __forceinline__ int cta_stride(const unsigned char* smem) {\n"
+       "  return reinterpret_cast<const int*>(smem + 240)[1];\n}\n"
+       "__device__ __forceinline__ void cta_place(unsigned char* smem, const SliceGrid& sgrid) {\n"
+       "  int s = 0;\n"
+       "  while (s + 1 < NSLICE && (int)blockIdx.x >= sgrid.start[s + 1]) ++s;\n"
+       "  int* h = reinterpret_cast<int*>(smem + 240);\n"
+       "  h[0] = (int)blockIdx.x - sgrid.start[s];\n"
+       "  h[1] = sgrid.start[s + 1] - sgrid.start[s];\n"
+       "  h[2] = s;\n"
+       "}\n";
+  o << "__device__ __forceinline__ unsigned char* stage_ptr(unsigned char* smem, int s) {\n"
+       "  return smem + OFF_STAGE + s * STAGE_BYTES;\n}\n";
+  o << "__device__ __forceinline__ int slice_chs(int s) { switch (s) {";
+  for (int s = 0; s < S; ++s) o << " case " << s << ": return " << SL[s].chs << ";";
+  o << " } return 0; }\n";
+
+  // ---- TMA warp: walks the CTA's receivers (first, first + stride, ...)
+  // and their chunks in the same order as the consumers; the running chunk
+  // counter q picks the stage (q % NSTAGE) and the phase parity.
+  o << "__device__ __noinline__ void tma_warp(const int* __restrict__ rowptr, int n_recv,\n"
+       "    const int* __restrict__ col, const float* __restrict__ x, const float* __restrict__ W,\n"
+       "    const float* __restrict__ g, int* __restrict__ err, unsigned char* smem, int slice, int lane) {\n"
+       "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
+       "  const u32 gfull0 = full0 + 2 * NSTAGE * 8, gempty0 = gfull0 + 16;\n"
+       "  (void)gfull0; (void)gempty0; (void)g;\n"
+       "  const u64 pol = policy_evict_first();\n"
+       "  (void)pol;\n"
+       "  int q = 0, k = 0;\n"
+       "  bool dead = false;\n"
+       "  for (int i = cta_first(smem); i < n_recv && !dead; i += cta_stride(smem)) {\n"
+       "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n";
+  if (backward) o << "    if (e1 == e0) continue;\n";
+  o << "    switch (slice) {\n";
+  for (int s = 0; s < S; ++s) {
+    const SliceLayout& sl = SL[s];
+    long wb = 0, xb = 0, gb = 0;
+    for (auto& q : sl.wseg) wb += q.len * 4;
+    for (auto& q : sl.xseg) xb += q.len * 4;
+    for (auto& q : sl.gseg) gb += q.len * 4;
+    const bool w_one = sl.wseg.size() == 1 && sl.wseg[0].src == 0 && sl.wseg[0].dst == 0 &&
+                       sl.wseg[0].len == P.U && sl.ws == P.U;
+    o << "    case " << s << ": {\n";
+    if (backward) {
+      o << "      {  // this receiver's grad_out pieces into buffer k & 1\n"
+           "        const int gb = k & 1;\n"
+           "        if (k >= 2 && !mbar_wait(gempty0 + 8 * gb, ((k >> 1) - 1) & 1)) { if (lane == 0) atomicOr(err, 10); dead = true; break; }\n"
+           "        float* sg = reinterpret_cast<float*>(smem + OFF_G) + gb * GS;\n"
+           "        const float* grow = g + (size_t)i * DOUT;\n";
+      if (K.g_bulk) {
+        o << "        if (lane == 0) {\n          mbar_expect_tx(gfull0 + 8 * gb, " << gb << ");\n";
+        for (auto& q : sl.gseg)
+          o << "          bulk_g2s(smem_u32(sg + " << q.dst << "), grow + " << q.src << ", " << q.len * 4
+            << ", gfull0 + 8 * gb);\n";
+        o << "        }\n";
+      } else {
+        for (auto& q : sl.gseg)
+          o << "        for (int t = lane; t < " << q.len << "; t += 32) sg[" << q.dst << " + t] = grow["
+            << q.src << " + t];\n";
+      }
+      o << "        mbar_arrive(gfull0 + 8 * gb);\n"
+           "        ++k;\n      }\n";
+    }
+    o << "      for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
+         "        const int s = q % NSTAGE;\n"
+         "        if (q >= NSTAGE && !mbar_wait(empty0 + 8 * s, ((q / NSTAGE) - 1) & 1)) { if (lane == 0) atomicOr(err, 10); dead = true; break; }\n"
+         "        const int nb = min(NB, e1 - eb);\n"
+         "        unsigned char* st = stage_ptr(smem, s);\n"
+         "        float* sW = reinterpret_cast<float*>(st + OFF_W);\n"
+         "        float* sX = reinterpret_cast<float*>(st + OFF_X);\n"
+         "        (void)sW; (void)sX;\n"
+         "        const int jj = (lane < nb) ? col[eb + lane] : 0;\n"
+         "        (void)jj;\n"
+         "        if (lane == 0) mbar_expect_tx(full0 + 8 * s, (u32)nb * "
+      << ((K.w_bulk ? wb : 0) + (K.x_bulk ? xb : 0)) << ");\n"
+      << "        __syncwarp();\n"
+         "#define WROW(b) (W + (size_t)(eb + (b)) * NU)\n";
+    std::ostringstream cp;
+    gen_copy_pieces(cp, sl.wseg, K.w_bulk, "sW", K.WS, "WROW", "full0 + 8 * s", w_one, P.U);
+    if (K.x_bulk) {
+      cp << "#undef WROW\n#define XROW(b) (x + (size_t)jj * DIN)\n";
+      gen_copy_pieces(cp, sl.xseg, true, "sX", K.XS, "XROW", "full0 + 8 * s", false, P.D_in);
+    } else {
+      cp << "#undef WROW\n#define XROW(b) (x + (size_t)col[eb + (b)] * DIN)\n";
+      gen_copy_pieces(cp, sl.xseg, false, "sX", K.XS, "XROW", "full0 + 8 * s", false, P.D_in);
+    }
+    // indent the copy code by two more spaces
+    std::string c = cp.str(), ind;
+    size_t pos = 0;
+    while (pos < c.size()) {
+      size_t e = c.find('\n', pos);
+      if (e == std::string::npos) e = c.size();
+      std::string line = c.substr(pos, e - pos);
+      ind += (line.rfind("#", 0) == 0 ? "" : "  ") + line + "\n";
+      pos = e + 1;
+    }
+    o << ind
+      << "#undef XROW\n"
+         "        mbar_arrive(full0 + 8 * s);\n"
+         "      }\n"
+         "      break;\n    }\n";
+  }
+  o << "    }\n"
+       "  }\n"
+       "  // bulk copies still in flight must land before the CTA may exit\n"
+       "  if (lane == 0)\n"
+       "    for (int c = max(0, q - NSTAGE); c < q; ++c) mbar_wait(full0 + 8 * (c % NSTAGE), (c / NSTAGE) & 1);\n"
+       "}\n";
+
+  // ---- helper warp
+  if (backward) {
+    o << "__device__ __forceinline__ void reduce_dy(unsigned char* smem, int s, int slice, int eb, int nb,\n"
+         "    float* __restrict__ dys, int lane) {\n"
+         "  const float* sdy = reinterpret_cast<const float*>(stage_ptr(smem, s) + OFF_DY);\n"
+         "  for (int t = lane; t < nb * DE; t += 32) {\n"
+         "    const int b = t / DE, k = t - b * DE;\n"
+         "    float v = 0.f;\n"
+         "#pragma unroll\n"
+         "    for (int w = 0; w < NW; ++w) {\n"
+         "      const int ph = kPh[slice * NW + w];\n"
+         "      if (ph >= 0 && (b & (kNph[slice * NW + w] - 1)) == ph) v += sdy[(w * NB + b) * DE + k];\n"
+         "    }\n"
+         "    dys[(size_t)(eb + b) * DE + k] = v;\n"
+         "  }\n"
+         "}\n";
+  }
+  o << "__device__ __noinline__ void helper_warp(const int* __restrict__ rowptr, int n_recv,\n"
+       "    const float* __restrict__ Y, const int4* __restrict__ rec, int nrec, float* __restrict__ dys,\n"
+       "    int* __restrict__ err, unsigned char* smem, int slice, int chs, int lane) {\n"
+       "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
+       "  int2* desc = reinterpret_cast<int2*>(smem + 2 * NSTAGE * 8 + 32);  // (eb, nb) of each stage\n"
+       "  (void)dys; (void)slice; (void)desc;\n"
+       "  // Chat elements without a CG term stay zero for the whole CTA\n"
+       "  for (int s = 0; s < NSTAGE; ++s) {\n"
+       "    float* ch = reinterpret_cast<float*>(stage_ptr(smem, s) + OFF_CH);\n"
+       "    for (int t = lane; t < NB * CHS; t += 32) ch[t] = 0.f;\n"
+       "  }\n"
+       "  int q = 0;\n"
+       "  bool dead = false;\n"
+       "  for (int i = cta_first(smem); i < n_recv && !dead; i += cta_stride(smem)) {\n"
+       "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
+       "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
+       "      const int s = q % NSTAGE;\n"
+       "      if (q >= NSTAGE) {\n"
+       "        if (!mbar_wait(empty0 + 8 * s, ((q / NSTAGE) - 1) & 1)) { if (lane == 0) atomicOr(err, 10); dead = true; break; }\n";
+  if (backward)
+    o << "        if (dys) { const int2 d = desc[s]; reduce_dy(smem, s, slice, d.x, d.y, dys, lane); }\n";
+  o << "      }\n"
+       "      const int nb = min(NB, e1 - eb);\n"
+       "      unsigned char* st = stage_ptr(smem, s);\n"
+       "      float* sY = reinterpret_cast<float*>(st + OFF_Y);\n"
+       "      float* ch = reinterpret_cast<float*>(st + OFF_CH);\n"
+       "      for (int t = lane; t < nb * DE; t += 32) sY[t] = Y[(size_t)eb * DE + t];\n"
+       "      if (lane == 0) desc[s] = make_int2(eb, nb);\n"
+       "      __syncwarp();\n"
+       "      for (int b = 0; b < nb; ++b) {\n"
+       "        const float* y = sY + b * DE;\n"
+       "        float* cb = ch + b * chs;\n"
+       "#pragma unroll 4\n"
+       "        for (int r0 = lane; r0 < nrec; r0 += 32) {\n"
+       "          const int4 r = __ldg(rec + r0);\n"
+       "          cb[r.x & 0xffff] = fmaf(__int_as_float(r.y), y[(r.x >> 16) & 0xff], __int_as_float(r.z) * y[(unsigned)r.x >> 24]);\n"
+       "        }\n"
+       "      }\n"
+       "      mbar_arrive(full0 + 8 * s);\n"
+       "    }\n"
+       "  }\n";
+  if (backward)
+    o << "  if (!dead && dys)\n"
+         "    for (int c = max(0, q - NSTAGE); c < q; ++c) {\n"
+         "      const int s = c % NSTAGE;\n"
+         "      if (!mbar_wait(empty0 + 8 * s, (c / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); break; }\n"
+         "      __syncwarp();\n"
+         "      const int2 d = desc[s];\n"
+         "      reduce_dy(smem, s, slice, d.x, d.y, dys, lane);\n"
+         "    }\n";
+  o << "}\n";
+  return o.str();
+}
+
+// One 16-byte record per non-zero Chat element of a slice's paths (real CG
+// blocks have at most two non-zero C[m1][m2][m3] for a given (m1, m3)):
+//   x = dst offset in the edge's Chat block | y0 << 16 | y1 << 24
+//   y = coefficient of Y[y0], z = coefficient of Y[y1] (FP32 bits), w = 0.
+// Elements with no term stay zero: the helper clears the Chat buffers once.
 cgtp_status upload_chat_tables(const Plan& P, const std::vector<SliceLayout>& SL, void** d_ent,
                                void** d_term, std::vector<int>& ent_begin) {
-  std::vector<int> ent, term;
+  std::vector<int> rec;
   ent_begin.assign(1, 0);
   for (const SliceLayout& sl : SL) {
     for (int pi : sl.paths) {
@@ -23,34 +379,38 @@ cgtp_status upload_chat_tables(const Plan& P, const std::vector<SliceLayout>& SL
       const double* C = P.coeff.data() + p.c_off;
       for (int m3 = 0; m3 < n3; ++m3)
         for (int m1 = 0; m1 < n1; ++m1) {
-          const int tb = (int)term.size() / 2;
+          int yi[2] = {0, 0};
+          float cf[2] = {0.f, 0.f};
           int cnt = 0;
           for (int m2 = 0; m2 < n2; ++m2) {
             const double c = C[((size_t)m1 * n2 + m2) * n3 + m3];
             if (c == 0.0) continue;
-            const float cf = (float)c;
-            int bits;
-            std::memcpy(&bits, &cf, 4);
-            term.push_back(p.l2 * p.l2 + m2);
-            term.push_back(bits);
+            if (cnt == 2) return fail(CGTP_ERR_SIZE, "a Chat element with more than two CG terms");
+            yi[cnt] = p.l2 * p.l2 + m2;
+            cf[cnt] = (float)c;
             ++cnt;
           }
-          ent.push_back(sl.ch_off.at(pi) + chat_pos(p.l1, p.l3, m1, m3));
-          ent.push_back(tb);
-          ent.push_back(cnt);
-          ent.push_back(0);
+          if (cnt == 0) continue;
+          const int dst = sl.ch_off.at(pi) + chat_pos(p.l1, p.l3, m1, m3);
+          if (dst >= (1 << 16) || yi[0] >= 256 || yi[1] >= 256)
+            return fail(CGTP_ERR_SIZE, "Chat block too large for the record format");
+          int b0, b1;
+          std::memcpy(&b0, &cf[0], 4);
+          std::memcpy(&b1, &cf[1], 4);
+          rec.push_back(dst | (yi[0] << 16) | (yi[1] << 24));
+          rec.push_back(b0);
+          rec.push_back(b1);
+          rec.push_back(0);
         }
     }
-    ent_begin.push_back((int)ent.size() / 4);
+    ent_begin.push_back((int)rec.size() / 4);
   }
+  *d_term = nullptr;
   if (P.host_only) return CGTP_OK;
-  if (ent.empty()) ent.assign(4, 0);
-  if (term.empty()) term.assign(2, 0);
-  if (cudaMalloc(d_ent, ent.size() * sizeof(int)) != cudaSuccess ||
-      cudaMalloc(d_term, term.size() * sizeof(int)) != cudaSuccess)
+  if (rec.empty()) rec.assign(4, 0);
+  if (cudaMalloc(d_ent, rec.size() * sizeof(int)) != cudaSuccess)
     return fail(CGTP_ERR_OOM, "cudaMalloc of the Chat tables");
-  CGTP_CUDA_TRY(cudaMemcpy(*d_ent, ent.data(), ent.size() * sizeof(int), cudaMemcpyHostToDevice));
-  CGTP_CUDA_TRY(cudaMemcpy(*d_term, term.data(), term.size() * sizeof(int), cudaMemcpyHostToDevice));
+  CGTP_CUDA_TRY(cudaMemcpy(*d_ent, rec.data(), rec.size() * sizeof(int), cudaMemcpyHostToDevice));
   return CGTP_OK;
 }
 

@@ -1,5 +1,6 @@
 // codegen_common.hpp -- pieces shared by the forward and backward code
-// generators: the device prelude, the per-edge Chat layout and its tables.
+// generators: the device prelude, per-slice staging layouts, the Chat tables,
+// and the two service warps of both kernels.
 #pragma once
 
 #include <map>
@@ -25,21 +26,56 @@ inline int chat_pos(int l1, int l3, int m1, int m3) {
   return n1 == 1 ? m3 : m3 * pad4(n1) + m1;
 }
 
-struct SliceLayout {
-  std::vector<int> paths;     // unique paths of the slice
-  std::map<int, int> ch_off;  // path -> Chat offset (floats)
-  int chs = 0;                // Chat floats per edge
-  std::vector<int> irreps;    // hidden irreps staged
-  std::map<int, int> x_st;    // irrep -> staged offset (floats)
-  int xs = 0;                 // staged x floats per edge
-  std::map<int, int> g_st;    // path -> staged offset of its grad_out block (backward)
-  int gs = 0;                 // staged grad_out floats per receiver (backward)
+// A contiguous piece of a global row copied into a staged row.
+struct Segment {
+  int src;  // float offset in the global row
+  int dst;  // float offset in the staged row
+  int len;  // floats
 };
 
-std::string gen_producer(const Plan& P, const FwdConfig& F);
-std::string gen_slice_helpers(const Plan& P, const FwdConfig& F, const std::vector<SliceLayout>& SL);
-std::string gen_layout(const Plan& P, const FwdConfig& F, const std::vector<SliceLayout>& SL,
-                       int extra_bytes, int& off_extra, int& smem_bytes);
+struct SliceLayout {
+  std::vector<int> paths;      // paths whose Chat the slice needs
+  std::map<int, int> ch_off;   // path -> Chat offset (floats, per edge)
+  int chs = 0;                 // Chat floats per edge
+  std::vector<int> irreps;     // hidden irreps of the slice
+  std::map<int, int> x_st;     // irrep -> staged x offset
+  std::vector<Segment> xseg;   // x row pieces
+  int xs = 0;                  // staged x floats per edge
+  std::map<int, int> w_st;     // path -> staged W offset of its channel 0
+  std::vector<Segment> wseg;   // W row pieces
+  int ws = 0;                  // staged W floats per edge
+  std::map<int, int> g_st;     // path -> staged grad_out offset (backward)
+  std::vector<Segment> gseg;   // grad_out row pieces (backward)
+  int gs = 0;                  // staged grad_out floats per receiver
+};
+
+// Builds the staging layout of one slice from its paths and irreps.
+void layout_slice(const Plan& P, SliceLayout& sl, bool with_g);
+
+// Whether every piece of the slice can move by bulk copy (16-byte aligned
+// starts and lengths in both the global and the staged row).
+bool segments_aligned(const std::vector<Segment>& segs, long row_len);
+
+struct KernelShape {
+  int S = 1, nw = 0, B = 2, stages = 3;
+  bool w_bulk = true, x_bulk = true, g_bulk = true;
+  int WS = 0, XS = 0, CHS = 0, GS = 0;
+  int sdy_floats = 0;  // per stage (backward)
+  // byte offsets in dynamic shared memory
+  int off_stage = 0, stage_bytes = 0, off_w = 0, off_x = 0, off_y = 0, off_ch = 0, off_dy = 0;
+  int off_g = 0, smem = 0;
+  int WB = 0;       // per-consumer-warp staging buffer for coalesced row stores (floats)
+  int off_wb = 0;
+};
+
+// Fills the shared-memory layout of a kernel; extra per-stage floats for the
+// backward's dY partials.
+void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape& K, bool backward);
+
+// Device code: #defines, per-slice staging switches, the TMA warp and the
+// helper warp.  (backward: grad_out staging and dY reduction.)
+std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
+                              const KernelShape& K, bool backward);
 
 cgtp_status upload_chat_tables(const Plan& P, const std::vector<SliceLayout>& SL, void** d_ent,
                                void** d_term, std::vector<int>& ent_begin);

@@ -76,6 +76,7 @@ struct JitKernel {
   std::string name;
   std::string log;
   unsigned long long hash = 0;  // of the generated source and compile options
+  int blocks_per_sm = 0;        // resident CTAs per SM (occupancy query)
 };
 
 struct FwdConfig {
@@ -87,6 +88,7 @@ struct FwdConfig {
   bool x_smem = true;    // x blocks staged by bulk copy
   int nacc = 0;          // accumulator registers per thread
   std::vector<std::vector<int>> slice_roles;  // role ids per slice
+  std::vector<double> weight;                 // relative work per receiver of each slice
 };
 
 struct Plan {
@@ -98,6 +100,7 @@ struct Plan {
   std::vector<Path> paths;
   std::vector<double> coeff;  // concatenated real CG blocks (FP64)
   int device = -1;
+  int num_sms = 0;
 
   // forward
   std::vector<FwdRole> fwd_roles;

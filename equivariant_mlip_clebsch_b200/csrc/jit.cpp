@@ -30,6 +30,7 @@ struct Driver {
   CUresult (*launchKernel)(CUfunction, unsigned, unsigned, unsigned, unsigned, unsigned, unsigned,
                            unsigned, CUstream, void**, void**) = nullptr;
   CUresult (*getErrorString)(CUresult, const char**) = nullptr;
+  CUresult (*occupancy)(int*, CUfunction, int, size_t) = nullptr;
   bool ok = false;
   std::string err;
 };
@@ -57,7 +58,8 @@ Driver& driver() {
            entry("cuModuleUnload", d.moduleUnload, err) &&
            entry("cuFuncSetAttribute", d.funcSetAttribute, err) &&
            entry("cuLaunchKernel", d.launchKernel, err) &&
-           entry("cuGetErrorString", d.getErrorString, err);
+           entry("cuGetErrorString", d.getErrorString, err) &&
+           entry("cuOccupancyMaxActiveBlocksPerMultiprocessor", d.occupancy, err);
     d.err = err;
   });
   return d;
@@ -172,6 +174,13 @@ cgtp_status jit_compile(const std::string& src, const std::string& name, JitKern
       return fail(CGTP_ERR_CUDA, "cuFuncSetAttribute(smem): " + cu_str(cr));
     }
   }
+  int nb = 0;
+  cr = d.occupancy(&nb, fn, k.threads, (size_t)k.smem);
+  if (cr != CUDA_SUCCESS || nb < 1) {
+    d.moduleUnload(mod);
+    return fail(CGTP_ERR_CUDA, "kernel " + name + " cannot be resident: " + cu_str(cr));
+  }
+  k.blocks_per_sm = nb;
   k.module = mod;
   k.function = fn;
   return CGTP_OK;
