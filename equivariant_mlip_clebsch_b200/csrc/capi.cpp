@@ -91,22 +91,11 @@ struct TimedScope {
   }
 };
 
-// Persistent grid: T resident CTAs shared among the slices in proportion to
-// their work; CTAs [start[s], start[s+1]) serve slice s.
-static std::vector<int> slice_partition(const FwdConfig& F, int blocks_per_sm, int num_sms,
-                                        int64_t n_recv) {
-  const int S = F.S;
-  const long T = std::max<long>(S, (long)blocks_per_sm * num_sms);
-  double W = 0.0;
-  for (int s = 0; s < S; ++s) W += (s < (int)F.weight.size() ? F.weight[s] : 1.0);
-  std::vector<int> start(S + 1, 0);
-  for (int s = 0; s < S; ++s) {
-    const double w = s < (int)F.weight.size() ? F.weight[s] : 1.0;
-    long g = (long)std::floor(T * w / std::max(W, 1e-30));
-    g = std::max<long>(1, std::min<long>(g, std::max<int64_t>(1, n_recv)));
-    start[s + 1] = start[s] + (int)g;
-  }
-  return start;
+// Persistent grid: about one wave of resident CTAs; each walks the slices in
+// order and, inside a slice, the receivers blockIdx.x, + gridDim.x, ...
+static unsigned persistent_grid(int blocks_per_sm, int num_sms, int64_t n_recv) {
+  const int64_t T = std::max<int64_t>(1, (int64_t)blocks_per_sm * num_sms);
+  return (unsigned)std::max<int64_t>(1, std::min<int64_t>(T, n_recv));
 }
 
 }  // namespace cgtp
@@ -265,10 +254,9 @@ cgtp_status cgtp_forward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t
   int nr = (int)n_recv;
   // persistent CTAs: about one wave of resident CTAs, each walking its slice's
   // receivers first, first + stride, ...
-  std::vector<int> part = slice_partition(P->fcfg, P->fwd.blocks_per_sm, P->num_sms, n_recv);
-  void* args[] = {&rowptr, &col, &x, &Y, &W, &out, &P->d_fwd_ent, &nr, &P->d_err, part.data()};
+  void* args[] = {&rowptr, &col, &x, &Y, &W, &out, &P->d_fwd_ent, &nr, &P->d_err};
   TimedScope ts(*P, 1, s);
-  return jit_launch(P->fwd, dim3((unsigned)part.back(), 1), args, s);
+  return jit_launch(P->fwd, dim3(persistent_grid(P->fwd.blocks_per_sm, P->num_sms, n_recv)), args, s);
 }
 
 cgtp_status cgtp_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
@@ -346,11 +334,9 @@ cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
   }
   if (n_recv > 0) {
     int nr = (int)n_recv;
-    std::vector<int> part = slice_partition(P->bcfg, P->bwd.blocks_per_sm, P->num_sms, n_recv);
-    void* args[] = {&rowptr, &col, &x, &Y, &W, &grad_out, &grad_W, &dyp, &m, &P->d_bwd_ent, &nr,
-                    &P->d_err, part.data()};
+    void* args[] = {&rowptr, &col, &x, &Y, &W, &grad_out, &grad_W, &dyp, &m, &P->d_bwd_ent, &nr, &P->d_err};
     TimedScope ts(*P, 2, s, allow_timing);
-    st = jit_launch(P->bwd, dim3((unsigned)part.back(), 1), args, s);
+    st = jit_launch(P->bwd, dim3(persistent_grid(P->bwd.blocks_per_sm, P->num_sms, n_recv)), args, s);
     if (st != CGTP_OK) return st;
   }
   if (grad_Y && P->bcfg.S > 1) {

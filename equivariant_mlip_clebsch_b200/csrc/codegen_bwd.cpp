@@ -51,7 +51,7 @@ std::string flt(double v) {
 }  // namespace
 
 static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>& SL, const KernelShape& K,
-                                  const std::string& kname) {
+                                  const std::string& kname, int min_blocks) {
   const FwdConfig& F = P.bcfg;
   const int S = K.S, NW = K.nw;
   std::ostringstream o;
@@ -78,7 +78,8 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
   }
   const std::string params =
       "(const int* __restrict__ rowptr, int n_recv, float* __restrict__ dW, float* __restrict__ msg,\n"
-      "    int* __restrict__ err, unsigned char* smem, int u0, int ph, int nph, int chs, bool want_dy)";
+      "    int* __restrict__ err, unsigned char* smem, int u0, int ph, int nph, int chs, bool want_dy,\n"
+      "    int* qp, int* kp)";
   for (size_t k = 0; k < shape_rep.size(); ++k) {
     const BwdRole& r = P.bwd_roles[shape_rep[k]];
     const SliceLayout& sl = SL[slice_of[shape_rep[k]]];
@@ -92,11 +93,11 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
     o << "__device__ __noinline__ void bcons_" << k << params << " {\n"
       << "  const int lane = threadIdx.x & 31;\n"
       << "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
-      << "  const u32 gfull0 = full0 + 2 * NSTAGE * 8, gempty0 = gfull0 + 16;\n"
+      << "  const u32 gfull0 = full0 + OFF_GFULL, gempty0 = full0 + OFF_GEMPTY;\n"
       << "  bool ok[" << R << "];\n"
       << "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) ok[r] = u0 + r * 32 + lane < " << MUL << ";\n"
-      << "  int q = 0, kr = 0;\n"
-      << "#pragma unroll 1\n  for (int i = cta_first(smem); i < n_recv; i += cta_stride(smem)) {\n"
+      << "  int q = *qp, kr = *kp;\n"
+      << "#pragma unroll 1\n  for (int i = blockIdx.x; i < n_recv; i += gridDim.x) {\n"
       << "  const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
       << "  if (e1 == e0) continue;\n"
       << "  const int gb = kr & 1;\n"
@@ -205,14 +206,14 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       << ", wbuf, min(" << 32 * R << ", " << MUL << " - u0) * " << N1 << ", lane);\n"
       << "        __syncwarp();\n      }\n";
     o << "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n"
-      << "  __syncwarp();\n  if (lane == 0) mbar_arrive(gempty0 + 8 * gb);\n  ++kr;\n  }\n}\n";
+      << "  __syncwarp();\n  if (lane == 0) mbar_arrive(gempty0 + 8 * gb);\n  ++kr;\n  }\n  *qp = q;\n  *kp = kr;\n}\n";
   }
   o << "__device__ __noinline__ void bcons_idle" << params << " {\n"
        "  const int lane = threadIdx.x & 31;\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
-       "  const u32 gempty0 = full0 + 2 * NSTAGE * 8 + 16;\n"
-       "  int q = 0, kr = 0;\n"
-       "#pragma unroll 1\n  for (int i = cta_first(smem); i < n_recv; i += cta_stride(smem)) {\n"
+       "  const u32 gempty0 = full0 + OFF_GEMPTY;\n"
+       "  int q = *qp, kr = *kp;\n"
+       "#pragma unroll 1\n  for (int i = blockIdx.x; i < n_recv; i += gridDim.x) {\n"
        "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
        "    if (e1 == e0) continue;\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
@@ -224,6 +225,8 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
        "    if (lane == 0) mbar_arrive(gempty0 + 8 * (kr & 1));\n"
        "    ++kr;\n"
        "  }\n"
+       "  *qp = q;\n"
+       "  *kp = kr;\n"
        "}\n";
   o << "__constant__ int kShape[" << S * NW << "] = {";
   for (int s = 0; s < S; ++s)
@@ -236,44 +239,33 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
   o << "};\n__constant__ int kEntBegin[" << S + 1 << "] = {";
   for (int v : P.bwd_ent_begin) o << v << ",";
   o << "};\n";
-  // resident CTAs to plan registers for: as many as shared memory allows (at
-  // most 3), or CGTP_MIN_BLOCKS when set (1 leaves registers uncapped)
-  int min_blocks = std::max(1, std::min(3, (228 * 1024) / (K.smem + 1024)));
-  if (const char* mb = std::getenv("CGTP_MIN_BLOCKS")) min_blocks = std::max(1, std::atoi(mb));
   o << "extern \"C\" __global__ void __launch_bounds__((NW + 2) * 32, " << min_blocks << ") " << kname
     << "(const int* __restrict__ rowptr, const int* __restrict__ col, const float* __restrict__ x,\n"
        "    const float* __restrict__ Y, const float* __restrict__ W, const float* __restrict__ g,\n"
        "    float* __restrict__ dW, float* __restrict__ dyp, float* __restrict__ msg,\n"
-       "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err, const SliceGrid sgrid) {\n"
+       "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err) {\n"
        "  extern __shared__ __align__(128) unsigned char smem[];\n"
-       "  (void)0;\n"
        "  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
-       "  const u32 gfull0 = full0 + 2 * NSTAGE * 8, gempty0 = gfull0 + 16;\n"
+       "  const u32 gfull0 = full0 + OFF_GFULL, gempty0 = full0 + OFF_GEMPTY;\n"
        "  if (threadIdx.x == 0) {\n"
        "    for (int s = 0; s < NSTAGE; ++s) { mbar_init(full0 + 8 * s, FULL_COUNT); mbar_init(empty0 + 8 * s, NW); }\n"
        "    for (int b = 0; b < 2; ++b) { mbar_init(gfull0 + 8 * b, 32); mbar_init(gempty0 + 8 * b, NW); }\n"
        "    fence_mbar_init();\n"
-       "    cta_place(smem, sgrid);\n"
        "  }\n"
        "  __syncthreads();\n"
-       "  const int slice = reinterpret_cast<const int*>(smem + 240)[2];\n"
-       "  const int chs = slice_chs(slice);\n"
-       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, g, err, smem, slice, lane); return; }\n"
-       "  if (warp == NW + 1) {\n"
-       "    const int E = rowptr[n_recv];\n"
-       "    float* dys = dyp ? dyp + (size_t)slice * E * DE : nullptr;\n"
-       "    helper_warp(rowptr, n_recv, Y, ent + kEntBegin[slice], kEntBegin[slice + 1] - kEntBegin[slice],\n"
-       "                dys, err, smem, slice, chs, lane);\n"
-       "    return;\n"
-       "  }\n"
-       "  const int slot = slice * NW + warp;\n"
-       "  const int u0 = kU0[slot], ph = kPh[slot], nph = kNph[slot];\n"
-       "  switch (kShape[slot]) {\n";
+       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, g, err, smem, lane); return; }\n"
+       "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, ent, kEntBegin, dyp, err, smem, lane); return; }\n"
+       "  int q = 0, kr = 0;\n"
+       "  for (int slice = 0; slice < NSLICE; ++slice) {\n"
+       "    const int slot = slice * NW + warp;\n"
+       "    const int u0 = kU0[slot], ph = kPh[slot], nph = kNph[slot], chs = kChs[slice];\n"
+       "    switch (kShape[slot]) {\n";
   for (size_t k = 0; k < shape_rep.size(); ++k)
-    o << "  case " << k << ": bcons_" << k
-      << "(rowptr, n_recv, dW, msg, err, smem, u0, ph, nph, chs, dyp != nullptr); break;\n";
-  o << "  default: bcons_idle(rowptr, n_recv, dW, msg, err, smem, u0, ph, nph, chs, dyp != nullptr); break;\n  }\n}\n";
+    o << "    case " << k << ": bcons_" << k
+      << "(rowptr, n_recv, dW, msg, err, smem, u0, ph, nph, chs, dyp != nullptr, &q, &kr); break;\n";
+  o << "    default: bcons_idle(rowptr, n_recv, dW, msg, err, smem, u0, ph, nph, chs, dyp != nullptr, &q, &kr); break;\n"
+       "    }\n  }\n}\n";
   return o.str();
 }
 
@@ -359,8 +351,22 @@ cgtp_status build_backward(Plan& P) {
   cgtp_status st = upload_chat_tables(P, SL, &P.d_bwd_ent, &P.d_bwd_term, P.bwd_ent_begin);
   if (st != CGTP_OK) return st;
   const std::string name = "cgtp_bwd";
-  std::string src = gen_bwd_source(P, SL, K, name);
+  // register cap from the resident CTAs shared memory allows; one CTA fewer
+  // (but not below two) when the compiler reports sizeable spills
   if (K.smem > 227 * 1024) return fail(CGTP_ERR_SIZE, "backward kernel needs too much shared memory");
+  bool fixed = false;
+  const int mb0 = initial_min_blocks(K.smem, &fixed);
+  const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
+  std::string src;
+  for (int mb = mb0; mb >= mb_floor; --mb) {
+    src = gen_bwd_source(P, SL, K, name, mb);
+    P.bwd.threads = (F.nw + 2) * 32;
+    P.bwd.smem = K.smem;
+    cgtp_status cst = jit_compile(src, name, P.bwd);
+    if (cst != CGTP_OK) return cst;
+    if (mb == mb_floor || max_spill_bytes(P.bwd.log) <= 160) break;
+    jit_unload(P.bwd);
+  }
   P.bwd.threads = (F.nw + 2) * 32;
   P.bwd.smem = K.smem;
   if (const char* d = std::getenv("CGTP_DUMP_SOURCE")) {
@@ -370,7 +376,7 @@ cgtp_status build_backward(Plan& P) {
       std::fclose(f);
     }
   }
-  return jit_compile(src, name, P.bwd);
+  return CGTP_OK;
 }
 
 }  // namespace cgtp

@@ -18,6 +18,8 @@
 #include "codegen_common.hpp"
 
 #include <algorithm>
+#include <cctype>
+#include <cstdlib>
 #include <cstring>
 #include <sstream>
 
@@ -26,6 +28,28 @@ namespace cgtp {
 const char* kPrelude =
 #include "device_prelude.inc"
     ;
+
+int max_spill_bytes(const std::string& log) {
+  int best = 0;
+  size_t pos = 0;
+  const std::string key = " bytes spill stores";
+  while ((pos = log.find(key, pos)) != std::string::npos) {
+    size_t b = pos;
+    while (b > 0 && std::isdigit((unsigned char)log[b - 1])) --b;
+    if (b < pos) best = std::max(best, std::atoi(log.substr(b, pos - b).c_str()));
+    pos += key.size();
+  }
+  return best;
+}
+
+int initial_min_blocks(int smem_bytes, bool* fixed) {
+  if (const char* mb = std::getenv("CGTP_MIN_BLOCKS")) {
+    *fixed = true;
+    return std::max(1, std::atoi(mb));
+  }
+  *fixed = false;
+  return std::max(1, std::min(3, (228 * 1024) / (smem_bytes + 1024)));
+}
 
 static void merge_segment(std::vector<Segment>& v, Segment s) {
   if (!v.empty() && v.back().src + v.back().len == s.src && v.back().dst + v.back().len == s.dst)
@@ -156,13 +180,16 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
   std::ostringstream o;
   const int S = K.S;
   o << "#define NW " << K.nw << "\n#define NB " << K.B << "\n#define NSTAGE " << K.stages
-    << "\n#define DIN " << P.D_in << "\n#define DE " << P.D_e << "\n#define DOUT " << P.D_out
-    << "\n#define NU " << P.U << "\n#define WS " << K.WS << "\n#define XS " << K.XS << "\n#define CHS "
-    << K.CHS << "\n#define STAGE_BYTES " << K.stage_bytes << "\n#define OFF_STAGE " << K.off_stage
-    << "\n#define OFF_W " << K.off_w << "\n#define OFF_X " << K.off_x << "\n#define OFF_Y " << K.off_y
-    << "\n#define OFF_CH " << K.off_ch << "\n#define OFF_DY " << K.off_dy << "\n#define OFF_G " << K.off_g
-    << "\n#define GS " << K.GS << "\n#define WB " << K.WB << "\n#define OFF_WB " << K.off_wb
-    << "\n#define FULL_COUNT 64\n";
+    << "\n#define NSLICE " << S << "\n#define DIN " << P.D_in << "\n#define DE " << P.D_e
+    << "\n#define DOUT " << P.D_out << "\n#define NU " << P.U << "\n#define WS " << K.WS
+    << "\n#define XS " << K.XS << "\n#define CHS " << K.CHS << "\n#define STAGE_BYTES " << K.stage_bytes
+    << "\n#define OFF_STAGE " << K.off_stage << "\n#define OFF_W " << K.off_w << "\n#define OFF_X "
+    << K.off_x << "\n#define OFF_Y " << K.off_y << "\n#define OFF_CH " << K.off_ch << "\n#define OFF_DY "
+    << K.off_dy << "\n#define OFF_G " << K.off_g << "\n#define GS " << K.GS << "\n#define WB " << K.WB
+    << "\n#define OFF_WB " << K.off_wb << "\n#define FULL_COUNT 64\n";
+  // shared-memory header: full[NSTAGE], empty[NSTAGE], gfull[2], gempty[2]
+  // mbarriers, then the helper's per-stage chunk descriptors
+  o << "#define OFF_GFULL (2 * NSTAGE * 8)\n#define OFF_GEMPTY (OFF_GFULL + 16)\n#define OFF_DESC (OFF_GEMPTY + 16)\n";
   if (backward) {
     o << "__constant__ int kPh[" << S * K.nw << "] = {";
     for (int s = 0; s < S; ++s)
@@ -178,42 +205,27 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
       }
     o << "};\n";
   }
-  // CTA -> (slice, first receiver, receiver stride): CTAs [start[s], start[s+1])
-  // of the one-dimensional persistent grid serve slice s
-  o << "struct SliceGrid { int start[" << S + 1 << "]; };\n"
-       "#define NSLICE " << S << "\n"
-       "__device__ __forceinline__ int cta_first(const unsigned char* smem) {\n"
-       "  return reinterpret_cast<const int*>(smem + 240)[0];\n}\n"
-       "__device__ __forceinline__ int cta_stride(const unsigned char* smem) {\n"
-       "  return reinterpret_cast<const int*>(smem + 240)[1];\n}\n"
-       "__device__ __forceinline__ void cta_place(unsigned char* smem, const SliceGrid& sgrid) {\n"
-       "  int s = 0;\n"
-       "  while (s + 1 < NSLICE && (int)blockIdx.x >= sgrid.start[s + 1]) ++s;\n"
-       "  int* h = reinterpret_cast<int*>(smem + 240);\n"
-       "  h[0] = (int)blockIdx.x - sgrid.start[s];\n"
-       "  h[1] = sgrid.start[s + 1] - sgrid.start[s];\n"
-       "  h[2] = s;\n"
-       "}\n";
+  o << "__constant__ int kChs[" << S << "] = {";
+  for (int s = 0; s < S; ++s) o << SL[s].chs << ",";
+  o << "};\n";
   o << "__device__ __forceinline__ unsigned char* stage_ptr(unsigned char* smem, int s) {\n"
        "  return smem + OFF_STAGE + s * STAGE_BYTES;\n}\n";
-  o << "__device__ __forceinline__ int slice_chs(int s) { switch (s) {";
-  for (int s = 0; s < S; ++s) o << " case " << s << ": return " << SL[s].chs << ";";
-  o << " } return 0; }\n";
 
-  // ---- TMA warp: walks the CTA's receivers (first, first + stride, ...)
-  // and their chunks in the same order as the consumers; the running chunk
-  // counter q picks the stage (q % NSTAGE) and the phase parity.
+  // ---- TMA warp.  Every warp of a CTA walks the same sequence: for each
+  // slice in order, the receivers blockIdx.x, + gridDim.x, ..., and their
+  // chunks; the running chunk counter q picks the stage and the phase.
   o << "__device__ __noinline__ void tma_warp(const int* __restrict__ rowptr, int n_recv,\n"
        "    const int* __restrict__ col, const float* __restrict__ x, const float* __restrict__ W,\n"
-       "    const float* __restrict__ g, int* __restrict__ err, unsigned char* smem, int slice, int lane) {\n"
+       "    const float* __restrict__ g, int* __restrict__ err, unsigned char* smem, int lane) {\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
-       "  const u32 gfull0 = full0 + 2 * NSTAGE * 8, gempty0 = gfull0 + 16;\n"
+       "  const u32 gfull0 = full0 + OFF_GFULL, gempty0 = full0 + OFF_GEMPTY;\n"
        "  (void)gfull0; (void)gempty0; (void)g;\n"
        "  const u64 pol = policy_evict_first();\n"
        "  (void)pol;\n"
        "  int q = 0, k = 0;\n"
        "  bool dead = false;\n"
-       "  for (int i = cta_first(smem); i < n_recv && !dead; i += cta_stride(smem)) {\n"
+       "  for (int slice = 0; slice < NSLICE && !dead; ++slice) {\n"
+       "  for (int i = blockIdx.x; i < n_recv && !dead; i += gridDim.x) {\n"
        "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n";
   if (backward) o << "    if (e1 == e0) continue;\n";
   o << "    switch (slice) {\n";
@@ -258,18 +270,19 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
          "        (void)jj;\n"
          "        if (lane == 0) mbar_expect_tx(full0 + 8 * s, (u32)nb * "
       << ((K.w_bulk ? wb : 0) + (K.x_bulk ? xb : 0)) << ");\n"
-      << "        __syncwarp();\n"
-         "#define WROW(b) (W + (size_t)(eb + (b)) * NU)\n";
+      << "        __syncwarp();\n";
     std::ostringstream cp;
+    cp << "#define WROW(b) (W + (size_t)(eb + (b)) * NU)\n";
     gen_copy_pieces(cp, sl.wseg, K.w_bulk, "sW", K.WS, "WROW", "full0 + 8 * s", w_one, P.U);
+    cp << "#undef WROW\n";
     if (K.x_bulk) {
-      cp << "#undef WROW\n#define XROW(b) (x + (size_t)jj * DIN)\n";
+      cp << "#define XROW(b) (x + (size_t)jj * DIN)\n";
       gen_copy_pieces(cp, sl.xseg, true, "sX", K.XS, "XROW", "full0 + 8 * s", false, P.D_in);
     } else {
-      cp << "#undef WROW\n#define XROW(b) (x + (size_t)col[eb + (b)] * DIN)\n";
+      cp << "#define XROW(b) (x + (size_t)col[eb + (b)] * DIN)\n";
       gen_copy_pieces(cp, sl.xseg, false, "sX", K.XS, "XROW", "full0 + 8 * s", false, P.D_in);
     }
-    // indent the copy code by two more spaces
+    cp << "#undef XROW\n";
     std::string c = cp.str(), ind;
     size_t pos = 0;
     while (pos < c.size()) {
@@ -280,12 +293,12 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
       pos = e + 1;
     }
     o << ind
-      << "#undef XROW\n"
-         "        mbar_arrive(full0 + 8 * s);\n"
+      << "        mbar_arrive(full0 + 8 * s);\n"
          "      }\n"
          "      break;\n    }\n";
   }
   o << "    }\n"
+       "  }\n"
        "  }\n"
        "  // bulk copies still in flight must land before the CTA may exit\n"
        "  if (lane == 0)\n"
@@ -294,70 +307,82 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
 
   // ---- helper warp
   if (backward) {
-    o << "__device__ __forceinline__ void reduce_dy(unsigned char* smem, int s, int slice, int eb, int nb,\n"
-         "    float* __restrict__ dys, int lane) {\n"
+    o << "__device__ __forceinline__ void reduce_dy(unsigned char* smem, int s, int4 d, float* __restrict__ dyp,\n"
+         "    int E, int lane) {\n"
+         "  // d = (first edge, edges, slice) of the chunk that stage s held\n"
          "  const float* sdy = reinterpret_cast<const float*>(stage_ptr(smem, s) + OFF_DY);\n"
-         "  for (int t = lane; t < nb * DE; t += 32) {\n"
+         "  float* dys = dyp + (size_t)d.z * E * DE;\n"
+         "  for (int t = lane; t < d.y * DE; t += 32) {\n"
          "    const int b = t / DE, k = t - b * DE;\n"
          "    float v = 0.f;\n"
          "#pragma unroll\n"
          "    for (int w = 0; w < NW; ++w) {\n"
-         "      const int ph = kPh[slice * NW + w];\n"
-         "      if (ph >= 0 && (b & (kNph[slice * NW + w] - 1)) == ph) v += sdy[(w * NB + b) * DE + k];\n"
+         "      const int ph = kPh[d.z * NW + w];\n"
+         "      if (ph >= 0 && (b & (kNph[d.z * NW + w] - 1)) == ph) v += sdy[(w * NB + b) * DE + k];\n"
          "    }\n"
-         "    dys[(size_t)(eb + b) * DE + k] = v;\n"
+         "    dys[(size_t)(d.x + b) * DE + k] = v;\n"
          "  }\n"
          "}\n";
   }
   o << "__device__ __noinline__ void helper_warp(const int* __restrict__ rowptr, int n_recv,\n"
-       "    const float* __restrict__ Y, const int4* __restrict__ rec, int nrec, float* __restrict__ dys,\n"
-       "    int* __restrict__ err, unsigned char* smem, int slice, int chs, int lane) {\n"
+       "    const float* __restrict__ Y, const int4* __restrict__ rec, const int* __restrict__ rec_begin,\n"
+       "    float* __restrict__ dyp, int* __restrict__ err, unsigned char* smem, int lane) {\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
-       "  int2* desc = reinterpret_cast<int2*>(smem + 2 * NSTAGE * 8 + 32);  // (eb, nb) of each stage\n"
-       "  (void)dys; (void)slice; (void)desc;\n"
-       "  // Chat elements without a CG term stay zero for the whole CTA\n"
-       "  for (int s = 0; s < NSTAGE; ++s) {\n"
-       "    float* ch = reinterpret_cast<float*>(stage_ptr(smem, s) + OFF_CH);\n"
-       "    for (int t = lane; t < NB * CHS; t += 32) ch[t] = 0.f;\n"
-       "  }\n"
+       "  int4* desc = reinterpret_cast<int4*>(smem + OFF_DESC);  // (eb, nb, slice, -) of each stage\n"
+       "  (void)dyp; (void)desc;\n"
+       "  const int E = rowptr[n_recv];\n"
+       "  (void)E;\n"
+       "  int last_slice[NSTAGE];\n"
+       "#pragma unroll\n"
+       "  for (int s = 0; s < NSTAGE; ++s) last_slice[s] = -1;\n"
        "  int q = 0;\n"
        "  bool dead = false;\n"
-       "  for (int i = cta_first(smem); i < n_recv && !dead; i += cta_stride(smem)) {\n"
+       "  for (int slice = 0; slice < NSLICE && !dead; ++slice) {\n"
+       "  const int chs = kChs[slice];\n"
+       "  const int4* srec = rec + rec_begin[slice];\n"
+       "  const int nrec = rec_begin[slice + 1] - rec_begin[slice];\n"
+       "  for (int i = blockIdx.x; i < n_recv && !dead; i += gridDim.x) {\n"
        "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
        "      const int s = q % NSTAGE;\n"
        "      if (q >= NSTAGE) {\n"
        "        if (!mbar_wait(empty0 + 8 * s, ((q / NSTAGE) - 1) & 1)) { if (lane == 0) atomicOr(err, 10); dead = true; break; }\n";
   if (backward)
-    o << "        if (dys) { const int2 d = desc[s]; reduce_dy(smem, s, slice, d.x, d.y, dys, lane); }\n";
+    o << "        if (dyp) { __syncwarp(); reduce_dy(smem, s, desc[s], dyp, E, lane); }\n";
   o << "      }\n"
        "      const int nb = min(NB, e1 - eb);\n"
        "      unsigned char* st = stage_ptr(smem, s);\n"
        "      float* sY = reinterpret_cast<float*>(st + OFF_Y);\n"
        "      float* ch = reinterpret_cast<float*>(st + OFF_CH);\n"
+       "      bool fresh = false;\n"
+       "#pragma unroll\n"
+       "      for (int t = 0; t < NSTAGE; ++t)\n"
+       "        if (t == s && last_slice[t] != slice) { last_slice[t] = slice; fresh = true; }\n"
+       "      if (fresh)  // Chat elements without a CG term are zero for this slice\n"
+       "        for (int t = lane; t < NB * CHS; t += 32) ch[t] = 0.f;\n"
        "      for (int t = lane; t < nb * DE; t += 32) sY[t] = Y[(size_t)eb * DE + t];\n"
-       "      if (lane == 0) desc[s] = make_int2(eb, nb);\n"
+       "      if (lane == 0) desc[s] = make_int4(eb, nb, slice, 0);\n"
        "      __syncwarp();\n"
        "      for (int b = 0; b < nb; ++b) {\n"
        "        const float* y = sY + b * DE;\n"
        "        float* cb = ch + b * chs;\n"
        "#pragma unroll 4\n"
        "        for (int r0 = lane; r0 < nrec; r0 += 32) {\n"
-       "          const int4 r = __ldg(rec + r0);\n"
+       "          const int4 r = __ldg(srec + r0);\n"
        "          cb[r.x & 0xffff] = fmaf(__int_as_float(r.y), y[(r.x >> 16) & 0xff], __int_as_float(r.z) * y[(unsigned)r.x >> 24]);\n"
        "        }\n"
        "      }\n"
        "      mbar_arrive(full0 + 8 * s);\n"
        "    }\n"
+       "  }\n"
        "  }\n";
   if (backward)
-    o << "  if (!dead && dys)\n"
+    o << "  if (!dead && dyp)\n"
          "    for (int c = max(0, q - NSTAGE); c < q; ++c) {\n"
          "      const int s = c % NSTAGE;\n"
          "      if (!mbar_wait(empty0 + 8 * s, (c / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); break; }\n"
          "      __syncwarp();\n"
-         "      const int2 d = desc[s];\n"
-         "      reduce_dy(smem, s, slice, d.x, d.y, dys, lane);\n"
+         "      reduce_dy(smem, s, desc[s], dyp, E, lane);\n"
          "    }\n";
   o << "}\n";
   return o.str();

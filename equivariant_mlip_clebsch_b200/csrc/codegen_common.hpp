@@ -77,6 +77,13 @@ void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape&
 std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
                               const KernelShape& K, bool backward);
 
+// Largest "N bytes spill stores" of a compiler log.
+int max_spill_bytes(const std::string& log);
+
+// Resident CTAs per SM the shared memory allows (at most 3): the starting
+// point of the register cap; CGTP_MIN_BLOCKS overrides it.
+int initial_min_blocks(int smem_bytes, bool* fixed);
+
 cgtp_status upload_chat_tables(const Plan& P, const std::vector<SliceLayout>& SL, void** d_ent,
                                void** d_term, std::vector<int>& ent_begin);
 

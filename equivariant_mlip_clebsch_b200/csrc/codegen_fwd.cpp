@@ -28,7 +28,7 @@
 namespace cgtp {
 
 static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>& SL, const KernelShape& K,
-                                  const std::string& kname) {
+                                  const std::string& kname, int min_blocks) {
   const FwdConfig& F = P.fcfg;
   const int S = K.S, NW = K.nw;
   std::ostringstream o;
@@ -64,13 +64,13 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
       << " paths, R=" << R << "\n";
     o << "__device__ __noinline__ void fcons_" << k
       << "(const int* __restrict__ rowptr, int n_recv, float* __restrict__ out, int* __restrict__ err,\n"
-         "    unsigned char* smem, int u0, int chs) {\n"
+         "    unsigned char* smem, int u0, int chs, int* qp) {\n"
          "  const int lane = threadIdx.x & 31;\n"
          "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
          "  bool ok[" << R << "];\n"
          "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) ok[r] = u0 + r * 32 + lane < " << MUL << ";\n"
-         "  int q = 0;\n"
-         "#pragma unroll 1\n  for (int i = cta_first(smem); i < n_recv; i += cta_stride(smem)) {\n"
+         "  int q = *qp;\n"
+         "#pragma unroll 1\n  for (int i = blockIdx.x; i < n_recv; i += gridDim.x) {\n"
          "  const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
          "  float acc[" << nacc << "];\n"
          "#pragma unroll\n  for (int k = 0; k < " << nacc << "; ++k) acc[k] = 0.f;\n"
@@ -102,30 +102,25 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
       A += R * N3;
     }
     o << "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n";
-    o << "  float* orow = out + (size_t)i * DOUT;\n"
-         "  float* wbuf = reinterpret_cast<float*>(smem + OFF_WB) + (threadIdx.x >> 5) * WB;\n"
-         "  const int nch = min(" << 32 * R << ", " << MUL << " - u0);\n";
+    o << "  float* orow = out + (size_t)i * DOUT;\n";
     A = 0;
     for (int pi : r.paths) {
       const Path& p = P.paths[pi];
       const int N3 = 2 * p.l3 + 1;
-      // through the warp's buffer so that the row segment is stored coalesced
-      o << "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) {\n"
-        << "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) wbuf[(r * 32 + lane) * " << N3
-        << " + m3] = acc[" << A << " + r * " << N3 << " + m3];\n  }\n"
-        << "  __syncwarp();\n  warp_copy_out(orow + " << p.o_off << " + u0 * " << N3 << ", wbuf, nch * " << N3
-        << ", lane);\n  __syncwarp();\n";
+      o << "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) if (ok[r]) {\n    const int u = u0 + r * 32 + lane;\n"
+        << "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) orow[" << p.o_off << " + u * " << N3
+        << " + m3] = acc[" << A << " + r * " << N3 << " + m3];\n  }\n";
       A += R * N3;
     }
-    o << "  }\n}\n";
+    o << "  }\n  *qp = q;\n}\n";
   }
   // idle consumer: keeps the stage accounting of the CTA
   o << "__device__ __noinline__ void fcons_idle(const int* __restrict__ rowptr, int n_recv,\n"
-       "    int* __restrict__ err, unsigned char* smem) {\n"
+       "    int* __restrict__ err, unsigned char* smem, int* qp) {\n"
        "  const int lane = threadIdx.x & 31;\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
-       "  int q = 0;\n"
-       "#pragma unroll 1\n  for (int i = cta_first(smem); i < n_recv; i += cta_stride(smem)) {\n"
+       "  int q = *qp;\n"
+       "#pragma unroll 1\n  for (int i = blockIdx.x; i < n_recv; i += gridDim.x) {\n"
        "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
        "      const int s = q % NSTAGE;\n"
@@ -134,6 +129,7 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
        "      if (lane == 0) mbar_arrive(empty0 + 8 * s);\n"
        "    }\n"
        "  }\n"
+       "  *qp = q;\n"
        "}\n";
   o << "__constant__ int kShape[" << S * NW << "] = {";
   for (int s = 0; s < S; ++s)
@@ -146,37 +142,28 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
   o << "};\n__constant__ int kEntBegin[" << S + 1 << "] = {";
   for (int v : P.fwd_ent_begin) o << v << ",";
   o << "};\n";
-  // resident CTAs to plan registers for: as many as shared memory allows (at
-  // most 3), or CGTP_MIN_BLOCKS when set (1 leaves registers uncapped)
-  int min_blocks = std::max(1, std::min(3, (228 * 1024) / (K.smem + 1024)));
-  if (const char* mb = std::getenv("CGTP_MIN_BLOCKS")) min_blocks = std::max(1, std::atoi(mb));
   o << "extern \"C\" __global__ void __launch_bounds__((NW + 2) * 32, " << min_blocks << ") " << kname
     << "(const int* __restrict__ rowptr, const int* __restrict__ col, const float* __restrict__ x,\n"
        "    const float* __restrict__ Y, const float* __restrict__ W, float* __restrict__ out,\n"
-       "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err, const SliceGrid sgrid) {\n"
+       "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err) {\n"
        "  extern __shared__ __align__(128) unsigned char smem[];\n"
-       "  (void)0;\n"
        "  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  if (threadIdx.x == 0) {\n"
        "    for (int s = 0; s < NSTAGE; ++s) { mbar_init(full0 + 8 * s, FULL_COUNT); mbar_init(empty0 + 8 * s, NW); }\n"
        "    fence_mbar_init();\n"
-       "    cta_place(smem, sgrid);\n"
        "  }\n"
        "  __syncthreads();\n"
-       "  const int slice = reinterpret_cast<const int*>(smem + 240)[2];\n"
-       "  const int chs = slice_chs(slice);\n"
-       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, nullptr, err, smem, slice, lane); return; }\n"
-       "  if (warp == NW + 1) {\n"
-       "    helper_warp(rowptr, n_recv, Y, ent + kEntBegin[slice], kEntBegin[slice + 1] - kEntBegin[slice],\n"
-       "                nullptr, err, smem, slice, chs, lane);\n"
-       "    return;\n"
-       "  }\n"
-       "  const int u0 = kU0[slice * NW + warp];\n"
-       "  switch (kShape[slice * NW + warp]) {\n";
+       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, nullptr, err, smem, lane); return; }\n"
+       "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, ent, kEntBegin, nullptr, err, smem, lane); return; }\n"
+       "  int q = 0;\n"
+       "  for (int slice = 0; slice < NSLICE; ++slice) {\n"
+       "    const int slot = slice * NW + warp;\n"
+       "    const int u0 = kU0[slot], chs = kChs[slice];\n"
+       "    switch (kShape[slot]) {\n";
   for (size_t k = 0; k < shape_rep.size(); ++k)
-    o << "  case " << k << ": fcons_" << k << "(rowptr, n_recv, out, err, smem, u0, chs); break;\n";
-  o << "  default: fcons_idle(rowptr, n_recv, err, smem); break;\n  }\n}\n";
+    o << "    case " << k << ": fcons_" << k << "(rowptr, n_recv, out, err, smem, u0, chs, &q); break;\n";
+  o << "    default: fcons_idle(rowptr, n_recv, err, smem, &q); break;\n    }\n  }\n}\n";
   return o.str();
 }
 
@@ -276,8 +263,22 @@ cgtp_status build_forward(Plan& P) {
   cgtp_status st = upload_chat_tables(P, SL, &P.d_fwd_ent, &P.d_fwd_term, P.fwd_ent_begin);
   if (st != CGTP_OK) return st;
   const std::string name = "cgtp_fwd";
-  std::string src = gen_fwd_source(P, SL, K, name);
+  // register cap from the resident CTAs shared memory allows; one CTA fewer
+  // (but not below two) when the compiler reports sizeable spills
   if (K.smem > 227 * 1024) return fail(CGTP_ERR_SIZE, "forward kernel needs too much shared memory");
+  bool fixed = false;
+  const int mb0 = initial_min_blocks(K.smem, &fixed);
+  const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
+  std::string src;
+  for (int mb = mb0; mb >= mb_floor; --mb) {
+    src = gen_fwd_source(P, SL, K, name, mb);
+    P.fwd.threads = (F.nw + 2) * 32;
+    P.fwd.smem = K.smem;
+    cgtp_status cst = jit_compile(src, name, P.fwd);
+    if (cst != CGTP_OK) return cst;
+    if (mb == mb_floor || max_spill_bytes(P.fwd.log) <= 64) break;
+    jit_unload(P.fwd);
+  }
   P.fwd.threads = (F.nw + 2) * 32;
   P.fwd.smem = K.smem;
   if (const char* d = std::getenv("CGTP_DUMP_SOURCE")) {
@@ -287,7 +288,7 @@ cgtp_status build_forward(Plan& P) {
       std::fclose(f);
     }
   }
-  return jit_compile(src, name, P.fwd);
+  return CGTP_OK;
 }
 
 }  // namespace cgtp
