@@ -100,8 +100,8 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       << "#pragma unroll 1\n  for (int i = blockIdx.x; i < n_recv; i += gridDim.x) {\n"
       << "  const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
       << "  if (e1 == e0) continue;\n"
-      << "  const int gb = kr & 1;\n"
-      << "  if (!mbar_wait(gfull0 + 8 * gb, (kr >> 1) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
+      << "  const int gb = kr % GBUF;\n"
+      << "  if (!mbar_wait(gfull0 + 8 * gb, (kr / GBUF) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
       << "  const float* sg = reinterpret_cast<const float*>(smem + OFF_G) + gb * GS;\n"
       << "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
       << "    const int s = q % NSTAGE;\n"
@@ -222,7 +222,7 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
        "      __syncwarp();\n"
        "      if (lane == 0) mbar_arrive(empty0 + 8 * s);\n"
        "    }\n"
-       "    if (lane == 0) mbar_arrive(gempty0 + 8 * (kr & 1));\n"
+       "    if (lane == 0) mbar_arrive(gempty0 + 8 * (kr % GBUF));\n"
        "    ++kr;\n"
        "  }\n"
        "  *qp = q;\n"

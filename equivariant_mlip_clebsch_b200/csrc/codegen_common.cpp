@@ -127,8 +127,11 @@ void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape&
     if (backward) b += r128(4L * K.nw * B * P.D_e);
     return b;
   };
-  const long fixed = 256 + (backward ? 2L * r128(4L * K.GS) : 0)  // two grad_out buffers
-                     + r128(4L * K.nw * K.WB);                      // store staging
+  // two grad_out buffers overlap the next receiver's load with this one's
+  // compute; wide rows (Lmax 6) keep one so more CTAs fit
+  K.gbufs = (backward && 2L * r128(4L * K.GS) > 48 * 1024) ? 1 : 2;
+  const long fixed = 256 + (backward ? (long)K.gbufs * r128(4L * K.GS) : 0)  // grad_out buffers
+                     + r128(4L * K.nw * K.WB);                                 // store staging
   // two or three CTAs per SM when it fits, at least two stages in flight
   // wide rows (Lmax 6) may take up to half an SM to keep two edges per chunk
   const long budget =
@@ -136,6 +139,10 @@ void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape&
   K.B = 4;
   while (K.B > 1 && fixed + 2 * stage_of(K.B) > budget) K.B /= 2;
   K.stages = (int)std::min<long>(6, std::max<long>(2, (budget - fixed) / stage_of(K.B)));
+  // tuning overrides: edges per chunk and ring depth
+  if (const char* v = std::getenv("CGTP_CHUNK")) K.B = std::max(1, std::min(8, std::atoi(v)));
+  if (const char* v = std::getenv("CGTP_STAGES")) K.stages = std::max(2, std::min(6, std::atoi(v)));
+  while (K.stages > 2 && fixed + K.stages * stage_of(K.B) > 220 * 1024) --K.stages;
   K.sdy_floats = backward ? K.nw * K.B * (int)P.D_e : 0;
   K.off_stage = 256;  // mbarriers first
   K.off_w = 0;
@@ -145,7 +152,7 @@ void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape&
   K.off_dy = K.off_ch + r128(4L * K.B * K.CHS);
   K.stage_bytes = K.off_dy + (backward ? r128(4L * K.sdy_floats) : 0);
   K.off_g = K.off_stage + K.stages * K.stage_bytes;
-  K.off_wb = K.off_g + (backward ? 2 * r128(4L * K.GS) : 0);
+  K.off_wb = K.off_g + (backward ? K.gbufs * r128(4L * K.GS) : 0);
   K.smem = K.off_wb + r128(4L * K.nw * K.WB);
 }
 
@@ -186,7 +193,8 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
     << "\n#define OFF_STAGE " << K.off_stage << "\n#define OFF_W " << K.off_w << "\n#define OFF_X "
     << K.off_x << "\n#define OFF_Y " << K.off_y << "\n#define OFF_CH " << K.off_ch << "\n#define OFF_DY "
     << K.off_dy << "\n#define OFF_G " << K.off_g << "\n#define GS " << K.GS << "\n#define WB " << K.WB
-    << "\n#define OFF_WB " << K.off_wb << "\n#define FULL_COUNT 64\n";
+    << "\n#define OFF_WB " << K.off_wb << "\n#define FULL_COUNT 64\n#define GBUF " << K.gbufs << "\n#define YPL "
+    << (K.B * P.D_e + 31) / 32 << "\n";
   // shared-memory header: full[NSTAGE], empty[NSTAGE], gfull[2], gempty[2]
   // mbarriers, then the helper's per-stage chunk descriptors
   o << "#define OFF_GFULL (2 * NSTAGE * 8)\n#define OFF_GEMPTY (OFF_GFULL + 16)\n#define OFF_DESC (OFF_GEMPTY + 16)\n";
@@ -239,9 +247,9 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
                        sl.wseg[0].len == P.U && sl.ws == P.U;
     o << "    case " << s << ": {\n";
     if (backward) {
-      o << "      {  // this receiver's grad_out pieces into buffer k & 1\n"
-           "        const int gb = k & 1;\n"
-           "        if (k >= 2 && !mbar_wait(gempty0 + 8 * gb, ((k >> 1) - 1) & 1)) { if (lane == 0) atomicOr(err, 10); dead = true; break; }\n"
+      o << "      {  // this receiver's grad_out pieces into buffer k % GBUF\n"
+           "        const int gb = k % GBUF;\n"
+           "        if (k >= GBUF && !mbar_wait(gempty0 + 8 * gb, ((k / GBUF) - 1) & 1)) { if (lane == 0) atomicOr(err, 10); dead = true; break; }\n"
            "        float* sg = reinterpret_cast<float*>(smem + OFF_G) + gb * GS;\n"
            "        const float* grow = g + (size_t)i * DOUT;\n";
       if (K.g_bulk) {
@@ -260,13 +268,13 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
     }
     o << "      for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
          "        const int s = q % NSTAGE;\n"
-         "        if (q >= NSTAGE && !mbar_wait(empty0 + 8 * s, ((q / NSTAGE) - 1) & 1)) { if (lane == 0) atomicOr(err, 10); dead = true; break; }\n"
          "        const int nb = min(NB, e1 - eb);\n"
+         "        const int jj = (lane < nb) ? __ldg(col + eb + lane) : 0;  // read before the wait\n"
+         "        if (q >= NSTAGE && !mbar_wait(empty0 + 8 * s, ((q / NSTAGE) - 1) & 1)) { if (lane == 0) atomicOr(err, 10); dead = true; break; }\n"
          "        unsigned char* st = stage_ptr(smem, s);\n"
          "        float* sW = reinterpret_cast<float*>(st + OFF_W);\n"
          "        float* sX = reinterpret_cast<float*>(st + OFF_X);\n"
          "        (void)sW; (void)sX;\n"
-         "        const int jj = (lane < nb) ? col[eb + lane] : 0;\n"
          "        (void)jj;\n"
          "        if (lane == 0) mbar_expect_tx(full0 + 8 * s, (u32)nb * "
       << ((K.w_bulk ? wb : 0) + (K.x_bulk ? xb : 0)) << ");\n"
@@ -345,12 +353,16 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
        "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
        "      const int s = q % NSTAGE;\n"
+       "      const int nb = min(NB, e1 - eb);\n"
+       "      // this chunk's Y values travel while the stage is still in use\n"
+       "      float yv[YPL];\n"
+       "#pragma unroll\n"
+       "      for (int k = 0; k < YPL; ++k) { const int t = lane + 32 * k; yv[k] = t < nb * DE ? __ldg(Y + (size_t)eb * DE + t) : 0.f; }\n"
        "      if (q >= NSTAGE) {\n"
        "        if (!mbar_wait(empty0 + 8 * s, ((q / NSTAGE) - 1) & 1)) { if (lane == 0) atomicOr(err, 10); dead = true; break; }\n";
   if (backward)
     o << "        if (dyp) { __syncwarp(); reduce_dy(smem, s, desc[s], dyp, E, lane); }\n";
   o << "      }\n"
-       "      const int nb = min(NB, e1 - eb);\n"
        "      unsigned char* st = stage_ptr(smem, s);\n"
        "      float* sY = reinterpret_cast<float*>(st + OFF_Y);\n"
        "      float* ch = reinterpret_cast<float*>(st + OFF_CH);\n"
@@ -360,7 +372,8 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
        "        if (t == s && last_slice[t] != slice) { last_slice[t] = slice; fresh = true; }\n"
        "      if (fresh)  // Chat elements without a CG term are zero for this slice\n"
        "        for (int t = lane; t < NB * CHS; t += 32) ch[t] = 0.f;\n"
-       "      for (int t = lane; t < nb * DE; t += 32) sY[t] = Y[(size_t)eb * DE + t];\n"
+       "#pragma unroll\n"
+       "      for (int k = 0; k < YPL; ++k) { const int t = lane + 32 * k; if (t < nb * DE) sY[t] = yv[k]; }\n"
        "      if (lane == 0) desc[s] = make_int4(eb, nb, slice, 0);\n"
        "      __syncwarp();\n"
        "      for (int b = 0; b < nb; ++b) {\n"

@@ -65,6 +65,7 @@ struct KernelShape {
   int off_stage = 0, stage_bytes = 0, off_w = 0, off_x = 0, off_y = 0, off_ch = 0, off_dy = 0;
   int off_g = 0, smem = 0;
   int WB = 0;       // per-consumer-warp staging buffer for coalesced row stores (floats)
+  int gbufs = 2;    // grad_out row buffers (backward)
   int off_wb = 0;
 };
 

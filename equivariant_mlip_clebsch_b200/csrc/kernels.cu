@@ -84,7 +84,8 @@ __global__ void __launch_bounds__(128) sph_harm_kernel(int64_t E, const float* _
   for (int t = threadIdx.x; t < n; t += 128) dst[t] = tile[t];
 }
 
-// dx[j][c] = sum over the sender's edges t (ascending) of m[perm_T[t]][c]
+// dx[j][c] = sum over the sender's edges t (ascending) of m[perm_T[t]][c];
+// the sum runs in edge order (bitwise reproducible), four rows in flight.
 __global__ void __launch_bounds__(128) segment_rows_kernel(int64_t width,
                                                            const int32_t* __restrict__ rowptr_T,
                                                            const int32_t* __restrict__ perm_T,
@@ -96,8 +97,22 @@ __global__ void __launch_bounds__(128) segment_rows_kernel(int64_t width,
     const int64_t w4 = width >> 2;
     for (int64_t c = threadIdx.x + (int64_t)blockIdx.y * 128; c < w4; c += 128 * (int64_t)gridDim.y) {
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int t = t0; t < t1; ++t) {
-        const float4 v = __ldcs(reinterpret_cast<const float4*>(m + (int64_t)perm_T[t] * width) + c);
+      int t = t0;
+      for (; t + 4 <= t1; t += 4) {
+        float4 v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          v[k] = __ldcs(reinterpret_cast<const float4*>(m + (int64_t)__ldg(perm_T + t + k) * width) + c);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          acc.x += v[k].x;
+          acc.y += v[k].y;
+          acc.z += v[k].z;
+          acc.w += v[k].w;
+        }
+      }
+      for (; t < t1; ++t) {
+        const float4 v = __ldcs(reinterpret_cast<const float4*>(m + (int64_t)__ldg(perm_T + t) * width) + c);
         acc.x += v.x;
         acc.y += v.y;
         acc.z += v.z;
