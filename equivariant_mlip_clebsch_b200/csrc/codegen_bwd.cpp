@@ -2,11 +2,10 @@
 //
 // Given g = dL/dout (LunaTP, arXiv 2610.18393, Table 11 lists the backward
 // outputs x-bar, y-bar, w-bar), per edge e = (i <- j), path p, channel u:
-//   t[m3]  = sum_m1 Chat[m3][m1] x[j][u][m1]            (as in the forward)
-//   dW[e][k0+u]      = sum_m3 g[i][u][m3] t[m3]
-//   h[m3]  = W[e][k0+u] g[i][u][m3]
-//   msg[e][u][m1]   += sum_m3 Chat[m3][m1] h[m3]        (over the paths of the irrep)
-//   dY[e][l2^2+m2]  += sum_{u,m1,m3} C[m1][m2][m3] x[j][u][m1] h[m3]
+//   s[m1]  = sum_m3 Chat[m3][m1] g[i][u][m3]
+//   dW[e][k0+u]      = sum_m1 x[j][u][m1] s[m1]   (= sum_m3 g (Chat x)[m3])
+//   msg[e][u][m1]   += W[e][k0+u] s[m1]           (over the paths of the irrep)
+//   dY[e][l2^2+m2]  += sum_{u,m1,m3} C[m1][m2][m3] W[e][k0+u] x[j][u][m1] g[i][u][m3]
 // and dx[j] = sum over the edges leaving j of msg[e] (a second, sender-major
 // pass over the transpose edge list, kernels.cu).
 //
@@ -25,6 +24,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
+#include <functional>
 #include <numeric>
 #include <sstream>
 
@@ -147,18 +147,19 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
         const int pi = ps[q];
         const Path& p = P.paths[pi];
         const int N3 = 2 * p.l3 + 1, n2 = 2 * p.l2 + 1;
-        o << "        {\n          float w[" << R << "], gv[" << R << "][" << N3 << "], hh[" << R << "][" << N3
-          << "], dw[" << R << "];\n"
+        o << "        {\n          float w[" << R << "], gv[" << R << "][" << N3 << "], dw[" << R << "];\n"
           << "#pragma unroll\n          for (int r = 0; r < " << R << "; ++r) {\n"
           << "            const int u = u0 + r * 32 + lane;\n"
           << "            w[r] = ok[r] ? wr[" << sl.w_st.at(pi) << " + u] : 0.f;\n"
           << "#pragma unroll\n            for (int m3 = 0; m3 < " << N3 << "; ++m3) gv[r][m3] = ok[r] ? sg["
           << sl.g_st.at(pi) << " + u * " << N3 << " + m3] : 0.f;\n          }\n"
           << "          bpath<" << N1 << "," << N3 << "," << R << ">(chb + " << sl.ch_off.at(pi)
-          << ", xv, w, gv, hh, mx, dw);\n"
+          << ", xv, w, gv, mx, dw);\n"
           << "          if (dWrow) {\n#pragma unroll\n            for (int r = 0; r < " << R
           << "; ++r) if (ok[r]) dWrow[" << p.k0 << " + u0 + r * 32 + lane] = dw[r];\n          }\n"
-          << "          if (sdy) {\n#pragma unroll\n            for (int r = 0; r < " << R << "; ++r) {\n";
+          << "          if (sdy) {\n#pragma unroll\n            for (int r = 0; r < " << R << "; ++r) {\n"
+          << "              float wx[" << N1 << "];\n#pragma unroll\n              for (int m1 = 0; m1 < " << N1
+          << "; ++m1) wx[m1] = w[r] * xv[r][m1];\n";
         const double* C = P.coeff.data() + p.c_off;
         for (int m1 = 0; m1 < N1; ++m1)
           for (int m3 = 0; m3 < N3; ++m3) {
@@ -168,7 +169,7 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
               if (c != 0.0) t.push_back({m2, c});
             }
             if (t.empty()) continue;
-            o << "              { const float pr = xv[r][" << m1 << "] * hh[r][" << m3 << "];";
+            o << "              { const float pr = wx[" << m1 << "] * gv[r][" << m3 << "];";
             for (auto& tc : t)
               o << " z[" << zo + tc.first << "] = fmaf(" << flt(tc.second) << ", pr, z[" << zo + tc.first << "]);";
             o << " }\n";
@@ -269,80 +270,254 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
   return o.str();
 }
 
+namespace {
+
+// One backward warp role option for a hidden irrep: R channels per lane,
+// nph edge phases.
+struct BwdOption {
+  int R, nph, roles;
+  double cost;  // instructions per chunk of the costliest role
+};
+
+struct BwdIrrep {
+  int a;
+  std::vector<BwdOption> opts;
+};
+
+// Instructions one warp issues per edge for R channel sets of irrep a (all
+// its paths): the s, dW, msg and dY arithmetic, shared loads, stores, and the
+// lane reduction of the dY partials.
+double bwd_edge_cost(const Plan& P, int a, int R) {
+  const int n1 = 2 * P.in[a].l + 1;
+  auto pow2 = [](int n) { int v = 1; while (v < n) v <<= 1; return v; };
+  double c = 2.0 * R * n1;  // x loads, msg staging
+  std::vector<char> l2seen(P.L + 1, 0);
+  for (size_t k = 0; k < P.paths.size(); ++k) {
+    const Path& p = P.paths[k];
+    if (p.irrep != a) continue;
+    const int n2 = 2 * p.l2 + 1, n3 = 2 * p.l3 + 1;
+    int nnz = 0, pairs = 0;
+    const double* C = P.coeff.data() + p.c_off;
+    for (int m1 = 0; m1 < n1; ++m1)
+      for (int m3 = 0; m3 < n3; ++m3) {
+        int t = 0;
+        for (int m2 = 0; m2 < n2; ++m2) t += C[((size_t)m1 * n2 + m2) * n3 + m3] != 0.0;
+        nnz += t;
+        pairs += t > 0;
+      }
+    c += R * ((double)n1 * n3 + 3.0 * n1 + n3 + 2.0 + pairs + nnz) + (double)n3 * ((n1 + 3) / 4);
+    l2seen[p.l2] = 1;
+  }
+  if (P.D_e <= 32) {
+    c += 2.0 * pow2((int)P.D_e) + 8.0;
+  } else {
+    for (int l2 = 0; l2 <= P.L; ++l2)
+      if (l2seen[l2]) c += 2.0 * pow2(2 * l2 + 1) + 8.0;
+  }
+  return c;
+}
+
+// Smallest per-chunk time of a slice holding the given irreps with NW warps:
+// the least bound T such that every irrep has an option no costlier than T
+// and the options' roles fit NW.  Returns -1 when nothing fits.
+double slice_time(const std::vector<BwdIrrep>& W, const std::vector<int>& members, int NW,
+                  std::vector<int>* choice) {
+  std::vector<double> cand;
+  for (int m : members)
+    for (auto& o : W[m].opts) cand.push_back(o.cost);
+  std::sort(cand.begin(), cand.end());
+  cand.erase(std::unique(cand.begin(), cand.end()), cand.end());
+  for (double T : cand) {
+    int roles = 0;
+    std::vector<int> pick;
+    bool ok = true;
+    for (int m : members) {
+      int best = -1;
+      for (size_t k = 0; k < W[m].opts.size(); ++k) {
+        const BwdOption& o = W[m].opts[k];
+        if (o.cost <= T && (best < 0 || o.roles < W[m].opts[best].roles ||
+                            (o.roles == W[m].opts[best].roles && o.cost < W[m].opts[best].cost)))
+          best = (int)k;
+      }
+      if (best < 0) {
+        ok = false;
+        break;
+      }
+      roles += W[m].opts[best].roles;
+      pick.push_back(best);
+    }
+    if (ok && roles <= NW) {
+      if (choice) *choice = pick;
+      return T;
+    }
+  }
+  return -1.0;
+}
+
+// Every set partition of {0..n-1} as restricted growth strings.
+void partitions(int n, std::vector<std::vector<int>>& out) {
+  std::vector<int> a(n, 0);
+  std::function<void(int, int)> rec = [&](int i, int mx) {
+    if (i == n) {
+      out.push_back(a);
+      return;
+    }
+    for (int v = 0; v <= mx + 1; ++v) {
+      a[i] = v;
+      rec(i + 1, std::max(mx, v));
+    }
+  };
+  if (n > 0) rec(0, -1);
+}
+
+}  // namespace
+
 cgtp_status build_backward(Plan& P) {
   P.bwd_roles.clear();
   FwdConfig& F = P.bcfg;
   F = FwdConfig();
   if (P.paths.empty()) return CGTP_OK;
-  // one slice per hidden irrep with paths; roles = channel blocks x edge phases
-  struct IrrepWork {
-    int a, R, nblk;
-    double cost;
-  };
-  std::vector<IrrepWork> iw;
+  // ---- per hidden irrep: the edge cost of each channel width per lane
+  std::vector<int> work_irreps;
   for (size_t a = 0; a < P.in.size(); ++a) {
-    const Irrep& h = P.in[a];
-    const int n1 = 2 * h.l + 1;
-    double c = 0.0;
     bool any = false;
-    for (size_t k = 0; k < P.paths.size(); ++k)
-      if (P.paths[k].irrep == (int)a) {
-        const int n3 = 2 * P.paths[k].l3 + 1;
-        c += 2.0 * n1 * n3 + 3.0 * n3 + 2.0 * path_nnz(P, (int)k);
-        any = true;
-      }
-    if (!any) {
+    for (auto& p : P.paths) any = any || p.irrep == (int)a;
+    if (any)
+      work_irreps.push_back((int)a);
+    else
       P.bwd_irrep_gap = true;
-      continue;
-    }
-    const int R = (h.mul >= 64 && h.l <= 3) ? 2 : 1;
-    const int nblk = (h.mul + 32 * R - 1) / (32 * R);
-    iw.push_back({(int)a, R, nblk, c * R});
   }
-  std::vector<SliceLayout> SL;
+  const int n = (int)work_irreps.size();
+  std::vector<std::vector<int>> parts;
+  if (n <= 8) {
+    partitions(n, parts);
+  } else {  // one slice per irrep
+    std::vector<int> a(n);
+    std::iota(a.begin(), a.end(), 0);
+    parts.push_back(a);
+  }
+  struct Best {
+    double score = 1e300;
+    int B = 0, NW = 0;
+    std::vector<std::vector<int>> slices;  // members (indices into work_irreps)
+    std::vector<std::vector<int>> pick;    // option per member
+    std::vector<BwdIrrep> W;
+  } best;
+  const int kB[] = {8, 4, 2, 1};
+  // barrier round trips, loop and address work of one chunk, in the units of
+  // bwd_edge_cost
+  const double kChunkOverhead = 80.0;
+  const int kNW[] = {4, 6, 8, 12, 16};
+  for (int B : kB) {
+    // options of every irrep for this chunk size
+    std::vector<BwdIrrep> W(n);
+    for (int i = 0; i < n; ++i) {
+      const int a = work_irreps[i];
+      const Irrep& h = P.in[a];
+      W[i].a = a;
+      std::vector<int> Rs = {1};
+      if (h.mul > 32 && h.l <= 3) Rs.push_back(2);
+      if (h.mul > 64 && h.l == 0) Rs.push_back(4);
+      for (int R : Rs) {
+        const double ce = bwd_edge_cost(P, a, R);
+        const int nblk = (h.mul + 32 * R - 1) / (32 * R);
+        for (int nph = 1; nph <= B; nph *= 2)
+          W[i].opts.push_back({R, nph, nblk * nph, ce * ((B + nph - 1) / nph)});
+      }
+    }
+    for (int NW : kNW) {
+      for (const auto& rgs : parts) {
+        const int ns = rgs.empty() ? 0 : *std::max_element(rgs.begin(), rgs.end()) + 1;
+        std::vector<std::vector<int>> slices(ns);
+        for (int i = 0; i < n; ++i) slices[rgs[i]].push_back(i);
+        double sumT = 0.0;
+        std::vector<std::vector<int>> pick(ns);
+        bool ok = true;
+        for (int s2 = 0; s2 < ns && ok; ++s2) {
+          const double T = slice_time(W, slices[s2], NW, &pick[s2]);
+          if (T < 0) ok = false;
+          sumT += T + kChunkOverhead;
+        }
+        if (!ok) continue;
+        // shared memory of this grouping at this chunk size
+        std::vector<SliceLayout> SL(ns);
+        KernelShape K;
+        K.S = ns;
+        K.nw = NW;
+        K.force_B = B;
+        int maxr = 0;
+        for (int s2 = 0; s2 < ns; ++s2) {
+          for (size_t k = 0; k < slices[s2].size(); ++k) {
+            const int a = W[slices[s2][k]].a;
+            const BwdOption& o = W[slices[s2][k]].opts[pick[s2][k]];
+            SL[s2].irreps.push_back(a);
+            for (size_t q = 0; q < P.paths.size(); ++q)
+              if (P.paths[q].irrep == a) SL[s2].paths.push_back((int)q);
+            K.WB = std::max(K.WB, 32 * o.R * (2 * P.in[a].l + 1));
+            maxr = std::max(maxr, o.R * (2 * P.in[a].l + 1));
+          }
+          std::sort(SL[s2].paths.begin(), SL[s2].paths.end());
+          layout_slice(P, SL[s2], true);
+        }
+        plan_layout(P, SL, K, true);
+        if (K.smem > 227 * 1024) continue;
+        // resident CTAs: shared memory, warps, and a register estimate
+        const int regs = std::min(255, (40 + 3 * maxr + (int)std::min<int64_t>(32, P.D_e) + 7) & ~7);
+        const int threads = (NW + 2) * 32;
+        const int ctas = std::max(
+            1, std::min({233472 / (K.smem + 1024), 64 / (NW + 2), 65536 / (threads * regs), 3}));
+        const double score = sumT / ((double)B * ctas) * (1.0 + 0.01 * NW);
+        if (score < best.score) {
+          best.score = score;
+          best.B = B;
+          best.NW = NW;
+          best.slices = slices;
+          best.pick = pick;
+          best.W = W;
+        }
+      }
+    }
+  }
+  if (best.B == 0) return fail(CGTP_ERR_SIZE, "backward kernel needs too much shared memory");
+  // ---- roles of the chosen plan: channel blocks x edge phases per irrep
+  F.S = (int)best.slices.size();
+  F.nw = best.NW;
+  F.slice_roles.assign(F.S, {});
+  std::vector<SliceLayout> SL(F.S);
   KernelShape K;
-  int maxnph = 4;
-  for (int attempt = 0; attempt < 3; ++attempt) {
-    P.bwd_roles.clear();
-    F.slice_roles.clear();
-    for (auto& w : iw) {
-      int nph = std::max(1, std::min(maxnph, 8 / std::max(1, w.nblk)));
-      while (nph & (nph - 1)) --nph;  // 1, 2 or 4
-      F.slice_roles.push_back({});
-      for (int blk = 0; blk < w.nblk; ++blk)
-        for (int ph = 0; ph < nph; ++ph) {
+  K.S = F.S;
+  K.nw = F.nw;
+  K.force_B = best.B;
+  for (int s2 = 0; s2 < F.S; ++s2) {
+    double wsum = 0.0;
+    for (size_t k = 0; k < best.slices[s2].size(); ++k) {
+      const BwdIrrep& wi = best.W[best.slices[s2][k]];
+      const BwdOption& o = wi.opts[best.pick[s2][k]];
+      const Irrep& h = P.in[wi.a];
+      const int nblk = (h.mul + 32 * o.R - 1) / (32 * o.R);
+      for (int blk = 0; blk < nblk; ++blk)
+        for (int ph = 0; ph < o.nph; ++ph) {
           BwdRole r;
-          r.irrep = w.a;
-          r.u0 = blk * 32 * w.R;
-          r.R = w.R;
+          r.irrep = wi.a;
+          r.u0 = blk * 32 * o.R;
+          r.R = o.R;
           r.ph = ph;
-          r.nph = nph;
-          r.cost = w.cost / nph;
-          F.slice_roles.back().push_back((int)P.bwd_roles.size());
+          r.nph = o.nph;
+          r.cost = o.cost;
+          F.slice_roles[s2].push_back((int)P.bwd_roles.size());
           P.bwd_roles.push_back(r);
         }
+      wsum += o.cost * o.roles;
+      SL[s2].irreps.push_back(wi.a);
+      for (size_t q = 0; q < P.paths.size(); ++q)
+        if (P.paths[q].irrep == wi.a) SL[s2].paths.push_back((int)q);
+      K.WB = std::max(K.WB, 32 * o.R * (2 * h.l + 1));
     }
-    F.S = (int)F.slice_roles.size();
-    F.weight.clear();
-    for (auto& w : iw) F.weight.push_back(w.cost * w.nblk);
-    F.nw = 0;
-    for (auto& v : F.slice_roles) F.nw = std::max<int>(F.nw, (int)v.size());
-    SL.assign(F.S, SliceLayout());
-    for (int s = 0; s < F.S; ++s) {
-      const int a = iw[s].a;
-      SL[s].irreps.push_back(a);
-      for (size_t k = 0; k < P.paths.size(); ++k)
-        if (P.paths[k].irrep == a) SL[s].paths.push_back((int)k);
-      layout_slice(P, SL[s], true);
-    }
-    K = KernelShape();
-    K.S = F.S;
-    K.nw = F.nw;
-    for (auto& r : P.bwd_roles) K.WB = std::max(K.WB, 32 * r.R * (2 * P.in[r.irrep].l + 1));
-    plan_layout(P, SL, K, true);
-    if (K.B >= maxnph) break;
-    maxnph = K.B;
+    std::sort(SL[s2].paths.begin(), SL[s2].paths.end());
+    layout_slice(P, SL[s2], true);
+    F.weight.push_back(wsum);
   }
+  plan_layout(P, SL, K, true);
   F.B = K.B;
   F.stages = K.stages;
   F.w_smem = K.w_bulk;

@@ -136,11 +136,15 @@ void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape&
   // wide rows (Lmax 6) may take up to half an SM to keep two edges per chunk
   const long budget =
       std::max<long>(72 * 1024, std::min<long>(112 * 1024, fixed + 2 * stage_of(2)));
-  K.B = 4;
-  while (K.B > 1 && fixed + 2 * stage_of(K.B) > budget) K.B /= 2;
+  if (K.force_B > 0) {
+    K.B = K.force_B;
+  } else {
+    K.B = 4;
+    while (K.B > 1 && fixed + 2 * stage_of(K.B) > budget) K.B /= 2;
+  }
   K.stages = (int)std::min<long>(6, std::max<long>(2, (budget - fixed) / stage_of(K.B)));
   // tuning overrides: edges per chunk and ring depth
-  if (const char* v = std::getenv("CGTP_CHUNK")) K.B = std::max(1, std::min(8, std::atoi(v)));
+  if (const char* v = std::getenv("CGTP_CHUNK"); v && K.force_B == 0) K.B = std::max(1, std::min(8, std::atoi(v)));
   if (const char* v = std::getenv("CGTP_STAGES")) K.stages = std::max(2, std::min(6, std::atoi(v)));
   while (K.stages > 2 && fixed + K.stages * stage_of(K.B) > 220 * 1024) --K.stages;
   K.sdy_floats = backward ? K.nw * K.B * (int)P.D_e : 0;

@@ -66,6 +66,7 @@ struct KernelShape {
   int off_g = 0, smem = 0;
   int WB = 0;       // per-consumer-warp staging buffer for coalesced row stores (floats)
   int gbufs = 2;    // grad_out row buffers (backward)
+  int force_B = 0;  // edges per chunk fixed by the caller (0: chosen from the budget)
   int off_wb = 0;
 };
 

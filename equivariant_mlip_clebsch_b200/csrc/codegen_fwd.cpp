@@ -167,6 +167,18 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
   return o.str();
 }
 
+// Instructions one warp issues per edge for a role (FMAs, shared loads).
+static double fwd_role_cost(const Plan& P, const FwdRole& r) {
+  const int n1 = 2 * P.in[r.irrep].l + 1;
+  double c = (double)r.R * n1;  // x
+  for (int pi : r.paths) {
+    const int n3 = 2 * P.paths[pi].l3 + 1;
+    const double fma = n1 == 1 ? 1 + n3 : (n1 < n3 ? n1 + n1 * n3 : n1 * n3 + n3);
+    c += r.R * (fma + 1) + (double)n3 * ((n1 + 3) / 4);
+  }
+  return c;
+}
+
 cgtp_status build_forward(Plan& P) {
   // ---- roles: per hidden irrep, channel blocks x path groups
   const int kAccBudget = 64;
@@ -191,7 +203,6 @@ cgtp_status build_forward(Plan& P) {
       sum += n3;
     }
     const int nblk = (h.mul + 32 * R - 1) / (32 * R);
-    const int n1 = 2 * h.l + 1;
     for (auto& g : groups)
       for (int blk = 0; blk < nblk; ++blk) {
         FwdRole r;
@@ -199,12 +210,14 @@ cgtp_status build_forward(Plan& P) {
         r.u0 = blk * 32 * R;
         r.R = R;
         r.paths = g;
-        double c = 0;
-        for (int pi : g) c += (double)(n1 + 1) * (2 * P.paths[pi].l3 + 1);
-        r.cost = c * R;
+        r.cost = fwd_role_cost(P, r);
         P.fwd_roles.push_back(r);
       }
   }
+  // Roles are not split further to balance them: measured on B200, more and
+  // smaller roles (single-block channel groups, split path groups) made the
+  // forward slower (more distinct code resident at once, x and Chat read by
+  // more warps), so the coarse roles above stand.
   const int NR = (int)P.fwd_roles.size();
   FwdConfig& F = P.fcfg;
   F = FwdConfig();
@@ -252,8 +265,7 @@ cgtp_status build_forward(Plan& P) {
   KernelShape K;
   K.S = F.S;
   K.nw = F.nw;
-  for (auto& r : P.fwd_roles)
-    for (int pi : r.paths) K.WB = std::max(K.WB, 32 * r.R * (2 * P.paths[pi].l3 + 1));
+  K.WB = 0;  // output rows go straight from registers to global memory
   plan_layout(P, SL, K, false);
   F.B = K.B;
   F.stages = K.stages;
