@@ -317,6 +317,34 @@ double bwd_edge_cost(const Plan& P, int a, int R) {
   return c;
 }
 
+// Registers per thread the compiler grants a block of `threads` threads when
+// `ctas` blocks share an SM (65536 registers; blocks counted in whole groups
+// of four warps; eight-register steps).
+int reg_cap(int threads, int ctas) {
+  const int t = (threads + 127) / 128 * 128;
+  return std::min(255, 65536 / (t * ctas) / 8 * 8);
+}
+
+// Registers a backward role of irrep a with R channels per lane keeps live:
+// the dY partials, x, msg and s per channel, grad_out of the widest path, the
+// Chat row, and about 28 for addresses, counters and temporaries.
+int bwd_role_regs(const Plan& P, int a, int R) {
+  const int n1 = 2 * P.in[a].l + 1;
+  int n3max = 1;
+  for (auto& p : P.paths)
+    if (p.irrep == a) n3max = std::max(n3max, 2 * p.l3 + 1);
+  auto pow2 = [](int n) { int v = 1; while (v < n) v <<= 1; return v; };
+  int vz = 0;
+  if (P.D_e <= 32) {
+    vz = pow2((int)P.D_e);
+  } else {
+    for (auto& p : P.paths)
+      if (p.irrep == a) vz = std::max(vz, pow2(2 * p.l2 + 1));
+  }
+  // a quarter on top: the compiler keeps more values live than these
+  return (28 + vz + R * (3 * n1 + n3max + 2) + n1 + ((n1 + 3) & ~3)) * 5 / 4;
+}
+
 // Smallest per-chunk time of a slice holding the given irreps with NW warps:
 // the least bound T such that every irrep has an option no costlier than T
 // and the options' roles fit NW.  Returns -1 when nothing fits.
@@ -398,17 +426,23 @@ cgtp_status build_backward(Plan& P) {
   }
   struct Best {
     double score = 1e300;
-    int B = 0, NW = 0;
+    int B = 0, NW = 0, ctas = 0;
     std::vector<std::vector<int>> slices;  // members (indices into work_irreps)
     std::vector<std::vector<int>> pick;    // option per member
     std::vector<BwdIrrep> W;
   } best;
+  // Order of preference, from measurements on B200: the largest chunk that
+  // fits (it sets how many edges each stage hands over per barrier round
+  // trip, and how many are in flight), then two resident CTAs per SM when
+  // that chunk allows it, then the shortest consumer critical path per SM.
   const int kB[] = {8, 4, 2, 1};
   // barrier round trips, loop and address work of one chunk, in the units of
   // bwd_edge_cost
   const double kChunkOverhead = 80.0;
-  const int kNW[] = {4, 6, 8, 12, 16};
+  // consumer warps per CTA (6 measured slower than 4 or 8 on the Lmax 2 case)
+  const int kNW[] = {4, 8, 12, 16};
   for (int B : kB) {
+    if (best.B != 0) break;
     // options of every irrep for this chunk size
     std::vector<BwdIrrep> W(n);
     for (int i = 0; i < n; ++i) {
@@ -425,6 +459,7 @@ cgtp_status build_backward(Plan& P) {
           W[i].opts.push_back({R, nph, nblk * nph, ce * ((B + nph - 1) / nph)});
       }
     }
+    for (int min_ctas = 2; min_ctas >= 1 && best.B == 0; --min_ctas)
     for (int NW : kNW) {
       for (const auto& rgs : parts) {
         const int ns = rgs.empty() ? 0 : *std::max_element(rgs.begin(), rgs.end()) + 1;
@@ -454,7 +489,7 @@ cgtp_status build_backward(Plan& P) {
             for (size_t q = 0; q < P.paths.size(); ++q)
               if (P.paths[q].irrep == a) SL[s2].paths.push_back((int)q);
             K.WB = std::max(K.WB, 32 * o.R * (2 * P.in[a].l + 1));
-            maxr = std::max(maxr, o.R * (2 * P.in[a].l + 1));
+            maxr = std::max(maxr, bwd_role_regs(P, a, o.R));
           }
           std::sort(SL[s2].paths.begin(), SL[s2].paths.end());
           layout_slice(P, SL[s2], true);
@@ -462,11 +497,16 @@ cgtp_status build_backward(Plan& P) {
         plan_layout(P, SL, K, true);
         if (K.smem > 227 * 1024) continue;
         // resident CTAs: shared memory, warps, and a register estimate
-        const int regs = std::min(255, (40 + 3 * maxr + (int)std::min<int64_t>(32, P.D_e) + 7) & ~7);
+        // the most CTAs (up to three) whose register share still holds the
+        // role's estimate; none: the roles would spill
         const int threads = (NW + 2) * 32;
-        const int ctas = std::max(
-            1, std::min({233472 / (K.smem + 1024), 64 / (NW + 2), 65536 / (threads * regs), 3}));
-        const double score = sumT / ((double)B * ctas) * (1.0 + 0.01 * NW);
+        int ctas = 0;
+        for (int c = std::min({3, 233472 / (K.smem + 1024), 64 / (NW + 2)}); c >= 1 && !ctas; --c)
+          if (maxr <= reg_cap(threads, c)) ctas = c;
+        if (ctas < min_ctas) continue;
+        // resident CTAs weigh more than their count: each brings its own ring
+        // of stages, so the SM keeps more loads in flight
+        const double score = sumT / std::pow((double)ctas, 1.5) * (1.0 + 0.01 * NW);
         if (score < best.score) {
           best.score = score;
           best.B = B;
@@ -474,6 +514,7 @@ cgtp_status build_backward(Plan& P) {
           best.slices = slices;
           best.pick = pick;
           best.W = W;
+          best.ctas = ctas;
         }
       }
     }
@@ -525,12 +566,15 @@ cgtp_status build_backward(Plan& P) {
 
   cgtp_status st = upload_chat_tables(P, SL, &P.d_bwd_ent, &P.d_bwd_term, P.bwd_ent_begin);
   if (st != CGTP_OK) return st;
+  for (size_t k = 0; k + 1 < P.bwd_ent_begin.size(); ++k)
+    K.rec_max = std::max(K.rec_max, P.bwd_ent_begin[k + 1] - P.bwd_ent_begin[k]);
   const std::string name = "cgtp_bwd";
   // register cap from the resident CTAs shared memory allows; one CTA fewer
   // (but not below two) when the compiler reports sizeable spills
   if (K.smem > 227 * 1024) return fail(CGTP_ERR_SIZE, "backward kernel needs too much shared memory");
   bool fixed = false;
-  const int mb0 = initial_min_blocks(K.smem, &fixed);
+  int mb0 = initial_min_blocks(K.smem, &fixed);
+  if (!fixed) mb0 = std::min(mb0, best.ctas);  // the planner's register share
   const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
   std::string src;
   for (int mb = mb0; mb >= mb_floor; --mb) {

@@ -353,6 +353,16 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
        "  const int chs = kChs[slice];\n"
        "  const int4* srec = rec + rec_begin[slice];\n"
        "  const int nrec = rec_begin[slice + 1] - rec_begin[slice];\n"
+       "  (void)srec; (void)nrec;\n";
+  const int KR = (K.rec_max + 31) / 32;
+  const bool rec_regs = KR <= 12;
+  if (rec_regs)  // the slice's records stay in registers: no loads in the Chat loop
+    o << "  int rd[" << KR << "];\n  float rc0[" << KR << "], rc1[" << KR << "];\n"
+      << "  const int nk = (nrec - lane + 31) >> 5;\n"
+      << "#pragma unroll\n  for (int k = 0; k < " << KR << "; ++k) {\n"
+      << "    const int4 r = k < nk ? __ldg(srec + lane + 32 * k) : make_int4(0, 0, 0, 0);\n"
+      << "    rd[k] = r.x;\n    rc0[k] = __int_as_float(r.y);\n    rc1[k] = __int_as_float(r.z);\n  }\n";
+  o <<
        "  for (int i = blockIdx.x; i < n_recv && !dead; i += gridDim.x) {\n"
        "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
@@ -380,16 +390,28 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
        "      for (int k = 0; k < YPL; ++k) { const int t = lane + 32 * k; if (t < nb * DE) sY[t] = yv[k]; }\n"
        "      if (lane == 0) desc[s] = make_int4(eb, nb, slice, 0);\n"
        "      __syncwarp();\n"
-       "      for (int b = 0; b < nb; ++b) {\n"
-       "        const float* y = sY + b * DE;\n"
-       "        float* cb = ch + b * chs;\n"
-       "#pragma unroll 4\n"
-       "        for (int r0 = lane; r0 < nrec; r0 += 32) {\n"
-       "          const int4 r = __ldg(srec + r0);\n"
-       "          cb[r.x & 0xffff] = fmaf(__int_as_float(r.y), y[(r.x >> 16) & 0xff], __int_as_float(r.z) * y[(unsigned)r.x >> 24]);\n"
-       "        }\n"
-       "      }\n"
-       "      mbar_arrive(full0 + 8 * s);\n"
+       "";
+  if (rec_regs)
+    o << "#pragma unroll\n"
+         "      for (int k = 0; k < " << KR << "; ++k) {\n"
+         "        if (k < nk) {\n"
+         "          const int d = rd[k] & 0xffff, ia = (rd[k] >> 16) & 0xff, ib = (unsigned)rd[k] >> 24;\n"
+         "#pragma unroll\n"
+         "          for (int b = 0; b < NB; ++b)\n"
+         "            if (b < nb) ch[b * chs + d] = fmaf(rc0[k], sY[b * DE + ia], rc1[k] * sY[b * DE + ib]);\n"
+         "        }\n"
+         "      }\n";
+  else
+    o << "      for (int b = 0; b < nb; ++b) {\n"
+         "        const float* y = sY + b * DE;\n"
+         "        float* cb = ch + b * chs;\n"
+         "#pragma unroll 4\n"
+         "        for (int r0 = lane; r0 < nrec; r0 += 32) {\n"
+         "          const int4 r = __ldg(srec + r0);\n"
+         "          cb[r.x & 0xffff] = fmaf(__int_as_float(r.y), y[(r.x >> 16) & 0xff], __int_as_float(r.z) * y[(unsigned)r.x >> 24]);\n"
+         "        }\n"
+         "      }\n";
+  o << "      mbar_arrive(full0 + 8 * s);\n"
        "    }\n"
        "  }\n"
        "  }\n";

@@ -67,6 +67,7 @@ struct KernelShape {
   int WB = 0;       // per-consumer-warp staging buffer for coalesced row stores (floats)
   int gbufs = 2;    // grad_out row buffers (backward)
   int force_B = 0;  // edges per chunk fixed by the caller (0: chosen from the budget)
+  int rec_max = 0;  // most Chat records of a slice
   int off_wb = 0;
 };
 

@@ -189,8 +189,12 @@ cgtp_status build_forward(Plan& P) {
     for (size_t k = 0; k < P.paths.size(); ++k)
       if (P.paths[k].irrep == (int)a) ps.push_back((int)k);
     if (ps.empty()) continue;
-    const int R = h.mul >= 64 ? 2 : 1;
-    const int beta = std::max(13, kAccBudget / R);
+    // wide inputs (l >= 3): one channel per lane and fewer accumulators, so
+    // that x, w*x and the Chat row still fit beside them without spilling
+    const int n1 = 2 * h.l + 1;
+    const int R = (h.mul >= 64 && h.l < 3) ? 2 : 1;
+    const int beta = h.l < 3 ? std::max(13, kAccBudget / R)
+                             : std::max(13, kAccBudget - 2 * n1 - ((n1 + 3) & ~3));
     std::vector<std::vector<int>> groups;
     int sum = 0;
     for (int pi : ps) {
@@ -203,6 +207,7 @@ cgtp_status build_forward(Plan& P) {
       sum += n3;
     }
     const int nblk = (h.mul + 32 * R - 1) / (32 * R);
+    (void)n1;
     for (auto& g : groups)
       for (int blk = 0; blk < nblk; ++blk) {
         FwdRole r;
@@ -222,7 +227,11 @@ cgtp_status build_forward(Plan& P) {
   FwdConfig& F = P.fcfg;
   F = FwdConfig();
   if (NR == 0) return CGTP_OK;  // no paths: forward writes zeros
-  const int kMaxWarps = 16;
+  // up to 16 consumer warps per CTA; 8 when the roles are register-heavy
+  // (wide inputs), so that two CTAs of (8 + 2) warps keep 96 registers each
+  int kMaxWarps = 16;
+  for (auto& r : P.fwd_roles)
+    if (P.in[r.irrep].l >= 3 && NR > 8) kMaxWarps = 8;
   F.S = (NR + kMaxWarps - 1) / kMaxWarps;
   // longest-processing-time assignment of roles to slices
   std::vector<int> order(NR);
@@ -274,6 +283,8 @@ cgtp_status build_forward(Plan& P) {
 
   cgtp_status st = upload_chat_tables(P, SL, &P.d_fwd_ent, &P.d_fwd_term, P.fwd_ent_begin);
   if (st != CGTP_OK) return st;
+  for (size_t k = 0; k + 1 < P.fwd_ent_begin.size(); ++k)
+    K.rec_max = std::max(K.rec_max, P.fwd_ent_begin[k + 1] - P.fwd_ent_begin[k]);
   const std::string name = "cgtp_fwd";
   // register cap from the resident CTAs shared memory allows; one CTA fewer
   // (but not below two) when the compiler reports sizeable spills
