@@ -59,7 +59,8 @@ def algorithmic(N, E, d_in, d_e, d_out, U, paths, coeff):
     backward: W, Y, col, rowptr, x, grad_out in; dW, dY out (the per-edge
               message buffer of the two-pass dx is an implementation choice and
               is not counted)
-    dx rows : the sender CSR in; dx out
+    bwd_reduce: the sender CSR in; dx out (the dY slice partials it also sums
+              are part of the same implementation choice and not counted)
     sph_harm: r in; Y out
     flops (factored evaluation): forward per edge and path 2 nnz(C) for
       Chat = C . Y plus u (2 (2l1+1)(2l3+1) + 2 (2l3+1)); backward per edge and
@@ -68,9 +69,8 @@ def algorithmic(N, E, d_in, d_e, d_out, U, paths, coeff):
     b = {
         "cgtp_fwd": 4 * (E * U + E * d_e + E + (N + 1) + N * d_in + N * d_out),
         "cgtp_bwd": 4 * (E * U + E * d_e + E + (N + 1) + N * d_in + N * d_out + E * U + E * d_e),
-        "bwd_dx_rows": 4 * (N + 1 + E + N * d_in),
+        "bwd_reduce": 4 * (N + 1 + E + N * d_in),
         "sph_harm": 4 * (3 * E + E * d_e),
-        "bwd_dy_slices": 4 * (2 * E * d_e),
     }
     ff = fb = 0.0
     for (l1, l2, l3, mul, xo, k0, oo, co) in paths:

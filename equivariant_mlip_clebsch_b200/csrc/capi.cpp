@@ -57,8 +57,7 @@ static cgtp_status check_device(const Plan& P) {
   return CGTP_OK;
 }
 
-static const char* kKindName[] = {"sph_harm", "cgtp_fwd", "cgtp_bwd", "bwd_dx_rows", "bwd_dy_slices",
-                                   "zero_fill"};
+static const char* kKindName[] = {"sph_harm", "cgtp_fwd", "cgtp_bwd", "bwd_reduce", "unused", "zero_fill"};
 
 // Brackets one internal launch with events when timing is on.
 struct TimedScope {
@@ -96,6 +95,17 @@ struct TimedScope {
 static unsigned persistent_grid(int blocks_per_sm, int num_sms, int64_t n_recv) {
   const int64_t T = std::max<int64_t>(1, (int64_t)blocks_per_sm * num_sms);
   return (unsigned)std::max<int64_t>(1, std::min<int64_t>(T, n_recv));
+}
+
+// Backward workspace: the per-edge messages for dx [E x D_in] and the
+// per-slice dY partials [S x E x D_e] when S > 1.  Returns the total bytes;
+// the partials' offset through the pointer when given.
+static size_t bwd_workspace_layout(const Plan& P, int64_t E, size_t* off_dyp) {
+  auto r256 = [](size_t v) { return (v + 255) & ~size_t(255); };
+  size_t b = r256((size_t)E * P.D_in * sizeof(float));
+  if (off_dyp) *off_dyp = b;
+  if (P.bcfg.S > 1) b += r256((size_t)P.bcfg.S * E * P.D_e * sizeof(float));
+  return b;
 }
 
 }  // namespace cgtp
@@ -265,9 +275,7 @@ cgtp_status cgtp_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t
   const Plan* P = reinterpret_cast<const Plan*>(plan);
   if (n_recv < 0 || n_send < 0 || E < 0) return fail(CGTP_ERR_SIZE, "negative size");
   auto r256 = [](size_t v) { return (v + 255) & ~size_t(255); };
-  size_t b = r256((size_t)E * P->D_in * sizeof(float));
-  if (P->bcfg.S > 1) b += r256((size_t)P->bcfg.S * E * P->D_e * sizeof(float));
-  *bytes = b;
+  *bytes = bwd_workspace_layout(*P, E, nullptr);
   return CGTP_OK;
 }
 
@@ -313,39 +321,33 @@ cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
     if (grad_Y) CGTP_CUDA_TRY(cudaMemsetAsync(grad_Y, 0, (size_t)E * P->D_e * sizeof(float), s));
     return CGTP_OK;
   }
-  size_t need = 0;
-  cgtp_backward_workspace_size(plan, n_recv, n_send, E, &need);
+  size_t off_dyp = 0;
+  const size_t need = bwd_workspace_layout(*P, E, &off_dyp);
   const bool need_ws = grad_x || (grad_Y && P->bcfg.S > 1);
   if (need_ws && (!workspace || workspace_bytes < need))
     return fail(CGTP_ERR_WORKSPACE, "workspace of " + std::to_string(need) + " bytes required");
   if (need_ws && ((uintptr_t)workspace & 255))
     return fail(CGTP_ERR_ALIGN, "workspace must be 256-byte aligned");
-  auto r256 = [](size_t v) { return (v + 255) & ~size_t(255); };
-  float* m = grad_x ? reinterpret_cast<float*>(workspace) : nullptr;
+  char* wsb = reinterpret_cast<char*>(workspace);
+  float* m = grad_x ? reinterpret_cast<float*>(wsb) : nullptr;
   float* dyp = nullptr;
-  if (grad_Y) {
-    dyp = P->bcfg.S > 1 ? reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
-                                                   r256((size_t)E * P->D_in * sizeof(float)))
-                        : grad_Y;
-  }
+  if (grad_Y) dyp = P->bcfg.S > 1 ? reinterpret_cast<float*>(wsb + off_dyp) : grad_Y;
   if (m && P->bwd_irrep_gap) {  // hidden irreps without paths receive zero gradient
     TimedScope ts(*P, 5, s, allow_timing);
     CGTP_CUDA_TRY(cudaMemsetAsync(m, 0, (size_t)E * P->D_in * sizeof(float), s));
   }
   if (n_recv > 0) {
     int nr = (int)n_recv;
+    const unsigned G = persistent_grid(P->bwd.blocks_per_sm, P->num_sms, n_recv);
     void* args[] = {&rowptr, &col, &x, &Y, &W, &grad_out, &grad_W, &dyp, &m, &P->d_bwd_ent, &nr, &P->d_err};
     TimedScope ts(*P, 2, s, allow_timing);
-    st = jit_launch(P->bwd, dim3(persistent_grid(P->bwd.blocks_per_sm, P->num_sms, n_recv)), args, s);
+    st = jit_launch(P->bwd, dim3(G), args, s);
     if (st != CGTP_OK) return st;
   }
-  if (grad_Y && P->bcfg.S > 1) {
-    TimedScope ts(*P, 4, s, allow_timing);
-    CGTP_CUDA_TRY(launch_sum_slices(P->bcfg.S, E * P->D_e, dyp, grad_Y, s));
-  }
-  if (grad_x) {
+  if (grad_x || (grad_Y && P->bcfg.S > 1)) {
     TimedScope ts(*P, 3, s, allow_timing);
-    CGTP_CUDA_TRY(launch_segment_rows(n_send, P->D_in, rowptr_T, perm_T, m, grad_x, s));
+    CGTP_CUDA_TRY(launch_bwd_reduce(n_send, P->D_in, rowptr_T, perm_T, m, grad_x, P->bcfg.S, E * P->D_e, dyp,
+                                    (grad_Y && P->bcfg.S > 1) ? grad_Y : nullptr, s));
   }
   return CGTP_OK;
 }

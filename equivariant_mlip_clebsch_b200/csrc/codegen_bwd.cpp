@@ -42,6 +42,15 @@ int path_nnz(const Plan& P, int pi) {
   return c;
 }
 
+// Channel blocks of a backward role unrolled together.  One: measured on
+// B200, unrolling two or four blocks (for l <= 1 inputs) was slower overall
+// than running every block in the loop, whose code is the smallest.
+int bwd_unroll(int n1, int R) {
+  (void)n1;
+  (void)R;
+  return 1;
+}
+
 std::string flt(double v) {
   char b[48];
   std::snprintf(b, sizeof b, "%.9ef", (double)(float)v);
@@ -94,12 +103,11 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       << "  const int lane = threadIdx.x & 31;\n"
       << "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
       << "  const u32 gfull0 = full0 + OFF_GFULL, gempty0 = full0 + OFF_GEMPTY;\n"
-      << "  bool ok[" << R << "];\n"
-      << "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) ok[r] = u0 + r * 32 + lane < " << MUL << ";\n"
+
       << "  int q = *qp, kr = *kp;\n"
-      << "#pragma unroll 1\n  for (int i = blockIdx.x; i < n_recv; i += gridDim.x) {\n"
-      << "  const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
-      << "  if (e1 == e0) continue;\n"
+      << "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
+      << "  const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
+      << "  if (e1 <= e0) continue;\n"
       << "  const int gb = kr % GBUF;\n"
       << "  if (!mbar_wait(gfull0 + 8 * gb, (kr / GBUF) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
       << "  const float* sg = reinterpret_cast<const float*>(smem + OFF_G) + gb * GS;\n"
@@ -119,19 +127,30 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       << "      const float* chb = sC + b * chs;\n"
       << "      float* dWrow = dW ? dW + (size_t)e * NU : nullptr;\n"
       << "      float* sdy = want_dy ? sdyw + b * DE : nullptr;\n"
-      << "      float xv[" << R << "][" << N1 << "], mx[" << R << "][" << N1 << "];\n"
-      << "#pragma unroll\n      for (int r = 0; r < " << R << "; ++r) {\n"
-      << "        const int u = u0 + r * 32 + lane;\n"
-      << "#pragma unroll\n        for (int m1 = 0; m1 < " << N1
-      << "; ++m1) { mx[r][m1] = 0.f; xv[r][m1] = ok[r] ? xr[u * " << N1 << " + m1] : 0.f; }\n"
-      << "      }\n";
-    // dY partials: one vector over every edge degree (reduced once) when
-    // (L+1)^2 <= 32, else one vector per edge degree
+      ;
+    // The R channel blocks of the role: RU of them unrolled together, the
+    // groups of RU one after another in a loop.  Few channels per lane at a
+    // time keep registers and code small; the Chat rows are read again per
+    // group (broadcast loads).
     auto pow2 = [](int n) { int v = 1; while (v < n) v <<= 1; return v; };
     const bool combined = P.D_e <= 32;
+    if (!combined && R != 1) {
+      std::fprintf(stderr, "cgtp: backward role with R > 1 needs D_e <= 32\n");
+      std::abort();
+    }
+    const int RU = bwd_unroll(N1, R);
     const int VZ = pow2((int)P.D_e);
     if (combined)
       o << "      float z[" << VZ << "];\n#pragma unroll\n      for (int t = 0; t < " << VZ << "; ++t) z[t] = 0.f;\n";
+    o << "#pragma unroll 1\n      for (int r = 0; r < " << R << "; r += " << RU << ") {\n"
+      << "      bool ok[" << RU << "];\n"
+      << "      float xv[" << RU << "][" << N1 << "], mx[" << RU << "][" << N1 << "];\n"
+      << "#pragma unroll\n      for (int v = 0; v < " << RU << "; ++v) {\n"
+      << "        const int u = u0 + (r + v) * 32 + lane;\n"
+      << "        ok[v] = u < " << MUL << ";\n"
+      << "#pragma unroll\n        for (int m1 = 0; m1 < " << N1
+      << "; ++m1) { mx[v][m1] = 0.f; xv[v][m1] = ok[v] ? xr[u * " << N1 << " + m1] : 0.f; }\n"
+      << "      }\n";
     std::vector<char> l2seen(P.L + 1, 0);
     size_t q = 0;
     while (q < ps.size()) {
@@ -147,19 +166,19 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
         const int pi = ps[q];
         const Path& p = P.paths[pi];
         const int N3 = 2 * p.l3 + 1, n2 = 2 * p.l2 + 1;
-        o << "        {\n          float w[" << R << "], gv[" << R << "][" << N3 << "], dw[" << R << "];\n"
-          << "#pragma unroll\n          for (int r = 0; r < " << R << "; ++r) {\n"
-          << "            const int u = u0 + r * 32 + lane;\n"
-          << "            w[r] = ok[r] ? wr[" << sl.w_st.at(pi) << " + u] : 0.f;\n"
-          << "#pragma unroll\n            for (int m3 = 0; m3 < " << N3 << "; ++m3) gv[r][m3] = ok[r] ? sg["
+        o << "        {\n          float w[" << RU << "], gv[" << RU << "][" << N3 << "], dw[" << RU << "];\n"
+          << "#pragma unroll\n          for (int v = 0; v < " << RU << "; ++v) {\n"
+          << "            const int u = u0 + (r + v) * 32 + lane;\n"
+          << "            w[v] = ok[v] ? wr[" << sl.w_st.at(pi) << " + u] : 0.f;\n"
+          << "#pragma unroll\n            for (int m3 = 0; m3 < " << N3 << "; ++m3) gv[v][m3] = ok[v] ? sg["
           << sl.g_st.at(pi) << " + u * " << N3 << " + m3] : 0.f;\n          }\n"
-          << "          bpath<" << N1 << "," << N3 << "," << R << ">(chb + " << sl.ch_off.at(pi)
+          << "          bpath<" << N1 << "," << N3 << "," << RU << ">(chb + " << sl.ch_off.at(pi)
           << ", xv, w, gv, mx, dw);\n"
-          << "          if (dWrow) {\n#pragma unroll\n            for (int r = 0; r < " << R
-          << "; ++r) if (ok[r]) dWrow[" << p.k0 << " + u0 + r * 32 + lane] = dw[r];\n          }\n"
-          << "          if (sdy) {\n#pragma unroll\n            for (int r = 0; r < " << R << "; ++r) {\n"
+          << "          if (dWrow) {\n#pragma unroll\n            for (int v = 0; v < " << RU
+          << "; ++v) if (ok[v]) dWrow[" << p.k0 << " + u0 + (r + v) * 32 + lane] = dw[v];\n          }\n"
+          << "          if (sdy) {\n#pragma unroll\n            for (int v = 0; v < " << RU << "; ++v) {\n"
           << "              float wx[" << N1 << "];\n#pragma unroll\n              for (int m1 = 0; m1 < " << N1
-          << "; ++m1) wx[m1] = w[r] * xv[r][m1];\n";
+          << "; ++m1) wx[m1] = w[v] * xv[v][m1];\n";
         const double* C = P.coeff.data() + p.c_off;
         for (int m1 = 0; m1 < N1; ++m1)
           for (int m3 = 0; m3 < N3; ++m3) {
@@ -169,7 +188,7 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
               if (c != 0.0) t.push_back({m2, c});
             }
             if (t.empty()) continue;
-            o << "              { const float pr = wx[" << m1 << "] * gv[r][" << m3 << "];";
+            o << "              { const float pr = wx[" << m1 << "] * gv[v][" << m3 << "];";
             for (auto& tc : t)
               o << " z[" << zo + tc.first << "] = fmaf(" << flt(tc.second) << ", pr, z[" << zo + tc.first << "]);";
             o << " }\n";
@@ -185,6 +204,18 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       }
       o << "      }\n";
     }
+    // this group's message row segment, through the warp's buffer
+    o << "      if (msg) {\n"
+      << "        float* wbuf = reinterpret_cast<float*>(smem + OFF_WB) + (threadIdx.x >> 5) * WB;\n"
+      << "#pragma unroll\n        for (int v = 0; v < " << RU << "; ++v) {\n"
+      << "#pragma unroll\n          for (int m1 = 0; m1 < " << N1 << "; ++m1) wbuf[(v * 32 + lane) * " << N1
+      << " + m1] = mx[v][m1];\n        }\n"
+      << "        __syncwarp();\n"
+      << "        const int nch = min(" << 32 * RU << ", " << MUL << " - u0 - r * 32);\n"
+      << "        if (nch > 0) warp_copy_out(msg + (size_t)e * DIN + " << P.x_off[r.irrep] << " + (u0 + r * 32) * "
+      << N1 << ", wbuf, nch * " << N1 << ", lane);\n"
+      << "        __syncwarp();\n      }\n"
+      << "      }\n";  // r
     if (combined) {
       const int LV = __builtin_ctz(VZ), sh = 5 - LV;
       o << "      if (sdy) {\n        const float v = warp_sum_many<" << VZ << ">(z, lane);\n"
@@ -196,16 +227,6 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
           o << "      if (sdy && lane == 0) {\n#pragma unroll\n        for (int t = 0; t < " << 2 * l2 + 1
             << "; ++t) sdy[" << l2 * l2 << " + t] = 0.f;\n      }\n";
     }
-    // the message row segment of this role, through the warp's buffer
-    o << "      if (msg) {\n"
-      << "        float* wbuf = reinterpret_cast<float*>(smem + OFF_WB) + (threadIdx.x >> 5) * WB;\n"
-      << "#pragma unroll\n        for (int r = 0; r < " << R << "; ++r) {\n"
-      << "#pragma unroll\n          for (int m1 = 0; m1 < " << N1 << "; ++m1) wbuf[(r * 32 + lane) * " << N1
-      << " + m1] = mx[r][m1];\n        }\n"
-      << "        __syncwarp();\n"
-      << "        warp_copy_out(msg + (size_t)e * DIN + " << P.x_off[r.irrep] << " + u0 * " << N1
-      << ", wbuf, min(" << 32 * R << ", " << MUL << " - u0) * " << N1 << ", lane);\n"
-      << "        __syncwarp();\n      }\n";
     o << "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n"
       << "  __syncwarp();\n  if (lane == 0) mbar_arrive(gempty0 + 8 * gb);\n  ++kr;\n  }\n  *qp = q;\n  *kp = kr;\n}\n";
   }
@@ -214,9 +235,9 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  const u32 gempty0 = full0 + OFF_GEMPTY;\n"
        "  int q = *qp, kr = *kp;\n"
-       "#pragma unroll 1\n  for (int i = blockIdx.x; i < n_recv; i += gridDim.x) {\n"
-       "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
-       "    if (e1 == e0) continue;\n"
+       "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
+       "    const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
+       "    if (e1 <= e0) continue;\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
        "      const int s = q % NSTAGE;\n"
        "      if (!mbar_wait(full0 + 8 * s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
@@ -290,7 +311,7 @@ struct BwdIrrep {
 double bwd_edge_cost(const Plan& P, int a, int R) {
   const int n1 = 2 * P.in[a].l + 1;
   auto pow2 = [](int n) { int v = 1; while (v < n) v <<= 1; return v; };
-  double c = 2.0 * R * n1;  // x loads, msg staging
+  double c = 2.0 * R * n1 + 12.0 * ((R + bwd_unroll(n1, R) - 1) / bwd_unroll(n1, R));  // x, msg, loop
   std::vector<char> l2seen(P.L + 1, 0);
   for (size_t k = 0; k < P.paths.size(); ++k) {
     const Path& p = P.paths[k];
@@ -305,7 +326,8 @@ double bwd_edge_cost(const Plan& P, int a, int R) {
         nnz += t;
         pairs += t > 0;
       }
-    c += R * ((double)n1 * n3 + 3.0 * n1 + n3 + 2.0 + pairs + nnz) + (double)n3 * ((n1 + 3) / 4);
+    const int groups = (R + bwd_unroll(n1, R) - 1) / bwd_unroll(n1, R);
+    c += R * ((double)n1 * n3 + 3.0 * n1 + n3 + 2.0 + pairs + nnz) + groups * (double)n3 * ((n1 + 3) / 4);
     l2seen[p.l2] = 1;
   }
   if (P.D_e <= 32) {
@@ -318,11 +340,11 @@ double bwd_edge_cost(const Plan& P, int a, int R) {
 }
 
 // Registers per thread the compiler grants a block of `threads` threads when
-// `ctas` blocks share an SM (65536 registers; blocks counted in whole groups
-// of four warps; eight-register steps).
+// `ctas` blocks share an SM: each of the four schedulers has 16384 registers
+// for its share of the warps (rounded up), in eight-register steps.
 int reg_cap(int threads, int ctas) {
-  const int t = (threads + 127) / 128 * 128;
-  return std::min(255, 65536 / (t * ctas) / 8 * 8);
+  const int warps_per_sched = ((threads / 32) * ctas + 3) / 4;
+  return std::min(255, 16384 / (warps_per_sched * 32) / 8 * 8);
 }
 
 // Registers a backward role of irrep a with R channels per lane keeps live:
@@ -341,8 +363,9 @@ int bwd_role_regs(const Plan& P, int a, int R) {
     for (auto& p : P.paths)
       if (p.irrep == a) vz = std::max(vz, pow2(2 * p.l2 + 1));
   }
-  // a quarter on top: the compiler keeps more values live than these
-  return (28 + vz + R * (3 * n1 + n3max + 2) + n1 + ((n1 + 3) & ~3)) * 5 / 4;
+  // a tenth on top: the compiler keeps a few more values live than these
+  const int RU = bwd_unroll(n1, R);  // blocks unrolled together; the rest loop
+  return (28 + vz + RU * (3 * n1 + n3max + 2) + n1 + ((n1 + 3) & ~3)) * 11 / 10;
 }
 
 // Smallest per-chunk time of a slice holding the given irreps with NW warps:
@@ -439,8 +462,8 @@ cgtp_status build_backward(Plan& P) {
   // barrier round trips, loop and address work of one chunk, in the units of
   // bwd_edge_cost
   const double kChunkOverhead = 80.0;
-  // consumer warps per CTA (6 measured slower than 4 or 8 on the Lmax 2 case)
-  const int kNW[] = {4, 8, 12, 16};
+  // consumer warps per CTA: 6, 12 and 16 measured slower than 4 or 8 on B200
+  const int kNW[] = {4, 8};
   for (int B : kB) {
     if (best.B != 0) break;
     // options of every irrep for this chunk size
@@ -449,9 +472,13 @@ cgtp_status build_backward(Plan& P) {
       const int a = work_irreps[i];
       const Irrep& h = P.in[a];
       W[i].a = a;
+      // channel blocks one warp takes in turn (the dY partials of all blocks
+      // must fit one reduction: only when (L+1)^2 <= 32)
       std::vector<int> Rs = {1};
-      if (h.mul > 32 && h.l <= 3) Rs.push_back(2);
-      if (h.mul > 64 && h.l == 0) Rs.push_back(4);
+      if (P.D_e <= 32) {
+        if (h.mul > 32) Rs.push_back(2);
+        if (h.mul > 64) Rs.push_back(4);
+      }
       for (int R : Rs) {
         const double ce = bwd_edge_cost(P, a, R);
         const int nblk = (h.mul + 32 * R - 1) / (32 * R);
@@ -488,7 +515,7 @@ cgtp_status build_backward(Plan& P) {
             SL[s2].irreps.push_back(a);
             for (size_t q = 0; q < P.paths.size(); ++q)
               if (P.paths[q].irrep == a) SL[s2].paths.push_back((int)q);
-            K.WB = std::max(K.WB, 32 * o.R * (2 * P.in[a].l + 1));
+            K.WB = std::max(K.WB, 32 * bwd_unroll(2 * P.in[a].l + 1, o.R) * (2 * P.in[a].l + 1));
             maxr = std::max(maxr, bwd_role_regs(P, a, o.R));
           }
           std::sort(SL[s2].paths.begin(), SL[s2].paths.end());
@@ -552,7 +579,7 @@ cgtp_status build_backward(Plan& P) {
       SL[s2].irreps.push_back(wi.a);
       for (size_t q = 0; q < P.paths.size(); ++q)
         if (P.paths[q].irrep == wi.a) SL[s2].paths.push_back((int)q);
-      K.WB = std::max(K.WB, 32 * o.R * (2 * h.l + 1));
+      K.WB = std::max(K.WB, 32 * bwd_unroll(2 * h.l + 1, o.R) * (2 * h.l + 1));
     }
     std::sort(SL[s2].paths.begin(), SL[s2].paths.end());
     layout_slice(P, SL[s2], true);

@@ -202,6 +202,12 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
   // shared-memory header: full[NSTAGE], empty[NSTAGE], gfull[2], gempty[2]
   // mbarriers, then the helper's per-stage chunk descriptors
   o << "#define OFF_GFULL (2 * NSTAGE * 8)\n#define OFF_GEMPTY (OFF_GFULL + 16)\n#define OFF_DESC (OFF_GEMPTY + 16)\n";
+  // the receivers a CTA walks: blockIdx.x, + gridDim.x, ...  (Edge-balanced
+  // ranges for the backward were measured on B200: faster on small graphs,
+  // but the range search, in the kernel or as a launch of its own, cost more
+  // than it saved on the larger cases.)
+  o << "#define RECV_FIRST ((int)blockIdx.x)\n#define RECV_END n_recv\n#define RECV_STEP ((int)gridDim.x)\n"
+       "#define EDGE_LO(i) rowptr[i]\n#define EDGE_HI(i) rowptr[(i) + 1]\n";
   if (backward) {
     o << "__constant__ int kPh[" << S * K.nw << "] = {";
     for (int s = 0; s < S; ++s)
@@ -237,9 +243,9 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
        "  int q = 0, k = 0;\n"
        "  bool dead = false;\n"
        "  for (int slice = 0; slice < NSLICE && !dead; ++slice) {\n"
-       "  for (int i = blockIdx.x; i < n_recv && !dead; i += gridDim.x) {\n"
-       "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n";
-  if (backward) o << "    if (e1 == e0) continue;\n";
+       "  for (int i = RECV_FIRST; i < RECV_END && !dead; i += RECV_STEP) {\n"
+       "    const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n";
+  if (backward) o << "    if (e1 <= e0) continue;\n";
   o << "    switch (slice) {\n";
   for (int s = 0; s < S; ++s) {
     const SliceLayout& sl = SL[s];
@@ -363,8 +369,8 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
       << "    const int4 r = k < nk ? __ldg(srec + lane + 32 * k) : make_int4(0, 0, 0, 0);\n"
       << "    rd[k] = r.x;\n    rc0[k] = __int_as_float(r.y);\n    rc1[k] = __int_as_float(r.z);\n  }\n";
   o <<
-       "  for (int i = blockIdx.x; i < n_recv && !dead; i += gridDim.x) {\n"
-       "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
+       "  for (int i = RECV_FIRST; i < RECV_END && !dead; i += RECV_STEP) {\n"
+       "    const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
        "      const int s = q % NSTAGE;\n"
        "      const int nb = min(NB, e1 - eb);\n"

@@ -70,8 +70,8 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
          "  bool ok[" << R << "];\n"
          "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) ok[r] = u0 + r * 32 + lane < " << MUL << ";\n"
          "  int q = *qp;\n"
-         "#pragma unroll 1\n  for (int i = blockIdx.x; i < n_recv; i += gridDim.x) {\n"
-         "  const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
+         "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
+         "  const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
          "  float acc[" << nacc << "];\n"
          "#pragma unroll\n  for (int k = 0; k < " << nacc << "; ++k) acc[k] = 0.f;\n"
          "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
@@ -120,8 +120,8 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
        "  const int lane = threadIdx.x & 31;\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  int q = *qp;\n"
-       "#pragma unroll 1\n  for (int i = blockIdx.x; i < n_recv; i += gridDim.x) {\n"
-       "    const int e0 = rowptr[i], e1 = rowptr[i + 1];\n"
+       "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
+       "    const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
        "      const int s = q % NSTAGE;\n"
        "      if (!mbar_wait(full0 + 8 * s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"

@@ -156,9 +156,10 @@ void jit_unload(JitKernel& k);
 
 // generic CUDA kernels (kernels.cu)
 cudaError_t launch_sph_harm(int L, int64_t E, const float* r, float* Y, cudaStream_t s);
-cudaError_t launch_segment_rows(int64_t n_send, int64_t width, const int32_t* rowptr_T,
-                                const int32_t* perm_T, const float* m, float* dx,
-                                cudaStream_t s);
-cudaError_t launch_sum_slices(int S, int64_t n, const float* parts, float* dst, cudaStream_t s);
+// dx row sums over the transpose edge list and the dY slice sums, one launch;
+// either part is skipped when its output is null (or S == 1 for dY).
+cudaError_t launch_bwd_reduce(int64_t n_send, int64_t width, const int32_t* rowptr_T, const int32_t* perm_T,
+                              const float* m, float* dx, int S, int64_t ny, const float* parts, float* dy,
+                              cudaStream_t s);
 
 }  // namespace cgtp

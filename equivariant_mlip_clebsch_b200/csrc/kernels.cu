@@ -1,8 +1,9 @@
 // kernels.cu -- the kernels that do not depend on the path structure:
-// real spherical harmonics of the edge vectors, and the two deterministic
-// reductions of the backward (sender-major row sums, slice sums).
+// real spherical harmonics of the edge vectors, and the deterministic closing
+// reductions of the backward (sender-major row sums, slice sums) in one launch.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 
@@ -84,58 +85,78 @@ __global__ void __launch_bounds__(128) sph_harm_kernel(int64_t E, const float* _
   for (int t = threadIdx.x; t < n; t += 128) dst[t] = tile[t];
 }
 
-// dx[j][c] = sum over the sender's edges t (ascending) of m[perm_T[t]][c];
-// the sum runs in edge order (bitwise reproducible), four rows in flight.
-__global__ void __launch_bounds__(128) segment_rows_kernel(int64_t width,
-                                                           const int32_t* __restrict__ rowptr_T,
-                                                           const int32_t* __restrict__ perm_T,
-                                                           const float* __restrict__ m,
-                                                           float* __restrict__ dx) {
-  const int64_t j = blockIdx.x;
-  const int t0 = rowptr_T[j], t1 = rowptr_T[j + 1];
-  if ((width & 3) == 0) {
-    const int64_t w4 = width >> 2;
-    for (int64_t c = threadIdx.x + (int64_t)blockIdx.y * 128; c < w4; c += 128 * (int64_t)gridDim.y) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      int t = t0;
-      for (; t + 4 <= t1; t += 4) {
-        float4 v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          v[k] = __ldcs(reinterpret_cast<const float4*>(m + (int64_t)__ldg(perm_T + t + k) * width) + c);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          acc.x += v[k].x;
-          acc.y += v[k].y;
-          acc.z += v[k].z;
-          acc.w += v[k].w;
-        }
-      }
-      for (; t < t1; ++t) {
-        const float4 v = __ldcs(reinterpret_cast<const float4*>(m + (int64_t)__ldg(perm_T + t) * width) + c);
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
-      }
-      reinterpret_cast<float4*>(dx + j * width)[c] = acc;
-    }
-  } else {
-    for (int64_t c = threadIdx.x + (int64_t)blockIdx.y * 128; c < width; c += 128 * (int64_t)gridDim.y) {
-      float acc = 0.f;
-      for (int t = t0; t < t1; ++t) acc += __ldcs(m + (int64_t)perm_T[t] * width + c);
-      dx[j * width + c] = acc;
-    }
-  }
+// The backward's closing reductions in one launch.
+//  blocks [0, n_send): dx[j][c] = sum over sender j's edges of m[perm_T[t]][c].
+//    Two groups of 128 threads take the even and the odd positions t0 + 2k of
+//    the sender's list, eight rows in flight each; the two partial sums are
+//    added in a fixed order, so the result is bitwise reproducible.
+//  blocks [n_send, n_send + dy_blocks): dY = sum over the S slice partials.
+constexpr int kEpiThreads = 256;
+
+__device__ __forceinline__ void add4(float4& a, const float4 v) {
+  a.x += v.x;
+  a.y += v.y;
+  a.z += v.z;
+  a.w += v.w;
 }
 
-__global__ void sum_slices_kernel(int S, int64_t n, const float* __restrict__ parts,
-                                  float* __restrict__ dst) {
-  for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < n;
-       k += (int64_t)gridDim.x * blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < S; ++s) acc += parts[(int64_t)s * n + k];
-    dst[k] = acc;
+__global__ void __launch_bounds__(kEpiThreads) bwd_reduce_kernel(
+    int64_t n_send, int64_t width, const int32_t* __restrict__ rowptr_T, const int32_t* __restrict__ perm_T,
+    const float* __restrict__ m, float* __restrict__ dx, int S, int64_t ny, const float* __restrict__ parts,
+    float* __restrict__ dy) {
+  __shared__ float4 part[128];
+  const int64_t blk = blockIdx.x;
+  if (blk >= n_send || dx == nullptr) {
+    const int64_t b0 = dx ? blk - n_send : blk;
+    const int64_t nblk = (int64_t)gridDim.x - (dx ? n_send : 0);
+    for (int64_t k = b0 * kEpiThreads + threadIdx.x; k < ny; k += nblk * kEpiThreads) {
+      float acc = 0.f;
+      for (int q = 0; q < S; ++q) acc += parts[(int64_t)q * ny + k];
+      dy[k] = acc;
+    }
+    return;
+  }
+  const int64_t j = blk;
+  const int t0 = rowptr_T[j], t1 = rowptr_T[j + 1];
+  const int g = threadIdx.x >> 7, c0 = threadIdx.x & 127;
+  if ((width & 3) == 0) {
+    const int64_t w4 = width >> 2;
+    for (int64_t cb = 0; cb < w4; cb += 128) {
+      const int64_t c = cb + c0;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c < w4) {
+        int t = t0 + g;
+        for (; t + 14 < t1; t += 16) {
+          float4 v[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            v[k] = __ldcs(reinterpret_cast<const float4*>(m + (int64_t)__ldg(perm_T + t + 2 * k) * width) + c);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) add4(acc, v[k]);
+        }
+        for (; t < t1; t += 2) add4(acc, __ldcs(reinterpret_cast<const float4*>(m + (int64_t)__ldg(perm_T + t) * width) + c));
+      }
+      if (g == 1) part[c0] = acc;
+      __syncthreads();
+      if (g == 0 && c < w4) {
+        const float4 o = part[c0];
+        add4(acc, o);
+        reinterpret_cast<float4*>(dx + j * width)[c] = acc;
+      }
+      __syncthreads();
+    }
+  } else {
+    float* pf = reinterpret_cast<float*>(part);
+    for (int64_t cb = 0; cb < width; cb += 128) {
+      const int64_t c = cb + c0;
+      float acc = 0.f;
+      if (c < width)
+        for (int t = t0 + g; t < t1; t += 2) acc += __ldcs(m + (int64_t)perm_T[t] * width + c);
+      if (g == 1) pf[c0] = acc;
+      __syncthreads();
+      if (g == 0 && c < width) dx[j * width + c] = acc + pf[c0];
+      __syncthreads();
+    }
   }
 }
 
@@ -176,19 +197,14 @@ cudaError_t launch_sph_harm(int L, int64_t E, const float* r, float* Y, cudaStre
   return cudaGetLastError();
 }
 
-cudaError_t launch_segment_rows(int64_t n_send, int64_t width, const int32_t* rowptr_T,
-                                const int32_t* perm_T, const float* m, float* dx, cudaStream_t s) {
-  if (n_send == 0 || width == 0) return cudaSuccess;
-  const int64_t cols = (width & 3) == 0 ? width / 4 : width;
-  const unsigned gy = (unsigned)((cols + 127) / 128);
-  segment_rows_kernel<<<dim3((unsigned)n_send, gy), 128, 0, s>>>(width, rowptr_T, perm_T, m, dx);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_sum_slices(int S, int64_t n, const float* parts, float* dst, cudaStream_t s) {
-  if (n == 0) return cudaSuccess;
-  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 16);
-  sum_slices_kernel<<<(unsigned)blocks, 256, 0, s>>>(S, n, parts, dst);
+cudaError_t launch_bwd_reduce(int64_t n_send, int64_t width, const int32_t* rowptr_T, const int32_t* perm_T,
+                              const float* m, float* dx, int S, int64_t ny, const float* parts, float* dy,
+                              cudaStream_t s) {
+  const int64_t nx = (dx && width > 0) ? n_send : 0;
+  const int64_t ndy = (dy && S > 1 && ny > 0) ? std::min<int64_t>((ny + kEpiThreads - 1) / kEpiThreads, 148 * 4) : 0;
+  if (nx + ndy == 0) return cudaSuccess;
+  bwd_reduce_kernel<<<(unsigned)(nx + ndy), kEpiThreads, 0, s>>>(nx, width, rowptr_T, perm_T, m, nx ? dx : nullptr,
+                                                                S, ndy ? ny : 0, parts, dy);
   return cudaGetLastError();
 }
 

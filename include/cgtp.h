@@ -148,7 +148,7 @@ cgtp_status cgtp_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t
  * sum for grad_x goes through the transpose edge list (rowptr_T, perm_T,
  * needed only when grad_x != NULL) and the workspace; no atomics, bitwise
  * reproducible.  workspace must hold cgtp_backward_workspace_size bytes and be
- * 256-byte aligned. */
+ * 256-byte aligned (NULL is accepted when grad_W is the only output wanted). */
 cgtp_status cgtp_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
                           const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
                           const int32_t* perm_T, const float* x, const float* Y,
