@@ -37,6 +37,7 @@ void destroy_plan_device(Plan& P) {
   P.tpool.clear();
   jit_unload(P.fwd);
   jit_unload(P.bwd);
+  jit_unload(P.bwd_er);
   for (void** p : {&P.d_fwd_ent, &P.d_fwd_term, &P.d_bwd_ent, &P.d_bwd_term}) {
     if (*p) cudaFree(*p);
     *p = nullptr;
@@ -338,10 +339,14 @@ cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
   }
   if (n_recv > 0) {
     int nr = (int)n_recv;
-    const unsigned G = persistent_grid(P->bwd.blocks_per_sm, P->num_sms, n_recv);
+    // few receivers per CTA: equal edge ranges keep the CTAs' work even
+    unsigned G = persistent_grid(P->bwd.blocks_per_sm, P->num_sms, n_recv);
+    const bool er = P->bwd_er.function && n_recv <= 8 * (int64_t)G;
+    JitKernel& JK = er ? P->bwd_er : P->bwd;
+    if (er) G = persistent_grid(P->bwd_er.blocks_per_sm, P->num_sms, n_recv);
     void* args[] = {&rowptr, &col, &x, &Y, &W, &grad_out, &grad_W, &dyp, &m, &P->d_bwd_ent, &nr, &P->d_err};
     TimedScope ts(*P, 2, s, allow_timing);
-    st = jit_launch(P->bwd, dim3(G), args, s);
+    st = jit_launch(JK, dim3(G), args, s);
     if (st != CGTP_OK) return st;
   }
   if (grad_x || (grad_Y && P->bcfg.S > 1)) {
@@ -396,6 +401,12 @@ cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* need
     t += "  brole " + std::to_string(r) + ": irrep " + std::to_string(q.irrep) + " u0=" +
          std::to_string(q.u0) + " R=" + std::to_string(q.R) + " ph=" + std::to_string(q.ph) + "/" +
          std::to_string(q.nph) + " cost=" + std::to_string((int)q.cost) + "\n";
+  }
+  {  // the edge-range variant of the backward (same roles and layout)
+    char hx[40];
+    std::snprintf(hx, sizeof hx, " hash=%016llx\n", P->bwd_er.hash);
+    t += "backward (edge ranges, for at most 8 receivers per CTA):" + std::string(hx) + P->bwd_er.log;
+    if (!P->bwd_er.log.empty() && P->bwd_er.log.back() != '\n') t += "\n";
   }
   if (needed) *needed = t.size() + 1;
   if (buf && n > 0) {

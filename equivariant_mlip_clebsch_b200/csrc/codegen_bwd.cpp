@@ -275,6 +275,16 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
        "    for (int b = 0; b < 2; ++b) { mbar_init(gfull0 + 8 * b, 32); mbar_init(gempty0 + 8 * b, NW); }\n"
        "    fence_mbar_init();\n"
        "  }\n"
+       << (K.edge_ranges
+           ? "  if (warp == 0) {  // this CTA's share of the edges and the receivers it touches\n"
+             "    const int E = __ldg(rowptr + n_recv);\n"
+             "    const int lo = (int)((long long)E * blockIdx.x / gridDim.x);\n"
+             "    const int hi = (int)((long long)E * (blockIdx.x + 1) / gridDim.x);\n"
+             "    const int i0 = warp_last_le(rowptr, 0, n_recv - 1, lo, lane);\n"
+             "    const int i1 = hi > lo ? warp_last_le(rowptr, 0, n_recv - 1, hi - 1, lane) + 1 : i0;\n"
+             "    if (lane == 0) *reinterpret_cast<int4*>(smem + OFF_RANGE) = make_int4(i0, i1, lo, hi);\n"
+             "  }\n"
+           : "") <<
        "  __syncthreads();\n"
        "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, g, err, smem, lane); return; }\n"
        "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, ent, kEntBegin, dyp, err, smem, lane); return; }\n"
@@ -595,7 +605,6 @@ cgtp_status build_backward(Plan& P) {
   if (st != CGTP_OK) return st;
   for (size_t k = 0; k + 1 < P.bwd_ent_begin.size(); ++k)
     K.rec_max = std::max(K.rec_max, P.bwd_ent_begin[k + 1] - P.bwd_ent_begin[k]);
-  const std::string name = "cgtp_bwd";
   // register cap from the resident CTAs shared memory allows; one CTA fewer
   // (but not below two) when the compiler reports sizeable spills
   if (K.smem > 227 * 1024) return fail(CGTP_ERR_SIZE, "backward kernel needs too much shared memory");
@@ -603,23 +612,32 @@ cgtp_status build_backward(Plan& P) {
   int mb0 = initial_min_blocks(K.smem, &fixed);
   if (!fixed) mb0 = std::min(mb0, best.ctas);  // the planner's register share
   const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
-  std::string src;
-  for (int mb = mb0; mb >= mb_floor; --mb) {
-    src = gen_bwd_source(P, SL, K, name, mb);
-    P.bwd.threads = (F.nw + 2) * 32;
-    P.bwd.smem = K.smem;
-    cgtp_status cst = jit_compile(src, name, P.bwd);
-    if (cst != CGTP_OK) return cst;
-    if (mb == mb_floor || max_spill_bytes(P.bwd.log) <= 160) break;
-    jit_unload(P.bwd);
-  }
-  P.bwd.threads = (F.nw + 2) * 32;
-  P.bwd.smem = K.smem;
-  if (const char* d = std::getenv("CGTP_DUMP_SOURCE")) {
-    FILE* f = std::fopen((std::string(d) + "/bwd.cu").c_str(), "w");
-    if (f) {
-      std::fputs(src.c_str(), f);
-      std::fclose(f);
+  // Two variants of the same kernel: CTAs over whole receivers, and CTAs
+  // over equal edge ranges.  The second balances graphs with few receivers
+  // per CTA; measured on B200, the range code in the first variant (even
+  // when not taken) slowed the large cases, hence two kernels.
+  for (int er = 0; er < 2; ++er) {
+    K.edge_ranges = er == 1;
+    const std::string name = er ? "cgtp_bwd_er" : "cgtp_bwd";
+    JitKernel& JK = er ? P.bwd_er : P.bwd;
+    std::string src;
+    for (int mb = mb0; mb >= mb_floor; --mb) {
+      src = gen_bwd_source(P, SL, K, name, mb);
+      JK.threads = (F.nw + 2) * 32;
+      JK.smem = K.smem;
+      cgtp_status cst = jit_compile(src, name, JK);
+      if (cst != CGTP_OK) return cst;
+      if (mb == mb_floor || max_spill_bytes(JK.log) <= 160) break;
+      jit_unload(JK);
+    }
+    JK.threads = (F.nw + 2) * 32;
+    JK.smem = K.smem;
+    if (const char* d = std::getenv("CGTP_DUMP_SOURCE")) {
+      FILE* f = std::fopen((std::string(d) + (er ? "/bwd_er.cu" : "/bwd.cu")).c_str(), "w");
+      if (f) {
+        std::fputs(src.c_str(), f);
+        std::fclose(f);
+      }
     }
   }
   return CGTP_OK;

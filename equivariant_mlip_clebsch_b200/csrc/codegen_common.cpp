@@ -202,12 +202,17 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
   // shared-memory header: full[NSTAGE], empty[NSTAGE], gfull[2], gempty[2]
   // mbarriers, then the helper's per-stage chunk descriptors
   o << "#define OFF_GFULL (2 * NSTAGE * 8)\n#define OFF_GEMPTY (OFF_GFULL + 16)\n#define OFF_DESC (OFF_GEMPTY + 16)\n";
-  // the receivers a CTA walks: blockIdx.x, + gridDim.x, ...  (Edge-balanced
-  // ranges for the backward were measured on B200: faster on small graphs,
-  // but the range search, in the kernel or as a launch of its own, cost more
-  // than it saved on the larger cases.)
-  o << "#define RECV_FIRST ((int)blockIdx.x)\n#define RECV_END n_recv\n#define RECV_STEP ((int)gridDim.x)\n"
-       "#define EDGE_LO(i) rowptr[i]\n#define EDGE_HI(i) rowptr[(i) + 1]\n";
+  // the receivers a CTA walks: whole receivers blockIdx.x, + gridDim.x, ...,
+  // or (backward, edge_ranges) an equal share of the edges, receivers clipped
+  // to it (the range sits in the header at OFF_RANGE)
+  if (backward && K.edge_ranges)
+    o << "#define OFF_RANGE 240\n"
+         "#define RANGE_AT(k) (reinterpret_cast<const int*>(smem + OFF_RANGE)[k])\n"
+         "#define RECV_FIRST RANGE_AT(0)\n#define RECV_END RANGE_AT(1)\n#define RECV_STEP 1\n"
+         "#define EDGE_LO(i) max(rowptr[i], RANGE_AT(2))\n#define EDGE_HI(i) min(rowptr[(i) + 1], RANGE_AT(3))\n";
+  else
+    o << "#define RECV_FIRST ((int)blockIdx.x)\n#define RECV_END n_recv\n#define RECV_STEP ((int)gridDim.x)\n"
+         "#define EDGE_LO(i) rowptr[i]\n#define EDGE_HI(i) rowptr[(i) + 1]\n";
   if (backward) {
     o << "__constant__ int kPh[" << S * K.nw << "] = {";
     for (int s = 0; s < S; ++s)

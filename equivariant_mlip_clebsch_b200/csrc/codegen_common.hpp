@@ -68,6 +68,7 @@ struct KernelShape {
   int gbufs = 2;    // grad_out row buffers (backward)
   int force_B = 0;  // edges per chunk fixed by the caller (0: chosen from the budget)
   int rec_max = 0;  // most Chat records of a slice
+  bool edge_ranges = false;  // backward CTAs take equal edge ranges
   int off_wb = 0;
 };
 

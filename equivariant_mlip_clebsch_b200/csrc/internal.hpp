@@ -115,7 +115,8 @@ struct Plan {
   // backward
   std::vector<BwdRole> bwd_roles;
   FwdConfig bcfg;
-  JitKernel bwd;
+  JitKernel bwd;     // CTAs walk receivers blockIdx.x, + gridDim.x, ...
+  JitKernel bwd_er;  // CTAs take equal edge ranges (for few receivers per CTA)
   void* d_bwd_ent = nullptr;
   void* d_bwd_term = nullptr;
   std::vector<int> bwd_ent_begin;
