@@ -346,8 +346,8 @@ def ncu_traffic(name, kernel, plan):
         return None
     desc = plan.describe()
     tag = "forward" if kernel == "cgtp_fwd" else "backward"
-    for line in desc.splitlines():
-        if line.startswith(tag + ":") and f"hash={d.get('kernel_hash')}" in line:
+    for line in desc.splitlines():  # either backward variant
+        if line.startswith(tag) and f"hash={d.get('kernel_hash')}" in line:
             return d.get("bytes_per_launch")
     return None
 
