@@ -139,7 +139,7 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       std::abort();
     }
     const int RU = bwd_unroll(N1, R);
-    const int VZ = pow2((int)P.D_e);
+    const int VZ = (int)P.D_e;  // reduced in power-of-two parts (9 = 8 + 1, 25 = 16 + 8 + 1)
     if (combined)
       o << "      float z[" << VZ << "];\n#pragma unroll\n      for (int t = 0; t < " << VZ << "; ++t) z[t] = 0.f;\n";
     o << "#pragma unroll 1\n      for (int r = 0; r < " << R << "; r += " << RU << ") {\n"
@@ -147,7 +147,8 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       << "      float xv[" << RU << "][" << N1 << "], mx[" << RU << "][" << N1 << "];\n"
       << "#pragma unroll\n      for (int v = 0; v < " << RU << "; ++v) {\n"
       << "        const int u = u0 + (r + v) * 32 + lane;\n"
-      << "        ok[v] = u < " << MUL << ";\n"
+      << "        ok[v] = " << (MUL % (32 * R) == 0 ? std::string("true") : "u < " + std::to_string(MUL))
+      << ";  // every lane holds a channel when the blocks are full\n"
       << "#pragma unroll\n        for (int m1 = 0; m1 < " << N1
       << "; ++m1) { mx[v][m1] = 0.f; xv[v][m1] = ok[v] ? xr[u * " << N1 << " + m1] : 0.f; }\n"
       << "      }\n";
@@ -217,10 +218,20 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       << "        __syncwarp();\n      }\n"
       << "      }\n";  // r
     if (combined) {
-      const int LV = __builtin_ctz(VZ), sh = 5 - LV;
-      o << "      if (sdy) {\n        const float v = warp_sum_many<" << VZ << ">(z, lane);\n"
-        << "        const int k = lane >> " << sh << ";\n"
-        << "        if ((lane & " << ((1 << sh) - 1) << ") == 0 && k < DE) sdy[k] = v;\n      }\n";
+      o << "      if (sdy) {\n";
+      for (int off = 0, rest = VZ; rest > 0;) {
+        int V = 1;
+        while (V * 2 <= rest && V * 2 <= 32) V *= 2;
+        const int LV = __builtin_ctz(V), sh = 5 - LV;
+        o << "        {\n          float zp[" << V << "];\n#pragma unroll\n          for (int t = 0; t < " << V
+          << "; ++t) zp[t] = z[" << off << " + t];\n"
+          << "          const float v = warp_sum_many<" << V << ">(zp, lane);\n"
+          << "          if ((lane & " << ((1 << sh) - 1) << ") == 0) sdy[" << off << " + (lane >> " << sh
+          << ")] = v;\n        }\n";
+        off += V;
+        rest -= V;
+      }
+      o << "      }\n";
     } else {
       for (int l2 = 0; l2 <= P.L; ++l2)
         if (!l2seen[l2])

@@ -68,7 +68,9 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
          "  const int lane = threadIdx.x & 31;\n"
          "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
          "  bool ok[" << R << "];\n"
-         "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) ok[r] = u0 + r * 32 + lane < " << MUL << ";\n"
+         "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) ok[r] = "
+      << (MUL % (32 * R) == 0 ? std::string("true") : "u0 + r * 32 + lane < " + std::to_string(MUL))
+      << ";  // every lane holds a channel when the blocks are full\n"
          "  int q = *qp;\n"
          "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
          "  const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
