@@ -59,6 +59,22 @@ CONFIGS = {
         cells=(4, 4, 6), sigma=0.05, rc=5.0,
         irreps_in=_L6_IN, irreps_edge=_L6_EDGE,
         irreps_out="448x0e+768x1o+1024x2e+1152x3o+1216x4e+1152x5o+1024x6e"),
+    # Table 1 Cases 4-6 (atom counts not given there: the 768-atom cell above)
+    "case4": dict(
+        desc="768 Si atoms, 4x4x6 cells, rc 5.0, Lmax 3, 256 channels per degree (Table 1 Case 4)",
+        cells=(4, 4, 6), sigma=0.05, rc=5.0,
+        irreps_in="256x0e+256x1o+256x2e+256x3o", irreps_edge="1x0e+1x1o+1x2e+1x3o",
+        irreps_out="1024x0e+1536x1o+1792x2e+1536x3o"),
+    "case5": dict(
+        desc="768 Si atoms, 4x4x6 cells, rc 5.0, Lmax 4 (Table 1 Case 5)",
+        cells=(4, 4, 6), sigma=0.05, rc=5.0,
+        irreps_in="320x0e+96x1o+64x2e+32x3o+32x4e", irreps_edge="1x0e+1x1o+1x2e+1x3o+1x4e",
+        irreps_out="544x0e+736x1o+832x2e+800x3o+704x4e"),
+    "case6": dict(
+        desc="768 Si atoms, 4x4x6 cells, rc 5.0, Lmax 4, 128 channels per degree (Table 1 Case 6)",
+        cells=(4, 4, 6), sigma=0.05, rc=5.0,
+        irreps_in="128x0e+128x1o+128x2e+128x3o+128x4e", irreps_edge="1x0e+1x1o+1x2e+1x3o+1x4e",
+        irreps_out="640x0e+1024x1o+1280x2e+1280x3o+1152x4e"),
 }
 
 

@@ -3,8 +3,9 @@
 Bar (from the acceptance criteria of the build): rel-L2 <= 1e-5 and
 max |err| <= 1e-4 * max |ref| for Y, out, dx, dW and dY; CSR and edge vectors
 bit-exact; GPU results bitwise repeatable run to run.  Every workload runs at
-its full size; the 6144-atom Lmax=3 case is compared on sampled receivers and
-senders (the oracle computes those rows exactly from a sub-list of edges).
+its full size (Table 1 Cases 4-6 on the 768-atom cell); the 6144-atom Lmax=3
+case is compared on sampled receivers and senders (the oracle computes those
+rows exactly from a sub-list of edges).
 """
 import numpy as np
 import pytest
@@ -16,7 +17,7 @@ from tests._cases import Workload, assert_close
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
-ALL = ["tiny", "lmax2", "lmax2_wide", "lmax3", "lmax6"]
+ALL = ["tiny", "lmax2", "lmax2_wide", "lmax3", "lmax6", "case4", "case5", "case6"]
 _plans, _cases = {}, {}
 
 

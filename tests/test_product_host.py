@@ -92,7 +92,7 @@ def compile_only(monkeypatch):
     monkeypatch.setenv("CGTP_JIT_COMPILE_ONLY", "1")
 
 
-@pytest.mark.parametrize("name", ["tiny", "lmax2", "lmax2_wide", "lmax3", "lmax6"])
+@pytest.mark.parametrize("name", ["tiny", "lmax2", "lmax2_wide", "lmax3", "lmax6", "case4", "case5", "case6"])
 def test_plan_builds_and_compiles(name, compile_only):
     c = WL.CONFIGS[name]
     plan = C.Plan(c["irreps_in"], c["irreps_edge"], c["irreps_out"], 6)
