@@ -15,7 +15,10 @@
  *     (theta, phi), component normalisation, m = -l..l, no Condon-Shortley
  *     phase,
  *   - a brute-force periodic neighbour search over all atom pairs and images,
- *   - the forward and backward CGTP convolution as nested sums.
+ *   - the forward and backward CGTP convolution as nested sums,
+ *   - the gradient of the harmonics with respect to the edge vector (forward-
+ *     mode differentiation of the harmonics above) and the force assembly
+ *     from it (the step after the backward: forces = -dE/dpos).
  *
  * Source of the operation: LunaTP (arXiv 2610.18393), Abstract (the CGTP
  * convolution), Table 1 (irreps configurations and hence the path set) and
@@ -214,6 +217,135 @@ void orc_sph_harm(int L, int64_t E, const double* r, double* Y) {
       }
     }
   }
+}
+
+/* ------------------------------------------------------------------ */
+/* gradient of the real spherical harmonics with respect to r           */
+/* ------------------------------------------------------------------ */
+/* Forward-mode differentiation of orc_sph_harm above: every quantity of that
+ * computation carries its value and its derivatives with respect to
+ * (x, y, z), propagated through each elementary operation by the chain rule
+ * (exact up to rounding).  J is [E][(L+1)^2][3], J[e][t][k] = dY_t/dr_k.
+ * r = 0 gives J = 0.  Undefined exactly on the z axis (x = y = 0, r != 0),
+ * where phi = atan2(y, x) has no derivative; returns -1 if such an edge
+ * occurs, else 0.  This is the step from dL/dY to dL/dr on the way to the
+ * forces (forces = minus the position gradient of the energy, the BranchIP
+ * page's force definition). */
+typedef struct {
+  double v, d[3];
+} dual3;
+
+static dual3 dconst(double v) {
+  dual3 a = {v, {0.0, 0.0, 0.0}};
+  return a;
+}
+static dual3 dadd(dual3 a, dual3 b) {
+  dual3 c = {a.v + b.v, {a.d[0] + b.d[0], a.d[1] + b.d[1], a.d[2] + b.d[2]}};
+  return c;
+}
+static dual3 dsub(dual3 a, dual3 b) {
+  dual3 c = {a.v - b.v, {a.d[0] - b.d[0], a.d[1] - b.d[1], a.d[2] - b.d[2]}};
+  return c;
+}
+static dual3 dmul(dual3 a, dual3 b) {
+  dual3 c;
+  c.v = a.v * b.v;
+  for (int k = 0; k < 3; ++k) c.d[k] = a.d[k] * b.v + a.v * b.d[k];
+  return c;
+}
+static dual3 dscale(double s, dual3 a) {
+  dual3 c = {s * a.v, {s * a.d[0], s * a.d[1], s * a.d[2]}};
+  return c;
+}
+static dual3 ddiv(dual3 a, dual3 b) {
+  dual3 c;
+  c.v = a.v / b.v;
+  for (int k = 0; k < 3; ++k) c.d[k] = (a.d[k] * b.v - a.v * b.d[k]) / (b.v * b.v);
+  return c;
+}
+/* f(a) with f' given: value f(a.v), derivative f'(a.v) * a.d */
+static dual3 dapply(dual3 a, double f, double fprime) {
+  dual3 c = {f, {fprime * a.d[0], fprime * a.d[1], fprime * a.d[2]}};
+  return c;
+}
+static dual3 dsqrt(dual3 a) { return dapply(a, sqrt(a.v), 0.5 / sqrt(a.v)); }
+static dual3 dacos(dual3 a) { return dapply(a, acos(a.v), -1.0 / sqrt(1.0 - a.v * a.v)); }
+static dual3 dsin(dual3 a) { return dapply(a, sin(a.v), cos(a.v)); }
+static dual3 dcos(dual3 a) { return dapply(a, cos(a.v), -sin(a.v)); }
+static dual3 datan2(dual3 y, dual3 x) {
+  /* d atan2(y, x) = (x dy - y dx) / (x^2 + y^2) */
+  dual3 c;
+  double q = x.v * x.v + y.v * y.v;
+  c.v = atan2(y.v, x.v);
+  for (int k = 0; k < 3; ++k) c.d[k] = (x.v * y.d[k] - y.v * x.d[k]) / q;
+  if (g_fault == 3) /* mutation: the phi dependence of the gradient dropped */
+    for (int k = 0; k < 3; ++k) c.d[k] = 0.0;
+  return c;
+}
+
+int orc_sph_harm_grad(int L, int64_t E, const double* r, double* J) {
+  int D = (L + 1) * (L + 1), bad = 0;
+  for (int64_t e = 0; e < E; ++e) {
+    double* out = J + e * D * 3;
+    for (int t = 0; t < 3 * D; ++t) out[t] = 0.0;
+    dual3 x = {r[3 * e], {1.0, 0.0, 0.0}};
+    dual3 y = {r[3 * e + 1], {0.0, 1.0, 0.0}};
+    dual3 z = {r[3 * e + 2], {0.0, 0.0, 1.0}};
+    dual3 rr = dsqrt(dadd(dadd(dmul(x, x), dmul(y, y)), dmul(z, z)));
+    if (rr.v == 0.0) continue;
+    if (x.v == 0.0 && y.v == 0.0) {
+      bad = 1;
+      continue;
+    }
+    dual3 ct = ddiv(z, rr);
+    dual3 th = dacos(ct);
+    dual3 ph = datan2(y, x);
+    dual3 st = dsin(th);
+    dual3 P[13][13];
+    for (int a = 0; a < 13; ++a)
+      for (int b = 0; b < 13; ++b) P[a][b] = dconst(0.0);
+    /* the same recurrences as orc_sph_harm, on dual numbers */
+    for (int m = 0; m <= L; ++m) {
+      dual3 pmm = dconst(1.0);
+      for (int k = 1; k <= m; ++k) pmm = dmul(pmm, dscale(2.0 * k - 1.0, st));
+      P[m][m] = pmm;
+      if (m + 1 <= L) P[m + 1][m] = dscale(2.0 * m + 1.0, dmul(ct, pmm));
+      for (int l = m + 2; l <= L; ++l)
+        P[l][m] = dscale(1.0 / (l - m), dsub(dscale(2.0 * l - 1.0, dmul(ct, P[l - 1][m])),
+                                             dscale(l + m - 1.0, P[l - 2][m])));
+    }
+    for (int l = 0; l <= L; ++l) {
+      double nl = sqrt(2.0 * l + 1.0);
+      dual3 y0 = dscale(nl, P[l][0]);
+      for (int k = 0; k < 3; ++k) out[(l * l + l) * 3 + k] = y0.d[k];
+      for (int m = 1; m <= l; ++m) {
+        double nm = nl * sqrt(2.0 * fact(l - m) / fact(l + m));
+        dual3 mph = dscale((double)m, ph);
+        dual3 yc = dscale(nm, dmul(P[l][m], dcos(mph)));
+        dual3 ys = dscale(nm, dmul(P[l][m], dsin(mph)));
+        for (int k = 0; k < 3; ++k) {
+          out[(l * l + l + m) * 3 + k] = yc.d[k];
+          out[(l * l + l - m) * 3 + k] = ys.d[k];
+        }
+      }
+    }
+  }
+  return bad ? -1 : 0;
+}
+
+/* Forces from the edge-vector gradient G = dL/dr [E][3], with
+ * r_e = pos[col[e]] - pos[i] (+ image shift) for the edges e of receiver i:
+ *   F[a] = -dL/dpos[a] = sum_{e of receiver a} G[e] - sum_{e with col[e] = a} G[e].
+ * Plain loops over the edges. */
+void orc_edge_forces(int64_t n_atoms, const int64_t* rowptr, const int32_t* col, const double* G,
+                     double* F) {
+  for (int64_t a = 0; a < 3 * n_atoms; ++a) F[a] = 0.0;
+  for (int64_t i = 0; i < n_atoms; ++i)
+    for (int64_t e = rowptr[i]; e < rowptr[i + 1]; ++e)
+      for (int k = 0; k < 3; ++k) {
+        F[3 * i + k] += G[3 * e + k];
+        F[3 * (int64_t)col[e] + k] -= (g_fault == 4 ? -1.0 : 1.0) * G[3 * e + k]; /* 4: sign mutation */
+      }
 }
 
 /* ------------------------------------------------------------------ */

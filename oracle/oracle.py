@@ -61,6 +61,10 @@ def lib():
         L.orc_real_cg.argtypes = [i, i, i, P]
         L.orc_sph_harm.restype = None
         L.orc_sph_harm.argtypes = [i, i64, P, P]
+        L.orc_sph_harm_grad.restype = i
+        L.orc_sph_harm_grad.argtypes = [i, i64, P, P]
+        L.orc_edge_forces.restype = None
+        L.orc_edge_forces.argtypes = [i64, P, P, P, P]
         L.orc_neighbor_list.restype = i64
         L.orc_neighbor_list.argtypes = [i64, P, P, d, P, P, P, P]
         L.orc_forward.restype = None
@@ -203,6 +207,33 @@ def sph_harm(L: int, r) -> np.ndarray:
     Y = np.zeros((r.shape[0], (L + 1) ** 2), dtype=np.float64)
     lib().orc_sph_harm(L, r.shape[0], _ptr(r), _ptr(Y))
     return Y
+
+
+def sph_harm_grad(L: int, r) -> np.ndarray:
+    """Jacobian dY/dr [E, (L+1)^2, 3] of sph_harm, by forward-mode
+    differentiation of the same (theta, phi) computation (exact up to
+    rounding).  Raises on an edge exactly on the z axis (no derivative of phi)."""
+    r = np.ascontiguousarray(np.asarray(r, dtype=np.float64).reshape(-1, 3))
+    J = np.zeros((r.shape[0], (L + 1) ** 2, 3), dtype=np.float64)
+    if lib().orc_sph_harm_grad(L, r.shape[0], _ptr(r), _ptr(J)) != 0:
+        raise ValueError("edge vector on the z axis: the (theta, phi) gradient is undefined there")
+    return J
+
+
+def sph_harm_backward(L: int, r, dY) -> np.ndarray:
+    """dL/dr [E, 3] = sum_m dL/dY[e, m] dY_m/dr (the SH step of the force chain)."""
+    J = sph_harm_grad(L, r)
+    return np.einsum("em,emk->ek", np.asarray(dY, dtype=np.float64), J)
+
+
+def edge_forces(n_atoms: int, rowptr, col, G) -> np.ndarray:
+    """F[a] = -dL/dpos[a] from G = dL/dr per edge (r = pos_sender - pos_receiver + shift)."""
+    rowptr = np.ascontiguousarray(rowptr, dtype=np.int64)
+    col = np.ascontiguousarray(col, dtype=np.int32)
+    G = np.ascontiguousarray(G, dtype=np.float64).reshape(-1, 3)
+    F = np.zeros((n_atoms, 3), dtype=np.float64)
+    lib().orc_edge_forces(int(n_atoms), _ptr(rowptr), _ptr(col), _ptr(G), _ptr(F))
+    return F
 
 
 # ---------------------------------------------------------------------------
