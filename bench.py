@@ -233,11 +233,26 @@ def run_cgtp(args, rank, world, local_rank):
         plan.sph_harm(T["r"], Y)
         plan.forward(T["rowptr"], T["col"], T["x"], Y, T["W"], out=out)
         b.record(stream)
+    # the force chain after the backward (dL/dY -> dL/dr -> forces), not in
+    # the step: reported beside it
+    from equivariant_mlip_clebsch_b200 import cgtp as C
+    gr = torch.empty((E, 3), device=dev)
+    Fo = torch.empty((N, 3), device=dev)
+    ev_c = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush.zero_()
+        a, b = ev_c[k]
+        a.record(stream)
+        plan.sph_harm_backward(T["r"], dY, grad_r=gr)
+        C.edge_forces(T["rowptr"], T["rpt"], T["perm"], gr, forces=Fo)
+        b.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
     plan.check_device_error()
     ms_steps = [a.elapsed_time(b) for a, b in ev]
     ms_fwd = [a.elapsed_time(b) for a, b in ev_f]
+    force_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_c]))
     ms_step = float(np.sum(ms_steps)) / args.steps
     if world > 1:
         t = torch.tensor([ms_step], device=dev)
@@ -296,6 +311,8 @@ def run_cgtp(args, rank, world, local_rank):
                        "parallelism": "replicas" if world > 1 else "single GPU"},
                atoms_per_s=world * N / (ms_step * 1e-3),
                fwd_edges_per_s=world * E / (fwd_ms * 1e-3), fwd_ms=fwd_ms,
+               force_chain={"ms": force_ms, "edges_per_s": world * E / (force_ms * 1e-3),
+                            "what": "sph_harm_backward + edge_forces after the step (not in it)"},
                roofline=roof, kernels=kernels, gpu_launches=int(gpu_launches), e2e=e2e, clocks=clocks)
     return res
 

@@ -37,6 +37,8 @@ _SIGS = {
     "cgtp_plan_describe": (_i, [_P, ctypes.c_char_p, _sz, ctypes.POINTER(_sz)]),
     "cgtp_real_cg": (_i, [_i, _i, _i, _P]),
     "cgtp_sph_harm": (_i, [_P, _i64, _P, _P, _P]),
+    "cgtp_sph_harm_backward": (_i, [_P, _i64, _P, _P, _P, _P]),
+    "cgtp_edge_forces": (_i, [_i64, _i64, _P, _P, _P, _P, _P, _P]),
     "cgtp_forward": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P, _P, _P]),
     "cgtp_backward_workspace_size": (_i, [_P, _i64, _i64, _i64, ctypes.POINTER(_sz)]),
     "cgtp_backward": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -110,6 +112,18 @@ def neighbor_list(pos, box, rc: float):
     _check(_lib.cgtp_neighbor_list(N, _np_ptr(pos), _np_ptr(box), float(rc), _np_ptr(rowptr),
                                    _np_ptr(col), _np_ptr(shift), _np_ptr(r), ctypes.byref(E)))
     return rowptr, col, shift, r
+
+
+def edge_forces(rowptr, rowptr_T, perm_T, grad_r, forces=None, stream=None):
+    """cgtp_edge_forces: forces [N,3] = -dL/dpos from grad_r [E,3] (device
+    tensors; r_e = pos_sender - pos_receiver + shift)."""
+    import torch
+    n_atoms, E = rowptr.shape[0] - 1, grad_r.shape[0]
+    if forces is None:
+        forces = torch.empty((n_atoms, 3), dtype=torch.float32, device=grad_r.device)
+    _check(_lib.cgtp_edge_forces(n_atoms, E, _tptr(rowptr), _tptr(rowptr_T), _tptr(perm_T), _tptr(grad_r),
+                                 _tptr(forces), _stream(stream)))
+    return forces
 
 
 def csr_transpose(rowptr, col, n_send: int):
@@ -209,6 +223,16 @@ class Plan:
             Y = torch.empty((E, self.d_edge), dtype=torch.float32, device=r.device)
         _check(_lib.cgtp_sph_harm(self._h, E, _tptr(r), _tptr(Y), _stream(stream)))
         return Y
+
+    def sph_harm_backward(self, r, grad_Y, grad_r=None, stream=None):
+        """cgtp_sph_harm_backward: grad_r [E,3] = sum_t grad_Y[:, t] dY_t/dr."""
+        import torch
+        E = r.shape[0]
+        if grad_r is None:
+            grad_r = torch.empty((E, 3), dtype=torch.float32, device=r.device)
+        _check(_lib.cgtp_sph_harm_backward(self._h, E, _tptr(r), _tptr(grad_Y), _tptr(grad_r),
+                                           _stream(stream)))
+        return grad_r
 
     def forward(self, rowptr, col, x, Y, W, out=None, stream=None):
         import torch

@@ -58,7 +58,7 @@ static cgtp_status check_device(const Plan& P) {
   return CGTP_OK;
 }
 
-static const char* kKindName[] = {"sph_harm", "cgtp_fwd", "cgtp_bwd", "bwd_reduce", "unused", "zero_fill"};
+static const char* kKindName[] = {"sph_harm", "cgtp_fwd", "cgtp_bwd", "bwd_reduce", "sph_harm_bwd", "zero_fill"};
 
 // Brackets one internal launch with events when timing is on.
 struct TimedScope {
@@ -238,6 +238,35 @@ cgtp_status cgtp_sph_harm(cgtp_plan plan, int64_t E, const float* r, float* Y, c
     TimedScope ts(*const_cast<Plan*>(P), 0, (cudaStream_t)stream);
     CGTP_CUDA_TRY(launch_sph_harm(P->L, E, r, Y, (cudaStream_t)stream));
   }
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_sph_harm_backward(cgtp_plan plan, int64_t E, const float* r, const float* grad_Y,
+                                   float* grad_r, cgtp_stream stream) {
+  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
+  const Plan* P = reinterpret_cast<const Plan*>(plan);
+  if (E < 0 || E >= (int64_t(1) << 31)) return fail(CGTP_ERR_SIZE, "E out of range");
+  if (E == 0) return CGTP_OK;
+  if (!r || !grad_Y || !grad_r) return fail(CGTP_ERR_NULL, "r, grad_Y or grad_r is NULL");
+  if (!aligned16(r) || !aligned16(grad_Y) || !aligned16(grad_r))
+    return fail(CGTP_ERR_ALIGN, "r, grad_Y and grad_r must be 16-byte aligned");
+  cgtp_status st = check_device(*P);
+  if (st != CGTP_OK) return st;
+  {
+    TimedScope ts(*const_cast<Plan*>(P), 4, (cudaStream_t)stream);
+    CGTP_CUDA_TRY(launch_sph_harm_backward(P->L, E, r, grad_Y, grad_r, (cudaStream_t)stream));
+  }
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_edge_forces(int64_t n_atoms, int64_t E, const int32_t* rowptr, const int32_t* rowptr_T,
+                             const int32_t* perm_T, const float* grad_r, float* forces, cgtp_stream stream) {
+  if (n_atoms < 0 || E < 0 || n_atoms >= (int64_t(1) << 31) || E >= (int64_t(1) << 31))
+    return fail(CGTP_ERR_SIZE, "sizes out of range");
+  if (n_atoms == 0) return CGTP_OK;
+  if (!rowptr || !rowptr_T || !forces) return fail(CGTP_ERR_NULL, "rowptr, rowptr_T or forces is NULL");
+  if (E > 0 && (!perm_T || !grad_r)) return fail(CGTP_ERR_NULL, "perm_T or grad_r is NULL");
+  CGTP_CUDA_TRY(launch_edge_forces(n_atoms, rowptr, rowptr_T, perm_T, grad_r, forces, (cudaStream_t)stream));
   return CGTP_OK;
 }
 

@@ -157,6 +157,13 @@ void jit_unload(JitKernel& k);
 
 // generic CUDA kernels (kernels.cu)
 cudaError_t launch_sph_harm(int L, int64_t E, const float* r, float* Y, cudaStream_t s);
+// dr = sum_t dY_t dY_t/dr per edge (harmonics up to L), and the per-atom forces
+// F = sum over receiver edges - sum over sender edges of dr.
+cudaError_t launch_sph_harm_backward(int L, int64_t E, const float* r, const float* dY, float* dr,
+                                     cudaStream_t s);
+cudaError_t launch_edge_forces(int64_t n_atoms, const int32_t* rowptr, const int32_t* rowptr_T,
+                               const int32_t* perm_T, const float* G, float* F, cudaStream_t s);
+
 // dx row sums over the transpose edge list and the dY slice sums, one launch;
 // either part is skipped when its output is null (or S == 1 for dY).
 cudaError_t launch_bwd_reduce(int64_t n_send, int64_t width, const int32_t* rowptr_T, const int32_t* perm_T,

@@ -85,6 +85,126 @@ __global__ void __launch_bounds__(128) sph_harm_kernel(int64_t E, const float* _
   for (int t = threadIdx.x; t < n; t += 128) dst[t] = tile[t];
 }
 
+// dL/dr of the harmonics, one thread per edge:
+//   dr[e] = sum_t dY[e][t] dY_t/dr(r_e).
+// Y_lm = N_lm Q_l^m(z) C_m(x,y) (or S_m) on the unit vector u = r/|r| (the
+// Cartesian form of sph_harm_kernel).  Any smooth extension F of Y off the
+// sphere has the same tangential gradient, so with g = sum_t dY_t grad_u F_t:
+//   dr = (g - (g.u) u) / |r|,
+// where grad C_m = m (C_{m-1}, -S_{m-1}, 0), grad S_m = m (S_{m-1}, C_{m-1}, 0),
+// and Q' follows from differentiating the z recurrence:
+//   (l-m) Q_l' = (2l-1)(Q_{l-1} + z Q_{l-1}') - (l+m-1) Q_{l-2}'.
+// dY rows are staged through shared memory (coalesced); r = 0 gives dr = 0.
+template <int L>
+__global__ void __launch_bounds__(128) sph_harm_backward_kernel(int64_t E, const float* __restrict__ r,
+                                                                const float* __restrict__ dY,
+                                                                float* __restrict__ dr) {
+  constexpr int D = (L + 1) * (L + 1);
+  __shared__ float tile[128 * D];
+  __shared__ float otile[128 * 3];
+  const int64_t e0 = (int64_t)blockIdx.x * 128;
+  const int64_t n = (E - e0 < 128 ? E - e0 : 128);
+  for (int64_t t = threadIdx.x; t < n * D; t += 128) tile[t] = dY[e0 * D + t];
+  __syncthreads();
+  const int64_t e = e0 + threadIdx.x;
+  if (e < E) {
+    const float* g_in = tile + threadIdx.x * D;
+    const float rx = r[3 * e], ry = r[3 * e + 1], rz = r[3 * e + 2];
+    const float r2 = rx * rx + ry * ry + rz * rz;
+    float gx = 0.f, gy = 0.f, gz = 0.f, inv = 0.f, x = 0.f, yy = 0.f, z = 0.f;
+    if (r2 > 0.f) {
+      inv = rsqrtf(r2);
+      x = rx * inv;
+      yy = ry * inv;
+      z = rz * inv;
+      float Cm[L + 1], Sm[L + 1];
+      Cm[0] = 1.f;
+      Sm[0] = 0.f;
+#pragma unroll
+      for (int m = 1; m <= L; ++m) {
+        Cm[m] = x * Cm[m - 1] - yy * Sm[m - 1];
+        Sm[m] = x * Sm[m - 1] + yy * Cm[m - 1];
+      }
+#pragma unroll
+      for (int m = 0; m <= L; ++m) {
+        float qmm = 1.f;
+#pragma unroll
+        for (int k = 1; k <= m; ++k) qmm *= (float)(2 * k - 1);
+        float q2 = 0.f, q1 = qmm, d2 = 0.f, d1 = 0.f;
+#pragma unroll
+        for (int l = m; l <= L; ++l) {
+          float q, dq;
+          if (l == m) {
+            q = qmm;
+            dq = 0.f;
+          } else if (l == m + 1) {
+            q = (float)(2 * m + 1) * z * qmm;
+            dq = (float)(2 * m + 1) * qmm;
+          } else {
+            q = ((float)(2 * l - 1) * z * q1 - (float)(l + m - 1) * q2) / (float)(l - m);
+            dq = ((float)(2 * l - 1) * (q1 + z * d1) - (float)(l + m - 1) * d2) / (float)(l - m);
+          }
+          if (l > m) {
+            q2 = q1;
+            q1 = q;
+            d2 = d1;
+            d1 = dq;
+          }
+          const float nn = c_norm[l * (l + 1) / 2 + m];
+          if (m == 0) {
+            const float w = g_in[l * l + l] * nn;
+            gz = fmaf(w, dq, gz);
+          } else {
+            const float wc = g_in[l * l + l + m] * nn, ws = g_in[l * l + l - m] * nn;
+            const float fm = (float)m;
+            // F_c = Q C_m, F_s = Q S_m
+            gx = fmaf(q * fm, fmaf(wc, Cm[m - 1], ws * Sm[m - 1]), gx);
+            gy = fmaf(q * fm, fmaf(ws, Cm[m - 1], -wc * Sm[m - 1]), gy);
+            gz = fmaf(dq, fmaf(wc, Cm[m], ws * Sm[m]), gz);
+          }
+        }
+      }
+      const float gu = gx * x + gy * yy + gz * z;
+      gx = (gx - gu * x) * inv;
+      gy = (gy - gu * yy) * inv;
+      gz = (gz - gu * z) * inv;
+    }
+    otile[3 * threadIdx.x] = gx;
+    otile[3 * threadIdx.x + 1] = gy;
+    otile[3 * threadIdx.x + 2] = gz;
+  }
+  __syncthreads();
+  for (int64_t t = threadIdx.x; t < n * 3; t += 128) dr[e0 * 3 + t] = otile[t];
+}
+
+// Forces from the edge-vector gradient, one thread per atom a:
+//   F[a] = sum over a's receiver edges of G[e] - sum over a's sender edges of G[e]
+// (r_e = pos_sender - pos_receiver + shift, F = -dL/dpos), each sum in edge
+// order: bitwise reproducible.
+__global__ void __launch_bounds__(128) edge_forces_kernel(int64_t n_atoms, const int32_t* __restrict__ rowptr,
+                                                          const int32_t* __restrict__ rowptr_T,
+                                                          const int32_t* __restrict__ perm_T,
+                                                          const float* __restrict__ G, float* __restrict__ F) {
+  const int64_t a = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (a >= n_atoms) return;
+  float fx = 0.f, fy = 0.f, fz = 0.f;
+  for (int e = rowptr[a]; e < rowptr[a + 1]; ++e) {
+    fx += G[3 * (int64_t)e];
+    fy += G[3 * (int64_t)e + 1];
+    fz += G[3 * (int64_t)e + 2];
+  }
+  float sx = 0.f, sy = 0.f, sz = 0.f;
+  for (int t = rowptr_T[a]; t < rowptr_T[a + 1]; ++t) {
+    const int64_t e = perm_T[t];
+    sx += G[3 * e];
+    sy += G[3 * e + 1];
+    sz += G[3 * e + 2];
+  }
+  F[3 * a] = fx - sx;
+  F[3 * a + 1] = fy - sy;
+  F[3 * a + 2] = fz - sz;
+}
+
 // The backward's closing reductions in one launch.
 //  blocks [0, n_send): dx[j][c] = sum over sender j's edges of m[perm_T[t]][c].
 //    Two groups of 128 threads take the even and the odd positions t0 + 2k of
@@ -194,6 +314,32 @@ cudaError_t launch_sph_harm(int L, int64_t E, const float* r, float* Y, cudaStre
     case 6: sph_harm_kernel<6><<<grid, 128, 0, s>>>(E, r, Y); break;
     default: return cudaErrorInvalidValue;
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sph_harm_backward(int L, int64_t E, const float* r, const float* dY, float* dr,
+                                     cudaStream_t s) {
+  cudaError_t e = ensure_norm();
+  if (e != cudaSuccess) return e;
+  if (E == 0) return cudaSuccess;
+  const dim3 grid((unsigned)((E + 127) / 128));
+  switch (L) {
+    case 0: sph_harm_backward_kernel<0><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
+    case 1: sph_harm_backward_kernel<1><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
+    case 2: sph_harm_backward_kernel<2><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
+    case 3: sph_harm_backward_kernel<3><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
+    case 4: sph_harm_backward_kernel<4><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
+    case 5: sph_harm_backward_kernel<5><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
+    case 6: sph_harm_backward_kernel<6><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_edge_forces(int64_t n_atoms, const int32_t* rowptr, const int32_t* rowptr_T,
+                               const int32_t* perm_T, const float* G, float* F, cudaStream_t s) {
+  if (n_atoms == 0) return cudaSuccess;
+  edge_forces_kernel<<<(unsigned)((n_atoms + 127) / 128), 128, 0, s>>>(n_atoms, rowptr, rowptr_T, perm_T, G, F);
   return cudaGetLastError();
 }
 

@@ -126,6 +126,27 @@ cgtp_status cgtp_real_cg(int l1, int l2, int l3, double* C);
 cgtp_status cgtp_sph_harm(cgtp_plan plan, int64_t E, const float* r, float* Y,
                           cgtp_stream stream);
 
+/* The harmonics' step of the force chain (after the backward's grad_Y):
+ *   grad_r[e][k] = sum_t grad_Y[e][t] dY_t(r_e)/dr_k
+ * r [E,3], grad_Y [E, d_edge], grad_r [E,3]: FP32 device, 16-byte aligned;
+ * grad_r is overwritten; r = 0 gives grad_r = 0.  Forces are minus the
+ * position gradient of the energy (BranchIP page, its force definition).
+ * The pages print no formula for this step; it is the chain rule through
+ * the harmonics of cgtp_sph_harm.  Errors: NULL, SIZE, ALIGN, DEVICE, CUDA. */
+cgtp_status cgtp_sph_harm_backward(cgtp_plan plan, int64_t E, const float* r, const float* grad_Y,
+                                   float* grad_r, cgtp_stream stream);
+
+/* Per-atom forces from the edge-vector gradient, for edges
+ * r_e = pos[col[e]] - pos[i] + shift (receiver CSR rowptr, sender lists
+ * rowptr_T/perm_T as from cgtp_csr_transpose; all int32 device arrays):
+ *   forces[a] = sum over a's receiver edges of grad_r[e]
+ *             - sum over a's sender edges of grad_r[e]      (= -dL/dpos[a]).
+ * grad_r [E,3], forces [n_atoms,3]: FP32 device; forces overwritten; each
+ * sum in edge order (bitwise reproducible, no atomics).  Needs no plan. */
+cgtp_status cgtp_edge_forces(int64_t n_atoms, int64_t E, const int32_t* rowptr, const int32_t* rowptr_T,
+                             const int32_t* perm_T, const float* grad_r, float* forces,
+                             cgtp_stream stream);
+
 /* Forward CGTP convolution (the x' of LunaTP Table 11), formula above.
  *   n_recv receivers, n_send senders, E edges (0 <= E < 2^31)
  *   rowptr [n_recv+1], col [E] (int32, device); x [n_send, d_in];

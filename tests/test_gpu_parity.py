@@ -135,6 +135,24 @@ def test_backward(name, dev):
         assert_close(dx[send_s], rdx[send_s], f"{name} dx (128 sampled senders)")
 
 
+@pytest.mark.parametrize("name", ALL)
+def test_force_chain(name, dev):
+    """grad_r = dL/dr through the harmonics, and the per-atom forces from it."""
+    c = case(name, dev)
+    w = c.w
+    dYg = np.random.default_rng(7).standard_normal((w.E, w.P.D_e)).astype(np.float32)
+    gr = c.plan.sph_harm_backward(c.r, T(dYg, dev))
+    ref = O.sph_harm_backward(w.P.L, w.r32, dYg)
+    assert_close(gr.cpu().numpy(), ref, f"{name} grad_r")
+    # forces on the same FP32 input, then the whole chain
+    g32 = ref.astype(np.float32)
+    F = C().edge_forces(c.rowptr, c.rpt, c.perm, T(g32, dev)).cpu().numpy()
+    assert_close(F, O.edge_forces(w.N, w.rowptr, w.col, g32), f"{name} forces")
+    Fc = C().edge_forces(c.rowptr, c.rpt, c.perm, gr).cpu().numpy()
+    assert_close(Fc, O.edge_forces(w.N, w.rowptr, w.col, ref), f"{name} forces (chain)")
+    assert np.abs(Fc.sum(0)).max() <= 1e-4 * np.abs(Fc).max() * np.sqrt(w.N)  # no net force
+
+
 @pytest.mark.parametrize("name", ["lmax2", "lmax6"])
 def test_bitwise_repeatable(name, dev):
     c = case(name, dev)
