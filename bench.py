@@ -205,10 +205,20 @@ def run_cgtp(args, rank, world, local_rank):
         for _ in range(20):
             step(T["r"], T["x"], T["W"], T["g"])
         torch.cuda.synchronize()
-    plan.kernel_times()  # discard
-    plan.set_timing(True)
+    # the step's four launches captured once in a CUDA graph (no launch gaps);
+    # the headline times K replays
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(T["r"], T["x"], T["W"], T["g"])
+        graph.replay()
+        torch.cuda.synchronize()
+        plan.check_device_error()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
+    ev_e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
     ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(args.steps)]
     if world > 1:
@@ -218,13 +228,28 @@ def run_cgtp(args, rank, world, local_rank):
         flush.zero_()  # L2 flush (not timed)
         a, b = ev[k]
         a.record(stream)
-        step(T["r"], T["x"], T["W"], T["g"])
+        if graph is not None:
+            graph.replay()
+        else:
+            step(T["r"], T["x"], T["W"], T["g"])
         b.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    # the same K steps launched one by one, with the library's per-kernel
+    # events on: the per-kernel breakdown and the roofline
+    plan.kernel_times()  # discard
+    plan.set_timing(True)
+    for k in range(args.steps):
+        flush.zero_()
+        a, b = ev_e[k]
+        a.record(stream)
+        step(T["r"], T["x"], T["W"], T["g"])
+        b.record(stream)
+    torch.cuda.synchronize()
     plan.set_timing(False)
-    kt = plan.kernel_times()  # the kernels of the K timed steps
+    kt = plan.kernel_times()  # the kernels of the K eager steps
+    ms_eager = float(np.mean([a.elapsed_time(b) for a, b in ev_e]))
     # forward-only steps (harmonics + forward), for the forward edges/s
     for k in range(args.steps):
         flush.zero_()
@@ -306,11 +331,13 @@ def run_cgtp(args, rank, world, local_rank):
                config={"workload": f"{name}: {c['desc']}", "atoms": N, "edges": E,
                        "irreps_in": c["irreps_in"], "irreps_edge": c["irreps_edge"],
                        "irreps_out": c["irreps_out"], "seed": 0,
-                       "step": "sph_harm + forward + backward (dx, dW, dY)",
+                       "step": "sph_harm + forward + backward (dx, dW, dY)"
+                               + (", replayed from one CUDA graph" if graph is not None else ""),
                        "l2": f"{L2_FLUSH_BYTES >> 20} MB buffer written before every timed step (not timed)",
                        "parallelism": "replicas" if world > 1 else "single GPU"},
                atoms_per_s=world * N / (ms_step * 1e-3),
                fwd_edges_per_s=world * E / (fwd_ms * 1e-3), fwd_ms=fwd_ms,
+               ms_per_step_launched=ms_eager,
                force_chain={"ms": force_ms, "edges_per_s": world * E / (force_ms * 1e-3),
                             "what": "sph_harm_backward + edge_forces after the step (not in it)"},
                roofline=roof, kernels=kernels, gpu_launches=int(gpu_launches), e2e=e2e, clocks=clocks)
@@ -517,6 +544,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cgtp", choices=["cgtp", "reference"])
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the step launched kernel by kernel instead of from a CUDA graph")
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(WL.CONFIGS))
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline field (0 to skip)")
