@@ -278,6 +278,8 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
        "    float* __restrict__ dW, float* __restrict__ dyp, float* __restrict__ msg,\n"
        "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err) {\n"
        "  extern __shared__ __align__(128) unsigned char smem[];\n"
+       "  grid_dependency_wait();  // the previous kernel's results are visible\n"
+       "  grid_launch_dependents();\n"
        "  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  const u32 gfull0 = full0 + OFF_GFULL, gempty0 = full0 + OFF_GEMPTY;\n"

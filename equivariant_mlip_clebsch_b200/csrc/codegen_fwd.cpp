@@ -149,6 +149,8 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
        "    const float* __restrict__ Y, const float* __restrict__ W, float* __restrict__ out,\n"
        "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err) {\n"
        "  extern __shared__ __align__(128) unsigned char smem[];\n"
+       "  grid_dependency_wait();  // the previous kernel's results are visible\n"
+       "  grid_launch_dependents();\n"
        "  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  if (threadIdx.x == 0) {\n"

@@ -29,6 +29,7 @@ struct Driver {
   CUresult (*funcSetAttribute)(CUfunction, CUfunction_attribute, int) = nullptr;
   CUresult (*launchKernel)(CUfunction, unsigned, unsigned, unsigned, unsigned, unsigned, unsigned,
                            unsigned, CUstream, void**, void**) = nullptr;
+  CUresult (*launchKernelEx)(const CUlaunchConfig*, CUfunction, void**, void**) = nullptr;
   CUresult (*getErrorString)(CUresult, const char**) = nullptr;
   CUresult (*occupancy)(int*, CUfunction, int, size_t) = nullptr;
   bool ok = false;
@@ -61,6 +62,8 @@ Driver& driver() {
            entry("cuGetErrorString", d.getErrorString, err) &&
            entry("cuOccupancyMaxActiveBlocksPerMultiprocessor", d.occupancy, err);
     d.err = err;
+    std::string ignore;  // optional: without it, launches are plain
+    entry("cuLaunchKernelEx", d.launchKernelEx, ignore);
   });
   return d;
 }
@@ -189,8 +192,30 @@ cgtp_status jit_compile(const std::string& src, const std::string& name, JitKern
 cgtp_status jit_launch(const JitKernel& k, dim3 grid, void** args, cudaStream_t stream) {
   if (!k.function) return fail(CGTP_ERR_CUDA, "kernel " + k.name + " is not loaded");
   Driver& d = driver();
-  CUresult cr = d.launchKernel((CUfunction)k.function, grid.x, grid.y, grid.z, k.threads, 1, 1,
-                               k.smem, (CUstream)stream, args, nullptr);
+  CUresult cr;
+  if (d.launchKernelEx) {
+    // programmatic dependent launch: the kernel may start while its
+    // predecessor on the stream finishes; it waits (griddepcontrol.wait)
+    // before touching any memory the predecessor writes
+    CUlaunchAttribute attr[1];
+    attr[0].id = CU_LAUNCH_ATTRIBUTE_PROGRAMMATIC_STREAM_SERIALIZATION;
+    attr[0].value.programmaticStreamSerializationAllowed = 1;
+    CUlaunchConfig cfg = {};
+    cfg.gridDimX = grid.x;
+    cfg.gridDimY = grid.y;
+    cfg.gridDimZ = grid.z;
+    cfg.blockDimX = (unsigned)k.threads;
+    cfg.blockDimY = 1;
+    cfg.blockDimZ = 1;
+    cfg.sharedMemBytes = (unsigned)k.smem;
+    cfg.hStream = (CUstream)stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cr = d.launchKernelEx(&cfg, (CUfunction)k.function, args, nullptr);
+  } else {
+    cr = d.launchKernel((CUfunction)k.function, grid.x, grid.y, grid.z, k.threads, 1, 1, k.smem,
+                        (CUstream)stream, args, nullptr);
+  }
   if (cr != CUDA_SUCCESS) return fail(CGTP_ERR_CUDA, "launch of " + k.name + ": " + cu_str(cr));
   return CGTP_OK;
 }

@@ -13,6 +13,28 @@ namespace cgtp {
 
 namespace {
 
+// Programmatic dependent launch (as for the generated kernels): wait for the
+// previous kernel on the stream and its writes, then let the next one launch.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, unsigned block, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Normalisation of the component-normalised real harmonics:
 //   N_l0 = sqrt(2l+1),  N_lm = sqrt(2l+1) sqrt(2 (l-m)!/(l+m)!)  (m > 0)
 // index l*(l+1)/2 + m, l <= 6.
@@ -22,6 +44,8 @@ bool g_norm_ready[64] = {false};
 template <int L>
 __global__ void __launch_bounds__(128) sph_harm_kernel(int64_t E, const float* __restrict__ r,
                                                        float* __restrict__ Y) {
+  grid_dependency_wait();
+  grid_launch_dependents();
   constexpr int D = (L + 1) * (L + 1);
   __shared__ float tile[128 * D];
   const int64_t e0 = (int64_t)blockIdx.x * 128;
@@ -99,6 +123,8 @@ template <int L>
 __global__ void __launch_bounds__(128) sph_harm_backward_kernel(int64_t E, const float* __restrict__ r,
                                                                 const float* __restrict__ dY,
                                                                 float* __restrict__ dr) {
+  grid_dependency_wait();
+  grid_launch_dependents();
   constexpr int D = (L + 1) * (L + 1);
   __shared__ float tile[128 * D];
   __shared__ float otile[128 * 3];
@@ -185,6 +211,8 @@ __global__ void __launch_bounds__(128) edge_forces_kernel(int64_t n_atoms, const
                                                           const int32_t* __restrict__ rowptr_T,
                                                           const int32_t* __restrict__ perm_T,
                                                           const float* __restrict__ G, float* __restrict__ F) {
+  grid_dependency_wait();
+  grid_launch_dependents();
   const int64_t a = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (a >= n_atoms) return;
   float fx = 0.f, fy = 0.f, fz = 0.f;
@@ -224,6 +252,8 @@ __global__ void __launch_bounds__(kEpiThreads) bwd_reduce_kernel(
     int64_t n_send, int64_t width, const int32_t* __restrict__ rowptr_T, const int32_t* __restrict__ perm_T,
     const float* __restrict__ m, float* __restrict__ dx, int S, int64_t ny, const float* __restrict__ parts,
     float* __restrict__ dy) {
+  grid_dependency_wait();
+  grid_launch_dependents();
   __shared__ float4 part[128];
   const int64_t blk = blockIdx.x;
   if (blk >= n_send || dx == nullptr) {
@@ -305,16 +335,15 @@ cudaError_t launch_sph_harm(int L, int64_t E, const float* r, float* Y, cudaStre
   if (E == 0) return cudaSuccess;
   const dim3 grid((unsigned)((E + 127) / 128));
   switch (L) {
-    case 0: sph_harm_kernel<0><<<grid, 128, 0, s>>>(E, r, Y); break;
-    case 1: sph_harm_kernel<1><<<grid, 128, 0, s>>>(E, r, Y); break;
-    case 2: sph_harm_kernel<2><<<grid, 128, 0, s>>>(E, r, Y); break;
-    case 3: sph_harm_kernel<3><<<grid, 128, 0, s>>>(E, r, Y); break;
-    case 4: sph_harm_kernel<4><<<grid, 128, 0, s>>>(E, r, Y); break;
-    case 5: sph_harm_kernel<5><<<grid, 128, 0, s>>>(E, r, Y); break;
-    case 6: sph_harm_kernel<6><<<grid, 128, 0, s>>>(E, r, Y); break;
+    case 0: return launch_pdl(sph_harm_kernel<0>, grid, 128, s, E, r, Y);
+    case 1: return launch_pdl(sph_harm_kernel<1>, grid, 128, s, E, r, Y);
+    case 2: return launch_pdl(sph_harm_kernel<2>, grid, 128, s, E, r, Y);
+    case 3: return launch_pdl(sph_harm_kernel<3>, grid, 128, s, E, r, Y);
+    case 4: return launch_pdl(sph_harm_kernel<4>, grid, 128, s, E, r, Y);
+    case 5: return launch_pdl(sph_harm_kernel<5>, grid, 128, s, E, r, Y);
+    case 6: return launch_pdl(sph_harm_kernel<6>, grid, 128, s, E, r, Y);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_sph_harm_backward(int L, int64_t E, const float* r, const float* dY, float* dr,
@@ -324,23 +353,22 @@ cudaError_t launch_sph_harm_backward(int L, int64_t E, const float* r, const flo
   if (E == 0) return cudaSuccess;
   const dim3 grid((unsigned)((E + 127) / 128));
   switch (L) {
-    case 0: sph_harm_backward_kernel<0><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
-    case 1: sph_harm_backward_kernel<1><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
-    case 2: sph_harm_backward_kernel<2><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
-    case 3: sph_harm_backward_kernel<3><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
-    case 4: sph_harm_backward_kernel<4><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
-    case 5: sph_harm_backward_kernel<5><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
-    case 6: sph_harm_backward_kernel<6><<<grid, 128, 0, s>>>(E, r, dY, dr); break;
+    case 0: return launch_pdl(sph_harm_backward_kernel<0>, grid, 128, s, E, r, dY, dr);
+    case 1: return launch_pdl(sph_harm_backward_kernel<1>, grid, 128, s, E, r, dY, dr);
+    case 2: return launch_pdl(sph_harm_backward_kernel<2>, grid, 128, s, E, r, dY, dr);
+    case 3: return launch_pdl(sph_harm_backward_kernel<3>, grid, 128, s, E, r, dY, dr);
+    case 4: return launch_pdl(sph_harm_backward_kernel<4>, grid, 128, s, E, r, dY, dr);
+    case 5: return launch_pdl(sph_harm_backward_kernel<5>, grid, 128, s, E, r, dY, dr);
+    case 6: return launch_pdl(sph_harm_backward_kernel<6>, grid, 128, s, E, r, dY, dr);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_edge_forces(int64_t n_atoms, const int32_t* rowptr, const int32_t* rowptr_T,
                                const int32_t* perm_T, const float* G, float* F, cudaStream_t s) {
   if (n_atoms == 0) return cudaSuccess;
-  edge_forces_kernel<<<(unsigned)((n_atoms + 127) / 128), 128, 0, s>>>(n_atoms, rowptr, rowptr_T, perm_T, G, F);
-  return cudaGetLastError();
+  return launch_pdl(edge_forces_kernel, dim3((unsigned)((n_atoms + 127) / 128)), 128, s, n_atoms, rowptr, rowptr_T,
+                    perm_T, G, F);
 }
 
 cudaError_t launch_bwd_reduce(int64_t n_send, int64_t width, const int32_t* rowptr_T, const int32_t* perm_T,
@@ -349,9 +377,8 @@ cudaError_t launch_bwd_reduce(int64_t n_send, int64_t width, const int32_t* rowp
   const int64_t nx = (dx && width > 0) ? n_send : 0;
   const int64_t ndy = (dy && S > 1 && ny > 0) ? std::min<int64_t>((ny + kEpiThreads - 1) / kEpiThreads, 148 * 4) : 0;
   if (nx + ndy == 0) return cudaSuccess;
-  bwd_reduce_kernel<<<(unsigned)(nx + ndy), kEpiThreads, 0, s>>>(nx, width, rowptr_T, perm_T, m, nx ? dx : nullptr,
-                                                                S, ndy ? ny : 0, parts, dy);
-  return cudaGetLastError();
+  return launch_pdl(bwd_reduce_kernel, dim3((unsigned)(nx + ndy)), kEpiThreads, s, nx, width, rowptr_T, perm_T, m,
+                    nx ? dx : nullptr, S, ndy ? ny : (int64_t)0, parts, dy);
 }
 
 }  // namespace cgtp

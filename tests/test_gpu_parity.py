@@ -164,6 +164,38 @@ def test_bitwise_repeatable(name, dev):
         assert torch.equal(p, q)
 
 
+@pytest.mark.parametrize("name", ["lmax2", "lmax3"])
+def test_cuda_graph_replay(name, dev):
+    """The step (harmonics, forward, backward) captured in a CUDA graph replays
+    to the same bits as the launched calls (no allocation or host sync inside
+    the calls)."""
+    c = case(name, dev)
+    w = c.w
+    Y = torch.empty_like(c.Y)
+    out = torch.empty((w.N, c.plan.d_out), device=dev)
+    grads = tuple(torch.empty_like(t) for t in (c.x, c.W, Y))
+    ws = torch.empty(max(c.plan.workspace_size(w.N, w.N, w.E), 256), dtype=torch.uint8, device=dev)
+
+    def step():
+        c.plan.sph_harm(c.r, Y)
+        c.plan.forward(c.rowptr, c.col, c.x, Y, c.W, out=out)
+        c.plan.backward(c.rowptr, c.col, c.rpt, c.perm, c.x, Y, c.W, c.g, grads=grads, workspace=ws)
+
+    step()
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in (Y, out) + grads]
+    for t in (Y, out) + grads:
+        t.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    g.replay()
+    torch.cuda.synchronize()
+    c.plan.check_device_error()
+    for a, b in zip(ref, (Y, out) + grads):
+        assert torch.equal(a, b)
+
+
 def test_partial_gradients(dev):
     c = case("lmax2_wide", dev)
     dx, dW, dY = c.backward()
