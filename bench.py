@@ -141,6 +141,40 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------
+# ranks: one process per GPU, independent replicas of the step
+# --------------------------------------------------------------------------
+def init_distributed(world: int, local_rank: int, backend: str = "nccl", timeout_s: int = 120) -> None:
+    """Process group for N > 1 (RANK, WORLD_SIZE, MASTER_* from the launcher's
+    environment).  The replicas exchange nothing on the data path: the group
+    only brackets the timed region with barriers and takes the max time."""
+    if world <= 1:
+        return
+    import datetime
+    import torch
+    import torch.distributed as dist
+    if backend == "nccl":
+        torch.cuda.set_device(local_rank)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The slowest rank's time (a number of one rank for world == 1)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_value(world: int, units_per_rank: int, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time (weak scaling: every rank runs the full workload)."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
+# --------------------------------------------------------------------------
 # workload (host side)
 # --------------------------------------------------------------------------
 def build_workload(name: str, seed: int = 0):
@@ -278,12 +312,8 @@ def run_cgtp(args, rank, world, local_rank):
     ms_steps = [a.elapsed_time(b) for a, b in ev]
     ms_fwd = [a.elapsed_time(b) for a, b in ev_f]
     force_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_c]))
-    ms_step = float(np.sum(ms_steps)) / args.steps
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
-    value = world * E / (ms_step * 1e-3)
+    ms_step = max_over_ranks(float(np.sum(ms_steps)) / args.steps, world, dev)
+    value = replica_value(world, E, ms_step)
     fwd_ms = float(np.mean(ms_fwd))
 
     # ---- per-kernel roofline (device time from the library's events)
@@ -335,7 +365,7 @@ def run_cgtp(args, rank, world, local_rank):
                                + (", replayed from one CUDA graph" if graph is not None else ""),
                        "l2": f"{L2_FLUSH_BYTES >> 20} MB buffer written before every timed step (not timed)",
                        "parallelism": "replicas" if world > 1 else "single GPU"},
-               atoms_per_s=world * N / (ms_step * 1e-3),
+               atoms_per_s=replica_value(world, N, ms_step),
                fwd_edges_per_s=world * E / (fwd_ms * 1e-3), fwd_ms=fwd_ms,
                ms_per_step_launched=ms_eager,
                force_chain={"ms": force_ms, "edges_per_s": world * E / (force_ms * 1e-3),
@@ -429,10 +459,10 @@ def run_e2e(args, plan, T, host, Y, out, dx, dW, dY, ws, E, dev, world):
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     run(steps, a, b)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world, dev)
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = sum(t.numel() * t.element_size() for t in hout)
-    return {"value": world * E / (ms * 1e-3), "unit": "edges/s", "h2d_bytes_per_step": int(h2d),
+    return {"value": replica_value(world, E, ms), "unit": "edges/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps,
             "pipelined": "host->device, compute and device->host on three streams, two buffer sets"}
 
@@ -562,12 +592,7 @@ def main():
         if res is not None:
             print(json.dumps(res), flush=True)
         return
-    if world > 1:
-        import datetime
-        import torch
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    init_distributed(world, local_rank, "nccl")
     res = run_cgtp(args, rank, world, local_rank)
     if rank == 0 and args.cpu_budget > 0 and not args.profile:
         s = oracle_sample(args.config, args.cpu_budget)
