@@ -22,10 +22,143 @@
 #include <cstring>
 #include <numeric>
 #include <sstream>
+#include <tuple>
 
 #include "codegen_common.hpp"
 
 namespace cgtp {
+
+// The kernel entry after the role functions: service warps, then each
+// consumer warp runs its slot's role in every slice.
+static void gen_fwd_entry(std::ostringstream& o, const std::string& kname, int min_blocks,
+                          const std::string& dispatch) {
+  o << "extern \"C\" __global__ void __launch_bounds__((NW + 2) * 32, " << min_blocks << ") " << kname
+    << "(const int* __restrict__ rowptr, const int* __restrict__ col, const float* __restrict__ x,\n"
+       "    const float* __restrict__ Y, const float* __restrict__ W, float* __restrict__ out,\n"
+       "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err) {\n"
+       "  extern __shared__ __align__(128) unsigned char smem[];\n"
+       "  grid_dependency_wait();  // the previous kernel's results are visible\n"
+       "  grid_launch_dependents();\n"
+       "  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;\n"
+       "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
+       "  if (threadIdx.x == 0) {\n"
+       "    for (int s = 0; s < NSTAGE; ++s) { mbar_init(full0 + 8 * s, FULL_COUNT); mbar_init(empty0 + 8 * s, NW); }\n"
+       "    fence_mbar_init();\n"
+       "  }\n"
+       "  __syncthreads();\n"
+       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, nullptr, err, smem, lane); return; }\n"
+       "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, ent, kEntBegin, nullptr, err, smem, lane); return; }\n"
+       "  int q = 0;\n"
+       "  for (int slice = 0; slice < NSLICE; ++slice) {\n"
+       "    const int slot = slice * NW + warp;\n"
+       "    const int u0 = kU0[slot], chs = kChs[slice];\n"
+       "    switch (kShape[slot]) {\n"
+    << dispatch << "    default: fcons_idle(rowptr, n_recv, err, smem, &q); break;\n    }\n  }\n}\n";
+}
+
+static void gen_fwd_idle(std::ostringstream& o) {
+  // idle consumer: keeps the stage accounting of the CTA
+  o << "__device__ __noinline__ void fcons_idle(const int* __restrict__ rowptr, int n_recv,\n"
+       "    int* __restrict__ err, unsigned char* smem, int* qp) {\n"
+       "  const int lane = threadIdx.x & 31;\n"
+       "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
+       "  int q = *qp;\n"
+       "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
+       "    const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
+       "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
+       "      const int s = q % NSTAGE;\n"
+       "      if (!mbar_wait(full0 + 8 * s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
+       "      __syncwarp();\n"
+       "      if (lane == 0) mbar_arrive(empty0 + 8 * s);\n"
+       "    }\n"
+       "  }\n"
+       "  *qp = q;\n"
+       "}\n";
+}
+
+// Wide plans: one function per (2l1+1, 2l3+1, full channel blocks) shape; a
+// role's path offsets come from per-slot tables.
+static std::string gen_fwd_generic(const Plan& P, const std::vector<SliceLayout>& SL, const KernelShape& K,
+                                   const std::string& kname, int min_blocks, std::ostringstream& o,
+                                   const std::vector<int>& slice_of) {
+  const FwdConfig& F = P.fcfg;
+  const int S = K.S, NW = K.nw;
+  std::vector<std::tuple<int, int, bool>> shapes;
+  std::vector<int> shape_of(P.fwd_roles.size(), -1);
+  for (size_t ri = 0; ri < P.fwd_roles.size(); ++ri) {
+    const FwdRole& r = P.fwd_roles[ri];
+    const Path& p = P.paths[r.paths[0]];
+    const auto key = std::make_tuple(2 * P.in[r.irrep].l + 1, 2 * p.l3 + 1, P.in[r.irrep].mul % 32 == 0);
+    auto it = std::find(shapes.begin(), shapes.end(), key);
+    shape_of[ri] = (int)(it - shapes.begin());
+    if (it == shapes.end()) shapes.push_back(key);
+  }
+  for (size_t k = 0; k < shapes.size(); ++k) {
+    const int N1 = std::get<0>(shapes[k]), N3 = std::get<1>(shapes[k]);
+    const bool full = std::get<2>(shapes[k]);
+    o << "// shape " << k << ": one path " << N1 << " x " << N3 << ", one channel per lane\n"
+      << "__device__ __noinline__ void fgen_" << k
+      << "(const int* __restrict__ rowptr, int n_recv, float* __restrict__ out, int* __restrict__ err,\n"
+         "    unsigned char* smem, int u0, int chs, int choff, int wst, int xst, int ooff, int mul, int* qp) {\n"
+         "  const int lane = threadIdx.x & 31;\n"
+         "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
+         "  const int u = u0 + lane;\n"
+         "  const bool ok = " << (full ? "true" : "u < mul") << ";\n"
+         "  (void)mul;\n"
+         "  int q = *qp;\n"
+         "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
+         "  const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
+         "  float acc[" << N3 << "];\n"
+         "#pragma unroll\n  for (int k = 0; k < " << N3 << "; ++k) acc[k] = 0.f;\n"
+         "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
+         "    const int s = q % NSTAGE;\n"
+         "    if (!mbar_wait(full0 + 8 * s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
+         "    const int nb = min(NB, e1 - eb);\n"
+         "    const unsigned char* st = stage_ptr(smem, s);\n"
+         "    const float* sW = reinterpret_cast<const float*>(st + OFF_W) + wst;\n"
+         "    const float* sX = reinterpret_cast<const float*>(st + OFF_X) + xst;\n"
+         "    const float* sC = reinterpret_cast<const float*>(st + OFF_CH) + choff;\n"
+         "#pragma unroll 1\n    for (int b = 0; b < nb; ++b) {\n"
+         "      float xv[1][" << N1 << "], w[1];\n"
+         "#pragma unroll\n      for (int m1 = 0; m1 < " << N1 << "; ++m1) xv[0][m1] = ok ? sX[b * XS + u * " << N1
+      << " + m1] : 0.f;\n"
+         "      w[0] = ok ? sW[b * WS + u] : 0.f;\n"
+         "      fpath<" << N1 << "," << N3 << ",1,0," << N3 << ">(acc, sC + b * chs, xv, w);\n"
+         "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n"
+         "  if (ok) {\n    float* orow = out + (size_t)i * DOUT + ooff;\n"
+         "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) orow[u * " << N3 << " + m3] = acc[m3];\n  }\n"
+         "  }\n  *qp = q;\n}\n";
+  }
+  gen_fwd_idle(o);
+  auto table = [&](const char* name, auto f) {
+    o << "__constant__ int " << name << "[" << S * NW << "] = {";
+    for (int s = 0; s < S; ++s)
+      for (int w = 0; w < NW; ++w) o << (w < (int)F.slice_roles[s].size() ? f(s, F.slice_roles[s][w]) : 0) << ",";
+    o << "};\n";
+  };
+  o << "__constant__ int kShape[" << S * NW << "] = {";
+  for (int s = 0; s < S; ++s)
+    for (int w = 0; w < NW; ++w)
+      o << (w < (int)F.slice_roles[s].size() ? shape_of[F.slice_roles[s][w]] : -1) << ",";
+  o << "};\n";
+  table("kU0", [&](int, int ri) { return P.fwd_roles[ri].u0; });
+  table("kChOff", [&](int s, int ri) { return SL[s].ch_off.at(P.fwd_roles[ri].paths[0]); });
+  table("kWst", [&](int s, int ri) { return SL[s].w_st.at(P.fwd_roles[ri].paths[0]); });
+  table("kXst", [&](int s, int ri) { return SL[s].x_st.at(P.fwd_roles[ri].irrep); });
+  table("kOoff", [&](int, int ri) { return P.paths[P.fwd_roles[ri].paths[0]].o_off; });
+  table("kMul", [&](int, int ri) { return P.in[P.fwd_roles[ri].irrep].mul; });
+  o << "__constant__ int kEntBegin[" << S + 1 << "] = {";
+  for (int v : P.fwd_ent_begin) o << v << ",";
+  o << "};\n";
+  (void)slice_of;
+  std::ostringstream d;
+  for (size_t k = 0; k < shapes.size(); ++k)
+    d << "    case " << k << ": fgen_" << k
+      << "(rowptr, n_recv, out, err, smem, u0, chs, kChOff[slot], kWst[slot], kXst[slot], kOoff[slot], kMul[slot], "
+         "&q); break;\n";
+  gen_fwd_entry(o, kname, min_blocks, d.str());
+  return o.str();
+}
 
 static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>& SL, const KernelShape& K,
                                   const std::string& kname, int min_blocks) {
@@ -38,6 +171,7 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
   std::vector<int> slice_of(P.fwd_roles.size(), -1);
   for (int s = 0; s < S; ++s)
     for (int v : F.slice_roles[s]) slice_of[v] = s;
+  if (F.generic) return gen_fwd_generic(P, SL, K, kname, min_blocks, o, slice_of);
   std::vector<int> shape_of(P.fwd_roles.size(), -1), shape_rep;
   for (size_t ri = 0; ri < P.fwd_roles.size(); ++ri) {
     const FwdRole& r = P.fwd_roles[ri];
@@ -116,23 +250,7 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
     }
     o << "  }\n  *qp = q;\n}\n";
   }
-  // idle consumer: keeps the stage accounting of the CTA
-  o << "__device__ __noinline__ void fcons_idle(const int* __restrict__ rowptr, int n_recv,\n"
-       "    int* __restrict__ err, unsigned char* smem, int* qp) {\n"
-       "  const int lane = threadIdx.x & 31;\n"
-       "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
-       "  int q = *qp;\n"
-       "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
-       "    const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
-       "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
-       "      const int s = q % NSTAGE;\n"
-       "      if (!mbar_wait(full0 + 8 * s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
-       "      __syncwarp();\n"
-       "      if (lane == 0) mbar_arrive(empty0 + 8 * s);\n"
-       "    }\n"
-       "  }\n"
-       "  *qp = q;\n"
-       "}\n";
+  gen_fwd_idle(o);
   o << "__constant__ int kShape[" << S * NW << "] = {";
   for (int s = 0; s < S; ++s)
     for (int w = 0; w < NW; ++w)
@@ -144,30 +262,10 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
   o << "};\n__constant__ int kEntBegin[" << S + 1 << "] = {";
   for (int v : P.fwd_ent_begin) o << v << ",";
   o << "};\n";
-  o << "extern \"C\" __global__ void __launch_bounds__((NW + 2) * 32, " << min_blocks << ") " << kname
-    << "(const int* __restrict__ rowptr, const int* __restrict__ col, const float* __restrict__ x,\n"
-       "    const float* __restrict__ Y, const float* __restrict__ W, float* __restrict__ out,\n"
-       "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err) {\n"
-       "  extern __shared__ __align__(128) unsigned char smem[];\n"
-       "  grid_dependency_wait();  // the previous kernel's results are visible\n"
-       "  grid_launch_dependents();\n"
-       "  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;\n"
-       "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
-       "  if (threadIdx.x == 0) {\n"
-       "    for (int s = 0; s < NSTAGE; ++s) { mbar_init(full0 + 8 * s, FULL_COUNT); mbar_init(empty0 + 8 * s, NW); }\n"
-       "    fence_mbar_init();\n"
-       "  }\n"
-       "  __syncthreads();\n"
-       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, nullptr, err, smem, lane); return; }\n"
-       "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, ent, kEntBegin, nullptr, err, smem, lane); return; }\n"
-       "  int q = 0;\n"
-       "  for (int slice = 0; slice < NSLICE; ++slice) {\n"
-       "    const int slot = slice * NW + warp;\n"
-       "    const int u0 = kU0[slot], chs = kChs[slice];\n"
-       "    switch (kShape[slot]) {\n";
+  std::ostringstream d;
   for (size_t k = 0; k < shape_rep.size(); ++k)
-    o << "    case " << k << ": fcons_" << k << "(rowptr, n_recv, out, err, smem, u0, chs, &q); break;\n";
-  o << "    default: fcons_idle(rowptr, n_recv, err, smem, &q); break;\n    }\n  }\n}\n";
+    d << "    case " << k << ": fcons_" << k << "(rowptr, n_recv, out, err, smem, u0, chs, &q); break;\n";
+  gen_fwd_entry(o, kname, min_blocks, d.str());
   return o.str();
 }
 
@@ -231,29 +329,74 @@ cgtp_status build_forward(Plan& P) {
   FwdConfig& F = P.fcfg;
   F = FwdConfig();
   if (NR == 0) return CGTP_OK;  // no paths: forward writes zeros
-  // up to 16 consumer warps per CTA; 8 when the roles are register-heavy
-  // (wide inputs), so that two CTAs of (8 + 2) warps keep 96 registers each
-  int kMaxWarps = 16;
-  for (auto& r : P.fwd_roles)
-    if (P.in[r.irrep].l >= 3 && NR > 8) kMaxWarps = 8;
-  F.S = (NR + kMaxWarps - 1) / kMaxWarps;
-  // longest-processing-time assignment of roles to slices
-  std::vector<int> order(NR);
-  std::iota(order.begin(), order.end(), 0);
-  std::stable_sort(order.begin(), order.end(),
-                   [&](int a, int b) { return P.fwd_roles[a].cost > P.fwd_roles[b].cost; });
-  const int cap = (NR + F.S - 1) / F.S;
-  F.slice_roles.assign(F.S, {});
-  std::vector<double> load(F.S, 0.0);
-  for (int ri : order) {
-    int best = -1;
-    for (int s = 0; s < F.S; ++s)
-      if ((int)F.slice_roles[s].size() < cap && (best < 0 || load[s] < load[best])) best = s;
-    F.slice_roles[best].push_back(ri);
-    load[best] += P.fwd_roles[ri].cost;
+  // Wide plans (an input of l >= 3 and more than 16 coarse roles): the coarse
+  // roles' fully unrolled multi-path code outgrows the instruction cache
+  // (measured on B200: most cycles stalled on instruction fetch).  There a
+  // role is one path and one block of 32 channels, and roles of the same
+  // (2l1+1, 2l3+1) shape share one function with the path's offsets as
+  // arguments; slices take roles in (shape, irrep) order, 8 per slice.
+  bool wide = false;
+  for (auto& r : P.fwd_roles) wide = wide || P.in[r.irrep].l >= 3;
+  F.generic = wide && NR > 16;
+  std::vector<FwdRole> roles;
+  if (F.generic) {
+    for (size_t k = 0; k < P.paths.size(); ++k) {
+      const Path& p = P.paths[k];
+      const int mul = P.in[p.irrep].mul;
+      for (int u0 = 0; u0 < mul; u0 += 32) {
+        FwdRole r;
+        r.irrep = p.irrep;
+        r.u0 = u0;
+        r.R = 1;
+        r.paths = {(int)k};
+        r.cost = fwd_role_cost(P, r);
+        roles.push_back(r);
+      }
+    }
+    auto key = [&](const FwdRole& r) {
+      const Path& p = P.paths[r.paths[0]];
+      return std::make_tuple(-(2 * P.in[r.irrep].l + 1) * (2 * p.l3 + 1), 2 * P.in[r.irrep].l + 1, 2 * p.l3 + 1,
+                             r.irrep, r.paths[0], r.u0);
+    };
+    std::stable_sort(roles.begin(), roles.end(), [&](const FwdRole& a, const FwdRole& b) { return key(a) < key(b); });
+    P.fwd_roles = roles;
   }
-  for (auto& v : F.slice_roles) std::sort(v.begin(), v.end());
-  F.weight = load;
+  const int NR2 = (int)P.fwd_roles.size();
+  if (F.generic) {
+    const int per = 8;
+    F.S = (NR2 + per - 1) / per;
+    F.slice_roles.assign(F.S, {});
+    std::vector<double> load(F.S, 0.0);
+    for (int ri = 0; ri < NR2; ++ri) {
+      F.slice_roles[ri / per].push_back(ri);
+      load[ri / per] = std::max(load[ri / per], P.fwd_roles[ri].cost);
+    }
+    F.weight = load;
+  } else {
+    // up to 16 consumer warps per CTA; 8 when the roles are register-heavy
+    // (wide inputs), so that two CTAs of (8 + 2) warps keep 96 registers each
+    int kMaxWarps = 16;
+    for (auto& r : P.fwd_roles)
+      if (P.in[r.irrep].l >= 3 && NR > 8) kMaxWarps = 8;
+    F.S = (NR + kMaxWarps - 1) / kMaxWarps;
+    // longest-processing-time assignment of roles to slices
+    std::vector<int> order(NR);
+    std::iota(order.begin(), order.end(), 0);
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int a, int b) { return P.fwd_roles[a].cost > P.fwd_roles[b].cost; });
+    const int cap = (NR + F.S - 1) / F.S;
+    F.slice_roles.assign(F.S, {});
+    std::vector<double> load(F.S, 0.0);
+    for (int ri : order) {
+      int best = -1;
+      for (int s = 0; s < F.S; ++s)
+        if ((int)F.slice_roles[s].size() < cap && (best < 0 || load[s] < load[best])) best = s;
+      F.slice_roles[best].push_back(ri);
+      load[best] += P.fwd_roles[ri].cost;
+    }
+    for (auto& v : F.slice_roles) std::sort(v.begin(), v.end());
+    F.weight = load;
+  }
   F.nw = 0;
   for (auto& v : F.slice_roles) F.nw = std::max<int>(F.nw, (int)v.size());
   F.nacc = 1;

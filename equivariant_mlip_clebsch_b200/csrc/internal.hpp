@@ -86,6 +86,7 @@ struct FwdConfig {
   int stages = 3;        // ring depth
   bool w_smem = true;    // W rows staged by bulk copy (needs S == 1)
   bool x_smem = true;    // x blocks staged by bulk copy
+  bool generic = false;  // forward roles of one path, one function per (2l1+1, 2l3+1) shape
   int nacc = 0;          // accumulator registers per thread
   std::vector<std::vector<int>> slice_roles;  // role ids per slice
   std::vector<double> weight;                 // relative work per receiver of each slice
