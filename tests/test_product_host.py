@@ -124,3 +124,17 @@ def test_lmax_bound(compile_only):
     with pytest.raises(C.CgtpError) as e:
         C.Plan("4x3e", "1x0e+1x1o", "4x3e+4x2o+4x4o", 2)
     assert e.value.status == 5
+
+
+def test_force_chain_argument_errors(compile_only):
+    """cgtp_sph_harm_backward / cgtp_edge_forces validate before any launch."""
+    OK, NULL, SIZE = 0, 1, 6  # cgtp_status codes of include/cgtp.h
+    lib = C._lib
+    plan = C.Plan("16x0e+16x1o", "1x0e+1x1o", "32x0e+32x1o", 6)
+    assert lib.cgtp_sph_harm_backward(None, 1, None, None, None, None) == NULL
+    assert lib.cgtp_sph_harm_backward(plan._h, -1, None, None, None, None) == SIZE
+    assert lib.cgtp_sph_harm_backward(plan._h, 4, None, None, None, None) == NULL
+    assert lib.cgtp_sph_harm_backward(plan._h, 0, None, None, None, None) == OK  # nothing to do
+    assert lib.cgtp_edge_forces(-1, 0, None, None, None, None, None, None) == SIZE
+    assert lib.cgtp_edge_forces(0, 0, None, None, None, None, None, None) == OK
+    assert lib.cgtp_edge_forces(4, 8, None, None, None, None, None, None) == NULL
