@@ -9,16 +9,19 @@
 // and dx[j] = sum over the edges leaving j of msg[e] (a second, sender-major
 // pass over the transpose edge list, kernels.cu).
 //
-// Execution: grid (n_recv, S) with one slice per hidden irrep, so that every
-// consumer warp of a CTA runs the same role function (instruction-cache
-// friendly, and CTAs of one slice are scheduled together).  The TMA warp
-// stages the receiver's grad_out pieces once and then, per chunk, the W and x
-// pieces of the irrep; the helper warp stages Y, builds Chat and sums the dY
-// partials of released stages.  A consumer owns R channels of the irrep, ALL
-// its paths (so msg is complete in registers) and the edges b of each chunk
-// with b % nph == ph.  dW and msg go straight to global memory; dY partials
-// are reduced over lanes by shuffles, over the CTA's warps by the helper in a
-// fixed order, and over slices by a small kernel: bitwise reproducible.
+// Execution: persistent CTAs (resident CTAs per SM x SMs) walk the slices
+// in turn; a slice is a group of hidden irreps, chosen with the chunk size and
+// warp count by the planner (build_backward).  Within a slice the TMA warp
+// stages each receiver's grad_out pieces once and, per chunk, the W and x
+// pieces of the slice; the helper warp stages Y, builds Chat and sums the dY
+// partials of released stages.  A consumer owns R blocks of 32 channels of one
+// irrep (run one after another), ALL its paths (so msg is complete in
+// registers) and the edges b of each chunk with b % nph == ph.  Two variants
+// are compiled: CTAs over receivers blockIdx.x, + gridDim.x, ..., and CTAs
+// over equal edge ranges (for graphs with few receivers per CTA).  dW and msg
+// go straight to global memory; dY partials are reduced over lanes by
+// shuffles, over the CTA's warps by the helper in a fixed order, and over
+// slices by the closing reduction kernel: bitwise reproducible.
 #include <algorithm>
 #include <array>
 #include <cmath>

@@ -1,14 +1,15 @@
 // codegen_common.cpp -- staging layouts, the Chat tables and the two service
 // warps shared by the generated forward and backward kernels.
 //
-// Warp organisation of both kernels (one CTA = one receiver x one slice of
-// the warp roles):
+// Warp organisation of both kernels (persistent CTAs; each walks the slices
+// of the warp roles in turn, and in each its receivers or edge range):
 //   warps 0..NW-1  consumers: pure compute on staged data
 //   warp NW        TMA warp: per chunk of NB edges, bulk copies (cp.async.bulk,
 //                  completion counted in bytes on the stage's "full" mbarrier)
 //                  of the W and x row pieces the slice needs; pieces that are
 //                  not 16-byte aligned are copied with plain loads instead.
-//                  The backward's grad_out row pieces are staged once per CTA.
+//                  The backward's grad_out row pieces are staged once per
+//                  receiver and slice, into one of two buffers.
 //   warp NW+1      helper warp: loads the chunk's Y rows and builds
 //                  Chat_{e,p} = sum_m2 C_p[m1][m2][m3] Y[e][m2] into the stage;
 //                  in the backward it also sums the consumers' dY partials of

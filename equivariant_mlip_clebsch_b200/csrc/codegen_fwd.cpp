@@ -1,19 +1,21 @@
 // codegen_fwd.cpp -- the forward CGTP convolution kernel, generated per plan.
 //
 // Node-centric execution (LunaTP Fig. 3a: every receiver's row is
-// accumulated on chip and stored once, no atomics).  Grid (n_recv, S): CTA
-// (i, s) owns receiver i and slice s of the warp roles.  The TMA warp and the
-// helper warp (codegen_common.cpp) stream the receiver's edges in chunks of NB
-// through a ring of NSTAGE stages holding, per edge, the W and x pieces of the
-// slice, the Y row and Chat = C.Y for the slice's paths.  Each consumer warp
-// runs one role: R channels per lane of one hidden irrep and a group of that
-// irrep's paths, accumulating
+// accumulated on chip and stored once, no atomics).  Persistent CTAs walk the
+// slices of the warp roles in turn and, in each, the receivers blockIdx.x,
+// + gridDim.x, ...  The TMA warp and the helper warp (codegen_common.cpp)
+// stream a receiver's edges in chunks of NB through a ring of NSTAGE stages
+// holding, per edge, the W and x pieces of the slice, the Y row and
+// Chat = C.Y for the slice's paths.  Each consumer warp runs one role: R
+// channels per lane of one hidden irrep and a group of that irrep's paths,
+// accumulating
 //     acc[p][u][m3] += W[e][k0_p+u] * sum_m1 Chat[m3][m1] x[j][u][m1]
 // in registers.  x is read once per edge for all paths of the group (the
 // cross-path input reuse of LunaTP Table 8); the paths of an irrep are
 // grouped under a register budget per lane (LunaTP's output-component budget,
 // Fig. 3b / Table 7).  Roles with the same irrep and path group share one
-// __noinline__ function with the channel block as an argument.
+// __noinline__ function with the channel block as an argument.  Wide plans
+// use one-path roles instead, one function per (2l1+1, 2l3+1) shape.
 #include <algorithm>
 #include <array>
 #include <cmath>

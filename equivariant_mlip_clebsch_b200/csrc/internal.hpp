@@ -80,7 +80,7 @@ struct JitKernel {
 };
 
 struct FwdConfig {
-  int S = 1;             // slices (CTAs per receiver)
+  int S = 1;             // slices (each CTA walks them in turn)
   int nw = 0;            // consumer warps per CTA
   int B = 4;             // edges per chunk
   int stages = 3;        // ring depth
