@@ -84,7 +84,7 @@ struct FwdConfig {
   int nw = 0;            // consumer warps per CTA
   int B = 4;             // edges per chunk
   int stages = 3;        // ring depth
-  bool w_smem = true;    // W rows staged by bulk copy (needs S == 1)
+  bool w_smem = true;    // W row pieces staged by bulk copy (16-byte aligned)
   bool x_smem = true;    // x blocks staged by bulk copy
   bool generic = false;  // forward roles of one path, one function per (2l1+1, 2l3+1) shape
   int nacc = 0;          // accumulator registers per thread
