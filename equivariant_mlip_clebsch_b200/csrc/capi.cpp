@@ -38,7 +38,7 @@ void destroy_plan_device(Plan& P) {
   jit_unload(P.fwd);
   jit_unload(P.bwd);
   jit_unload(P.bwd_er);
-  for (void** p : {&P.d_fwd_ent, &P.d_fwd_term, &P.d_bwd_ent, &P.d_bwd_term}) {
+  for (void** p : {&P.d_fwd_ent, &P.d_bwd_ent}) {
     if (*p) cudaFree(*p);
     *p = nullptr;
   }

@@ -583,7 +583,6 @@ cgtp_status build_backward(Plan& P) {
   K.nw = F.nw;
   K.force_B = best.B;
   for (int s2 = 0; s2 < F.S; ++s2) {
-    double wsum = 0.0;
     for (size_t k = 0; k < best.slices[s2].size(); ++k) {
       const BwdIrrep& wi = best.W[best.slices[s2][k]];
       const BwdOption& o = wi.opts[best.pick[s2][k]];
@@ -601,7 +600,6 @@ cgtp_status build_backward(Plan& P) {
           F.slice_roles[s2].push_back((int)P.bwd_roles.size());
           P.bwd_roles.push_back(r);
         }
-      wsum += o.cost * o.roles;
       SL[s2].irreps.push_back(wi.a);
       for (size_t q = 0; q < P.paths.size(); ++q)
         if (P.paths[q].irrep == wi.a) SL[s2].paths.push_back((int)q);
@@ -609,7 +607,6 @@ cgtp_status build_backward(Plan& P) {
     }
     std::sort(SL[s2].paths.begin(), SL[s2].paths.end());
     layout_slice(P, SL[s2], true);
-    F.weight.push_back(wsum);
   }
   plan_layout(P, SL, K, true);
   F.B = K.B;
@@ -617,7 +614,7 @@ cgtp_status build_backward(Plan& P) {
   F.w_smem = K.w_bulk;
   F.x_smem = K.x_bulk;
 
-  cgtp_status st = upload_chat_tables(P, SL, &P.d_bwd_ent, &P.d_bwd_term, P.bwd_ent_begin);
+  cgtp_status st = upload_chat_tables(P, SL, &P.d_bwd_ent, P.bwd_ent_begin);
   if (st != CGTP_OK) return st;
   for (size_t k = 0; k + 1 < P.bwd_ent_begin.size(); ++k)
     K.rec_max = std::max(K.rec_max, P.bwd_ent_begin[k + 1] - P.bwd_ent_begin[k]);

@@ -445,7 +445,7 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
 //   y = coefficient of Y[y0], z = coefficient of Y[y1] (FP32 bits), w = 0.
 // Elements with no term stay zero: the helper clears the Chat buffers once.
 cgtp_status upload_chat_tables(const Plan& P, const std::vector<SliceLayout>& SL, void** d_ent,
-                               void** d_term, std::vector<int>& ent_begin) {
+                               std::vector<int>& ent_begin) {
   std::vector<int> rec;
   ent_begin.assign(1, 0);
   for (const SliceLayout& sl : SL) {
@@ -481,7 +481,6 @@ cgtp_status upload_chat_tables(const Plan& P, const std::vector<SliceLayout>& SL
     }
     ent_begin.push_back((int)rec.size() / 4);
   }
-  *d_term = nullptr;
   if (P.host_only) return CGTP_OK;
   if (rec.empty()) rec.assign(4, 0);
   if (cudaMalloc(d_ent, rec.size() * sizeof(int)) != cudaSuccess)

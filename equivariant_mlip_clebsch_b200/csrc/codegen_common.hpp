@@ -88,7 +88,9 @@ int max_spill_bytes(const std::string& log);
 // point of the register cap; CGTP_MIN_BLOCKS overrides it.
 int initial_min_blocks(int smem_bytes, bool* fixed);
 
+// The Chat records of every slice (16 bytes each: target | y index a |
+// y index b, c_a, c_b) uploaded to the device; ent_begin[s] is slice s's first.
 cgtp_status upload_chat_tables(const Plan& P, const std::vector<SliceLayout>& SL, void** d_ent,
-                               void** d_term, std::vector<int>& ent_begin);
+                               std::vector<int>& ent_begin);
 
 }  // namespace cgtp

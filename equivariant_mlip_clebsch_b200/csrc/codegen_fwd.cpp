@@ -368,12 +368,7 @@ cgtp_status build_forward(Plan& P) {
     const int per = 8;
     F.S = (NR2 + per - 1) / per;
     F.slice_roles.assign(F.S, {});
-    std::vector<double> load(F.S, 0.0);
-    for (int ri = 0; ri < NR2; ++ri) {
-      F.slice_roles[ri / per].push_back(ri);
-      load[ri / per] = std::max(load[ri / per], P.fwd_roles[ri].cost);
-    }
-    F.weight = load;
+    for (int ri = 0; ri < NR2; ++ri) F.slice_roles[ri / per].push_back(ri);
   } else {
     // up to 16 consumer warps per CTA; 8 when the roles are register-heavy
     // (wide inputs), so that two CTAs of (8 + 2) warps keep 96 registers each
@@ -397,7 +392,6 @@ cgtp_status build_forward(Plan& P) {
       load[best] += P.fwd_roles[ri].cost;
     }
     for (auto& v : F.slice_roles) std::sort(v.begin(), v.end());
-    F.weight = load;
   }
   F.nw = 0;
   for (auto& v : F.slice_roles) F.nw = std::max<int>(F.nw, (int)v.size());
@@ -430,7 +424,7 @@ cgtp_status build_forward(Plan& P) {
   F.w_smem = K.w_bulk;
   F.x_smem = K.x_bulk;
 
-  cgtp_status st = upload_chat_tables(P, SL, &P.d_fwd_ent, &P.d_fwd_term, P.fwd_ent_begin);
+  cgtp_status st = upload_chat_tables(P, SL, &P.d_fwd_ent, P.fwd_ent_begin);
   if (st != CGTP_OK) return st;
   for (size_t k = 0; k + 1 < P.fwd_ent_begin.size(); ++k)
     K.rec_max = std::max(K.rec_max, P.fwd_ent_begin[k + 1] - P.fwd_ent_begin[k]);

@@ -89,7 +89,6 @@ struct FwdConfig {
   bool generic = false;  // forward roles of one path, one function per (2l1+1, 2l3+1) shape
   int nacc = 0;          // accumulator registers per thread
   std::vector<std::vector<int>> slice_roles;  // role ids per slice
-  std::vector<double> weight;                 // relative work per receiver of each slice
 };
 
 struct Plan {
@@ -109,7 +108,6 @@ struct Plan {
   JitKernel fwd;
   // Chat build tables per slice (device): entry -> (dst offset, term begin, term count)
   void* d_fwd_ent = nullptr;   // int4 [n]
-  void* d_fwd_term = nullptr;  // int2 [n] (y index, coeff bits)
   std::vector<int> fwd_ent_begin;  // per slice, into d_fwd_ent (size S+1)
   std::vector<int> fwd_chs;        // Chat floats per edge per slice
 
@@ -119,7 +117,6 @@ struct Plan {
   JitKernel bwd;     // CTAs walk receivers blockIdx.x, + gridDim.x, ...
   JitKernel bwd_er;  // CTAs take equal edge ranges (for few receivers per CTA)
   void* d_bwd_ent = nullptr;
-  void* d_bwd_term = nullptr;
   std::vector<int> bwd_ent_begin;
   std::vector<int> bwd_chs;
   bool bwd_irrep_gap = false;  // some hidden irrep has no path
