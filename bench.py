@@ -306,12 +306,33 @@ def run_cgtp(args, rank, world, local_rank):
         plan.sph_harm_backward(T["r"], dY, grad_r=gr)
         C.edge_forces(T["rowptr"], T["rpt"], T["perm"], gr, forces=Fo)
         b.record(stream)
+    # the strain derivative (virial) from the same grad_r, timed on its own
+    Vo = torch.empty((3, 3), device=dev)
+    ev_v = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    virial_err = None
+    try:
+        for k in range(args.steps):
+            flush.zero_()
+            a, b = ev_v[k]
+            a.record(stream)
+            C.edge_virial(T["r"], gr, virial=Vo)
+            b.record(stream)
+    except C.CgtpError as e:
+        virial_err = str(e)
     torch.cuda.synchronize()
     clocks = sampler.stop()
     plan.check_device_error()
     ms_steps = [a.elapsed_time(b) for a, b in ev]
     ms_fwd = [a.elapsed_time(b) for a, b in ev_f]
     force_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_c]))
+    if virial_err is None:
+        virial_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_v]))
+        virial = {"ms": virial_ms, "edges_per_s": world * E / (virial_ms * 1e-3),
+                  "achieved_gbs": 24.0 * E / (virial_ms * 1e-3) / 1e9,
+                  "what": "edge_virial from grad_r (24 B/edge read), after the step (not in it)"}
+    else:
+        virial = {"error": virial_err}
     ms_step = max_over_ranks(float(np.sum(ms_steps)) / args.steps, world, dev)
     value = replica_value(world, E, ms_step)
     fwd_ms = float(np.mean(ms_fwd))
@@ -370,6 +391,7 @@ def run_cgtp(args, rank, world, local_rank):
                ms_per_step_launched=ms_eager,
                force_chain={"ms": force_ms, "edges_per_s": world * E / (force_ms * 1e-3),
                             "what": "sph_harm_backward + edge_forces after the step (not in it)"},
+               virial=virial,
                roofline=roof, kernels=kernels, gpu_launches=int(gpu_launches), e2e=e2e, clocks=clocks)
     return res
 

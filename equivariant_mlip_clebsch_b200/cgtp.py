@@ -39,6 +39,7 @@ _SIGS = {
     "cgtp_sph_harm": (_i, [_P, _i64, _P, _P, _P]),
     "cgtp_sph_harm_backward": (_i, [_P, _i64, _P, _P, _P, _P]),
     "cgtp_edge_forces": (_i, [_i64, _i64, _P, _P, _P, _P, _P, _P]),
+    "cgtp_edge_virial": (_i, [_i64, _P, _P, _P, _P]),
     "cgtp_forward": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P, _P, _P]),
     "cgtp_backward_workspace_size": (_i, [_P, _i64, _i64, _i64, ctypes.POINTER(_sz)]),
     "cgtp_backward": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -124,6 +125,19 @@ def edge_forces(rowptr, rowptr_T, perm_T, grad_r, forces=None, stream=None):
     _check(_lib.cgtp_edge_forces(n_atoms, E, _tptr(rowptr), _tptr(rowptr_T), _tptr(perm_T), _tptr(grad_r),
                                  _tptr(forces), _stream(stream)))
     return forces
+
+
+def edge_virial(r, grad_r, virial=None, stream=None):
+    """cgtp_edge_virial: the strain derivative V [3,3], V[a,b] = sum_e
+    grad_r[e,a] r[e,b] (device tensors; stress = V / cell volume)."""
+    import torch
+    E = r.shape[0]
+    if grad_r.shape[0] != E:
+        raise ValueError("r and grad_r have different edge counts")
+    if virial is None:
+        virial = torch.empty((3, 3), dtype=torch.float32, device=r.device)
+    _check(_lib.cgtp_edge_virial(E, _tptr(r), _tptr(grad_r), _tptr(virial), _stream(stream)))
+    return virial
 
 
 def csr_transpose(rowptr, col, n_send: int):

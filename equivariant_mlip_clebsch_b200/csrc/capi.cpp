@@ -270,6 +270,16 @@ cgtp_status cgtp_edge_forces(int64_t n_atoms, int64_t E, const int32_t* rowptr, 
   return CGTP_OK;
 }
 
+cgtp_status cgtp_edge_virial(int64_t E, const float* r, const float* grad_r, float* virial, cgtp_stream stream) {
+  if (E < 0 || E >= (int64_t(1) << 31)) return fail(CGTP_ERR_SIZE, "E out of range");
+  if (!virial) return fail(CGTP_ERR_NULL, "virial is NULL");
+  if (E > 0 && (!r || !grad_r)) return fail(CGTP_ERR_NULL, "r or grad_r is NULL");
+  if (E > 0 && (!aligned16(r) || !aligned16(grad_r)))
+    return fail(CGTP_ERR_ALIGN, "r and grad_r must be 16-byte aligned");
+  CGTP_CUDA_TRY(launch_edge_virial(E, r, grad_r, virial, (cudaStream_t)stream));
+  return CGTP_OK;
+}
+
 cgtp_status cgtp_forward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
                          const int32_t* rowptr, const int32_t* col, const float* x, const float* Y,
                          const float* W, float* out, cgtp_stream stream) {

@@ -1,6 +1,9 @@
 // kernels.cu -- the kernels that do not depend on the path structure:
-// real spherical harmonics of the edge vectors, and the deterministic closing
-// reductions of the backward (sender-major row sums, slice sums) in one launch.
+// real spherical harmonics of the edge vectors and their gradient, the force
+// and strain-derivative (virial) assembly from the edge-vector gradient, and
+// the deterministic closing reductions of the backward (sender-major row sums,
+// slice sums) in one launch.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -233,6 +236,78 @@ __global__ void __launch_bounds__(128) edge_forces_kernel(int64_t n_atoms, const
   F[3 * a + 2] = fz - sz;
 }
 
+// Strain derivative of the loss from the edge-vector gradient:
+//   V[3a+b] = sum_e G[e][a] r[e][b]      (= dL/d eps_ab for r_e -> (1 + eps) r_e).
+// One cluster of kVirCtas CTAs.  Thread t of the cluster takes the groups of
+// four edges t, t + kVirCtas*kVirThreads, ... (three float4 loads per array and
+// group: 48 bytes, 16-byte aligned when r and G are), and the last E % 4 edges
+// one each; products and sums are in FP64.  Each CTA sums its warps in warp
+// order, then CTA 0 adds the CTAs' sums in rank order through distributed
+// shared memory, so the result depends on E only (no atomics).
+constexpr int kVirCtas = 8;
+constexpr int kVirThreads = 512;
+
+__global__ void __cluster_dims__(kVirCtas, 1, 1) __launch_bounds__(kVirThreads)
+    edge_virial_kernel(int64_t E, const float* __restrict__ r, const float* __restrict__ G, float* __restrict__ V) {
+  namespace cg = cooperative_groups;
+  grid_dependency_wait();
+  grid_launch_dependents();
+  __shared__ double warp_sum[kVirThreads / 32][9];
+  __shared__ double cta_sum[9];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int64_t t = (int64_t)cluster.block_rank() * kVirThreads + threadIdx.x;
+  constexpr int64_t kStride = (int64_t)kVirCtas * kVirThreads;
+  double acc[9];
+#pragma unroll
+  for (int k = 0; k < 9; ++k) acc[k] = 0.0;
+  const int64_t groups = E / 4;
+  for (int64_t q = t; q < groups; q += kStride) {
+    float rf[12], gf[12];
+    const float4* r4 = reinterpret_cast<const float4*>(r + 12 * q);
+    const float4* g4 = reinterpret_cast<const float4*>(G + 12 * q);
+#pragma unroll
+    for (int v = 0; v < 3; ++v) {
+      const float4 a = __ldg(r4 + v), b = __ldg(g4 + v);
+      rf[4 * v] = a.x, rf[4 * v + 1] = a.y, rf[4 * v + 2] = a.z, rf[4 * v + 3] = a.w;
+      gf[4 * v] = b.x, gf[4 * v + 1] = b.y, gf[4 * v + 2] = b.z, gf[4 * v + 3] = b.w;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int a = 0; a < 3; ++a)
+#pragma unroll
+        for (int b = 0; b < 3; ++b) acc[3 * a + b] += (double)gf[3 * k + a] * (double)rf[3 * k + b];
+  }
+  if (t < E - 4 * groups) {
+    const int64_t e = 4 * groups + t;
+#pragma unroll
+    for (int a = 0; a < 3; ++a)
+#pragma unroll
+      for (int b = 0; b < 3; ++b) acc[3 * a + b] += (double)G[3 * e + a] * (double)r[3 * e + b];
+  }
+#pragma unroll
+  for (int k = 0; k < 9; ++k)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], off);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0)
+#pragma unroll
+    for (int k = 0; k < 9; ++k) warp_sum[warp][k] = acc[k];
+  __syncthreads();
+  if (threadIdx.x < 9) {
+    double s = 0.0;
+    for (int w = 0; w < kVirThreads / 32; ++w) s += warp_sum[w][threadIdx.x];
+    cta_sum[threadIdx.x] = s;
+  }
+  cluster.sync();  // every CTA's cta_sum is written
+  if (cluster.block_rank() == 0 && threadIdx.x < 9) {
+    double s = 0.0;
+    for (unsigned q = 0; q < (unsigned)kVirCtas; ++q) s += cluster.map_shared_rank(cta_sum, q)[threadIdx.x];
+    V[threadIdx.x] = (float)s;
+  }
+  cluster.sync();  // no CTA leaves (and frees its shared memory) before CTA 0 has read it
+}
+
 // The backward's closing reductions in one launch.
 //  blocks [0, n_send): dx[j][c] = sum over sender j's edges of m[perm_T[t]][c].
 //    Two groups of 128 threads take the even and the odd positions t0 + 2k of
@@ -369,6 +444,10 @@ cudaError_t launch_edge_forces(int64_t n_atoms, const int32_t* rowptr, const int
   if (n_atoms == 0) return cudaSuccess;
   return launch_pdl(edge_forces_kernel, dim3((unsigned)((n_atoms + 127) / 128)), 128, s, n_atoms, rowptr, rowptr_T,
                     perm_T, G, F);
+}
+
+cudaError_t launch_edge_virial(int64_t E, const float* r, const float* G, float* V, cudaStream_t s) {
+  return launch_pdl(edge_virial_kernel, dim3(kVirCtas), kVirThreads, s, E, r, G, V);
 }
 
 cudaError_t launch_bwd_reduce(int64_t n_send, int64_t width, const int32_t* rowptr_T, const int32_t* perm_T,

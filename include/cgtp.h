@@ -147,6 +147,21 @@ cgtp_status cgtp_edge_forces(int64_t n_atoms, int64_t E, const int32_t* rowptr, 
                              const int32_t* perm_T, const float* grad_r, float* forces,
                              cgtp_stream stream);
 
+/* Strain derivative of the loss (the virial), for stresses, from the same
+ * edge-vector gradient as cgtp_edge_forces:
+ *   virial[3a+b] = sum_e grad_r[e][a] r[e][b]   (a, b = x, y, z)
+ * which is dL/d eps_ab when every edge vector (and so the cell) is strained
+ * as r_e -> (1 + eps) r_e; the stress is virial / cell volume.  The pages
+ * name stresses beside forces as derivatives of the energy (BranchIP page,
+ * its MLIP background) but print no formula: this is the chain rule through
+ * the edge vectors, the same reading as the forces.
+ * r, grad_r [E,3] FP32 device, 16-byte aligned; virial [9] FP32 device,
+ * overwritten (zeros for E = 0).  Products and sums in FP64, in an order fixed
+ * by E (bitwise reproducible, no atomics).  Needs no plan.
+ * Errors: SIZE (E < 0 or E >= 2^31), NULL, ALIGN, CUDA. */
+cgtp_status cgtp_edge_virial(int64_t E, const float* r, const float* grad_r, float* virial,
+                             cgtp_stream stream);
+
 /* Forward CGTP convolution (the x' of LunaTP Table 11), formula above.
  *   n_recv receivers, n_send senders, E edges (0 <= E < 2^31)
  *   rowptr [n_recv+1], col [E] (int32, device); x [n_send, d_in];

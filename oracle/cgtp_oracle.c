@@ -17,8 +17,9 @@
  *   - a brute-force periodic neighbour search over all atom pairs and images,
  *   - the forward and backward CGTP convolution as nested sums,
  *   - the gradient of the harmonics with respect to the edge vector (forward-
- *     mode differentiation of the harmonics above) and the force assembly
- *     from it (the step after the backward: forces = -dE/dpos).
+ *     mode differentiation of the harmonics above), and the force and
+ *     strain-derivative (virial) assembly from it (the steps after the
+ *     backward: forces = -dE/dpos, stress = dE/d strain / volume).
  *
  * Source of the operation: LunaTP (arXiv 2610.18393), Abstract (the CGTP
  * convolution), Table 1 (irreps configurations and hence the path set) and
@@ -345,6 +346,20 @@ void orc_edge_forces(int64_t n_atoms, const int64_t* rowptr, const int32_t* col,
       for (int k = 0; k < 3; ++k) {
         F[3 * i + k] += G[3 * e + k];
         F[3 * (int64_t)col[e] + k] -= (g_fault == 4 ? -1.0 : 1.0) * G[3 * e + k]; /* 4: sign mutation */
+      }
+}
+
+/* Strain derivative of the loss from G = dL/dr [E][3]: straining every
+ * edge vector (and with it the cell) as r_e -> (1 + eps) r_e gives
+ *   V[3a+b] = dL/d eps_ab = sum_e G[e][a] r[e][b].
+ * The stress is V / volume.  Chain rule through the edge vectors, plain loop. */
+void orc_edge_virial(int64_t E, const double* r, const double* G, double* V) {
+  for (int k = 0; k < 9; ++k) V[k] = 0.0;
+  for (int64_t e = 0; e < E; ++e)
+    for (int a = 0; a < 3; ++a)
+      for (int b = 0; b < 3; ++b) {
+        int k = g_fault == 5 ? 3 * b + a : 3 * a + b; /* 5: transposed mutation */
+        V[k] += G[3 * e + a] * r[3 * e + b];
       }
 }
 

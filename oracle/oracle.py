@@ -65,6 +65,8 @@ def lib():
         L.orc_sph_harm_grad.argtypes = [i, i64, P, P]
         L.orc_edge_forces.restype = None
         L.orc_edge_forces.argtypes = [i64, P, P, P, P]
+        L.orc_edge_virial.restype = None
+        L.orc_edge_virial.argtypes = [i64, P, P, P]
         L.orc_neighbor_list.restype = i64
         L.orc_neighbor_list.argtypes = [i64, P, P, d, P, P, P, P]
         L.orc_forward.restype = None
@@ -234,6 +236,18 @@ def edge_forces(n_atoms: int, rowptr, col, G) -> np.ndarray:
     F = np.zeros((n_atoms, 3), dtype=np.float64)
     lib().orc_edge_forces(int(n_atoms), _ptr(rowptr), _ptr(col), _ptr(G), _ptr(F))
     return F
+
+
+def edge_virial(r, G) -> np.ndarray:
+    """V [3,3] = dL/d strain = sum_e G[e] (outer) r[e], with G = dL/dr per edge
+    and every edge vector strained as r -> (1 + eps) r."""
+    r = np.ascontiguousarray(r, dtype=np.float64).reshape(-1, 3)
+    G = np.ascontiguousarray(G, dtype=np.float64).reshape(-1, 3)
+    if r.shape != G.shape:
+        raise ValueError("r and G have different edge counts")
+    V = np.zeros((3, 3), dtype=np.float64)
+    lib().orc_edge_virial(r.shape[0], _ptr(r), _ptr(G), _ptr(V))
+    return V
 
 
 # ---------------------------------------------------------------------------

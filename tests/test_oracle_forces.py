@@ -11,8 +11,11 @@ harmonics; these tests pin it to things other than itself:
   * rotation: dY/dr(R r) = D(R) dY/dr(r) R^T,
   * forces: they sum to zero, and equal minus the finite-difference position
     gradient of an energy built from the harmonics on a periodic cell,
+  * the virial (strain derivative): it equals the finite-difference strain
+    derivative of such an energy (with a radial factor, so the isotropic part
+    counts), and its trace vanishes for an energy of the directions alone,
   * planted mistakes (the phi term dropped, a sign flipped in the force
-    assembly) fail these pins.
+    assembly, the virial transposed) fail these pins.
 """
 import numpy as np
 import pytest
@@ -144,3 +147,56 @@ def test_pins_catch_planted_mistakes():
     assert np.abs(fd - J[:, :, 0]).max() > 1e-3
     F, got, fd = _cell_energy_and_forces(fault=4)  # sign of the sender term flipped
     assert np.abs(got - fd).max() > 1e-3
+
+
+def _strained_energy_and_virial(seed=0, L=3, h=1e-6, fault=0):
+    """E(eps) = sum_e |r_e|^2 sum_m c[e,m] Y_m(r_e) over the tiny Si cell's
+    edges with every edge vector strained, r_e -> (1 + eps) r_e (edge list and
+    images held fixed).  Returns the oracle's virial of G = dE/dr and the
+    central differences of E over the nine strain components."""
+    c = WL.CONFIGS["tiny"]
+    pos, box = WL.si_diamond(c["cells"], c["sigma"], seed)
+    _, col, _, vec = O.neighbor_list(pos, box, c["rc"])
+    coef = np.random.default_rng(seed + 9).standard_normal((len(col), (L + 1) ** 2))
+
+    def energy(eps):
+        r = vec @ (np.eye(3) + eps).T
+        return float(((r * r).sum(1)[:, None] * coef * O.sph_harm(L, r)).sum())
+
+    # dE/dr_e = |r|^2 sum_m c dY_m/dr + 2 r sum_m c Y_m (product rule)
+    s = (coef * O.sph_harm(L, vec)).sum(1)
+    G = (vec * vec).sum(1)[:, None] * O.sph_harm_backward(L, vec, coef) + 2.0 * vec * s[:, None]
+    try:
+        O.set_fault(fault)
+        V = O.edge_virial(vec, G)
+    finally:
+        O.set_fault(0)
+    fd = np.zeros((3, 3))
+    for a in range(3):
+        for b in range(3):
+            d = np.zeros((3, 3))
+            d[a, b] = h
+            fd[a, b] = (energy(d) - energy(-d)) / (2 * h)
+    return V, fd
+
+
+def test_virial_against_strain_differences():
+    V, fd = _strained_energy_and_virial()
+    assert np.abs(V - V.T).max() > 1e-2 * np.abs(V).max()  # asymmetric: a transposition shows
+    assert abs(np.trace(V)) > 1e-2 * np.abs(V).max()      # the isotropic part is exercised
+    assert np.abs(V - fd).max() < 1e-6 * np.abs(fd).max()
+
+
+def test_virial_trace_vanishes_for_directions_only():
+    """Y depends on the direction alone, so a uniform dilation leaves an
+    energy of the harmonics unchanged: sum_e G_e . r_e = trace V = 0."""
+    r = _vectors(200, 41)
+    coef = np.random.default_rng(42).standard_normal((200, 16))
+    V = O.edge_virial(r, O.sph_harm_backward(3, r, coef))
+    assert abs(np.trace(V)) < 1e-12 * np.abs(V).sum()
+    assert np.abs(V).max() > 1.0
+
+
+def test_virial_pin_catches_transposition():
+    V, fd = _strained_energy_and_virial(fault=5)
+    assert np.abs(V - fd).max() > 1e-2 * np.abs(fd).max()

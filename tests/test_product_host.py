@@ -9,6 +9,7 @@
   * every workload's plan builds and its kernels compile for sm_100a (the
     compile-only mode skips all device work), with the oracle's path table.
 """
+import ctypes
 import os
 import re
 
@@ -127,8 +128,9 @@ def test_lmax_bound(compile_only):
 
 
 def test_force_chain_argument_errors(compile_only):
-    """cgtp_sph_harm_backward / cgtp_edge_forces validate before any launch."""
-    OK, NULL, SIZE = 0, 1, 6  # cgtp_status codes of include/cgtp.h
+    """cgtp_sph_harm_backward / cgtp_edge_forces / cgtp_edge_virial validate
+    before any launch."""
+    OK, NULL, ALIGN, SIZE = 0, 1, 2, 6  # cgtp_status codes of include/cgtp.h
     lib = C._lib
     plan = C.Plan("16x0e+16x1o", "1x0e+1x1o", "32x0e+32x1o", 6)
     assert lib.cgtp_sph_harm_backward(None, 1, None, None, None, None) == NULL
@@ -138,3 +140,11 @@ def test_force_chain_argument_errors(compile_only):
     assert lib.cgtp_edge_forces(-1, 0, None, None, None, None, None, None) == SIZE
     assert lib.cgtp_edge_forces(0, 0, None, None, None, None, None, None) == OK
     assert lib.cgtp_edge_forces(4, 8, None, None, None, None, None, None) == NULL
+    p16, p4 = ctypes.c_void_p(16), ctypes.c_void_p(4)  # never dereferenced: refused first
+    assert lib.cgtp_edge_virial(-1, None, None, p16, None) == SIZE
+    assert lib.cgtp_edge_virial(1 << 31, p16, p16, p16, None) == SIZE
+    assert lib.cgtp_edge_virial(4, p16, p16, None, None) == NULL
+    assert lib.cgtp_edge_virial(4, None, p16, p16, None) == NULL
+    assert lib.cgtp_edge_virial(4, p16, None, p16, None) == NULL
+    assert lib.cgtp_edge_virial(4, p4, p16, p16, None) == ALIGN
+    assert lib.cgtp_edge_virial(4, p16, p4, p16, None) == ALIGN
