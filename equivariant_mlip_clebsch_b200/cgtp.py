@@ -76,13 +76,38 @@ def _np_ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
-def _tptr(t):
-    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
-    if t is None:
-        return None
+def _require_device(t, name, dev):
     if not t.is_cuda or not t.is_contiguous():
-        raise ValueError("expected a contiguous CUDA tensor")
-    return ctypes.c_void_p(t.data_ptr())
+        raise ValueError(f"{name}: expected a contiguous CUDA tensor")
+    if dev is not None and t.device != dev:
+        raise ValueError(f"{name}: on {t.device}, the other arguments on {dev}")
+
+
+def _args(dev, *specs):
+    """Device pointers of tensor arguments, each spec (tensor, name, count,
+    kind), after the checks that keep the kernels' flat indexing inside
+    them: first dtype (kind "f32" or "i32") and exactly `count` elements for
+    every argument, then a contiguous CUDA tensor on `dev`.  None passes as
+    NULL (the library then reports a required argument as CGTP_ERR_NULL)."""
+    import torch
+    for t, name, count, kind in specs:
+        if t is None:
+            continue
+        want = torch.float32 if kind == "f32" else torch.int32
+        if t.dtype != want:
+            raise TypeError(f"{name}: expected {want}, got {t.dtype}")
+        if t.numel() != count:
+            raise ValueError(f"{name}: expected {count} elements, got shape {tuple(t.shape)}")
+    for t, name, _, _ in specs:
+        if t is not None:
+            _require_device(t, name, dev)
+    return [None if t is None else ctypes.c_void_p(t.data_ptr()) for t, _, _, _ in specs]
+
+
+def _workspace(t, dev):
+    """Pointer and byte size of a caller workspace (any dtype)."""
+    _require_device(t, "workspace", dev)
+    return ctypes.c_void_p(t.data_ptr()), t.numel() * t.element_size()
 
 
 def _stream(stream=None):
@@ -119,11 +144,13 @@ def edge_forces(rowptr, rowptr_T, perm_T, grad_r, forces=None, stream=None):
     """cgtp_edge_forces: forces [N,3] = -dL/dpos from grad_r [E,3] (device
     tensors; r_e = pos_sender - pos_receiver + shift)."""
     import torch
-    n_atoms, E = rowptr.shape[0] - 1, grad_r.shape[0]
+    n_atoms, E, dev = rowptr.shape[0] - 1, grad_r.shape[0], grad_r.device
     if forces is None:
-        forces = torch.empty((n_atoms, 3), dtype=torch.float32, device=grad_r.device)
-    _check(_lib.cgtp_edge_forces(n_atoms, E, _tptr(rowptr), _tptr(rowptr_T), _tptr(perm_T), _tptr(grad_r),
-                                 _tptr(forces), _stream(stream)))
+        forces = torch.empty((n_atoms, 3), dtype=torch.float32, device=dev)
+    ptrs = _args(dev, (rowptr, "rowptr", n_atoms + 1, "i32"), (rowptr_T, "rowptr_T", n_atoms + 1, "i32"),
+                 (perm_T, "perm_T", E, "i32"), (grad_r, "grad_r", 3 * E, "f32"),
+                 (forces, "forces", 3 * n_atoms, "f32"))
+    _check(_lib.cgtp_edge_forces(n_atoms, E, *ptrs, _stream(stream)))
     return forces
 
 
@@ -131,12 +158,11 @@ def edge_virial(r, grad_r, virial=None, stream=None):
     """cgtp_edge_virial: the strain derivative V [3,3], V[a,b] = sum_e
     grad_r[e,a] r[e,b] (device tensors; stress = V / cell volume)."""
     import torch
-    E = r.shape[0]
-    if grad_r.shape[0] != E:
-        raise ValueError("r and grad_r have different edge counts")
+    E, dev = r.shape[0], r.device
     if virial is None:
-        virial = torch.empty((3, 3), dtype=torch.float32, device=r.device)
-    _check(_lib.cgtp_edge_virial(E, _tptr(r), _tptr(grad_r), _tptr(virial), _stream(stream)))
+        virial = torch.empty((3, 3), dtype=torch.float32, device=dev)
+    ptrs = _args(dev, (r, "r", 3 * E, "f32"), (grad_r, "grad_r", 3 * E, "f32"), (virial, "virial", 9, "f32"))
+    _check(_lib.cgtp_edge_virial(E, *ptrs, _stream(stream)))
     return virial
 
 
@@ -232,31 +258,43 @@ class Plan:
     # ---- device calls
     def sph_harm(self, r, Y=None, stream=None):
         import torch
-        E = r.shape[0]
+        E, dev = r.shape[0], r.device
         if Y is None:
-            Y = torch.empty((E, self.d_edge), dtype=torch.float32, device=r.device)
-        _check(_lib.cgtp_sph_harm(self._h, E, _tptr(r), _tptr(Y), _stream(stream)))
+            Y = torch.empty((E, self.d_edge), dtype=torch.float32, device=dev)
+        ptrs = _args(dev, (r, "r", 3 * E, "f32"), (Y, "Y", E * self.d_edge, "f32"))
+        _check(_lib.cgtp_sph_harm(self._h, E, *ptrs, _stream(stream)))
         return Y
 
     def sph_harm_backward(self, r, grad_Y, grad_r=None, stream=None):
         """cgtp_sph_harm_backward: grad_r [E,3] = sum_t grad_Y[:, t] dY_t/dr."""
         import torch
-        E = r.shape[0]
+        E, dev = r.shape[0], r.device
         if grad_r is None:
-            grad_r = torch.empty((E, 3), dtype=torch.float32, device=r.device)
-        _check(_lib.cgtp_sph_harm_backward(self._h, E, _tptr(r), _tptr(grad_Y), _tptr(grad_r),
-                                           _stream(stream)))
+            grad_r = torch.empty((E, 3), dtype=torch.float32, device=dev)
+        ptrs = _args(dev, (r, "r", 3 * E, "f32"), (grad_Y, "grad_Y", E * self.d_edge, "f32"),
+                     (grad_r, "grad_r", 3 * E, "f32"))
+        _check(_lib.cgtp_sph_harm_backward(self._h, E, *ptrs, _stream(stream)))
         return grad_r
 
     def forward(self, rowptr, col, x, Y, W, out=None, stream=None):
         import torch
-        n_recv = rowptr.shape[0] - 1
+        n_recv, n_send, E, dev = rowptr.shape[0] - 1, x.shape[0], col.shape[0], x.device
         if out is None:
-            out = torch.empty((n_recv, self.d_out), dtype=torch.float32, device=x.device)
-        _check(_lib.cgtp_forward(self._h, n_recv, x.shape[0], col.shape[0], _tptr(rowptr),
-                                 _tptr(col), _tptr(x), _tptr(Y), _tptr(W), _tptr(out),
-                                 _stream(stream)))
+            out = torch.empty((n_recv, self.d_out), dtype=torch.float32, device=dev)
+        ptrs = _args(dev, (rowptr, "rowptr", n_recv + 1, "i32"), (col, "col", E, "i32"),
+                     (x, "x", n_send * self.d_in, "f32"), (Y, "Y", E * self.d_edge, "f32"),
+                     (W, "W", E * self.n_weights, "f32"), (out, "out", n_recv * self.d_out, "f32"))
+        _check(_lib.cgtp_forward(self._h, n_recv, n_send, E, *ptrs, _stream(stream)))
         return out
+
+    def _backward_args(self, rowptr, col, rowptr_T, perm_T, x, Y, W, grad_out, dx, dW, dY, dev,
+                       n_recv, n_send, E):
+        return _args(dev, (rowptr, "rowptr", n_recv + 1, "i32"), (col, "col", E, "i32"),
+                     (rowptr_T, "rowptr_T", n_send + 1, "i32"), (perm_T, "perm_T", E, "i32"),
+                     (x, "x", n_send * self.d_in, "f32"), (Y, "Y", E * self.d_edge, "f32"),
+                     (W, "W", E * self.n_weights, "f32"), (grad_out, "grad_out", n_recv * self.d_out, "f32"),
+                     (dx, "grad_x", n_send * self.d_in, "f32"), (dW, "grad_W", E * self.n_weights, "f32"),
+                     (dY, "grad_Y", E * self.d_edge, "f32"))
 
     def workspace_size(self, n_recv: int, n_send: int, E: int) -> int:
         b = ctypes.c_size_t()
@@ -274,13 +312,13 @@ class Plan:
             dY = torch.empty((E, self.d_edge), dtype=torch.float32, device=dev) if "Y" in want else None
         else:
             dx, dW, dY = grads
-        nbytes = self.workspace_size(n_recv, n_send, E)
         if workspace is None:
+            nbytes = self.workspace_size(n_recv, n_send, E)
             workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
-        _check(_lib.cgtp_backward(self._h, n_recv, n_send, E, _tptr(rowptr), _tptr(col),
-                                  _tptr(rowptr_T), _tptr(perm_T), _tptr(x), _tptr(Y), _tptr(W),
-                                  _tptr(grad_out), _tptr(dx), _tptr(dW), _tptr(dY),
-                                  _tptr(workspace), workspace.numel(), _stream(stream)))
+        _check(_lib.cgtp_backward(self._h, n_recv, n_send, E,
+                                  *self._backward_args(rowptr, col, rowptr_T, perm_T, x, Y, W, grad_out,
+                                                       dx, dW, dY, dev, n_recv, n_send, E),
+                                  *_workspace(workspace, dev), _stream(stream)))
         return dx, dW, dY
 
     def backward_static_scratch(self, rowptr, col, rowptr_T, perm_T, x, Y, W, grad_out,
@@ -297,8 +335,9 @@ class Plan:
             dY = torch.empty((E, self.d_edge), dtype=torch.float32, device=dev) if "Y" in want else None
         else:
             dx, dW, dY = grads
-        _check(_lib.cgtp_backward_static_scratch(self._h, n_recv, n_send, E, _tptr(rowptr), _tptr(col),
-                                                 _tptr(rowptr_T), _tptr(perm_T), _tptr(x), _tptr(Y),
-                                                 _tptr(W), _tptr(grad_out), _tptr(dx), _tptr(dW),
-                                                 _tptr(dY), _stream(stream)))
+        _check(_lib.cgtp_backward_static_scratch(self._h, n_recv, n_send, E,
+                                                 *self._backward_args(rowptr, col, rowptr_T, perm_T, x, Y, W,
+                                                                      grad_out, dx, dW, dY, dev, n_recv,
+                                                                      n_send, E),
+                                                 _stream(stream)))
         return dx, dW, dY

@@ -42,7 +42,13 @@
  *
  * Errors: every entry point returns a cgtp_status.  Arguments are validated
  * on the host before any launch (null pointers, 16-byte alignment of float
- * arrays, sizes, irreps, lmax).  No exception crosses the ABI.
+ * arrays, sizes, irreps, lmax).  No exception crosses the ABI.  What the ABI
+ * cannot see is trusted: each device buffer holds at least the elements its
+ * layout above implies (the Python binding checks dtype, element count and
+ * device of every tensor before the call), and the graph is a valid CSR
+ * (rowptr non-decreasing from 0 to E, every col in [0, n_send), perm_T a
+ * permutation grouped by sender) -- cgtp_csr_transpose checks exactly this
+ * on the host while it builds rowptr_T and perm_T.
  * cgtp_last_error() returns a message for the calling thread's last failure.
  * Calls are ordered on the given stream; a plan may be used from several
  * threads for concurrent launches.
@@ -260,7 +266,9 @@ cgtp_status cgtp_neighbor_list(int64_t N, const double* pos, const double* box, 
                                int64_t* n_edges);
 
 /* Transpose of a receiver CSR: rowptr_T [n_send+1] and perm_T [E] listing, for
- * every sender, the ids of its edges in ascending order.  Host pointers. */
+ * every sender, the ids of its edges in ascending order.  Host pointers.
+ * Checks the CSR on the way: CGTP_ERR_INVALID_CSR when rowptr does not run
+ * non-decreasing from 0 to E or a col entry lies outside [0, n_send). */
 cgtp_status cgtp_csr_transpose(int64_t n_recv, int64_t n_send, int64_t E,
                                const int32_t* rowptr, const int32_t* col, int32_t* rowptr_T,
                                int32_t* perm_T);

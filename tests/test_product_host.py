@@ -148,3 +148,41 @@ def test_force_chain_argument_errors(compile_only):
     assert lib.cgtp_edge_virial(4, p16, None, p16, None) == NULL
     assert lib.cgtp_edge_virial(4, p4, p16, p16, None) == ALIGN
     assert lib.cgtp_edge_virial(4, p16, p4, p16, None) == ALIGN
+
+
+def test_binding_checks_tensors_before_the_abi(compile_only):
+    """The binding refuses a tensor whose dtype, element count or device
+    would let a kernel's flat indexing leave it, before any pointer crosses
+    the C ABI (checked in that order, so CPU tensors reach each check)."""
+    torch = pytest.importorskip("torch")
+    plan = C.Plan("16x0e+16x1o", "1x0e+1x1o", "32x0e+32x1o", 6)
+    n, E = 3, 5
+    rowptr = torch.tensor([0, 2, 4, 5], dtype=torch.int32)
+    col = torch.tensor([1, 2, 0, 2, 1], dtype=torch.int32)
+    x = torch.zeros(n, plan.d_in)
+    Y = torch.zeros(E, plan.d_edge)
+    W = torch.zeros(E, plan.n_weights)
+    with pytest.raises(TypeError, match="x: expected torch.float32"):
+        plan.forward(rowptr, col, x.double(), Y, W)
+    with pytest.raises(TypeError, match="rowptr: expected torch.int32"):
+        plan.forward(rowptr.long(), col, x, Y, W)
+    with pytest.raises(ValueError, match="W: expected"):
+        plan.forward(rowptr, col, x, Y, W[:, 1:].contiguous())
+    with pytest.raises(ValueError, match="out: expected"):
+        plan.forward(rowptr, col, x, Y, W, out=torch.zeros(n, plan.d_out - 1))
+    with pytest.raises(ValueError, match="contiguous CUDA tensor"):
+        plan.forward(rowptr, col, x, Y, W)
+    g = torch.zeros(n, plan.d_out)
+    with pytest.raises(ValueError, match="rowptr_T: expected"):
+        plan.backward(rowptr, col, rowptr[:-1].contiguous(), col, x, Y, W, g)
+    with pytest.raises(ValueError, match="grad_out: expected"):
+        plan.backward(rowptr, col, rowptr, col, x, Y, W, g[:-1])
+    r = torch.zeros(E, 3)
+    with pytest.raises(ValueError, match="grad_Y: expected"):
+        plan.sph_harm_backward(r, torch.zeros(E, plan.d_edge + 1))
+    with pytest.raises(TypeError, match="r: expected torch.float32"):
+        C.edge_virial(r.int(), r)
+    with pytest.raises(ValueError, match="grad_r: expected"):
+        C.edge_virial(r, r[:-1])
+    with pytest.raises(ValueError, match="perm_T: expected"):
+        C.edge_forces(rowptr, rowptr, col[:-1], r)
