@@ -314,7 +314,6 @@ cgtp_status cgtp_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t
   if (!plan || !bytes) return fail(CGTP_ERR_NULL, "null argument");
   const Plan* P = reinterpret_cast<const Plan*>(plan);
   if (n_recv < 0 || n_send < 0 || E < 0) return fail(CGTP_ERR_SIZE, "negative size");
-  auto r256 = [](size_t v) { return (v + 255) & ~size_t(255); };
   *bytes = bwd_workspace_layout(*P, E, nullptr);
   return CGTP_OK;
 }
@@ -459,8 +458,7 @@ cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* need
 cgtp_status cgtp_plan_set_timing(cgtp_plan plan, int enable) {
   if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
   Plan* P = reinterpret_cast<Plan*>(plan);
-  std::lock_guard<std::mutex> g(P->tmu);
-  P->timing = enable != 0;
+  P->timing.store(enable != 0);
   return CGTP_OK;
 }
 

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <memory>
 #include <mutex>
@@ -123,7 +124,7 @@ struct Plan {
 
   int* d_err = nullptr;  // device error word
   // kernel timing (cgtp_plan_set_timing)
-  bool timing = false;
+  std::atomic<bool> timing{false};  // read by launches on any thread
   std::mutex tmu;
   struct TimedLaunch {
     int kind;
