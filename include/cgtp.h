@@ -97,7 +97,13 @@ const char* cgtp_last_error(void);
  * Parses and checks the irreps, enumerates the paths, builds the real CG
  * tables in FP64 (rounded to FP32 for the device), generates and compiles the
  * path-specialised forward and backward kernels for sm_100a, and uploads the
- * tables.  On failure *out is set to NULL. */
+ * tables.  On failure *out is set to NULL.
+ * Capacity: the backward keeps the grad_out rows of all paths of one hidden
+ * irrep in shared memory, beside two edge stages, within the 227 KB a CTA
+ * can hold: a plan whose single hidden irrep feeds more than roughly 30,000
+ * output floats per atom (mul x the sum of 2 l3 + 1 over its paths; 256x6e
+ * against L = 6 edges feeds 51,456) is refused with CGTP_ERR_SIZE.
+ * Errors: NULL, IRREPS_PARSE, IRREPS_MISMATCH, LMAX, SIZE, CUDA, OOM, JIT. */
 cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge,
                              const char* irreps_out, int lmax, cgtp_plan* out);
 

@@ -8,6 +8,8 @@ plans, no GPU):
   * backward: for each hidden irrep with paths, its roles share one phase
     count nph and cover every (32-channel block, edge phase) pair once, all
     in one slice; a slice has no more roles than consumer warps.
+The same on irreps sets unlike the workloads, and the one refusal the
+planner has (a hidden irrep too wide for shared memory).
 """
 import re
 from collections import Counter
@@ -19,6 +21,16 @@ from equivariant_mlip_clebsch_b200 import cgtp as C
 from equivariant_mlip_clebsch_b200 import workloads as WL
 
 NAMES = ["tiny", "lmax2", "lmax2_wide", "lmax3", "lmax6", "case4", "case5", "case6"]
+# irreps sets unlike the workloads: multiplicities 1, 3, 17, 33 and 96 (partial
+# warps and blocks), one irrep without any path, missing outputs, odd parities
+ODD = [
+    ("3x2o", "1x0e+1x1o", "3x1e+3x2o+3x2e+3x3e"),
+    ("1x0e", "1x0e+1x1o+1x2e", "1x1o+1x2e"),
+    ("96x1e", "1x0e+1x1o", "96x0o+96x1o"),
+    ("128x0e+17x1e+1x2e", "1x0e+1x1o+1x2e", "17x0o+129x0e+35x1e+18x2o+147x2e+1x3o+18x3e+1x4e"),
+    ("33x0e", "1x0e+1x1o+1x2e+1x3o+1x4e", "33x0e+33x1o+33x3o+33x4e"),
+    ("16x0e+16x1o+8x2e", "1x0e+1x1o", "32x0e+16x1e"),  # 8x2e feeds no output
+]
 
 
 @pytest.fixture
@@ -40,9 +52,11 @@ def _parse(text, kind):
     return nroles, nw, slices[:nslices]
 
 
-@pytest.mark.parametrize("name", NAMES)
-def test_role_coverage(name, compile_only):
-    c = WL.CONFIGS[name]
+@pytest.mark.parametrize("irreps", [WL.CONFIGS[n] for n in NAMES] + [
+    dict(irreps_in=a, irreps_edge=b, irreps_out=c) for a, b, c in ODD], ids=NAMES + [f"odd{k}" for k in range(len(ODD))])
+def test_role_coverage(irreps, compile_only):
+    c = irreps
+    name = c["irreps_in"]
     plan = C.Plan(c["irreps_in"], c["irreps_edge"], c["irreps_out"], 6)
     P = O.enumerate_paths(c["irreps_in"], c["irreps_edge"], c["irreps_out"])
     text = plan.describe()
@@ -95,3 +109,13 @@ def test_role_coverage(name, compile_only):
                     pairs[(u0 + 32 * k, ph)] += 1
         blocks = range(0, muls[a], 32)
         assert pairs == Counter({(b, ph): 1 for b in blocks for ph in range(nph)}), (name, a)
+
+
+def test_backward_capacity_refusal(compile_only):
+    """One hidden irrep whose grad_out rows do not fit shared memory beside two
+    edge stages (256x6e against L = 6 edges: 21 paths, 51,456 floats per atom)
+    is refused with CGTP_ERR_SIZE, not planned into an invalid kernel."""
+    with pytest.raises(C.CgtpError) as e:
+        C.Plan("33x1o+17x4o+256x6e", "1x0e+1x1o+1x2e+1x3o+1x4e+1x5o+1x6e",
+               "339x1o+340x2o+612x2e+596x3e+613x4o+885x4e+885x5o+852x6o+1091x6e", 6)
+    assert e.value.status == 6 and "shared memory" in str(e.value)
