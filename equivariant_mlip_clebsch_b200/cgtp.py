@@ -287,6 +287,16 @@ class Plan:
         _check(_lib.cgtp_forward(self._h, n_recv, n_send, E, *ptrs, _stream(stream)))
         return out
 
+    def _grads(self, want, grads, n_send, E, dev):
+        """The caller's (dx, dW, dY), or new tensors for the gradients in `want`."""
+        if grads is not None:
+            return grads
+        import torch
+        f = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
+        return (f(n_send, self.d_in) if "x" in want else None,
+                f(E, self.n_weights) if "W" in want else None,
+                f(E, self.d_edge) if "Y" in want else None)
+
     def _backward_args(self, rowptr, col, rowptr_T, perm_T, x, Y, W, grad_out, dx, dW, dY, dev,
                        n_recv, n_send, E):
         return _args(dev, (rowptr, "rowptr", n_recv + 1, "i32"), (col, "col", E, "i32"),
@@ -306,12 +316,7 @@ class Plan:
         import torch
         n_recv, n_send, E = rowptr.shape[0] - 1, x.shape[0], col.shape[0]
         dev = x.device
-        if grads is None:
-            dx = torch.empty((n_send, self.d_in), dtype=torch.float32, device=dev) if "x" in want else None
-            dW = torch.empty((E, self.n_weights), dtype=torch.float32, device=dev) if "W" in want else None
-            dY = torch.empty((E, self.d_edge), dtype=torch.float32, device=dev) if "Y" in want else None
-        else:
-            dx, dW, dY = grads
+        dx, dW, dY = self._grads(want, grads, n_send, E, dev)
         if workspace is None:
             nbytes = self.workspace_size(n_recv, n_send, E)
             workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
@@ -326,15 +331,9 @@ class Plan:
         """cgtp_backward_static_scratch: the backward with the library's fixed
         device scratch instead of a workspace (no device allocation in the call
         when ``grads`` are given)."""
-        import torch
         n_recv, n_send, E = rowptr.shape[0] - 1, x.shape[0], col.shape[0]
         dev = x.device
-        if grads is None:
-            dx = torch.empty((n_send, self.d_in), dtype=torch.float32, device=dev) if "x" in want else None
-            dW = torch.empty((E, self.n_weights), dtype=torch.float32, device=dev) if "W" in want else None
-            dY = torch.empty((E, self.d_edge), dtype=torch.float32, device=dev) if "Y" in want else None
-        else:
-            dx, dW, dY = grads
+        dx, dW, dY = self._grads(want, grads, n_send, E, dev)
         _check(_lib.cgtp_backward_static_scratch(self._h, n_recv, n_send, E,
                                                  *self._backward_args(rowptr, col, rowptr_T, perm_T, x, Y, W,
                                                                       grad_out, dx, dW, dY, dev, n_recv,
