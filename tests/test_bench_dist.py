@@ -80,6 +80,8 @@ def test_reference_arm_under_torchrun_prints_one_line():
     prints one JSON line; rank 1 exits 0 without work."""
     import json
     import subprocess
+
+    import bench
     port = _free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
@@ -91,3 +93,7 @@ def test_reference_arm_under_torchrun_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    # the same metric, unit, direction and workload as the CUDA arm
+    assert d["metric"] == bench.METRIC and d["unit"] == "edges/s" and d["higher_is_better"] is True
+    assert d["config"]["workload"].startswith(bench.DEFAULT_CONFIG + ":")
+    assert d["steps"] == 1 and d["warmup"] == 3 and d["cpu_baseline"]["cores"] >= 1
