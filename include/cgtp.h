@@ -266,7 +266,9 @@ cgtp_status cgtp_plan_check_device_error(cgtp_plan plan, int* code);
  * Edges are ordered by (receiver i, sender j, n_x, n_y, n_z).  Positions must
  * lie in [0, box).  Call with col == NULL to get *n_edges (and rowptr); then
  * with col/shift/r sized for it.  r [E,3] FP32 = the rounded edge vectors,
- * shift [E,3] int32 = n.  rowptr has N+1 entries. */
+ * shift [E,3] int32 = n.  rowptr has N+1 entries.  Receivers are split over
+ * host threads (CGTP_HOST_THREADS, default the hardware threads, one below
+ * 4096 atoms); the result does not depend on their number. */
 cgtp_status cgtp_neighbor_list(int64_t N, const double* pos, const double* box, double rc,
                                int32_t* rowptr, int32_t* col, int32_t* shift, float* r,
                                int64_t* n_edges);

@@ -68,6 +68,18 @@ def test_neighbor_list_small_boxes_many_images(cells, rc):
     assert np.array_equal(sh, sh_o) and np.array_equal(r, vec_o.astype(np.float32))
 
 
+@pytest.mark.parametrize("threads", ["1", "3", "7"])
+def test_neighbor_list_independent_of_host_threads(threads, monkeypatch):
+    """Receivers split over host threads (uneven ranges here) give the
+    oracle's brute-force list bit for bit."""
+    pos, box = WL.si_diamond((2, 2, 3), 0.07, 4)
+    rp_o, col_o, sh_o, vec_o = O.neighbor_list(pos, box, 5.0)
+    monkeypatch.setenv("CGTP_HOST_THREADS", threads)
+    rp, col, sh, r = C.neighbor_list(pos, box, 5.0)
+    assert np.array_equal(rp.astype(np.int64), rp_o) and np.array_equal(col, col_o)
+    assert np.array_equal(sh, sh_o) and np.array_equal(r, vec_o.astype(np.float32))
+
+
 def test_neighbor_list_rejects_unwrapped_positions():
     with pytest.raises(C.CgtpError):
         C.neighbor_list(np.array([[0.0, 0.0, 5.0]]), np.array([4.0, 4.0, 4.0]), 3.0)
