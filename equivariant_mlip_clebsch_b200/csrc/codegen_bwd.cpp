@@ -30,6 +30,7 @@
 #include <functional>
 #include <numeric>
 #include <sstream>
+#include <thread>
 
 #include "codegen_common.hpp"
 
@@ -629,26 +630,55 @@ cgtp_status build_backward(Plan& P) {
   // over equal edge ranges.  The second balances graphs with few receivers
   // per CTA; measured on B200, the range code in the first variant (even
   // when not taken) slowed the large cases, hence two kernels.
-  for (int er = 0; er < 2; ++er) {
-    K.edge_ranges = er == 1;
-    const std::string name = er ? "cgtp_bwd_er" : "cgtp_bwd";
-    JitKernel& JK = er ? P.bwd_er : P.bwd;
+  // Both are compiled at once on two host threads (NVRTC needs no CUDA
+  // context; each takes tens of seconds at Lmax 6), then loaded here.  Each
+  // lowers its resident-CTA target while the compiler reports spills.
+  struct Variant {
     std::string src;
-    for (int mb = mb0; mb >= mb_floor; --mb) {
-      src = gen_bwd_source(P, SL, K, name, mb);
-      JK.threads = (F.nw + 2) * 32;
-      JK.smem = K.smem;
-      cgtp_status cst = jit_compile(src, name, JK);
-      if (cst != CGTP_OK) return cst;
-      if (mb == mb_floor || max_spill_bytes(JK.log) <= 160) break;
-      jit_unload(JK);
+    JitBinary bin;
+    cgtp_status st = CGTP_OK;
+  } var[2];
+  auto build = [&](int er) {
+    try {
+      KernelShape Kv = K;
+      Kv.edge_ranges = er == 1;
+      const std::string name = er ? "cgtp_bwd_er" : "cgtp_bwd";
+      for (int mb = mb0; mb >= mb_floor; --mb) {
+        var[er].src = gen_bwd_source(P, SL, Kv, name, mb);
+        var[er].st = jit_build(var[er].src, name, var[er].bin);
+        if (var[er].st != CGTP_OK || mb == mb_floor || max_spill_bytes(var[er].bin.log) <= 160) break;
+      }
+    } catch (const std::exception& e) {
+      var[er].st = CGTP_ERR_OOM;
+      var[er].bin.err = std::string("exception while building the backward: ") + e.what();
     }
+  };
+  {
+    std::thread second;
+    try {
+      second = std::thread(build, 1);
+    } catch (...) {
+    }
+    build(0);
+    if (second.joinable())
+      second.join();
+    else
+      build(1);
+  }
+  for (int er = 0; er < 2; ++er) {
+    if (var[er].st != CGTP_OK) {
+      set_error(var[er].bin.err);
+      return var[er].st;
+    }
+    JitKernel& JK = er ? P.bwd_er : P.bwd;
     JK.threads = (F.nw + 2) * 32;
     JK.smem = K.smem;
+    cgtp_status cst = jit_load(var[er].bin, er ? "cgtp_bwd_er" : "cgtp_bwd", JK);
+    if (cst != CGTP_OK) return cst;
     if (const char* d = std::getenv("CGTP_DUMP_SOURCE")) {
       FILE* f = std::fopen((std::string(d) + (er ? "/bwd_er.cu" : "/bwd.cu")).c_str(), "w");
       if (f) {
-        std::fputs(src.c_str(), f);
+        std::fputs(var[er].src.c_str(), f);
         std::fclose(f);
       }
     }

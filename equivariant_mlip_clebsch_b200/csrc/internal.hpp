@@ -150,6 +150,14 @@ cgtp_status build_backward(Plan& P);
 void destroy_plan_device(Plan& P);
 
 // JIT
+// A compiled kernel before loading: building needs no CUDA context and may
+// run on any thread; loading uses the calling thread's current context.
+struct JitBinary {
+  std::string cubin, log, err;  // err: the failing thread's message
+  unsigned long long hash = 0;
+};
+cgtp_status jit_build(const std::string& src, const std::string& name, JitBinary& b);
+cgtp_status jit_load(const JitBinary& b, const std::string& name, JitKernel& k);
 cgtp_status jit_compile(const std::string& src, const std::string& name, JitKernel& k);
 cgtp_status jit_launch(const JitKernel& k, dim3 grid, void** args, cudaStream_t stream);
 void jit_unload(JitKernel& k);

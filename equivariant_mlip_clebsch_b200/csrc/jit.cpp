@@ -13,7 +13,9 @@
 #include <cstdlib>
 #include <cstring>
 #include <fstream>
+#include <functional>
 #include <sstream>
+#include <thread>
 #include <unistd.h>
 
 #include "internal.hpp"
@@ -92,7 +94,8 @@ bool read_file(const std::string& path, std::string& out) {
 }
 
 void write_file_atomic(const std::string& path, const std::string& data) {
-  std::string tmp = path + ".tmp" + std::to_string((long)::getpid());
+  std::string tmp = path + ".tmp" + std::to_string((long)::getpid()) + "_" +
+                    std::to_string(std::hash<std::thread::id>()(std::this_thread::get_id()));
   {
     std::ofstream f(tmp, std::ios::binary);
     if (!f) return;
@@ -153,16 +156,28 @@ static cgtp_status compile_cubin(const std::string& src, const std::string& name
   return CGTP_OK;
 }
 
+cgtp_status jit_build(const std::string& src, const std::string& name, JitBinary& b) {
+  const cgtp_status st = compile_cubin(src, name, b.cubin, b.log, b.hash);
+  if (st != CGTP_OK) b.err = cgtp_last_error();  // this thread's message, for the caller's
+  return st;
+}
+
 cgtp_status jit_compile(const std::string& src, const std::string& name, JitKernel& k) {
-  std::string cubin;
-  cgtp_status st = compile_cubin(src, name, cubin, k.log, k.hash);
+  JitBinary b;
+  const cgtp_status st = jit_build(src, name, b);
   if (st != CGTP_OK) return st;
+  return jit_load(b, name, k);
+}
+
+cgtp_status jit_load(const JitBinary& b, const std::string& name, JitKernel& k) {
+  k.log = b.log;
+  k.hash = b.hash;
   k.name = name;
   if (std::getenv("CGTP_JIT_COMPILE_ONLY")) return CGTP_OK;  // host-only checks
   Driver& d = driver();
   if (!d.ok) return fail(CGTP_ERR_CUDA, d.err);
   CUmodule mod;
-  CUresult cr = d.moduleLoadData(&mod, cubin.data());
+  CUresult cr = d.moduleLoadData(&mod, b.cubin.data());
   if (cr != CUDA_SUCCESS) return fail(CGTP_ERR_CUDA, "cuModuleLoadData: " + cu_str(cr));
   CUfunction fn;
   cr = d.moduleGetFunction(&fn, mod, name.c_str());
