@@ -9,7 +9,9 @@ plans, no GPU):
     count nph and cover every (32-channel block, edge phase) pair once, all
     in one slice; a slice has no more roles than consumer warps.
 The same on irreps sets unlike the workloads, and the one refusal the
-planner has (a hidden irrep too wide for shared memory).
+planner has (a hidden irrep too wide for shared memory).  And, read from the
+generated source, every row copy into shared memory stays inside its global
+row and its staging slot, with bulk (TMA) copies on 16-byte boundaries.
 """
 import re
 from collections import Counter
@@ -119,3 +121,91 @@ def test_backward_capacity_refusal(compile_only):
         C.Plan("33x1o+17x4o+256x6e", "1x0e+1x1o+1x2e+1x3o+1x4e+1x5o+1x6e",
                "339x1o+340x2o+612x2e+596x3e+613x4o+885x4e+885x5o+852x6o+1091x6e", 6)
     assert e.value.status == 6 and "shared memory" in str(e.value)
+
+
+def _defines(src):
+    return {m.group(1): int(m.group(2)) for m in re.finditer(r"^#define (\w+) (-?\d+)\s*$", src, re.M)}
+
+
+def _check_copies(src):
+    """Every row copy the generated kernel makes into shared memory: the
+    source range inside its global row (W: NU, x: DIN, grad_out: DOUT), the
+    destination inside its staging slot (WS, XS, GS per edge), and every bulk
+    (TMA) copy on 16-byte boundaries with a multiple of 16 bytes.  Returns
+    (copies checked, problems)."""
+    d = _defines(src)
+    DIN, DOUT, NU = d["DIN"], d["DOUT"], d["NU"]
+    WS, XS, GS = d.get("WS", 0), d.get("XS", 0), d.get("GS", 0)
+    bad, n = [], 0
+    for m in re.finditer(r"t < (\d+); t \+= 32\) sg\[(\d+) \+ t\] = grow\[(\d+) \+ t\]", src):
+        N, D, S = map(int, m.groups())
+        n += 1
+        if not (S + N <= DOUT and D + N <= GS):
+            bad.append(m.group(0))
+    recognised = 0
+    for arr, row, width, slot in (("sW", "WROW", NU, WS), ("sX", "XROW", DIN, XS)):
+        for m in re.finditer(r"t < nb \* (\d+); t \+= 32\) \{ const int b = t / \d+, q = t - b \* \d+; " + arr
+                             + r"\[b \* (\d+) \+ (\d+) \+ q\] = " + row + r"\(b\)\[(\d+) \+ q\]", src):
+            N, stride, D, S = map(int, m.groups())
+            n += 1
+            if not (S + N <= width and D + N <= stride == slot):
+                bad.append(m.group(0))
+        for m in re.finditer(r"bulk_g2s(?:_stream)?\(smem_u32\(" + arr + r" \+ b \* (\d+) \+ (\d+)\), " + row
+                             + r"\(b\) \+ (\d+), (\d+),", src):
+            stride, D, S, B = map(int, m.groups())
+            n += 1
+            recognised += 1
+            if not (B % 16 == 0 and S % 4 == 0 and D % 4 == 0 and width % 4 == 0 and stride % 4 == 0
+                    and S + B // 4 <= width and D + B // 4 <= stride == slot):
+                bad.append(m.group(0))
+    for m in re.finditer(r"bulk_g2s(?:_stream)?\(smem_u32\(sg \+ (\d+)\), grow \+ (\d+), (\d+),", src):
+        D, S, B = map(int, m.groups())
+        n += 1
+        recognised += 1
+        if not (B % 16 == 0 and S % 4 == 0 and D % 4 == 0 and DOUT % 4 == 0
+                and S + B // 4 <= DOUT and D + B // 4 <= GS):
+            bad.append(m.group(0))
+    # one copy for a chunk's consecutive W rows (only W rows are contiguous)
+    for m in re.finditer(r"bulk_g2s_stream\(smem_u32\((sW|sX)\), (WROW|XROW)\(0\), \(u32\)nb \* (\d+),", src):
+        B = int(m.group(3))
+        n += 1
+        recognised += 1
+        if not (m.group(1) == "sW" and B == 4 * NU and WS == NU and B % 16 == 0):
+            bad.append(m.group(0))
+    total = len(re.findall(r"\bbulk_g2s(?:_stream)?\(smem_u32", src))
+    if total != recognised:
+        bad.append(f"{total - recognised} bulk copies of an unrecognised form")
+    return n, bad
+
+
+@pytest.mark.parametrize("irreps", [WL.CONFIGS[n] for n in NAMES] + [
+    dict(irreps_in=a, irreps_edge=b, irreps_out=c) for a, b, c in ODD], ids=NAMES + [f"odd{k}" for k in range(len(ODD))])
+def test_generated_copies_stay_in_bounds(irreps, compile_only, monkeypatch, tmp_path):
+    """The generated kernels' row copies into shared memory, read from the
+    generated source (checked here so that a mistake fails on the CPU rather
+    than faulting a GPU)."""
+    monkeypatch.setenv("CGTP_DUMP_SOURCE", str(tmp_path))
+    C.Plan(irreps["irreps_in"], irreps["irreps_edge"], irreps["irreps_out"], 6)
+    files = sorted(p.name for p in tmp_path.iterdir())
+    assert files == ["bwd.cu", "bwd_er.cu", "fwd.cu"]
+    for f in files:
+        n, bad = _check_copies((tmp_path / f).read_text())
+        assert n > 0 and not bad, (f, bad[:3])
+
+
+def test_copy_check_catches_planted_mistakes():
+    head = "#define DIN 64\n#define DOUT 128\n#define NU 96\n#define WS 96\n#define XS 64\n#define GS 128\n"
+    ok = head + ("bulk_g2s(smem_u32(sW + b * 96 + 0), WROW(b) + 32, 256, bar);\n"
+                 "for (int t = lane; t < 16; t += 32) sg[0 + t] = grow[100 + t];\n")
+    assert _check_copies(ok) == (2, [])
+    planted = [
+        "bulk_g2s(smem_u32(sW + b * 96 + 0), WROW(b) + 33, 256, bar);\n",   # source off 16 bytes
+        "bulk_g2s(smem_u32(sW + b * 96 + 0), WROW(b) + 32, 260, bar);\n",   # size not 16-byte multiple
+        "bulk_g2s(smem_u32(sW + b * 96 + 64), WROW(b) + 32, 256, bar);\n",  # past the W slot
+        "for (int t = lane; t < 16; t += 32) sg[0 + t] = grow[120 + t];\n",  # past the grad_out row
+        "if (lane == 0) bulk_g2s_stream(smem_u32(sX), XROW(0), (u32)nb * 256, bar, pol);\n",  # gathered rows
+        "bulk_g2s(smem_u32(sY + 4), yrow, 64, bar);\n",                      # unknown form
+    ]
+    for p in planted:
+        n, bad = _check_copies(head + p)
+        assert bad, p
