@@ -11,8 +11,8 @@ pinned host memory and the outputs copied back inside the timed region.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
   python bench.py --impl reference ...     # the FP64 oracle on the host cores
 
-Multi-GPU: the workload does not shard across GPUs in this build; N ranks run
-N independent replicas ("weak" scaling), timed on the device, max over ranks.
+Multi-GPU: the convolution is not sharded across GPUs; N ranks run N
+independent replicas ("weak" scaling), timed on the device, max over ranks.
 Prints one JSON line on rank 0 (details for humans go to stderr).
 """
 from __future__ import annotations
