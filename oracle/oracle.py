@@ -307,3 +307,36 @@ def backward(paths: Paths, rowptr, col, n_send: int, x, Y, W, g, want=("x", "W",
                        _ptr(np.ascontiguousarray(paths.table)), _ptr(paths.cg), _ptr(dx),
                        _ptr(dW), _ptr(dY), int(nthreads))
     return dx, dW, dY
+
+
+def double_backward(paths: Paths, rowptr, col, n_send: int, x, Y, W, g, h_x=None, h_W=None, h_Y=None):
+    """Gradients of S = <h_x, dx> + <h_W, dW> + <h_Y, dY>, (dx, dW, dY) the
+    backward of the convolution at (x, Y, W) with cotangent g, with respect
+    to g, x, W and Y (None cotangents are zero).  The convolution is linear
+    in each of x, Y and W, so each term of S is the pairing of g with a
+    forward in which one argument is replaced by its cotangent:
+        S = <g, fwd(h_x, Y, W) + fwd(x, Y, h_W) + fwd(x, h_Y, W)>
+    and every gradient is a forward or a backward with that substitution.
+    Written as those calls of forward() and backward() above."""
+    n_recv = len(rowptr) - 1
+    E = len(col)
+    gg = np.zeros((n_recv, paths.D_out))
+    gx = np.zeros((n_send, paths.D_in))
+    gW = np.zeros((E, paths.U))
+    gY = np.zeros((E, paths.D_e))
+    if h_x is not None:  # <g, fwd(h_x, Y, W)>: depends on g, Y, W
+        gg += forward(paths, rowptr, col, h_x, Y, W)
+        _, dW, dY = backward(paths, rowptr, col, n_send, h_x, Y, W, g, want=("W", "Y"))
+        gW += dW
+        gY += dY
+    if h_W is not None:  # <g, fwd(x, Y, h_W)>: depends on g, x, Y
+        gg += forward(paths, rowptr, col, x, Y, h_W)
+        dx, _, dY = backward(paths, rowptr, col, n_send, x, Y, h_W, g, want=("x", "Y"))
+        gx += dx
+        gY += dY
+    if h_Y is not None:  # <g, fwd(x, h_Y, W)>: depends on g, x, W
+        gg += forward(paths, rowptr, col, x, h_Y, W)
+        dx, dW, _ = backward(paths, rowptr, col, n_send, x, h_Y, W, g, want=("x", "W"))
+        gx += dx
+        gW += dW
+    return gg, gx, gW, gY
