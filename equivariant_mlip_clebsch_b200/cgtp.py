@@ -40,6 +40,8 @@ _SIGS = {
     "cgtp_sph_harm_backward": (_i, [_P, _i64, _P, _P, _P, _P]),
     "cgtp_edge_forces": (_i, [_i64, _i64, _P, _P, _P, _P, _P, _P]),
     "cgtp_edge_virial": (_i, [_i64, _P, _P, _P, _P]),
+    "cgtp_double_backward_workspace_size": (_i, [_P, _i64, _i64, _i64, ctypes.POINTER(_sz)]),
+    "cgtp_double_backward": (_i, [_P, _i64, _i64, _i64] + [_P] * 16 + [_sz, _P]),
     "cgtp_forward": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P, _P, _P]),
     "cgtp_backward_workspace_size": (_i, [_P, _i64, _i64, _i64, ctypes.POINTER(_sz)]),
     "cgtp_backward": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -325,6 +327,41 @@ class Plan:
                                                        dx, dW, dY, dev, n_recv, n_send, E),
                                   *_workspace(workspace, dev), _stream(stream)))
         return dx, dW, dY
+
+    def double_backward_workspace_size(self, n_recv: int, n_send: int, E: int) -> int:
+        b = ctypes.c_size_t()
+        _check(_lib.cgtp_double_backward_workspace_size(self._h, n_recv, n_send, E, ctypes.byref(b)))
+        return b.value
+
+    def double_backward(self, rowptr, col, rowptr_T, perm_T, x, Y, W, grad_out, h_x=None, h_W=None,
+                        h_Y=None, want=("g", "x", "W", "Y"), grads=None, workspace=None, stream=None):
+        """cgtp_double_backward: the gradients (d grad_out, dx, dW, dY) of
+        S = <h_x, grad_x> + <h_W, grad_W> + <h_Y, grad_Y> over the backward
+        at (x, Y, W, grad_out); None cotangents are zero."""
+        import torch
+        n_recv, n_send, E = rowptr.shape[0] - 1, x.shape[0], col.shape[0]
+        dev = x.device
+        if grads is None:
+            f = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
+            grads = (f(n_recv, self.d_out) if "g" in want else None,
+                     f(n_send, self.d_in) if "x" in want else None,
+                     f(E, self.n_weights) if "W" in want else None,
+                     f(E, self.d_edge) if "Y" in want else None)
+        gg, gx, gW, gY = grads
+        if workspace is None:
+            nbytes = self.double_backward_workspace_size(n_recv, n_send, E)
+            workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        ptrs = _args(dev, (rowptr, "rowptr", n_recv + 1, "i32"), (col, "col", E, "i32"),
+                     (rowptr_T, "rowptr_T", n_send + 1, "i32"), (perm_T, "perm_T", E, "i32"),
+                     (x, "x", n_send * self.d_in, "f32"), (Y, "Y", E * self.d_edge, "f32"),
+                     (W, "W", E * self.n_weights, "f32"), (grad_out, "grad_out", n_recv * self.d_out, "f32"),
+                     (h_x, "h_x", n_send * self.d_in, "f32"), (h_W, "h_W", E * self.n_weights, "f32"),
+                     (h_Y, "h_Y", E * self.d_edge, "f32"), (gg, "grad_grad_out", n_recv * self.d_out, "f32"),
+                     (gx, "grad_x", n_send * self.d_in, "f32"), (gW, "grad_W", E * self.n_weights, "f32"),
+                     (gY, "grad_Y", E * self.d_edge, "f32"))
+        _check(_lib.cgtp_double_backward(self._h, n_recv, n_send, E, *ptrs, *_workspace(workspace, dev),
+                                         _stream(stream)))
+        return gg, gx, gW, gY
 
     def backward_static_scratch(self, rowptr, col, rowptr_T, perm_T, x, Y, W, grad_out,
                                 want=("x", "W", "Y"), grads=None, stream=None):

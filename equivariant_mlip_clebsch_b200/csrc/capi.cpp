@@ -109,6 +109,23 @@ static size_t bwd_workspace_layout(const Plan& P, int64_t E, size_t* off_dyp) {
   return b;
 }
 
+// Double-backward workspace: the backward's own workspace, then one scratch
+// buffer per output (grad_out, x, W, Y) for a term added to an earlier one.
+struct DbwdLayout {
+  size_t bwd, f, x, w, y, total;
+};
+static DbwdLayout dbwd_workspace_layout(const Plan& P, int64_t n_recv, int64_t n_send, int64_t E) {
+  auto r256 = [](size_t v) { return (v + 255) & ~size_t(255); };
+  DbwdLayout L;
+  L.bwd = 0;
+  L.f = r256(bwd_workspace_layout(P, E, nullptr));
+  L.x = L.f + r256((size_t)n_recv * P.D_out * sizeof(float));
+  L.w = L.x + r256((size_t)n_send * P.D_in * sizeof(float));
+  L.y = L.w + r256((size_t)E * P.U * sizeof(float));
+  L.total = L.y + r256((size_t)E * P.D_e * sizeof(float));
+  return L;
+}
+
 }  // namespace cgtp
 
 using namespace cgtp;
@@ -517,6 +534,89 @@ cgtp_status cgtp_plan_check_device_error(cgtp_plan plan, int* code) {
   CGTP_CUDA_TRY(cudaMemset(P->d_err, 0, sizeof(int)));
   *code = v;
   if (v != 0) return fail(CGTP_ERR_TIMEOUT, "a bounded wait inside a kernel expired");
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_double_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                                                size_t* bytes) {
+  if (!plan || !bytes) return fail(CGTP_ERR_NULL, "null argument");
+  if (n_recv < 0 || n_send < 0 || E < 0) return fail(CGTP_ERR_SIZE, "negative size");
+  *bytes = dbwd_workspace_layout(*reinterpret_cast<const Plan*>(plan), n_recv, n_send, E).total;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                                 const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
+                                 const int32_t* perm_T, const float* x, const float* Y, const float* W,
+                                 const float* grad_out, const float* h_x, const float* h_W, const float* h_Y,
+                                 float* gg_out, float* gx, float* gW, float* gY, void* workspace,
+                                 size_t workspace_bytes, cgtp_stream stream) {
+  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
+  Plan* P = reinterpret_cast<Plan*>(plan);
+  if (n_recv < 0 || n_send < 0 || E < 0 || n_recv >= (int64_t(1) << 31) ||
+      n_send >= (int64_t(1) << 31) || E >= (int64_t(1) << 31) - 1)
+    return fail(CGTP_ERR_SIZE, "sizes out of range");
+  cgtp_status st = check_device(*P);
+  if (st != CGTP_OK) return st;
+  for (const void* p : {(const void*)x, (const void*)Y, (const void*)W, (const void*)grad_out, (const void*)h_x,
+                        (const void*)h_W, (const void*)h_Y, (const void*)gg_out, (const void*)gx, (const void*)gW,
+                        (const void*)gY})
+    if (p && !aligned16(p)) return fail(CGTP_ERR_ALIGN, "float arrays must be 16-byte aligned");
+  if (n_recv > 0 && !rowptr) return fail(CGTP_ERR_NULL, "rowptr is NULL");
+  if (E > 0 && (!col || !x || !Y || !W || !grad_out))
+    return fail(CGTP_ERR_NULL, "col, x, Y, W or grad_out is NULL");
+  if (gx && (h_W || h_Y) && E > 0 && (!rowptr_T || !perm_T))
+    return fail(CGTP_ERR_NULL, "grad_x needs rowptr_T and perm_T");
+  const DbwdLayout L = dbwd_workspace_layout(*P, n_recv, n_send, E);
+  if (!workspace || workspace_bytes < L.total)
+    return fail(CGTP_ERR_WORKSPACE, "workspace of " + std::to_string(L.total) + " bytes required");
+  if ((uintptr_t)workspace & 255) return fail(CGTP_ERR_ALIGN, "workspace must be 256-byte aligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  char* ws = reinterpret_cast<char*>(workspace);
+  float* tF = reinterpret_cast<float*>(ws + L.f);
+  float* tX = reinterpret_cast<float*>(ws + L.x);
+  float* tW = reinterpret_cast<float*>(ws + L.w);
+  float* tY = reinterpret_cast<float*>(ws + L.y);
+  // S = <g, fwd(h_x, Y, W) + fwd(x, Y, h_W) + fwd(x, h_Y, W)>: one term per
+  // given cotangent, each a forward or backward with one argument replaced
+  const float* tx[3] = {h_x, x, x};
+  const float* ty[3] = {Y, Y, h_Y};
+  const float* tw[3] = {W, h_W, W};
+  const bool on[3] = {h_x != nullptr, h_W != nullptr, h_Y != nullptr};
+  if (gg_out && n_recv > 0) {  // d S / d grad_out: the three forwards
+    bool written = false;
+    for (int k = 0; k < 3; ++k) {
+      if (!on[k]) continue;
+      float* dst = written ? tF : gg_out;
+      st = cgtp_forward(plan, n_recv, n_send, E, rowptr, col, tx[k], ty[k], tw[k], dst, stream);
+      if (st != CGTP_OK) return st;
+      if (written) CGTP_CUDA_TRY(launch_add(n_recv * P->D_out, tF, gg_out, s));
+      written = true;
+    }
+    if (!written) CGTP_CUDA_TRY(cudaMemsetAsync(gg_out, 0, (size_t)n_recv * P->D_out * sizeof(float), s));
+  }
+  // d S / d (x, W, Y): term k gives the gradients of the two arguments it
+  // kept (h_x: W and Y; h_W: x and Y; h_Y: x and W)
+  bool wx = false, ww = false, wy = false;
+  for (int k = 0; k < 3; ++k) {
+    if (!on[k]) continue;
+    float* ox = (k != 0 && gx) ? (wx ? tX : gx) : nullptr;
+    float* ow = (k != 1 && gW) ? (ww ? tW : gW) : nullptr;
+    float* oy = (k != 2 && gY) ? (wy ? tY : gY) : nullptr;
+    if (!ox && !ow && !oy) continue;
+    st = backward_impl(plan, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, tx[k], ty[k], tw[k], grad_out, ox,
+                       ow, oy, ws + L.bwd, L.f - L.bwd, stream, true);
+    if (st != CGTP_OK) return st;
+    if (ox == tX) CGTP_CUDA_TRY(launch_add(n_send * P->D_in, tX, gx, s));
+    if (ow == tW) CGTP_CUDA_TRY(launch_add(E * P->U, tW, gW, s));
+    if (oy == tY) CGTP_CUDA_TRY(launch_add(E * P->D_e, tY, gY, s));
+    wx = wx || ox;
+    ww = ww || ow;
+    wy = wy || oy;
+  }
+  if (gx && !wx && n_send > 0) CGTP_CUDA_TRY(cudaMemsetAsync(gx, 0, (size_t)n_send * P->D_in * sizeof(float), s));
+  if (gW && !ww && E > 0) CGTP_CUDA_TRY(cudaMemsetAsync(gW, 0, (size_t)E * P->U * sizeof(float), s));
+  if (gY && !wy && E > 0) CGTP_CUDA_TRY(cudaMemsetAsync(gY, 0, (size_t)E * P->D_e * sizeof(float), s));
   return CGTP_OK;
 }
 

@@ -171,6 +171,7 @@ cudaError_t launch_sph_harm_backward(int L, int64_t E, const float* r, const flo
 cudaError_t launch_edge_forces(int64_t n_atoms, const int32_t* rowptr, const int32_t* rowptr_T,
                                const int32_t* perm_T, const float* G, float* F, cudaStream_t s);
 cudaError_t launch_edge_virial(int64_t E, const float* r, const float* G, float* V, cudaStream_t s);
+cudaError_t launch_add(int64_t n, const float* src, float* dst, cudaStream_t s);
 
 // dx row sums over the transpose edge list and the dY slice sums, one launch;
 // either part is skipped when its output is null (or S == 1 for dY).

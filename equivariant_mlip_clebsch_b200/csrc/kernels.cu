@@ -308,6 +308,15 @@ __global__ void __cluster_dims__(kVirCtas, 1, 1) __launch_bounds__(kVirThreads)
   cluster.sync();  // no CTA leaves (and frees its shared memory) before CTA 0 has read it
 }
 
+// dst += src over n floats (grid-stride), for the sums of the double
+// backward's terms.
+__global__ void __launch_bounds__(256) add_kernel(int64_t n, const float* __restrict__ src, float* __restrict__ dst) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int64_t stride = (int64_t)gridDim.x * 256;
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += stride) dst[i] += src[i];
+}
+
 // The backward's closing reductions in one launch.
 //  blocks [0, n_send): dx[j][c] = sum over sender j's edges of m[perm_T[t]][c].
 //    Two groups of 128 threads take the even and the odd positions t0 + 2k of
@@ -448,6 +457,12 @@ cudaError_t launch_edge_forces(int64_t n_atoms, const int32_t* rowptr, const int
 
 cudaError_t launch_edge_virial(int64_t E, const float* r, const float* G, float* V, cudaStream_t s) {
   return launch_pdl(edge_virial_kernel, dim3(kVirCtas), kVirThreads, s, E, r, G, V);
+}
+
+cudaError_t launch_add(int64_t n, const float* src, float* dst, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 8);
+  return launch_pdl(add_kernel, dim3((unsigned)blocks), 256, s, n, src, dst);
 }
 
 cudaError_t launch_bwd_reduce(int64_t n_send, int64_t width, const int32_t* rowptr_T, const int32_t* perm_T,

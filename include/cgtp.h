@@ -258,6 +258,34 @@ cgtp_status cgtp_plan_check_device_error(cgtp_plan plan, int* code);
 
 /* ---- graph utilities (host, no GPU needed) ----------------------------- */
 
+/* Second-order backward ("double backward"; LunaTP Table 11 lists its
+ * outputs h_x and h_y, and its Figure 5 trains through it with a Hessian
+ * objective; no formula is printed): given cotangents of the
+ * backward's outputs, h_x [n_send, d_in], h_W [E, n_weights], h_Y [E, d_edge]
+ * (each nullable = zero), the gradients of
+ *   S = <h_x, grad_x> + <h_W, grad_W> + <h_Y, grad_Y>
+ * (grad_* the backward at x, Y, W with cotangent grad_out) with respect to
+ * grad_out, x, W and Y.  The convolution is linear in each of x, Y, W, so
+ *   S = <grad_out, fwd(h_x, Y, W) + fwd(x, Y, h_W) + fwd(x, h_Y, W)>
+ * and the gradients are forwards and backwards of this library with one
+ * argument replaced by its cotangent:
+ *   gg_out = fwd(h_x, Y, W) + fwd(x, Y, h_W) + fwd(x, h_Y, W)
+ *   gx = bwd_x(Y, h_W) + bwd_x(h_Y, W)      gW = bwd_W(h_x, Y) + bwd_W(x, h_Y)
+ *   gY = bwd_Y(h_x, W) + bwd_Y(x, h_W)       (all with grad_out)
+ * Outputs gg_out [n_recv, d_out], gx, gW, gY (shapes of grad_out, x, W, Y;
+ * each nullable = not computed) are overwritten and must not alias inputs.
+ * workspace: cgtp_double_backward_workspace_size bytes, 256-byte aligned.
+ * Graph arrays as for cgtp_backward (rowptr_T/perm_T needed for gx).
+ * Errors: NULL, SIZE, ALIGN, WORKSPACE, DEVICE, CUDA. */
+cgtp_status cgtp_double_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                                                size_t* bytes);
+cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                                 const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
+                                 const int32_t* perm_T, const float* x, const float* Y, const float* W,
+                                 const float* grad_out, const float* h_x, const float* h_W, const float* h_Y,
+                                 float* gg_out, float* gx, float* gW, float* gY, void* workspace,
+                                 size_t workspace_bytes, cgtp_stream stream);
+
 /* Periodic neighbour list by cell list, FP64.  Host pointers.
  * Edge i <- j with image n (integers, |n_a| <= ceil(rc / box_a)) exists iff
  * (i,j,n) != (i,i,0) and |(pos_j + n*box) - pos_i|^2 < rc^2, each component

@@ -1,7 +1,7 @@
 """Pins of the oracle's double backward (the gradients of a functional of
 the backward's outputs: the second-order pass that force and Hessian
-training run through the CGTP convolution; LunaTP benchmarks it beside the
-forward and backward).
+training run through the CGTP convolution; LunaTP Table 11 lists its outputs
+h_x and h_y beside the forward's and backward's).
 
 S(g, x, Y, W) = <h_x, dx> + <h_W, dW> + <h_Y, dY>, with (dx, dW, dY) the
 oracle's backward, is linear in each of g, x, Y and W separately, so a

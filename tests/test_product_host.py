@@ -198,3 +198,28 @@ def test_binding_checks_tensors_before_the_abi(compile_only):
         C.edge_virial(r, r[:-1])
     with pytest.raises(ValueError, match="perm_T: expected"):
         C.edge_forces(rowptr, rowptr, col[:-1], r)
+
+
+def test_double_backward_host_checks(compile_only):
+    torch = pytest.importorskip("torch")
+    NULL, SIZE = 1, 6
+    lib = C._lib
+    plan = C.Plan("16x0e+16x1o", "1x0e+1x1o", "32x0e+32x1o", 6)
+    args = [None] * 16 + [0, None]
+    assert lib.cgtp_double_backward(None, 1, 1, 1, *args) == NULL
+    assert lib.cgtp_double_backward(plan._h, -1, 1, 1, *args) == SIZE
+    # the workspace holds the backward's and one scratch row set per output
+    n_recv, n_send, E = 7, 5, 40
+    need = plan.double_backward_workspace_size(n_recv, n_send, E)
+    floats = n_recv * plan.d_out + n_send * plan.d_in + E * plan.n_weights + E * plan.d_edge
+    assert need >= plan.workspace_size(n_recv, n_send, E) + 4 * floats
+    assert plan.double_backward_workspace_size(n_recv, n_send, 2 * E) > need
+    # the binding checks the cotangents like every other tensor
+    rowptr = torch.tensor([0, 2, 4, 5], dtype=torch.int32)
+    col = torch.tensor([1, 2, 0, 2, 1], dtype=torch.int32)
+    x, Y, W = torch.zeros(3, plan.d_in), torch.zeros(5, plan.d_edge), torch.zeros(5, plan.n_weights)
+    g = torch.zeros(3, plan.d_out)
+    with pytest.raises(ValueError, match="h_W: expected"):
+        plan.double_backward(rowptr, col, rowptr, col, x, Y, W, g, h_W=W[:4])
+    with pytest.raises(TypeError, match="h_Y: expected torch.float32"):
+        plan.double_backward(rowptr, col, rowptr, col, x, Y, W, g, h_Y=Y.double())
