@@ -320,6 +320,24 @@ def run_cgtp(args, rank, world, local_rank):
             b.record(stream)
     except C.CgtpError as e:
         virial_err = str(e)
+    # the double backward (all three cotangents), timed on its own
+    ev_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    dbl_err = None
+    try:
+        gen = torch.Generator(device=dev).manual_seed(3)
+        hx, hW, hY = (torch.randn(t.shape, device=dev, generator=gen) for t in (T["x"], T["W"], Y))
+        dgrads = tuple(torch.empty_like(t) for t in (T["g"], T["x"], T["W"], Y))
+        dws = torch.empty(max(plan.double_backward_workspace_size(N, N, E), 256), dtype=torch.uint8, device=dev)
+        for k in range(args.steps):
+            flush.zero_()
+            a, b = ev_d[k]
+            a.record(stream)
+            plan.double_backward(T["rowptr"], T["col"], T["rpt"], T["perm"], T["x"], Y, T["W"], T["g"],
+                                 h_x=hx, h_W=hW, h_Y=hY, grads=dgrads, workspace=dws)
+            b.record(stream)
+    except C.CgtpError as e:
+        dbl_err = str(e)
     torch.cuda.synchronize()
     clocks = sampler.stop()
     plan.check_device_error()
@@ -333,6 +351,13 @@ def run_cgtp(args, rank, world, local_rank):
                   "what": "edge_virial from grad_r (24 B/edge read), after the step (not in it)"}
     else:
         virial = {"error": virial_err}
+    if dbl_err is None:
+        dbl_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_d]))
+        double_backward = {"ms": dbl_ms, "edges_per_s": world * E / (dbl_ms * 1e-3),
+                           "what": "double_backward with h_x, h_W, h_Y (3 forwards, 3 backwards, adds), "
+                                   "after the step (not in it)"}
+    else:
+        double_backward = {"error": dbl_err}
     ms_step = max_over_ranks(float(np.sum(ms_steps)) / args.steps, world, dev)
     value = replica_value(world, E, ms_step)
     fwd_ms = float(np.mean(ms_fwd))
@@ -391,7 +416,7 @@ def run_cgtp(args, rank, world, local_rank):
                ms_per_step_launched=ms_eager,
                force_chain={"ms": force_ms, "edges_per_s": world * E / (force_ms * 1e-3),
                             "what": "sph_harm_backward + edge_forces after the step (not in it)"},
-               virial=virial,
+               virial=virial, double_backward=double_backward,
                roofline=roof, kernels=kernels, gpu_launches=int(gpu_launches), e2e=e2e, clocks=clocks)
     return res
 
