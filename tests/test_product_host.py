@@ -223,3 +223,23 @@ def test_double_backward_host_checks(compile_only):
         plan.double_backward(rowptr, col, rowptr, col, x, Y, W, g, h_W=W[:4])
     with pytest.raises(TypeError, match="h_Y: expected torch.float32"):
         plan.double_backward(rowptr, col, rowptr, col, x, Y, W, g, h_Y=Y.double())
+
+
+@pytest.mark.parametrize("lang,std", [("c", "-std=c99"), ("c++", "-std=c++11")])
+def test_header_is_plain_c(lang, std, tmp_path):
+    """include/cgtp.h compiles on its own as strict C99 and as C++11 (no CUDA
+    or torch headers needed by a caller of the C ABI)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    src = tmp_path / "use.c"
+    src.write_text('#include "cgtp.h"\n'
+                   "static cgtp_status (*destroy)(cgtp_plan) = cgtp_plan_destroy;\n"
+                   "static const char* (*name)(cgtp_status) = cgtp_status_string;\n"
+                   "int main(void) { return destroy(0) != CGTP_OK || name(CGTP_OK) == 0; }\n")
+    p = subprocess.run([cc, "-x", lang, std, "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.dirname(HEADER), "-c", str(src), "-o", str(tmp_path / "use.o")],
+                       capture_output=True, text=True)
+    assert p.returncode == 0, p.stderr
