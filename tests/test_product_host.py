@@ -243,3 +243,63 @@ def test_header_is_plain_c(lang, std, tmp_path):
                         "-I", os.path.dirname(HEADER), "-c", str(src), "-o", str(tmp_path / "use.o")],
                        capture_output=True, text=True)
     assert p.returncode == 0, p.stderr
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <stdlib.h>
+#include "cgtp.h"
+int main(void) {
+  /* one diamond-cubic cell (a = 5.43): every atom has 4 neighbours within 2.5 */
+  const double a = 5.43, box[3] = {5.43, 5.43, 5.43};
+  const double f[8][3] = {{0, 0, 0}, {0, .5, .5}, {.5, 0, .5}, {.5, .5, 0},
+                          {.25, .25, .25}, {.25, .75, .75}, {.75, .25, .75}, {.75, .75, .25}};
+  double pos[24];
+  for (int i = 0; i < 24; ++i) pos[i] = a * f[i / 3][i % 3];
+  int32_t rowptr[9], rpt[9];
+  int64_t E = 0;
+  if (cgtp_neighbor_list(8, pos, box, 2.5, rowptr, NULL, NULL, NULL, &E) != CGTP_OK) return 1;
+  int32_t* col = malloc(sizeof(int32_t) * E);
+  int32_t* perm = malloc(sizeof(int32_t) * E);
+  float* r = malloc(sizeof(float) * 3 * E);
+  if (cgtp_neighbor_list(8, pos, box, 2.5, rowptr, col, NULL, r, &E) != CGTP_OK) return 2;
+  if (cgtp_csr_transpose(8, 8, E, rowptr, col, rpt, perm) != CGTP_OK) return 3;
+  cgtp_plan plan = NULL;
+  if (cgtp_plan_create("16x0e+16x1o", "1x0e+1x1o", "32x0e+32x1o", 6, &plan) != CGTP_OK) {
+    fprintf(stderr, "%s\n", cgtp_last_error());
+    return 4;
+  }
+  int64_t din, de, dout, nw, np;
+  cgtp_plan_info(plan, &din, &de, &dout, &nw, &np);
+  printf("E=%lld rpt8=%d din=%lld de=%lld dout=%lld nw=%lld paths=%lld\n", (long long)E, rpt[8],
+         (long long)din, (long long)de, (long long)dout, (long long)nw, (long long)np);
+  cgtp_status bad = cgtp_plan_create("16x0e+", "1x0e", "16x0e", 6, &plan);
+  printf("bad=%s\n", cgtp_status_string(bad));
+  free(col);
+  free(perm);
+  free(r);
+  return 0;
+}
+"""
+
+
+def test_c_program_uses_the_abi(tmp_path):
+    """A C program linked against libcgtp.so alone (no Python, no torch)
+    builds a neighbour list and its transpose and a compile-only plan."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no host compiler")
+    from equivariant_mlip_clebsch_b200 import build as B
+    src = tmp_path / "prog.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "prog"
+    libdir = os.path.dirname(B.LIB)
+    p = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-o",
+                        str(exe), "-L", libdir, "-lcgtp", "-Wl,-rpath," + libdir], capture_output=True, text=True)
+    assert p.returncode == 0, p.stderr
+    env = dict(os.environ, CGTP_JIT_COMPILE_ONLY="1", CGTP_JIT_CACHE=str(tmp_path / "cache"))
+    run = subprocess.run([str(exe)], capture_output=True, text=True, env=env, timeout=600)
+    assert run.returncode == 0, run.stderr
+    assert run.stdout.splitlines() == ["E=32 rpt8=32 din=64 de=4 dout=128 nw=64 paths=4",
+                                       "bad=CGTP_ERR_IRREPS_PARSE"]
