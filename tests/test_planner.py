@@ -11,7 +11,9 @@ plans, no GPU):
 The same on irreps sets unlike the workloads, and the one refusal the
 planner has (a hidden irrep too wide for shared memory).  And, read from the
 generated source, every row copy into shared memory stays inside its global
-row and its staging slot, with bulk (TMA) copies on 16-byte boundaries.
+row and its staging slot, with bulk (TMA) copies on 16-byte boundaries, and
+the shared-memory regions are ordered, disjoint, aligned and within the
+planned size.
 """
 import re
 from collections import Counter
@@ -178,6 +180,35 @@ def _check_copies(src):
     return n, bad
 
 
+def _check_layout(src, smem, backward):
+    """Shared-memory layout of a generated kernel, from its defines: the
+    regions of a stage (W, x, Y, C-hat, dY partials) in order without
+    overlap; mbarriers and stage records below the first stage; the stage
+    ring, the grad_out buffers and the store staging after one another
+    within the planned dynamic shared memory; every offset a multiple of 16
+    bytes (TMA destinations)."""
+    d = _defines(src)
+    NB, NW, NS, DE = d["NB"], d["NW"], d["NSTAGE"], d["DE"]
+    off = [d["OFF_W"], d["OFF_X"], d["OFF_Y"], d["OFF_CH"], d["OFF_DY"]]
+    size = [4 * NB * d["WS"], 4 * NB * d["XS"], 4 * NB * DE, 4 * NB * d["CHS"],
+            4 * NW * NB * DE if backward else 0]
+    bad = [f"region {k}" for k in range(4) if off[k] + size[k] > off[k + 1]]
+    if off[4] + size[4] > d["STAGE_BYTES"]:
+        bad.append("dY partials past the stage")
+    if any(v % 16 for v in off + [d["STAGE_BYTES"], d["OFF_STAGE"], d["OFF_G"], d["OFF_WB"]]):
+        bad.append("offset not 16-byte aligned")
+    if 32 * NS + 32 > d["OFF_STAGE"]:  # full/empty barriers, grad_out barriers, stage records
+        bad.append("barriers past the first stage")
+    if d["OFF_STAGE"] + NS * d["STAGE_BYTES"] > d["OFF_G"]:
+        bad.append("stage ring past the grad_out buffers")
+    gbytes = d.get("GBUF", 0) * 4 * d.get("GS", 0) if backward else 0
+    if d["OFF_G"] + gbytes > d["OFF_WB"]:
+        bad.append("grad_out buffers past the store staging")
+    if not (d["OFF_WB"] + 4 * NW * d.get("WB", 0) <= smem <= 227 * 1024):
+        bad.append(f"end {d['OFF_WB'] + 4 * NW * d.get('WB', 0)} vs planned {smem}")
+    return bad
+
+
 @pytest.mark.parametrize("irreps", [WL.CONFIGS[n] for n in NAMES] + [
     dict(irreps_in=a, irreps_edge=b, irreps_out=c) for a, b, c in ODD], ids=NAMES + [f"odd{k}" for k in range(len(ODD))])
 def test_generated_copies_stay_in_bounds(irreps, compile_only, monkeypatch, tmp_path):
@@ -185,12 +216,17 @@ def test_generated_copies_stay_in_bounds(irreps, compile_only, monkeypatch, tmp_
     generated source (checked here so that a mistake fails on the CPU rather
     than faulting a GPU)."""
     monkeypatch.setenv("CGTP_DUMP_SOURCE", str(tmp_path))
-    C.Plan(irreps["irreps_in"], irreps["irreps_edge"], irreps["irreps_out"], 6)
+    plan = C.Plan(irreps["irreps_in"], irreps["irreps_edge"], irreps["irreps_out"], 6)
+    smem = {k: int(v) for k, v in re.findall(r"^(forward|backward): .* smem=(\d+)", plan.describe(), re.M)}
     files = sorted(p.name for p in tmp_path.iterdir())
     assert files == ["bwd.cu", "bwd_er.cu", "fwd.cu"]
     for f in files:
-        n, bad = _check_copies((tmp_path / f).read_text())
+        src = (tmp_path / f).read_text()
+        n, bad = _check_copies(src)
         assert n > 0 and not bad, (f, bad[:3])
+        bwd = f.startswith("bwd")
+        bad = _check_layout(src, smem["backward" if bwd else "forward"], bwd)
+        assert not bad, (f, bad)
 
 
 def test_copy_check_catches_planted_mistakes():
@@ -209,3 +245,21 @@ def test_copy_check_catches_planted_mistakes():
     for p in planted:
         n, bad = _check_copies(head + p)
         assert bad, p
+
+
+def test_layout_check_catches_planted_mistakes():
+    # W 1024 B, x 512, Y 144, C-hat 256, dY partials 576 per stage; two stages
+    good = {"NB": 4, "NW": 4, "NSTAGE": 2, "DE": 9, "WS": 64, "XS": 32, "CHS": 16, "OFF_W": 0, "OFF_X": 1024,
+            "OFF_Y": 1536, "OFF_CH": 1792, "OFF_DY": 2048, "STAGE_BYTES": 2688, "OFF_STAGE": 256,
+            "OFF_G": 5632, "GS": 128, "GBUF": 2, "OFF_WB": 6656, "WB": 32}
+    text = lambda d: "".join(f"#define {k} {v}\n" for k, v in d.items())
+    assert _check_layout(text(good), 7168, True) == []
+    for key, val, smem in (("OFF_X", 768, 7168),      # W region overlaps x
+                           ("OFF_Y", 1544, 7168),     # not 16-byte aligned
+                           ("OFF_G", 5120, 7168),     # stage ring overlaps grad_out
+                           ("OFF_WB", 6400, 7168),    # grad_out buffers overlap staging
+                           ("OFF_STAGE", 64, 7168),   # barriers overlap stage 0
+                           ("WB", 64, 7168)):         # past the planned size
+        d = dict(good)
+        d[key] = val
+        assert _check_layout(text(d), smem, True), key
