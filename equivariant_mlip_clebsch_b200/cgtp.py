@@ -1,8 +1,10 @@
-"""Python binding of libcgtp (include/cgtp.h): argument marshalling only.
+"""Python binding of libcgtp (include/cgtp.h): argument checks and
+marshalling only.
 
 Every step of the convolution runs in the library's CUDA kernels; torch is used
-for device memory and the current stream.  There is no fallback: if the
-library is missing this module raises on import.
+for device memory and the current stream.  Each tensor's dtype, element count
+and device are checked before its pointer crosses the ABI.  There is no
+fallback: if the library is missing this module raises on import.
 """
 from __future__ import annotations
 
