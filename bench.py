@@ -318,7 +318,7 @@ def run_cgtp(args, rank, world, local_rank):
             a.record(stream)
             C.edge_virial(T["r"], gr, virial=Vo)
             b.record(stream)
-    except C.CgtpError as e:
+    except (C.CgtpError, ValueError, TypeError) as e:  # reported, the headline stands
         virial_err = str(e)
     # the double backward (all three cotangents), timed on its own
     ev_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -336,7 +336,7 @@ def run_cgtp(args, rank, world, local_rank):
             plan.double_backward(T["rowptr"], T["col"], T["rpt"], T["perm"], T["x"], Y, T["W"], T["g"],
                                  h_x=hx, h_W=hW, h_Y=hY, grads=dgrads, workspace=dws)
             b.record(stream)
-    except C.CgtpError as e:
+    except (C.CgtpError, ValueError, TypeError) as e:  # reported, the headline stands
         dbl_err = str(e)
     torch.cuda.synchronize()
     clocks = sampler.stop()
