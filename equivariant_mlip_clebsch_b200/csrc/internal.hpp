@@ -18,11 +18,17 @@ namespace cgtp {
 void set_error(const std::string& msg);
 cgtp_status fail(cgtp_status s, const std::string& msg);
 
+// A failed runtime call returns CGTP_ERR_CUDA and clears the runtime's
+// per-thread last error, so that a non-sticky failure here (an invalid launch
+// configuration, say) is reported once, through the status, and not again by
+// the caller's next unrelated CUDA check.
 #define CGTP_CUDA_TRY(expr)                                                          \
   do {                                                                               \
     cudaError_t _e = (expr);                                                         \
-    if (_e != cudaSuccess)                                                           \
+    if (_e != cudaSuccess) {                                                         \
+      (void)cudaGetLastError();                                                      \
       return ::cgtp::fail(CGTP_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(_e)); \
+    }                                                                                \
   } while (0)
 
 // ---------------------------------------------------------------- irreps
