@@ -537,9 +537,11 @@ def ncu_traffic(name, kernel, plan):
 # --------------------------------------------------------------------------
 # the oracle on the host cores: cpu_baseline and the reference arm
 # --------------------------------------------------------------------------
-def oracle_sample(name: str, budget_s: float, rows: int | None = None):
-    """Time the FP64 oracle (forward + backward, all three gradients) on the
-    sub-graph of the first ``rows`` receivers, repeated until ``budget_s``."""
+def oracle_sample(name: str, budget_s: float, rows: int | None = None, nthreads: int = 0,
+                  backward: bool = True):
+    """Time the FP64 oracle (forward + backward, all three gradients; the
+    forward alone with backward=False) on the sub-graph of the first ``rows``
+    receivers, repeated until ``budget_s``; nthreads 0 = all host cores."""
     import oracle as O
     c = WL.CONFIGS[name]
     pos, box = WL.si_diamond(c["cells"], c["sigma"], 0)
@@ -556,30 +558,31 @@ def oracle_sample(name: str, budget_s: float, rows: int | None = None):
         rows = min(N, 32)
         rp = rowptr[:rows + 1]
         t = time.time()
-        _oracle_pass(O, P, rp, col, vec, N, std, pos)
+        _oracle_pass(O, P, rp, col, vec, N, std, pos, nthreads, backward)
         dt = max(time.time() - t, 1e-3)
         rows = int(min(N, max(8, rows * (budget_s / 3) / dt)))
     rp = rowptr[:rows + 1]
     nE = int(rp[-1])
     reps, t0 = 0, time.time()
     while True:
-        _oracle_pass(O, P, rp, col, vec, N, std, pos)
+        _oracle_pass(O, P, rp, col, vec, N, std, pos, nthreads, backward)
         reps += 1
         if time.time() - t0 >= budget_s or reps >= 50:
             break
     dt = time.time() - t0
     return {"edges_per_s": reps * nE / dt, "rows": rows, "edges": nE, "reps": reps, "seconds": dt,
-            "cores": O.max_threads()}
+            "cores": nthreads or O.max_threads()}
 
 
-def _oracle_pass(O, P, rp, col, vec, N, std, pos):
+def _oracle_pass(O, P, rp, col, vec, N, std, pos, nthreads=0, backward=True):
     E = int(rp[-1])
     x = WL.draw_x(N, P.D_in)
     W = WL.draw_W(E, P.U, std)
     g = WL.draw_g(len(rp) - 1, P.D_out)
     Y = O.sph_harm(P.L, vec[:E].astype(np.float32))
-    O.forward(P, rp, col[:E], x, Y, W)
-    O.backward(P, rp, col[:E], N, x, Y, W, g)
+    O.forward(P, rp, col[:E], x, Y, W, nthreads=nthreads)
+    if backward:
+        O.backward(P, rp, col[:E], N, x, Y, W, g, nthreads=nthreads)
 
 
 def run_reference(args, rank, world):
@@ -647,6 +650,12 @@ def main():
                                "kind": "oracle",
                                "sample": f"receivers 0..{s['rows'] - 1} ({s['edges']} edges), harmonics + "
                                          f"forward + backward, {s['reps']} passes in {s['seconds']:.1f}s, FP64"}
+        # the same step on one host thread, and the forward alone on all cores
+        for key, kw in (("single_thread", dict(nthreads=1)), ("forward_only", dict(backward=False))):
+            v = oracle_sample(args.config, args.cpu_budget / 4, **kw)
+            res["cpu_baseline"][key] = {"value": v["edges_per_s"], "unit": "edges/s", "cores": v["cores"],
+                                        "sample": f"receivers 0..{v['rows'] - 1} ({v['edges']} edges), "
+                                                  f"{v['reps']} passes in {v['seconds']:.1f}s"}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

@@ -45,9 +45,24 @@ static int g_fault = 0;
 void orc_set_fault(int f) { g_fault = f; }
 int orc_get_fault(void) { return g_fault; }
 
+/* Threads of a parallel loop: the caller's count when positive, else the
+ * process default read once (never changed here, so a one-thread call does
+ * not lower later ones).  Loops write disjoint outputs, so results do not
+ * depend on the count. */
+static int orc_threads(int nthreads) {
+#ifdef _OPENMP
+  static int deflt = 0;
+  if (deflt == 0) deflt = omp_get_max_threads();
+  return nthreads > 0 ? nthreads : deflt;
+#else
+  (void)nthreads;
+  return 1;
+#endif
+}
+
 int orc_max_threads(void) {
 #ifdef _OPENMP
-  return omp_get_max_threads();
+  return orc_threads(0);
 #else
   return 1;
 #endif
@@ -446,12 +461,9 @@ enum { PI_L1, PI_L2, PI_L3, PI_MUL, PI_XOFF, PI_K0, PI_OOFF, PI_COFF, PI_N };
 void orc_forward(int64_t n_recv, const int64_t* rowptr, const int32_t* col, int D_in, int D_e,
                  int D_out, int U, const double* x, const double* Y, const double* W, int npaths,
                  const int32_t* paths, const double* cg, double* out, int nthreads) {
-#ifdef _OPENMP
-  if (nthreads > 0) omp_set_num_threads(nthreads);
-#else
-  (void)nthreads;
-#endif
-#pragma omp parallel for schedule(dynamic, 4)
+  const int nt = orc_threads(nthreads);
+  (void)nt;
+#pragma omp parallel for schedule(dynamic, 4) num_threads(nt)
   for (int64_t i = 0; i < n_recv; ++i) {
     double* oi = out + i * (int64_t)D_out;
     for (int t = 0; t < D_out; ++t) oi[t] = 0.0;
@@ -494,17 +506,14 @@ void orc_backward(int64_t n_recv, int64_t n_send, int64_t E, const int64_t* rowp
                   const double* Y, const double* W, const double* g, int npaths,
                   const int32_t* paths, const double* cg, double* grad_x, double* grad_W,
                   double* grad_Y, int nthreads) {
-#ifdef _OPENMP
-  if (nthreads > 0) omp_set_num_threads(nthreads);
-#else
-  (void)nthreads;
-#endif
+  const int nt = orc_threads(nthreads);
+  (void)nt;
   int64_t* recv_of = malloc(sizeof(int64_t) * (E > 0 ? E : 1));
   for (int64_t i = 0; i < n_recv; ++i)
     for (int64_t e = rowptr[i]; e < rowptr[i + 1]; ++e) recv_of[e] = i;
 
   if (grad_W || grad_Y) {
-#pragma omp parallel for schedule(dynamic, 64)
+#pragma omp parallel for schedule(dynamic, 64) num_threads(nt)
     for (int64_t e = 0; e < E; ++e) {
       int64_t i = recv_of[e], j = col[e];
       if (grad_W)
@@ -545,7 +554,7 @@ void orc_backward(int64_t n_recv, int64_t n_send, int64_t E, const int64_t* rowp
     for (int64_t j = 0; j < n_send; ++j) fill[j] = tptr[j];
     for (int64_t e = 0; e < E; ++e) tedge[fill[col[e]]++] = e;
     free(fill);
-#pragma omp parallel for schedule(dynamic, 4)
+#pragma omp parallel for schedule(dynamic, 4) num_threads(nt)
     for (int64_t j = 0; j < n_send; ++j) {
       double* dxj = grad_x + j * (int64_t)D_in;
       for (int t = 0; t < D_in; ++t) dxj[t] = 0.0;
