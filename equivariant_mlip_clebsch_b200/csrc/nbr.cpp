@@ -110,8 +110,8 @@ static void visit_row(const CellList& L, const double* pos, const double* box, d
           const double dx = (pos[3 * j] + (double)n[0] * box[0]) - pos[3 * i];
           const double dy = (pos[3 * j + 1] + (double)n[1] * box[1]) - pos[3 * i + 1];
           const double dz = (pos[3 * j + 2] + (double)n[2] * box[2]) - pos[3 * i + 2];
-          const double d2 = dx * dx + dy * dy + dz * dz;
-          if (d2 < rc2) fn(j, n, dx, dy, dz);
+          const double r2 = dx * dx + dy * dy + dz * dz;
+          if (r2 < rc2) fn(j, n, dx, dy, dz);
         }
       }
 }
