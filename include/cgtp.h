@@ -144,7 +144,8 @@ cgtp_status cgtp_sph_harm(cgtp_plan plan, int64_t E, const float* r, float* Y,
  * grad_r is overwritten; r = 0 gives grad_r = 0.  Forces are minus the
  * position gradient of the energy (BranchIP page, its force definition).
  * The pages print no formula for this step; it is the chain rule through
- * the harmonics of cgtp_sph_harm.  Errors: NULL, SIZE, ALIGN, DEVICE, CUDA. */
+ * the harmonics of cgtp_sph_harm.  Errors: NULL, SIZE, ALIGN, CUDA (also for a
+ * plan of another device or a compile-only plan). */
 cgtp_status cgtp_sph_harm_backward(cgtp_plan plan, int64_t E, const float* r, const float* grad_Y,
                                    float* grad_r, cgtp_stream stream);
 
@@ -276,7 +277,8 @@ cgtp_status cgtp_plan_check_device_error(cgtp_plan plan, int* code);
  * each nullable = not computed) are overwritten and must not alias inputs.
  * workspace: cgtp_double_backward_workspace_size bytes, 256-byte aligned.
  * Graph arrays as for cgtp_backward (rowptr_T/perm_T needed for gx).
- * Errors: NULL, SIZE, ALIGN, WORKSPACE, DEVICE, CUDA. */
+ * Errors: NULL, SIZE, ALIGN, WORKSPACE, CUDA (also for a plan of another
+ * device or a compile-only plan). */
 cgtp_status cgtp_double_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
                                                 size_t* bytes);
 cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
