@@ -303,3 +303,14 @@ def test_c_program_uses_the_abi(tmp_path):
     assert run.returncode == 0, run.stderr
     assert run.stdout.splitlines() == ["E=32 rpt8=32 din=64 de=4 dout=128 nw=64 paths=4",
                                        "bad=CGTP_ERR_IRREPS_PARSE"]
+
+
+def test_header_error_lists_name_real_statuses():
+    """Every status an entry's "Errors:" list names exists in cgtp_status."""
+    text = open(HEADER).read()
+    enum = set(re.findall(r"CGTP_ERR_(\w+)\s*=", text))
+    lists = re.findall(r"Errors:\s*([A-Z_, ]+)", text)
+    assert lists
+    for lst in lists:
+        for name in re.findall(r"[A-Z][A-Z_]+", lst):
+            assert name in enum, (name, lst)
