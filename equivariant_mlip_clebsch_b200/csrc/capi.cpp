@@ -180,9 +180,14 @@ cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge, con
       if (cudaMalloc(&P->d_err, sizeof(int)) != cudaSuccess) return fail(CGTP_ERR_OOM, "cudaMalloc");
       CGTP_CUDA_TRY(cudaMemset(P->d_err, 0, sizeof(int)));
     }
-    st = build_forward(*P);
+    st = build_forward(*P);  // leaves the forward compiling on a host thread
     if (st == CGTP_OK) st = build_backward(*P);
+    if (st == CGTP_OK)
+      st = finish_forward(*P);
+    else
+      P->fwd_pending.reset();  // joins; its result is not needed
   } catch (const std::exception& e) {
+    P->fwd_pending.reset();
     destroy_plan_device(*P);
     return fail(CGTP_ERR_OOM, std::string("exception in plan create: ") + e.what());
   }

@@ -22,8 +22,10 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <memory>
 #include <numeric>
 #include <sstream>
+#include <thread>
 #include <tuple>
 
 #include "codegen_common.hpp"
@@ -435,22 +437,49 @@ cgtp_status build_forward(Plan& P) {
   bool fixed = false;
   const int mb0 = initial_min_blocks(K.smem, &fixed);
   const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
-  std::string src;
-  for (int mb = mb0; mb >= mb_floor; --mb) {
-    src = gen_fwd_source(P, SL, K, name, mb);
-    P.fwd.threads = (F.nw + 2) * 32;
-    P.fwd.smem = K.smem;
-    cgtp_status cst = jit_compile(src, name, P.fwd);
-    if (cst != CGTP_OK) return cst;
-    if (mb == mb_floor || max_spill_bytes(P.fwd.log) <= 64) break;
-    jit_unload(P.fwd);
+  // The compile runs on a host thread while the backward is planned and
+  // compiled (NVRTC needs no CUDA context); finish_forward joins and loads.
+  // It reads only the plan's paths, irreps and forward fields, all set by now.
+  auto pend = std::make_unique<PendingCompile>();
+  PendingCompile* pc = pend.get();
+  const Plan& CP = P;
+  auto body = [pc, &CP, SL, K, mb0, mb_floor, name]() {
+    try {
+      for (int mb = mb0; mb >= mb_floor; --mb) {
+        pc->src = gen_fwd_source(CP, SL, K, name, mb);
+        pc->st = jit_build(pc->src, name, pc->bin);
+        if (pc->st != CGTP_OK || mb == mb_floor || max_spill_bytes(pc->bin.log) <= 64) break;
+      }
+    } catch (const std::exception& e) {
+      pc->st = CGTP_ERR_OOM;
+      pc->bin.err = std::string("exception while building the forward: ") + e.what();
+    }
+  };
+  try {
+    pend->th = std::thread(body);
+  } catch (...) {
+    body();
   }
   P.fwd.threads = (F.nw + 2) * 32;
   P.fwd.smem = K.smem;
+  P.fwd_pending = std::move(pend);
+  return CGTP_OK;
+}
+
+cgtp_status finish_forward(Plan& P) {
+  if (!P.fwd_pending) return CGTP_OK;
+  std::unique_ptr<PendingCompile> pc = std::move(P.fwd_pending);
+  pc->join();
+  if (pc->st != CGTP_OK) {
+    set_error(pc->bin.err);
+    return pc->st;
+  }
+  const cgtp_status st = jit_load(pc->bin, "cgtp_fwd", P.fwd);
+  if (st != CGTP_OK) return st;
   if (const char* d = std::getenv("CGTP_DUMP_SOURCE")) {
     FILE* f = std::fopen((std::string(d) + "/fwd.cu").c_str(), "w");
     if (f) {
-      std::fputs(src.c_str(), f);
+      std::fputs(pc->src.c_str(), f);
       std::fclose(f);
     }
   }

@@ -8,6 +8,7 @@
 #include <memory>
 #include <mutex>
 #include <string>
+#include <thread>
 #include <vector>
 
 #include "cgtp.h"
@@ -86,6 +87,26 @@ struct JitKernel {
   int blocks_per_sm = 0;        // resident CTAs per SM (occupancy query)
 };
 
+// A compiled kernel before loading: building needs no CUDA context and may
+// run on any thread; loading uses the calling thread's current context.
+struct JitBinary {
+  std::string cubin, log, err;  // err: the failing thread's message
+  unsigned long long hash = 0;
+};
+
+// A kernel compiling on a host thread during plan creation; the destructor
+// joins, so no exit path leaves the thread running.
+struct PendingCompile {
+  std::thread th;
+  std::string src;
+  JitBinary bin;
+  cgtp_status st = CGTP_OK;
+  void join() {
+    if (th.joinable()) th.join();
+  }
+  ~PendingCompile() { join(); }
+};
+
 struct FwdConfig {
   int S = 1;             // slices (each CTA walks them in turn)
   int nw = 0;            // consumer warps per CTA
@@ -140,6 +161,9 @@ struct Plan {
   std::vector<cudaEvent_t> tpool;
   bool host_only = false;  // built for compile checks only: no device state
   int L_sh = 0;
+  // the forward's compile while the backward is built (reads the fields
+  // above; the last member, so it is joined before they are destroyed)
+  std::unique_ptr<PendingCompile> fwd_pending;
 };
 
 cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
@@ -153,15 +177,10 @@ cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
 cgtp_status build_paths(Plan& P);
 cgtp_status build_forward(Plan& P);
 cgtp_status build_backward(Plan& P);
+cgtp_status finish_forward(Plan& P);  // joins the forward's compile and loads it
 void destroy_plan_device(Plan& P);
 
 // JIT
-// A compiled kernel before loading: building needs no CUDA context and may
-// run on any thread; loading uses the calling thread's current context.
-struct JitBinary {
-  std::string cubin, log, err;  // err: the failing thread's message
-  unsigned long long hash = 0;
-};
 cgtp_status jit_build(const std::string& src, const std::string& name, JitBinary& b);
 cgtp_status jit_load(const JitBinary& b, const std::string& name, JitKernel& k);
 cgtp_status jit_compile(const std::string& src, const std::string& name, JitKernel& k);
