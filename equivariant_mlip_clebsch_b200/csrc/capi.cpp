@@ -9,6 +9,7 @@
 #include <cstring>
 #include <string>
 
+#include "double_backward.hpp"
 #include "internal.hpp"
 
 namespace cgtp {
@@ -576,53 +577,39 @@ cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send,
   if (!workspace || workspace_bytes < L.total)
     return fail(CGTP_ERR_WORKSPACE, "workspace of " + std::to_string(L.total) + " bytes required");
   if ((uintptr_t)workspace & 255) return fail(CGTP_ERR_ALIGN, "workspace must be 256-byte aligned");
-  cudaStream_t s = (cudaStream_t)stream;
   char* ws = reinterpret_cast<char*>(workspace);
   float* tF = reinterpret_cast<float*>(ws + L.f);
   float* tX = reinterpret_cast<float*>(ws + L.x);
   float* tW = reinterpret_cast<float*>(ws + L.w);
   float* tY = reinterpret_cast<float*>(ws + L.y);
-  // S = <g, fwd(h_x, Y, W) + fwd(x, Y, h_W) + fwd(x, h_Y, W)>: one term per
-  // given cotangent, each a forward or backward with one argument replaced
-  const float* tx[3] = {h_x, x, x};
-  const float* ty[3] = {Y, Y, h_Y};
-  const float* tw[3] = {W, h_W, W};
-  const bool on[3] = {h_x != nullptr, h_W != nullptr, h_Y != nullptr};
-  if (gg_out && n_recv > 0) {  // d S / d grad_out: the three forwards
-    bool written = false;
-    for (int k = 0; k < 3; ++k) {
-      if (!on[k]) continue;
-      float* dst = written ? tF : gg_out;
-      st = cgtp_forward(plan, n_recv, n_send, E, rowptr, col, tx[k], ty[k], tw[k], dst, stream);
-      if (st != CGTP_OK) return st;
-      if (written) CGTP_CUDA_TRY(launch_add(n_recv * P->D_out, tF, gg_out, s));
-      written = true;
+  // the term structure (double_backward.hpp) on the library's kernels
+  struct DeviceOps {
+    cgtp_plan plan;
+    int64_t n_recv, n_send, E;
+    const int32_t *rowptr, *col, *rowptr_T, *perm_T;
+    const float* g;
+    void* bws;
+    size_t bw_bytes;
+    cgtp_stream stream;
+    int forward(const float* xx, const float* yy, const float* ww, float* out) {
+      return cgtp_forward(plan, n_recv, n_send, E, rowptr, col, xx, yy, ww, out, stream);
     }
-    if (!written) CGTP_CUDA_TRY(cudaMemsetAsync(gg_out, 0, (size_t)n_recv * P->D_out * sizeof(float), s));
-  }
-  // d S / d (x, W, Y): term k gives the gradients of the two arguments it
-  // kept (h_x: W and Y; h_W: x and Y; h_Y: x and W)
-  bool wx = false, ww = false, wy = false;
-  for (int k = 0; k < 3; ++k) {
-    if (!on[k]) continue;
-    float* ox = (k != 0 && gx) ? (wx ? tX : gx) : nullptr;
-    float* ow = (k != 1 && gW) ? (ww ? tW : gW) : nullptr;
-    float* oy = (k != 2 && gY) ? (wy ? tY : gY) : nullptr;
-    if (!ox && !ow && !oy) continue;
-    st = backward_impl(plan, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, tx[k], ty[k], tw[k], grad_out, ox,
-                       ow, oy, ws + L.bwd, L.f - L.bwd, stream, true);
-    if (st != CGTP_OK) return st;
-    if (ox == tX) CGTP_CUDA_TRY(launch_add(n_send * P->D_in, tX, gx, s));
-    if (ow == tW) CGTP_CUDA_TRY(launch_add(E * P->U, tW, gW, s));
-    if (oy == tY) CGTP_CUDA_TRY(launch_add(E * P->D_e, tY, gY, s));
-    wx = wx || ox;
-    ww = ww || ow;
-    wy = wy || oy;
-  }
-  if (gx && !wx && n_send > 0) CGTP_CUDA_TRY(cudaMemsetAsync(gx, 0, (size_t)n_send * P->D_in * sizeof(float), s));
-  if (gW && !ww && E > 0) CGTP_CUDA_TRY(cudaMemsetAsync(gW, 0, (size_t)E * P->U * sizeof(float), s));
-  if (gY && !wy && E > 0) CGTP_CUDA_TRY(cudaMemsetAsync(gY, 0, (size_t)E * P->D_e * sizeof(float), s));
-  return CGTP_OK;
+    int backward(const float* xx, const float* yy, const float* ww, float* ox, float* ow, float* oy) {
+      return backward_impl(plan, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, xx, yy, ww, g, ox, ow, oy, bws,
+                           bw_bytes, stream, true);
+    }
+    int add(float* dst, const float* src, int64_t n) {
+      CGTP_CUDA_TRY(launch_add(n, src, dst, (cudaStream_t)stream));
+      return CGTP_OK;
+    }
+    int zero(float* dst, int64_t n) {
+      CGTP_CUDA_TRY(cudaMemsetAsync(dst, 0, (size_t)n * sizeof(float), (cudaStream_t)stream));
+      return CGTP_OK;
+    }
+  } ops{plan, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, grad_out, ws + L.bwd, L.f - L.bwd, stream};
+  const DbwdDims dims{n_recv, n_send, E, P->D_in, P->D_e, P->D_out, P->U};
+  return (cgtp_status)compose_double_backward(ops, dims, x, Y, W, h_x, h_W, h_Y, gg_out, gx, gW, gY, tF, tX, tW,
+                                              tY);
 }
 
 cgtp_status cgtp_neighbor_list(int64_t N, const double* pos, const double* box, double rc,

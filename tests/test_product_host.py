@@ -314,3 +314,121 @@ def test_header_error_lists_name_real_statuses():
     for lst in lists:
         for name in re.findall(r"[A-Z][A-Z_]+", lst):
             assert name in enum, (name, lst)
+
+
+COMPOSE_HOST = r"""
+#include <cstdint>
+#include <vector>
+#include "double_backward.hpp"
+extern "C" {
+void orc_forward(int64_t, const int64_t*, const int32_t*, int, int, int, int, const double*, const double*,
+                 const double*, int, const int32_t*, const double*, double*, int);
+void orc_backward(int64_t, int64_t, int64_t, const int64_t*, const int32_t*, int, int, int, int, const double*,
+                  const double*, const double*, const double*, int, const int32_t*, const double*, double*,
+                  double*, double*, int);
+}
+struct HostOps {  // the oracle's forward and backward on host buffers
+  cgtp::DbwdDims d;
+  const int64_t* rowptr;
+  const int32_t* col;
+  int npaths;
+  const int32_t* paths;
+  const double* cg;
+  const float* g;
+  static std::vector<double> up(const float* p, int64_t n) { return std::vector<double>(p, p + n); }
+  static void down(const std::vector<double>& v, float* p) {
+    for (size_t i = 0; i < v.size(); ++i) p[i] = (float)v[i];
+  }
+  int forward(const float* x, const float* Y, const float* W, float* out) {
+    auto xd = up(x, d.n_send * d.D_in), yd = up(Y, d.E * d.D_e), wd = up(W, d.E * d.U);
+    std::vector<double> o(d.n_recv * d.D_out);
+    orc_forward(d.n_recv, rowptr, col, (int)d.D_in, (int)d.D_e, (int)d.D_out, (int)d.U, xd.data(), yd.data(),
+                wd.data(), npaths, paths, cg, o.data(), 0);
+    down(o, out);
+    return 0;
+  }
+  int backward(const float* x, const float* Y, const float* W, float* ox, float* ow, float* oy) {
+    auto xd = up(x, d.n_send * d.D_in), yd = up(Y, d.E * d.D_e), wd = up(W, d.E * d.U);
+    auto gd = up(g, d.n_recv * d.D_out);
+    std::vector<double> vx(ox ? d.n_send * d.D_in : 0), vw(ow ? d.E * d.U : 0), vy(oy ? d.E * d.D_e : 0);
+    orc_backward(d.n_recv, d.n_send, d.E, rowptr, col, (int)d.D_in, (int)d.D_e, (int)d.D_out, (int)d.U, xd.data(),
+                 yd.data(), wd.data(), gd.data(), npaths, paths, cg, ox ? vx.data() : nullptr,
+                 ow ? vw.data() : nullptr, oy ? vy.data() : nullptr, 0);
+    if (ox) down(vx, ox);
+    if (ow) down(vw, ow);
+    if (oy) down(vy, oy);
+    return 0;
+  }
+  int add(float* dst, const float* src, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) dst[i] += src[i];
+    return 0;
+  }
+  int zero(float* dst, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) dst[i] = 0.f;
+    return 0;
+  }
+};
+extern "C" int run_compose(const int64_t* dims, const int64_t* rowptr, const int32_t* col, int npaths,
+                           const int32_t* paths, const double* cg, const float* x, const float* Y, const float* W,
+                           const float* g, const float* h_x, const float* h_W, const float* h_Y, float* gg,
+                           float* gx, float* gW, float* gY) {
+  const cgtp::DbwdDims d{dims[0], dims[1], dims[2], dims[3], dims[4], dims[5], dims[6]};
+  std::vector<float> tF(d.n_recv * d.D_out), tX(d.n_send * d.D_in), tW(d.E * d.U), tY(d.E * d.D_e);
+  HostOps ops{d, rowptr, col, npaths, paths, cg, g};
+  return cgtp::compose_double_backward(ops, d, x, Y, W, h_x, h_W, h_Y, gg, gx, gW, gY, tF.data(), tX.data(),
+                                       tW.data(), tY.data());
+}
+"""
+
+
+@pytest.mark.parametrize("keys", [(), ("h_x",), ("h_W",), ("h_Y",), ("h_x", "h_W"), ("h_W", "h_Y"),
+                                  ("h_x", "h_Y"), ("h_x", "h_W", "h_Y")])
+def test_double_backward_composition_on_host(keys, tmp_path):
+    """The library's double-backward term structure (csrc/double_backward.hpp,
+    the code cgtp_double_backward runs on the kernels) driven by the oracle's
+    forward and backward on the host equals the oracle's own composition:
+    which term writes an output in place, which adds through scratch, which
+    output is zeroed.  Outputs start as NaN; two are left out in one case."""
+    import ctypes
+    import shutil
+    import subprocess
+    if shutil.which("g++") is None:
+        pytest.skip("no host compiler")
+    src = tmp_path / "compose.cpp"
+    src.write_text(COMPOSE_HOST)
+    so = tmp_path / "libcompose.so"
+    orc = O.build()
+    csrc = os.path.join(os.path.dirname(os.path.dirname(__file__)), "equivariant_mlip_clebsch_b200", "csrc")
+    p = subprocess.run(["g++", "-std=c++17", "-O1", "-shared", "-fPIC", "-I", csrc, str(src), "-o", str(so),
+                        orc, "-Wl,-rpath," + os.path.dirname(orc)], capture_output=True, text=True)
+    assert p.returncode == 0, p.stderr
+    lib = ctypes.CDLL(str(so))
+    rng = np.random.default_rng(5)
+    P = O.enumerate_paths("16x0e+16x1o", "1x0e+1x1o", "32x0e+32x1o")
+    n_recv, n_send = 7, 6
+    deg = rng.integers(0, 5, size=n_recv)
+    rowptr = np.concatenate([[0], np.cumsum(deg)]).astype(np.int64)
+    E = int(rowptr[-1])
+    col = rng.integers(0, n_send, size=E).astype(np.int32)
+    f32 = lambda *s: rng.standard_normal(s).astype(np.float32)
+    x, Y, W, g = f32(n_send, P.D_in), f32(E, P.D_e), f32(E, P.U), f32(n_recv, P.D_out)
+    h = {"h_x": f32(n_send, P.D_in), "h_W": f32(E, P.U), "h_Y": f32(E, P.D_e)}
+    h = {k: (v if k in keys else None) for k, v in h.items()}
+    want = {"gg": (n_recv, P.D_out), "gx": (n_send, P.D_in), "gW": (E, P.U), "gY": (E, P.D_e)}
+    skip = {"gx", "gY"} if keys == ("h_x", "h_W") else set()  # outputs not asked for
+    outs = {k: (None if k in skip else np.full(s, np.nan, dtype=np.float32)) for k, s in want.items()}
+    ptr = lambda a: None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+    dims = np.array([n_recv, n_send, E, P.D_in, P.D_e, P.D_out, P.U], dtype=np.int64)
+    table = np.ascontiguousarray(P.table, dtype=np.int32)
+    cg = np.ascontiguousarray(P.cg, dtype=np.float64)
+    lib.run_compose.restype = ctypes.c_int
+    rc = lib.run_compose(ptr(dims), ptr(rowptr), ptr(col), ctypes.c_int(P.npaths), ptr(table), ptr(cg), ptr(x),
+                         ptr(Y), ptr(W), ptr(g), ptr(h["h_x"]), ptr(h["h_W"]), ptr(h["h_Y"]), ptr(outs["gg"]),
+                         ptr(outs["gx"]), ptr(outs["gW"]), ptr(outs["gY"]))
+    assert rc == 0
+    ref = O.double_backward(P, rowptr, col, n_send, x, Y, W, g, **h)
+    for k, r in zip(("gg", "gx", "gW", "gY"), ref):
+        if outs[k] is None:
+            continue
+        assert np.isfinite(outs[k]).all(), k
+        assert np.allclose(outs[k], r, rtol=1e-5, atol=1e-5 * max(1.0, np.abs(r).max())), k
