@@ -7,6 +7,10 @@ harmonics of the edge vectors, the forward CGTP convolution and its backward
 built once before timing.  Inputs are resident in HBM for ``value``; ``e2e``
 repeats the step through the same public API with the inputs copied from
 pinned host memory and the outputs copied back inside the timed region.
+The headline is the Lmax=3 workload (6,144 atoms, the largest on one GPU);
+``per_workload`` gives forward and forward+backward edges/s and atoms/s,
+each kernel's fraction of its binding roof and the oracle's CPU rate for the
+five workloads (tiny, lmax2, lmax2_wide, lmax3, lmax6).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
   python bench.py --impl reference ...     # the FP64 oracle on the host cores
@@ -33,7 +37,10 @@ sys.path.insert(0, ROOT)
 from equivariant_mlip_clebsch_b200 import workloads as WL  # noqa: E402
 
 METRIC = "CGTP conv edges/s (fwd, fwd+bwd) on 1 B200; % of HBM/FP32 roofline"
-DEFAULT_CONFIG = "lmax2"  # the Lmax=2 channelwise workload the metric is quoted on
+# the headline workload: the largest that fits one GPU (Table 1 Case 3 on
+# 6,144 atoms); the five workloads of PER_WORKLOAD are measured beside it
+DEFAULT_CONFIG = "lmax3"
+PER_WORKLOAD = ("tiny", "lmax2", "lmax2_wide", "lmax3", "lmax6")
 L2_FLUSH_BYTES = 512 << 20
 
 
@@ -193,39 +200,212 @@ def build_workload(name: str, seed: int = 0):
     return plan, host, N, E, c
 
 
+def workload_config(name: str, N: int, E: int, U: int, world: int) -> dict:
+    """The ``config`` of both arms' JSON lines (identical dicts): the workload
+    and what one step computes; how each arm times it is outside."""
+    c = WL.CONFIGS[name]
+    w_mb = 4.0 * E * U / 1e6
+    return {"workload": f"{name}: {c['desc']}", "atoms": N, "edges": E,
+            "irreps_in": c["irreps_in"], "irreps_edge": c["irreps_edge"], "irreps_out": c["irreps_out"],
+            "seed": 0, "step": "sph_harm + forward + backward (dx, dW, dY)",
+            "l2": (f"inputs larger than L2 (W alone {w_mb:.0f} MB)" if w_mb > 126 else
+                   f"W is {w_mb:.0f} MB") + "; the GPU arm also writes a 512 MB buffer before every timed step",
+            "parallelism": "replicas" if world > 1 else "single GPU"}
+
+
+def fp32_peaks(dev, smax_mhz: float) -> dict:
+    """FP32 peaks: derived (SMs from the device properties x 128 FP32 lanes x 2
+    flop x the max SM clock) and measured (the library's FMA probe, best of
+    three ~50 ms launches)."""
+    import ctypes
+    import torch
+    from equivariant_mlip_clebsch_b200 import cgtp as C
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    derived = sms * 128 * 2 * smax_mhz * 1e6 / 1e12
+    n = ctypes.c_int64()
+    C._check(C._lib.cgtp_fma_peak_sink_floats(ctypes.byref(n)))
+    sink = torch.empty(n.value, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    flops = ctypes.c_double()
+    best = 0.0
+    for iters in (2000, 100000, 100000, 100000):  # the first launch warms up
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        C._check(C._lib.cgtp_fma_peak(iters, ctypes.c_void_p(sink.data_ptr()), n.value,
+                                      ctypes.c_void_p(stream.cuda_stream), ctypes.byref(flops)))
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if iters > 2000:
+            best = max(best, flops.value / (e0.elapsed_time(e1) * 1e-3) / 1e12)
+    return {"derived_tflops": derived, "measured_tflops": best, "sms": sms, "sm_max_mhz": smax_mhz,
+            "derived": f"{sms} SMs x 128 FP32 lanes x 2 flop x {smax_mhz:.0f} MHz",
+            "measured": "cgtp_fma_peak: 2 CTAs x 512 threads per SM, 8 independent FMA chains, best of 3"}
+
+
+def kernel_roofs(kt: dict, alg_b: dict, alg_f: dict, hbm: float, fp32: dict) -> dict:
+    """Per kernel: average device time, achieved GB/s and TFLOP/s, the binding
+    roof (HBM unless its flops at the derived FP32 peak take longer) and the
+    fractions of HBM and of both FP32 peaks."""
+    out = {}
+    for nm, (ms, cnt) in kt.items():
+        avg = ms / max(cnt, 1)
+        d = {"avg_ms": avg, "launches": cnt}
+        t = avg * 1e-3
+        if nm in alg_b:
+            d["GB/s"] = alg_b[nm] / t / 1e9
+            d["frac_hbm"] = d["GB/s"] / hbm
+        if nm in alg_f:
+            d["TFLOP/s"] = alg_f[nm] / t / 1e12
+            d["frac_fp32_derived"] = d["TFLOP/s"] / fp32["derived_tflops"]
+            if fp32["measured_tflops"] > 0:
+                d["frac_fp32_measured"] = d["TFLOP/s"] / fp32["measured_tflops"]
+        if nm in alg_b and nm in alg_f:
+            alu = alg_f[nm] / (fp32["derived_tflops"] * 1e12) > alg_b[nm] / (hbm * 1e9)
+            d["bound"] = "alu" if alu else "hbm"
+            d["frac_bound"] = d["frac_fp32_derived"] if alu else d["frac_hbm"]
+        elif nm in alg_b:
+            d["bound"] = "hbm"
+            d["frac_bound"] = d["frac_hbm"]
+        out[nm] = d
+    return out
+
+
+class Timer:
+    """K timed repetitions of a callable on one stream, the L2 flushed before
+    each (not timed); mean device milliseconds."""
+
+    def __init__(self, flush, stream):
+        self.flush, self.stream = flush, stream
+
+    def __call__(self, fn, k: int) -> float:
+        import torch
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
+        for a, b in ev:
+            self.flush.zero_()
+            a.record(self.stream)
+            fn()
+            b.record(self.stream)
+        torch.cuda.synchronize()
+        return float(np.mean([a.elapsed_time(b) for a, b in ev]))
+
+
+class Workbench:
+    """One workload resident on the device, with its step, forward and the
+    per-kernel breakdown."""
+
+    def __init__(self, name, dev, flush):
+        import torch
+        t0 = time.time()
+        self.name, self.dev = name, dev
+        self.plan, self.host, self.N, self.E, self.c = build_workload(name)
+        self.setup_s = time.time() - t0
+        plan, N, E = self.plan, self.N, self.E
+        self.T = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in self.host.items()}
+        self.Y = torch.empty((E, plan.d_edge), device=dev)
+        self.out = torch.empty((N, plan.d_out), device=dev)
+        self.dx = torch.empty((N, plan.d_in), device=dev)
+        self.dW = torch.empty((E, plan.n_weights), device=dev)
+        self.dY = torch.empty((E, plan.d_edge), device=dev)
+        self.ws = torch.empty(max(plan.workspace_size(N, N, E), 256), dtype=torch.uint8, device=dev)
+        self.stream = torch.cuda.current_stream()
+        self.timer = Timer(flush, self.stream)
+        self.graph = None
+
+    def step(self):
+        T, plan = self.T, self.plan
+        plan.sph_harm(T["r"], self.Y)
+        plan.forward(T["rowptr"], T["col"], T["x"], self.Y, T["W"], out=self.out)
+        plan.backward(T["rowptr"], T["col"], T["rpt"], T["perm"], T["x"], self.Y, T["W"], T["g"],
+                      grads=(self.dx, self.dW, self.dY), workspace=self.ws)
+
+    def fwd(self):
+        T = self.T
+        self.plan.sph_harm(T["r"], self.Y)
+        self.plan.forward(T["rowptr"], T["col"], T["x"], self.Y, T["W"], out=self.out)
+
+    def warm(self, n):
+        import torch
+        for _ in range(n):
+            self.step()
+        torch.cuda.synchronize()
+        self.plan.check_device_error()
+
+    def capture(self):
+        import torch
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step()
+        self.graph.replay()
+        torch.cuda.synchronize()
+        self.plan.check_device_error()
+
+    def measure(self, k: int, use_graph: bool):
+        """(step ms, launched step ms, forward ms, kernel times {name: (ms, n)})."""
+        if use_graph and self.graph is None:
+            self.capture()
+        ms_step = self.timer(self.graph.replay if use_graph else self.step, k)
+        self.plan.kernel_times()  # discard
+        self.plan.set_timing(True)
+        ms_eager = self.timer(self.step, k)
+        self.plan.set_timing(False)
+        kt = self.plan.kernel_times()
+        ms_fwd = self.timer(self.fwd, k)
+        self.plan.check_device_error()
+        return ms_step, ms_eager, ms_fwd, kt
+
+    def algorithmic(self):
+        p = self.plan
+        return algorithmic(self.N, self.E, p.d_in, p.d_edge, p.d_out, p.n_weights, p.paths(), p.coefficients())
+
+    def close(self):
+        self.graph = None
+        self.T = self.Y = self.out = self.dx = self.dW = self.dY = self.ws = None
+        self.plan.close()
+
+
+def per_workload_entry(wb: "Workbench", k: int, use_graph: bool, hbm: float, fp32: dict, world: int,
+                       cpu_budget: float) -> dict:
+    ms_step, ms_eager, ms_fwd, kt = wb.measure(k, use_graph)
+    alg_b, alg_f = wb.algorithmic()
+    N, E = wb.N, wb.E
+    d = {"atoms": N, "edges": E, "steps": k,
+         "fwd": {"ms": ms_fwd, "edges_per_s": world * E / (ms_fwd * 1e-3),
+                 "atoms_per_s": world * N / (ms_fwd * 1e-3), "what": "sph_harm + forward"},
+         "fwd_bwd": {"ms": ms_step, "edges_per_s": world * E / (ms_step * 1e-3),
+                     "atoms_per_s": world * N / (ms_step * 1e-3),
+                     "what": "sph_harm + forward + backward (dx, dW, dY)"
+                             + (", replayed from one CUDA graph" if use_graph else "")},
+         "ms_per_step_launched": ms_eager,
+         "kernels": kernel_roofs(kt, alg_b, alg_f, hbm, fp32)}
+    if cpu_budget > 0:
+        try:
+            s = oracle_sample(wb.name, cpu_budget)
+            d["cpu_baseline"] = {"value": s["edges_per_s"], "unit": "edges/s",
+                                 "atoms_per_s": s["edges_per_s"] * N / E, "cores": s["cores"],
+                                 "kind": "oracle",
+                                 "sample": f"receivers 0..{s['rows'] - 1} ({s['edges']} edges), harmonics + "
+                                           f"forward + backward, {s['reps']} passes in {s['seconds']:.1f}s, FP64"}
+        except Exception as e:  # reported; the GPU figures stand
+            d["cpu_baseline"] = {"error": str(e)}
+    return d
+
+
 def run_cgtp(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     name = args.config
-    t0 = time.time()
-    plan, host, N, E, c = build_workload(name)
-    log(f"[rank {rank}] plan + workload {name}: N={N} E={E} ({time.time() - t0:.1f}s)")
-    T = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in host.items()}
-    Y = torch.empty((E, plan.d_edge), device=dev)
-    out = torch.empty((N, plan.d_out), device=dev)
-    dx = torch.empty((N, plan.d_in), device=dev)
-    dW = torch.empty((E, plan.n_weights), device=dev)
-    dY = torch.empty((E, plan.d_edge), device=dev)
-    ws = torch.empty(max(plan.workspace_size(N, N, E), 256), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
-
-    def step(r_, x_, W_, g_):
-        plan.sph_harm(r_, Y)
-        plan.forward(T["rowptr"], T["col"], x_, Y, W_, out=out)
-        plan.backward(T["rowptr"], T["col"], T["rpt"], T["perm"], x_, Y, W_, g_, grads=(dx, dW, dY),
-                      workspace=ws)
-
-    for _ in range(args.warmup):
-        step(T["r"], T["x"], T["W"], T["g"])
-    torch.cuda.synchronize()
-    plan.check_device_error()
+    wb = Workbench(name, dev, flush)
+    plan, T, N, E, c = wb.plan, wb.T, wb.N, wb.E, wb.c
+    log(f"[rank {rank}] plan + workload {name}: N={N} E={E} ({wb.setup_s:.1f}s)")
+    stream = wb.stream
+    wb.warm(args.warmup)
     if args.profile:  # for ncu: warm-up plus K plain steps, nothing else
         for _ in range(args.steps):
             flush.zero_()
-            step(T["r"], T["x"], T["W"], T["g"])
+            wb.step()
         torch.cuda.synchronize()
         plan.check_device_error()
         return {"profile": name, "steps": args.steps, "warmup": args.warmup, "N": N, "E": E}
@@ -236,123 +416,53 @@ def run_cgtp(args, rank, world, local_rank):
     sampler.start()
     t_end = time.time() + 1.0
     while time.time() < t_end:
-        for _ in range(20):
-            step(T["r"], T["x"], T["W"], T["g"])
+        for _ in range(5):
+            wb.step()
         torch.cuda.synchronize()
-    # the step's four launches captured once in a CUDA graph (no launch gaps);
-    # the headline times K replays
-    graph = None
-    if not args.no_graph:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            step(T["r"], T["x"], T["W"], T["g"])
-        graph.replay()
-        torch.cuda.synchronize()
-        plan.check_device_error()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    ev_e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
-    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
+    use_graph = not args.no_graph
+    if use_graph:
+        wb.capture()
+    # ---- the headline: K steps, barrier + synchronize on both sides
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    for k in range(args.steps):
-        flush.zero_()  # L2 flush (not timed)
-        a, b = ev[k]
-        a.record(stream)
-        if graph is not None:
-            graph.replay()
-        else:
-            step(T["r"], T["x"], T["W"], T["g"])
-        b.record(stream)
+    ms_step_local = wb.timer(wb.graph.replay if use_graph else wb.step, args.steps)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    # the same K steps launched one by one, with the library's per-kernel
-    # events on: the per-kernel breakdown and the roofline
-    plan.kernel_times()  # discard
-    plan.set_timing(True)
-    for k in range(args.steps):
-        flush.zero_()
-        a, b = ev_e[k]
-        a.record(stream)
-        step(T["r"], T["x"], T["W"], T["g"])
-        b.record(stream)
-    torch.cuda.synchronize()
-    plan.set_timing(False)
-    kt = plan.kernel_times()  # the kernels of the K eager steps
-    ms_eager = float(np.mean([a.elapsed_time(b) for a, b in ev_e]))
-    # forward-only steps (harmonics + forward), for the forward edges/s
-    for k in range(args.steps):
-        flush.zero_()
-        a, b = ev_f[k]
-        a.record(stream)
-        plan.sph_harm(T["r"], Y)
-        plan.forward(T["rowptr"], T["col"], T["x"], Y, T["W"], out=out)
-        b.record(stream)
+    ms_step = max_over_ranks(ms_step_local, world, dev)
+    value = replica_value(world, E, ms_step)
+    # ---- the per-kernel breakdown and the forward on the same workload
+    _, ms_eager, fwd_ms, kt = wb.measure(args.steps, use_graph)
+
     # the force chain after the backward (dL/dY -> dL/dr -> forces), not in
     # the step: reported beside it
     from equivariant_mlip_clebsch_b200 import cgtp as C
     gr = torch.empty((E, 3), device=dev)
     Fo = torch.empty((N, 3), device=dev)
-    ev_c = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
-    for k in range(args.steps):
-        flush.zero_()
-        a, b = ev_c[k]
-        a.record(stream)
-        plan.sph_harm_backward(T["r"], dY, grad_r=gr)
+
+    def force_chain():
+        plan.sph_harm_backward(T["r"], wb.dY, grad_r=gr)
         C.edge_forces(T["rowptr"], T["rpt"], T["perm"], gr, forces=Fo)
-        b.record(stream)
+    force_ms = wb.timer(force_chain, args.steps)
     # the strain derivative (virial) from the same grad_r, timed on its own
     Vo = torch.empty((3, 3), device=dev)
-    ev_v = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
-    virial_err = None
     try:
-        for k in range(args.steps):
-            flush.zero_()
-            a, b = ev_v[k]
-            a.record(stream)
-            C.edge_virial(T["r"], gr, virial=Vo)
-            b.record(stream)
-    except (C.CgtpError, ValueError, TypeError) as e:  # reported, the headline stands
-        virial_err = str(e)
-    # the double backward (all three cotangents), timed on its own
-    ev_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
-    dbl_err = None
-    try:
-        gen = torch.Generator(device=dev).manual_seed(3)
-        hx, hW, hY = (torch.randn(t.shape, device=dev, generator=gen) for t in (T["x"], T["W"], Y))
-        dgrads = tuple(torch.empty_like(t) for t in (T["g"], T["x"], T["W"], Y))
-        dws = torch.empty(max(plan.double_backward_workspace_size(N, N, E), 256), dtype=torch.uint8, device=dev)
-        for k in range(args.steps):
-            flush.zero_()
-            a, b = ev_d[k]
-            a.record(stream)
-            plan.double_backward(T["rowptr"], T["col"], T["rpt"], T["perm"], T["x"], Y, T["W"], T["g"],
-                                 h_x=hx, h_W=hW, h_Y=hY, grads=dgrads, workspace=dws)
-            b.record(stream)
-    except (C.CgtpError, ValueError, TypeError) as e:  # reported, the headline stands
-        dbl_err = str(e)
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
-    plan.check_device_error()
-    ms_steps = [a.elapsed_time(b) for a, b in ev]
-    ms_fwd = [a.elapsed_time(b) for a, b in ev_f]
-    force_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_c]))
-    if virial_err is None:
-        virial_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_v]))
+        virial_ms = wb.timer(lambda: C.edge_virial(T["r"], gr, virial=Vo), args.steps)
         virial = {"ms": virial_ms, "edges_per_s": world * E / (virial_ms * 1e-3),
                   "achieved_gbs": 24.0 * E / (virial_ms * 1e-3) / 1e9,
                   "what": "edge_virial from grad_r (24 B/edge read), after the step (not in it)"}
-    else:
-        virial = {"error": virial_err}
-    if dbl_err is None:
-        dbl_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_d]))
+    except (C.CgtpError, ValueError, TypeError) as e:  # reported, the headline stands
+        virial = {"error": str(e)}
+    # the double backward (all three cotangents), timed on its own
+    try:
+        gen = torch.Generator(device=dev).manual_seed(3)
+        hx, hW, hY = (torch.randn(t.shape, device=dev, generator=gen) for t in (T["x"], T["W"], wb.Y))
+        dgrads = tuple(torch.empty_like(t) for t in (T["g"], T["x"], T["W"], wb.Y))
+        dws = torch.empty(max(plan.double_backward_workspace_size(N, N, E), 256), dtype=torch.uint8, device=dev)
+        dbl_ms = wb.timer(lambda: plan.double_backward(T["rowptr"], T["col"], T["rpt"], T["perm"], T["x"], wb.Y,
+                                                       T["W"], T["g"], h_x=hx, h_W=hW, h_Y=hY, grads=dgrads,
+                                                       workspace=dws), args.steps)
         # the operation's own bytes: x, Y, W, grad_out and the three cotangents
         # read once, the four gradients written once, both CSRs read
         dbl_bytes = 4 * (2 * N * plan.d_in + 2 * E * plan.d_edge + 2 * E * plan.n_weights + N * plan.d_out
@@ -360,73 +470,82 @@ def run_cgtp(args, rank, world, local_rank):
                          + 2 * (N + 1 + E))
         double_backward = {"ms": dbl_ms, "edges_per_s": world * E / (dbl_ms * 1e-3),
                            "algorithmic_bytes": dbl_bytes, "achieved_gbs": dbl_bytes / (dbl_ms * 1e-3) / 1e9,
-                           "what": "double_backward with h_x, h_W, h_Y (3 forwards, 3 backwards, adds), "
-                                   "after the step (not in it); achieved_gbs counts the operation's own "
-                                   "bytes, so the composition's extra passes show as a low fraction"}
-    else:
-        double_backward = {"error": dbl_err}
-    ms_step = max_over_ranks(float(np.sum(ms_steps)) / args.steps, world, dev)
-    value = replica_value(world, E, ms_step)
-    fwd_ms = float(np.mean(ms_fwd))
-
-    # ---- per-kernel roofline (device time from the library's events)
+                           "vs_step": dbl_ms / ms_step_local,
+                           "what": "double_backward with h_x, h_W, h_Y, after the step (not in it)"}
+        del hx, hW, hY, dgrads, dws
+    except (C.CgtpError, ValueError, TypeError) as e:  # reported, the headline stands
+        double_backward = {"error": str(e)}
     hbm, smax, pk_kind = peaks()
     if "achieved_gbs" in double_backward:
         double_backward["frac_hbm"] = double_backward["achieved_gbs"] / hbm
-    paths = plan.paths()
-    coeff = plan.coefficients()
-    alg_b, alg_f = algorithmic(N, E, plan.d_in, plan.d_edge, plan.d_out, plan.n_weights, paths, coeff)
-    kernels = {}
-    for nm, (ms, cnt) in kt.items():
-        avg = ms / max(cnt, 1)
-        d = {"avg_ms": avg, "launches": cnt}
-        if nm in alg_b:
-            d["GB/s"] = alg_b[nm] / (avg * 1e-3) / 1e9
-        if nm in alg_f:
-            d["TFLOP/s"] = alg_f[nm] / (avg * 1e-3) / 1e12
-        kernels[nm] = d
+    fp32 = fp32_peaks(dev, smax)
+    clocks_main = sampler.stop()
+    plan.check_device_error()
+
+    # ---- roofline of the dominant kernel
+    alg_b, alg_f = wb.algorithmic()
+    kernels = kernel_roofs(kt, alg_b, alg_f, hbm, fp32)
     timed_names = [n for n in kt if n in ("cgtp_fwd", "cgtp_bwd")]
     dom = max(timed_names, key=lambda n: kt[n][0]) if timed_names else max(kt, key=lambda n: kt[n][0])
-    fp32_peak = 148 * 128 * 2 * smax * 1e6 / 1e12  # TFLOP/s at the max SM clock
-    avg_dom = kt[dom][0] / kt[dom][1]
-    bytes_dom = alg_b.get(dom, 0)
-    flops_dom = alg_f.get(dom, 0.0)
-    t_hbm = bytes_dom / (hbm * 1e9)
-    t_alu = flops_dom / (fp32_peak * 1e12)
-    if t_alu > t_hbm:
-        roof = {"bound": "alu", "achieved": flops_dom / (avg_dom * 1e-3) / 1e12, "peak": fp32_peak,
-                "unit": "TFLOP/s"}
+    kd = kernels[dom]
+    if kd.get("bound") == "alu":
+        roof = {"bound": "alu", "achieved": kd["TFLOP/s"], "peak": fp32["derived_tflops"], "unit": "TFLOP/s",
+                "peak_source": fp32["derived"], "measured_fma_peak": fp32["measured_tflops"],
+                "frac_of_measured_fma_peak": kd.get("frac_fp32_measured")}
     else:
-        roof = {"bound": "hbm", "achieved": bytes_dom / (avg_dom * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s"}
+        roof = {"bound": "hbm", "achieved": kd["GB/s"], "peak": hbm, "unit": "GB/s",
+                "peak_source": pk_kind + " (MEASURED_PEAKS.json hbm_gbs)",
+                "frac_vs_spec_8000": kd["GB/s"] / 8000.0}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    if roof["bound"] == "hbm":  # against the ~8 TB/s spec as well
-        roof["frac_vs_spec_8000"] = roof["achieved"] / 8000.0
-    roof["fp32_sgemm_tflops"] = sgemm_tflops(dev)  # measured FP32 (CUDA cores), context
     roof["kernel"] = dom
-    roof["peak_source"] = pk_kind if roof["bound"] == "hbm" else \
-        "148 SMs x 128 FP32 lanes x 2 flop x max SM clock"
+    roof["algorithmic_bytes_per_launch"] = alg_b.get(dom)
     roof["traffic"] = ncu_traffic(name, dom, plan)
+    roof["fp32_sgemm_tflops"] = sgemm_tflops(dev)  # measured cuBLAS FP32 (CUDA cores), context
     gpu_launches = sum(cnt for nm, (ms, cnt) in kt.items() if nm != "zero_fill")
 
     # ---- end to end through the same API with host buffers
-    e2e = run_e2e(args, plan, T, host, Y, out, dx, dW, dY, ws, E, dev, world)
+    e2e = run_e2e(args, plan, T, wb.host, wb.Y, wb.out, wb.dx, wb.dW, wb.dY, wb.ws, E, dev, world)
     res = dict(metric=METRIC, value=value, unit="edges/s", n_gpus=world, steps=args.steps,
                warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
                vs_baseline=None, dtype="f32", data="synthetic",
-               config={"workload": f"{name}: {c['desc']}", "atoms": N, "edges": E,
-                       "irreps_in": c["irreps_in"], "irreps_edge": c["irreps_edge"],
-                       "irreps_out": c["irreps_out"], "seed": 0,
-                       "step": "sph_harm + forward + backward (dx, dW, dY)"
-                               + (", replayed from one CUDA graph" if graph is not None else ""),
-                       "l2": f"{L2_FLUSH_BYTES >> 20} MB buffer written before every timed step (not timed)",
-                       "parallelism": "replicas" if world > 1 else "single GPU"},
+               config=workload_config(name, N, E, plan.n_weights, world),
+               timing={"device": "CUDA events on the launching stream, K steps"
+                                 + (" replayed from one CUDA graph" if use_graph else " launched call by call"),
+                       "l2_flush": f"{L2_FLUSH_BYTES >> 20} MB buffer written before every timed step (not timed)"},
                atoms_per_s=replica_value(world, N, ms_step),
-               fwd_edges_per_s=world * E / (fwd_ms * 1e-3), fwd_ms=fwd_ms,
-               ms_per_step_launched=ms_eager,
+               fwd_edges_per_s=world * E / (fwd_ms * 1e-3), fwd_atoms_per_s=world * N / (fwd_ms * 1e-3),
+               fwd_ms=fwd_ms, ms_per_step_launched=ms_eager,
                force_chain={"ms": force_ms, "edges_per_s": world * E / (force_ms * 1e-3),
                             "what": "sph_harm_backward + edge_forces after the step (not in it)"},
                virial=virial, double_backward=double_backward,
-               roofline=roof, kernels=kernels, gpu_launches=int(gpu_launches), e2e=e2e, clocks=clocks)
+               roofline=roof, fp32_peak=fp32, kernels=kernels, gpu_launches=int(gpu_launches), e2e=e2e,
+               clocks=clocks_main)
+    # the five workloads of the target, each measured on its own (the headline
+    # workload's figures are taken again in the same way, for one table)
+    if not args.no_per_workload:
+        per = {}
+        k = max(3, min(args.steps, 10))
+        wb.close()
+        del wb
+        torch.cuda.empty_cache()
+        sampler2 = ClockSampler(sampler.idx)
+        sampler2.start()
+        for nm in PER_WORKLOAD:
+            try:
+                w2 = Workbench(nm, dev, flush)
+                w2.warm(3)
+                per[nm] = per_workload_entry(w2, k, use_graph, hbm, fp32, world,
+                                             args.cpu_budget / 4 if rank == 0 else 0.0)
+                per[nm]["plan_and_graph_s"] = w2.setup_s
+                w2.close()
+                del w2
+                torch.cuda.empty_cache()
+            except Exception as e:  # reported, the headline stands
+                per[nm] = {"error": f"{type(e).__name__}: {e}"}
+            log(f"[rank {rank}] per-workload {nm}: "
+                + (f"{per[nm]['fwd_bwd']['edges_per_s']:.3e} edges/s" if "fwd_bwd" in per[nm] else per[nm]["error"]))
+        per["clocks"] = sampler2.stop()
+        res["per_workload"] = per
     return res
 
 
@@ -621,7 +740,9 @@ def run_reference(args, rank, world):
     return dict(impl="reference", metric=METRIC, value=value, unit="edges/s", n_gpus=world,
                 steps=args.steps, warmup=args.warmup, ms_per_step=float(np.mean(times)) * 1e3,
                 higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
-                config={"workload": f"{name}: {c['desc']}", "atoms": len(pos), "edges": int(len(col))},
+                config=workload_config(name, len(pos), int(len(col)), P.U, world),
+                timing={"host": "wall clock per step of the FP64 oracle on the host cores, on a bounded "
+                                "sample of the workload's receivers"},
                 cpu_baseline={"value": value, "unit": "edges/s", "cores": s["cores"], "kind": "oracle",
                               "sample": sample},
                 e2e={"value": value, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
@@ -638,6 +759,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(WL.CONFIGS))
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline field (0 to skip)")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the per-workload figures of the five workloads")
     ap.add_argument("--profile", action="store_true",
                     help="warm-up + K steps only (no clock loop, e2e or CPU baseline), for ncu")
     args = ap.parse_args()

@@ -53,6 +53,8 @@ _SIGS = {
     "cgtp_plan_check_device_error": (_i, [_P, ctypes.POINTER(_i)]),
     "cgtp_plan_set_timing": (_i, [_P, _i]),
     "cgtp_plan_kernel_times": (_i, [_P, _i, ctypes.c_char_p, _P, _P, ctypes.POINTER(_i)]),
+    "cgtp_fma_peak_sink_floats": (_i, [_pi64]),
+    "cgtp_fma_peak": (_i, [_i64, _P, _i64, _P, ctypes.POINTER(_d)]),
     "cgtp_neighbor_list": (_i, [_i64, _P, _P, _d, _P, _P, _P, _P, _pi64]),
     "cgtp_csr_transpose": (_i, [_i64, _i64, _i64, _P, _P, _P, _P]),
 }

@@ -180,6 +180,7 @@ cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge, con
       CGTP_CUDA_TRY(cudaFree(0));  // make the primary context current
       if (cudaMalloc(&P->d_err, sizeof(int)) != cudaSuccess) return fail(CGTP_ERR_OOM, "cudaMalloc");
       CGTP_CUDA_TRY(cudaMemset(P->d_err, 0, sizeof(int)));
+      CGTP_CUDA_TRY(upload_sph_norm());  // once per device, before any capture
     }
     st = build_forward(*P);  // leaves the forward compiling on a host thread
     if (st == CGTP_OK) st = build_backward(*P);
@@ -355,6 +356,38 @@ cgtp_status cgtp_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
 
 namespace cgtp {
 
+cgtp_status check_plan_device(const Plan& P) { return check_device(P); }
+
+// The scratch bytes one backward call uses: the per-edge messages when grad_x
+// is wanted (first), and the slice parts of dY when grad_Y is wanted from a
+// plan of several slices (after the messages, or at offset 0 without them).
+size_t backward_scratch_bytes(const Plan& P, int64_t E, bool want_x, bool want_Y, size_t* off_dyp) {
+  auto r256 = [](size_t v) { return (v + 255) & ~size_t(255); };
+  const size_t msg = want_x ? r256((size_t)E * P.D_in * sizeof(float)) : 0;
+  if (off_dyp) *off_dyp = msg;
+  const size_t parts = (want_Y && P.bcfg.S > 1) ? r256((size_t)P.bcfg.S * E * P.D_e * sizeof(float)) : 0;
+  return msg + parts;
+}
+
+cgtp_status backward_validate(const Plan& P, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
+                              const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, const float* x,
+                              const float* Y, const float* W, const float* grad_out, const float* grad_x,
+                              const float* grad_W, const float* grad_Y) {
+  if (n_recv < 0 || n_send < 0 || E < 0 || n_recv >= (int64_t(1) << 31) ||
+      n_send >= (int64_t(1) << 31) || E >= (int64_t(1) << 31) - 1)
+    return fail(CGTP_ERR_SIZE, "sizes out of range");
+  cgtp_status st = check_device(P);
+  if (st != CGTP_OK) return st;
+  for (const void* p : {(const void*)x, (const void*)Y, (const void*)W, (const void*)grad_out,
+                        (const void*)grad_x, (const void*)grad_W, (const void*)grad_Y})
+    if (p && !aligned16(p)) return fail(CGTP_ERR_ALIGN, "float arrays must be 16-byte aligned");
+  if (E == 0) return CGTP_OK;
+  if (!rowptr || !col || !x || !Y || !W || !grad_out)
+    return fail(CGTP_ERR_NULL, "rowptr, col, x, Y, W or grad_out is NULL");
+  if (grad_x && (!rowptr_T || !perm_T)) return fail(CGTP_ERR_NULL, "grad_x needs rowptr_T and perm_T");
+  return CGTP_OK;
+}
+
 cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
                           const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
                           const int32_t* perm_T, const float* x, const float* Y, const float* W,
@@ -363,29 +396,21 @@ cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
                           bool allow_timing) {
   if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
   Plan* P = reinterpret_cast<Plan*>(plan);
-  if (n_recv < 0 || n_send < 0 || E < 0 || n_recv >= (int64_t(1) << 31) ||
-      n_send >= (int64_t(1) << 31) || E >= (int64_t(1) << 31) - 1)
-    return fail(CGTP_ERR_SIZE, "sizes out of range");
-  cudaStream_t s = (cudaStream_t)stream;
-  cgtp_status st = check_device(*P);
+  cgtp_status st = backward_validate(*P, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, x, Y, W, grad_out,
+                                     grad_x, grad_W, grad_Y);
   if (st != CGTP_OK) return st;
-  for (const void* p : {(const void*)x, (const void*)Y, (const void*)W, (const void*)grad_out,
-                        (const void*)grad_x, (const void*)grad_W, (const void*)grad_Y})
-    if (p && !aligned16(p)) return fail(CGTP_ERR_ALIGN, "float arrays must be 16-byte aligned");
+  cudaStream_t s = (cudaStream_t)stream;
   if (grad_x && n_send > 0 && (E == 0 || P->bwd_roles.empty()))
     CGTP_CUDA_TRY(cudaMemsetAsync(grad_x, 0, (size_t)n_send * P->D_in * sizeof(float), s));
   if (E == 0) return CGTP_OK;
-  if (!rowptr || !col || !x || !Y || !W || !grad_out)
-    return fail(CGTP_ERR_NULL, "rowptr, col, x, Y, W or grad_out is NULL");
-  if (grad_x && (!rowptr_T || !perm_T)) return fail(CGTP_ERR_NULL, "grad_x needs rowptr_T and perm_T");
   if (P->bwd_roles.empty()) {
     if (grad_W) CGTP_CUDA_TRY(cudaMemsetAsync(grad_W, 0, (size_t)E * P->U * sizeof(float), s));
     if (grad_Y) CGTP_CUDA_TRY(cudaMemsetAsync(grad_Y, 0, (size_t)E * P->D_e * sizeof(float), s));
     return CGTP_OK;
   }
   size_t off_dyp = 0;
-  const size_t need = bwd_workspace_layout(*P, E, &off_dyp);
-  const bool need_ws = grad_x || (grad_Y && P->bcfg.S > 1);
+  const size_t need = backward_scratch_bytes(*P, E, grad_x != nullptr, grad_Y != nullptr, &off_dyp);
+  const bool need_ws = need > 0;
   if (need_ws && (!workspace || workspace_bytes < need))
     return fail(CGTP_ERR_WORKSPACE, "workspace of " + std::to_string(need) + " bytes required");
   if (need_ws && ((uintptr_t)workspace & 255))
@@ -610,6 +635,27 @@ cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send,
   const DbwdDims dims{n_recv, n_send, E, P->D_in, P->D_e, P->D_out, P->U};
   return (cgtp_status)compose_double_backward(ops, dims, x, Y, W, h_x, h_W, h_Y, gg_out, gx, gW, gY, tF, tX, tW,
                                               tY);
+}
+
+cgtp_status cgtp_fma_peak_sink_floats(int64_t* floats) {
+  if (!floats) return fail(CGTP_ERR_NULL, "floats is NULL");
+  int dev = 0, sms = 0;
+  CGTP_CUDA_TRY(cudaGetDevice(&dev));
+  CGTP_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  *floats = fma_peak_sink_floats(sms);
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_fma_peak(int64_t iters, float* sink, int64_t sink_floats, cgtp_stream stream, double* flops) {
+  if (!sink || !flops) return fail(CGTP_ERR_NULL, "sink or flops is NULL");
+  if (iters < 1 || iters > (int64_t(1) << 24)) return fail(CGTP_ERR_SIZE, "iters must be in 1..2^24");
+  int dev = 0, sms = 0;
+  CGTP_CUDA_TRY(cudaGetDevice(&dev));
+  CGTP_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  if (sink_floats < fma_peak_sink_floats(sms))
+    return fail(CGTP_ERR_SIZE, "sink holds fewer floats than cgtp_fma_peak_sink_floats");
+  CGTP_CUDA_TRY(launch_fma_peak(sms, iters, 1.0f - 1e-7f, 1e-7f, sink, (cudaStream_t)stream, flops));
+  return CGTP_OK;
 }
 
 cgtp_status cgtp_neighbor_list(int64_t N, const double* pos, const double* box, double rc,

@@ -173,6 +173,17 @@ cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
                           void* workspace, size_t workspace_bytes, cgtp_stream stream,
                           bool allow_timing);
 
+// The plan's device is current and the plan has device state.
+cgtp_status check_plan_device(const Plan& P);
+// Host checks of a backward call (sizes, device, alignment, required pointers).
+cgtp_status backward_validate(const Plan& P, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
+                              const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, const float* x,
+                              const float* Y, const float* W, const float* grad_out, const float* grad_x,
+                              const float* grad_W, const float* grad_Y);
+// Scratch bytes a backward call uses for the gradients it is asked for (at
+// most cgtp_backward_workspace_size); off_dyp receives the dY parts' offset.
+size_t backward_scratch_bytes(const Plan& P, int64_t E, bool want_x, bool want_Y, size_t* off_dyp);
+
 // construction steps
 cgtp_status build_paths(Plan& P);
 cgtp_status build_forward(Plan& P);
@@ -197,6 +208,12 @@ cudaError_t launch_edge_forces(int64_t n_atoms, const int32_t* rowptr, const int
                                const int32_t* perm_T, const float* G, float* F, cudaStream_t s);
 cudaError_t launch_edge_virial(int64_t E, const float* r, const float* G, float* V, cudaStream_t s);
 cudaError_t launch_add(int64_t n, const float* src, float* dst, cudaStream_t s);
+// c_norm of the harmonics kernels, uploaded once per device (plan creation)
+cudaError_t upload_sph_norm();
+// FP32 FMA throughput probe: 2 CTAs per SM; flops receives the launch's FLOPs
+int64_t fma_peak_sink_floats(int num_sms);
+cudaError_t launch_fma_peak(int num_sms, int64_t iters, float m, float c, float* sink, cudaStream_t s,
+                            double* flops);
 
 // dx row sums over the transpose edge list and the dY slice sums, one launch;
 // either part is skipped when its output is null (or S == 1 for dY).

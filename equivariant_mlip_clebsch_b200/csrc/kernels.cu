@@ -7,8 +7,10 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "internal.hpp"
 
@@ -42,7 +44,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, unsigned block, cuda
 //   N_l0 = sqrt(2l+1),  N_lm = sqrt(2l+1) sqrt(2 (l-m)!/(l+m)!)  (m > 0)
 // index l*(l+1)/2 + m, l <= 6.
 __constant__ float c_norm[28];
-bool g_norm_ready[64] = {false};
+constexpr int kMaxDevices = 256;
+std::atomic<bool> g_norm_ready[kMaxDevices];
+std::mutex g_norm_mu;
 
 template <int L>
 __global__ void __launch_bounds__(128) sph_harm_kernel(int64_t E, const float* __restrict__ r,
@@ -317,6 +321,34 @@ __global__ void __launch_bounds__(256) add_kernel(int64_t n, const float* __rest
   for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += stride) dst[i] += src[i];
 }
 
+// FP32 FMA throughput probe (the measured FP32 peak the Lmax >= 4 workloads
+// are compared with).  Every thread runs kFmaChains independent dependency
+// chains a <- a * m + c, kFmaUnroll steps per loop trip; with 512 threads per
+// CTA and two CTAs per SM each scheduler has eight warps of eight independent
+// FMAs in flight, more than the pipeline latency needs.  m and c come from
+// the caller (the compiler cannot fold the chains); the chains' sum is stored
+// per thread so that none is dead.  FLOPs = 2 x threads x iters x chains x unroll.
+constexpr int kFmaChains = 8;
+constexpr int kFmaUnroll = 16;
+constexpr int kFmaThreads = 512;
+
+__global__ void __launch_bounds__(kFmaThreads) fma_peak_kernel(int64_t iters, float m, float c,
+                                                               float* __restrict__ sink) {
+  float a[kFmaChains];
+#pragma unroll
+  for (int k = 0; k < kFmaChains; ++k) a[k] = (float)(threadIdx.x + k) * 1e-3f;
+  for (int64_t it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int u = 0; u < kFmaUnroll; ++u)
+#pragma unroll
+      for (int k = 0; k < kFmaChains; ++k) a[k] = fmaf(a[k], m, c);
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < kFmaChains; ++k) s += a[k];
+  sink[(int64_t)blockIdx.x * kFmaThreads + threadIdx.x] = s;
+}
+
 // The backward's closing reductions in one launch.
 //  blocks [0, n_send): dx[j][c] = sum over sender j's edges of m[perm_T[t]][c].
 //    Two groups of 128 threads take the even and the odd positions t0 + 2k of
@@ -396,11 +428,17 @@ __global__ void __launch_bounds__(kEpiThreads) bwd_reduce_kernel(
 
 }  // namespace
 
-static cudaError_t ensure_norm() {
+// Uploads c_norm to the current device once (plan creation calls this with
+// the plan's device current).  A synchronous copy: it must not run inside a
+// stream capture, which is why the launches below never do it themselves.
+cudaError_t upload_sph_norm() {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && g_norm_ready[dev]) return cudaSuccess;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (g_norm_ready[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  std::lock_guard<std::mutex> g(g_norm_mu);
+  if (g_norm_ready[dev].load(std::memory_order_relaxed)) return cudaSuccess;
   float h[28];
   for (int l = 0; l <= 6; ++l)
     for (int m = 0; m <= l; ++m) {
@@ -409,13 +447,11 @@ static cudaError_t ensure_norm() {
       h[l * (l + 1) / 2 + m] = (float)(std::sqrt(2.0 * l + 1.0) * (m == 0 ? 1.0 : std::sqrt(2.0 * f)));
     }
   e = cudaMemcpyToSymbol(c_norm, h, sizeof h);
-  if (e == cudaSuccess && dev >= 0 && dev < 64) g_norm_ready[dev] = true;
+  if (e == cudaSuccess) g_norm_ready[dev].store(true, std::memory_order_release);
   return e;
 }
 
 cudaError_t launch_sph_harm(int L, int64_t E, const float* r, float* Y, cudaStream_t s) {
-  cudaError_t e = ensure_norm();
-  if (e != cudaSuccess) return e;
   if (E == 0) return cudaSuccess;
   const dim3 grid((unsigned)((E + 127) / 128));
   switch (L) {
@@ -432,8 +468,6 @@ cudaError_t launch_sph_harm(int L, int64_t E, const float* r, float* Y, cudaStre
 
 cudaError_t launch_sph_harm_backward(int L, int64_t E, const float* r, const float* dY, float* dr,
                                      cudaStream_t s) {
-  cudaError_t e = ensure_norm();
-  if (e != cudaSuccess) return e;
   if (E == 0) return cudaSuccess;
   const dim3 grid((unsigned)((E + 127) / 128));
   switch (L) {
@@ -457,6 +491,16 @@ cudaError_t launch_edge_forces(int64_t n_atoms, const int32_t* rowptr, const int
 
 cudaError_t launch_edge_virial(int64_t E, const float* r, const float* G, float* V, cudaStream_t s) {
   return launch_pdl(edge_virial_kernel, dim3(kVirCtas), kVirThreads, s, E, r, G, V);
+}
+
+int64_t fma_peak_sink_floats(int num_sms) { return (int64_t)num_sms * 2 * kFmaThreads; }
+
+cudaError_t launch_fma_peak(int num_sms, int64_t iters, float m, float c, float* sink, cudaStream_t s,
+                            double* flops) {
+  const int64_t blocks = (int64_t)num_sms * 2;
+  *flops = 2.0 * (double)blocks * kFmaThreads * (double)iters * kFmaChains * kFmaUnroll;
+  fma_peak_kernel<<<(unsigned)blocks, kFmaThreads, 0, s>>>(iters, m, c, sink);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_add(int64_t n, const float* src, float* dst, cudaStream_t s) {

@@ -56,9 +56,15 @@ extern "C" cgtp_status cgtp_backward_static_scratch(
     const float* Y, const float* W, const float* grad_out, float* grad_x, float* grad_W,
     float* grad_Y, cgtp_stream stream) {
   if (!plan) return cgtp::fail(CGTP_ERR_NULL, "plan is NULL");
-  size_t need = 0;
-  cgtp_status st = cgtp_backward_workspace_size(plan, n_recv, n_send, E, &need);
+  const cgtp::Plan& P = *reinterpret_cast<const cgtp::Plan*>(plan);
+  // every host check first: a call with the wrong device current, a bad size
+  // or pointer is refused before the array's address is looked up
+  cgtp_status st = cgtp::backward_validate(P, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, x, Y, W,
+                                           grad_out, grad_x, grad_W, grad_Y);
   if (st != CGTP_OK) return st;
+  // only the scratch this call uses counts against the array: a grad_W-only
+  // call needs none, whatever the graph's size
+  const size_t need = cgtp::backward_scratch_bytes(P, E, grad_x != nullptr, grad_Y != nullptr, nullptr);
   if (need > kScratchBytes) {
     char msg[200];
     std::snprintf(msg, sizeof msg,
@@ -68,11 +74,13 @@ extern "C" cgtp_status cgtp_backward_static_scratch(
     return cgtp::fail(CGTP_ERR_WORKSPACE, msg);
   }
   void* ws = nullptr;
-  st = scratch_address(&ws);
-  if (st != CGTP_OK) return st;
+  if (need > 0) {
+    st = scratch_address(&ws);
+    if (st != CGTP_OK) return st;
+  }
   // the scratch needs no initial contents: every byte the backward reads
   // from it is written earlier in the same call
   return cgtp::backward_impl(plan, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, x, Y, W,
-                             grad_out, grad_x, grad_W, grad_Y, ws, kScratchBytes, stream,
+                             grad_out, grad_x, grad_W, grad_Y, ws, need > 0 ? kScratchBytes : 0, stream,
                              /*allow_timing=*/false);
 }

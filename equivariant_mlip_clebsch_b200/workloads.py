@@ -33,7 +33,8 @@ _L6_IN = "+".join(f"64x{l}{'e' if l % 2 == 0 else 'o'}" for l in range(7))
 _L6_EDGE = "+".join(f"1x{l}{'e' if l % 2 == 0 else 'o'}" for l in range(7))
 
 # name -> workload.  ``metric_config`` marks the one the headline number is
-# quoted on; the others are parity cases and secondary bench lines.
+# quoted on (the largest that fits one GPU); the others are parity cases and
+# the per-workload bench figures.
 CONFIGS = {
     "tiny": dict(
         desc="64 Si atoms, 2x2x2 cells, rc 5.0, Lmax 1",
@@ -43,7 +44,7 @@ CONFIGS = {
         desc="768 Si atoms, 4x4x6 cells, rc 5.0, Lmax 2 (Table 1 Case 1)",
         cells=(4, 4, 6), sigma=0.05, rc=5.0,
         irreps_in="128x0e+64x1e+32x2e", irreps_edge="1x0e+1x1e+1x2e",
-        irreps_out="224x0e+384x1e+352x2e", metric_config=True),
+        irreps_out="224x0e+384x1e+352x2e"),
     "lmax2_wide": dict(
         desc="768 Si atoms, 4x4x6 cells, rc 6.0, Lmax 2 wide (Table 1 Case 2)",
         cells=(4, 4, 6), sigma=0.05, rc=6.0,
@@ -53,7 +54,7 @@ CONFIGS = {
         desc="6144 Si atoms, 8x8x12 cells, sigma 0.1, rc 5.0, Lmax 3 (Table 1 Case 3)",
         cells=(8, 8, 12), sigma=0.1, rc=5.0,
         irreps_in="128x0e+64x1o+32x2e+32x3o", irreps_edge="1x0e+1x1o+1x2e+1x3o",
-        irreps_out="256x0e+352x1o+384x2e+320x3o"),
+        irreps_out="256x0e+352x1o+384x2e+320x3o", metric_config=True),
     "lmax6": dict(
         desc="768 Si atoms, 4x4x6 cells, rc 5.0, Lmax 6, 64 channels per degree (Fig. 1)",
         cells=(4, 4, 6), sigma=0.05, rc=5.0,

@@ -234,8 +234,12 @@ cgtp_status cgtp_plan_kernel_times(cgtp_plan plan, int max, char* names, double*
  * The scratch is a fixed array of CGTP_STATIC_SCRATCH_BYTES inside the
  * library's device code: every GPU that loads the library holds it until the
  * process exits.  The call allocates nothing (no cudaMalloc/cudaFree, no
- * library allocator).  Sizes whose cgtp_backward_workspace_size exceeds the
- * array are rejected with CGTP_ERR_WORKSPACE before any launch.
+ * library allocator).  Only the scratch the requested gradients use counts
+ * against the array: the per-edge messages (E x d_in floats) when grad_x is
+ * wanted, and the slice parts of grad_Y for plans of several slices; a
+ * grad_W-only call uses none.  A call that needs more is rejected with
+ * CGTP_ERR_WORKSPACE before any launch, and every argument check of
+ * cgtp_backward runs before the array is touched.
  *   - The first call on a device looks up the array's device address with
  *     that device current (cudaGetSymbolAddress) and caches it; make that
  *     first call before any stream capture on the device.
@@ -256,6 +260,23 @@ cgtp_status cgtp_backward_static_scratch(cgtp_plan plan, int64_t n_recv, int64_t
  * kernels launched since the last call completed; CGTP_ERR_TIMEOUT is
  * returned otherwise. */
 cgtp_status cgtp_plan_check_device_error(cgtp_plan plan, int* code);
+
+/* ---- measurement ----------------------------------------------------- */
+
+/* FP32 FMA throughput probe of the current device, the measured FP32 peak
+ * that the FP32-bound workloads (Lmax >= 4) are compared with.  It is not
+ * part of the convolution: the pages quote only relative speedups, and the
+ * roofline of the FP32-bound kernels needs the device's own FMA rate.
+ * cgtp_fma_peak launches, on the given stream, 2 CTAs per SM of 512 threads,
+ * each running 8 independent FMA chains for iters x 16 steps, and stores each
+ * thread's chain sum in sink (device FP32, at least
+ * cgtp_fma_peak_sink_floats elements; contents meaningless).  *flops
+ * receives the launch's floating-point operations (2 per FMA); the caller
+ * times the launch (CUDA events on the same stream) and divides.
+ * Errors: NULL, SIZE (iters outside 1..2^24, sink too small), CUDA. */
+cgtp_status cgtp_fma_peak_sink_floats(int64_t* floats);
+cgtp_status cgtp_fma_peak(int64_t iters, float* sink, int64_t sink_floats, cgtp_stream stream,
+                          double* flops);
 
 /* ---- graph utilities (host, no GPU needed) ----------------------------- */
 

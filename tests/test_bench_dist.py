@@ -96,4 +96,11 @@ def test_reference_arm_under_torchrun_prints_one_line():
     # the same metric, unit, direction and workload as the CUDA arm
     assert d["metric"] == bench.METRIC and d["unit"] == "edges/s" and d["higher_is_better"] is True
     assert d["config"]["workload"].startswith(bench.DEFAULT_CONFIG + ":")
+    # the config dict is the one the CUDA arm prints for the same workload
+    import oracle as O
+    from equivariant_mlip_clebsch_b200 import workloads as WL
+    c = WL.CONFIGS[bench.DEFAULT_CONFIG]
+    U = O.enumerate_paths(c["irreps_in"], c["irreps_edge"], c["irreps_out"]).U
+    assert d["config"] == bench.workload_config(bench.DEFAULT_CONFIG, d["config"]["atoms"],
+                                                d["config"]["edges"], U, 2)
     assert d["steps"] == 1 and d["warmup"] == 3 and d["cpu_baseline"]["cores"] >= 1
