@@ -340,3 +340,72 @@ def double_backward(paths: Paths, rowptr, col, n_send: int, x, Y, W, g, h_x=None
         gx += dx
         gW += dW
     return gg, gx, gW, gY
+
+
+# ---------------------------------------------------------------------------
+# BranchIP sparse evaluation (BranchIP page, section "BranchIP" and the
+# Branchlegro paragraph): a router gives every edge a continuation gate
+# f_e in [0, 1]; the gate multiplies the edge's feature before the TP, so the
+# edge's TP term is scaled by f_e (the convolution is linear in W, so the gate
+# is applied to the edge's weight row here).  Dense evaluation keeps every
+# edge; sparse evaluation omits the zero-gated edges from the TP and pads the
+# skipped per-edge outputs with zeros over the full edge set.
+# ---------------------------------------------------------------------------
+def gated_forward(paths: Paths, rowptr, col, x, Y, W, gate) -> np.ndarray:
+    """Dense evaluation: every edge, its TP term scaled by its gate."""
+    gate = np.asarray(gate, dtype=np.float64)
+    return forward(paths, rowptr, col, x, Y, gate[:, None] * _f64(W))
+
+
+def gated_backward(paths: Paths, rowptr, col, n_send: int, x, Y, W, gate, g):
+    """Gradients of <g, gated_forward> with respect to x, W, Y and the gate,
+    every edge evaluated (dense).  With W' = gate * W: dW = gate * dL/dW',
+    dgate[e] = <W[e], dL/dW'[e]> (= <g[i], the edge's ungated TP term>)."""
+    gate = np.asarray(gate, dtype=np.float64)
+    W = _f64(W)
+    dx, dWp, dY = backward(paths, rowptr, col, n_send, x, Y, gate[:, None] * W, g)
+    return dx, gate[:, None] * dWp, dY, np.sum(W * dWp, axis=1)
+
+
+def active_edges(rowptr, gate):
+    """The sparse evaluation's edge set: the edges with a non-zero gate, in
+    their original (receiver-sorted) order, and the receiver CSR over them.
+    Returns (act int64 [E_A] edge ids, rowptr_A int64 [n_recv+1])."""
+    rowptr = np.asarray(rowptr, dtype=np.int64)
+    gate = np.asarray(gate, dtype=np.float64)
+    n_recv = len(rowptr) - 1
+    recv = np.repeat(np.arange(n_recv), np.diff(rowptr))
+    act = np.nonzero(gate > 0)[0]
+    rowptr_A = np.concatenate([[0], np.cumsum(np.bincount(recv[act], minlength=n_recv))]).astype(np.int64)
+    return act, rowptr_A
+
+
+def sparse_forward(paths: Paths, rowptr, col, x, Y, W, gate) -> np.ndarray:
+    """Sparse evaluation: the TP runs on the active edges only."""
+    gate = np.asarray(gate, dtype=np.float64)
+    act, rowptr_A = active_edges(rowptr, gate)
+    col = np.asarray(col)
+    return forward(paths, rowptr_A, col[act], x, _f64(Y)[act], gate[act, None] * _f64(W)[act])
+
+
+def sparse_backward(paths: Paths, rowptr, col, n_send: int, x, Y, W, gate, g):
+    """Sparse evaluation of the gradients: the backward runs on the active
+    edges only, and dW, dY and dgate of the skipped edges are zero (no
+    backward branch is built for them).  dx, dW and dY equal the dense ones
+    exactly (a zero gate scales the skipped edges' terms to zero); dgate
+    equals the dense one on active edges and is zero on skipped ones, which
+    is exact for any loss reaching the gate through a function with zero
+    slope wherever it is zero (the pages' flat-zero gate)."""
+    gate = np.asarray(gate, dtype=np.float64)
+    W, Y = _f64(W), _f64(Y)
+    act, rowptr_A = active_edges(rowptr, gate)
+    col = np.asarray(col)
+    E = len(col)
+    dx, dWp, dYa = backward(paths, rowptr_A, col[act], n_send, x, Y[act], gate[act, None] * W[act], g)
+    dW = np.zeros((E, paths.U))
+    dY = np.zeros((E, paths.D_e))
+    dgate = np.zeros(E)
+    dW[act] = gate[act, None] * dWp
+    dY[act] = dYa
+    dgate[act] = np.sum(W[act] * dWp, axis=1)
+    return dx, dW, dY, dgate
