@@ -390,6 +390,52 @@ def per_workload_entry(wb: "Workbench", k: int, use_graph: bool, hbm: float, fp3
     return d
 
 
+def sparse_field(wb: "Workbench", k: int, ms_dense_step: float, ms_dense_fwd: float) -> dict:
+    """The BranchIP sparse evaluation (cgtp_sparse_forward / _backward, all
+    four gradients) on the workload with 25, 50 and 75 % of the edges
+    active, timed like the step (harmonics included, L2 flushed)."""
+    import torch
+    plan, T, E = wb.plan, wb.T, wb.E
+    ws = torch.empty(max(plan.sparse_workspace_size(wb.N, wb.N, E), 256), dtype=torch.uint8, device=wb.dev)
+    dg = torch.empty(E, device=wb.dev)
+    out = {"what": "sph_harm + sparse forward (+ sparse backward: dx, dW, dY, dgate, zero-padded); gate "
+                   "~ workloads.draw_gate (random edges, gate U(0,1] when active)"}
+    for frac in (0.25, 0.5, 0.75):
+        gate = torch.from_numpy(WL.draw_gate(E, frac)).to(wb.dev)
+        n_act = int((gate > 0).sum().item())
+
+        def fwd():
+            plan.sph_harm(T["r"], wb.Y)
+            plan.sparse_forward(T["rowptr"], T["col"], T["x"], wb.Y, T["W"], gate, out=wb.out, workspace=ws)
+
+        def step():
+            fwd()
+            plan.sparse_backward(T["rowptr"], T["col"], T["rpt"], T["perm"], T["x"], wb.Y, T["W"], gate, T["g"],
+                                 grads=(wb.dx, wb.dW, wb.dY, dg), workspace=ws)
+        step()
+        torch.cuda.synchronize()
+        ms_f = wb.timer(fwd, k)
+        ms_s = wb.timer(step, k)
+        plan.check_device_error()
+        out[f"{int(frac * 100)}%"] = {
+            "active_edges": n_act, "fwd_ms": ms_f, "fwd_bwd_ms": ms_s,
+            "fwd_bwd_edges_per_s": E / (ms_s * 1e-3), "active_edges_per_s": n_act / (ms_s * 1e-3),
+            "speedup_vs_dense_fwd_bwd": ms_dense_step / ms_s, "speedup_vs_dense_fwd": ms_dense_fwd / ms_f}
+    return out
+
+
+def graph_check_cost(wb: "Workbench", k: int) -> dict:
+    """Device time the plan's graph checks add to one forward call (the
+    checks, the read-back of their result and the wait for it)."""
+    ms_off = wb.timer(wb.fwd, k)
+    wb.plan.set_checks(True)
+    try:
+        ms_on = wb.timer(wb.fwd, k)
+    finally:
+        wb.plan.set_checks(False)
+    return {"fwd_ms_checks_off": ms_off, "fwd_ms_checks_on": ms_on, "ms_added": ms_on - ms_off}
+
+
 def run_cgtp(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -475,6 +521,11 @@ def run_cgtp(args, rank, world, local_rank):
         del hx, hW, hY, dgrads, dws
     except (C.CgtpError, ValueError, TypeError) as e:  # reported, the headline stands
         double_backward = {"error": str(e)}
+    # BranchIP sparse evaluation at 25 / 50 / 75 % active edges, after the step
+    try:
+        sparse = sparse_field(wb, args.steps, ms_step_local, fwd_ms)
+    except (C.CgtpError, ValueError, TypeError) as e:  # reported, the headline stands
+        sparse = {"error": str(e)}
     hbm, smax, pk_kind = peaks()
     if "achieved_gbs" in double_backward:
         double_backward["frac_hbm"] = double_backward["achieved_gbs"] / hbm
@@ -517,7 +568,7 @@ def run_cgtp(args, rank, world, local_rank):
                fwd_ms=fwd_ms, ms_per_step_launched=ms_eager,
                force_chain={"ms": force_ms, "edges_per_s": world * E / (force_ms * 1e-3),
                             "what": "sph_harm_backward + edge_forces after the step (not in it)"},
-               virial=virial, double_backward=double_backward,
+               virial=virial, double_backward=double_backward, sparse=sparse,
                roofline=roof, fp32_peak=fp32, kernels=kernels, gpu_launches=int(gpu_launches), e2e=e2e,
                clocks=clocks_main)
     # the five workloads of the target, each measured on its own (the headline
@@ -536,6 +587,7 @@ def run_cgtp(args, rank, world, local_rank):
                 w2.warm(3)
                 per[nm] = per_workload_entry(w2, k, use_graph, hbm, fp32, world,
                                              args.cpu_budget / 4 if rank == 0 else 0.0)
+                per[nm]["graph_checks"] = graph_check_cost(w2, k)
                 per[nm]["plan_and_graph_s"] = w2.setup_s
                 w2.close()
                 del w2

@@ -52,7 +52,11 @@ _SIGS = {
                                           _P, _P, _P]),
     "cgtp_plan_check_device_error": (_i, [_P, ctypes.POINTER(_i)]),
     "cgtp_plan_set_timing": (_i, [_P, _i]),
+    "cgtp_plan_set_checks": (_i, [_P, _i]),
     "cgtp_plan_kernel_times": (_i, [_P, _i, ctypes.c_char_p, _P, _P, ctypes.POINTER(_i)]),
+    "cgtp_sparse_workspace_size": (_i, [_P, _i64, _i64, _i64, ctypes.POINTER(_sz)]),
+    "cgtp_sparse_forward": (_i, [_P, _i64, _i64, _i64] + [_P] * 8 + [_sz, _P]),
+    "cgtp_sparse_backward": (_i, [_P, _i64, _i64, _i64] + [_P] * 14 + [_sz, _P]),
     "cgtp_fma_peak_sink_floats": (_i, [_pi64]),
     "cgtp_fma_peak": (_i, [_i64, _P, _i64, _P, ctypes.POINTER(_d)]),
     "cgtp_neighbor_list": (_i, [_i64, _P, _P, _d, _P, _P, _P, _P, _pi64]),
@@ -244,6 +248,11 @@ class Plan:
         code = ctypes.c_int()
         _check(_lib.cgtp_plan_check_device_error(self._h, ctypes.byref(code)))
 
+    def set_checks(self, enable: bool) -> None:
+        """cgtp_plan_set_checks: device checks of the graph before every call
+        (each call then waits for their result)."""
+        _check(_lib.cgtp_plan_set_checks(self._h, 1 if enable else 0))
+
     def set_timing(self, enable: bool) -> None:
         _check(_lib.cgtp_plan_set_timing(self._h, int(bool(enable))))
 
@@ -366,6 +375,58 @@ class Plan:
         _check(_lib.cgtp_double_backward(self._h, n_recv, n_send, E, *ptrs, *_workspace(workspace, dev),
                                          _stream(stream)))
         return gg, gx, gW, gY
+
+    # ---- BranchIP sparse evaluation (zero-gated edges skipped)
+    def sparse_workspace_size(self, n_recv: int, n_send: int, E: int) -> int:
+        b = ctypes.c_size_t()
+        _check(_lib.cgtp_sparse_workspace_size(self._h, n_recv, n_send, E, ctypes.byref(b)))
+        return b.value
+
+    def _sparse_ws(self, workspace, n_recv, n_send, E, dev):
+        if workspace is None:
+            import torch
+            workspace = torch.empty(max(self.sparse_workspace_size(n_recv, n_send, E), 256),
+                                    dtype=torch.uint8, device=dev)
+        return _workspace(workspace, dev)
+
+    def sparse_forward(self, rowptr, col, x, Y, W, gate, out=None, workspace=None, stream=None):
+        """cgtp_sparse_forward: out[i] = sum_e gate[e] TP_e over the edges with
+        gate > 0 only (the full graph and full W, Y, gate are passed)."""
+        import torch
+        n_recv, n_send, E, dev = rowptr.shape[0] - 1, x.shape[0], col.shape[0], x.device
+        if out is None:
+            out = torch.empty((n_recv, self.d_out), dtype=torch.float32, device=dev)
+        ptrs = _args(dev, (rowptr, "rowptr", n_recv + 1, "i32"), (col, "col", E, "i32"),
+                     (x, "x", n_send * self.d_in, "f32"), (Y, "Y", E * self.d_edge, "f32"),
+                     (W, "W", E * self.n_weights, "f32"), (gate, "gate", E, "f32"),
+                     (out, "out", n_recv * self.d_out, "f32"))
+        _check(_lib.cgtp_sparse_forward(self._h, n_recv, n_send, E, *ptrs,
+                                        *self._sparse_ws(workspace, n_recv, n_send, E, dev), _stream(stream)))
+        return out
+
+    def sparse_backward(self, rowptr, col, rowptr_T, perm_T, x, Y, W, gate, grad_out,
+                        want=("x", "W", "Y", "gate"), grads=None, workspace=None, stream=None):
+        """cgtp_sparse_backward: (dx, dW, dY, dgate) over the full edge set,
+        zero on the skipped edges."""
+        import torch
+        n_recv, n_send, E, dev = rowptr.shape[0] - 1, x.shape[0], col.shape[0], x.device
+        if grads is None:
+            f = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
+            grads = (f(n_send, self.d_in) if "x" in want else None,
+                     f(E, self.n_weights) if "W" in want else None,
+                     f(E, self.d_edge) if "Y" in want else None,
+                     f(E) if "gate" in want else None)
+        dx, dW, dY, dg = grads
+        ptrs = _args(dev, (rowptr, "rowptr", n_recv + 1, "i32"), (col, "col", E, "i32"),
+                     (rowptr_T, "rowptr_T", n_send + 1, "i32"), (perm_T, "perm_T", E, "i32"),
+                     (x, "x", n_send * self.d_in, "f32"), (Y, "Y", E * self.d_edge, "f32"),
+                     (W, "W", E * self.n_weights, "f32"), (gate, "gate", E, "f32"),
+                     (grad_out, "grad_out", n_recv * self.d_out, "f32"),
+                     (dx, "grad_x", n_send * self.d_in, "f32"), (dW, "grad_W", E * self.n_weights, "f32"),
+                     (dY, "grad_Y", E * self.d_edge, "f32"), (dg, "grad_gate", E, "f32"))
+        _check(_lib.cgtp_sparse_backward(self._h, n_recv, n_send, E, *ptrs,
+                                         *self._sparse_ws(workspace, n_recv, n_send, E, dev), _stream(stream)))
+        return dx, dW, dY, dg
 
     def backward_static_scratch(self, rowptr, col, rowptr_T, perm_T, x, Y, W, grad_out,
                                 want=("x", "W", "Y"), grads=None, stream=None):

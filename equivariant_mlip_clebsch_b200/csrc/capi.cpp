@@ -45,6 +45,8 @@ void destroy_plan_device(Plan& P) {
   }
   if (P.d_err) cudaFree(P.d_err);
   P.d_err = nullptr;
+  if (P.d_csr) cudaFree(P.d_csr);
+  P.d_csr = nullptr;
 }
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
@@ -180,7 +182,9 @@ cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge, con
       CGTP_CUDA_TRY(cudaFree(0));  // make the primary context current
       if (cudaMalloc(&P->d_err, sizeof(int)) != cudaSuccess) return fail(CGTP_ERR_OOM, "cudaMalloc");
       CGTP_CUDA_TRY(cudaMemset(P->d_err, 0, sizeof(int)));
+      if (cudaMalloc(&P->d_csr, sizeof(int)) != cudaSuccess) return fail(CGTP_ERR_OOM, "cudaMalloc");
       CGTP_CUDA_TRY(upload_sph_norm());  // once per device, before any capture
+      if (const char* d = std::getenv("CGTP_DEBUG"); d && *d && *d != '0') P->checks.store(CGTP_CHECK_GRAPH);
     }
     st = build_forward(*P);  // leaves the forward compiling on a host thread
     if (st == CGTP_OK) st = build_backward(*P);
@@ -307,30 +311,7 @@ cgtp_status cgtp_edge_virial(int64_t E, const float* r, const float* grad_r, flo
 cgtp_status cgtp_forward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
                          const int32_t* rowptr, const int32_t* col, const float* x, const float* Y,
                          const float* W, float* out, cgtp_stream stream) {
-  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
-  Plan* P = reinterpret_cast<Plan*>(plan);
-  if (n_recv < 0 || n_send < 0 || E < 0 || n_recv >= (int64_t(1) << 31) ||
-      n_send >= (int64_t(1) << 31) || E >= (int64_t(1) << 31) - 1)
-    return fail(CGTP_ERR_SIZE, "sizes out of range");
-  if (n_recv == 0) return CGTP_OK;
-  if (!rowptr || !out) return fail(CGTP_ERR_NULL, "rowptr or out is NULL");
-  if (E > 0 && (!col || !Y || !W || !x)) return fail(CGTP_ERR_NULL, "col, x, Y or W is NULL");
-  if (E > 0 && n_send == 0) return fail(CGTP_ERR_SIZE, "edges without senders");
-  for (const void* p : {(const void*)x, (const void*)Y, (const void*)W, (const void*)out})
-    if (p && !aligned16(p)) return fail(CGTP_ERR_ALIGN, "float arrays must be 16-byte aligned");
-  cgtp_status st = check_device(*P);
-  if (st != CGTP_OK) return st;
-  cudaStream_t s = (cudaStream_t)stream;
-  if (P->fwd_roles.empty()) {
-    CGTP_CUDA_TRY(cudaMemsetAsync(out, 0, (size_t)n_recv * P->D_out * sizeof(float), s));
-    return CGTP_OK;
-  }
-  int nr = (int)n_recv;
-  // persistent CTAs: about one wave of resident CTAs, each walking its slice's
-  // receivers first, first + stride, ...
-  void* args[] = {&rowptr, &col, &x, &Y, &W, &out, &P->d_fwd_ent, &nr, &P->d_err};
-  TimedScope ts(*P, 1, s);
-  return jit_launch(P->fwd, dim3(persistent_grid(P->fwd.blocks_per_sm, P->num_sms, n_recv)), args, s);
+  return cgtp::forward_impl(plan, n_recv, n_send, E, rowptr, col, x, Y, W, nullptr, out, stream, true);
 }
 
 cgtp_status cgtp_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
@@ -349,14 +330,75 @@ cgtp_status cgtp_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
                           void* workspace, size_t workspace_bytes, cgtp_stream stream) {
   return cgtp::backward_impl(plan, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, x, Y, W,
                              grad_out, grad_x, grad_W, grad_Y, workspace, workspace_bytes, stream,
-                             true);
+                             true, nullptr, true);
 }
 
 }  // extern "C"
 
 namespace cgtp {
 
+cgtp_status forward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
+                         const int32_t* col, const float* x, const float* Y, const float* W, const int32_t* eid,
+                         float* out, cgtp_stream stream, bool graph_checks) {
+  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
+  Plan* P = reinterpret_cast<Plan*>(plan);
+  if (n_recv < 0 || n_send < 0 || E < 0 || n_recv >= (int64_t(1) << 31) ||
+      n_send >= (int64_t(1) << 31) || E >= (int64_t(1) << 31) - 1)
+    return fail(CGTP_ERR_SIZE, "sizes out of range");
+  if (n_recv == 0) return CGTP_OK;
+  if (!rowptr || !out) return fail(CGTP_ERR_NULL, "rowptr or out is NULL");
+  if (E > 0 && (!col || !Y || !W || !x)) return fail(CGTP_ERR_NULL, "col, x, Y or W is NULL");
+  if (E > 0 && n_send == 0) return fail(CGTP_ERR_SIZE, "edges without senders");
+  for (const void* p : {(const void*)x, (const void*)Y, (const void*)W, (const void*)out})
+    if (p && !aligned16(p)) return fail(CGTP_ERR_ALIGN, "float arrays must be 16-byte aligned");
+  cgtp_status st = check_device(*P);
+  if (st != CGTP_OK) return st;
+  if (graph_checks && E > 0) {
+    st = check_graph(*P, n_recv, n_send, E, rowptr, col, nullptr, nullptr, stream);
+    if (st != CGTP_OK) return st;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  if (P->fwd_roles.empty()) {
+    CGTP_CUDA_TRY(cudaMemsetAsync(out, 0, (size_t)n_recv * P->D_out * sizeof(float), s));
+    return CGTP_OK;
+  }
+  int nr = (int)n_recv;
+  // persistent CTAs: about one wave of resident CTAs, each walking its slice's
+  // receivers first, first + stride, ...
+  void* args[] = {&rowptr, &col, &x, &Y, &W, &eid, &out, &P->d_fwd_ent, &nr, &P->d_err};
+  TimedScope ts(*P, 1, s);
+  return jit_launch(P->fwd, dim3(persistent_grid(P->fwd.blocks_per_sm, P->num_sms, n_recv)), args, s);
+}
+
 cgtp_status check_plan_device(const Plan& P) { return check_device(P); }
+
+cgtp_status check_graph(Plan& P, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
+                        const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, cgtp_stream stream) {
+  if (!(P.checks.load() & CGTP_CHECK_GRAPH) || (n_recv == 0 && E == 0)) return CGTP_OK;
+  if (!rowptr || (E > 0 && !col)) return fail(CGTP_ERR_NULL, "rowptr or col is NULL");
+  if (!rowptr_T || !perm_T) rowptr_T = nullptr, perm_T = nullptr;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  CGTP_CUDA_TRY(cudaStreamIsCapturing(s, &cs));
+  if (cs != cudaStreamCaptureStatusNone)
+    return fail(CGTP_ERR_CUDA, "the graph checks wait for their result; turn them off under stream capture");
+  std::lock_guard<std::mutex> g(P.csr_mu);  // one result word per plan
+  int h = 0;
+  CGTP_CUDA_TRY(cudaMemsetAsync(P.d_csr, 0, sizeof(int), s));
+  CGTP_CUDA_TRY(launch_csr_check(P.num_sms, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, P.d_csr, s));
+  CGTP_CUDA_TRY(cudaMemcpyAsync(&h, P.d_csr, sizeof(int), cudaMemcpyDeviceToHost, s));
+  CGTP_CUDA_TRY(cudaStreamSynchronize(s));
+  if (h == 0) return CGTP_OK;
+  static const char* what[] = {"rowptr does not run from 0 to E", "rowptr decreases",
+                               "a col entry lies outside [0, n_send)", "rowptr_T does not run from 0 to E",
+                               "rowptr_T decreases", "a perm_T entry lies outside [0, E)",
+                               "a perm_T entry lists an edge of another sender",
+                               "perm_T is not ascending within a sender"};
+  std::string msg = "graph checks failed:";
+  for (int b = 0; b < 8; ++b)
+    if (h & (1 << b)) msg += std::string(" ") + what[b] + ";";
+  return fail(CGTP_ERR_INVALID_CSR, msg);
+}
 
 // The scratch bytes one backward call uses: the per-edge messages when grad_x
 // is wanted (first), and the slice parts of dY when grad_Y is wanted from a
@@ -393,12 +435,17 @@ cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
                           const int32_t* perm_T, const float* x, const float* Y, const float* W,
                           const float* grad_out, float* grad_x, float* grad_W, float* grad_Y,
                           void* workspace, size_t workspace_bytes, cgtp_stream stream,
-                          bool allow_timing) {
+                          bool allow_timing, const int32_t* eid, bool graph_checks) {
   if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
   Plan* P = reinterpret_cast<Plan*>(plan);
   cgtp_status st = backward_validate(*P, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, x, Y, W, grad_out,
                                      grad_x, grad_W, grad_Y);
   if (st != CGTP_OK) return st;
+  if (graph_checks && E > 0) {
+    st = check_graph(*P, n_recv, n_send, E, rowptr, col, grad_x ? rowptr_T : nullptr, grad_x ? perm_T : nullptr,
+                     stream);
+    if (st != CGTP_OK) return st;
+  }
   cudaStream_t s = (cudaStream_t)stream;
   if (grad_x && n_send > 0 && (E == 0 || P->bwd_roles.empty()))
     CGTP_CUDA_TRY(cudaMemsetAsync(grad_x, 0, (size_t)n_send * P->D_in * sizeof(float), s));
@@ -430,7 +477,7 @@ cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
     const bool er = P->bwd_er.function && n_recv <= 8 * (int64_t)G;
     JitKernel& JK = er ? P->bwd_er : P->bwd;
     if (er) G = persistent_grid(P->bwd_er.blocks_per_sm, P->num_sms, n_recv);
-    void* args[] = {&rowptr, &col, &x, &Y, &W, &grad_out, &grad_W, &dyp, &m, &P->d_bwd_ent, &nr, &P->d_err};
+    void* args[] = {&rowptr, &col, &x, &Y, &W, &eid, &grad_out, &grad_W, &dyp, &m, &P->d_bwd_ent, &nr, &P->d_err};
     TimedScope ts(*P, 2, s, allow_timing);
     st = jit_launch(JK, dim3(G), args, s);
     if (st != CGTP_OK) return st;
@@ -500,6 +547,13 @@ cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* need
     std::memcpy(buf, t.data(), k);
     buf[k] = '\0';
   }
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_set_checks(cgtp_plan plan, int flags) {
+  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
+  if (flags & ~CGTP_CHECK_GRAPH) return fail(CGTP_ERR_SIZE, "unknown check flags");
+  reinterpret_cast<Plan*>(plan)->checks.store(flags);
   return CGTP_OK;
 }
 
@@ -598,6 +652,12 @@ cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send,
     return fail(CGTP_ERR_NULL, "col, x, Y, W or grad_out is NULL");
   if (gx && (h_W || h_Y) && E > 0 && (!rowptr_T || !perm_T))
     return fail(CGTP_ERR_NULL, "grad_x needs rowptr_T and perm_T");
+  if (n_recv > 0 && E > 0) {
+    const bool need_T = gx && (h_W || h_Y);
+    st = check_graph(*P, n_recv, n_send, E, rowptr, col, need_T ? rowptr_T : nullptr, need_T ? perm_T : nullptr,
+                     stream);
+    if (st != CGTP_OK) return st;
+  }
   const DbwdLayout L = dbwd_workspace_layout(*P, n_recv, n_send, E);
   if (!workspace || workspace_bytes < L.total)
     return fail(CGTP_ERR_WORKSPACE, "workspace of " + std::to_string(L.total) + " bytes required");
@@ -617,11 +677,11 @@ cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send,
     size_t bw_bytes;
     cgtp_stream stream;
     int forward(const float* xx, const float* yy, const float* ww, float* out) {
-      return cgtp_forward(plan, n_recv, n_send, E, rowptr, col, xx, yy, ww, out, stream);
+      return forward_impl(plan, n_recv, n_send, E, rowptr, col, xx, yy, ww, nullptr, out, stream, false);
     }
     int backward(const float* xx, const float* yy, const float* ww, float* ox, float* ow, float* oy) {
       return backward_impl(plan, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, xx, yy, ww, g, ox, ow, oy, bws,
-                           bw_bytes, stream, true);
+                           bw_bytes, stream, true, nullptr, false);
     }
     int add(float* dst, const float* src, int64_t n) {
       CGTP_CUDA_TRY(launch_add(n, src, dst, (cudaStream_t)stream));

@@ -68,7 +68,7 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
   const FwdConfig& F = P.bcfg;
   const int S = K.S, NW = K.nw;
   std::ostringstream o;
-  o << kPrelude;
+  o << spin_limit_define() << kPrelude;
   o << gen_common_device(P, SL, K, true);
 
   std::vector<int> slice_of(P.bwd_roles.size(), -1);
@@ -90,9 +90,9 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
     }
   }
   const std::string params =
-      "(const int* __restrict__ rowptr, int n_recv, float* __restrict__ dW, float* __restrict__ msg,\n"
-      "    int* __restrict__ err, unsigned char* smem, int u0, int ph, int nph, int chs, bool want_dy,\n"
-      "    int* qp, int* kp)";
+      "(const int* __restrict__ rowptr, int n_recv, const int* __restrict__ eid, float* __restrict__ dW,\n"
+      "    float* __restrict__ msg, int* __restrict__ err, unsigned char* smem, int u0, int ph, int nph, int chs,\n"
+      "    bool want_dy, int* qp, int* kp)";
   for (size_t k = 0; k < shape_rep.size(); ++k) {
     const BwdRole& r = P.bwd_roles[shape_rep[k]];
     const SliceLayout& sl = SL[slice_of[shape_rep[k]]];
@@ -113,11 +113,11 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       << "  const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
       << "  if (e1 <= e0) continue;\n"
       << "  const int gb = kr % GBUF;\n"
-      << "  if (!mbar_wait(gfull0 + 8 * gb, (kr / GBUF) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
+      << "  if (!mbar_wait(gfull0 + 8 * gb, (kr / GBUF) & 1)) { if (lane == 0) atomicOr(err, 10); *qp = -1; return; }\n"
       << "  const float* sg = reinterpret_cast<const float*>(smem + OFF_G) + gb * GS;\n"
       << "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
       << "    const int s = q % NSTAGE;\n"
-      << "    if (!mbar_wait(full0 + 8 * s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
+      << "    if (!stage_ready(full0, s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); *qp = -1; return; }\n"
       << "    const int nb = min(NB, e1 - eb);\n"
       << "    unsigned char* st = stage_ptr(smem, s);\n"
       << "    const float* sW = reinterpret_cast<const float*>(st + OFF_W);\n"
@@ -129,7 +129,7 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       << "      const float* wr = sW + b * WS;\n"
       << "      const float* xr = sX + b * XS;\n"
       << "      const float* chb = sC + b * chs;\n"
-      << "      float* dWrow = dW ? dW + (size_t)e * NU : nullptr;\n"
+      << "      float* dWrow = dW ? dW + (size_t)(eid ? __ldg(eid + e) : e) * NU : nullptr;\n"
       << "      float* sdy = want_dy ? sdyw + b * DE : nullptr;\n"
       ;
     // The R channel blocks of the role: RU of them unrolled together, the
@@ -255,7 +255,7 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
        "    if (e1 <= e0) continue;\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
        "      const int s = q % NSTAGE;\n"
-       "      if (!mbar_wait(full0 + 8 * s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
+       "      if (!stage_ready(full0, s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); *qp = -1; return; }\n"
        "      __syncwarp();\n"
        "      if (lane == 0) mbar_arrive(empty0 + 8 * s);\n"
        "    }\n"
@@ -278,8 +278,8 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
   o << "};\n";
   o << "extern \"C\" __global__ void __launch_bounds__((NW + 2) * 32, " << min_blocks << ") " << kname
     << "(const int* __restrict__ rowptr, const int* __restrict__ col, const float* __restrict__ x,\n"
-       "    const float* __restrict__ Y, const float* __restrict__ W, const float* __restrict__ g,\n"
-       "    float* __restrict__ dW, float* __restrict__ dyp, float* __restrict__ msg,\n"
+       "    const float* __restrict__ Y, const float* __restrict__ W, const int* __restrict__ eid,\n"
+       "    const float* __restrict__ g, float* __restrict__ dW, float* __restrict__ dyp, float* __restrict__ msg,\n"
        "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err) {\n"
        "  extern __shared__ __align__(128) unsigned char smem[];\n"
        "  grid_dependency_wait();  // the previous kernel's results are visible\n"
@@ -288,7 +288,9 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  const u32 gfull0 = full0 + OFF_GFULL, gempty0 = full0 + OFF_GEMPTY;\n"
        "  if (threadIdx.x == 0) {\n"
-       "    for (int s = 0; s < NSTAGE; ++s) { mbar_init(full0 + 8 * s, FULL_COUNT); mbar_init(empty0 + 8 * s, NW); }\n"
+       "    for (int s = 0; s < NSTAGE; ++s) {\n"
+       "      mbar_init(full0 + 8 * s, FULL_COUNT); mbar_init(empty0 + 8 * s, NW); mbar_init(full0 + OFF_CHAT + 8 * s, CHAT_COUNT);\n"
+       "    }\n"
        "    for (int b = 0; b < 2; ++b) { mbar_init(gfull0 + 8 * b, 32); mbar_init(gempty0 + 8 * b, NW); }\n"
        "    fence_mbar_init();\n"
        "  }\n"
@@ -303,7 +305,7 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
              "  }\n"
            : "") <<
        "  __syncthreads();\n"
-       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, g, err, smem, lane); return; }\n"
+       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, eid, g, err, smem, lane); return; }\n"
        "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, ent, kEntBegin, dyp, err, smem, lane); return; }\n"
        "  int q = 0, kr = 0;\n"
        "  for (int slice = 0; slice < NSLICE; ++slice) {\n"
@@ -312,9 +314,10 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
        "    switch (kShape[slot]) {\n";
   for (size_t k = 0; k < shape_rep.size(); ++k)
     o << "    case " << k << ": bcons_" << k
-      << "(rowptr, n_recv, dW, msg, err, smem, u0, ph, nph, chs, dyp != nullptr, &q, &kr); break;\n";
-  o << "    default: bcons_idle(rowptr, n_recv, dW, msg, err, smem, u0, ph, nph, chs, dyp != nullptr, &q, &kr); break;\n"
-       "    }\n  }\n}\n";
+      << "(rowptr, n_recv, eid, dW, msg, err, smem, u0, ph, nph, chs, dyp != nullptr, &q, &kr); break;\n";
+  o << "    default: bcons_idle(rowptr, n_recv, eid, dW, msg, err, smem, u0, ph, nph, chs, dyp != nullptr, &q, &kr); break;\n"
+       "    }\n"
+       "    if (q < 0) break;  // a wait expired: this warp stops\n  }\n}\n";
   return o.str();
 }
 

@@ -30,6 +30,13 @@ const char* kPrelude =
 #include "device_prelude.inc"
     ;
 
+std::string spin_limit_define() {
+  const char* v = std::getenv("CGTP_SPIN_LIMIT");
+  if (!v || !*v) return "";
+  const unsigned long n = std::strtoul(v, nullptr, 10);
+  return "#define CGTP_SPIN_LIMIT " + std::to_string(std::max(1ul, std::min(n, 1ul << 30))) + "u\n";
+}
+
 int max_spill_bytes(const std::string& log) {
   int best = 0;
   size_t pos = 0;
@@ -149,7 +156,7 @@ void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape&
   if (const char* v = std::getenv("CGTP_STAGES")) K.stages = std::max(2, std::min(6, std::atoi(v)));
   while (K.stages > 2 && fixed + K.stages * stage_of(K.B) > 220 * 1024) --K.stages;
   K.sdy_floats = backward ? K.nw * K.B * (int)P.D_e : 0;
-  K.off_stage = 256;  // mbarriers first
+  K.off_stage = 512;  // mbarriers, chunk descriptors and the edge range first
   K.off_w = 0;
   K.off_x = r128(4L * K.B * K.WS);
   K.off_y = K.off_x + r128(4L * K.B * K.XS);
@@ -198,17 +205,24 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
     << "\n#define OFF_STAGE " << K.off_stage << "\n#define OFF_W " << K.off_w << "\n#define OFF_X "
     << K.off_x << "\n#define OFF_Y " << K.off_y << "\n#define OFF_CH " << K.off_ch << "\n#define OFF_DY "
     << K.off_dy << "\n#define OFF_G " << K.off_g << "\n#define GS " << K.GS << "\n#define WB " << K.WB
-    << "\n#define OFF_WB " << K.off_wb << "\n#define FULL_COUNT 64\n#define GBUF " << K.gbufs << "\n#define YPL "
+    << "\n#define OFF_WB " << K.off_wb << "\n#define FULL_COUNT 32\n#define CHAT_COUNT 32\n#define GBUF " << K.gbufs << "\n#define YPL "
     << (K.B * P.D_e + 31) / 32 << "\n";
-  // shared-memory header: full[NSTAGE], empty[NSTAGE], gfull[2], gempty[2]
-  // mbarriers, then the helper's per-stage chunk descriptors
-  o << "#define OFF_GFULL (2 * NSTAGE * 8)\n#define OFF_GEMPTY (OFF_GFULL + 16)\n#define OFF_DESC (OFF_GEMPTY + 16)\n";
+  // shared-memory header: full[NSTAGE] (the TMA warp's 32 lanes and the
+  // bytes of its copies), empty[NSTAGE] (one arrival per consumer warp),
+  // chat[NSTAGE] (the helper's 32 lanes: Y and Chat of the stage written),
+  // gfull[2], gempty[2] mbarriers, the helper's per-stage chunk descriptors,
+  // and the edge range of the edge-range variant, all below OFF_STAGE
+  o << "#define OFF_CHAT (2 * NSTAGE * 8)\n#define OFF_GFULL (3 * NSTAGE * 8)\n#define OFF_GEMPTY (OFF_GFULL + 16)\n"
+       "#define OFF_DESC (OFF_GEMPTY + 16)\n#define OFF_RANGE (OFF_DESC + 16 * NSTAGE)\n";
+  // a stage is ready for the consumers when its copies have landed and its
+  // Chat is built
+  o << "__device__ __forceinline__ bool stage_ready(u32 full0, int s, u32 parity) {\n"
+       "  return mbar_wait(full0 + 8 * s, parity) && mbar_wait(full0 + OFF_CHAT + 8 * s, parity);\n}\n";
   // the receivers a CTA walks: whole receivers blockIdx.x, + gridDim.x, ...,
   // or (backward, edge_ranges) an equal share of the edges, receivers clipped
   // to it (the range sits in the header at OFF_RANGE)
   if (backward && K.edge_ranges)
-    o << "#define OFF_RANGE 240\n"
-         "#define RANGE_AT(k) (reinterpret_cast<const int*>(smem + OFF_RANGE)[k])\n"
+    o << "#define RANGE_AT(k) (reinterpret_cast<const int*>(smem + OFF_RANGE)[k])\n"
          "#define RECV_FIRST RANGE_AT(0)\n#define RECV_END RANGE_AT(1)\n#define RECV_STEP 1\n"
          "#define EDGE_LO(i) max(rowptr[i], RANGE_AT(2))\n#define EDGE_HI(i) min(rowptr[(i) + 1], RANGE_AT(3))\n";
   else
@@ -238,15 +252,19 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
   // ---- TMA warp.  Every warp of a CTA walks the same sequence: for each
   // slice in order, the receivers blockIdx.x, + gridDim.x, ..., and their
   // chunks; the running chunk counter q picks the stage and the phase.
+  // eid (nullable): the edges' ids in the full edge set, whose W rows the
+  // chunk reads (the sparse evaluation's active edges); NULL: W row = edge
   o << "__device__ __noinline__ void tma_warp(const int* __restrict__ rowptr, int n_recv,\n"
        "    const int* __restrict__ col, const float* __restrict__ x, const float* __restrict__ W,\n"
-       "    const float* __restrict__ g, int* __restrict__ err, unsigned char* smem, int lane) {\n"
+       "    const int* __restrict__ eid, const float* __restrict__ g, int* __restrict__ err,\n"
+       "    unsigned char* smem, int lane) {\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  const u32 gfull0 = full0 + OFF_GFULL, gempty0 = full0 + OFF_GEMPTY;\n"
        "  (void)gfull0; (void)gempty0; (void)g;\n"
        "  const u64 pol = policy_evict_first();\n"
        "  (void)pol;\n"
-       "  int q = 0, k = 0;\n"
+       "  int q = 0, k = 0;  // chunks and grad_out loads issued\n"
+       "  (void)k;\n"
        "  bool dead = false;\n"
        "  for (int slice = 0; slice < NSLICE && !dead; ++slice) {\n"
        "  for (int i = RECV_FIRST; i < RECV_END && !dead; i += RECV_STEP) {\n"
@@ -296,9 +314,13 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
       << ((K.w_bulk ? wb : 0) + (K.x_bulk ? xb : 0)) << ");\n"
       << "        __syncwarp();\n";
     std::ostringstream cp;
-    cp << "#define WROW(b) (W + (size_t)(eb + (b)) * NU)\n";
+    // W rows: consecutive for a chunk of one receiver's edges, or (eid) the
+    // rows of the listed edges, one copy per edge
+    cp << "if (eid == nullptr) {\n#define WROW(b) (W + (size_t)(eb + (b)) * NU)\n";
     gen_copy_pieces(cp, sl.wseg, K.w_bulk, "sW", K.WS, "WROW", "full0 + 8 * s", w_one, P.U);
-    cp << "#undef WROW\n";
+    cp << "#undef WROW\n} else {\n#define WROW(b) (W + (size_t)__ldg(eid + eb + (b)) * NU)\n";
+    gen_copy_pieces(cp, sl.wseg, K.w_bulk, "sW", K.WS, "WROW", "full0 + 8 * s", false, P.U);
+    cp << "#undef WROW\n}\n";
     if (K.x_bulk) {
       cp << "#define XROW(b) (x + (size_t)jj * DIN)\n";
       gen_copy_pieces(cp, sl.xseg, true, "sX", K.XS, "XROW", "full0 + 8 * s", false, P.D_in);
@@ -324,9 +346,16 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
   o << "    }\n"
        "  }\n"
        "  }\n"
-       "  // bulk copies still in flight must land before the CTA may exit\n"
-       "  if (lane == 0)\n"
-       "    for (int c = max(0, q - NSTAGE); c < q; ++c) mbar_wait(full0 + 8 * (c % NSTAGE), (c / NSTAGE) & 1);\n"
+       "  // every bulk copy this warp issued must land before the CTA may exit:\n"
+       "  // the last NSTAGE chunks' and the last GBUF grad_out loads' barriers\n"
+       "  // complete on this warp's own arrivals and bytes alone\n"
+       "  if (lane == 0) {\n"
+       "    for (int c = max(0, q - NSTAGE); c < q; ++c)\n"
+       "      if (!mbar_wait_drain(full0 + 8 * (c % NSTAGE), (c / NSTAGE) & 1)) atomicOr(err, 10);\n";
+  if (backward)
+    o << "    for (int c = max(0, k - GBUF); c < k; ++c)\n"
+         "      if (!mbar_wait_drain(gfull0 + 8 * (c % GBUF), (c / GBUF) & 1)) atomicOr(err, 10);\n";
+  o << "  }\n"
        "}\n";
 
   // ---- helper warp
@@ -423,7 +452,7 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
          "          cb[r.x & 0xffff] = fmaf(__int_as_float(r.y), y[(r.x >> 16) & 0xff], __int_as_float(r.z) * y[(unsigned)r.x >> 24]);\n"
          "        }\n"
          "      }\n";
-  o << "      mbar_arrive(full0 + 8 * s);\n"
+  o << "      mbar_arrive(full0 + OFF_CHAT + 8 * s);\n"
        "    }\n"
        "  }\n"
        "  }\n";

@@ -13,6 +13,11 @@ namespace cgtp {
 
 extern const char* kPrelude;
 
+// "#define CGTP_SPIN_LIMIT n" when the CGTP_SPIN_LIMIT environment variable
+// is set at plan creation (a smaller bound for the pipeline waits, for tests
+// of the kernels' wind-down after an expired wait), else "".
+std::string spin_limit_define();
+
 inline int pad4(int n) { return (n + 3) & ~3; }
 
 // Chat_{e,p} = sum_m2 C_p[m1][m2][m3] Y[e][l2^2+m2], stored per edge and path

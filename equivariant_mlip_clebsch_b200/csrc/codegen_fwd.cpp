@@ -38,26 +38,29 @@ static void gen_fwd_entry(std::ostringstream& o, const std::string& kname, int m
                           const std::string& dispatch) {
   o << "extern \"C\" __global__ void __launch_bounds__((NW + 2) * 32, " << min_blocks << ") " << kname
     << "(const int* __restrict__ rowptr, const int* __restrict__ col, const float* __restrict__ x,\n"
-       "    const float* __restrict__ Y, const float* __restrict__ W, float* __restrict__ out,\n"
-       "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err) {\n"
+       "    const float* __restrict__ Y, const float* __restrict__ W, const int* __restrict__ eid,\n"
+       "    float* __restrict__ out, const int4* __restrict__ ent, int n_recv, int* __restrict__ err) {\n"
        "  extern __shared__ __align__(128) unsigned char smem[];\n"
        "  grid_dependency_wait();  // the previous kernel's results are visible\n"
        "  grid_launch_dependents();\n"
        "  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  if (threadIdx.x == 0) {\n"
-       "    for (int s = 0; s < NSTAGE; ++s) { mbar_init(full0 + 8 * s, FULL_COUNT); mbar_init(empty0 + 8 * s, NW); }\n"
+       "    for (int s = 0; s < NSTAGE; ++s) {\n"
+       "      mbar_init(full0 + 8 * s, FULL_COUNT); mbar_init(empty0 + 8 * s, NW); mbar_init(full0 + OFF_CHAT + 8 * s, CHAT_COUNT);\n"
+       "    }\n"
        "    fence_mbar_init();\n"
        "  }\n"
        "  __syncthreads();\n"
-       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, nullptr, err, smem, lane); return; }\n"
+       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, eid, nullptr, err, smem, lane); return; }\n"
        "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, ent, kEntBegin, nullptr, err, smem, lane); return; }\n"
        "  int q = 0;\n"
        "  for (int slice = 0; slice < NSLICE; ++slice) {\n"
        "    const int slot = slice * NW + warp;\n"
        "    const int u0 = kU0[slot], chs = kChs[slice];\n"
        "    switch (kShape[slot]) {\n"
-    << dispatch << "    default: fcons_idle(rowptr, n_recv, err, smem, &q); break;\n    }\n  }\n}\n";
+    << dispatch << "    default: fcons_idle(rowptr, n_recv, err, smem, &q); break;\n    }\n"
+       "    if (q < 0) break;  // a wait expired: this warp stops\n  }\n}\n";
 }
 
 static void gen_fwd_idle(std::ostringstream& o) {
@@ -71,7 +74,7 @@ static void gen_fwd_idle(std::ostringstream& o) {
        "    const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
        "      const int s = q % NSTAGE;\n"
-       "      if (!mbar_wait(full0 + 8 * s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
+       "      if (!stage_ready(full0, s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); *qp = -1; return; }\n"
        "      __syncwarp();\n"
        "      if (lane == 0) mbar_arrive(empty0 + 8 * s);\n"
        "    }\n"
@@ -116,7 +119,7 @@ static std::string gen_fwd_generic(const Plan& P, const std::vector<SliceLayout>
          "#pragma unroll\n  for (int k = 0; k < " << N3 << "; ++k) acc[k] = 0.f;\n"
          "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
          "    const int s = q % NSTAGE;\n"
-         "    if (!mbar_wait(full0 + 8 * s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
+         "    if (!stage_ready(full0, s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); *qp = -1; return; }\n"
          "    const int nb = min(NB, e1 - eb);\n"
          "    const unsigned char* st = stage_ptr(smem, s);\n"
          "    const float* sW = reinterpret_cast<const float*>(st + OFF_W) + wst;\n"
@@ -169,7 +172,7 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
   const FwdConfig& F = P.fcfg;
   const int S = K.S, NW = K.nw;
   std::ostringstream o;
-  o << kPrelude;
+  o << spin_limit_define() << kPrelude;
   o << gen_common_device(P, SL, K, false);
 
   std::vector<int> slice_of(P.fwd_roles.size(), -1);
@@ -216,7 +219,7 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
          "#pragma unroll\n  for (int k = 0; k < " << nacc << "; ++k) acc[k] = 0.f;\n"
          "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
          "    const int s = q % NSTAGE;\n"
-         "    if (!mbar_wait(full0 + 8 * s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); return; }\n"
+         "    if (!stage_ready(full0, s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); *qp = -1; return; }\n"
          "    const int nb = min(NB, e1 - eb);\n"
          "    const unsigned char* st = stage_ptr(smem, s);\n"
          "    const float* sW = reinterpret_cast<const float*>(st + OFF_W);\n"

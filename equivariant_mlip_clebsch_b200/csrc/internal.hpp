@@ -150,6 +150,11 @@ struct Plan {
   bool bwd_irrep_gap = false;  // some hidden irrep has no path
 
   int* d_err = nullptr;  // device error word
+  // device checks of the graph before each call (cgtp_plan_set_checks;
+  // CGTP_DEBUG=1 at plan creation): flags, the result word, its lock
+  std::atomic<int> checks{0};
+  int* d_csr = nullptr;
+  std::mutex csr_mu;
   // kernel timing (cgtp_plan_set_timing)
   std::atomic<bool> timing{false};  // read by launches on any thread
   std::mutex tmu;
@@ -166,15 +171,28 @@ struct Plan {
   std::unique_ptr<PendingCompile> fwd_pending;
 };
 
+// The forward and backward behind the C ABI.  eid (nullable, device int32
+// [E]): the full-set ids of the listed edges, whose W rows (and grad_W rows)
+// the kernels read (write) instead of row e (the sparse evaluation's active
+// edges); NULL for the plain convolution.
+// graph_checks: run the plan's graph checks (when on) on this call's graph.
+cgtp_status forward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
+                         const int32_t* col, const float* x, const float* Y, const float* W, const int32_t* eid,
+                         float* out, cgtp_stream stream, bool graph_checks);
 cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
                           const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
                           const int32_t* perm_T, const float* x, const float* Y, const float* W,
                           const float* grad_out, float* grad_x, float* grad_W, float* grad_Y,
                           void* workspace, size_t workspace_bytes, cgtp_stream stream,
-                          bool allow_timing);
+                          bool allow_timing, const int32_t* eid, bool graph_checks);
 
 // The plan's device is current and the plan has device state.
 cgtp_status check_plan_device(const Plan& P);
+// With the plan's CSR checks on: runs them on the stream, waits for their
+// result and returns CGTP_ERR_INVALID_CSR (with the failed checks in the
+// message) before any kernel reads through the graph.  OK when checks are off.
+cgtp_status check_graph(Plan& P, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
+                        const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, cgtp_stream stream);
 // Host checks of a backward call (sizes, device, alignment, required pointers).
 cgtp_status backward_validate(const Plan& P, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
                               const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, const float* x,
@@ -210,6 +228,11 @@ cudaError_t launch_edge_virial(int64_t E, const float* r, const float* G, float*
 cudaError_t launch_add(int64_t n, const float* src, float* dst, cudaStream_t s);
 // c_norm of the harmonics kernels, uploaded once per device (plan creation)
 cudaError_t upload_sph_norm();
+// The graph's device checks (bits in *flag, see kernels.cu); the sender
+// lists are checked when rowptr_T and perm_T are given.
+cudaError_t launch_csr_check(int num_sms, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
+                             const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, int* flag,
+                             cudaStream_t s);
 // FP32 FMA throughput probe: 2 CTAs per SM; flops receives the launch's FLOPs
 int64_t fma_peak_sink_floats(int num_sms);
 cudaError_t launch_fma_peak(int num_sms, int64_t iters, float m, float c, float* sink, cudaStream_t s,

@@ -321,6 +321,62 @@ __global__ void __launch_bounds__(256) add_kernel(int64_t n, const float* __rest
   for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += stride) dst[i] += src[i];
 }
 
+// Device checks of the graph (a plan's CSR checks, cgtp_plan_set_checks).
+// Bits of the flag word: 1 rowptr does not run from 0 to E, 2 rowptr
+// decreases, 4 a col outside [0, n_send), 8 rowptr_T does not run from 0 to E,
+// 16 rowptr_T decreases, 32 a perm_T entry outside [0, E), 64 a perm_T entry
+// whose edge has another sender, 128 perm_T not strictly ascending within a
+// sender.  Phase 1 reads only the arrays' own extents; phase 2 (the sender
+// lists) runs only when phase 1 found nothing, so its loops follow validated
+// bounds.
+__global__ void __launch_bounds__(256) csr_check_kernel(int64_t n_recv, int64_t n_send, int64_t E,
+                                                        const int32_t* __restrict__ rowptr,
+                                                        const int32_t* __restrict__ col,
+                                                        const int32_t* __restrict__ rowptr_T,
+                                                        int* __restrict__ flag) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  int bad = 0;
+  if (t0 == 0) {
+    if (rowptr[0] != 0 || rowptr[n_recv] != E) bad |= 1;
+    if (rowptr_T && (rowptr_T[0] != 0 || rowptr_T[n_send] != E)) bad |= 8;
+  }
+  for (int64_t i = t0; i < n_recv; i += stride)
+    if (rowptr[i] > rowptr[i + 1]) bad |= 2;
+  for (int64_t e = t0; e < E; e += stride) {
+    const int32_t j = col[e];
+    if (j < 0 || j >= n_send) bad |= 4;
+  }
+  if (rowptr_T)
+    for (int64_t j = t0; j < n_send; j += stride)
+      if (rowptr_T[j] > rowptr_T[j + 1]) bad |= 16;
+  if (bad) atomicOr(flag, bad);
+}
+
+__global__ void __launch_bounds__(256) csr_perm_check_kernel(int64_t n_send, int64_t E,
+                                                             const int32_t* __restrict__ col,
+                                                             const int32_t* __restrict__ rowptr_T,
+                                                             const int32_t* __restrict__ perm_T,
+                                                             int* __restrict__ flag) {
+  if (*(volatile int*)flag) return;  // phase 1 failed: the bounds below are not trusted
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  int bad = 0;
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n_send; j += stride) {
+    int32_t prev = -1;
+    for (int32_t t = rowptr_T[j]; t < rowptr_T[j + 1]; ++t) {
+      const int32_t e = perm_T[t];
+      if (e < 0 || e >= E) {
+        bad |= 32;
+        break;
+      }
+      if (col[e] != j) bad |= 64;
+      if (e <= prev) bad |= 128;
+      prev = e;
+    }
+  }
+  if (bad) atomicOr(flag, bad);
+}
+
 // FP32 FMA throughput probe (the measured FP32 peak the Lmax >= 4 workloads
 // are compared with).  Every thread runs kFmaChains independent dependency
 // chains a <- a * m + c, kFmaUnroll steps per loop trip; with 512 threads per
@@ -491,6 +547,17 @@ cudaError_t launch_edge_forces(int64_t n_atoms, const int32_t* rowptr, const int
 
 cudaError_t launch_edge_virial(int64_t E, const float* r, const float* G, float* V, cudaStream_t s) {
   return launch_pdl(edge_virial_kernel, dim3(kVirCtas), kVirThreads, s, E, r, G, V);
+}
+
+cudaError_t launch_csr_check(int num_sms, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
+                             const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, int* flag,
+                             cudaStream_t s) {
+  const int64_t work = std::max<int64_t>({n_recv, n_send, E, 1});
+  const unsigned blocks = (unsigned)std::min<int64_t>((work + 255) / 256, (int64_t)num_sms * 8);
+  csr_check_kernel<<<blocks, 256, 0, s>>>(n_recv, n_send, E, rowptr, col, rowptr_T, flag);
+  if (rowptr_T && perm_T)
+    csr_perm_check_kernel<<<blocks, 256, 0, s>>>(n_send, E, col, rowptr_T, perm_T, flag);
+  return cudaGetLastError();
 }
 
 int64_t fma_peak_sink_floats(int num_sms) { return (int64_t)num_sms * 2 * kFmaThreads; }

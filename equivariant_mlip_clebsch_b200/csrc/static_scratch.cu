@@ -82,5 +82,5 @@ extern "C" cgtp_status cgtp_backward_static_scratch(
   // from it is written earlier in the same call
   return cgtp::backward_impl(plan, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, x, Y, W,
                              grad_out, grad_x, grad_W, grad_Y, ws, need > 0 ? kScratchBytes : 0, stream,
-                             /*allow_timing=*/false);
+                             /*allow_timing=*/false, /*eid=*/nullptr, /*graph_checks=*/true);
 }

@@ -134,3 +134,14 @@ def draw_W(E: int, U: int, col_std, seed: int = 0) -> np.ndarray:
 
 def draw_g(n: int, d_out: int, seed: int = 0) -> np.ndarray:
     return normal_f32((n, d_out), seed, 3)
+
+
+def draw_gate(E: int, active_frac: float, seed: int = 0) -> np.ndarray:
+    """Continuation gates for the sparse evaluation: with u ~ U(0,1) per edge
+    (stream 4), an edge is active when u < active_frac and its gate is then
+    (active_frac - u) / active_frac in (0, 1]; skipped edges get exactly 0.
+    FP32."""
+    u = rng(seed, 4).uniform(0.0, 1.0, size=int(E))
+    a = float(active_frac)
+    f = np.where(u < a, (a - u) / max(a, 1e-300), 0.0)
+    return f.astype(np.float32)

@@ -48,7 +48,9 @@
  * device of every tensor before the call), and the graph is a valid CSR
  * (rowptr non-decreasing from 0 to E, every col in [0, n_send), perm_T a
  * permutation grouped by sender) -- cgtp_csr_transpose checks exactly this
- * on the host while it builds rowptr_T and perm_T.
+ * on the host while it builds rowptr_T and perm_T, and a plan's device
+ * graph checks (cgtp_plan_set_checks, or CGTP_DEBUG) check it before each
+ * call.
  * cgtp_last_error() returns a message for the calling thread's last failure.
  * Calls are ordered on the given stream; a plan may be used from several
  * threads for concurrent launches.
@@ -74,7 +76,7 @@ typedef enum {
   CGTP_ERR_IRREPS_MISMATCH = 4, /* output multiplicities disagree with the paths */
   CGTP_ERR_LMAX = 5,            /* some l exceeds lmax, or lmax > 6 */
   CGTP_ERR_SIZE = 6,            /* a size is negative, too large, or inconsistent */
-  CGTP_ERR_INVALID_CSR = 7,     /* rowptr/col/perm inconsistent (host checks) */
+  CGTP_ERR_INVALID_CSR = 7,     /* rowptr/col/perm inconsistent (host or device checks) */
   CGTP_ERR_CUDA = 8,            /* a CUDA runtime or driver call failed */
   CGTP_ERR_OOM = 9,             /* host or device allocation failed in plan create */
   CGTP_ERR_TIMEOUT = 10,        /* a bounded wait inside a kernel gave up */
@@ -218,6 +220,25 @@ cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* need
  * in milliseconds and the launch count since the previous call (which resets
  * them).  names receives up to max entries of 32 bytes each. */
 cgtp_status cgtp_plan_set_timing(cgtp_plan plan, int enable);
+
+/* Device checks of the graph (off by default; on for every plan created
+ * while the environment variable CGTP_DEBUG is set to anything but "0").
+ * With CGTP_CHECK_GRAPH set, every convolution call of the plan (forward,
+ * backward, its static-scratch form, the double backward and the sparse
+ * evaluation) first checks on the device, on the call's stream, that rowptr
+ * runs non-decreasing from 0 to E and every col lies in [0, n_send), and,
+ * when the call reads the sender lists (grad_x wanted), that rowptr_T runs
+ * non-decreasing from 0 to E and perm_T lists, for each sender, ids of its own
+ * edges in strictly ascending order (which makes it a permutation).  The
+ * call then WAITS for the result (a stream synchronize: not usable under
+ * stream capture, which is refused with CGTP_ERR_CUDA) and returns
+ * CGTP_ERR_INVALID_CSR, naming the failed checks, before any kernel reads
+ * through the graph.  The checks read only the arrays' declared extents
+ * (n_recv + 1, E, n_send + 1 entries); the sender lists are walked only
+ * after their bounds passed.  flags: 0 or CGTP_CHECK_GRAPH.
+ * Errors: NULL, SIZE (unknown flags). */
+#define CGTP_CHECK_GRAPH 1
+cgtp_status cgtp_plan_set_checks(cgtp_plan plan, int flags);
 cgtp_status cgtp_plan_kernel_times(cgtp_plan plan, int max, char* names, double* ms,
                                    int64_t* launches, int* n);
 
@@ -260,6 +281,50 @@ cgtp_status cgtp_backward_static_scratch(cgtp_plan plan, int64_t n_recv, int64_t
  * kernels launched since the last call completed; CGTP_ERR_TIMEOUT is
  * returned otherwise. */
 cgtp_status cgtp_plan_check_device_error(cgtp_plan plan, int* code);
+
+/* ---- BranchIP sparse evaluation -------------------------------------- */
+
+/* The BranchIP page (section "BranchIP", the Branchlegro paragraph) gives
+ * every edge a continuation gate f_e in [0, 1] that multiplies the edge's
+ * feature before the TP; at inference the zero-gated edges are omitted from
+ * the TP and the skipped per-edge outputs are zero-padded to the full edge
+ * set ("sparse evaluation"), which reproduces the dense evaluation exactly.
+ * Here the gate scales each edge's whole TP term:
+ *   out[i] = sum_{e in row i} f_e TP(x[col e], Y[e], W[e])
+ * (the convolution is linear in each input, so this is the gate applied to
+ * any one of them), and only the edges with f_e > 0 are evaluated.
+ *   gate [E] FP32 device, 16-byte aligned; f_e > 0 marks an active edge (a
+ *   NaN gate is inactive).  Other arguments and layouts as for cgtp_forward /
+ *   cgtp_backward; the graph is the full (ungated) CSR.
+ * Steps, all on the stream and deterministic (no atomics, no host sync): a
+ * scan compacts the active edges (receiver CSR, their ids, their gated
+ * harmonics f_e Y_e, and with grad_x the sender lists) into the workspace;
+ * the plan's kernels run over them, reading W rows and writing grad_W rows
+ * of the full set through the edge ids; the backward then pads.
+ * Workspace: cgtp_sparse_workspace_size bytes, 256-byte aligned, caller
+ * owned; nothing in it needs initialising, and a call leaves nothing in it
+ * that a later call needs (each call compacts again).
+ * Backward outputs (each nullable = skipped), overwritten over the FULL edge
+ * set: grad_x [n_send, d_in]; grad_W [E, n_weights] = f_e dL/dW' (zero rows
+ * for skipped edges); grad_Y [E, d_edge] (zero rows for skipped edges);
+ * grad_gate [E] = <g[i], TP_e> on active edges and 0 on skipped ones (the
+ * sparse path builds no backward branch for them; exact for a loss that
+ * reaches the gate through a function with zero slope where it is zero, the
+ * page's flat-zero gate).  rowptr_T/perm_T are needed only with grad_x.
+ * Errors: NULL, SIZE, ALIGN, WORKSPACE, CUDA (also for a plan of another
+ * device or a compile-only plan). */
+cgtp_status cgtp_sparse_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                                       size_t* bytes);
+cgtp_status cgtp_sparse_forward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                                const int32_t* rowptr, const int32_t* col, const float* x,
+                                const float* Y, const float* W, const float* gate, float* out,
+                                void* workspace, size_t workspace_bytes, cgtp_stream stream);
+cgtp_status cgtp_sparse_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                                 const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
+                                 const int32_t* perm_T, const float* x, const float* Y,
+                                 const float* W, const float* gate, const float* grad_out,
+                                 float* grad_x, float* grad_W, float* grad_Y, float* grad_gate,
+                                 void* workspace, size_t workspace_bytes, cgtp_stream stream);
 
 /* ---- measurement ----------------------------------------------------- */
 

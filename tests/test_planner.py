@@ -197,7 +197,8 @@ def _check_layout(src, smem, backward):
         bad.append("dY partials past the stage")
     if any(v % 16 for v in off + [d["STAGE_BYTES"], d["OFF_STAGE"], d["OFF_G"], d["OFF_WB"]]):
         bad.append("offset not 16-byte aligned")
-    if 32 * NS + 32 > d["OFF_STAGE"]:  # full/empty barriers, grad_out barriers, stage records
+    # full/empty/chat barriers, grad_out barriers, stage records, edge range
+    if 3 * 8 * NS + 32 + 16 * NS + 16 > d["OFF_STAGE"]:
         bad.append("barriers past the first stage")
     if d["OFF_STAGE"] + NS * d["STAGE_BYTES"] > d["OFF_G"]:
         bad.append("stage ring past the grad_out buffers")
