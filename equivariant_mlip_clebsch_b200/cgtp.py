@@ -44,6 +44,7 @@ _SIGS = {
     "cgtp_edge_virial": (_i, [_i64, _P, _P, _P, _P]),
     "cgtp_double_backward_workspace_size": (_i, [_P, _i64, _i64, _i64, ctypes.POINTER(_sz)]),
     "cgtp_double_backward": (_i, [_P, _i64, _i64, _i64] + [_P] * 16 + [_sz, _P]),
+    "cgtp_plan_prepare_double_backward": (_i, [_P, ctypes.POINTER(_i)]),
     "cgtp_forward": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P, _P, _P]),
     "cgtp_backward_workspace_size": (_i, [_P, _i64, _i64, _i64, ctypes.POINTER(_sz)]),
     "cgtp_backward": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -340,6 +341,13 @@ class Plan:
                                                        dx, dW, dY, dev, n_recv, n_send, E),
                                   *_workspace(workspace, dev), _stream(stream)))
         return dx, dW, dY
+
+    def prepare_double_backward(self) -> bool:
+        """cgtp_plan_prepare_double_backward: build the tangent kernels now;
+        True when the double backward will use them."""
+        t = ctypes.c_int()
+        _check(_lib.cgtp_plan_prepare_double_backward(self._h, ctypes.byref(t)))
+        return bool(t.value)
 
     def double_backward_workspace_size(self, n_recv: int, n_send: int, E: int) -> int:
         b = ctypes.c_size_t()

@@ -39,6 +39,8 @@ void destroy_plan_device(Plan& P) {
   jit_unload(P.fwd);
   jit_unload(P.bwd);
   jit_unload(P.bwd_er);
+  jit_unload(P.fwd_tan);
+  jit_unload(P.bwd_tan);
   for (void** p : {&P.d_fwd_ent, &P.d_bwd_ent}) {
     if (*p) cudaFree(*p);
     *p = nullptr;
@@ -61,7 +63,8 @@ static cgtp_status check_device(const Plan& P) {
   return CGTP_OK;
 }
 
-static const char* kKindName[] = {"sph_harm", "cgtp_fwd", "cgtp_bwd", "bwd_reduce", "sph_harm_bwd", "zero_fill"};
+static const char* kKindName[] = {"sph_harm",     "cgtp_fwd",  "cgtp_bwd",    "bwd_reduce",
+                                  "sph_harm_bwd", "zero_fill", "cgtp_fwd_tan", "cgtp_bwd_tan"};
 
 // Brackets one internal launch with events when timing is on.
 struct TimedScope {
@@ -158,6 +161,7 @@ const char* cgtp_last_error(void) { return t_err.c_str(); }
 
 cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge, const char* irreps_out,
                              int lmax, cgtp_plan* out) {
+  NvtxRange nvtx_range("cgtp_plan_create");
   if (!out) return fail(CGTP_ERR_NULL, "out is NULL");
   *out = nullptr;
   if (!irreps_in || !irreps_edge || !irreps_out) return fail(CGTP_ERR_NULL, "irreps string is NULL");
@@ -254,6 +258,7 @@ cgtp_status cgtp_real_cg(int l1, int l2, int l3, double* C) {
 }
 
 cgtp_status cgtp_sph_harm(cgtp_plan plan, int64_t E, const float* r, float* Y, cgtp_stream stream) {
+  NvtxRange nvtx_range("cgtp_sph_harm");
   if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
   const Plan* P = reinterpret_cast<const Plan*>(plan);
   if (E < 0 || E >= (int64_t(1) << 31)) return fail(CGTP_ERR_SIZE, "E out of range");
@@ -271,6 +276,7 @@ cgtp_status cgtp_sph_harm(cgtp_plan plan, int64_t E, const float* r, float* Y, c
 
 cgtp_status cgtp_sph_harm_backward(cgtp_plan plan, int64_t E, const float* r, const float* grad_Y,
                                    float* grad_r, cgtp_stream stream) {
+  NvtxRange nvtx_range("cgtp_sph_harm_backward");
   if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
   const Plan* P = reinterpret_cast<const Plan*>(plan);
   if (E < 0 || E >= (int64_t(1) << 31)) return fail(CGTP_ERR_SIZE, "E out of range");
@@ -289,6 +295,7 @@ cgtp_status cgtp_sph_harm_backward(cgtp_plan plan, int64_t E, const float* r, co
 
 cgtp_status cgtp_edge_forces(int64_t n_atoms, int64_t E, const int32_t* rowptr, const int32_t* rowptr_T,
                              const int32_t* perm_T, const float* grad_r, float* forces, cgtp_stream stream) {
+  NvtxRange nvtx_range("cgtp_edge_forces");
   if (n_atoms < 0 || E < 0 || n_atoms >= (int64_t(1) << 31) || E >= (int64_t(1) << 31))
     return fail(CGTP_ERR_SIZE, "sizes out of range");
   if (n_atoms == 0) return CGTP_OK;
@@ -299,6 +306,7 @@ cgtp_status cgtp_edge_forces(int64_t n_atoms, int64_t E, const int32_t* rowptr, 
 }
 
 cgtp_status cgtp_edge_virial(int64_t E, const float* r, const float* grad_r, float* virial, cgtp_stream stream) {
+  NvtxRange nvtx_range("cgtp_edge_virial");
   if (E < 0 || E >= (int64_t(1) << 31)) return fail(CGTP_ERR_SIZE, "E out of range");
   if (!virial) return fail(CGTP_ERR_NULL, "virial is NULL");
   if (E > 0 && (!r || !grad_r)) return fail(CGTP_ERR_NULL, "r or grad_r is NULL");
@@ -311,6 +319,7 @@ cgtp_status cgtp_edge_virial(int64_t E, const float* r, const float* grad_r, flo
 cgtp_status cgtp_forward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
                          const int32_t* rowptr, const int32_t* col, const float* x, const float* Y,
                          const float* W, float* out, cgtp_stream stream) {
+  NvtxRange nvtx_range("cgtp_forward");
   return cgtp::forward_impl(plan, n_recv, n_send, E, rowptr, col, x, Y, W, nullptr, out, stream, true);
 }
 
@@ -328,6 +337,7 @@ cgtp_status cgtp_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
                           const int32_t* perm_T, const float* x, const float* Y, const float* W,
                           const float* grad_out, float* grad_x, float* grad_W, float* grad_Y,
                           void* workspace, size_t workspace_bytes, cgtp_stream stream) {
+  NvtxRange nvtx_range("cgtp_backward");
   return cgtp::backward_impl(plan, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, x, Y, W,
                              grad_out, grad_x, grad_W, grad_Y, workspace, workspace_bytes, stream,
                              true, nullptr, true);
@@ -336,6 +346,45 @@ cgtp_status cgtp_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
 }  // extern "C"
 
 namespace cgtp {
+
+// The double backward's tangent kernels, built once per plan under its lock
+// (CGTP_DBWD_COMPOSE=1 at build time keeps the composition of plain calls).
+// Returns whether they are available; a build failure is remembered, not
+// returned: the composition remains.
+static bool ensure_tangent(Plan& P) {
+  std::lock_guard<std::mutex> g(P.tan_mu);
+  if (P.tan_state != 0) return P.tan_state > 0;
+  if (const char* v = std::getenv("CGTP_DBWD_COMPOSE"); v && *v && *v != '0') {
+    P.tan_state = -1;
+    P.tan_msg = "tangent kernels switched off (CGTP_DBWD_COMPOSE)";
+    return false;
+  }
+  if (P.fwd_roles.empty() || P.bwd_roles.empty()) {
+    P.tan_state = -1;
+    P.tan_msg = "no paths";
+    return false;
+  }
+  std::string fsrc, bsrc;
+  cgtp_status st = build_forward_tangent(P, P.fwd_tan, &fsrc);
+  if (st == CGTP_OK) st = build_backward_tangent(P, P.bwd_tan, &bsrc);
+  if (st != CGTP_OK) {
+    P.tan_msg = cgtp_last_error();
+    jit_unload(P.fwd_tan);
+    jit_unload(P.bwd_tan);
+    P.tan_state = -1;
+    return false;
+  }
+  if (const char* d = std::getenv("CGTP_DUMP_SOURCE")) {
+    for (auto [name, src] : {std::pair<const char*, std::string*>{"/fwd_tan.cu", &fsrc}, {"/bwd_tan.cu", &bsrc}}) {
+      if (FILE* f = std::fopen((std::string(d) + name).c_str(), "w")) {
+        std::fputs(src->c_str(), f);
+        std::fclose(f);
+      }
+    }
+  }
+  P.tan_state = 1;
+  return true;
+}
 
 cgtp_status forward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
                          const int32_t* col, const float* x, const float* Y, const float* W, const int32_t* eid,
@@ -535,6 +584,13 @@ cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* need
          std::to_string(q.u0) + " R=" + std::to_string(q.R) + " ph=" + std::to_string(q.ph) + "/" +
          std::to_string(q.nph) + " cost=" + std::to_string((int)q.cost) + "\n";
   }
+  for (const JitKernel* k : {&P->fwd_tan, &P->bwd_tan}) {  // tangent kernels, once built
+    if (k->name.empty()) continue;
+    char hx[64];
+    std::snprintf(hx, sizeof hx, " smem=%d threads=%d hash=%016llx\n", k->smem, k->threads, k->hash);
+    t += k->name + " (tangent, double backward):" + std::string(hx) + k->log;
+    if (!k->log.empty() && k->log.back() != '\n') t += "\n";
+  }
   {  // the edge-range variant of the backward (same roles and layout)
     char hx[40];
     std::snprintf(hx, sizeof hx, " hash=%016llx\n", P->bwd_er.hash);
@@ -547,6 +603,19 @@ cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* need
     std::memcpy(buf, t.data(), k);
     buf[k] = '\0';
   }
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_prepare_double_backward(cgtp_plan plan, int* tangent) {
+  NvtxRange nvtx_range("cgtp_plan_prepare_double_backward");
+  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
+  Plan* P = reinterpret_cast<Plan*>(plan);
+  if (!P->host_only) {  // a compile-only plan builds (and checks) the kernels' code only
+    cgtp_status st = check_device(*P);
+    if (st != CGTP_OK) return st;
+  }
+  const bool ok = ensure_tangent(*P);
+  if (tangent) *tangent = ok ? 1 : 0;
   return CGTP_OK;
 }
 
@@ -636,6 +705,7 @@ cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send,
                                  const float* grad_out, const float* h_x, const float* h_W, const float* h_Y,
                                  float* gg_out, float* gx, float* gW, float* gY, void* workspace,
                                  size_t workspace_bytes, cgtp_stream stream) {
+  NvtxRange nvtx_range("cgtp_double_backward");
   if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
   Plan* P = reinterpret_cast<Plan*>(plan);
   if (n_recv < 0 || n_send < 0 || E < 0 || n_recv >= (int64_t(1) << 31) ||
@@ -667,6 +737,39 @@ cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send,
   float* tX = reinterpret_cast<float*>(ws + L.x);
   float* tW = reinterpret_cast<float*>(ws + L.w);
   float* tY = reinterpret_cast<float*>(ws + L.y);
+  cudaStream_t cs = (cudaStream_t)stream;
+  if (h_x && h_W && h_Y && E > 0 && n_recv > 0 && ensure_tangent(*P)) {
+    // one tangent forward and one tangent backward: the derivatives along
+    // (h_x, h_Y, h_W) of the forward and of the backward at fixed grad_out
+    int nr = (int)n_recv;
+    const int32_t* no_eid = nullptr;
+    if (gg_out) {
+      void* args[] = {&rowptr, &col, &x, &Y, &W, &no_eid, &gg_out, &P->d_fwd_ent, &nr, &P->d_err, &h_x, &h_Y, &h_W};
+      TimedScope ts(*P, 6, cs);
+      st = jit_launch(P->fwd_tan, dim3(persistent_grid(P->fwd_tan.blocks_per_sm, P->num_sms, n_recv)), args, cs);
+      if (st != CGTP_OK) return st;
+    }
+    if (gx || gW || gY) {
+      size_t off_dyp = 0;
+      backward_scratch_bytes(*P, E, gx != nullptr, gY != nullptr, &off_dyp);
+      float* m = gx ? reinterpret_cast<float*>(ws + L.bwd) : nullptr;
+      float* dyp = gY ? (P->bcfg.S > 1 ? reinterpret_cast<float*>(ws + L.bwd + off_dyp) : gY) : nullptr;
+      if (m && P->bwd_irrep_gap) CGTP_CUDA_TRY(cudaMemsetAsync(m, 0, (size_t)E * P->D_in * sizeof(float), cs));
+      void* args[] = {&rowptr, &col, &x, &Y, &W, &no_eid, &grad_out, &gW, &dyp, &m, &P->d_bwd_ent, &nr, &P->d_err,
+                      &h_x, &h_Y, &h_W};
+      {
+        TimedScope ts(*P, 7, cs);
+        st = jit_launch(P->bwd_tan, dim3(persistent_grid(P->bwd_tan.blocks_per_sm, P->num_sms, n_recv)), args, cs);
+        if (st != CGTP_OK) return st;
+      }
+      if (gx || (gY && P->bcfg.S > 1)) {
+        TimedScope ts(*P, 3, cs);
+        CGTP_CUDA_TRY(launch_bwd_reduce(n_send, P->D_in, rowptr_T, perm_T, m, gx, P->bcfg.S, E * P->D_e, dyp,
+                                        (gY && P->bcfg.S > 1) ? gY : nullptr, cs));
+      }
+    }
+    return CGTP_OK;
+  }
   // the term structure (double_backward.hpp) on the library's kernels
   struct DeviceOps {
     cgtp_plan plan;

@@ -129,6 +129,11 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       << "      const float* wr = sW + b * WS;\n"
       << "      const float* xr = sX + b * XS;\n"
       << "      const float* chb = sC + b * chs;\n"
+      << (K.tangent ? "      const float* chtb = reinterpret_cast<const float*>(st + OFF_CHT) + b * chs;\n"
+                      "      const float* wtr = reinterpret_cast<const float*>(st + OFF_WT) + b * WS;\n"
+                      "      const float* xtr = reinterpret_cast<const float*>(st + OFF_XT) + " +
+                          std::to_string(sl.x_st.at(r.irrep)) + " + b * XS;\n"
+                    : "")
       << "      float* dWrow = dW ? dW + (size_t)(eid ? __ldg(eid + e) : e) * NU : nullptr;\n"
       << "      float* sdy = want_dy ? sdyw + b * DE : nullptr;\n"
       ;
@@ -149,13 +154,17 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
     o << "#pragma unroll 1\n      for (int r = 0; r < " << R << "; r += " << RU << ") {\n"
       << "      bool ok[" << RU << "];\n"
       << "      float xv[" << RU << "][" << N1 << "], mx[" << RU << "][" << N1 << "];\n"
+      << (K.tangent ? "      float xtv[" + std::to_string(RU) + "][" + std::to_string(N1) + "];\n" : "")
       << "#pragma unroll\n      for (int v = 0; v < " << RU << "; ++v) {\n"
       << "        const int u = u0 + (r + v) * 32 + lane;\n"
       << "        ok[v] = " << (MUL % (32 * R) == 0 ? std::string("true") : "u < " + std::to_string(MUL))
       << ";  // every lane holds a channel when the blocks are full\n"
       << "#pragma unroll\n        for (int m1 = 0; m1 < " << N1
-      << "; ++m1) { mx[v][m1] = 0.f; xv[v][m1] = ok[v] ? xr[u * " << N1 << " + m1] : 0.f; }\n"
-      << "      }\n";
+      << "; ++m1) { mx[v][m1] = 0.f; xv[v][m1] = ok[v] ? xr[u * " << N1 << " + m1] : 0.f; }\n";
+    if (K.tangent)
+      o << "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) xtv[v][m1] = ok[v] ? xtr[u * " << N1
+        << " + m1] : 0.f;\n";
+    o << "      }\n";
     std::vector<char> l2seen(P.L + 1, 0);
     size_t q = 0;
     while (q < ps.size()) {
@@ -172,18 +181,26 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
         const Path& p = P.paths[pi];
         const int N3 = 2 * p.l3 + 1, n2 = 2 * p.l2 + 1;
         o << "        {\n          float w[" << RU << "], gv[" << RU << "][" << N3 << "], dw[" << RU << "];\n"
+          << (K.tangent ? "          float wt[" + std::to_string(RU) + "];\n" : "")
           << "#pragma unroll\n          for (int v = 0; v < " << RU << "; ++v) {\n"
           << "            const int u = u0 + (r + v) * 32 + lane;\n"
           << "            w[v] = ok[v] ? wr[" << sl.w_st.at(pi) << " + u] : 0.f;\n"
+          << (K.tangent ? "            wt[v] = ok[v] ? wtr[" + std::to_string(sl.w_st.at(pi)) + " + u] : 0.f;\n" : "")
           << "#pragma unroll\n            for (int m3 = 0; m3 < " << N3 << "; ++m3) gv[v][m3] = ok[v] ? sg["
-          << sl.g_st.at(pi) << " + u * " << N3 << " + m3] : 0.f;\n          }\n"
-          << "          bpath<" << N1 << "," << N3 << "," << RU << ">(chb + " << sl.ch_off.at(pi)
-          << ", xv, w, gv, mx, dw);\n"
+          << sl.g_st.at(pi) << " + u * " << N3 << " + m3] : 0.f;\n          }\n";
+        if (K.tangent)
+          o << "          bpath_tan<" << N1 << "," << N3 << "," << RU << ">(chb + " << sl.ch_off.at(pi) << ", chtb + "
+            << sl.ch_off.at(pi) << ", xv, xtv, w, wt, gv, mx, dw);\n";
+        else
+          o << "          bpath<" << N1 << "," << N3 << "," << RU << ">(chb + " << sl.ch_off.at(pi)
+            << ", xv, w, gv, mx, dw);\n";
+        o
           << "          if (dWrow) {\n#pragma unroll\n            for (int v = 0; v < " << RU
           << "; ++v) if (ok[v]) dWrow[" << p.k0 << " + u0 + (r + v) * 32 + lane] = dw[v];\n          }\n"
           << "          if (sdy) {\n#pragma unroll\n            for (int v = 0; v < " << RU << "; ++v) {\n"
           << "              float wx[" << N1 << "];\n#pragma unroll\n              for (int m1 = 0; m1 < " << N1
-          << "; ++m1) wx[m1] = w[v] * xv[v][m1];\n";
+          << (K.tangent ? "; ++m1) wx[m1] = fmaf(w[v], xtv[v][m1], wt[v] * xv[v][m1]);  // d (w x)\n"
+                        : "; ++m1) wx[m1] = w[v] * xv[v][m1];\n");
         const double* C = P.coeff.data() + p.c_off;
         for (int m1 = 0; m1 < N1; ++m1)
           for (int m3 = 0; m3 < N3; ++m3) {
@@ -280,7 +297,10 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
     << "(const int* __restrict__ rowptr, const int* __restrict__ col, const float* __restrict__ x,\n"
        "    const float* __restrict__ Y, const float* __restrict__ W, const int* __restrict__ eid,\n"
        "    const float* __restrict__ g, float* __restrict__ dW, float* __restrict__ dyp, float* __restrict__ msg,\n"
-       "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err) {\n"
+       "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err"
+    << (K.tangent ? ",\n    const float* __restrict__ xt, const float* __restrict__ Yt, const float* __restrict__ Wt"
+                  : "")
+    << ") {\n"
        "  extern __shared__ __align__(128) unsigned char smem[];\n"
        "  grid_dependency_wait();  // the previous kernel's results are visible\n"
        "  grid_launch_dependents();\n"
@@ -305,8 +325,9 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
              "  }\n"
            : "") <<
        "  __syncthreads();\n"
-       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, eid, g, err, smem, lane); return; }\n"
-       "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, ent, kEntBegin, dyp, err, smem, lane); return; }\n"
+    << (K.tangent ? "" : "  const float* xt = nullptr; const float* Yt = nullptr; const float* Wt = nullptr;\n")
+    << "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, xt, Wt, eid, g, err, smem, lane); return; }\n"
+       "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, Yt, ent, kEntBegin, dyp, err, smem, lane); return; }\n"
        "  int q = 0, kr = 0;\n"
        "  for (int slice = 0; slice < NSLICE; ++slice) {\n"
        "    const int slot = slice * NW + warp;\n"
@@ -488,12 +509,16 @@ cgtp_status build_backward(Plan& P) {
   // fits (it sets how many edges each stage hands over per barrier round
   // trip, and how many are in flight), then two resident CTAs per SM when
   // that chunk allows it, then the shortest consumer critical path per SM.
-  const int kB[] = {8, 4, 2, 1};
+  int kB[] = {8, 4, 2, 1};
+  if (const char* v = std::getenv("CGTP_BWD_CHUNK"))  // tuning override: one chunk size
+    kB[0] = kB[1] = kB[2] = kB[3] = std::max(1, std::min(8, std::atoi(v)));
   // barrier round trips, loop and address work of one chunk, in the units of
   // bwd_edge_cost
   const double kChunkOverhead = 80.0;
   // consumer warps per CTA: 6, 12 and 16 measured slower than 4 or 8 on B200
-  const int kNW[] = {4, 8};
+  int kNW[] = {4, 8};
+  if (const char* v = std::getenv("CGTP_BWD_NW"))  // tuning override: one warp count
+    kNW[0] = kNW[1] = std::max(1, std::min(16, std::atoi(v)));
   for (int B : kB) {
     if (best.B != 0) break;
     // options of every irrep for this chunk size
@@ -628,6 +653,10 @@ cgtp_status build_backward(Plan& P) {
   bool fixed = false;
   int mb0 = initial_min_blocks(K.smem, &fixed);
   if (!fixed) mb0 = std::min(mb0, best.ctas);  // the planner's register share
+  if (const char* v = std::getenv("CGTP_BWD_MIN_BLOCKS")) {
+    mb0 = std::max(1, std::atoi(v));
+    fixed = true;
+  }
   const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
   // Two variants of the same kernel: CTAs over whole receivers, and CTAs
   // over equal edge ranges.  The second balances graphs with few receivers
@@ -687,6 +716,62 @@ cgtp_status build_backward(Plan& P) {
     }
   }
   return CGTP_OK;
+}
+
+// The backward's tangent kernel (cgtp_bwd_tan): the same roles and slices
+// as cgtp_bwd, every W, x and Y piece staged with its directional
+// derivative, so that one pass gives d/dt of (dW, dY, the dx messages) at
+// (x + t xt, Y + t Yt, W + t Wt) for a fixed grad_out.  The chunk is halved
+// while the doubled stages do not fit.  Built on first use.
+cgtp_status build_backward_tangent(Plan& P, JitKernel& out, std::string* src_out) {
+  const FwdConfig& F = P.bcfg;
+  std::vector<SliceLayout> SL(F.S);
+  KernelShape K;
+  K.S = F.S;
+  K.nw = F.nw;
+  K.tangent = true;
+  for (int s2 = 0; s2 < F.S; ++s2) {
+    for (int ri : F.slice_roles[s2]) {
+      const BwdRole& r = P.bwd_roles[ri];
+      auto& irr = SL[s2].irreps;
+      if (std::find(irr.begin(), irr.end(), r.irrep) == irr.end()) {
+        irr.push_back(r.irrep);
+        for (size_t q = 0; q < P.paths.size(); ++q)
+          if (P.paths[q].irrep == r.irrep) SL[s2].paths.push_back((int)q);
+      }
+      K.WB = std::max(K.WB, 32 * bwd_unroll(2 * P.in[r.irrep].l + 1, r.R) * (2 * P.in[r.irrep].l + 1));
+    }
+    std::sort(SL[s2].paths.begin(), SL[s2].paths.end());
+    layout_slice(P, SL[s2], true);
+  }
+  for (K.force_B = F.B; K.force_B >= 1; K.force_B /= 2) {
+    plan_layout(P, SL, K, true);
+    if (K.smem <= 227 * 1024) break;
+  }
+  if (K.force_B < 1 || K.smem > 227 * 1024)
+    return fail(CGTP_ERR_SIZE, "tangent backward needs too much shared memory");
+  for (size_t k = 0; k + 1 < P.bwd_ent_begin.size(); ++k)
+    K.rec_max = std::max(K.rec_max, P.bwd_ent_begin[k + 1] - P.bwd_ent_begin[k]);
+  bool fixed = false;
+  const int mb0 = initial_min_blocks(K.smem, &fixed);
+  const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
+  const std::string name = "cgtp_bwd_tan";
+  std::string src;
+  JitBinary bin;
+  cgtp_status st = CGTP_OK;
+  for (int mb = mb0; mb >= mb_floor; --mb) {
+    src = gen_bwd_source(P, SL, K, name, mb);
+    st = jit_build(src, name, bin);
+    if (st != CGTP_OK || mb == mb_floor || max_spill_bytes(bin.log) <= 160) break;
+  }
+  if (st != CGTP_OK) {
+    set_error(bin.err);
+    return st;
+  }
+  out.threads = (F.nw + 2) * 32;
+  out.smem = K.smem;
+  if (src_out) *src_out = src;
+  return jit_load(bin, name, out);
 }
 
 }  // namespace cgtp

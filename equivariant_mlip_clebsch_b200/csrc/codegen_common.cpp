@@ -130,15 +130,17 @@ void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape&
     K.g_bulk = K.g_bulk && segments_aligned(sl.gseg, P.D_out);
   }
   auto r128 = [](long v) { return (int)((v + 127) & ~127L); };
+  const long mt = K.tangent ? 2 : 1;  // tangent kernels stage each piece twice
   auto stage_of = [&](int B) {
-    long b = r128(4L * B * K.WS) + r128(4L * B * K.XS) + r128(4L * B * P.D_e) + r128(4L * B * K.CHS);
+    long b = r128(4L * mt * B * K.WS) + r128(4L * mt * B * K.XS) + r128(4L * mt * B * P.D_e) +
+             r128(4L * mt * B * K.CHS);
     if (backward) b += r128(4L * K.nw * B * P.D_e);
     return b;
   };
   // two grad_out buffers overlap the next receiver's load with this one's
   // compute; wide rows (Lmax 6) keep one so more CTAs fit
   K.gbufs = (backward && 2L * r128(4L * K.GS) > 48 * 1024) ? 1 : 2;
-  const long fixed = 256 + (backward ? (long)K.gbufs * r128(4L * K.GS) : 0)  // grad_out buffers
+  const long fixed = 512 + (backward ? (long)K.gbufs * r128(4L * K.GS) : 0)  // grad_out buffers
                      + r128(4L * K.nw * K.WB);                                 // store staging
   // two or three CTAs per SM when it fits, at least two stages in flight
   // wide rows (Lmax 6) may take up to half an SM to keep two edges per chunk
@@ -158,10 +160,10 @@ void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape&
   K.sdy_floats = backward ? K.nw * K.B * (int)P.D_e : 0;
   K.off_stage = 512;  // mbarriers, chunk descriptors and the edge range first
   K.off_w = 0;
-  K.off_x = r128(4L * K.B * K.WS);
-  K.off_y = K.off_x + r128(4L * K.B * K.XS);
-  K.off_ch = K.off_y + r128(4L * K.B * P.D_e);
-  K.off_dy = K.off_ch + r128(4L * K.B * K.CHS);
+  K.off_x = r128(4L * mt * K.B * K.WS);
+  K.off_y = K.off_x + r128(4L * mt * K.B * K.XS);
+  K.off_ch = K.off_y + r128(4L * mt * K.B * P.D_e);
+  K.off_dy = K.off_ch + r128(4L * mt * K.B * K.CHS);
   K.stage_bytes = K.off_dy + (backward ? r128(4L * K.sdy_floats) : 0);
   K.off_g = K.off_stage + K.stages * K.stage_bytes;
   K.off_wb = K.off_g + (backward ? K.gbufs * r128(4L * K.GS) : 0);
@@ -206,14 +208,25 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
     << K.off_x << "\n#define OFF_Y " << K.off_y << "\n#define OFF_CH " << K.off_ch << "\n#define OFF_DY "
     << K.off_dy << "\n#define OFF_G " << K.off_g << "\n#define GS " << K.GS << "\n#define WB " << K.WB
     << "\n#define OFF_WB " << K.off_wb << "\n#define FULL_COUNT 32\n#define CHAT_COUNT 32\n#define GBUF " << K.gbufs << "\n#define YPL "
-    << (K.B * P.D_e + 31) / 32 << "\n";
+    << (K.B * P.D_e + 31) / 32 << "\n#define TAN " << (K.tangent ? 1 : 0) << "\n";
+  // tangent copies of a stage's regions, right after the plain ones
+  o << "#define OFF_WT (OFF_W + 4 * NB * WS)\n#define OFF_XT (OFF_X + 4 * NB * XS)\n"
+       "#define OFF_YT (OFF_Y + 4 * NB * DE)\n#define OFF_CHT (OFF_CH + 4 * NB * CHS)\n";
   // shared-memory header: full[NSTAGE] (the TMA warp's 32 lanes and the
   // bytes of its copies), empty[NSTAGE] (one arrival per consumer warp),
   // chat[NSTAGE] (the helper's 32 lanes: Y and Chat of the stage written),
   // gfull[2], gempty[2] mbarriers, the helper's per-stage chunk descriptors,
   // and the edge range of the edge-range variant, all below OFF_STAGE
-  o << "#define OFF_CHAT (2 * NSTAGE * 8)\n#define OFF_GFULL (3 * NSTAGE * 8)\n#define OFF_GEMPTY (OFF_GFULL + 16)\n"
-       "#define OFF_DESC (OFF_GEMPTY + 16)\n#define OFF_RANGE (OFF_DESC + 16 * NSTAGE)\n";
+  // (mbarriers 8-byte aligned; the int4 descriptors and range 16-byte aligned)
+  {
+    const int off_chat = 2 * K.stages * 8;
+    const int off_gfull = (3 * K.stages * 8 + 15) & ~15;
+    const int off_gempty = off_gfull + 16;
+    const int off_desc = off_gempty + 16;
+    const int off_range = off_desc + 16 * K.stages;
+    o << "#define OFF_CHAT " << off_chat << "\n#define OFF_GFULL " << off_gfull << "\n#define OFF_GEMPTY "
+      << off_gempty << "\n#define OFF_DESC " << off_desc << "\n#define OFF_RANGE " << off_range << "\n";
+  }
   // a stage is ready for the consumers when its copies have landed and its
   // Chat is built
   o << "__device__ __forceinline__ bool stage_ready(u32 full0, int s, u32 parity) {\n"
@@ -254,10 +267,13 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
   // chunks; the running chunk counter q picks the stage and the phase.
   // eid (nullable): the edges' ids in the full edge set, whose W rows the
   // chunk reads (the sparse evaluation's active edges); NULL: W row = edge
+  // xt, Wt: the tangent inputs of tangent kernels (unused otherwise)
   o << "__device__ __noinline__ void tma_warp(const int* __restrict__ rowptr, int n_recv,\n"
        "    const int* __restrict__ col, const float* __restrict__ x, const float* __restrict__ W,\n"
+       "    const float* __restrict__ xt, const float* __restrict__ Wt,\n"
        "    const int* __restrict__ eid, const float* __restrict__ g, int* __restrict__ err,\n"
        "    unsigned char* smem, int lane) {\n"
+       "  (void)xt; (void)Wt;\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  const u32 gfull0 = full0 + OFF_GFULL, gempty0 = full0 + OFF_GEMPTY;\n"
        "  (void)gfull0; (void)gempty0; (void)g;\n"
@@ -308,25 +324,49 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
          "        unsigned char* st = stage_ptr(smem, s);\n"
          "        float* sW = reinterpret_cast<float*>(st + OFF_W);\n"
          "        float* sX = reinterpret_cast<float*>(st + OFF_X);\n"
-         "        (void)sW; (void)sX;\n"
+         "        float* sWt = reinterpret_cast<float*>(st + OFF_WT);\n"
+         "        float* sXt = reinterpret_cast<float*>(st + OFF_XT);\n"
+         "        (void)sW; (void)sX; (void)sWt; (void)sXt;\n"
          "        (void)jj;\n"
          "        if (lane == 0) mbar_expect_tx(full0 + 8 * s, (u32)nb * "
-      << ((K.w_bulk ? wb : 0) + (K.x_bulk ? xb : 0)) << ");\n"
+      << (K.tangent ? 2 : 1) * ((K.w_bulk ? wb : 0) + (K.x_bulk ? xb : 0)) << ");\n"
       << "        __syncwarp();\n";
     std::ostringstream cp;
     // W rows: consecutive for a chunk of one receiver's edges, or (eid) the
     // rows of the listed edges, one copy per edge
     cp << "if (eid == nullptr) {\n#define WROW(b) (W + (size_t)(eb + (b)) * NU)\n";
     gen_copy_pieces(cp, sl.wseg, K.w_bulk, "sW", K.WS, "WROW", "full0 + 8 * s", w_one, P.U);
-    cp << "#undef WROW\n} else {\n#define WROW(b) (W + (size_t)__ldg(eid + eb + (b)) * NU)\n";
+    cp << "#undef WROW\n";
+    if (K.tangent) {
+      cp << "#define WTROW(b) (Wt + (size_t)(eb + (b)) * NU)\n";
+      gen_copy_pieces(cp, sl.wseg, K.w_bulk, "sWt", K.WS, "WTROW", "full0 + 8 * s", w_one, P.U);
+      cp << "#undef WTROW\n";
+    }
+    cp << "} else {\n#define WROW(b) (W + (size_t)__ldg(eid + eb + (b)) * NU)\n";
     gen_copy_pieces(cp, sl.wseg, K.w_bulk, "sW", K.WS, "WROW", "full0 + 8 * s", false, P.U);
-    cp << "#undef WROW\n}\n";
+    cp << "#undef WROW\n";
+    if (K.tangent) {
+      cp << "#define WTROW(b) (Wt + (size_t)__ldg(eid + eb + (b)) * NU)\n";
+      gen_copy_pieces(cp, sl.wseg, K.w_bulk, "sWt", K.WS, "WTROW", "full0 + 8 * s", false, P.U);
+      cp << "#undef WTROW\n";
+    }
+    cp << "}\n";
     if (K.x_bulk) {
       cp << "#define XROW(b) (x + (size_t)jj * DIN)\n";
       gen_copy_pieces(cp, sl.xseg, true, "sX", K.XS, "XROW", "full0 + 8 * s", false, P.D_in);
+      if (K.tangent) {
+        cp << "#define XTROW(b) (xt + (size_t)jj * DIN)\n";
+        gen_copy_pieces(cp, sl.xseg, true, "sXt", K.XS, "XTROW", "full0 + 8 * s", false, P.D_in);
+        cp << "#undef XTROW\n";
+      }
     } else {
       cp << "#define XROW(b) (x + (size_t)col[eb + (b)] * DIN)\n";
       gen_copy_pieces(cp, sl.xseg, false, "sX", K.XS, "XROW", "full0 + 8 * s", false, P.D_in);
+      if (K.tangent) {
+        cp << "#define XTROW(b) (xt + (size_t)col[eb + (b)] * DIN)\n";
+        gen_copy_pieces(cp, sl.xseg, false, "sXt", K.XS, "XTROW", "full0 + 8 * s", false, P.D_in);
+        cp << "#undef XTROW\n";
+      }
     }
     cp << "#undef XROW\n";
     std::string c = cp.str(), ind;
@@ -377,9 +417,12 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
          "  }\n"
          "}\n";
   }
+  // Yt: the tangent harmonics of tangent kernels (unused otherwise)
   o << "__device__ __noinline__ void helper_warp(const int* __restrict__ rowptr, int n_recv,\n"
-       "    const float* __restrict__ Y, const int4* __restrict__ rec, const int* __restrict__ rec_begin,\n"
-       "    float* __restrict__ dyp, int* __restrict__ err, unsigned char* smem, int lane) {\n"
+       "    const float* __restrict__ Y, const float* __restrict__ Yt, const int4* __restrict__ rec,\n"
+       "    const int* __restrict__ rec_begin, float* __restrict__ dyp, int* __restrict__ err,\n"
+       "    unsigned char* smem, int lane) {\n"
+       "  (void)Yt;\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  int4* desc = reinterpret_cast<int4*>(smem + OFF_DESC);  // (eb, nb, slice, -) of each stage\n"
        "  (void)dyp; (void)desc;\n"
@@ -410,9 +453,14 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
        "      const int s = q % NSTAGE;\n"
        "      const int nb = min(NB, e1 - eb);\n"
        "      // this chunk's Y values travel while the stage is still in use\n"
-       "      float yv[YPL];\n"
+       "      float yv[YPL], ytv[TAN ? YPL : 1];\n"
+       "      (void)ytv;\n"
        "#pragma unroll\n"
        "      for (int k = 0; k < YPL; ++k) { const int t = lane + 32 * k; yv[k] = t < nb * DE ? __ldg(Y + (size_t)eb * DE + t) : 0.f; }\n"
+       "#if TAN\n"
+       "#pragma unroll\n"
+       "      for (int k = 0; k < YPL; ++k) { const int t = lane + 32 * k; ytv[k] = t < nb * DE ? __ldg(Yt + (size_t)eb * DE + t) : 0.f; }\n"
+       "#endif\n"
        "      if (q >= NSTAGE) {\n"
        "        if (!mbar_wait(empty0 + 8 * s, ((q / NSTAGE) - 1) & 1)) { if (lane == 0) atomicOr(err, 10); dead = true; break; }\n";
   if (backward)
@@ -425,10 +473,17 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
        "#pragma unroll\n"
        "      for (int t = 0; t < NSTAGE; ++t)\n"
        "        if (t == s && last_slice[t] != slice) { last_slice[t] = slice; fresh = true; }\n"
+       "      float* sYt = reinterpret_cast<float*>(st + OFF_YT);\n"
+       "      float* cht = reinterpret_cast<float*>(st + OFF_CHT);\n"
+       "      (void)sYt; (void)cht;\n"
        "      if (fresh)  // Chat elements without a CG term are zero for this slice\n"
-       "        for (int t = lane; t < NB * CHS; t += 32) ch[t] = 0.f;\n"
+       "        for (int t = lane; t < (TAN ? 2 : 1) * NB * CHS; t += 32) ch[t] = 0.f;\n"
        "#pragma unroll\n"
        "      for (int k = 0; k < YPL; ++k) { const int t = lane + 32 * k; if (t < nb * DE) sY[t] = yv[k]; }\n"
+       "#if TAN\n"
+       "#pragma unroll\n"
+       "      for (int k = 0; k < YPL; ++k) { const int t = lane + 32 * k; if (t < nb * DE) sYt[t] = ytv[k]; }\n"
+       "#endif\n"
        "      if (lane == 0) desc[s] = make_int4(eb, nb, slice, 0);\n"
        "      __syncwarp();\n"
        "";
@@ -439,7 +494,12 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
          "          const int d = rd[k] & 0xffff, ia = (rd[k] >> 16) & 0xff, ib = (unsigned)rd[k] >> 24;\n"
          "#pragma unroll\n"
          "          for (int b = 0; b < NB; ++b)\n"
-         "            if (b < nb) ch[b * chs + d] = fmaf(rc0[k], sY[b * DE + ia], rc1[k] * sY[b * DE + ib]);\n"
+         "            if (b < nb) {\n"
+         "              ch[b * chs + d] = fmaf(rc0[k], sY[b * DE + ia], rc1[k] * sY[b * DE + ib]);\n"
+         "#if TAN\n"
+         "              cht[b * chs + d] = fmaf(rc0[k], sYt[b * DE + ia], rc1[k] * sYt[b * DE + ib]);\n"
+         "#endif\n"
+         "            }\n"
          "        }\n"
          "      }\n";
   else
@@ -450,6 +510,10 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
          "        for (int r0 = lane; r0 < nrec; r0 += 32) {\n"
          "          const int4 r = __ldg(srec + r0);\n"
          "          cb[r.x & 0xffff] = fmaf(__int_as_float(r.y), y[(r.x >> 16) & 0xff], __int_as_float(r.z) * y[(unsigned)r.x >> 24]);\n"
+         "#if TAN\n"
+         "          cht[b * chs + (r.x & 0xffff)] = fmaf(__int_as_float(r.y), sYt[b * DE + ((r.x >> 16) & 0xff)],\n"
+         "                                              __int_as_float(r.z) * sYt[b * DE + ((unsigned)r.x >> 24)]);\n"
+         "#endif\n"
          "        }\n"
          "      }\n";
   o << "      mbar_arrive(full0 + OFF_CHAT + 8 * s);\n"

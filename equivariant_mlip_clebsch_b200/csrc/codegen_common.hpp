@@ -74,6 +74,9 @@ struct KernelShape {
   int force_B = 0;  // edges per chunk fixed by the caller (0: chosen from the budget)
   int rec_max = 0;  // most Chat records of a slice
   bool edge_ranges = false;  // backward CTAs take equal edge ranges
+  // tangent kernels: every staged W, x and Y piece (and so Chat) has a
+  // second copy holding its directional derivative (the double backward)
+  bool tangent = false;
   int off_wb = 0;
 };
 

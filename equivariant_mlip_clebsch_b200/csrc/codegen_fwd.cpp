@@ -35,11 +35,14 @@ namespace cgtp {
 // The kernel entry after the role functions: service warps, then each
 // consumer warp runs its slot's role in every slice.
 static void gen_fwd_entry(std::ostringstream& o, const std::string& kname, int min_blocks,
-                          const std::string& dispatch) {
+                          const std::string& dispatch, bool tangent) {
   o << "extern \"C\" __global__ void __launch_bounds__((NW + 2) * 32, " << min_blocks << ") " << kname
     << "(const int* __restrict__ rowptr, const int* __restrict__ col, const float* __restrict__ x,\n"
        "    const float* __restrict__ Y, const float* __restrict__ W, const int* __restrict__ eid,\n"
-       "    float* __restrict__ out, const int4* __restrict__ ent, int n_recv, int* __restrict__ err) {\n"
+       "    float* __restrict__ out, const int4* __restrict__ ent, int n_recv, int* __restrict__ err"
+    << (tangent ? ",\n    const float* __restrict__ xt, const float* __restrict__ Yt, const float* __restrict__ Wt"
+                : "")
+    << ") {\n"
        "  extern __shared__ __align__(128) unsigned char smem[];\n"
        "  grid_dependency_wait();  // the previous kernel's results are visible\n"
        "  grid_launch_dependents();\n"
@@ -52,8 +55,9 @@ static void gen_fwd_entry(std::ostringstream& o, const std::string& kname, int m
        "    fence_mbar_init();\n"
        "  }\n"
        "  __syncthreads();\n"
-       "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, eid, nullptr, err, smem, lane); return; }\n"
-       "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, ent, kEntBegin, nullptr, err, smem, lane); return; }\n"
+    << (tangent ? "" : "  const float* xt = nullptr; const float* Yt = nullptr; const float* Wt = nullptr;\n")
+    << "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, xt, Wt, eid, nullptr, err, smem, lane); return; }\n"
+       "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, Yt, ent, kEntBegin, nullptr, err, smem, lane); return; }\n"
        "  int q = 0;\n"
        "  for (int slice = 0; slice < NSLICE; ++slice) {\n"
        "    const int slot = slice * NW + warp;\n"
@@ -129,9 +133,19 @@ static std::string gen_fwd_generic(const Plan& P, const std::vector<SliceLayout>
          "      float xv[1][" << N1 << "], w[1];\n"
          "#pragma unroll\n      for (int m1 = 0; m1 < " << N1 << "; ++m1) xv[0][m1] = ok ? sX[b * XS + u * " << N1
       << " + m1] : 0.f;\n"
-         "      w[0] = ok ? sW[b * WS + u] : 0.f;\n"
-         "      fpath<" << N1 << "," << N3 << ",1,0," << N3 << ">(acc, sC + b * chs, xv, w);\n"
-         "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n"
+         "      w[0] = ok ? sW[b * WS + u] : 0.f;\n";
+    if (K.tangent)
+      o << "      float xtv[1][" << N1 << "], wt[1];\n"
+           "      const float* sXt = reinterpret_cast<const float*>(st + OFF_XT) + xst;\n"
+           "      const float* sWt = reinterpret_cast<const float*>(st + OFF_WT) + wst;\n"
+           "      const float* sCt = reinterpret_cast<const float*>(st + OFF_CHT) + choff;\n"
+           "#pragma unroll\n      for (int m1 = 0; m1 < " << N1 << "; ++m1) xtv[0][m1] = ok ? sXt[b * XS + u * " << N1
+        << " + m1] : 0.f;\n"
+           "      wt[0] = ok ? sWt[b * WS + u] : 0.f;\n"
+           "      fpath_tan<" << N1 << "," << N3 << ",1,0," << N3 << ">(acc, sC + b * chs, sCt + b * chs, xv, xtv, w, wt);\n";
+    else
+      o << "      fpath<" << N1 << "," << N3 << ",1,0," << N3 << ">(acc, sC + b * chs, xv, w);\n";
+    o << "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n"
          "  if (ok) {\n    float* orow = out + (size_t)i * DOUT + ooff;\n"
          "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) orow[u * " << N3 << " + m3] = acc[m3];\n  }\n"
          "  }\n  *qp = q;\n}\n";
@@ -163,7 +177,7 @@ static std::string gen_fwd_generic(const Plan& P, const std::vector<SliceLayout>
     d << "    case " << k << ": fgen_" << k
       << "(rowptr, n_recv, out, err, smem, u0, chs, kChOff[slot], kWst[slot], kXst[slot], kOoff[slot], kMul[slot], "
          "&q); break;\n";
-  gen_fwd_entry(o, kname, min_blocks, d.str());
+  gen_fwd_entry(o, kname, min_blocks, d.str(), K.tangent);
   return o.str();
 }
 
@@ -234,14 +248,30 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
          "        const int u = u0 + r * 32 + lane;\n"
          "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) xv[r][m1] = ok[r] ? xr[u * " << N1
       << " + m1] : 0.f;\n      }\n";
+    if (K.tangent)  // the tangent copies of the same pieces
+      o << "      const float* chtb = reinterpret_cast<const float*>(st + OFF_CHT) + b * chs;\n"
+           "      const float* wtr = reinterpret_cast<const float*>(st + OFF_WT) + b * WS;\n"
+           "      const float* xtr = reinterpret_cast<const float*>(st + OFF_XT) + " << sl.x_st.at(r.irrep)
+        << " + b * XS;\n"
+           "      float xtv[" << R << "][" << N1 << "];\n"
+           "#pragma unroll\n      for (int r = 0; r < " << R << "; ++r) {\n"
+           "        const int u = u0 + r * 32 + lane;\n"
+           "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) xtv[r][m1] = ok[r] ? xtr[u * " << N1
+        << " + m1] : 0.f;\n      }\n";
     int A = 0;
     for (int pi : r.paths) {
       const Path& p = P.paths[pi];
       const int N3 = 2 * p.l3 + 1;
       o << "      { float w[" << R << "];\n#pragma unroll\n        for (int r = 0; r < " << R
-        << "; ++r) w[r] = ok[r] ? wr[" << sl.w_st.at(pi) << " + u0 + r * 32 + lane] : 0.f;\n"
-        << "        fpath<" << N1 << "," << N3 << "," << R << "," << A << "," << nacc << ">(acc, chb + "
-        << sl.ch_off.at(pi) << ", xv, w); }\n";
+        << "; ++r) w[r] = ok[r] ? wr[" << sl.w_st.at(pi) << " + u0 + r * 32 + lane] : 0.f;\n";
+      if (K.tangent)
+        o << "        float wt[" << R << "];\n#pragma unroll\n        for (int r = 0; r < " << R
+          << "; ++r) wt[r] = ok[r] ? wtr[" << sl.w_st.at(pi) << " + u0 + r * 32 + lane] : 0.f;\n"
+          << "        fpath_tan<" << N1 << "," << N3 << "," << R << "," << A << "," << nacc << ">(acc, chb + "
+          << sl.ch_off.at(pi) << ", chtb + " << sl.ch_off.at(pi) << ", xv, xtv, w, wt); }\n";
+      else
+        o << "        fpath<" << N1 << "," << N3 << "," << R << "," << A << "," << nacc << ">(acc, chb + "
+          << sl.ch_off.at(pi) << ", xv, w); }\n";
       A += R * N3;
     }
     o << "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n";
@@ -272,7 +302,7 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
   std::ostringstream d;
   for (size_t k = 0; k < shape_rep.size(); ++k)
     d << "    case " << k << ": fcons_" << k << "(rowptr, n_recv, out, err, smem, u0, chs, &q); break;\n";
-  gen_fwd_entry(o, kname, min_blocks, d.str());
+  gen_fwd_entry(o, kname, min_blocks, d.str(), K.tangent);
   return o.str();
 }
 
@@ -288,9 +318,33 @@ static double fwd_role_cost(const Plan& P, const FwdRole& r) {
   return c;
 }
 
+// The staging layout of each forward slice: the paths and hidden irreps of
+// its roles.
+static std::vector<SliceLayout> forward_slices(const Plan& P) {
+  const FwdConfig& F = P.fcfg;
+  std::vector<SliceLayout> SL(F.S);
+  for (int s = 0; s < F.S; ++s) {
+    std::vector<char> pseen(P.paths.size(), 0), iseen(P.in.size(), 0);
+    for (int ri : F.slice_roles[s]) {
+      for (int pi : P.fwd_roles[ri].paths) pseen[pi] = 1;
+      iseen[P.fwd_roles[ri].irrep] = 1;
+    }
+    for (size_t k = 0; k < P.paths.size(); ++k)
+      if (pseen[k]) SL[s].paths.push_back((int)k);
+    for (size_t a = 0; a < P.in.size(); ++a)
+      if (iseen[a]) SL[s].irreps.push_back((int)a);
+    layout_slice(P, SL[s], false);
+  }
+  return SL;
+}
+
 cgtp_status build_forward(Plan& P) {
   // ---- roles: per hidden irrep, channel blocks x path groups
-  const int kAccBudget = 64;
+  // accumulator budget per lane (tuning override CGTP_FWD_BUDGET)
+  int kAccBudget = 64;
+  if (const char* v = std::getenv("CGTP_FWD_BUDGET")) kAccBudget = std::max(13, std::min(128, std::atoi(v)));
+  int force_R = 0;  // channels per lane (tuning override CGTP_FWD_R: 1 or 2)
+  if (const char* v = std::getenv("CGTP_FWD_R")) force_R = std::max(1, std::min(2, std::atoi(v)));
   P.fwd_roles.clear();
   for (size_t a = 0; a < P.in.size(); ++a) {
     const Irrep& h = P.in[a];
@@ -301,7 +355,7 @@ cgtp_status build_forward(Plan& P) {
     // wide inputs (l >= 3): one channel per lane and fewer accumulators, so
     // that x, w*x and the Chat row still fit beside them without spilling
     const int n1 = 2 * h.l + 1;
-    const int R = (h.mul >= 64 && h.l < 3) ? 2 : 1;
+    const int R = force_R ? std::min(force_R, std::max(1, h.mul / 32)) : ((h.mul >= 64 && h.l < 3) ? 2 : 1);
     const int beta = h.l < 3 ? std::max(13, kAccBudget / R)
                              : std::max(13, kAccBudget - 2 * n1 - ((n1 + 3) & ~3));
     std::vector<std::vector<int>> groups;
@@ -406,19 +460,7 @@ cgtp_status build_forward(Plan& P) {
     for (int pi : r.paths) n += r.R * (2 * P.paths[pi].l3 + 1);
     F.nacc = std::max(F.nacc, n);
   }
-  std::vector<SliceLayout> SL(F.S);
-  for (int s = 0; s < F.S; ++s) {
-    std::vector<char> pseen(P.paths.size(), 0), iseen(P.in.size(), 0);
-    for (int ri : F.slice_roles[s]) {
-      for (int pi : P.fwd_roles[ri].paths) pseen[pi] = 1;
-      iseen[P.fwd_roles[ri].irrep] = 1;
-    }
-    for (size_t k = 0; k < P.paths.size(); ++k)
-      if (pseen[k]) SL[s].paths.push_back((int)k);
-    for (size_t a = 0; a < P.in.size(); ++a)
-      if (iseen[a]) SL[s].irreps.push_back((int)a);
-    layout_slice(P, SL[s], false);
-  }
+  std::vector<SliceLayout> SL = forward_slices(P);
   KernelShape K;
   K.S = F.S;
   K.nw = F.nw;
@@ -438,7 +480,11 @@ cgtp_status build_forward(Plan& P) {
   // (but not below two) when the compiler reports sizeable spills
   if (K.smem > 227 * 1024) return fail(CGTP_ERR_SIZE, "forward kernel needs too much shared memory");
   bool fixed = false;
-  const int mb0 = initial_min_blocks(K.smem, &fixed);
+  int mb0 = initial_min_blocks(K.smem, &fixed);
+  if (const char* v = std::getenv("CGTP_FWD_MIN_BLOCKS")) {
+    mb0 = std::max(1, std::atoi(v));
+    fixed = true;
+  }
   const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
   // The compile runs on a host thread while the backward is planned and
   // compiled (NVRTC needs no CUDA context); finish_forward joins and loads.
@@ -467,6 +513,43 @@ cgtp_status build_forward(Plan& P) {
   P.fwd.smem = K.smem;
   P.fwd_pending = std::move(pend);
   return CGTP_OK;
+}
+
+// The forward's tangent kernel (cgtp_fwd_tan): the same roles and slices,
+// every W, x and Y piece staged with its directional derivative, so that one
+// pass gives d/dt fwd(x + t xt, Y + t Yt, W + t Wt).  Built on first use.
+cgtp_status build_forward_tangent(Plan& P, JitKernel& out, std::string* src_out) {
+  const FwdConfig& F = P.fcfg;
+  std::vector<SliceLayout> SL = forward_slices(P);
+  KernelShape K;
+  K.S = F.S;
+  K.nw = F.nw;
+  K.WB = 0;
+  K.tangent = true;
+  plan_layout(P, SL, K, false);
+  for (size_t k = 0; k + 1 < P.fwd_ent_begin.size(); ++k)
+    K.rec_max = std::max(K.rec_max, P.fwd_ent_begin[k + 1] - P.fwd_ent_begin[k]);
+  if (K.smem > 227 * 1024) return fail(CGTP_ERR_SIZE, "tangent forward needs too much shared memory");
+  bool fixed = false;
+  const int mb0 = initial_min_blocks(K.smem, &fixed);
+  const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
+  const std::string name = "cgtp_fwd_tan";
+  std::string src;
+  JitBinary bin;
+  cgtp_status st = CGTP_OK;
+  for (int mb = mb0; mb >= mb_floor; --mb) {
+    src = gen_fwd_source(P, SL, K, name, mb);
+    st = jit_build(src, name, bin);
+    if (st != CGTP_OK || mb == mb_floor || max_spill_bytes(bin.log) <= 64) break;
+  }
+  if (st != CGTP_OK) {
+    set_error(bin.err);
+    return st;
+  }
+  out.threads = (F.nw + 2) * 32;
+  out.smem = K.smem;
+  if (src_out) *src_out = src;
+  return jit_load(bin, name, out);
 }
 
 cgtp_status finish_forward(Plan& P) {

@@ -11,9 +11,21 @@
 #include <thread>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "cgtp.h"
 
 namespace cgtp {
+
+// An NVTX range over one C-ABI call, named after the entry point: it shows
+// each call (and the kernels it launched) on a profiler's timeline.  NVTX v3
+// is header-only and does nothing unless a profiling tool is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // ---------------------------------------------------------------- errors
 void set_error(const std::string& msg);
@@ -149,6 +161,13 @@ struct Plan {
   std::vector<int> bwd_chs;
   bool bwd_irrep_gap = false;  // some hidden irrep has no path
 
+  // tangent kernels of the double backward, built on first use (tan_state:
+  // 0 not built, 1 ready, -1 unavailable: the composition is used)
+  JitKernel fwd_tan, bwd_tan;
+  std::mutex tan_mu;
+  int tan_state = 0;
+  std::string tan_msg;
+
   int* d_err = nullptr;  // device error word
   // device checks of the graph before each call (cgtp_plan_set_checks;
   // CGTP_DEBUG=1 at plan creation): flags, the result word, its lock
@@ -207,6 +226,9 @@ cgtp_status build_paths(Plan& P);
 cgtp_status build_forward(Plan& P);
 cgtp_status build_backward(Plan& P);
 cgtp_status finish_forward(Plan& P);  // joins the forward's compile and loads it
+// tangent kernels (the double backward): built and loaded on the calling thread
+cgtp_status build_forward_tangent(Plan& P, JitKernel& out, std::string* src);
+cgtp_status build_backward_tangent(Plan& P, JitKernel& out, std::string* src);
 void destroy_plan_device(Plan& P);
 
 // JIT

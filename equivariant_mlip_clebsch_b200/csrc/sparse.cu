@@ -339,6 +339,7 @@ cgtp_status cgtp_sparse_forward(cgtp_plan plan, int64_t n_recv, int64_t n_send, 
                                 const int32_t* col, const float* x, const float* Y, const float* W,
                                 const float* gate, float* out, void* workspace, size_t workspace_bytes,
                                 cgtp_stream stream) {
+  NvtxRange nvtx_range("cgtp_sparse_forward");
   if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
   const Plan& P = *reinterpret_cast<const Plan*>(plan);
   const SparseLayout L = sparse_layout(P, std::max<int64_t>(n_recv, 0), std::max<int64_t>(n_send, 0),
@@ -367,6 +368,7 @@ cgtp_status cgtp_sparse_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send,
                                  const float* x, const float* Y, const float* W, const float* gate,
                                  const float* grad_out, float* grad_x, float* grad_W, float* grad_Y,
                                  float* grad_gate, void* workspace, size_t workspace_bytes, cgtp_stream stream) {
+  NvtxRange nvtx_range("cgtp_sparse_backward");
   if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
   const Plan& P = *reinterpret_cast<const Plan*>(plan);
   const SparseLayout L = sparse_layout(P, std::max<int64_t>(n_recv, 0), std::max<int64_t>(n_send, 0),

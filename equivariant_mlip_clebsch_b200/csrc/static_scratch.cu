@@ -55,6 +55,7 @@ extern "C" cgtp_status cgtp_backward_static_scratch(
     const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, const float* x,
     const float* Y, const float* W, const float* grad_out, float* grad_x, float* grad_W,
     float* grad_Y, cgtp_stream stream) {
+  cgtp::NvtxRange nvtx_range("cgtp_backward_static_scratch");
   if (!plan) return cgtp::fail(CGTP_ERR_NULL, "plan is NULL");
   const cgtp::Plan& P = *reinterpret_cast<const cgtp::Plan*>(plan);
   // every host check first: a call with the wrong device current, a bad size

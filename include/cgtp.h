@@ -367,6 +367,19 @@ cgtp_status cgtp_fma_peak(int64_t iters, float* sink, int64_t sink_floats, cgtp_
  * device or a compile-only plan). */
 cgtp_status cgtp_double_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
                                                 size_t* bytes);
+
+/* With all three cotangents given, cgtp_double_backward runs two tangent
+ * kernels instead of the calls above: the forward and the backward compiled
+ * with every W, x and Y piece staged beside its direction (h_W, h_x, h_Y),
+ * which give d/dt fwd(x + t h_x, Y + t h_Y, W + t h_W) = gg_out and
+ * d/dt bwd(x + t h_x, Y + t h_Y, W + t h_W; grad_out) = (gx, gW, gY) in one
+ * pass each (the same sums as above, every input read once).  They are
+ * compiled on the plan's first such call; cgtp_plan_prepare_double_backward
+ * compiles them ahead (call it before any stream capture).  *tangent (may be
+ * NULL) receives 1 when they are available, 0 when the plan keeps the
+ * composition (a tangent stage that does not fit shared memory, or
+ * CGTP_DBWD_COMPOSE set at the first call).  Errors: NULL, CUDA. */
+cgtp_status cgtp_plan_prepare_double_backward(cgtp_plan plan, int* tangent);
 cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
                                  const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
                                  const int32_t* perm_T, const float* x, const float* Y, const float* W,

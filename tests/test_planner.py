@@ -145,7 +145,8 @@ def _check_copies(src):
         if not (S + N <= DOUT and D + N <= GS):
             bad.append(m.group(0))
     recognised = 0
-    for arr, row, width, slot in (("sW", "WROW", NU, WS), ("sX", "XROW", DIN, XS)):
+    for arr, row, width, slot in (("sW", "WROW", NU, WS), ("sX", "XROW", DIN, XS),
+                                  ("sWt", "WTROW", NU, WS), ("sXt", "XTROW", DIN, XS)):
         for m in re.finditer(r"t < nb \* (\d+); t \+= 32\) \{ const int b = t / \d+, q = t - b \* \d+; " + arr
                              + r"\[b \* (\d+) \+ (\d+) \+ q\] = " + row + r"\(b\)\[(\d+) \+ q\]", src):
             N, stride, D, S = map(int, m.groups())
@@ -168,11 +169,12 @@ def _check_copies(src):
                 and S + B // 4 <= DOUT and D + B // 4 <= GS):
             bad.append(m.group(0))
     # one copy for a chunk's consecutive W rows (only W rows are contiguous)
-    for m in re.finditer(r"bulk_g2s_stream\(smem_u32\((sW|sX)\), (WROW|XROW)\(0\), \(u32\)nb \* (\d+),", src):
+    for m in re.finditer(r"bulk_g2s_stream\(smem_u32\((sWt?|sXt?)\), (WT?ROW|XT?ROW)\(0\), \(u32\)nb \* (\d+),", src):
         B = int(m.group(3))
         n += 1
         recognised += 1
-        if not (m.group(1) == "sW" and B == 4 * NU and WS == NU and B % 16 == 0):
+        if not (m.group(1) in ("sW", "sWt") and m.group(2) in ("WROW", "WTROW") and B == 4 * NU and WS == NU
+                and B % 16 == 0):
             bad.append(m.group(0))
     total = len(re.findall(r"\bbulk_g2s(?:_stream)?\(smem_u32", src))
     if total != recognised:
@@ -189,17 +191,28 @@ def _check_layout(src, smem, backward):
     bytes (TMA destinations)."""
     d = _defines(src)
     NB, NW, NS, DE = d["NB"], d["NW"], d["NSTAGE"], d["DE"]
+    mt = 2 if d.get("TAN", 0) else 1  # tangent kernels stage every piece twice
     off = [d["OFF_W"], d["OFF_X"], d["OFF_Y"], d["OFF_CH"], d["OFF_DY"]]
-    size = [4 * NB * d["WS"], 4 * NB * d["XS"], 4 * NB * DE, 4 * NB * d["CHS"],
+    size = [4 * mt * NB * d["WS"], 4 * mt * NB * d["XS"], 4 * mt * NB * DE, 4 * mt * NB * d["CHS"],
             4 * NW * NB * DE if backward else 0]
     bad = [f"region {k}" for k in range(4) if off[k] + size[k] > off[k + 1]]
     if off[4] + size[4] > d["STAGE_BYTES"]:
         bad.append("dY partials past the stage")
     if any(v % 16 for v in off + [d["STAGE_BYTES"], d["OFF_STAGE"], d["OFF_G"], d["OFF_WB"]]):
         bad.append("offset not 16-byte aligned")
-    # full/empty/chat barriers, grad_out barriers, stage records, edge range
-    if 3 * 8 * NS + 32 + 16 * NS + 16 > d["OFF_STAGE"]:
-        bad.append("barriers past the first stage")
+    # the header below the first stage: full/empty/chat barriers (8 bytes
+    # each, 8-byte aligned), the grad_out barriers, the int4 stage records and
+    # the edge range (16-byte aligned), in order and without overlap
+    hdr = [(0, 8 * NS, 8), (8 * NS, 8 * NS, 8), (d["OFF_CHAT"], 8 * NS, 8), (d["OFF_GFULL"], 16, 8),
+           (d["OFF_GEMPTY"], 16, 8), (d["OFF_DESC"], 16 * NS, 16), (d["OFF_RANGE"], 16, 16)]
+    for (o0, n0, a0), (o1, _, _) in zip(hdr, hdr[1:]):
+        if o0 + n0 > o1:
+            bad.append(f"header region at {o0} overlaps the next at {o1}")
+    for o0, n0, a0 in hdr:
+        if o0 % a0:
+            bad.append(f"header region at {o0} not {a0}-byte aligned")
+    if hdr[-1][0] + hdr[-1][1] > d["OFF_STAGE"]:
+        bad.append("header past the first stage")
     if d["OFF_STAGE"] + NS * d["STAGE_BYTES"] > d["OFF_G"]:
         bad.append("stage ring past the grad_out buffers")
     gbytes = d.get("GBUF", 0) * 4 * d.get("GS", 0) if backward else 0
@@ -230,6 +243,25 @@ def test_generated_copies_stay_in_bounds(irreps, compile_only, monkeypatch, tmp_
         assert not bad, (f, bad)
 
 
+@pytest.mark.parametrize("name", ["tiny", "lmax2", "lmax2_wide", "lmax3", "case5"])
+def test_tangent_kernels_copies_and_layout(name, compile_only, monkeypatch, tmp_path):
+    """The double backward's tangent kernels (built on request): the same
+    copy and layout checks, with every staged piece doubled."""
+    monkeypatch.setenv("CGTP_DUMP_SOURCE", str(tmp_path))
+    c = WL.CONFIGS[name]
+    plan = C.Plan(c["irreps_in"], c["irreps_edge"], c["irreps_out"], 6)
+    assert plan.prepare_double_backward()
+    desc = plan.describe()
+    smem = {k: int(v) for k, v in re.findall(r"^(cgtp_fwd_tan|cgtp_bwd_tan) .* smem=(\d+)", desc, re.M)}
+    for f, kname in (("fwd_tan.cu", "cgtp_fwd_tan"), ("bwd_tan.cu", "cgtp_bwd_tan")):
+        src = (tmp_path / f).read_text()
+        assert "#define TAN 1" in src
+        n, bad = _check_copies(src)
+        assert n > 0 and not bad, (f, bad[:3])
+        bad = _check_layout(src, smem[kname], f.startswith("bwd"))
+        assert not bad, (f, bad)
+
+
 def test_copy_check_catches_planted_mistakes():
     head = "#define DIN 64\n#define DOUT 128\n#define NU 96\n#define WS 96\n#define XS 64\n#define GS 128\n"
     ok = head + ("bulk_g2s(smem_u32(sW + b * 96 + 0), WROW(b) + 32, 256, bar);\n"
@@ -248,11 +280,26 @@ def test_copy_check_catches_planted_mistakes():
         assert bad, p
 
 
+def test_layout_check_catches_a_misaligned_header():
+    """A three-stage header whose stage records would start off a 16-byte
+    boundary (int4 stores) fails the layout check."""
+    good = ("#define NB 2\n#define NW 5\n#define NSTAGE 3\n#define DE 16\n#define WS 64\n#define XS 64\n"
+            "#define CHS 64\n#define OFF_W 0\n#define OFF_X 512\n#define OFF_Y 1024\n#define OFF_CH 1152\n"
+            "#define OFF_DY 1664\n#define STAGE_BYTES 1664\n#define OFF_STAGE 512\n#define OFF_G 5504\n"
+            "#define OFF_WB 5504\n#define OFF_CHAT 48\n#define OFF_GFULL 80\n#define OFF_GEMPTY 96\n"
+            "#define OFF_DESC 112\n#define OFF_RANGE 160\n")
+    assert not _check_layout(good, 5504, False)
+    bad = good.replace("#define OFF_GFULL 80\n#define OFF_GEMPTY 96\n#define OFF_DESC 112\n#define OFF_RANGE 160",
+                       "#define OFF_GFULL 72\n#define OFF_GEMPTY 88\n#define OFF_DESC 104\n#define OFF_RANGE 152")
+    assert any("16-byte aligned" in b for b in _check_layout(bad, 5504, False))
+
+
 def test_layout_check_catches_planted_mistakes():
     # W 1024 B, x 512, Y 144, C-hat 256, dY partials 576 per stage; two stages
     good = {"NB": 4, "NW": 4, "NSTAGE": 2, "DE": 9, "WS": 64, "XS": 32, "CHS": 16, "OFF_W": 0, "OFF_X": 1024,
             "OFF_Y": 1536, "OFF_CH": 1792, "OFF_DY": 2048, "STAGE_BYTES": 2688, "OFF_STAGE": 256,
-            "OFF_G": 5632, "GS": 128, "GBUF": 2, "OFF_WB": 6656, "WB": 32}
+            "OFF_G": 5632, "GS": 128, "GBUF": 2, "OFF_WB": 6656, "WB": 32,
+            "OFF_CHAT": 32, "OFF_GFULL": 48, "OFF_GEMPTY": 64, "OFF_DESC": 80, "OFF_RANGE": 112}
     text = lambda d: "".join(f"#define {k} {v}\n" for k, v in d.items())
     assert _check_layout(text(good), 7168, True) == []
     for key, val, smem in (("OFF_X", 768, 7168),      # W region overlaps x
