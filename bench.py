@@ -506,9 +506,14 @@ def run_cgtp(args, rank, world, local_rank):
         hx, hW, hY = (torch.randn(t.shape, device=dev, generator=gen) for t in (T["x"], T["W"], wb.Y))
         dgrads = tuple(torch.empty_like(t) for t in (T["g"], T["x"], T["W"], wb.Y))
         dws = torch.empty(max(plan.double_backward_workspace_size(N, N, E), 256), dtype=torch.uint8, device=dev)
-        dbl_ms = wb.timer(lambda: plan.double_backward(T["rowptr"], T["col"], T["rpt"], T["perm"], T["x"], wb.Y,
-                                                       T["W"], T["g"], h_x=hx, h_W=hW, h_Y=hY, grads=dgrads,
-                                                       workspace=dws), args.steps)
+        tangent = plan.prepare_double_backward()  # builds the tangent kernels outside the timing
+
+        def dbl():
+            plan.double_backward(T["rowptr"], T["col"], T["rpt"], T["perm"], T["x"], wb.Y, T["W"], T["g"],
+                                 h_x=hx, h_W=hW, h_Y=hY, grads=dgrads, workspace=dws)
+        dbl()
+        torch.cuda.synchronize()
+        dbl_ms = wb.timer(dbl, args.steps)
         # the operation's own bytes: x, Y, W, grad_out and the three cotangents
         # read once, the four gradients written once, both CSRs read
         dbl_bytes = 4 * (2 * N * plan.d_in + 2 * E * plan.d_edge + 2 * E * plan.n_weights + N * plan.d_out
@@ -517,6 +522,8 @@ def run_cgtp(args, rank, world, local_rank):
         double_backward = {"ms": dbl_ms, "edges_per_s": world * E / (dbl_ms * 1e-3),
                            "algorithmic_bytes": dbl_bytes, "achieved_gbs": dbl_bytes / (dbl_ms * 1e-3) / 1e9,
                            "vs_step": dbl_ms / ms_step_local,
+                           "path": "tangent kernels (one forward, one backward pass)" if tangent else
+                                   "composition of forwards and backwards",
                            "what": "double_backward with h_x, h_W, h_Y, after the step (not in it)"}
         del hx, hW, hY, dgrads, dws
     except (C.CgtpError, ValueError, TypeError) as e:  # reported, the headline stands
