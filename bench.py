@@ -556,6 +556,7 @@ def run_cgtp(args, rank, world, local_rank):
                 "frac_vs_spec_8000": kd["GB/s"] / 8000.0}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel"] = dom
+    roof["kernel_hashes"] = kernel_hashes(plan)
     roof["algorithmic_bytes_per_launch"] = alg_b.get(dom)
     roof["traffic"] = ncu_traffic(name, dom, plan)
     roof["fp32_sgemm_tflops"] = sgemm_tflops(dev)  # measured cuBLAS FP32 (CUDA cores), context
@@ -699,6 +700,17 @@ def run_e2e(args, plan, T, host, Y, out, dx, dW, dY, ws, E, dev, world):
     return {"value": replica_value(world, E, ms), "unit": "edges/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps,
             "pipelined": "host->device, compute and device->host on three streams, two buffer sets"}
+
+
+def kernel_hashes(plan) -> dict:
+    """The generated kernels' source hashes (as compiled in this process),
+    which key the committed ncu traffic figures."""
+    out = {}
+    for line in plan.describe().splitlines():
+        for tag, key in (("forward:", "cgtp_fwd"), ("backward:", "cgtp_bwd"), ("backward (edge ranges", "cgtp_bwd_er")):
+            if line.startswith(tag) and "hash=" in line:
+                out[key] = line.split("hash=")[1].split()[0]
+    return out
 
 
 def ncu_traffic(name, kernel, plan):

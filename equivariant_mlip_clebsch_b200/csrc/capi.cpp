@@ -526,7 +526,9 @@ cgtp_status backward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_
     const bool er = P->bwd_er.function && n_recv <= 8 * (int64_t)G;
     JitKernel& JK = er ? P->bwd_er : P->bwd;
     if (er) G = persistent_grid(P->bwd_er.blocks_per_sm, P->num_sms, n_recv);
-    void* args[] = {&rowptr, &col, &x, &Y, &W, &eid, &grad_out, &grad_W, &dyp, &m, &P->d_bwd_ent, &nr, &P->d_err};
+    int e_stride = (int)E;  // the slices' dY parts lie E edges apart
+    void* args[] = {&rowptr, &col, &x, &Y, &W, &eid, &grad_out, &grad_W, &dyp, &m, &P->d_bwd_ent, &nr, &P->d_err,
+                    &e_stride};
     TimedScope ts(*P, 2, s, allow_timing);
     st = jit_launch(JK, dim3(G), args, s);
     if (st != CGTP_OK) return st;
@@ -755,8 +757,9 @@ cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send,
       float* m = gx ? reinterpret_cast<float*>(ws + L.bwd) : nullptr;
       float* dyp = gY ? (P->bcfg.S > 1 ? reinterpret_cast<float*>(ws + L.bwd + off_dyp) : gY) : nullptr;
       if (m && P->bwd_irrep_gap) CGTP_CUDA_TRY(cudaMemsetAsync(m, 0, (size_t)E * P->D_in * sizeof(float), cs));
+      int e_stride = (int)E;
       void* args[] = {&rowptr, &col, &x, &Y, &W, &no_eid, &grad_out, &gW, &dyp, &m, &P->d_bwd_ent, &nr, &P->d_err,
-                      &h_x, &h_Y, &h_W};
+                      &e_stride, &h_x, &h_Y, &h_W};
       {
         TimedScope ts(*P, 7, cs);
         st = jit_launch(P->bwd_tan, dim3(persistent_grid(P->bwd_tan.blocks_per_sm, P->num_sms, n_recv)), args, cs);

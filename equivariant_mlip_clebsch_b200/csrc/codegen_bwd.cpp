@@ -297,7 +297,7 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
     << "(const int* __restrict__ rowptr, const int* __restrict__ col, const float* __restrict__ x,\n"
        "    const float* __restrict__ Y, const float* __restrict__ W, const int* __restrict__ eid,\n"
        "    const float* __restrict__ g, float* __restrict__ dW, float* __restrict__ dyp, float* __restrict__ msg,\n"
-       "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err"
+       "    const int4* __restrict__ ent, int n_recv, int* __restrict__ err, int e_stride"
     << (K.tangent ? ",\n    const float* __restrict__ xt, const float* __restrict__ Yt, const float* __restrict__ Wt"
                   : "")
     << ") {\n"
@@ -327,7 +327,7 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
        "  __syncthreads();\n"
     << (K.tangent ? "" : "  const float* xt = nullptr; const float* Yt = nullptr; const float* Wt = nullptr;\n")
     << "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, xt, Wt, eid, g, err, smem, lane); return; }\n"
-       "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, Yt, ent, kEntBegin, dyp, err, smem, lane); return; }\n"
+       "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, Yt, ent, kEntBegin, dyp, err, smem, lane, e_stride); return; }\n"
        "  int q = 0, kr = 0;\n"
        "  for (int slice = 0; slice < NSLICE; ++slice) {\n"
        "    const int slot = slice * NW + warp;\n"

@@ -418,15 +418,17 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
          "}\n";
   }
   // Yt: the tangent harmonics of tangent kernels (unused otherwise)
+  // E (backward): the edge stride between the slices' dY parts, the host's
+  // edge count (for the sparse evaluation an upper bound of the compact
+  // count the device CSR holds)
   o << "__device__ __noinline__ void helper_warp(const int* __restrict__ rowptr, int n_recv,\n"
        "    const float* __restrict__ Y, const float* __restrict__ Yt, const int4* __restrict__ rec,\n"
        "    const int* __restrict__ rec_begin, float* __restrict__ dyp, int* __restrict__ err,\n"
-       "    unsigned char* smem, int lane) {\n"
+       "    unsigned char* smem, int lane, int E) {\n"
        "  (void)Yt;\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  int4* desc = reinterpret_cast<int4*>(smem + OFF_DESC);  // (eb, nb, slice, -) of each stage\n"
        "  (void)dyp; (void)desc;\n"
-       "  const int E = rowptr[n_recv];\n"
        "  (void)E;\n"
        "  int last_slice[NSTAGE];\n"
        "#pragma unroll\n"

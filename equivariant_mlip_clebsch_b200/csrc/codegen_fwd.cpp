@@ -57,7 +57,7 @@ static void gen_fwd_entry(std::ostringstream& o, const std::string& kname, int m
        "  __syncthreads();\n"
     << (tangent ? "" : "  const float* xt = nullptr; const float* Yt = nullptr; const float* Wt = nullptr;\n")
     << "  if (warp == NW) { tma_warp(rowptr, n_recv, col, x, W, xt, Wt, eid, nullptr, err, smem, lane); return; }\n"
-       "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, Yt, ent, kEntBegin, nullptr, err, smem, lane); return; }\n"
+       "  if (warp == NW + 1) { helper_warp(rowptr, n_recv, Y, Yt, ent, kEntBegin, nullptr, err, smem, lane, 0); return; }\n"
        "  int q = 0;\n"
        "  for (int slice = 0; slice < NSLICE; ++slice) {\n"
        "    const int slot = slice * NW + warp;\n"
@@ -381,6 +381,111 @@ cgtp_status build_forward(Plan& P) {
         r.cost = fwd_role_cost(P, r);
         P.fwd_roles.push_back(r);
       }
+  }
+  // Balanced roles (CGTP_FWD_BALANCE=1): per hidden irrep, the channels per
+  // lane and the runs of its paths chosen so that the costliest role is as
+  // cheap as the warp budget allows (one slice of at most 16 warps, 8 with
+  // inputs of l >= 3).  A stage is released only when every warp has
+  // finished it, so the costliest role sets the pace.
+  if (const char* v = std::getenv("CGTP_FWD_BALANCE"); v && *v == '1') {
+    bool wide_in = false;
+    for (auto& h : P.in) wide_in = wide_in || h.l >= 3;
+    const int cap_roles = wide_in ? 8 : 16;
+    struct Opt {
+      int a, R, nblk;
+      std::vector<int> ps;
+      int acc_cap;
+    };
+    std::vector<Opt> opts;
+    for (size_t a = 0; a < P.in.size(); ++a) {
+      const Irrep& h = P.in[a];
+      std::vector<int> ps;
+      for (size_t k = 0; k < P.paths.size(); ++k)
+        if (P.paths[k].irrep == (int)a) ps.push_back((int)k);
+      if (ps.empty()) continue;
+      const int n1 = 2 * h.l + 1;
+      for (int R = 1; R <= 2; ++R) {
+        if (R == 2 && (h.mul < 64 || h.l >= 3)) continue;
+        const int cap = h.l < 3 ? kAccBudget : std::max(13, kAccBudget - 2 * n1 - ((n1 + 3) & ~3));
+        opts.push_back({(int)a, R, (h.mul + 32 * R - 1) / (32 * R), ps, cap});
+      }
+    }
+    auto run_cost = [&](const Opt& o, size_t i, size_t j) {
+      FwdRole r;
+      r.irrep = o.a;
+      r.u0 = 0;
+      r.R = o.R;
+      r.paths.assign(o.ps.begin() + i, o.ps.begin() + j);
+      return fwd_role_cost(P, r);
+    };
+    // the greedy runs of an option under a cost bound T (empty: infeasible)
+    auto groups_for = [&](const Opt& o, double T) {
+      std::vector<std::pair<size_t, size_t>> g;
+      size_t i = 0;
+      while (i < o.ps.size()) {
+        size_t j = i;
+        int acc = 0;
+        while (j < o.ps.size()) {
+          const int add = o.R * (2 * P.paths[o.ps[j]].l3 + 1);
+          if (j > i && (acc + add > o.acc_cap || run_cost(o, i, j + 1) > T)) break;
+          acc += add;
+          ++j;
+        }
+        if (run_cost(o, i, j) > T) return std::vector<std::pair<size_t, size_t>>();
+        g.push_back({i, j});
+        i = j;
+      }
+      return g;
+    };
+    std::vector<double> cand;
+    for (auto& o : opts)
+      for (size_t i = 0; i < o.ps.size(); ++i)
+        for (size_t j = i + 1; j <= o.ps.size(); ++j) cand.push_back(run_cost(o, i, j));
+    std::sort(cand.begin(), cand.end());
+    cand.erase(std::unique(cand.begin(), cand.end()), cand.end());
+    std::vector<FwdRole> best;
+    for (double T : cand) {
+      std::vector<FwdRole> roles;
+      bool ok = true;
+      for (size_t a = 0; a < P.in.size() && ok; ++a) {
+        int best_n = -1;
+        const Opt* bo = nullptr;
+        std::vector<std::pair<size_t, size_t>> bg;
+        for (auto& o : opts) {
+          if (o.a != (int)a) continue;
+          auto g = groups_for(o, T);
+          if (g.empty()) continue;
+          const int n = (int)g.size() * o.nblk;
+          if (best_n < 0 || n < best_n || (n == best_n && o.R > bo->R)) {
+            best_n = n;
+            bo = &o;
+            bg = g;
+          }
+        }
+        bool has_paths = false;
+        for (auto& o : opts) has_paths = has_paths || o.a == (int)a;
+        if (!has_paths) continue;
+        if (!bo) {
+          ok = false;
+          break;
+        }
+        for (auto& gr : bg)
+          for (int blk = 0; blk < bo->nblk; ++blk) {
+            FwdRole r;
+            r.irrep = bo->a;
+            r.u0 = blk * 32 * bo->R;
+            r.R = bo->R;
+            r.paths.assign(bo->ps.begin() + gr.first, bo->ps.begin() + gr.second);
+            r.cost = fwd_role_cost(P, r);
+            roles.push_back(r);
+          }
+      }
+      if (ok && (int)roles.size() <= cap_roles) {
+        best = roles;
+        break;
+      }
+    }
+    if (!best.empty()) P.fwd_roles = best;
   }
   // Roles are not split further to balance them: measured on B200, more and
   // smaller roles (single-block channel groups, split path groups) made the
