@@ -744,12 +744,22 @@ cgtp_status build_backward_tangent(Plan& P, JitKernel& out, std::string* src_out
     std::sort(SL[s2].paths.begin(), SL[s2].paths.end());
     layout_slice(P, SL[s2], true);
   }
-  for (K.force_B = F.B; K.force_B >= 1; K.force_B /= 2) {
+  // the largest chunk (at most the plain kernel's) whose doubled stages
+  // leave room for two CTAs per SM; else the largest that fits one
+  int pick = 0;
+  for (int B = F.B; B >= 1 && !pick; B /= 2) {
+    K.force_B = B;
     plan_layout(P, SL, K, true);
-    if (K.smem <= 227 * 1024) break;
+    if (2 * (K.smem + 1024) <= 228 * 1024) pick = B;
   }
-  if (K.force_B < 1 || K.smem > 227 * 1024)
-    return fail(CGTP_ERR_SIZE, "tangent backward needs too much shared memory");
+  for (int B = F.B; B >= 1 && !pick; B /= 2) {
+    K.force_B = B;
+    plan_layout(P, SL, K, true);
+    if (K.smem <= 227 * 1024) pick = B;
+  }
+  if (!pick) return fail(CGTP_ERR_SIZE, "tangent backward needs too much shared memory");
+  K.force_B = pick;
+  plan_layout(P, SL, K, true);
   for (size_t k = 0; k + 1 < P.bwd_ent_begin.size(); ++k)
     K.rec_max = std::max(K.rec_max, P.bwd_ent_begin[k + 1] - P.bwd_ent_begin[k]);
   bool fixed = false;

@@ -117,6 +117,10 @@ void layout_slice(const Plan& P, SliceLayout& sl, bool with_g) {
   }
 }
 
+// Chunks ahead of the stage ring whose W rows the TMA warp prefetches into
+// L2 (tuning override CGTP_PREFETCH).
+static const int kDefaultPrefetch = 0;
+
 void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape& K, bool backward) {
   K.WS = K.XS = K.CHS = K.GS = 0;
   K.w_bulk = K.x_bulk = K.g_bulk = true;
@@ -156,6 +160,8 @@ void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape&
   // tuning overrides: edges per chunk and ring depth
   if (const char* v = std::getenv("CGTP_CHUNK"); v && K.force_B == 0) K.B = std::max(1, std::min(8, std::atoi(v)));
   if (const char* v = std::getenv("CGTP_STAGES")) K.stages = std::max(2, std::min(6, std::atoi(v)));
+  K.prefetch = kDefaultPrefetch;  // W rows prefetched into L2, in chunks ahead
+  if (const char* v = std::getenv("CGTP_PREFETCH")) K.prefetch = std::max(0, std::min(64, std::atoi(v)));
   while (K.stages > 2 && fixed + K.stages * stage_of(K.B) > 220 * 1024) --K.stages;
   K.sdy_floats = backward ? K.nw * K.B * (int)P.D_e : 0;
   K.off_stage = 512;  // mbarriers, chunk descriptors and the edge range first
@@ -208,7 +214,8 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
     << K.off_x << "\n#define OFF_Y " << K.off_y << "\n#define OFF_CH " << K.off_ch << "\n#define OFF_DY "
     << K.off_dy << "\n#define OFF_G " << K.off_g << "\n#define GS " << K.GS << "\n#define WB " << K.WB
     << "\n#define OFF_WB " << K.off_wb << "\n#define FULL_COUNT 32\n#define CHAT_COUNT 32\n#define GBUF " << K.gbufs << "\n#define YPL "
-    << (K.B * P.D_e + 31) / 32 << "\n#define TAN " << (K.tangent ? 1 : 0) << "\n";
+    << (K.B * P.D_e + 31) / 32 << "\n#define TAN " << (K.tangent ? 1 : 0) << "\n#define PF " << K.prefetch
+    << "\n";
   // tangent copies of a stage's regions, right after the plain ones
   o << "#define OFF_WT (OFF_W + 4 * NB * WS)\n#define OFF_XT (OFF_X + 4 * NB * XS)\n"
        "#define OFF_YT (OFF_Y + 4 * NB * DE)\n#define OFF_CHT (OFF_CH + 4 * NB * CHS)\n";
@@ -316,10 +323,39 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
       o << "        mbar_arrive(gfull0 + 8 * gb);\n"
            "        ++k;\n      }\n";
     }
+    // W rows PF chunks ahead (into the CTA's next receiver near the end of
+    // this one) are prefetched into L2 before the wait for a free stage
+    std::ostringstream pf;
+    if (K.prefetch > 0 && K.w_bulk) {
+      pf << "        {\n"
+            "          int pe = eb + PF * NB, pe1 = e1;\n"
+            "          if (pe >= e1) {  // past this receiver: the next one's edges\n"
+            "            const int i2 = i + RECV_STEP;\n"
+            "            pe1 = 0;\n"
+            "            if (i2 < RECV_END) { const int a2 = EDGE_LO(i2); pe1 = EDGE_HI(i2); pe = a2 + (pe - e1); }\n"
+            "          }\n"
+            "          const int npf = min(NB, pe1 - pe);\n"
+            "          if (npf > 0) {\n";
+      if (w_one)
+        pf << "            if (eid == nullptr) {\n"
+              "              if (lane == 0) bulk_prefetch_l2(W + (size_t)pe * NU, (u32)npf * " << P.U * 4 << ");\n"
+              "            } else if (lane < npf) {\n"
+              "              bulk_prefetch_l2(W + (size_t)__ldg(eid + pe + lane) * NU, " << P.U * 4 << ");\n"
+              "            }\n";
+      else {
+        pf << "            if (lane < npf) {\n"
+              "              const float* wrow = W + (size_t)(eid ? __ldg(eid + pe + lane) : pe + lane) * NU;\n";
+        for (auto& q : sl.wseg) pf << "              bulk_prefetch_l2(wrow + " << q.src << ", " << q.len * 4 << ");\n";
+        pf << "            }\n";
+      }
+      pf << "          }\n        }\n";
+    }
     o << "      for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
          "        const int s = q % NSTAGE;\n"
          "        const int nb = min(NB, e1 - eb);\n"
          "        const int jj = (lane < nb) ? __ldg(col + eb + lane) : 0;  // read before the wait\n"
+      << pf.str();
+    o << ""
          "        if (q >= NSTAGE && !mbar_wait(empty0 + 8 * s, ((q / NSTAGE) - 1) & 1)) { if (lane == 0) atomicOr(err, 10); dead = true; break; }\n"
          "        unsigned char* st = stage_ptr(smem, s);\n"
          "        float* sW = reinterpret_cast<float*>(st + OFF_W);\n"

@@ -77,6 +77,8 @@ struct KernelShape {
   // tangent kernels: every staged W, x and Y piece (and so Chat) has a
   // second copy holding its directional derivative (the double backward)
   bool tangent = false;
+  // W rows prefetched into L2 this many chunks ahead (0: off)
+  int prefetch = 0;
   int off_wb = 0;
 };
 

@@ -179,6 +179,23 @@ def _check_copies(src):
     total = len(re.findall(r"\bbulk_g2s(?:_stream)?\(smem_u32", src))
     if total != recognised:
         bad.append(f"{total - recognised} bulk copies of an unrecognised form")
+    # L2 prefetches of W: whole rows of the chunk, or row pieces, inside the
+    # row, 16-byte aligned, multiples of 16 bytes
+    pre = 0
+    for m in re.finditer(r"bulk_prefetch_l2\(wrow \+ (\d+), (\d+)\)", src):
+        S, B = map(int, m.groups())
+        n += 1
+        pre += 1
+        if not (S % 4 == 0 and B % 16 == 0 and S + B // 4 <= NU):
+            bad.append(m.group(0))
+    for m in re.finditer(r"bulk_prefetch_l2\(W \+ \(size_t\)(?:pe|__ldg\(eid \+ pe \+ lane\)) \* NU, "
+                         r"(?:\(u32\)npf \* )?(\d+)\)", src):
+        n += 1
+        pre += 1
+        if not (int(m.group(1)) == 4 * NU and NU % 4 == 0):
+            bad.append(m.group(0))
+    if pre != len(re.findall(r"\bbulk_prefetch_l2\((?!const void)", src)):  # calls, not the definition
+        bad.append("prefetches of an unrecognised form")
     return n, bad
 
 
@@ -225,11 +242,13 @@ def _check_layout(src, smem, backward):
 
 @pytest.mark.parametrize("irreps", [WL.CONFIGS[n] for n in NAMES] + [
     dict(irreps_in=a, irreps_edge=b, irreps_out=c) for a, b, c in ODD], ids=NAMES + [f"odd{k}" for k in range(len(ODD))])
-def test_generated_copies_stay_in_bounds(irreps, compile_only, monkeypatch, tmp_path):
-    """The generated kernels' row copies into shared memory, read from the
-    generated source (checked here so that a mistake fails on the CPU rather
-    than faulting a GPU)."""
+@pytest.mark.parametrize("prefetch", ["0", "4"])
+def test_generated_copies_stay_in_bounds(irreps, prefetch, compile_only, monkeypatch, tmp_path):
+    """The generated kernels' row copies into shared memory and their L2
+    prefetches, read from the generated source (checked here so that a
+    mistake fails on the CPU rather than faulting a GPU)."""
     monkeypatch.setenv("CGTP_DUMP_SOURCE", str(tmp_path))
+    monkeypatch.setenv("CGTP_PREFETCH", prefetch)
     plan = C.Plan(irreps["irreps_in"], irreps["irreps_edge"], irreps["irreps_out"], 6)
     smem = {k: int(v) for k, v in re.findall(r"^(forward|backward): .* smem=(\d+)", plan.describe(), re.M)}
     files = sorted(p.name for p in tmp_path.iterdir())
