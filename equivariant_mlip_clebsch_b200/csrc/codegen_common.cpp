@@ -290,8 +290,22 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
        "  (void)k;\n"
        "  bool dead = false;\n"
        "  for (int slice = 0; slice < NSLICE && !dead; ++slice) {\n"
+       "  // The receivers' edge ranges are loaded two receivers ahead and their\n"
+       "  // first 32 sender ids (one per lane) one receiver ahead, so that no\n"
+       "  // chunk waits on a dependent global load before its copies are issued.\n"
+       "  int e0n = 0, e1n = 0, e0nn = 0, e1nn = 0, cnext = 0;\n"
+       "  if (RECV_FIRST < RECV_END) {\n"
+       "    e0n = EDGE_LO(RECV_FIRST); e1n = EDGE_HI(RECV_FIRST);\n"
+       "    cnext = (e0n + lane < e1n) ? __ldg(col + e0n + lane) : 0;\n"
+       "    if (RECV_FIRST + RECV_STEP < RECV_END) { e0nn = EDGE_LO(RECV_FIRST + RECV_STEP); e1nn = EDGE_HI(RECV_FIRST + RECV_STEP); }\n"
+       "  }\n"
        "  for (int i = RECV_FIRST; i < RECV_END && !dead; i += RECV_STEP) {\n"
-       "    const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n";
+       "    const int e0 = e0n, e1 = e1n;\n"
+       "    int cbase = e0, cwin = cnext;  // sender ids of edges [cbase, cbase + 32), one per lane\n"
+       "    e0n = e0nn; e1n = e1nn;\n"
+       "    cnext = (i + RECV_STEP < RECV_END && e0n + lane < e1n) ? __ldg(col + e0n + lane) : 0;\n"
+       "    if (i + 2 * RECV_STEP < RECV_END) { e0nn = EDGE_LO(i + 2 * RECV_STEP); e1nn = EDGE_HI(i + 2 * RECV_STEP); }\n"
+       "    (void)cbase; (void)cwin;\n";
   if (backward) o << "    if (e1 <= e0) continue;\n";
   o << "    switch (slice) {\n";
   for (int s = 0; s < S; ++s) {
@@ -353,7 +367,11 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
     o << "      for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
          "        const int s = q % NSTAGE;\n"
          "        const int nb = min(NB, e1 - eb);\n"
-         "        const int jj = (lane < nb) ? __ldg(col + eb + lane) : 0;  // read before the wait\n"
+         "        if (eb + nb > cbase + 32) {  // the next 32 sender ids of this receiver\n"
+         "          cbase = eb;\n"
+         "          cwin = (eb + lane < e1) ? __ldg(col + eb + lane) : 0;\n"
+         "        }\n"
+         "        const int jj = __shfl_sync(0xffffffffu, cwin, (eb - cbase + lane) & 31);  // edge eb + lane's sender\n"
       << pf.str();
     o << ""
          "        if (q >= NSTAGE && !mbar_wait(empty0 + 8 * s, ((q / NSTAGE) - 1) & 1)) { if (lane == 0) atomicOr(err, 10); dead = true; break; }\n"
