@@ -266,6 +266,10 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
   o << "__constant__ int kChs[" << S << "] = {";
   for (int s = 0; s < S; ++s) o << SL[s].chs << ",";
   o << "};\n";
+  // a consumer's receiver loop: the next receiver's edge range is loaded
+  // one receiver ahead (e0n_, e1n_), off the critical path
+  o << "#define RECV_AHEAD_INIT int e0n_ = 0, e1n_ = 0; if (RECV_FIRST < RECV_END) { e0n_ = EDGE_LO(RECV_FIRST); e1n_ = EDGE_HI(RECV_FIRST); }\n"
+       "#define RECV_AHEAD_NEXT if (i + RECV_STEP < RECV_END) { e0n_ = EDGE_LO(i + RECV_STEP); e1n_ = EDGE_HI(i + RECV_STEP); }\n";
   o << "__device__ __forceinline__ unsigned char* stage_ptr(unsigned char* smem, int s) {\n"
        "  return smem + OFF_STAGE + s * STAGE_BYTES;\n}\n";
 
