@@ -507,8 +507,10 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
       << "    const int4 r = k < nk ? __ldg(srec + lane + 32 * k) : make_int4(0, 0, 0, 0);\n"
       << "    rd[k] = r.x;\n    rc0[k] = __int_as_float(r.y);\n    rc1[k] = __int_as_float(r.z);\n  }\n";
   o <<
+       "  RECV_AHEAD_INIT\n"
        "  for (int i = RECV_FIRST; i < RECV_END && !dead; i += RECV_STEP) {\n"
-       "    const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
+       "    const int e0 = e0n_, e1 = e1n_;\n"
+       "    RECV_AHEAD_NEXT\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
        "      const int s = q % NSTAGE;\n"
        "      const int nb = min(NB, e1 - eb);\n"
