@@ -109,9 +109,8 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       << "  const u32 gfull0 = full0 + OFF_GFULL, gempty0 = full0 + OFF_GEMPTY;\n"
 
       << "  int q = *qp, kr = *kp;\n"
-      << "  RECV_AHEAD_INIT\n#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
-      << "  const int e0 = e0n_, e1 = e1n_;\n"
-      << "  RECV_AHEAD_NEXT\n"
+      << "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
+      << "  const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
       << "  if (e1 <= e0) continue;\n"
       << "  const int gb = kr % GBUF;\n"
       << "  if (!mbar_wait(gfull0 + 8 * gb, (kr / GBUF) & 1)) { if (lane == 0) atomicOr(err, 10); *qp = -1; return; }\n"
@@ -268,9 +267,8 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  const u32 gempty0 = full0 + OFF_GEMPTY;\n"
        "  int q = *qp, kr = *kp;\n"
-       "  RECV_AHEAD_INIT\n#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
-       "    const int e0 = e0n_, e1 = e1n_;\n"
-       "    RECV_AHEAD_NEXT\n"
+       "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
+       "    const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
        "    if (e1 <= e0) continue;\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
        "      const int s = q % NSTAGE;\n"

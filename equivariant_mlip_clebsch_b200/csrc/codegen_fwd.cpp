@@ -74,9 +74,8 @@ static void gen_fwd_idle(std::ostringstream& o) {
        "  const int lane = threadIdx.x & 31;\n"
        "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
        "  int q = *qp;\n"
-       "  RECV_AHEAD_INIT\n#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
-       "    const int e0 = e0n_, e1 = e1n_;\n"
-       "    RECV_AHEAD_NEXT\n"
+       "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
+       "    const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
        "      const int s = q % NSTAGE;\n"
        "      if (!stage_ready(full0, s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); *qp = -1; return; }\n"
@@ -118,9 +117,8 @@ static std::string gen_fwd_generic(const Plan& P, const std::vector<SliceLayout>
          "  const bool ok = " << (full ? "true" : "u < mul") << ";\n"
          "  (void)mul;\n"
          "  int q = *qp;\n"
-         "  RECV_AHEAD_INIT\n#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
-         "  const int e0 = e0n_, e1 = e1n_;\n"
-         "  RECV_AHEAD_NEXT\n"
+         "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
+         "  const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
          "  float acc[" << N3 << "];\n"
          "#pragma unroll\n  for (int k = 0; k < " << N3 << "; ++k) acc[k] = 0.f;\n"
          "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
@@ -229,9 +227,8 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
       << (MUL % (32 * R) == 0 ? std::string("true") : "u0 + r * 32 + lane < " + std::to_string(MUL))
       << ";  // every lane holds a channel when the blocks are full\n"
          "  int q = *qp;\n"
-         "  RECV_AHEAD_INIT\n#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
-         "  const int e0 = e0n_, e1 = e1n_;\n"
-         "  RECV_AHEAD_NEXT\n"
+         "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
+         "  const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
          "  float acc[" << nacc << "];\n"
          "#pragma unroll\n  for (int k = 0; k < " << nacc << "; ++k) acc[k] = 0.f;\n"
          "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
