@@ -266,10 +266,6 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
   o << "__constant__ int kChs[" << S << "] = {";
   for (int s = 0; s < S; ++s) o << SL[s].chs << ",";
   o << "};\n";
-  // a consumer's receiver loop: the next receiver's edge range is loaded
-  // one receiver ahead (e0n_, e1n_), off the critical path
-  o << "#define RECV_AHEAD_INIT int e0n_ = 0, e1n_ = 0; if (RECV_FIRST < RECV_END) { e0n_ = EDGE_LO(RECV_FIRST); e1n_ = EDGE_HI(RECV_FIRST); }\n"
-       "#define RECV_AHEAD_NEXT if (i + RECV_STEP < RECV_END) { e0n_ = EDGE_LO(i + RECV_STEP); e1n_ = EDGE_HI(i + RECV_STEP); }\n";
   o << "__device__ __forceinline__ unsigned char* stage_ptr(unsigned char* smem, int s) {\n"
        "  return smem + OFF_STAGE + s * STAGE_BYTES;\n}\n";
 
@@ -507,10 +503,8 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
       << "    const int4 r = k < nk ? __ldg(srec + lane + 32 * k) : make_int4(0, 0, 0, 0);\n"
       << "    rd[k] = r.x;\n    rc0[k] = __int_as_float(r.y);\n    rc1[k] = __int_as_float(r.z);\n  }\n";
   o <<
-       "  RECV_AHEAD_INIT\n"
        "  for (int i = RECV_FIRST; i < RECV_END && !dead; i += RECV_STEP) {\n"
-       "    const int e0 = e0n_, e1 = e1n_;\n"
-       "    RECV_AHEAD_NEXT\n"
+       "    const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
        "    for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
        "      const int s = q % NSTAGE;\n"
        "      const int nb = min(NB, e1 - eb);\n"
