@@ -190,6 +190,7 @@ cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge, con
       CGTP_CUDA_TRY(upload_sph_norm());  // once per device, before any capture
       if (const char* d = std::getenv("CGTP_DEBUG"); d && *d && *d != '0') P->checks.store(CGTP_CHECK_GRAPH);
     }
+    if (const char* v = std::getenv("CGTP_BWD_TFORM"); v && *v == '1') P->bwd_tform = true;
     st = build_forward(*P);  // leaves the forward compiling on a host thread
     if (st == CGTP_OK) st = build_backward(*P);
     if (st == CGTP_OK)

@@ -134,6 +134,10 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
                       "      const float* xtr = reinterpret_cast<const float*>(st + OFF_XT) + " +
                           std::to_string(sl.x_st.at(r.irrep)) + " + b * XS;\n"
                     : "")
+      << (K.no_chat ? std::string("      const float* yr = reinterpret_cast<const float*>(st + OFF_Y) + b * DE;\n") +
+                          (K.tangent ? "      const float* ytr = reinterpret_cast<const float*>(st + OFF_YT) + b * DE;\n"
+                                     : "")
+                    : std::string())
       << "      float* dWrow = dW ? dW + (size_t)(eid ? __ldg(eid + e) : e) * NU : nullptr;\n"
       << "      float* sdy = want_dy ? sdyw + b * DE : nullptr;\n"
       ;
@@ -176,6 +180,13 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       if (!combined)
         o << "        float z[" << pow2(N2) << "];\n#pragma unroll\n        for (int t = 0; t < " << pow2(N2)
           << "; ++t) z[t] = 0.f;\n";
+      if (K.no_chat) {  // this degree's harmonics of the edge (the same for every lane)
+        o << "        float yl[" << N2 << "];\n#pragma unroll\n        for (int m2 = 0; m2 < " << N2
+          << "; ++m2) yl[m2] = yr[" << l2 * l2 << " + m2];\n";
+        if (K.tangent)
+          o << "        float ytl[" << N2 << "];\n#pragma unroll\n        for (int m2 = 0; m2 < " << N2
+            << "; ++m2) ytl[m2] = ytr[" << l2 * l2 << " + m2];\n";
+      }
       for (; q < ps.size() && P.paths[ps[q]].l2 == l2; ++q) {
         const int pi = ps[q];
         const Path& p = P.paths[pi];
@@ -188,6 +199,62 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
           << (K.tangent ? "            wt[v] = ok[v] ? wtr[" + std::to_string(sl.w_st.at(pi)) + " + u] : 0.f;\n" : "")
           << "#pragma unroll\n            for (int m3 = 0; m3 < " << N3 << "; ++m3) gv[v][m3] = ok[v] ? sg["
           << sl.g_st.at(pi) << " + u * " << N3 << " + m3] : 0.f;\n          }\n";
+        if (K.no_chat) {
+          // t[m1][m2] = sum_m3 C[m1][m2][m3] g[m3] (CG coefficients as
+          // immediates), one row m1 at a time; from it s[m1] = sum_m2 Y t,
+          // dW = sum x s, msg += w s and the dY partial z[m2] += (w x)[m1] t
+          const double* C = P.coeff.data() + p.c_off;
+          o << "#pragma unroll\n          for (int v = 0; v < " << RU << "; ++v) {\n"
+            << "            float d = 0.f;\n";
+          for (int m1 = 0; m1 < N1; ++m1) {
+            std::vector<int> m2s;
+            o << "            {\n";
+            for (int m2 = 0; m2 < n2; ++m2) {
+              std::vector<std::pair<int, double>> t;
+              for (int m3 = 0; m3 < N3; ++m3) {
+                const double c = C[((size_t)m1 * n2 + m2) * N3 + m3];
+                if (c != 0.0) t.push_back({m3, c});
+              }
+              if (t.empty()) continue;
+              m2s.push_back(m2);
+              o << "              const float t" << m2 << " = ";
+              std::string e = flt(t[0].second) + " * gv[v][" + std::to_string(t[0].first) + "]";
+              for (size_t k = 1; k < t.size(); ++k)
+                e = "fmaf(" + flt(t[k].second) + ", gv[v][" + std::to_string(t[k].first) + "], " + e + ")";
+              o << e << ";\n";
+            }
+            if (m2s.empty()) {
+              o << "            }\n";
+              continue;
+            }
+            auto dot = [&](const char* y) {
+              std::string e = std::string(y) + "[" + std::to_string(m2s[0]) + "] * t" + std::to_string(m2s[0]);
+              for (size_t k = 1; k < m2s.size(); ++k)
+                e = "fmaf(" + std::string(y) + "[" + std::to_string(m2s[k]) + "], t" + std::to_string(m2s[k]) + ", " +
+                    e + ")";
+              return e;
+            };
+            o << "              const float s = " << dot("yl") << ";\n";
+            if (K.tangent) {
+              o << "              const float st = " << dot("ytl") << ";\n"
+                << "              d = fmaf(xtv[v][" << m1 << "], s, fmaf(xv[v][" << m1 << "], st, d));\n"
+                << "              mx[v][" << m1 << "] = fmaf(wt[v], s, fmaf(w[v], st, mx[v][" << m1 << "]));\n"
+                << "              const float wx = fmaf(w[v], xtv[v][" << m1 << "], wt[v] * xv[v][" << m1 << "]);\n";
+            } else {
+              o << "              d = fmaf(xv[v][" << m1 << "], s, d);\n"
+                << "              mx[v][" << m1 << "] = fmaf(w[v], s, mx[v][" << m1 << "]);\n"
+                << "              const float wx = w[v] * xv[v][" << m1 << "];\n";
+            }
+            for (int m2 : m2s)
+              o << "              z[" << zo + m2 << "] = fmaf(wx, t" << m2 << ", z[" << zo + m2 << "]);\n";
+            o << "            }\n";
+          }
+          o << "            dw[v] = d;\n          }\n";
+          o << "          if (dWrow) {\n#pragma unroll\n            for (int v = 0; v < " << RU
+            << "; ++v) if (ok[v]) dWrow[" << p.k0 << " + u0 + (r + v) * 32 + lane] = dw[v];\n          }\n"
+            << "        }\n";
+          continue;
+        }
         if (K.tangent)
           o << "          bpath_tan<" << N1 << "," << N3 << "," << RU << ">(chb + " << sl.ch_off.at(pi) << ", chtb + "
             << sl.ch_off.at(pi) << ", xv, xtv, w, wt, gv, mx, dw);\n";
@@ -562,6 +629,7 @@ cgtp_status build_backward(Plan& P) {
         K.S = ns;
         K.nw = NW;
         K.force_B = B;
+        K.no_chat = P.bwd_tform;
         int maxr = 0;
         for (int s2 = 0; s2 < ns; ++s2) {
           for (size_t k = 0; k < slices[s2].size(); ++k) {
@@ -611,6 +679,7 @@ cgtp_status build_backward(Plan& P) {
   K.S = F.S;
   K.nw = F.nw;
   K.force_B = best.B;
+  K.no_chat = P.bwd_tform;
   for (int s2 = 0; s2 < F.S; ++s2) {
     for (size_t k = 0; k < best.slices[s2].size(); ++k) {
       const BwdIrrep& wi = best.W[best.slices[s2][k]];
@@ -730,6 +799,7 @@ cgtp_status build_backward_tangent(Plan& P, JitKernel& out, std::string* src_out
   K.S = F.S;
   K.nw = F.nw;
   K.tangent = true;
+  K.no_chat = P.bwd_tform;
   for (int s2 = 0; s2 < F.S; ++s2) {
     for (int ri : F.slice_roles[s2]) {
       const BwdRole& r = P.bwd_roles[ri];

@@ -127,7 +127,7 @@ void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape&
   for (const auto& sl : SL) {
     K.WS = std::max(K.WS, sl.ws);
     K.XS = std::max(K.XS, sl.xs);
-    K.CHS = std::max(K.CHS, sl.chs);
+    if (!K.no_chat) K.CHS = std::max(K.CHS, sl.chs);
     K.GS = std::max(K.GS, sl.gs);
     K.w_bulk = K.w_bulk && segments_aligned(sl.wseg, P.U);
     K.x_bulk = K.x_bulk && segments_aligned(sl.xseg, P.D_in);
@@ -496,7 +496,7 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
        "  (void)srec; (void)nrec;\n";
   const int KR = (K.rec_max + 31) / 32;
   const bool rec_regs = KR <= 12;
-  if (rec_regs)  // the slice's records stay in registers: no loads in the Chat loop
+  if (rec_regs && !K.no_chat)  // the slice's records stay in registers: no loads in the Chat loop
     o << "  int rd[" << KR << "];\n  float rc0[" << KR << "], rc1[" << KR << "];\n"
       << "  const int nk = (nrec - lane + 31) >> 5;\n"
       << "#pragma unroll\n  for (int k = 0; k < " << KR << "; ++k) {\n"
@@ -532,8 +532,10 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
        "      float* sYt = reinterpret_cast<float*>(st + OFF_YT);\n"
        "      float* cht = reinterpret_cast<float*>(st + OFF_CHT);\n"
        "      (void)sYt; (void)cht;\n"
-       "      if (fresh)  // Chat elements without a CG term are zero for this slice\n"
-       "        for (int t = lane; t < (TAN ? 2 : 1) * NB * CHS; t += 32) ch[t] = 0.f;\n"
+    << (K.no_chat ? "      (void)fresh; (void)ch;\n"
+                  : "      if (fresh)  // Chat elements without a CG term are zero for this slice\n"
+                    "        for (int t = lane; t < (TAN ? 2 : 1) * NB * CHS; t += 32) ch[t] = 0.f;\n")
+    <<
        "#pragma unroll\n"
        "      for (int k = 0; k < YPL; ++k) { const int t = lane + 32 * k; if (t < nb * DE) sY[t] = yv[k]; }\n"
        "#if TAN\n"
@@ -543,7 +545,9 @@ std::string gen_common_device(const Plan& P, const std::vector<SliceLayout>& SL,
        "      if (lane == 0) desc[s] = make_int4(eb, nb, slice, 0);\n"
        "      __syncwarp();\n"
        "";
-  if (rec_regs)
+  if (K.no_chat)
+    ;  // the consumers contract with the CG table and Y directly
+  else if (rec_regs)
     o << "#pragma unroll\n"
          "      for (int k = 0; k < " << KR << "; ++k) {\n"
          "        if (k < nk) {\n"

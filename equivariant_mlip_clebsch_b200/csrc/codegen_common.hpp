@@ -79,6 +79,9 @@ struct KernelShape {
   bool tangent = false;
   // W rows prefetched into L2 this many chunks ahead (0: off)
   int prefetch = 0;
+  // backward roles that contract with the CG table and Y directly: no Chat
+  // is staged or built (CGTP_BWD_TFORM)
+  bool no_chat = false;
   int off_wb = 0;
 };
 

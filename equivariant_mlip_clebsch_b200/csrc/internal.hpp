@@ -160,6 +160,9 @@ struct Plan {
   std::vector<int> bwd_ent_begin;
   std::vector<int> bwd_chs;
   bool bwd_irrep_gap = false;  // some hidden irrep has no path
+  // backward roles contract with the CG table and Y directly instead of a
+  // staged Chat (tuning override CGTP_BWD_TFORM=1 at plan creation)
+  bool bwd_tform = false;
 
   // tangent kernels of the double backward, built on first use (tan_state:
   // 0 not built, 1 ready, -1 unavailable: the composition is used)
