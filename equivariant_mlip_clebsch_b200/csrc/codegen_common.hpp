@@ -80,7 +80,7 @@ struct KernelShape {
   // W rows prefetched into L2 this many chunks ahead (0: off)
   int prefetch = 0;
   // backward roles that contract with the CG table and Y directly: no Chat
-  // is staged or built (CGTP_BWD_TFORM)
+  // is staged or built (the default; CGTP_BWD_TFORM=0 turns it off)
   bool no_chat = false;
   int off_wb = 0;
 };

@@ -160,9 +160,10 @@ struct Plan {
   std::vector<int> bwd_ent_begin;
   std::vector<int> bwd_chs;
   bool bwd_irrep_gap = false;  // some hidden irrep has no path
-  // backward roles contract with the CG table and Y directly instead of a
-  // staged Chat (tuning override CGTP_BWD_TFORM=1 at plan creation)
-  bool bwd_tform = false;
+  // backward roles contract grad_out with the CG table first and then with
+  // Y, so no Chat is staged; CGTP_BWD_TFORM=0 at plan creation selects the
+  // staged-Chat form instead (kept for comparison)
+  bool bwd_tform = true;
 
   // tangent kernels of the double backward, built on first use (tan_state:
   // 0 not built, 1 ready, -1 unavailable: the composition is used)

@@ -135,6 +135,23 @@ def test_backward(name, dev):
         assert_close(dx[send_s], rdx[send_s], f"{name} dx (128 sampled senders)")
 
 
+@pytest.mark.parametrize("name", ["tiny", "lmax2"])
+def test_backward_staged_chat(name, dev, monkeypatch):
+    """The staged-Chat form of the backward (CGTP_BWD_TFORM=0), kept beside
+    the default for comparison, against the oracle."""
+    c = case(name, dev)
+    w = c.w
+    monkeypatch.setenv("CGTP_BWD_TFORM", "0")
+    cfg = w.cfg
+    plan = C().Plan(cfg["irreps_in"], cfg["irreps_edge"], cfg["irreps_out"], 6)
+    assert "backward form=staged_chat" in plan.describe()
+    grads = plan.backward(c.rowptr, c.col, c.rpt, c.perm, c.x, c.Y, c.W, c.g)
+    plan.check_device_error()
+    refs = O.backward(w.P, w.rowptr, w.col, w.N, w.x, c.Y_ref, w.W, w.g)
+    for k, a, b in zip("xWY", grads, refs):
+        assert_close(a.cpu().numpy(), b, f"{name} d{k} (staged Chat)")
+
+
 @pytest.mark.parametrize("name", ALL)
 def test_force_chain(name, dev):
     """grad_r = dL/dr through the harmonics, and the per-atom forces from it."""
