@@ -61,6 +61,222 @@ std::string flt(double v) {
   return b;
 }
 
+// One consumer role of the CG-first backward (no staged Chat).  Per path and
+// channel, with g = grad_out of the receiver:
+//   t[m1][m2] = sum_m3 C[m1][m2][m3] g[m3]      (CG coefficients as immediates)
+//   s[m1]     = sum_m2 Y[m2] t[m1][m2]           (= sum_m3 Chat[m3][m1] g[m3])
+//   dW += x[m1] s[m1],  msg[m1] += w s[m1],  dY[m2] += w x[m1] t[m1][m2].
+// t depends on the receiver only, so a pass takes NE edges of the receiver
+// (b, b + nph, ...) and computes t once for all of them; an edge past the
+// chunk's end is skipped.
+void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K, const BwdRole& r,
+                           const SliceLayout& sl, size_t k, const std::string& params) {
+  const Irrep& h = P.in[r.irrep];
+  const int N1 = 2 * h.l + 1, R = r.R, MUL = h.mul;
+  const int NE = K.tangent ? 1 : K.pair;
+  const bool tan = K.tangent;
+  auto pow2 = [](int n) { int v = 1; while (v < n) v <<= 1; return v; };
+  const bool combined = P.D_e <= 32;
+  if (!combined && R != 1) {
+    std::fprintf(stderr, "cgtp: backward role with R > 1 needs D_e <= 32\n");
+    std::abort();
+  }
+  const int VZ = (int)P.D_e;
+  std::vector<int> ps;
+  for (size_t q = 0; q < P.paths.size(); ++q)
+    if (P.paths[q].irrep == r.irrep) ps.push_back((int)q);
+  const std::string sNE = std::to_string(NE), sN1 = std::to_string(N1);
+  o << "// shape " << k << ": irrep " << r.irrep << " (" << h.mul << "x" << h.l << "), R=" << R << ", " << ps.size()
+    << " paths, CG first, " << NE << " edge(s) per pass\n"
+    << "__device__ __noinline__ void bcons_" << k << params << " {\n"
+    << "  const int lane = threadIdx.x & 31;\n"
+    << "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
+    << "  const u32 gfull0 = full0 + OFF_GFULL, gempty0 = full0 + OFF_GEMPTY;\n"
+    << "  (void)chs;\n"
+    << "  int q = *qp, kr = *kp;\n"
+    << "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
+    << "  const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
+    << "  if (e1 <= e0) continue;\n"
+    << "  const int gb = kr % GBUF;\n"
+    << "  if (!mbar_wait(gfull0 + 8 * gb, (kr / GBUF) & 1)) { if (lane == 0) atomicOr(err, 10); *qp = -1; return; }\n"
+    << "  const float* sg = reinterpret_cast<const float*>(smem + OFF_G) + gb * GS;\n"
+    << "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
+    << "    const int s = q % NSTAGE;\n"
+    << "    if (!stage_ready(full0, s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); *qp = -1; return; }\n"
+    << "    const int nb = min(NB, e1 - eb);\n"
+    << "    unsigned char* st = stage_ptr(smem, s);\n"
+    << "    float* sdyw = reinterpret_cast<float*>(st + OFF_DY) + (threadIdx.x >> 5) * NB * DE;\n"
+    << "#pragma unroll 1\n    for (int b = ph; b < nb; b += " << NE << " * nph) {\n"
+    << "      int bj[" << NE << "];\n      bool vj[" << NE << "];\n"
+    << "      const float* wr[" << NE << "];\n      const float* xr[" << NE << "];\n      const float* yr[" << NE
+    << "];\n"
+    << (tan ? "      const float* wtr[1];\n      const float* xtr[1];\n      const float* ytr[1];\n" : "")
+    << "      float* dWrow[" << NE << "];\n      float* sdy[" << NE << "];\n"
+    << "#pragma unroll\n      for (int j = 0; j < " << NE << "; ++j) {\n"
+    << "        bj[j] = b + j * nph;\n"
+    << "        vj[j] = bj[j] < nb;\n"
+    << "        if (!vj[j]) bj[j] = b;  // past the chunk: rows of the first edge, results dropped\n"
+    << "        wr[j] = reinterpret_cast<const float*>(st + OFF_W) + bj[j] * WS;\n"
+    << "        xr[j] = reinterpret_cast<const float*>(st + OFF_X) + " << sl.x_st.at(r.irrep) << " + bj[j] * XS;\n"
+    << "        yr[j] = reinterpret_cast<const float*>(st + OFF_Y) + bj[j] * DE;\n"
+    << (tan ? "        wtr[j] = reinterpret_cast<const float*>(st + OFF_WT) + bj[j] * WS;\n"
+              "        xtr[j] = reinterpret_cast<const float*>(st + OFF_XT) + " +
+                  std::to_string(sl.x_st.at(r.irrep)) +
+                  " + bj[j] * XS;\n"
+                  "        ytr[j] = reinterpret_cast<const float*>(st + OFF_YT) + bj[j] * DE;\n"
+            : "")
+    << "        const int e = eb + bj[j];\n"
+    << "        dWrow[j] = (dW && vj[j]) ? dW + (size_t)(eid ? __ldg(eid + e) : e) * NU : nullptr;\n"
+    << "        sdy[j] = (want_dy && vj[j]) ? sdyw + bj[j] * DE : nullptr;\n"
+    << "      }\n";
+  if (combined)
+    o << "      float z[" << NE << "][" << VZ << "];\n#pragma unroll\n      for (int j = 0; j < " << NE
+      << "; ++j)\n#pragma unroll\n        for (int t = 0; t < " << VZ << "; ++t) z[j][t] = 0.f;\n";
+  o << "#pragma unroll 1\n      for (int r = 0; r < " << R << "; ++r) {\n"
+    << "      const int u = u0 + r * 32 + lane;\n"
+    << "      const bool ok = " << (MUL % (32 * R) == 0 ? std::string("true") : "u < " + std::to_string(MUL))
+    << ";  // every lane holds a channel when the blocks are full\n"
+    << "      float xv[" << NE << "][" << N1 << "], mx[" << NE << "][" << N1 << "];\n"
+    << (tan ? "      float xtv[1][" + sN1 + "];\n" : "")
+    << "#pragma unroll\n      for (int j = 0; j < " << NE << "; ++j)\n"
+    << "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) {\n"
+    << "          mx[j][m1] = 0.f;\n"
+    << "          xv[j][m1] = ok ? xr[j][u * " << N1 << " + m1] : 0.f;\n"
+    << (tan ? "          xtv[j][m1] = ok ? xtr[j][u * " + sN1 + " + m1] : 0.f;\n" : "")
+    << "        }\n";
+  std::vector<char> l2seen(P.L + 1, 0);
+  size_t q = 0;
+  while (q < ps.size()) {
+    const int l2 = P.paths[ps[q]].l2;
+    const int N2 = 2 * l2 + 1;
+    const int zo = combined ? l2 * l2 : 0;  // offset of degree l2 inside z
+    l2seen[l2] = 1;
+    o << "      {\n";
+    if (!combined)
+      o << "        float z[" << NE << "][" << pow2(N2) << "];\n#pragma unroll\n        for (int j = 0; j < " << NE
+        << "; ++j)\n#pragma unroll\n          for (int t = 0; t < " << pow2(N2) << "; ++t) z[j][t] = 0.f;\n";
+    // this degree's harmonics of the edges (the same for every lane)
+    o << "        float yl[" << NE << "][" << N2 << "];\n#pragma unroll\n        for (int j = 0; j < " << NE
+      << "; ++j)\n#pragma unroll\n          for (int m2 = 0; m2 < " << N2 << "; ++m2) yl[j][m2] = yr[j][" << l2 * l2
+      << " + m2];\n";
+    if (tan)
+      o << "        float ytl[1][" << N2 << "];\n#pragma unroll\n        for (int m2 = 0; m2 < " << N2
+        << "; ++m2) ytl[0][m2] = ytr[0][" << l2 * l2 << " + m2];\n";
+    for (; q < ps.size() && P.paths[ps[q]].l2 == l2; ++q) {
+      const int pi = ps[q];
+      const Path& p = P.paths[pi];
+      const int N3 = 2 * p.l3 + 1, n2 = 2 * p.l2 + 1;
+      o << "        {\n          float w[" << NE << "], gv[" << N3 << "], d[" << NE << "];\n"
+        << (tan ? "          float wt[1];\n" : "")
+        << "#pragma unroll\n          for (int m3 = 0; m3 < " << N3 << "; ++m3) gv[m3] = ok ? sg[" << sl.g_st.at(pi)
+        << " + u * " << N3 << " + m3] : 0.f;\n"
+        << "#pragma unroll\n          for (int j = 0; j < " << NE << "; ++j) {\n"
+        << "            w[j] = ok ? wr[j][" << sl.w_st.at(pi) << " + u] : 0.f;\n"
+        << (tan ? "            wt[j] = ok ? wtr[j][" + std::to_string(sl.w_st.at(pi)) + " + u] : 0.f;\n" : "")
+        << "            d[j] = 0.f;\n          }\n";
+      const double* C = P.coeff.data() + p.c_off;
+      for (int m1 = 0; m1 < N1; ++m1) {
+        std::vector<int> m2s;
+        std::ostringstream tdef;
+        for (int m2 = 0; m2 < n2; ++m2) {
+          std::vector<std::pair<int, double>> t;
+          for (int m3 = 0; m3 < N3; ++m3) {
+            const double c = C[((size_t)m1 * n2 + m2) * N3 + m3];
+            if (c != 0.0) t.push_back({m3, c});
+          }
+          if (t.empty()) continue;
+          m2s.push_back(m2);
+          std::string e = flt(t[0].second) + " * gv[" + std::to_string(t[0].first) + "]";
+          for (size_t c = 1; c < t.size(); ++c)
+            e = "fmaf(" + flt(t[c].second) + ", gv[" + std::to_string(t[c].first) + "], " + e + ")";
+          tdef << "            const float t" << m2 << " = " << e << ";\n";
+        }
+        if (m2s.empty()) continue;
+        o << "          {\n" << tdef.str();
+        for (int j = 0; j < NE; ++j) {
+          const std::string J = std::to_string(j);
+          auto dot = [&](const std::string& y) {
+            std::string e = y + "[" + J + "][" + std::to_string(m2s[0]) + "] * t" + std::to_string(m2s[0]);
+            for (size_t c = 1; c < m2s.size(); ++c)
+              e = "fmaf(" + y + "[" + J + "][" + std::to_string(m2s[c]) + "], t" + std::to_string(m2s[c]) + ", " +
+                  e + ")";
+            return e;
+          };
+          const std::string xm = "xv[" + J + "][" + std::to_string(m1) + "]";
+          const std::string mm = "mx[" + J + "][" + std::to_string(m1) + "]";
+          o << (j == 0 ? "            {\n" : "            if (vj[" + J + "]) {\n")
+            << "              const float s = " << dot("yl") << ";\n";
+          if (tan) {
+            const std::string xt = "xtv[0][" + std::to_string(m1) + "]";
+            o << "              const float st = " << dot("ytl") << ";\n"
+              << "              d[0] = fmaf(" << xt << ", s, fmaf(" << xm << ", st, d[0]));\n"
+              << "              " << mm << " = fmaf(wt[0], s, fmaf(w[0], st, " << mm << "));\n"
+              << "              const float wx = fmaf(w[0], " << xt << ", wt[0] * " << xm << ");\n";
+          } else {
+            o << "              d[" << J << "] = fmaf(" << xm << ", s, d[" << J << "]);\n"
+              << "              " << mm << " = fmaf(w[" << J << "], s, " << mm << ");\n"
+              << "              const float wx = w[" << J << "] * " << xm << ";\n";
+          }
+          for (int m2 : m2s)
+            o << "              z[" << J << "][" << zo + m2 << "] = fmaf(wx, t" << m2 << ", z[" << J << "]["
+              << zo + m2 << "]);\n";
+          o << "            }\n";
+        }
+        o << "          }\n";
+      }
+      o << "#pragma unroll\n          for (int j = 0; j < " << NE << "; ++j)\n"
+        << "            if (dWrow[j] && ok) dWrow[j][" << p.k0 << " + u] = d[j];\n"
+        << "        }\n";
+    }
+    if (!combined) {
+      const int V = pow2(N2), LV = __builtin_ctz(V), sh = 5 - LV;
+      o << "#pragma unroll\n        for (int j = 0; j < " << NE << "; ++j)\n"
+        << "          if (sdy[j]) {\n            const float v = warp_sum_many<" << V << ">(z[j], lane);\n"
+        << "            const int c = lane >> " << sh << ";\n"
+        << "            if ((lane & " << ((1 << sh) - 1) << ") == 0 && c < " << N2 << ") sdy[j][" << l2 * l2
+        << " + c] = v;\n          }\n";
+    }
+    o << "      }\n";
+  }
+  // the message rows of this channel block, through the warp's buffer
+  o << "      if (msg) {\n"
+    << "        float* wbuf = reinterpret_cast<float*>(smem + OFF_WB) + (threadIdx.x >> 5) * WB;\n"
+    << "        const int nch = min(32, " << MUL << " - u0 - r * 32);\n"
+    << "#pragma unroll\n        for (int j = 0; j < " << NE << "; ++j) {\n"
+    << "          if (!vj[j]) continue;\n"
+    << "#pragma unroll\n          for (int m1 = 0; m1 < " << N1 << "; ++m1) wbuf[lane * " << N1
+    << " + m1] = mx[j][m1];\n"
+    << "          __syncwarp();\n"
+    << "          if (nch > 0) warp_copy_out(msg + (size_t)(eb + bj[j]) * DIN + " << P.x_off[r.irrep]
+    << " + (u0 + r * 32) * " << N1 << ", wbuf, nch * " << N1 << ", lane);\n"
+    << "          __syncwarp();\n        }\n      }\n"
+    << "      }\n";  // r
+  if (combined) {
+    o << "#pragma unroll\n      for (int j = 0; j < " << NE << "; ++j)\n      if (sdy[j]) {\n";
+    for (int off = 0, rest = VZ; rest > 0;) {
+      int V = 1;
+      while (V * 2 <= rest && V * 2 <= 32) V *= 2;
+      const int LV = __builtin_ctz(V), sh = 5 - LV;
+      o << "        {\n          float zp[" << V << "];\n#pragma unroll\n          for (int t = 0; t < " << V
+        << "; ++t) zp[t] = z[j][" << off << " + t];\n"
+        << "          const float v = warp_sum_many<" << V << ">(zp, lane);\n"
+        << "          if ((lane & " << ((1 << sh) - 1) << ") == 0) sdy[j][" << off << " + (lane >> " << sh
+        << ")] = v;\n        }\n";
+      off += V;
+      rest -= V;
+    }
+    o << "      }\n";
+  } else {
+    for (int l2 = 0; l2 <= P.L; ++l2)
+      if (!l2seen[l2])
+        o << "#pragma unroll\n      for (int j = 0; j < " << NE << "; ++j)\n"
+          << "        if (sdy[j] && lane == 0) {\n#pragma unroll\n          for (int t = 0; t < " << 2 * l2 + 1
+          << "; ++t) sdy[j][" << l2 * l2 << " + t] = 0.f;\n        }\n";
+  }
+  o << "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n"
+    << "  __syncwarp();\n  if (lane == 0) mbar_arrive(gempty0 + 8 * gb);\n  ++kr;\n  }\n  *qp = q;\n  *kp = kr;\n}\n";
+}
+
 }  // namespace
 
 static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>& SL, const KernelShape& K,
@@ -96,6 +312,10 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
   for (size_t k = 0; k < shape_rep.size(); ++k) {
     const BwdRole& r = P.bwd_roles[shape_rep[k]];
     const SliceLayout& sl = SL[slice_of[shape_rep[k]]];
+    if (K.no_chat) {
+      gen_bwd_role_cg_first(o, P, K, r, sl, k, params);
+      continue;
+    }
     const Irrep& h = P.in[r.irrep];
     const int N1 = 2 * h.l + 1, R = r.R, MUL = h.mul;
     std::vector<int> ps;
@@ -134,10 +354,6 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
                       "      const float* xtr = reinterpret_cast<const float*>(st + OFF_XT) + " +
                           std::to_string(sl.x_st.at(r.irrep)) + " + b * XS;\n"
                     : "")
-      << (K.no_chat ? std::string("      const float* yr = reinterpret_cast<const float*>(st + OFF_Y) + b * DE;\n") +
-                          (K.tangent ? "      const float* ytr = reinterpret_cast<const float*>(st + OFF_YT) + b * DE;\n"
-                                     : "")
-                    : std::string())
       << "      float* dWrow = dW ? dW + (size_t)(eid ? __ldg(eid + e) : e) * NU : nullptr;\n"
       << "      float* sdy = want_dy ? sdyw + b * DE : nullptr;\n"
       ;
@@ -180,13 +396,6 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
       if (!combined)
         o << "        float z[" << pow2(N2) << "];\n#pragma unroll\n        for (int t = 0; t < " << pow2(N2)
           << "; ++t) z[t] = 0.f;\n";
-      if (K.no_chat) {  // this degree's harmonics of the edge (the same for every lane)
-        o << "        float yl[" << N2 << "];\n#pragma unroll\n        for (int m2 = 0; m2 < " << N2
-          << "; ++m2) yl[m2] = yr[" << l2 * l2 << " + m2];\n";
-        if (K.tangent)
-          o << "        float ytl[" << N2 << "];\n#pragma unroll\n        for (int m2 = 0; m2 < " << N2
-            << "; ++m2) ytl[m2] = ytr[" << l2 * l2 << " + m2];\n";
-      }
       for (; q < ps.size() && P.paths[ps[q]].l2 == l2; ++q) {
         const int pi = ps[q];
         const Path& p = P.paths[pi];
@@ -199,62 +408,6 @@ static std::string gen_bwd_source(const Plan& P, const std::vector<SliceLayout>&
           << (K.tangent ? "            wt[v] = ok[v] ? wtr[" + std::to_string(sl.w_st.at(pi)) + " + u] : 0.f;\n" : "")
           << "#pragma unroll\n            for (int m3 = 0; m3 < " << N3 << "; ++m3) gv[v][m3] = ok[v] ? sg["
           << sl.g_st.at(pi) << " + u * " << N3 << " + m3] : 0.f;\n          }\n";
-        if (K.no_chat) {
-          // t[m1][m2] = sum_m3 C[m1][m2][m3] g[m3] (CG coefficients as
-          // immediates), one row m1 at a time; from it s[m1] = sum_m2 Y t,
-          // dW = sum x s, msg += w s and the dY partial z[m2] += (w x)[m1] t
-          const double* C = P.coeff.data() + p.c_off;
-          o << "#pragma unroll\n          for (int v = 0; v < " << RU << "; ++v) {\n"
-            << "            float d = 0.f;\n";
-          for (int m1 = 0; m1 < N1; ++m1) {
-            std::vector<int> m2s;
-            o << "            {\n";
-            for (int m2 = 0; m2 < n2; ++m2) {
-              std::vector<std::pair<int, double>> t;
-              for (int m3 = 0; m3 < N3; ++m3) {
-                const double c = C[((size_t)m1 * n2 + m2) * N3 + m3];
-                if (c != 0.0) t.push_back({m3, c});
-              }
-              if (t.empty()) continue;
-              m2s.push_back(m2);
-              o << "              const float t" << m2 << " = ";
-              std::string e = flt(t[0].second) + " * gv[v][" + std::to_string(t[0].first) + "]";
-              for (size_t k = 1; k < t.size(); ++k)
-                e = "fmaf(" + flt(t[k].second) + ", gv[v][" + std::to_string(t[k].first) + "], " + e + ")";
-              o << e << ";\n";
-            }
-            if (m2s.empty()) {
-              o << "            }\n";
-              continue;
-            }
-            auto dot = [&](const char* y) {
-              std::string e = std::string(y) + "[" + std::to_string(m2s[0]) + "] * t" + std::to_string(m2s[0]);
-              for (size_t k = 1; k < m2s.size(); ++k)
-                e = "fmaf(" + std::string(y) + "[" + std::to_string(m2s[k]) + "], t" + std::to_string(m2s[k]) + ", " +
-                    e + ")";
-              return e;
-            };
-            o << "              const float s = " << dot("yl") << ";\n";
-            if (K.tangent) {
-              o << "              const float st = " << dot("ytl") << ";\n"
-                << "              d = fmaf(xtv[v][" << m1 << "], s, fmaf(xv[v][" << m1 << "], st, d));\n"
-                << "              mx[v][" << m1 << "] = fmaf(wt[v], s, fmaf(w[v], st, mx[v][" << m1 << "]));\n"
-                << "              const float wx = fmaf(w[v], xtv[v][" << m1 << "], wt[v] * xv[v][" << m1 << "]);\n";
-            } else {
-              o << "              d = fmaf(xv[v][" << m1 << "], s, d);\n"
-                << "              mx[v][" << m1 << "] = fmaf(w[v], s, mx[v][" << m1 << "]);\n"
-                << "              const float wx = w[v] * xv[v][" << m1 << "];\n";
-            }
-            for (int m2 : m2s)
-              o << "              z[" << zo + m2 << "] = fmaf(wx, t" << m2 << ", z[" << zo + m2 << "]);\n";
-            o << "            }\n";
-          }
-          o << "            dw[v] = d;\n          }\n";
-          o << "          if (dWrow) {\n#pragma unroll\n            for (int v = 0; v < " << RU
-            << "; ++v) if (ok[v]) dWrow[" << p.k0 << " + u0 + (r + v) * 32 + lane] = dw[v];\n          }\n"
-            << "        }\n";
-          continue;
-        }
         if (K.tangent)
           o << "          bpath_tan<" << N1 << "," << N3 << "," << RU << ">(chb + " << sl.ch_off.at(pi) << ", chtb + "
             << sl.ch_off.at(pi) << ", xv, xtv, w, wt, gv, mx, dw);\n";
@@ -630,6 +783,7 @@ cgtp_status build_backward(Plan& P) {
         K.nw = NW;
         K.force_B = B;
         K.no_chat = P.bwd_tform;
+  K.pair = P.bwd_pair;
         int maxr = 0;
         for (int s2 = 0; s2 < ns; ++s2) {
           for (size_t k = 0; k < slices[s2].size(); ++k) {
@@ -680,6 +834,7 @@ cgtp_status build_backward(Plan& P) {
   K.nw = F.nw;
   K.force_B = best.B;
   K.no_chat = P.bwd_tform;
+  K.pair = P.bwd_pair;
   for (int s2 = 0; s2 < F.S; ++s2) {
     for (size_t k = 0; k < best.slices[s2].size(); ++k) {
       const BwdIrrep& wi = best.W[best.slices[s2][k]];
@@ -800,7 +955,7 @@ cgtp_status build_backward_tangent(Plan& P, JitKernel& out, std::string* src_out
   K.nw = F.nw;
   K.tangent = true;
   K.no_chat = P.bwd_tform;
-  for (int s2 = 0; s2 < F.S; ++s2) {
+    for (int s2 = 0; s2 < F.S; ++s2) {
     for (int ri : F.slice_roles[s2]) {
       const BwdRole& r = P.bwd_roles[ri];
       auto& irr = SL[s2].irreps;
