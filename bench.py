@@ -517,6 +517,11 @@ def run_cgtp(args, rank, world, local_rank):
         dbl()
         torch.cuda.synchronize()
         dbl_ms = wb.timer(dbl, args.steps)
+        plan.kernel_times()  # discard
+        plan.set_timing(True)
+        wb.timer(dbl, args.steps)
+        plan.set_timing(False)
+        dbl_kernels = {nm: {"avg_ms": ms / max(n, 1), "launches": n} for nm, (ms, n) in plan.kernel_times().items()}
         # the operation's own bytes: x, Y, W, grad_out and the three cotangents
         # read once, the four gradients written once, both CSRs read
         dbl_bytes = 4 * (2 * N * plan.d_in + 2 * E * plan.d_edge + 2 * E * plan.n_weights + N * plan.d_out
@@ -527,7 +532,8 @@ def run_cgtp(args, rank, world, local_rank):
                            "vs_step": dbl_ms / ms_step_local,
                            "path": "tangent kernels (one forward, one backward pass)" if tangent else
                                    "composition of forwards and backwards",
-                           "what": "double_backward with h_x, h_W, h_Y, after the step (not in it)"}
+                           "what": "double_backward with h_x, h_W, h_Y, after the step (not in it)",
+                           "kernels": dbl_kernels}
         del hx, hW, hY, dgrads, dws
     except (C.CgtpError, ValueError, TypeError) as e:  # reported, the headline stands
         double_backward = {"error": str(e)}

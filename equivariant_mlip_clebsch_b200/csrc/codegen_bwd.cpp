@@ -66,14 +66,13 @@ std::string flt(double v) {
 //   t[m1][m2] = sum_m3 C[m1][m2][m3] g[m3]      (CG coefficients as immediates)
 //   s[m1]     = sum_m2 Y[m2] t[m1][m2]           (= sum_m3 Chat[m3][m1] g[m3])
 //   dW += x[m1] s[m1],  msg[m1] += w s[m1],  dY[m2] += w x[m1] t[m1][m2].
-// t depends on the receiver only, so a pass takes NE edges of the receiver
-// (b, b + nph, ...) and computes t once for all of them; an edge past the
-// chunk's end is skipped.
+// The tangent form (double backward) adds the directional derivatives along
+// (xt, Yt, wt): st = sum_m2 Yt t, dW += xt s + x st, msg += wt s + w st and
+// dY += (w xt + wt x) t.
 void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K, const BwdRole& r,
                            const SliceLayout& sl, size_t k, const std::string& params) {
   const Irrep& h = P.in[r.irrep];
   const int N1 = 2 * h.l + 1, R = r.R, MUL = h.mul;
-  const int NE = K.tangent ? 1 : K.pair;
   const bool tan = K.tangent;
   auto pow2 = [](int n) { int v = 1; while (v < n) v <<= 1; return v; };
   const bool combined = P.D_e <= 32;
@@ -85,9 +84,9 @@ void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K,
   std::vector<int> ps;
   for (size_t q = 0; q < P.paths.size(); ++q)
     if (P.paths[q].irrep == r.irrep) ps.push_back((int)q);
-  const std::string sNE = std::to_string(NE), sN1 = std::to_string(N1);
+  const std::string sN1 = std::to_string(N1);
   o << "// shape " << k << ": irrep " << r.irrep << " (" << h.mul << "x" << h.l << "), R=" << R << ", " << ps.size()
-    << " paths, CG first, " << NE << " edge(s) per pass\n"
+    << " paths, CG first\n"
     << "__device__ __noinline__ void bcons_" << k << params << " {\n"
     << "  const int lane = threadIdx.x & 31;\n"
     << "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
@@ -106,44 +105,32 @@ void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K,
     << "    const int nb = min(NB, e1 - eb);\n"
     << "    unsigned char* st = stage_ptr(smem, s);\n"
     << "    float* sdyw = reinterpret_cast<float*>(st + OFF_DY) + (threadIdx.x >> 5) * NB * DE;\n"
-    << "#pragma unroll 1\n    for (int b = ph; b < nb; b += " << NE << " * nph) {\n"
-    << "      int bj[" << NE << "];\n      bool vj[" << NE << "];\n"
-    << "      const float* wr[" << NE << "];\n      const float* xr[" << NE << "];\n      const float* yr[" << NE
-    << "];\n"
-    << (tan ? "      const float* wtr[1];\n      const float* xtr[1];\n      const float* ytr[1];\n" : "")
-    << "      float* dWrow[" << NE << "];\n      float* sdy[" << NE << "];\n"
-    << "#pragma unroll\n      for (int j = 0; j < " << NE << "; ++j) {\n"
-    << "        bj[j] = b + j * nph;\n"
-    << "        vj[j] = bj[j] < nb;\n"
-    << "        if (!vj[j]) bj[j] = b;  // past the chunk: rows of the first edge, results dropped\n"
-    << "        wr[j] = reinterpret_cast<const float*>(st + OFF_W) + bj[j] * WS;\n"
-    << "        xr[j] = reinterpret_cast<const float*>(st + OFF_X) + " << sl.x_st.at(r.irrep) << " + bj[j] * XS;\n"
-    << "        yr[j] = reinterpret_cast<const float*>(st + OFF_Y) + bj[j] * DE;\n"
-    << (tan ? "        wtr[j] = reinterpret_cast<const float*>(st + OFF_WT) + bj[j] * WS;\n"
-              "        xtr[j] = reinterpret_cast<const float*>(st + OFF_XT) + " +
+    << "#pragma unroll 1\n    for (int b = ph; b < nb; b += nph) {\n"
+    << "      const int e = eb + b;\n"
+    << "      const float* wr = reinterpret_cast<const float*>(st + OFF_W) + b * WS;\n"
+    << "      const float* xr = reinterpret_cast<const float*>(st + OFF_X) + " << sl.x_st.at(r.irrep) << " + b * XS;\n"
+    << "      const float* yr = reinterpret_cast<const float*>(st + OFF_Y) + b * DE;\n"
+    << (tan ? "      const float* wtr = reinterpret_cast<const float*>(st + OFF_WT) + b * WS;\n"
+              "      const float* xtr = reinterpret_cast<const float*>(st + OFF_XT) + " +
                   std::to_string(sl.x_st.at(r.irrep)) +
-                  " + bj[j] * XS;\n"
-                  "        ytr[j] = reinterpret_cast<const float*>(st + OFF_YT) + bj[j] * DE;\n"
+                  " + b * XS;\n"
+                  "      const float* ytr = reinterpret_cast<const float*>(st + OFF_YT) + b * DE;\n"
             : "")
-    << "        const int e = eb + bj[j];\n"
-    << "        dWrow[j] = (dW && vj[j]) ? dW + (size_t)(eid ? __ldg(eid + e) : e) * NU : nullptr;\n"
-    << "        sdy[j] = (want_dy && vj[j]) ? sdyw + bj[j] * DE : nullptr;\n"
-    << "      }\n";
+    << "      float* dWrow = dW ? dW + (size_t)(eid ? __ldg(eid + e) : e) * NU : nullptr;\n"
+    << "      float* sdy = want_dy ? sdyw + b * DE : nullptr;\n";
   if (combined)
-    o << "      float z[" << NE << "][" << VZ << "];\n#pragma unroll\n      for (int j = 0; j < " << NE
-      << "; ++j)\n#pragma unroll\n        for (int t = 0; t < " << VZ << "; ++t) z[j][t] = 0.f;\n";
+    o << "      float z[" << VZ << "];\n#pragma unroll\n      for (int t = 0; t < " << VZ << "; ++t) z[t] = 0.f;\n";
   o << "#pragma unroll 1\n      for (int r = 0; r < " << R << "; ++r) {\n"
     << "      const int u = u0 + r * 32 + lane;\n"
     << "      const bool ok = " << (MUL % (32 * R) == 0 ? std::string("true") : "u < " + std::to_string(MUL))
     << ";  // every lane holds a channel when the blocks are full\n"
-    << "      float xv[" << NE << "][" << N1 << "], mx[" << NE << "][" << N1 << "];\n"
-    << (tan ? "      float xtv[1][" + sN1 + "];\n" : "")
-    << "#pragma unroll\n      for (int j = 0; j < " << NE << "; ++j)\n"
-    << "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) {\n"
-    << "          mx[j][m1] = 0.f;\n"
-    << "          xv[j][m1] = ok ? xr[j][u * " << N1 << " + m1] : 0.f;\n"
-    << (tan ? "          xtv[j][m1] = ok ? xtr[j][u * " + sN1 + " + m1] : 0.f;\n" : "")
-    << "        }\n";
+    << "      float xv[" << N1 << "], mx[" << N1 << "];\n"
+    << (tan ? "      float xtv[" + sN1 + "];\n" : "")
+    << "#pragma unroll\n      for (int m1 = 0; m1 < " << N1 << "; ++m1) {\n"
+    << "        mx[m1] = 0.f;\n"
+    << "        xv[m1] = ok ? xr[u * " << N1 << " + m1] : 0.f;\n"
+    << (tan ? "        xtv[m1] = ok ? xtr[u * " + sN1 + " + m1] : 0.f;\n" : "")
+    << "      }\n";
   std::vector<char> l2seen(P.L + 1, 0);
   size_t q = 0;
   while (q < ps.size()) {
@@ -153,27 +140,24 @@ void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K,
     l2seen[l2] = 1;
     o << "      {\n";
     if (!combined)
-      o << "        float z[" << NE << "][" << pow2(N2) << "];\n#pragma unroll\n        for (int j = 0; j < " << NE
-        << "; ++j)\n#pragma unroll\n          for (int t = 0; t < " << pow2(N2) << "; ++t) z[j][t] = 0.f;\n";
-    // this degree's harmonics of the edges (the same for every lane)
-    o << "        float yl[" << NE << "][" << N2 << "];\n#pragma unroll\n        for (int j = 0; j < " << NE
-      << "; ++j)\n#pragma unroll\n          for (int m2 = 0; m2 < " << N2 << "; ++m2) yl[j][m2] = yr[j][" << l2 * l2
-      << " + m2];\n";
+      o << "        float z[" << pow2(N2) << "];\n#pragma unroll\n        for (int t = 0; t < " << pow2(N2)
+        << "; ++t) z[t] = 0.f;\n";
+    // this degree's harmonics of the edge (the same for every lane)
+    o << "        float yl[" << N2 << "];\n#pragma unroll\n        for (int m2 = 0; m2 < " << N2
+      << "; ++m2) yl[m2] = yr[" << l2 * l2 << " + m2];\n";
     if (tan)
-      o << "        float ytl[1][" << N2 << "];\n#pragma unroll\n        for (int m2 = 0; m2 < " << N2
-        << "; ++m2) ytl[0][m2] = ytr[0][" << l2 * l2 << " + m2];\n";
+      o << "        float ytl[" << N2 << "];\n#pragma unroll\n        for (int m2 = 0; m2 < " << N2
+        << "; ++m2) ytl[m2] = ytr[" << l2 * l2 << " + m2];\n";
     for (; q < ps.size() && P.paths[ps[q]].l2 == l2; ++q) {
       const int pi = ps[q];
       const Path& p = P.paths[pi];
       const int N3 = 2 * p.l3 + 1, n2 = 2 * p.l2 + 1;
-      o << "        {\n          float w[" << NE << "], gv[" << N3 << "], d[" << NE << "];\n"
-        << (tan ? "          float wt[1];\n" : "")
+      o << "        {\n          float gv[" << N3 << "];\n"
         << "#pragma unroll\n          for (int m3 = 0; m3 < " << N3 << "; ++m3) gv[m3] = ok ? sg[" << sl.g_st.at(pi)
         << " + u * " << N3 << " + m3] : 0.f;\n"
-        << "#pragma unroll\n          for (int j = 0; j < " << NE << "; ++j) {\n"
-        << "            w[j] = ok ? wr[j][" << sl.w_st.at(pi) << " + u] : 0.f;\n"
-        << (tan ? "            wt[j] = ok ? wtr[j][" + std::to_string(sl.w_st.at(pi)) + " + u] : 0.f;\n" : "")
-        << "            d[j] = 0.f;\n          }\n";
+        << "          const float w = ok ? wr[" << sl.w_st.at(pi) << " + u] : 0.f;\n"
+        << (tan ? "          const float wt = ok ? wtr[" + std::to_string(sl.w_st.at(pi)) + " + u] : 0.f;\n" : "")
+        << "          float d = 0.f;\n";
       const double* C = P.coeff.data() + p.c_off;
       for (int m1 = 0; m1 < N1; ++m1) {
         std::vector<int> m2s;
@@ -192,75 +176,60 @@ void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K,
           tdef << "            const float t" << m2 << " = " << e << ";\n";
         }
         if (m2s.empty()) continue;
-        o << "          {\n" << tdef.str();
-        for (int j = 0; j < NE; ++j) {
-          const std::string J = std::to_string(j);
-          auto dot = [&](const std::string& y) {
-            std::string e = y + "[" + J + "][" + std::to_string(m2s[0]) + "] * t" + std::to_string(m2s[0]);
-            for (size_t c = 1; c < m2s.size(); ++c)
-              e = "fmaf(" + y + "[" + J + "][" + std::to_string(m2s[c]) + "], t" + std::to_string(m2s[c]) + ", " +
-                  e + ")";
-            return e;
-          };
-          const std::string xm = "xv[" + J + "][" + std::to_string(m1) + "]";
-          const std::string mm = "mx[" + J + "][" + std::to_string(m1) + "]";
-          o << (j == 0 ? "            {\n" : "            if (vj[" + J + "]) {\n")
-            << "              const float s = " << dot("yl") << ";\n";
-          if (tan) {
-            const std::string xt = "xtv[0][" + std::to_string(m1) + "]";
-            o << "              const float st = " << dot("ytl") << ";\n"
-              << "              d[0] = fmaf(" << xt << ", s, fmaf(" << xm << ", st, d[0]));\n"
-              << "              " << mm << " = fmaf(wt[0], s, fmaf(w[0], st, " << mm << "));\n"
-              << "              const float wx = fmaf(w[0], " << xt << ", wt[0] * " << xm << ");\n";
-          } else {
-            o << "              d[" << J << "] = fmaf(" << xm << ", s, d[" << J << "]);\n"
-              << "              " << mm << " = fmaf(w[" << J << "], s, " << mm << ");\n"
-              << "              const float wx = w[" << J << "] * " << xm << ";\n";
-          }
-          for (int m2 : m2s)
-            o << "              z[" << J << "][" << zo + m2 << "] = fmaf(wx, t" << m2 << ", z[" << J << "]["
-              << zo + m2 << "]);\n";
-          o << "            }\n";
+        auto dot = [&](const std::string& y) {
+          std::string e = y + "[" + std::to_string(m2s[0]) + "] * t" + std::to_string(m2s[0]);
+          for (size_t c = 1; c < m2s.size(); ++c)
+            e = "fmaf(" + y + "[" + std::to_string(m2s[c]) + "], t" + std::to_string(m2s[c]) + ", " + e + ")";
+          return e;
+        };
+        const std::string xm = "xv[" + std::to_string(m1) + "]", mm = "mx[" + std::to_string(m1) + "]";
+        o << "          {\n" << tdef.str() << "            const float s = " << dot("yl") << ";\n";
+        if (tan) {
+          const std::string xt = "xtv[" + std::to_string(m1) + "]";
+          o << "            const float st = " << dot("ytl") << ";\n"
+            << "            d = fmaf(" << xt << ", s, fmaf(" << xm << ", st, d));\n"
+            << "            " << mm << " = fmaf(wt, s, fmaf(w, st, " << mm << "));\n"
+            << "            const float wx = fmaf(w, " << xt << ", wt * " << xm << ");\n";
+        } else {
+          o << "            d = fmaf(" << xm << ", s, d);\n"
+            << "            " << mm << " = fmaf(w, s, " << mm << ");\n"
+            << "            const float wx = w * " << xm << ";\n";
         }
+        for (int m2 : m2s)
+          o << "            z[" << zo + m2 << "] = fmaf(wx, t" << m2 << ", z[" << zo + m2 << "]);\n";
         o << "          }\n";
       }
-      o << "#pragma unroll\n          for (int j = 0; j < " << NE << "; ++j)\n"
-        << "            if (dWrow[j] && ok) dWrow[j][" << p.k0 << " + u] = d[j];\n"
-        << "        }\n";
+      o << "          if (dWrow && ok) dWrow[" << p.k0 << " + u] = d;\n        }\n";
     }
     if (!combined) {
       const int V = pow2(N2), LV = __builtin_ctz(V), sh = 5 - LV;
-      o << "#pragma unroll\n        for (int j = 0; j < " << NE << "; ++j)\n"
-        << "          if (sdy[j]) {\n            const float v = warp_sum_many<" << V << ">(z[j], lane);\n"
-        << "            const int c = lane >> " << sh << ";\n"
-        << "            if ((lane & " << ((1 << sh) - 1) << ") == 0 && c < " << N2 << ") sdy[j][" << l2 * l2
-        << " + c] = v;\n          }\n";
+      o << "        if (sdy) {\n          const float v = warp_sum_many<" << V << ">(z, lane);\n"
+        << "          const int c = lane >> " << sh << ";\n"
+        << "          if ((lane & " << ((1 << sh) - 1) << ") == 0 && c < " << N2 << ") sdy[" << l2 * l2
+        << " + c] = v;\n        }\n";
     }
     o << "      }\n";
   }
-  // the message rows of this channel block, through the warp's buffer
+  // the message row segment of this channel block, through the warp's buffer
   o << "      if (msg) {\n"
     << "        float* wbuf = reinterpret_cast<float*>(smem + OFF_WB) + (threadIdx.x >> 5) * WB;\n"
+    << "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) wbuf[lane * " << N1 << " + m1] = mx[m1];\n"
+    << "        __syncwarp();\n"
     << "        const int nch = min(32, " << MUL << " - u0 - r * 32);\n"
-    << "#pragma unroll\n        for (int j = 0; j < " << NE << "; ++j) {\n"
-    << "          if (!vj[j]) continue;\n"
-    << "#pragma unroll\n          for (int m1 = 0; m1 < " << N1 << "; ++m1) wbuf[lane * " << N1
-    << " + m1] = mx[j][m1];\n"
-    << "          __syncwarp();\n"
-    << "          if (nch > 0) warp_copy_out(msg + (size_t)(eb + bj[j]) * DIN + " << P.x_off[r.irrep]
-    << " + (u0 + r * 32) * " << N1 << ", wbuf, nch * " << N1 << ", lane);\n"
-    << "          __syncwarp();\n        }\n      }\n"
+    << "        if (nch > 0) warp_copy_out(msg + (size_t)e * DIN + " << P.x_off[r.irrep] << " + (u0 + r * 32) * "
+    << N1 << ", wbuf, nch * " << N1 << ", lane);\n"
+    << "        __syncwarp();\n      }\n"
     << "      }\n";  // r
   if (combined) {
-    o << "#pragma unroll\n      for (int j = 0; j < " << NE << "; ++j)\n      if (sdy[j]) {\n";
+    o << "      if (sdy) {\n";
     for (int off = 0, rest = VZ; rest > 0;) {
       int V = 1;
       while (V * 2 <= rest && V * 2 <= 32) V *= 2;
       const int LV = __builtin_ctz(V), sh = 5 - LV;
       o << "        {\n          float zp[" << V << "];\n#pragma unroll\n          for (int t = 0; t < " << V
-        << "; ++t) zp[t] = z[j][" << off << " + t];\n"
+        << "; ++t) zp[t] = z[" << off << " + t];\n"
         << "          const float v = warp_sum_many<" << V << ">(zp, lane);\n"
-        << "          if ((lane & " << ((1 << sh) - 1) << ") == 0) sdy[j][" << off << " + (lane >> " << sh
+        << "          if ((lane & " << ((1 << sh) - 1) << ") == 0) sdy[" << off << " + (lane >> " << sh
         << ")] = v;\n        }\n";
       off += V;
       rest -= V;
@@ -269,9 +238,8 @@ void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K,
   } else {
     for (int l2 = 0; l2 <= P.L; ++l2)
       if (!l2seen[l2])
-        o << "#pragma unroll\n      for (int j = 0; j < " << NE << "; ++j)\n"
-          << "        if (sdy[j] && lane == 0) {\n#pragma unroll\n          for (int t = 0; t < " << 2 * l2 + 1
-          << "; ++t) sdy[j][" << l2 * l2 << " + t] = 0.f;\n        }\n";
+        o << "      if (sdy && lane == 0) {\n#pragma unroll\n        for (int t = 0; t < " << 2 * l2 + 1
+          << "; ++t) sdy[" << l2 * l2 << " + t] = 0.f;\n      }\n";
   }
   o << "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n"
     << "  __syncwarp();\n  if (lane == 0) mbar_arrive(gempty0 + 8 * gb);\n  ++kr;\n  }\n  *qp = q;\n  *kp = kr;\n}\n";
@@ -783,7 +751,6 @@ cgtp_status build_backward(Plan& P) {
         K.nw = NW;
         K.force_B = B;
         K.no_chat = P.bwd_tform;
-  K.pair = P.bwd_pair;
         int maxr = 0;
         for (int s2 = 0; s2 < ns; ++s2) {
           for (size_t k = 0; k < slices[s2].size(); ++k) {
@@ -834,7 +801,6 @@ cgtp_status build_backward(Plan& P) {
   K.nw = F.nw;
   K.force_B = best.B;
   K.no_chat = P.bwd_tform;
-  K.pair = P.bwd_pair;
   for (int s2 = 0; s2 < F.S; ++s2) {
     for (size_t k = 0; k < best.slices[s2].size(); ++k) {
       const BwdIrrep& wi = best.W[best.slices[s2][k]];

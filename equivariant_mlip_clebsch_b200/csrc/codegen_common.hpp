@@ -82,8 +82,6 @@ struct KernelShape {
   // backward roles that contract with the CG table and Y directly: no Chat
   // is staged or built (the default; CGTP_BWD_TFORM=0 turns it off)
   bool no_chat = false;
-  // CG-first roles: edges of a receiver per pass, sharing t = C g (1 or 2)
-  int pair = 1;
   int off_wb = 0;
 };
 

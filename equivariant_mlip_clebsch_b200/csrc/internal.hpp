@@ -164,8 +164,6 @@ struct Plan {
   // Y, so no Chat is staged; CGTP_BWD_TFORM=0 at plan creation selects the
   // staged-Chat form instead (kept for comparison)
   bool bwd_tform = true;
-  // edges per pass of a CG-first role (CGTP_BWD_PAIR at plan creation)
-  int bwd_pair = 1;
 
   // tangent kernels of the double backward, built on first use (tan_state:
   // 0 not built, 1 ready, -1 unavailable: the composition is used)
