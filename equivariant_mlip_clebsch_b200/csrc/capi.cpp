@@ -191,6 +191,7 @@ cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge, con
       if (const char* d = std::getenv("CGTP_DEBUG"); d && *d && *d != '0') P->checks.store(CGTP_CHECK_GRAPH);
     }
     if (const char* v = std::getenv("CGTP_BWD_TFORM"); v && *v == '0') P->bwd_tform = false;
+    if (const char* v = std::getenv("CGTP_FWD_PACKED"); v && *v) P->fwd_packed = *v == '1';
     st = build_forward(*P);  // leaves the forward compiling on a host thread
     if (st == CGTP_OK) st = build_backward(*P);
     if (st == CGTP_OK)
@@ -581,6 +582,7 @@ cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* need
          std::to_string(q.paths.size()) + " cost=" + std::to_string((int)q.cost) + "\n";
   }
   cfg("backward", P->bcfg, P->bwd, P->bwd_roles.size());
+  t += std::string("forward form=") + (P->fcfg.packed ? "packed" : "scalar") + "\n";
   t += std::string("backward form=") + (P->bwd_tform ? "cg_first" : "staged_chat") + "\n";
   for (size_t r = 0; r < P->bwd_roles.size(); ++r) {
     const BwdRole& q = P->bwd_roles[r];

@@ -693,13 +693,19 @@ cgtp_status build_backward(Plan& P) {
     std::vector<std::vector<int>> pick;    // option per member
     std::vector<BwdIrrep> W;
   } best;
-  // Order of preference, from measurements on B200: the largest chunk that
-  // fits (it sets how many edges each stage hands over per barrier round
-  // trip, and how many are in flight), then two resident CTAs per SM when
-  // that chunk allows it, then the shortest consumer critical path per SM.
-  int kB[] = {8, 4, 2, 1};
-  if (const char* v = std::getenv("CGTP_BWD_CHUNK"))  // tuning override: one chunk size
-    kB[0] = kB[1] = kB[2] = kB[3] = std::max(1, std::min(8, std::atoi(v)));
+  // Candidates (chunk, least resident CTAs per SM) in order of preference,
+  // from measurements on B200: the largest chunk of at least four edges that
+  // leaves two CTAs per SM (the chunk sets how many edges each stage hands
+  // over per barrier round trip, and how many are in flight); when none
+  // does, four edges at one CTA (wide rows: Lmax 2 wide 297 -> 270 us, Lmax 6
+  // 2130 -> 1917 us against eight edges at one CTA), then smaller chunks.
+  // Among the plans of a candidate: the shortest consumer critical path per
+  // SM.
+  std::vector<std::pair<int, int>> cand = {{8, 2}, {4, 2}, {4, 1}, {2, 1}, {1, 1}};
+  if (const char* v = std::getenv("CGTP_BWD_CHUNK")) {  // tuning override: one chunk size
+    const int B0 = std::max(1, std::min(8, std::atoi(v)));
+    cand = {{B0, 2}, {B0, 1}};
+  }
   // barrier round trips, loop and address work of one chunk, in the units of
   // bwd_edge_cost
   const double kChunkOverhead = 80.0;
@@ -707,7 +713,7 @@ cgtp_status build_backward(Plan& P) {
   int kNW[] = {4, 8};
   if (const char* v = std::getenv("CGTP_BWD_NW"))  // tuning override: one warp count
     kNW[0] = kNW[1] = std::max(1, std::min(16, std::atoi(v)));
-  for (int B : kB) {
+  for (const auto& [B, min_ctas] : cand) {
     if (best.B != 0) break;
     // options of every irrep for this chunk size
     std::vector<BwdIrrep> W(n);
@@ -729,7 +735,6 @@ cgtp_status build_backward(Plan& P) {
           W[i].opts.push_back({R, nph, nblk * nph, ce * ((B + nph - 1) / nph)});
       }
     }
-    for (int min_ctas = 2; min_ctas >= 1 && best.B == 0; --min_ctas)
     for (int NW : kNW) {
       for (const auto& rgs : parts) {
         const int ns = rgs.empty() ? 0 : *std::max_element(rgs.begin(), rgs.end()) + 1;

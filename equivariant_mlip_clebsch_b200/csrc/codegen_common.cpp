@@ -78,7 +78,7 @@ void layout_slice(const Plan& P, SliceLayout& sl, bool with_g) {
   sl.chs = 0;
   for (int pi : sl.paths) {
     sl.ch_off[pi] = sl.chs;
-    sl.chs += chat_size(P.paths[pi].l1, P.paths[pi].l3);
+    sl.chs += chat_size(P.paths[pi].l1, P.paths[pi].l3, sl.m1_major);
   }
   sl.x_st.clear();
   sl.xseg.clear();
@@ -620,7 +620,7 @@ cgtp_status upload_chat_tables(const Plan& P, const std::vector<SliceLayout>& SL
             ++cnt;
           }
           if (cnt == 0) continue;
-          const int dst = sl.ch_off.at(pi) + chat_pos(p.l1, p.l3, m1, m3);
+          const int dst = sl.ch_off.at(pi) + chat_pos(p.l1, p.l3, m1, m3, sl.m1_major);
           if (dst >= (1 << 16) || yi[0] >= 256 || yi[1] >= 256)
             return fail(CGTP_ERR_SIZE, "Chat block too large for the record format");
           int b0, b1;

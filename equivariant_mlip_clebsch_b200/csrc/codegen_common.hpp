@@ -21,14 +21,16 @@ std::string spin_limit_define();
 inline int pad4(int n) { return (n + 3) & ~3; }
 
 // Chat_{e,p} = sum_m2 C_p[m1][m2][m3] Y[e][l2^2+m2], stored per edge and path
-// as [N3][pad4(N1)] when N1 > 1 and as one padded row [pad4(N3)] when N1 == 1.
-inline int chat_size(int l1, int l3) {
+// as [N3][pad4(N1)] (m3-major) or [N1][pad4(N3)] (m1-major, rows of m3 pairs
+// for the packed forward) when N1 > 1, and as one padded row [pad4(N3)] when
+// N1 == 1.
+inline int chat_size(int l1, int l3, bool m1_major) {
   const int n1 = 2 * l1 + 1, n3 = 2 * l3 + 1;
-  return n1 == 1 ? pad4(n3) : n3 * pad4(n1);
+  return n1 == 1 ? pad4(n3) : m1_major ? n1 * pad4(n3) : n3 * pad4(n1);
 }
-inline int chat_pos(int l1, int l3, int m1, int m3) {
-  const int n1 = 2 * l1 + 1;
-  return n1 == 1 ? m3 : m3 * pad4(n1) + m1;
+inline int chat_pos(int l1, int l3, int m1, int m3, bool m1_major) {
+  const int n1 = 2 * l1 + 1, n3 = 2 * l3 + 1;
+  return n1 == 1 ? m3 : m1_major ? m1 * pad4(n3) + m3 : m3 * pad4(n1) + m1;
 }
 
 // A contiguous piece of a global row copied into a staged row.
@@ -39,6 +41,7 @@ struct Segment {
 };
 
 struct SliceLayout {
+  bool m1_major = false;       // Chat layout (see chat_pos)
   std::vector<int> paths;      // paths whose Chat the slice needs
   std::map<int, int> ch_off;   // path -> Chat offset (floats, per edge)
   int chs = 0;                 // Chat floats per edge
@@ -79,6 +82,9 @@ struct KernelShape {
   bool tangent = false;
   // W rows prefetched into L2 this many chunks ahead (0: off)
   int prefetch = 0;
+  // forward roles with float2 accumulators of m3 pairs and packed FMAs over
+  // an m1-major Chat (fpath2, fpath_tan2)
+  bool packed = false;
   // backward roles that contract with the CG table and Y directly: no Chat
   // is staged or built (the default; CGTP_BWD_TFORM=0 turns it off)
   bool no_chat = false;

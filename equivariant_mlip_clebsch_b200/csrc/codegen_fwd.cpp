@@ -213,10 +213,14 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
     const SliceLayout& sl = SL[slice_of[shape_rep[k]]];
     const Irrep& h = P.in[r.irrep];
     const int N1 = 2 * h.l + 1, R = r.R, MUL = h.mul;
+    // accumulators: floats, or float2 pairs of consecutive m3 (packed)
+    const bool pk = K.packed;
+    auto np = [&](int pi) { return pk ? P.paths[pi].l3 + 1 : 2 * P.paths[pi].l3 + 1; };
     int nacc = 0;
-    for (int pi : r.paths) nacc += R * (2 * P.paths[pi].l3 + 1);
+    for (int pi : r.paths) nacc += R * np(pi);
+    const std::string AT = pk ? "float2" : "float";
     o << "// shape " << k << ": irrep " << r.irrep << " (" << h.mul << "x" << h.l << "), " << r.paths.size()
-      << " paths, R=" << R << "\n";
+      << " paths, R=" << R << (pk ? ", packed" : "") << "\n";
     o << "__device__ __noinline__ void fcons_" << k
       << "(const int* __restrict__ rowptr, int n_recv, float* __restrict__ out, int* __restrict__ err,\n"
          "    unsigned char* smem, int u0, int chs, int* qp) {\n"
@@ -229,8 +233,9 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
          "  int q = *qp;\n"
          "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
          "  const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
-         "  float acc[" << nacc << "];\n"
-         "#pragma unroll\n  for (int k = 0; k < " << nacc << "; ++k) acc[k] = 0.f;\n"
+         "  " << AT << " acc[" << nacc << "];\n"
+         "#pragma unroll\n  for (int k = 0; k < " << nacc << "; ++k) acc[k] = "
+      << (pk ? "make_float2(0.f, 0.f)" : "0.f") << ";\n"
          "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
          "    const int s = q % NSTAGE;\n"
          "    if (!stage_ready(full0, s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); *qp = -1; return; }\n"
@@ -243,21 +248,25 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
          "      const float* chb = sC + b * chs;\n"
          "      const float* wr = sW + b * WS;\n"
          "      const float* xr = sX + b * XS;\n"
-         "      float xv[" << R << "][" << N1 << "];\n"
+         "      " << (pk ? "float2" : "float") << " xv[" << R << "][" << N1 << "];\n"
          "#pragma unroll\n      for (int r = 0; r < " << R << "; ++r) {\n"
          "        const int u = u0 + r * 32 + lane;\n"
-         "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) xv[r][m1] = ok[r] ? xr[u * " << N1
-      << " + m1] : 0.f;\n      }\n";
+         "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) "
+      << (pk ? "{ const float v = ok[r] ? xr[u * " + std::to_string(N1) + " + m1] : 0.f; xv[r][m1] = make_float2(v, v); }"
+             : "xv[r][m1] = ok[r] ? xr[u * " + std::to_string(N1) + " + m1] : 0.f;")
+      << "\n      }\n";
     if (K.tangent)  // the tangent copies of the same pieces
       o << "      const float* chtb = reinterpret_cast<const float*>(st + OFF_CHT) + b * chs;\n"
            "      const float* wtr = reinterpret_cast<const float*>(st + OFF_WT) + b * WS;\n"
            "      const float* xtr = reinterpret_cast<const float*>(st + OFF_XT) + " << sl.x_st.at(r.irrep)
         << " + b * XS;\n"
-           "      float xtv[" << R << "][" << N1 << "];\n"
+           "      " << (pk ? "float2" : "float") << " xtv[" << R << "][" << N1 << "];\n"
            "#pragma unroll\n      for (int r = 0; r < " << R << "; ++r) {\n"
            "        const int u = u0 + r * 32 + lane;\n"
-           "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) xtv[r][m1] = ok[r] ? xtr[u * " << N1
-        << " + m1] : 0.f;\n      }\n";
+           "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) "
+        << (pk ? "{ const float v = ok[r] ? xtr[u * " + std::to_string(N1) + " + m1] : 0.f; xtv[r][m1] = make_float2(v, v); }"
+               : "xtv[r][m1] = ok[r] ? xtr[u * " + std::to_string(N1) + " + m1] : 0.f;")
+        << "\n      }\n";
     int A = 0;
     for (int pi : r.paths) {
       const Path& p = P.paths[pi];
@@ -267,12 +276,12 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
       if (K.tangent)
         o << "        float wt[" << R << "];\n#pragma unroll\n        for (int r = 0; r < " << R
           << "; ++r) wt[r] = ok[r] ? wtr[" << sl.w_st.at(pi) << " + u0 + r * 32 + lane] : 0.f;\n"
-          << "        fpath_tan<" << N1 << "," << N3 << "," << R << "," << A << "," << nacc << ">(acc, chb + "
-          << sl.ch_off.at(pi) << ", chtb + " << sl.ch_off.at(pi) << ", xv, xtv, w, wt); }\n";
+          << "        fpath_tan" << (pk ? "2<" : "<") << N1 << "," << N3 << "," << R << "," << A << "," << nacc
+          << ">(acc, chb + " << sl.ch_off.at(pi) << ", chtb + " << sl.ch_off.at(pi) << ", xv, xtv, w, wt); }\n";
       else
-        o << "        fpath<" << N1 << "," << N3 << "," << R << "," << A << "," << nacc << ">(acc, chb + "
-          << sl.ch_off.at(pi) << ", xv, w); }\n";
-      A += R * N3;
+        o << "        fpath" << (pk ? "2<" : "<") << N1 << "," << N3 << "," << R << "," << A << "," << nacc
+          << ">(acc, chb + " << sl.ch_off.at(pi) << ", xv, w); }\n";
+      A += R * np(pi);
     }
     o << "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n";
     o << "  float* orow = out + (size_t)i * DOUT;\n";
@@ -282,8 +291,12 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
       const int N3 = 2 * p.l3 + 1;
       o << "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) if (ok[r]) {\n    const int u = u0 + r * 32 + lane;\n"
         << "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) orow[" << p.o_off << " + u * " << N3
-        << " + m3] = acc[" << A << " + r * " << N3 << " + m3];\n  }\n";
-      A += R * N3;
+        << " + m3] = "
+        << (pk ? "(m3 & 1) ? acc[" + std::to_string(A) + " + r * " + std::to_string(np(pi)) + " + (m3 >> 1)].y : acc[" +
+                     std::to_string(A) + " + r * " + std::to_string(np(pi)) + " + (m3 >> 1)].x"
+               : "acc[" + std::to_string(A) + " + r * " + std::to_string(N3) + " + m3]")
+        << ";\n  }\n";
+      A += R * np(pi);
     }
     o << "  }\n  *qp = q;\n}\n";
   }
@@ -320,10 +333,11 @@ static double fwd_role_cost(const Plan& P, const FwdRole& r) {
 
 // The staging layout of each forward slice: the paths and hidden irreps of
 // its roles.
-static std::vector<SliceLayout> forward_slices(const Plan& P) {
+static std::vector<SliceLayout> forward_slices(const Plan& P, bool m1_major) {
   const FwdConfig& F = P.fcfg;
   std::vector<SliceLayout> SL(F.S);
   for (int s = 0; s < F.S; ++s) {
+    SL[s].m1_major = m1_major;
     std::vector<char> pseen(P.paths.size(), 0), iseen(P.in.size(), 0);
     for (int ri : F.slice_roles[s]) {
       for (int pi : P.fwd_roles[ri].paths) pseen[pi] = 1;
@@ -565,11 +579,14 @@ cgtp_status build_forward(Plan& P) {
     for (int pi : r.paths) n += r.R * (2 * P.paths[pi].l3 + 1);
     F.nacc = std::max(F.nacc, n);
   }
-  std::vector<SliceLayout> SL = forward_slices(P);
+  // packed roles (float2 accumulators, m1-major Chat) for the coarse roles
+  F.packed = P.fwd_packed && !F.generic;
+  std::vector<SliceLayout> SL = forward_slices(P, F.packed);
   KernelShape K;
   K.S = F.S;
   K.nw = F.nw;
   K.WB = 0;  // output rows go straight from registers to global memory
+  K.packed = F.packed;
   plan_layout(P, SL, K, false);
   F.B = K.B;
   F.stages = K.stages;
@@ -625,12 +642,13 @@ cgtp_status build_forward(Plan& P) {
 // pass gives d/dt fwd(x + t xt, Y + t Yt, W + t Wt).  Built on first use.
 cgtp_status build_forward_tangent(Plan& P, JitKernel& out, std::string* src_out) {
   const FwdConfig& F = P.fcfg;
-  std::vector<SliceLayout> SL = forward_slices(P);
+  std::vector<SliceLayout> SL = forward_slices(P, F.packed);  // the plain forward's Chat records
   KernelShape K;
   K.S = F.S;
   K.nw = F.nw;
   K.WB = 0;
   K.tangent = true;
+  K.packed = F.packed;
   plan_layout(P, SL, K, false);
   for (size_t k = 0; k + 1 < P.fwd_ent_begin.size(); ++k)
     K.rec_max = std::max(K.rec_max, P.fwd_ent_begin[k + 1] - P.fwd_ent_begin[k]);

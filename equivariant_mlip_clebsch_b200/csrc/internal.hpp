@@ -127,6 +127,7 @@ struct FwdConfig {
   bool w_smem = true;    // W row pieces staged by bulk copy (16-byte aligned)
   bool x_smem = true;    // x blocks staged by bulk copy
   bool generic = false;  // forward roles of one path, one function per (2l1+1, 2l3+1) shape
+  bool packed = false;   // forward roles with packed FMAs over an m1-major Chat
   int nacc = 0;          // accumulator registers per thread
   std::vector<std::vector<int>> slice_roles;  // role ids per slice
 };
@@ -164,6 +165,9 @@ struct Plan {
   // Y, so no Chat is staged; CGTP_BWD_TFORM=0 at plan creation selects the
   // staged-Chat form instead (kept for comparison)
   bool bwd_tform = true;
+  // forward roles with float2 accumulators and packed FMAs (CGTP_FWD_PACKED
+  // at plan creation)
+  bool fwd_packed = false;
 
   // tangent kernels of the double backward, built on first use (tan_state:
   // 0 not built, 1 ready, -1 unavailable: the composition is used)
