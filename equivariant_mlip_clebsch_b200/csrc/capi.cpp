@@ -191,7 +191,7 @@ cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge, con
       if (const char* d = std::getenv("CGTP_DEBUG"); d && *d && *d != '0') P->checks.store(CGTP_CHECK_GRAPH);
     }
     if (const char* v = std::getenv("CGTP_BWD_TFORM"); v && *v == '0') P->bwd_tform = false;
-    if (const char* v = std::getenv("CGTP_FWD_PACKED"); v && *v) P->fwd_packed = *v == '1';
+    if (const char* v = std::getenv("CGTP_FWD_PACKED"); v && (*v == '0' || *v == '1')) P->fwd_packed = *v - '0';
     st = build_forward(*P);  // leaves the forward compiling on a host thread
     if (st == CGTP_OK) st = build_backward(*P);
     if (st == CGTP_OK)

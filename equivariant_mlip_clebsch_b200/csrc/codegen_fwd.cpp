@@ -579,8 +579,13 @@ cgtp_status build_forward(Plan& P) {
     for (int pi : r.paths) n += r.R * (2 * P.paths[pi].l3 + 1);
     F.nacc = std::max(F.nacc, n);
   }
-  // packed roles (float2 accumulators, m1-major Chat) for the coarse roles
-  F.packed = P.fwd_packed && !F.generic;
+  // Packed roles (float2 accumulators of m3 pairs, m1-major Chat) for coarse
+  // plans with a hidden irrep of l >= 3, whose long m3 rows pack well.
+  // Measured on B200: Lmax 3 470 -> 433 us, Case 5 470 -> 402 us; plans with
+  // l <= 2 inputs lose (Lmax 2 35 -> 43 us, Lmax 2 wide 137 -> 148 us).
+  int lmax_in = 0;
+  for (const Irrep& h : P.in) lmax_in = std::max(lmax_in, h.l);
+  F.packed = !F.generic && (P.fwd_packed < 0 ? lmax_in >= 3 : P.fwd_packed == 1);
   std::vector<SliceLayout> SL = forward_slices(P, F.packed);
   KernelShape K;
   K.S = F.S;

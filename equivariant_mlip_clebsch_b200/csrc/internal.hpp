@@ -165,9 +165,9 @@ struct Plan {
   // Y, so no Chat is staged; CGTP_BWD_TFORM=0 at plan creation selects the
   // staged-Chat form instead (kept for comparison)
   bool bwd_tform = true;
-  // forward roles with float2 accumulators and packed FMAs (CGTP_FWD_PACKED
-  // at plan creation)
-  bool fwd_packed = false;
+  // forward roles with float2 accumulators and packed FMAs: -1 chosen by the
+  // planner, 0 off, 1 on (CGTP_FWD_PACKED at plan creation)
+  int fwd_packed = -1;
 
   // tangent kernels of the double backward, built on first use (tan_state:
   // 0 not built, 1 ready, -1 unavailable: the composition is used)

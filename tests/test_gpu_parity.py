@@ -232,6 +232,7 @@ RAGGED = [
     ("96x0e+40x1o", "1x0e+1x1o+1x2e", None),                          # ragged channel blocks
     ("64x0e+64x1o+64x2e+64x3o+64x4e+64x5o+64x6e",
      "1x0e+1x1o+1x2e+1x3o+1x4e+1x5o+1x6e", "lmax6"),                  # several slices
+    ("32x0e+17x1o+8x2e+33x3o", "1x0e+1x1o+1x2e+1x3o", None),           # l = 3, partial blocks
 ]
 
 
@@ -242,7 +243,7 @@ def _out_irreps(hid, edge):
                     zip(P0.out_mul_from_paths, P0.irreps_out) if m > 0)
 
 
-@pytest.mark.parametrize("spec", RAGGED, ids=["partial_warps", "unaligned", "ragged_blocks", "slices"])
+@pytest.mark.parametrize("spec", RAGGED, ids=["partial_warps", "unaligned", "ragged_blocks", "slices", "l3_partial"])
 def test_random_ragged_graphs(spec, dev):
     hid, edge, out = spec
     if out == "lmax6":
@@ -252,11 +253,11 @@ def test_random_ragged_graphs(spec, dev):
     check_random_graph(hid, edge, out, dev)
 
 
-def check_random_graph(hid, edge, out, dev):
+def check_random_graph(hid, edge, out, dev, plan=None):
     """Y, forward and all three gradients on a random ragged graph (37
     receivers, 3 of them without edges, 29 senders, degrees 0-45, one zero
     edge vector) against the oracle."""
-    plan = plan_for(hid, edge, out)
+    plan = plan or plan_for(hid, edge, out)
     P = O.enumerate_paths(hid, edge, out)
     rng = np.random.default_rng(5)
     n_recv, n_send = 37, 29
@@ -284,6 +285,19 @@ def check_random_graph(hid, edge, out, dev):
     for k, a, b in zip("xWY", grads, refs):
         assert_close(a.cpu().numpy(), b, f"d{k}")
     plan.check_device_error()
+
+
+@pytest.mark.parametrize("form", ["0", "1"], ids=["scalar_fwd", "packed_fwd"])
+@pytest.mark.parametrize("spec", [RAGGED[1], RAGGED[2], RAGGED[4]], ids=["unaligned", "ragged_blocks", "l3_partial"])
+def test_forward_forms_on_ragged_graphs(spec, form, dev, monkeypatch):
+    """Both forward forms (scalar, and packed FMAs over an m1-major Chat),
+    whichever the planner would pick, on ragged graphs and channel blocks."""
+    hid, edge, out = spec
+    out = out or _out_irreps(hid, edge)
+    monkeypatch.setenv("CGTP_FWD_PACKED", form)
+    plan = C().Plan(hid, edge, out, 6)
+    assert ("forward form=packed" in plan.describe()) == (form == "1")
+    check_random_graph(hid, edge, out, dev, plan)
 
 
 def test_empty_graph(dev):

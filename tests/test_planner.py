@@ -242,16 +242,18 @@ def _check_layout(src, smem, backward):
 
 @pytest.mark.parametrize("irreps", [WL.CONFIGS[n] for n in NAMES] + [
     dict(irreps_in=a, irreps_edge=b, irreps_out=c) for a, b, c in ODD], ids=NAMES + [f"odd{k}" for k in range(len(ODD))])
-@pytest.mark.parametrize("prefetch,tform", [("0", "1"), ("4", "1"), ("0", "0")],
-                         ids=["default", "prefetch4", "staged_chat"])
-def test_generated_copies_stay_in_bounds(irreps, prefetch, tform, compile_only, monkeypatch, tmp_path):
+@pytest.mark.parametrize("prefetch,tform,packed", [("0", "1", ""), ("4", "1", ""), ("0", "0", "0"), ("0", "1", "1")],
+                         ids=["default", "prefetch4", "staged_chat_scalar_fwd", "packed_fwd"])
+def test_generated_copies_stay_in_bounds(irreps, prefetch, tform, packed, compile_only, monkeypatch, tmp_path):
     """The generated kernels' row copies into shared memory and their L2
     prefetches, read from the generated source (checked here so that a
     mistake fails on the CPU rather than faulting a GPU), for the default
-    kernels, with W prefetch, and with the staged-Chat backward."""
+    kernels, with W prefetch, with the staged-Chat backward and the scalar
+    forward, and with the packed forward on every plan."""
     monkeypatch.setenv("CGTP_DUMP_SOURCE", str(tmp_path))
     monkeypatch.setenv("CGTP_PREFETCH", prefetch)
     monkeypatch.setenv("CGTP_BWD_TFORM", tform)
+    monkeypatch.setenv("CGTP_FWD_PACKED", packed)
     plan = C.Plan(irreps["irreps_in"], irreps["irreps_edge"], irreps["irreps_out"], 6)
     assert f"backward form={'cg_first' if tform == '1' else 'staged_chat'}" in plan.describe()
     smem = {k: int(v) for k, v in re.findall(r"^(forward|backward): .* smem=(\d+)", plan.describe(), re.M)}
