@@ -40,6 +40,7 @@ void destroy_plan_device(Plan& P) {
   jit_unload(P.bwd);
   jit_unload(P.bwd_er);
   jit_unload(P.fwd_tan);
+  jit_unload(P.fwd_acc);
   jit_unload(P.bwd_tan);
   for (void** p : {&P.d_fwd_ent, &P.d_bwd_ent}) {
     if (*p) cudaFree(*p);
@@ -63,8 +64,8 @@ static cgtp_status check_device(const Plan& P) {
   return CGTP_OK;
 }
 
-static const char* kKindName[] = {"sph_harm",     "cgtp_fwd",  "cgtp_bwd",    "bwd_reduce",
-                                  "sph_harm_bwd", "zero_fill", "cgtp_fwd_tan", "cgtp_bwd_tan"};
+static const char* kKindName[] = {"sph_harm",     "cgtp_fwd",  "cgtp_bwd",     "bwd_reduce",  "sph_harm_bwd",
+                                  "zero_fill",    "cgtp_fwd_tan", "cgtp_bwd_tan", "cgtp_fwd_acc"};
 
 // Brackets one internal launch with events when timing is on.
 struct TimedScope {
@@ -192,6 +193,11 @@ cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge, con
     }
     if (const char* v = std::getenv("CGTP_BWD_TFORM"); v && *v == '0') P->bwd_tform = false;
     if (const char* v = std::getenv("CGTP_FWD_PACKED"); v && (*v == '0' || *v == '1')) P->fwd_packed = *v - '0';
+    if (const char* v = std::getenv("CGTP_DBWD_FWD")) {
+      if (std::string(v) == "tangent") P->dbwd_fwd_sum = 0;
+      if (std::string(v) == "sum") P->dbwd_fwd_sum = 1;
+    }
+    if (const char* v = std::getenv("CGTP_BWD_PACKED"); v && (*v == '0' || *v == '1')) P->bwd_packed = *v == '1';
     st = build_forward(*P);  // leaves the forward compiling on a host thread
     if (st == CGTP_OK) st = build_backward(*P);
     if (st == CGTP_OK)
@@ -366,18 +372,26 @@ static bool ensure_tangent(Plan& P) {
     P.tan_msg = "no paths";
     return false;
   }
+  // gg_out: the tangent forward, or (packed plans, where the tangent
+  // forward's doubled per-edge work on a shallower ring measured slower than
+  // three forwards: Lmax 3 1773 us against 3 x 453) the sum of one plain and
+  // two accumulating forwards
+  if (P.dbwd_fwd_sum < 0) P.dbwd_fwd_sum = P.fcfg.packed ? 1 : 0;
   std::string fsrc, bsrc;
-  cgtp_status st = build_forward_tangent(P, P.fwd_tan, &fsrc);
+  cgtp_status st = P.dbwd_fwd_sum ? build_forward_accumulate(P, P.fwd_acc, &fsrc)
+                                  : build_forward_tangent(P, P.fwd_tan, &fsrc);
   if (st == CGTP_OK) st = build_backward_tangent(P, P.bwd_tan, &bsrc);
   if (st != CGTP_OK) {
     P.tan_msg = cgtp_last_error();
     jit_unload(P.fwd_tan);
+    jit_unload(P.fwd_acc);
     jit_unload(P.bwd_tan);
     P.tan_state = -1;
     return false;
   }
   if (const char* d = std::getenv("CGTP_DUMP_SOURCE")) {
-    for (auto [name, src] : {std::pair<const char*, std::string*>{"/fwd_tan.cu", &fsrc}, {"/bwd_tan.cu", &bsrc}}) {
+    const char* fname = P.dbwd_fwd_sum ? "/fwd_acc.cu" : "/fwd_tan.cu";
+    for (auto [name, src] : {std::pair<const char*, std::string*>{fname, &fsrc}, {"/bwd_tan.cu", &bsrc}}) {
       if (FILE* f = std::fopen((std::string(d) + name).c_str(), "w")) {
         std::fputs(src->c_str(), f);
         std::fclose(f);
@@ -590,11 +604,11 @@ cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* need
          std::to_string(q.u0) + " R=" + std::to_string(q.R) + " ph=" + std::to_string(q.ph) + "/" +
          std::to_string(q.nph) + " cost=" + std::to_string((int)q.cost) + "\n";
   }
-  for (const JitKernel* k : {&P->fwd_tan, &P->bwd_tan}) {  // tangent kernels, once built
+  for (const JitKernel* k : {&P->fwd_tan, &P->fwd_acc, &P->bwd_tan}) {  // double-backward kernels, once built
     if (k->name.empty()) continue;
     char hx[64];
     std::snprintf(hx, sizeof hx, " smem=%d threads=%d hash=%016llx\n", k->smem, k->threads, k->hash);
-    t += k->name + " (tangent, double backward):" + std::string(hx) + k->log;
+    t += k->name + " (double backward):" + std::string(hx) + k->log;
     if (!k->log.empty() && k->log.back() != '\n') t += "\n";
   }
   {  // the edge-range variant of the backward (same roles and layout)
@@ -749,7 +763,20 @@ cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send,
     // (h_x, h_Y, h_W) of the forward and of the backward at fixed grad_out
     int nr = (int)n_recv;
     const int32_t* no_eid = nullptr;
-    if (gg_out) {
+    if (gg_out && P->dbwd_fwd_sum == 1) {
+      // the forward is trilinear: its derivative is the sum of three
+      // forwards, each with one input replaced by its direction (the first
+      // writes gg_out, the other two add to it)
+      st = forward_impl(plan, n_recv, n_send, E, rowptr, col, h_x, Y, W, nullptr, gg_out, stream, false);
+      if (st != CGTP_OK) return st;
+      const float* ins[2][3] = {{x, h_Y, W}, {x, Y, h_W}};
+      for (auto& in : ins) {
+        void* args[] = {&rowptr, &col, &in[0], &in[1], &in[2], &no_eid, &gg_out, &P->d_fwd_ent, &nr, &P->d_err};
+        TimedScope ts(*P, 8, cs);
+        st = jit_launch(P->fwd_acc, dim3(persistent_grid(P->fwd_acc.blocks_per_sm, P->num_sms, n_recv)), args, cs);
+        if (st != CGTP_OK) return st;
+      }
+    } else if (gg_out) {
       void* args[] = {&rowptr, &col, &x, &Y, &W, &no_eid, &gg_out, &P->d_fwd_ent, &nr, &P->d_err, &h_x, &h_Y, &h_W};
       TimedScope ts(*P, 6, cs);
       st = jit_launch(P->fwd_tan, dim3(persistent_grid(P->fwd_tan.blocks_per_sm, P->num_sms, n_recv)), args, cs);

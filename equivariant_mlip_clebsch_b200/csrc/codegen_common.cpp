@@ -160,6 +160,7 @@ void plan_layout(const Plan& P, const std::vector<SliceLayout>& SL, KernelShape&
   // tuning overrides: edges per chunk and ring depth
   if (const char* v = std::getenv("CGTP_CHUNK"); v && K.force_B == 0) K.B = std::max(1, std::min(8, std::atoi(v)));
   if (const char* v = std::getenv("CGTP_STAGES")) K.stages = std::max(2, std::min(6, std::atoi(v)));
+  if (K.force_stages > 0) K.stages = K.force_stages;
   K.prefetch = kDefaultPrefetch;  // W rows prefetched into L2, in chunks ahead
   if (const char* v = std::getenv("CGTP_PREFETCH")) K.prefetch = std::max(0, std::min(64, std::atoi(v)));
   while (K.stages > 2 && fixed + K.stages * stage_of(K.B) > 220 * 1024) --K.stages;

@@ -75,15 +75,19 @@ struct KernelShape {
   int WB = 0;       // per-consumer-warp staging buffer for coalesced row stores (floats)
   int gbufs = 2;    // grad_out row buffers (backward)
   int force_B = 0;  // edges per chunk fixed by the caller (0: chosen from the budget)
+  int force_stages = 0;  // ring depth fixed by the caller (0: chosen from the budget)
   int rec_max = 0;  // most Chat records of a slice
   bool edge_ranges = false;  // backward CTAs take equal edge ranges
   // tangent kernels: every staged W, x and Y piece (and so Chat) has a
   // second copy holding its directional derivative (the double backward)
   bool tangent = false;
+  // forward: add the result to the output rows instead of writing them
+  bool accumulate = false;
   // W rows prefetched into L2 this many chunks ahead (0: off)
   int prefetch = 0;
-  // forward roles with float2 accumulators of m3 pairs and packed FMAs over
-  // an m1-major Chat (fpath2, fpath_tan2)
+  // forward: roles with float2 accumulators of m3 pairs and packed FMAs over
+  // an m1-major Chat (fpath2, fpath_tan2); backward: CG-first roles with
+  // pairs of m1 rows in float2 halves
   bool packed = false;
   // backward roles that contract with the CG table and Y directly: no Chat
   // is staged or built (the default; CGTP_BWD_TFORM=0 turns it off)

@@ -147,7 +147,8 @@ static std::string gen_fwd_generic(const Plan& P, const std::vector<SliceLayout>
       o << "      fpath<" << N1 << "," << N3 << ",1,0," << N3 << ">(acc, sC + b * chs, xv, w);\n";
     o << "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n"
          "  if (ok) {\n    float* orow = out + (size_t)i * DOUT + ooff;\n"
-         "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) orow[u * " << N3 << " + m3] = acc[m3];\n  }\n"
+         "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) orow[u * " << N3 << " + m3] "
+      << (K.accumulate ? "+=" : "=") << " acc[m3];\n  }\n"
          "  }\n  *qp = q;\n}\n";
   }
   gen_fwd_idle(o);
@@ -291,7 +292,7 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
       const int N3 = 2 * p.l3 + 1;
       o << "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) if (ok[r]) {\n    const int u = u0 + r * 32 + lane;\n"
         << "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) orow[" << p.o_off << " + u * " << N3
-        << " + m3] = "
+        << " + m3] " << (K.accumulate ? "+= " : "= ")
         << (pk ? "(m3 & 1) ? acc[" + std::to_string(A) + " + r * " + std::to_string(np(pi)) + " + (m3 >> 1)].y : acc[" +
                      std::to_string(A) + " + r * " + std::to_string(np(pi)) + " + (m3 >> 1)].x"
                : "acc[" + std::to_string(A) + " + r * " + std::to_string(N3) + " + m3]")
@@ -654,6 +655,9 @@ cgtp_status build_forward_tangent(Plan& P, JitKernel& out, std::string* src_out)
   K.WB = 0;
   K.tangent = true;
   K.packed = F.packed;
+  // tuning overrides for this kernel alone: edges per chunk and ring depth
+  if (const char* v = std::getenv("CGTP_FWD_TAN_CHUNK")) K.force_B = std::max(1, std::min(8, std::atoi(v)));
+  if (const char* v = std::getenv("CGTP_FWD_TAN_STAGES")) K.force_stages = std::max(2, std::min(6, std::atoi(v)));
   plan_layout(P, SL, K, false);
   for (size_t k = 0; k + 1 < P.fwd_ent_begin.size(); ++k)
     K.rec_max = std::max(K.rec_max, P.fwd_ent_begin[k + 1] - P.fwd_ent_begin[k]);
@@ -662,6 +666,45 @@ cgtp_status build_forward_tangent(Plan& P, JitKernel& out, std::string* src_out)
   const int mb0 = initial_min_blocks(K.smem, &fixed);
   const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
   const std::string name = "cgtp_fwd_tan";
+  std::string src;
+  JitBinary bin;
+  cgtp_status st = CGTP_OK;
+  for (int mb = mb0; mb >= mb_floor; --mb) {
+    src = gen_fwd_source(P, SL, K, name, mb);
+    st = jit_build(src, name, bin);
+    if (st != CGTP_OK || mb == mb_floor || max_spill_bytes(bin.log) <= 64) break;
+  }
+  if (st != CGTP_OK) {
+    set_error(bin.err);
+    return st;
+  }
+  out.threads = (F.nw + 2) * 32;
+  out.smem = K.smem;
+  if (src_out) *src_out = src;
+  return jit_load(bin, name, out);
+}
+
+// The accumulating forward (cgtp_fwd_acc): the plain forward's roles, slices
+// and layout, adding its result to the output rows.  The double backward sums
+// three forwards with it where that beats the tangent forward.  Built on
+// first use.
+cgtp_status build_forward_accumulate(Plan& P, JitKernel& out, std::string* src_out) {
+  const FwdConfig& F = P.fcfg;
+  std::vector<SliceLayout> SL = forward_slices(P, F.packed);
+  KernelShape K;
+  K.S = F.S;
+  K.nw = F.nw;
+  K.WB = 0;
+  K.packed = F.packed;
+  K.accumulate = true;
+  plan_layout(P, SL, K, false);
+  for (size_t k = 0; k + 1 < P.fwd_ent_begin.size(); ++k)
+    K.rec_max = std::max(K.rec_max, P.fwd_ent_begin[k + 1] - P.fwd_ent_begin[k]);
+  if (K.smem > 227 * 1024) return fail(CGTP_ERR_SIZE, "forward kernel needs too much shared memory");
+  bool fixed = false;
+  const int mb0 = initial_min_blocks(K.smem, &fixed);
+  const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
+  const std::string name = "cgtp_fwd_acc";
   std::string src;
   JitBinary bin;
   cgtp_status st = CGTP_OK;

@@ -168,10 +168,18 @@ struct Plan {
   // forward roles with float2 accumulators and packed FMAs: -1 chosen by the
   // planner, 0 off, 1 on (CGTP_FWD_PACKED at plan creation)
   int fwd_packed = -1;
+  // double backward: gg_out as three forwards summed (-1: the planner's
+  // choice, 0: the tangent forward, 1: the sum; CGTP_DBWD_FWD=tangent|sum at
+  // plan creation)
+  int dbwd_fwd_sum = -1;
+  // CG-first backward roles with rows m1 paired in float2 halves and packed
+  // FMAs (CGTP_BWD_PACKED=1 at plan creation)
+  bool bwd_packed = false;
 
   // tangent kernels of the double backward, built on first use (tan_state:
   // 0 not built, 1 ready, -1 unavailable: the composition is used)
   JitKernel fwd_tan, bwd_tan;
+  JitKernel fwd_acc;  // accumulating forward (double backward on packed plans)
   std::mutex tan_mu;
   int tan_state = 0;
   std::string tan_msg;
@@ -235,6 +243,7 @@ cgtp_status build_forward(Plan& P);
 cgtp_status build_backward(Plan& P);
 cgtp_status finish_forward(Plan& P);  // joins the forward's compile and loads it
 // tangent kernels (the double backward): built and loaded on the calling thread
+cgtp_status build_forward_accumulate(Plan& P, JitKernel& out, std::string* src_out);
 cgtp_status build_forward_tangent(Plan& P, JitKernel& out, std::string* src);
 cgtp_status build_backward_tangent(Plan& P, JitKernel& out, std::string* src);
 void destroy_plan_device(Plan& P);

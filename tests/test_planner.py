@@ -268,19 +268,28 @@ def test_generated_copies_stay_in_bounds(irreps, prefetch, tform, packed, compil
         assert not bad, (f, bad)
 
 
+@pytest.mark.parametrize("fwd", ["", "tangent", "sum"], ids=["planner", "tangent_fwd", "sum_fwd"])
 @pytest.mark.parametrize("name", ["tiny", "lmax2", "lmax2_wide", "lmax3", "case5"])
-def test_tangent_kernels_copies_and_layout(name, compile_only, monkeypatch, tmp_path):
-    """The double backward's tangent kernels (built on request): the same
-    copy and layout checks, with every staged piece doubled."""
+def test_tangent_kernels_copies_and_layout(name, fwd, compile_only, monkeypatch, tmp_path):
+    """The double backward's kernels (built on request): the tangent backward
+    and either the tangent forward (every staged piece doubled) or the
+    accumulating forward; the same copy and layout checks.  The planner takes
+    the sum of forwards for plans with packed forward roles."""
     monkeypatch.setenv("CGTP_DUMP_SOURCE", str(tmp_path))
+    monkeypatch.setenv("CGTP_DBWD_FWD", fwd)
     c = WL.CONFIGS[name]
     plan = C.Plan(c["irreps_in"], c["irreps_edge"], c["irreps_out"], 6)
     assert plan.prepare_double_backward()
     desc = plan.describe()
-    smem = {k: int(v) for k, v in re.findall(r"^(cgtp_fwd_tan|cgtp_bwd_tan) .* smem=(\d+)", desc, re.M)}
-    for f, kname in (("fwd_tan.cu", "cgtp_fwd_tan"), ("bwd_tan.cu", "cgtp_bwd_tan")):
+    use_sum = fwd == "sum" or (fwd == "" and "forward form=packed" in desc)
+    fk = "cgtp_fwd_acc" if use_sum else "cgtp_fwd_tan"
+    smem = {k: int(v) for k, v in re.findall(r"^(cgtp_fwd_tan|cgtp_fwd_acc|cgtp_bwd_tan) .* smem=(\d+)", desc, re.M)}
+    assert set(smem) == {fk, "cgtp_bwd_tan"}, smem
+    for f, kname in ((fk[5:] + ".cu", fk), ("bwd_tan.cu", "cgtp_bwd_tan")):
         src = (tmp_path / f).read_text()
-        assert "#define TAN 1" in src
+        assert ("#define TAN 1" in src) == (kname != "cgtp_fwd_acc")
+        if kname == "cgtp_fwd_acc":
+            assert "orow[" in src and "+=" in src.split("orow[", 1)[1].split(";", 1)[0]
         n, bad = _check_copies(src)
         assert n > 0 and not bad, (f, bad[:3])
         bad = _check_layout(src, smem[kname], f.startswith("bwd"))

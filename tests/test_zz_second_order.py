@@ -38,7 +38,27 @@ def _compare(plan, P, d, host, h, dev):
 def test_double_backward_random_graph(keys, dev):
     hid, edge = "96x0e+40x1o", "1x0e+1x1o+1x2e"
     out = _out_irreps(hid, edge)
-    plan = plan_for(hid, edge, out)
+    _random_graph_case(plan_for(hid, edge, out), hid, edge, out, keys, dev)
+
+
+@pytest.mark.parametrize("fwd", ["tangent", "sum"])
+@pytest.mark.parametrize("hid,edge", [("96x0e+40x1o", "1x0e+1x1o+1x2e"),
+                                      ("32x0e+17x1o+8x2e+33x3o", "1x0e+1x1o+1x2e+1x3o")],
+                         ids=["l1", "l3_partial"])
+def test_double_backward_forward_paths(hid, edge, fwd, dev, monkeypatch):
+    """Both ways of forming d grad_out: the tangent forward, and one plain
+    plus two accumulating forwards (the planner's choice for plans with packed
+    forward roles)."""
+    out = _out_irreps(hid, edge)
+    monkeypatch.setenv("CGTP_DBWD_FWD", fwd)
+    from equivariant_mlip_clebsch_b200 import cgtp as C
+    plan = C.Plan(hid, edge, out, 6)
+    assert plan.prepare_double_backward()
+    assert ("cgtp_fwd_acc" in plan.describe()) == (fwd == "sum")
+    _random_graph_case(plan, hid, edge, out, ("h_x", "h_W", "h_Y"), dev)
+
+
+def _random_graph_case(plan, hid, edge, out, keys, dev):
     P = O.enumerate_paths(hid, edge, out)
     rng = np.random.default_rng(11)
     n_recv, n_send = 37, 29
