@@ -425,18 +425,16 @@ def sparse_field(wb: "Workbench", k: int, ms_dense_step: float, ms_dense_fwd: fl
 
 
 def graph_check_cost(wb: "Workbench", k: int) -> dict:
-    """Device time the plan's graph checks add to one forward call (the
-    checks, the read-back of their result and the wait for it)."""
-    offs, ons = [], []
-    for _ in range(2):  # alternated, the lower of two runs each
-        offs.append(wb.timer(wb.fwd, k))
-        wb.plan.set_checks(True)
-        try:
-            ons.append(wb.timer(wb.fwd, k))
-        finally:
-            wb.plan.set_checks(False)
-    ms_off, ms_on = min(offs), min(ons)
-    return {"fwd_ms_checks_off": ms_off, "fwd_ms_checks_on": ms_on, "ms_added": ms_on - ms_off}
+    """Time of the device graph checks a checked call adds (the checks of
+    the receiver CSR and of the sender lists, the read-back of their result
+    and the wait for it), timed directly through cgtp_validate_graph."""
+    T = wb.T
+
+    def check():
+        wb.plan.validate_graph(T["rowptr"], T["col"], wb.N, T["rpt"], T["perm"], stream=wb.stream)
+    check()
+    return {"ms_added": wb.timer(check, k), "what": "cgtp_validate_graph on the step's graph (receiver CSR "
+            "and sender lists), host round trip included"}
 
 
 def run_cgtp(args, rank, world, local_rank):

@@ -54,6 +54,7 @@ _SIGS = {
     "cgtp_plan_check_device_error": (_i, [_P, ctypes.POINTER(_i)]),
     "cgtp_plan_set_timing": (_i, [_P, _i]),
     "cgtp_plan_set_checks": (_i, [_P, _i]),
+    "cgtp_validate_graph": (_i, [_P, _i64, _i64, _i64, _P, _P, _P, _P, _P]),
     "cgtp_plan_kernel_times": (_i, [_P, _i, ctypes.c_char_p, _P, _P, ctypes.POINTER(_i)]),
     "cgtp_sparse_workspace_size": (_i, [_P, _i64, _i64, _i64, ctypes.POINTER(_sz)]),
     "cgtp_sparse_forward": (_i, [_P, _i64, _i64, _i64] + [_P] * 8 + [_sz, _P]),
@@ -253,6 +254,17 @@ class Plan:
         """cgtp_plan_set_checks: device checks of the graph before every call
         (each call then waits for their result)."""
         _check(_lib.cgtp_plan_set_checks(self._h, 1 if enable else 0))
+
+    def validate_graph(self, rowptr, col, n_send: int, rowptr_T=None, perm_T=None, stream=None) -> None:
+        """cgtp_validate_graph: the device graph checks once, whatever the
+        plan's flags (raises CgtpError with status 7 naming the failed
+        checks)."""
+        if (rowptr_T is None) != (perm_T is None):
+            raise ValueError("rowptr_T and perm_T go together")
+        n_recv, E, dev = rowptr.shape[0] - 1, col.shape[0], rowptr.device
+        ptrs = _args(dev, (rowptr, "rowptr", n_recv + 1, "i32"), (col, "col", E, "i32"),
+                     (rowptr_T, "rowptr_T", n_send + 1, "i32"), (perm_T, "perm_T", E, "i32"))
+        _check(_lib.cgtp_validate_graph(self._h, n_recv, n_send, E, *ptrs, _stream(stream)))
 
     def set_timing(self, enable: bool) -> None:
         _check(_lib.cgtp_plan_set_timing(self._h, int(bool(enable))))

@@ -438,8 +438,9 @@ cgtp_status forward_impl(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t
 cgtp_status check_plan_device(const Plan& P) { return check_device(P); }
 
 cgtp_status check_graph(Plan& P, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
-                        const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, cgtp_stream stream) {
-  if (!(P.checks.load() & CGTP_CHECK_GRAPH) || (n_recv == 0 && E == 0)) return CGTP_OK;
+                        const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, cgtp_stream stream,
+                        bool always) {
+  if ((!always && !(P.checks.load() & CGTP_CHECK_GRAPH)) || (n_recv == 0 && E == 0)) return CGTP_OK;
   if (!rowptr || (E > 0 && !col)) return fail(CGTP_ERR_NULL, "rowptr or col is NULL");
   if (!rowptr_T || !perm_T) rowptr_T = nullptr, perm_T = nullptr;
   cudaStream_t s = (cudaStream_t)stream;
@@ -644,6 +645,21 @@ cgtp_status cgtp_plan_set_checks(cgtp_plan plan, int flags) {
   if (flags & ~CGTP_CHECK_GRAPH) return fail(CGTP_ERR_SIZE, "unknown check flags");
   reinterpret_cast<Plan*>(plan)->checks.store(flags);
   return CGTP_OK;
+}
+
+cgtp_status cgtp_validate_graph(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                                const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
+                                const int32_t* perm_T, cgtp_stream stream) {
+  NvtxRange nvtx_range("cgtp_validate_graph");
+  if (!plan) return fail(CGTP_ERR_NULL, "plan is NULL");
+  Plan* P = reinterpret_cast<Plan*>(plan);
+  if (n_recv < 0 || n_send < 0 || E < 0 || n_recv >= (int64_t(1) << 31) ||
+      n_send >= (int64_t(1) << 31) || E >= (int64_t(1) << 31) - 1)
+    return fail(CGTP_ERR_SIZE, "sizes out of range");
+  if ((rowptr_T == nullptr) != (perm_T == nullptr)) return fail(CGTP_ERR_NULL, "rowptr_T and perm_T go together");
+  cgtp_status st = check_device(*P);
+  if (st != CGTP_OK) return st;
+  return check_graph(*P, n_recv, n_send, E, rowptr, col, rowptr_T, perm_T, stream, true);
 }
 
 cgtp_status cgtp_plan_set_timing(cgtp_plan plan, int enable) {

@@ -227,7 +227,8 @@ cgtp_status check_plan_device(const Plan& P);
 // result and returns CGTP_ERR_INVALID_CSR (with the failed checks in the
 // message) before any kernel reads through the graph.  OK when checks are off.
 cgtp_status check_graph(Plan& P, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
-                        const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, cgtp_stream stream);
+                        const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, cgtp_stream stream,
+                        bool always = false);
 // Host checks of a backward call (sizes, device, alignment, required pointers).
 cgtp_status backward_validate(const Plan& P, int64_t n_recv, int64_t n_send, int64_t E, const int32_t* rowptr,
                               const int32_t* col, const int32_t* rowptr_T, const int32_t* perm_T, const float* x,

@@ -239,6 +239,19 @@ cgtp_status cgtp_plan_set_timing(cgtp_plan plan, int enable);
  * Errors: NULL, SIZE (unknown flags). */
 #define CGTP_CHECK_GRAPH 1
 cgtp_status cgtp_plan_set_checks(cgtp_plan plan, int flags);
+
+/* The same device graph checks once, whatever the plan's flags: rowptr
+ * [n_recv+1] runs non-decreasing from 0 to E and every col [E] lies in
+ * [0, n_send); when rowptr_T [n_send+1] and perm_T [E] are both given, they
+ * form the sender lists as above (both NULL: not checked).  On the stream;
+ * the call waits for the result, so it is refused under stream capture
+ * (CGTP_ERR_CUDA).  A caller that builds a graph once and calls the
+ * convolutions many times can validate it here instead of turning the
+ * per-call checks on.  Errors: NULL, SIZE, INVALID_CSR (naming the failed
+ * checks), CUDA. */
+cgtp_status cgtp_validate_graph(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
+                                const int32_t* rowptr, const int32_t* col, const int32_t* rowptr_T,
+                                const int32_t* perm_T, cgtp_stream stream);
 cgtp_status cgtp_plan_kernel_times(cgtp_plan plan, int max, char* names, double* ms,
                                    int64_t* launches, int* n);
 

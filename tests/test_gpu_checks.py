@@ -100,6 +100,32 @@ def test_graph_checks_refuse_bad_graphs(tiny):
         plan.set_checks(False)
 
 
+def test_validate_graph(tiny):
+    """cgtp_validate_graph runs the same checks once, whatever the plan's
+    flags: a valid graph passes, a bad col, rowptr or perm_T is named."""
+    w, plan, d = tiny
+    T = d["T"]
+    plan.validate_graph(T(d["rowptr"]), T(d["col"]), w.N)
+    plan.validate_graph(T(d["rowptr"]), T(d["col"]), w.N, T(d["rpt"]), T(d["perm"]))
+    col = d["col"].copy()
+    col[7] = w.N
+    with pytest.raises(C().CgtpError) as e:
+        plan.validate_graph(T(d["rowptr"]), T(col), w.N)
+    assert e.value.status == 7 and "col" in str(e.value)
+    rp = d["rowptr"].copy()
+    rp[10], rp[11] = rp[11], rp[10]
+    with pytest.raises(C().CgtpError) as e:
+        plan.validate_graph(T(rp), T(d["col"]), w.N)
+    assert e.value.status == 7 and "rowptr decreases" in str(e.value)
+    perm = d["perm"].copy()
+    a, b = d["rpt"][3], d["rpt"][40]
+    perm[a], perm[b] = perm[b], perm[a]
+    with pytest.raises(C().CgtpError) as e:
+        plan.validate_graph(T(d["rowptr"]), T(d["col"]), w.N, T(d["rpt"]), T(perm))
+    assert e.value.status == 7 and "perm_T" in str(e.value)
+    _valid_calls(w, plan, d)  # the plan's own calls are unaffected
+
+
 def test_checks_flags_are_validated(tiny):
     w, plan, d = tiny
     with pytest.raises(C().CgtpError) as e:
