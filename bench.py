@@ -529,7 +529,7 @@ def run_cgtp(args, rank, world, local_rank):
                            "algorithmic_bytes": dbl_bytes, "achieved_gbs": dbl_bytes / (dbl_ms * 1e-3) / 1e9,
                            "vs_step": dbl_ms / ms_step_local,
                            "path": ("tangent backward + one plain and two accumulating forwards"
-                                    if "cgtp_fwd_acc" in plan.describe() else
+                                    if "double backward forward=sum" in plan.describe() else
                                     "tangent kernels (one forward, one backward pass)") if tangent else
                                    "composition of forwards and backwards",
                            "what": "double_backward with h_x, h_W, h_Y, after the step (not in it)",

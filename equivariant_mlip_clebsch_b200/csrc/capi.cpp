@@ -372,14 +372,22 @@ static bool ensure_tangent(Plan& P) {
     P.tan_msg = "no paths";
     return false;
   }
-  // gg_out: the tangent forward, or (packed plans, where the tangent
-  // forward's doubled per-edge work on a shallower ring measured slower than
-  // three forwards: Lmax 3 1773 us against 3 x 453) the sum of one plain and
-  // two accumulating forwards
-  if (P.dbwd_fwd_sum < 0) P.dbwd_fwd_sum = P.fcfg.packed ? 1 : 0;
-  std::string fsrc, bsrc;
-  cgtp_status st = P.dbwd_fwd_sum ? build_forward_accumulate(P, P.fwd_acc, &fsrc)
-                                  : build_forward_tangent(P, P.fwd_tan, &fsrc);
+  // gg_out: the tangent forward, or the sum of one plain and two
+  // accumulating forwards.  Which is faster depends on the plan (Lmax 3: the
+  // tangent forward 1773 us against 3 x 453; Case 5: 1019 against 1193), so
+  // both are built unless CGTP_DBWD_FWD fixes one, and the first double
+  // backward timed outside stream capture chooses (dbwd_fwd_sum).
+  std::string fsrc, asrc, bsrc;
+  cgtp_status st = CGTP_OK;
+  if (P.dbwd_fwd_sum != 1) {
+    st = build_forward_tangent(P, P.fwd_tan, &fsrc);
+    if (st != CGTP_OK && P.dbwd_fwd_sum < 0) {  // e.g. doubled stages too large: the sum remains
+      jit_unload(P.fwd_tan);
+      P.dbwd_fwd_sum = 1;
+      st = CGTP_OK;
+    }
+  }
+  if (st == CGTP_OK && P.dbwd_fwd_sum != 0) st = build_forward_accumulate(P, P.fwd_acc, &asrc);
   if (st == CGTP_OK) st = build_backward_tangent(P, P.bwd_tan, &bsrc);
   if (st != CGTP_OK) {
     P.tan_msg = cgtp_last_error();
@@ -390,8 +398,9 @@ static bool ensure_tangent(Plan& P) {
     return false;
   }
   if (const char* d = std::getenv("CGTP_DUMP_SOURCE")) {
-    const char* fname = P.dbwd_fwd_sum ? "/fwd_acc.cu" : "/fwd_tan.cu";
-    for (auto [name, src] : {std::pair<const char*, std::string*>{fname, &fsrc}, {"/bwd_tan.cu", &bsrc}}) {
+    for (auto [name, src] : {std::pair<const char*, std::string*>{"/fwd_tan.cu", &fsrc}, {"/fwd_acc.cu", &asrc},
+                             {"/bwd_tan.cu", &bsrc}}) {
+      if (src->empty()) continue;
       if (FILE* f = std::fopen((std::string(d) + name).c_str(), "w")) {
         std::fputs(src->c_str(), f);
         std::fclose(f);
@@ -605,6 +614,9 @@ cgtp_status cgtp_plan_describe(cgtp_plan plan, char* buf, size_t n, size_t* need
          std::to_string(q.u0) + " R=" + std::to_string(q.R) + " ph=" + std::to_string(q.ph) + "/" +
          std::to_string(q.nph) + " cost=" + std::to_string((int)q.cost) + "\n";
   }
+  if (P->tan_state > 0)
+    t += std::string("double backward forward=") +
+         (P->dbwd_fwd_sum < 0 ? "undecided" : P->dbwd_fwd_sum ? "sum" : "tangent") + "\n";
   for (const JitKernel* k : {&P->fwd_tan, &P->fwd_acc, &P->bwd_tan}) {  // double-backward kernels, once built
     if (k->name.empty()) continue;
     char hx[64];
@@ -779,23 +791,56 @@ cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send,
     // (h_x, h_Y, h_W) of the forward and of the backward at fixed grad_out
     int nr = (int)n_recv;
     const int32_t* no_eid = nullptr;
-    if (gg_out && P->dbwd_fwd_sum == 1) {
-      // the forward is trilinear: its derivative is the sum of three
-      // forwards, each with one input replaced by its direction (the first
-      // writes gg_out, the other two add to it)
-      st = forward_impl(plan, n_recv, n_send, E, rowptr, col, h_x, Y, W, nullptr, gg_out, stream, false);
-      if (st != CGTP_OK) return st;
-      const float* ins[2][3] = {{x, h_Y, W}, {x, Y, h_W}};
-      for (auto& in : ins) {
-        void* args[] = {&rowptr, &col, &in[0], &in[1], &in[2], &no_eid, &gg_out, &P->d_fwd_ent, &nr, &P->d_err};
-        TimedScope ts(*P, 8, cs);
-        st = jit_launch(P->fwd_acc, dim3(persistent_grid(P->fwd_acc.blocks_per_sm, P->num_sms, n_recv)), args, cs);
-        if (st != CGTP_OK) return st;
+    if (gg_out) {
+      // d grad_out along (h_x, h_Y, h_W): the tangent forward, or (the
+      // forward is trilinear) one plain forward with h_x plus two
+      // accumulating forwards with h_Y and h_W
+      auto run_tangent = [&]() -> cgtp_status {
+        void* args[] = {&rowptr, &col, &x, &Y, &W, &no_eid, &gg_out, &P->d_fwd_ent, &nr, &P->d_err, &h_x, &h_Y, &h_W};
+        TimedScope ts(*P, 6, cs);
+        return jit_launch(P->fwd_tan, dim3(persistent_grid(P->fwd_tan.blocks_per_sm, P->num_sms, n_recv)), args, cs);
+      };
+      auto run_sum = [&]() -> cgtp_status {
+        cgtp_status r = forward_impl(plan, n_recv, n_send, E, rowptr, col, h_x, Y, W, nullptr, gg_out, stream, false);
+        const float* ins[2][3] = {{x, h_Y, W}, {x, Y, h_W}};
+        for (auto& in : ins) {
+          if (r != CGTP_OK) break;
+          void* args[] = {&rowptr, &col, &in[0], &in[1], &in[2], &no_eid, &gg_out, &P->d_fwd_ent, &nr, &P->d_err};
+          TimedScope ts(*P, 8, cs);
+          r = jit_launch(P->fwd_acc, dim3(persistent_grid(P->fwd_acc.blocks_per_sm, P->num_sms, n_recv)), args, cs);
+        }
+        return r;
+      };
+      int mode = P->dbwd_fwd_sum.load();
+      if (mode < 0) {
+        cudaStreamCaptureStatus capst = cudaStreamCaptureStatusNone;
+        CGTP_CUDA_TRY(cudaStreamIsCapturing(cs, &capst));
+        if (capst != cudaStreamCaptureStatusNone) {
+          mode = 0;  // no timing under capture: the tangent forward, undecided
+        } else {
+          // time each way once on this call's inputs, keep the faster; the
+          // chosen one then runs last, so every call's gg_out comes from it
+          std::lock_guard<std::mutex> g(P->tan_mu);
+          if (P->dbwd_fwd_sum < 0) {
+            cudaEvent_t ev[3];
+            for (auto& e : ev) CGTP_CUDA_TRY(cudaEventCreate(&e));
+            cudaEventRecord(ev[0], cs);
+            st = run_tangent();
+            cudaEventRecord(ev[1], cs);
+            if (st == CGTP_OK) st = run_sum();
+            cudaEventRecord(ev[2], cs);
+            float t_tan = 0.f, t_sum = 0.f;
+            if (st == CGTP_OK && cudaEventSynchronize(ev[2]) == cudaSuccess &&
+                cudaEventElapsedTime(&t_tan, ev[0], ev[1]) == cudaSuccess &&
+                cudaEventElapsedTime(&t_sum, ev[1], ev[2]) == cudaSuccess)
+              P->dbwd_fwd_sum = t_sum < t_tan ? 1 : 0;
+            for (auto& e : ev) cudaEventDestroy(e);
+            if (st != CGTP_OK) return st;
+          }
+          mode = std::max(0, P->dbwd_fwd_sum.load());
+        }
       }
-    } else if (gg_out) {
-      void* args[] = {&rowptr, &col, &x, &Y, &W, &no_eid, &gg_out, &P->d_fwd_ent, &nr, &P->d_err, &h_x, &h_Y, &h_W};
-      TimedScope ts(*P, 6, cs);
-      st = jit_launch(P->fwd_tan, dim3(persistent_grid(P->fwd_tan.blocks_per_sm, P->num_sms, n_recv)), args, cs);
+      st = mode == 1 ? run_sum() : run_tangent();
       if (st != CGTP_OK) return st;
     }
     if (gx || gW || gY) {

@@ -1031,7 +1031,7 @@ cgtp_status build_backward_tangent(Plan& P, JitKernel& out, std::string* src_out
     K.rec_max = std::max(K.rec_max, P.bwd_ent_begin[k + 1] - P.bwd_ent_begin[k]);
   bool fixed = false;
   const int mb0 = initial_min_blocks(K.smem, &fixed);
-  const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
+  const int mb_floor = fixed ? mb0 : 1;  // down to one CTA while the doubled roles spill
   const std::string name = "cgtp_bwd_tan";
   std::string src;
   JitBinary bin;

@@ -104,10 +104,14 @@ static std::string gen_fwd_generic(const Plan& P, const std::vector<SliceLayout>
     shape_of[ri] = (int)(it - shapes.begin());
     if (it == shapes.end()) shapes.push_back(key);
   }
+  const bool pk = K.packed;  // float2 accumulators of m3 pairs (fpath2)
   for (size_t k = 0; k < shapes.size(); ++k) {
     const int N1 = std::get<0>(shapes[k]), N3 = std::get<1>(shapes[k]);
+    const int NA = pk ? (N3 + 1) / 2 : N3;  // accumulators
+    const std::string FT = pk ? "float2" : "float";
     const bool full = std::get<2>(shapes[k]);
-    o << "// shape " << k << ": one path " << N1 << " x " << N3 << ", one channel per lane\n"
+    o << "// shape " << k << ": one path " << N1 << " x " << N3 << ", one channel per lane" << (pk ? ", packed" : "")
+      << "\n"
       << "__device__ __noinline__ void fgen_" << k
       << "(const int* __restrict__ rowptr, int n_recv, float* __restrict__ out, int* __restrict__ err,\n"
          "    unsigned char* smem, int u0, int chs, int choff, int wst, int xst, int ooff, int mul, int* qp) {\n"
@@ -119,8 +123,9 @@ static std::string gen_fwd_generic(const Plan& P, const std::vector<SliceLayout>
          "  int q = *qp;\n"
          "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
          "  const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
-         "  float acc[" << N3 << "];\n"
-         "#pragma unroll\n  for (int k = 0; k < " << N3 << "; ++k) acc[k] = 0.f;\n"
+         "  " << FT << " acc[" << NA << "];\n"
+         "#pragma unroll\n  for (int k = 0; k < " << NA << "; ++k) acc[k] = " << (pk ? "make_float2(0.f, 0.f)" : "0.f")
+      << ";\n"
          "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
          "    const int s = q % NSTAGE;\n"
          "    if (!stage_ready(full0, s, (q / NSTAGE) & 1)) { if (lane == 0) atomicOr(err, 10); *qp = -1; return; }\n"
@@ -130,25 +135,29 @@ static std::string gen_fwd_generic(const Plan& P, const std::vector<SliceLayout>
          "    const float* sX = reinterpret_cast<const float*>(st + OFF_X) + xst;\n"
          "    const float* sC = reinterpret_cast<const float*>(st + OFF_CH) + choff;\n"
          "#pragma unroll 1\n    for (int b = 0; b < nb; ++b) {\n"
-         "      float xv[1][" << N1 << "], w[1];\n"
-         "#pragma unroll\n      for (int m1 = 0; m1 < " << N1 << "; ++m1) xv[0][m1] = ok ? sX[b * XS + u * " << N1
-      << " + m1] : 0.f;\n"
-         "      w[0] = ok ? sW[b * WS + u] : 0.f;\n";
+         "      " << FT << " xv[1][" << N1 << "];\n      float w[1];\n"
+         "#pragma unroll\n      for (int m1 = 0; m1 < " << N1 << "; ++m1) "
+      << (pk ? "{ const float v = ok ? sX[b * XS + u * " + std::to_string(N1) + " + m1] : 0.f; xv[0][m1] = make_float2(v, v); }"
+             : "xv[0][m1] = ok ? sX[b * XS + u * " + std::to_string(N1) + " + m1] : 0.f;")
+      << "\n      w[0] = ok ? sW[b * WS + u] : 0.f;\n";
+    const std::string fp = pk ? "2<" : "<";
     if (K.tangent)
-      o << "      float xtv[1][" << N1 << "], wt[1];\n"
+      o << "      " << FT << " xtv[1][" << N1 << "];\n      float wt[1];\n"
            "      const float* sXt = reinterpret_cast<const float*>(st + OFF_XT) + xst;\n"
            "      const float* sWt = reinterpret_cast<const float*>(st + OFF_WT) + wst;\n"
            "      const float* sCt = reinterpret_cast<const float*>(st + OFF_CHT) + choff;\n"
-           "#pragma unroll\n      for (int m1 = 0; m1 < " << N1 << "; ++m1) xtv[0][m1] = ok ? sXt[b * XS + u * " << N1
-        << " + m1] : 0.f;\n"
-           "      wt[0] = ok ? sWt[b * WS + u] : 0.f;\n"
-           "      fpath_tan<" << N1 << "," << N3 << ",1,0," << N3 << ">(acc, sC + b * chs, sCt + b * chs, xv, xtv, w, wt);\n";
+           "#pragma unroll\n      for (int m1 = 0; m1 < " << N1 << "; ++m1) "
+        << (pk ? "{ const float v = ok ? sXt[b * XS + u * " + std::to_string(N1) + " + m1] : 0.f; xtv[0][m1] = make_float2(v, v); }"
+               : "xtv[0][m1] = ok ? sXt[b * XS + u * " + std::to_string(N1) + " + m1] : 0.f;")
+        << "\n      wt[0] = ok ? sWt[b * WS + u] : 0.f;\n"
+           "      fpath_tan" << fp << N1 << "," << N3 << ",1,0," << NA << ">(acc, sC + b * chs, sCt + b * chs, xv, xtv, w, wt);\n";
     else
-      o << "      fpath<" << N1 << "," << N3 << ",1,0," << N3 << ">(acc, sC + b * chs, xv, w);\n";
+      o << "      fpath" << fp << N1 << "," << N3 << ",1,0," << NA << ">(acc, sC + b * chs, xv, w);\n";
     o << "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n"
          "  if (ok) {\n    float* orow = out + (size_t)i * DOUT + ooff;\n"
-         "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) orow[u * " << N3 << " + m3] "
-      << (K.accumulate ? "+=" : "=") << " acc[m3];\n  }\n"
+         "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) "
+      << (K.accumulate ? "red_add(&orow[u * " : "orow[u * ") << N3 << " + m3]" << (K.accumulate ? ", " : " = ")
+      << (pk ? "(m3 & 1) ? acc[m3 >> 1].y : acc[m3 >> 1].x" : "acc[m3]") << (K.accumulate ? ")" : "") << ";\n  }\n"
          "  }\n  *qp = q;\n}\n";
   }
   gen_fwd_idle(o);
@@ -291,12 +300,13 @@ static std::string gen_fwd_source(const Plan& P, const std::vector<SliceLayout>&
       const Path& p = P.paths[pi];
       const int N3 = 2 * p.l3 + 1;
       o << "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) if (ok[r]) {\n    const int u = u0 + r * 32 + lane;\n"
-        << "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) orow[" << p.o_off << " + u * " << N3
-        << " + m3] " << (K.accumulate ? "+= " : "= ")
+        << "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) " << (K.accumulate ? "red_add(&orow[" : "orow[")
+        << p.o_off << " + u * " << N3
+        << " + m3]" << (K.accumulate ? ", " : " = ")
         << (pk ? "(m3 & 1) ? acc[" + std::to_string(A) + " + r * " + std::to_string(np(pi)) + " + (m3 >> 1)].y : acc[" +
                      std::to_string(A) + " + r * " + std::to_string(np(pi)) + " + (m3 >> 1)].x"
                : "acc[" + std::to_string(A) + " + r * " + std::to_string(N3) + " + m3]")
-        << ";\n  }\n";
+        << (K.accumulate ? ")" : "") << ";\n  }\n";
       A += R * np(pi);
     }
     o << "  }\n  *qp = q;\n}\n";
@@ -586,7 +596,7 @@ cgtp_status build_forward(Plan& P) {
   // l <= 2 inputs lose (Lmax 2 35 -> 43 us, Lmax 2 wide 137 -> 148 us).
   int lmax_in = 0;
   for (const Irrep& h : P.in) lmax_in = std::max(lmax_in, h.l);
-  F.packed = !F.generic && (P.fwd_packed < 0 ? lmax_in >= 3 : P.fwd_packed == 1);
+  F.packed = P.fwd_packed < 0 ? !F.generic && lmax_in >= 3 : P.fwd_packed == 1;
   std::vector<SliceLayout> SL = forward_slices(P, F.packed);
   KernelShape K;
   K.S = F.S;
@@ -664,7 +674,7 @@ cgtp_status build_forward_tangent(Plan& P, JitKernel& out, std::string* src_out)
   if (K.smem > 227 * 1024) return fail(CGTP_ERR_SIZE, "tangent forward needs too much shared memory");
   bool fixed = false;
   const int mb0 = initial_min_blocks(K.smem, &fixed);
-  const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
+  const int mb_floor = fixed ? mb0 : 1;  // down to one CTA while the doubled roles spill
   const std::string name = "cgtp_fwd_tan";
   std::string src;
   JitBinary bin;

@@ -168,10 +168,11 @@ struct Plan {
   // forward roles with float2 accumulators and packed FMAs: -1 chosen by the
   // planner, 0 off, 1 on (CGTP_FWD_PACKED at plan creation)
   int fwd_packed = -1;
-  // double backward: gg_out as three forwards summed (-1: the planner's
-  // choice, 0: the tangent forward, 1: the sum; CGTP_DBWD_FWD=tangent|sum at
-  // plan creation)
-  int dbwd_fwd_sum = -1;
+  // double backward: gg_out from the tangent forward (0) or as one plain and
+  // two accumulating forwards (1); -1: chosen by timing both on the first
+  // all-cotangent call outside stream capture (CGTP_DBWD_FWD=tangent|sum at
+  // plan creation fixes it)
+  std::atomic<int> dbwd_fwd_sum{-1};
   // CG-first backward roles with rows m1 paired in float2 halves and packed
   // FMAs (CGTP_BWD_PACKED=1 at plan creation)
   bool bwd_packed = false;

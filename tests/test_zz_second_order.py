@@ -32,6 +32,7 @@ def _compare(plan, P, d, host, h, dev):
     for name, a, b in zip(("d grad_out", "dx", "dW", "dY"), got, ref):
         assert_close(a.cpu().numpy(), b, name)
     plan.check_device_error()
+    return got
 
 
 @pytest.mark.parametrize("keys", [("h_x", "h_W", "h_Y"), ("h_x",), ("h_W",), ("h_Y",), ("h_W", "h_Y")])
@@ -58,6 +59,23 @@ def test_double_backward_forward_paths(hid, edge, fwd, dev, monkeypatch):
     _random_graph_case(plan, hid, edge, out, ("h_x", "h_W", "h_Y"), dev)
 
 
+def test_double_backward_first_call_chooses(dev):
+    """With both ways of forming d grad_out built, the first call times them
+    and keeps the faster; that call and the next give the same bits."""
+    hid, edge = "32x0e+17x1o+8x2e+33x3o", "1x0e+1x1o+1x2e+1x3o"
+    out = _out_irreps(hid, edge)
+    from equivariant_mlip_clebsch_b200 import cgtp as C
+    plan = C.Plan(hid, edge, out, 6)
+    assert plan.prepare_double_backward()
+    assert "double backward forward=undecided" in plan.describe()
+    first = _random_graph_case(plan, hid, edge, out, ("h_x", "h_W", "h_Y"), dev)
+    desc = plan.describe()
+    assert "double backward forward=tangent" in desc or "double backward forward=sum" in desc
+    second = _random_graph_case(plan, hid, edge, out, ("h_x", "h_W", "h_Y"), dev)
+    for a, b in zip(first, second):
+        assert torch.equal(a, b)
+
+
 def _random_graph_case(plan, hid, edge, out, keys, dev):
     P = O.enumerate_paths(hid, edge, out)
     rng = np.random.default_rng(11)
@@ -78,7 +96,7 @@ def _random_graph_case(plan, hid, edge, out, keys, dev):
     rpt, perm = C.csr_transpose(rowptr.astype(np.int32), col, n_send)
     d = dict(rowptr=T(rowptr.astype(np.int32), dev), col=T(col, dev), rpt=T(rpt, dev), perm=T(perm, dev),
              x=T(host["x"], dev), Y=T(Y, dev), W=T(host["W"], dev), g=T(host["g"], dev))
-    _compare(plan, P, d, host, h, dev)
+    return _compare(plan, P, d, host, h, dev)
 
 
 @pytest.mark.parametrize("name", ["tiny", "lmax2"])
