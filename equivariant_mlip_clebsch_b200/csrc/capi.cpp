@@ -197,7 +197,6 @@ cgtp_status cgtp_plan_create(const char* irreps_in, const char* irreps_edge, con
       if (std::string(v) == "tangent") P->dbwd_fwd_sum = 0;
       if (std::string(v) == "sum") P->dbwd_fwd_sum = 1;
     }
-    if (const char* v = std::getenv("CGTP_BWD_PACKED"); v && (*v == '0' || *v == '1')) P->bwd_packed = *v == '1';
     st = build_forward(*P);  // leaves the forward compiling on a host thread
     if (st == CGTP_OK) st = build_backward(*P);
     if (st == CGTP_OK)

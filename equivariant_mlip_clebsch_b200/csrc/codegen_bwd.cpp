@@ -69,19 +69,11 @@ std::string flt(double v) {
 // The tangent form (double backward) adds the directional derivatives along
 // (xt, Yt, wt): st = sum_m2 Yt t, dW += xt s + x st, msg += wt s + w st and
 // dY += (w xt + wt x) t.
-// Packed form (K.packed, l1 >= 1, not tangent): rows m1 = 2h and 2h + 1 go
-// as the halves of float2 values, so s, dW, msg, w x and the dY partial take
-// one packed FMA (__ffma2_rn) for both rows; t of the two rows is formed by
-// scalar FMAs into the halves (zero where a row has no term, and for the
-// missing row of an odd count).  dW and the dY partials sum the two halves at
-// the end: the same products in another order of summation.
 void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K, const BwdRole& r,
                            const SliceLayout& sl, size_t k, const std::string& params) {
   const Irrep& h = P.in[r.irrep];
   const int N1 = 2 * h.l + 1, R = r.R, MUL = h.mul;
   const bool tan = K.tangent;
-  const bool pk = K.packed && !tan && N1 > 1;
-  const int NH = (N1 + 1) / 2;  // row pairs (packed form)
   auto pow2 = [](int n) { int v = 1; while (v < n) v <<= 1; return v; };
   const bool combined = P.D_e <= 32;
   if (!combined && R != 1) {
@@ -126,30 +118,19 @@ void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K,
             : "")
     << "      float* dWrow = dW ? dW + (size_t)(eid ? __ldg(eid + e) : e) * NU : nullptr;\n"
     << "      float* sdy = want_dy ? sdyw + b * DE : nullptr;\n";
-  const std::string ZT = pk ? "float2" : "float", Z0 = pk ? "make_float2(0.f, 0.f)" : "0.f";
   if (combined)
-    o << "      " << ZT << " z[" << VZ << "];\n#pragma unroll\n      for (int t = 0; t < " << VZ << "; ++t) z[t] = "
-      << Z0 << ";\n";
+    o << "      float z[" << VZ << "];\n#pragma unroll\n      for (int t = 0; t < " << VZ << "; ++t) z[t] = 0.f;\n";
   o << "#pragma unroll 1\n      for (int r = 0; r < " << R << "; ++r) {\n"
     << "      const int u = u0 + r * 32 + lane;\n"
     << "      const bool ok = " << (MUL % (32 * R) == 0 ? std::string("true") : "u < " + std::to_string(MUL))
     << ";  // every lane holds a channel when the blocks are full\n"
-    ;
-  if (pk) {
-    o << "      float2 xv[" << NH << "], mx[" << NH << "];\n";
-    for (int hh = 0; hh < NH; ++hh)
-      o << "      xv[" << hh << "] = make_float2(ok ? xr[u * " << N1 << " + " << 2 * hh << "] : 0.f, "
-        << (2 * hh + 1 < N1 ? "ok ? xr[u * " + sN1 + " + " + std::to_string(2 * hh + 1) + "] : 0.f" : std::string("0.f"))
-        << ");\n      mx[" << hh << "] = make_float2(0.f, 0.f);\n";
-  } else {
-    o << "      float xv[" << N1 << "], mx[" << N1 << "];\n"
-      << (tan ? "      float xtv[" + sN1 + "];\n" : "")
-      << "#pragma unroll\n      for (int m1 = 0; m1 < " << N1 << "; ++m1) {\n"
-      << "        mx[m1] = 0.f;\n"
-      << "        xv[m1] = ok ? xr[u * " << N1 << " + m1] : 0.f;\n"
-      << (tan ? "        xtv[m1] = ok ? xtr[u * " + sN1 + " + m1] : 0.f;\n" : "")
-      << "      }\n";
-  }
+    << "      float xv[" << N1 << "], mx[" << N1 << "];\n"
+    << (tan ? "      float xtv[" + sN1 + "];\n" : "")
+    << "#pragma unroll\n      for (int m1 = 0; m1 < " << N1 << "; ++m1) {\n"
+    << "        mx[m1] = 0.f;\n"
+    << "        xv[m1] = ok ? xr[u * " << N1 << " + m1] : 0.f;\n"
+    << (tan ? "        xtv[m1] = ok ? xtr[u * " + sN1 + " + m1] : 0.f;\n" : "")
+    << "      }\n";
   std::vector<char> l2seen(P.L + 1, 0);
   size_t q = 0;
   while (q < ps.size()) {
@@ -159,16 +140,11 @@ void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K,
     l2seen[l2] = 1;
     o << "      {\n";
     if (!combined)
-      o << "        " << ZT << " z[" << pow2(N2) << "];\n#pragma unroll\n        for (int t = 0; t < " << pow2(N2)
-        << "; ++t) z[t] = " << Z0 << ";\n";
-    // this degree's harmonics of the edge (the same for every lane; in both
-    // halves for the packed form)
-    if (pk)
-      o << "        float2 yl[" << N2 << "];\n#pragma unroll\n        for (int m2 = 0; m2 < " << N2
-        << "; ++m2) { const float v = yr[" << l2 * l2 << " + m2]; yl[m2] = make_float2(v, v); }\n";
-    else
-      o << "        float yl[" << N2 << "];\n#pragma unroll\n        for (int m2 = 0; m2 < " << N2
-        << "; ++m2) yl[m2] = yr[" << l2 * l2 << " + m2];\n";
+      o << "        float z[" << pow2(N2) << "];\n#pragma unroll\n        for (int t = 0; t < " << pow2(N2)
+        << "; ++t) z[t] = 0.f;\n";
+    // this degree's harmonics of the edge (the same for every lane)
+    o << "        float yl[" << N2 << "];\n#pragma unroll\n        for (int m2 = 0; m2 < " << N2
+      << "; ++m2) yl[m2] = yr[" << l2 * l2 << " + m2];\n";
     if (tan)
       o << "        float ytl[" << N2 << "];\n#pragma unroll\n        for (int m2 = 0; m2 < " << N2
         << "; ++m2) ytl[m2] = ytr[" << l2 * l2 << " + m2];\n";
@@ -181,47 +157,9 @@ void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K,
         << " + u * " << N3 << " + m3] : 0.f;\n"
         << "          const float w = ok ? wr[" << sl.w_st.at(pi) << " + u] : 0.f;\n"
         << (tan ? "          const float wt = ok ? wtr[" + std::to_string(sl.w_st.at(pi)) + " + u] : 0.f;\n" : "")
-        << (pk ? "          const float2 w2 = make_float2(w, w);\n          float2 d = make_float2(0.f, 0.f);\n"
-               : "          float d = 0.f;\n");
+        << "          float d = 0.f;\n";
       const double* C = P.coeff.data() + p.c_off;
-      // t[m1][m2] as an expression of gv (empty when the row has no term)
-      auto texpr = [&](int m1, int m2) {
-        std::vector<std::pair<int, double>> t;
-        for (int m3 = 0; m3 < N3; ++m3) {
-          const double c = C[((size_t)m1 * n2 + m2) * N3 + m3];
-          if (c != 0.0) t.push_back({m3, c});
-        }
-        if (t.empty()) return std::string();
-        std::string e = flt(t[0].second) + " * gv[" + std::to_string(t[0].first) + "]";
-        for (size_t c = 1; c < t.size(); ++c)
-          e = "fmaf(" + flt(t[c].second) + ", gv[" + std::to_string(t[c].first) + "], " + e + ")";
-        return e;
-      };
-      for (int hh = 0; pk && hh < NH; ++hh) {  // packed: rows 2hh and 2hh + 1
-        const int ra = 2 * hh, rb = 2 * hh + 1;
-        std::vector<int> m2s;
-        std::ostringstream tdef;
-        for (int m2 = 0; m2 < n2; ++m2) {
-          const std::string ea = texpr(ra, m2), eb = rb < N1 ? texpr(rb, m2) : std::string();
-          if (ea.empty() && eb.empty()) continue;
-          m2s.push_back(m2);
-          tdef << "            const float2 t" << m2 << " = make_float2(" << (ea.empty() ? "0.f" : ea) << ", "
-               << (eb.empty() ? "0.f" : eb) << ");\n";
-        }
-        if (m2s.empty()) continue;
-        std::string sv = "__fmul2_rn(yl[" + std::to_string(m2s[0]) + "], t" + std::to_string(m2s[0]) + ")";
-        for (size_t c = 1; c < m2s.size(); ++c)
-          sv = "__ffma2_rn(yl[" + std::to_string(m2s[c]) + "], t" + std::to_string(m2s[c]) + ", " + sv + ")";
-        const std::string xm = "xv[" + std::to_string(hh) + "]", mm = "mx[" + std::to_string(hh) + "]";
-        o << "          {\n" << tdef.str() << "            const float2 s = " << sv << ";\n"
-          << "            d = __ffma2_rn(" << xm << ", s, d);\n"
-          << "            " << mm << " = __ffma2_rn(w2, s, " << mm << ");\n"
-          << "            const float2 wx = __fmul2_rn(w2, " << xm << ");\n";
-        for (int m2 : m2s)
-          o << "            z[" << zo + m2 << "] = __ffma2_rn(wx, t" << m2 << ", z[" << zo + m2 << "]);\n";
-        o << "          }\n";
-      }
-      for (int m1 = 0; !pk && m1 < N1; ++m1) {
+      for (int m1 = 0; m1 < N1; ++m1) {
         std::vector<int> m2s;
         std::ostringstream tdef;
         for (int m2 = 0; m2 < n2; ++m2) {
@@ -261,17 +199,12 @@ void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K,
           o << "            z[" << zo + m2 << "] = fmaf(wx, t" << m2 << ", z[" << zo + m2 << "]);\n";
         o << "          }\n";
       }
-      o << "          if (dWrow && ok) dWrow[" << p.k0 << " + u] = " << (pk ? "d.x + d.y" : "d") << ";\n        }\n";
+      o << "          if (dWrow && ok) dWrow[" << p.k0 << " + u] = d;\n        }\n";
     }
     if (!combined) {
       const int V = pow2(N2), LV = __builtin_ctz(V), sh = 5 - LV;
-      o << "        if (sdy) {\n";
-      if (pk)
-        o << "          float zs[" << V << "];\n#pragma unroll\n          for (int t = 0; t < " << V
-          << "; ++t) zs[t] = z[t].x + z[t].y;\n          const float v = warp_sum_many<" << V << ">(zs, lane);\n";
-      else
-        o << "          const float v = warp_sum_many<" << V << ">(z, lane);\n";
-      o << "          const int c = lane >> " << sh << ";\n"
+      o << "        if (sdy) {\n          const float v = warp_sum_many<" << V << ">(z, lane);\n"
+        << "          const int c = lane >> " << sh << ";\n"
         << "          if ((lane & " << ((1 << sh) - 1) << ") == 0 && c < " << N2 << ") sdy[" << l2 * l2
         << " + c] = v;\n        }\n";
     }
@@ -280,8 +213,7 @@ void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K,
   // the message row segment of this channel block, through the warp's buffer
   o << "      if (msg) {\n"
     << "        float* wbuf = reinterpret_cast<float*>(smem + OFF_WB) + (threadIdx.x >> 5) * WB;\n"
-    << "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) wbuf[lane * " << N1 << " + m1] = "
-    << (pk ? "(m1 & 1) ? mx[m1 >> 1].y : mx[m1 >> 1].x" : "mx[m1]") << ";\n"
+    << "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) wbuf[lane * " << N1 << " + m1] = mx[m1];\n"
     << "        __syncwarp();\n"
     << "        const int nch = min(32, " << MUL << " - u0 - r * 32);\n"
     << "        if (nch > 0) warp_copy_out(msg + (size_t)e * DIN + " << P.x_off[r.irrep] << " + (u0 + r * 32) * "
@@ -295,8 +227,7 @@ void gen_bwd_role_cg_first(std::ostream& o, const Plan& P, const KernelShape& K,
       while (V * 2 <= rest && V * 2 <= 32) V *= 2;
       const int LV = __builtin_ctz(V), sh = 5 - LV;
       o << "        {\n          float zp[" << V << "];\n#pragma unroll\n          for (int t = 0; t < " << V
-        << "; ++t) zp[t] = " << (pk ? "z[" + std::to_string(off) + " + t].x + z[" + std::to_string(off) + " + t].y"
-                                    : "z[" + std::to_string(off) + " + t]") << ";\n"
+        << "; ++t) zp[t] = z[" << off << " + t];\n"
         << "          const float v = warp_sum_many<" << V << ">(zp, lane);\n"
         << "          if ((lane & " << ((1 << sh) - 1) << ") == 0) sdy[" << off << " + (lane >> " << sh
         << ")] = v;\n        }\n";
@@ -825,7 +756,6 @@ cgtp_status build_backward(Plan& P) {
         K.nw = NW;
         K.force_B = B;
         K.no_chat = P.bwd_tform;
-        K.packed = P.bwd_packed;
         int maxr = 0;
         for (int s2 = 0; s2 < ns; ++s2) {
           for (size_t k = 0; k < slices[s2].size(); ++k) {
@@ -876,7 +806,6 @@ cgtp_status build_backward(Plan& P) {
   K.nw = F.nw;
   K.force_B = best.B;
   K.no_chat = P.bwd_tform;
-  K.packed = P.bwd_packed;
   for (int s2 = 0; s2 < F.S; ++s2) {
     for (size_t k = 0; k < best.slices[s2].size(); ++k) {
       const BwdIrrep& wi = best.W[best.slices[s2][k]];

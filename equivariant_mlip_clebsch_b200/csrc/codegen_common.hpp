@@ -85,9 +85,8 @@ struct KernelShape {
   bool accumulate = false;
   // W rows prefetched into L2 this many chunks ahead (0: off)
   int prefetch = 0;
-  // forward: roles with float2 accumulators of m3 pairs and packed FMAs over
-  // an m1-major Chat (fpath2, fpath_tan2); backward: CG-first roles with
-  // pairs of m1 rows in float2 halves
+  // forward roles with float2 accumulators of m3 pairs and packed FMAs over
+  // an m1-major Chat (fpath2, fpath_tan2)
   bool packed = false;
   // backward roles that contract with the CG table and Y directly: no Chat
   // is staged or built (the default; CGTP_BWD_TFORM=0 turns it off)

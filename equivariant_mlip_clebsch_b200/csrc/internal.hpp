@@ -173,9 +173,6 @@ struct Plan {
   // all-cotangent call outside stream capture (CGTP_DBWD_FWD=tangent|sum at
   // plan creation fixes it)
   std::atomic<int> dbwd_fwd_sum{-1};
-  // CG-first backward roles with rows m1 paired in float2 halves and packed
-  // FMAs (CGTP_BWD_PACKED=1 at plan creation)
-  bool bwd_packed = false;
 
   // tangent kernels of the double backward, built on first use (tan_state:
   // 0 not built, 1 ready, -1 unavailable: the composition is used)
