@@ -817,10 +817,14 @@ cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send,
         if (capst != cudaStreamCaptureStatusNone) {
           mode = 0;  // no timing under capture: the tangent forward, undecided
         } else {
-          // time each way once on this call's inputs, keep the faster; the
-          // chosen one then runs last, so every call's gg_out comes from it
+          // run each way once untimed (first launches carry one-time costs),
+          // then time each once on this call's inputs and keep the faster;
+          // the chosen one runs last, so every call's gg_out comes from it
           std::lock_guard<std::mutex> g(P->tan_mu);
           if (P->dbwd_fwd_sum < 0) {
+            st = run_tangent();
+            if (st == CGTP_OK) st = run_sum();
+            if (st != CGTP_OK) return st;
             cudaEvent_t ev[3];
             for (auto& e : ev) CGTP_CUDA_TRY(cudaEventCreate(&e));
             cudaEventRecord(ev[0], cs);

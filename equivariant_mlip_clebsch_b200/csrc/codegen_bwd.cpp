@@ -941,14 +941,19 @@ cgtp_status build_backward_tangent(Plan& P, JitKernel& out, std::string* src_out
     layout_slice(P, SL[s2], true);
   }
   // the largest chunk (at most the plain kernel's) whose doubled stages
-  // leave room for two CTAs per SM; else the largest that fits one
+  // leave room for two CTAs per SM; else the largest that fits one.  Never
+  // below the roles' edge phases: a role takes the edges b of a chunk with
+  // b % nph == ph, so a chunk of fewer than nph edges would leave the roles
+  // of the higher phases without work.
+  int min_B = 1;
+  for (const BwdRole& r : P.bwd_roles) min_B = std::max(min_B, r.nph);
   int pick = 0;
-  for (int B = F.B; B >= 1 && !pick; B /= 2) {
+  for (int B = F.B; B >= min_B && !pick; B /= 2) {
     K.force_B = B;
     plan_layout(P, SL, K, true);
     if (2 * (K.smem + 1024) <= 228 * 1024) pick = B;
   }
-  for (int B = F.B; B >= 1 && !pick; B /= 2) {
+  for (int B = F.B; B >= min_B && !pick; B /= 2) {
     K.force_B = B;
     plan_layout(P, SL, K, true);
     if (K.smem <= 227 * 1024) pick = B;

@@ -590,13 +590,14 @@ cgtp_status build_forward(Plan& P) {
     for (int pi : r.paths) n += r.R * (2 * P.paths[pi].l3 + 1);
     F.nacc = std::max(F.nacc, n);
   }
-  // Packed roles (float2 accumulators of m3 pairs, m1-major Chat) for coarse
-  // plans with a hidden irrep of l >= 3, whose long m3 rows pack well.
-  // Measured on B200: Lmax 3 470 -> 433 us, Case 5 470 -> 402 us; plans with
-  // l <= 2 inputs lose (Lmax 2 35 -> 43 us, Lmax 2 wide 137 -> 148 us).
+  // Packed roles (float2 accumulators of m3 pairs, m1-major Chat) for plans
+  // with a hidden irrep of l >= 3, whose long m3 rows pack well.  Measured on
+  // B200: Lmax 3 470 -> 433 us, Case 5 470 -> 402 us, Lmax 6 2035 -> 1631 us,
+  // Case 6 821 -> 721 us, Case 4 unchanged; plans with l <= 2 inputs lose
+  // (Lmax 2 35 -> 43 us, Lmax 2 wide 137 -> 148 us).
   int lmax_in = 0;
   for (const Irrep& h : P.in) lmax_in = std::max(lmax_in, h.l);
-  F.packed = P.fwd_packed < 0 ? !F.generic && lmax_in >= 3 : P.fwd_packed == 1;
+  F.packed = P.fwd_packed < 0 ? lmax_in >= 3 : P.fwd_packed == 1;
   std::vector<SliceLayout> SL = forward_slices(P, F.packed);
   KernelShape K;
   K.S = F.S;
@@ -674,7 +675,7 @@ cgtp_status build_forward_tangent(Plan& P, JitKernel& out, std::string* src_out)
   if (K.smem > 227 * 1024) return fail(CGTP_ERR_SIZE, "tangent forward needs too much shared memory");
   bool fixed = false;
   const int mb0 = initial_min_blocks(K.smem, &fixed);
-  const int mb_floor = fixed ? mb0 : 1;  // down to one CTA while the doubled roles spill
+  const int mb_floor = fixed ? mb0 : std::min(mb0, 2);
   const std::string name = "cgtp_fwd_tan";
   std::string src;
   JitBinary bin;
