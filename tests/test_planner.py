@@ -285,6 +285,11 @@ def test_tangent_kernels_copies_and_layout(name, fwd, compile_only, monkeypatch,
     smem = {k: int(v) for k, v in re.findall(r"^(cgtp_fwd_tan|cgtp_fwd_acc|cgtp_bwd_tan) .* smem=(\d+)", desc, re.M)}
     assert set(smem) == set(built) | {"cgtp_bwd_tan"}, smem
     assert ("double backward forward=undecided" in desc) == (fwd == "")
+    # every backward role has edges in the tangent backward's chunks: a role
+    # takes the edges b with b % nph == ph, so the chunk must hold nph edges
+    nph = max(int(v) for v in re.findall(r"^  brole \d+: .* ph=\d+/(\d+)", desc, re.M))
+    nb = int(re.search(r"^#define NB (\d+)", (tmp_path / "bwd_tan.cu").read_text(), re.M).group(1))
+    assert nb >= nph, (nb, nph)
     for f, kname in [(k[5:] + ".cu", k) for k in built] + [("bwd_tan.cu", "cgtp_bwd_tan")]:
         src = (tmp_path / f).read_text()
         assert ("#define TAN 1" in src) == (kname != "cgtp_fwd_acc")
