@@ -604,6 +604,9 @@ cgtp_status build_forward(Plan& P) {
   K.nw = F.nw;
   K.WB = 0;  // output rows go straight from registers to global memory
   K.packed = F.packed;
+  // tuning overrides for the plain forward alone: edges per chunk and ring depth
+  if (const char* v = std::getenv("CGTP_FWD_CHUNK")) K.force_B = std::max(1, std::min(8, std::atoi(v)));
+  if (const char* v = std::getenv("CGTP_FWD_STAGES")) K.force_stages = std::max(2, std::min(6, std::atoi(v)));
   plan_layout(P, SL, K, false);
   F.B = K.B;
   F.stages = K.stages;
