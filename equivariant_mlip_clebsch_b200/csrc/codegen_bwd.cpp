@@ -1,20 +1,25 @@
 // codegen_bwd.cpp -- the backward CGTP convolution kernel, generated per plan.
 //
 // Given g = dL/dout (LunaTP, arXiv 2610.18393, Table 11 lists the backward
-// outputs x-bar, y-bar, w-bar), per edge e = (i <- j), path p, channel u:
+// outputs x-bar, y-bar, w-bar), per edge e = (i <- j), path p, channel u,
+// with Chat[m3][m1] = sum_m2 C[m1][m2][m3] Y[e][l2^2+m2]:
 //   s[m1]  = sum_m3 Chat[m3][m1] g[i][u][m3]
 //   dW[e][k0+u]      = sum_m1 x[j][u][m1] s[m1]   (= sum_m3 g (Chat x)[m3])
 //   msg[e][u][m1]   += W[e][k0+u] s[m1]           (over the paths of the irrep)
 //   dY[e][l2^2+m2]  += sum_{u,m1,m3} C[m1][m2][m3] W[e][k0+u] x[j][u][m1] g[i][u][m3]
 // and dx[j] = sum over the edges leaving j of msg[e] (a second, sender-major
-// pass over the transpose edge list, kernels.cu).
+// pass over the transpose edge list, kernels.cu).  The default roles form
+// these "CG first" (gen_bwd_role_cg_first: t = C g per channel, then s and
+// the dY partial from t and Y, no Chat); the staged-Chat roles (the helper
+// builds Chat per edge in shared memory) remain behind CGTP_BWD_TFORM=0.
 //
 // Execution: persistent CTAs (resident CTAs per SM x SMs) walk the slices
 // in turn; a slice is a group of hidden irreps, chosen with the chunk size and
 // warp count by the planner (build_backward).  Within a slice the TMA warp
 // stages each receiver's grad_out pieces once and, per chunk, the W and x
-// pieces of the slice; the helper warp stages Y, builds Chat and sums the dY
-// partials of released stages.  A consumer owns R blocks of 32 channels of one
+// pieces of the slice; the helper warp stages Y (and builds Chat for the
+// staged-Chat roles) and sums the dY partials of released stages.  A
+// consumer owns R blocks of 32 channels of one
 // irrep (run one after another), ALL its paths (so msg is complete in
 // registers) and the edges b of each chunk with b % nph == ph.  Two variants
 // are compiled: CTAs over receivers blockIdx.x, + gridDim.x, ..., and CTAs

@@ -15,7 +15,13 @@
 // grouped under a register budget per lane (LunaTP's output-component budget,
 // Fig. 3b / Table 7).  Roles with the same irrep and path group share one
 // __noinline__ function with the channel block as an argument.  Wide plans
-// use one-path roles instead, one function per (2l1+1, 2l3+1) shape.
+// use one-path roles instead, one function per (2l1+1, 2l3+1) shape.  Plans
+// with a hidden irrep of l >= 3 use packed roles (fpath2: float2 accumulators
+// of m3 pairs over an m1-major Chat, one packed FMA per m1 and pair).  Two
+// more kernels come from the same generator for the double backward: the
+// tangent forward (every staged piece doubled) and the accumulating forward,
+// which adds its rows to the output with red.global.add (one add per element
+// per launch, so still deterministic).
 #include <algorithm>
 #include <array>
 #include <cmath>
