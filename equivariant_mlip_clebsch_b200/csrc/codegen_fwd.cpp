@@ -100,12 +100,12 @@ static std::string gen_fwd_generic(const Plan& P, const std::vector<SliceLayout>
                                    const std::vector<int>& slice_of) {
   const FwdConfig& F = P.fcfg;
   const int S = K.S, NW = K.nw;
-  std::vector<std::tuple<int, int, bool, int>> shapes;
+  std::vector<std::tuple<int, int, bool>> shapes;
   std::vector<int> shape_of(P.fwd_roles.size(), -1);
   for (size_t ri = 0; ri < P.fwd_roles.size(); ++ri) {
     const FwdRole& r = P.fwd_roles[ri];
     const Path& p = P.paths[r.paths[0]];
-    const auto key = std::make_tuple(2 * P.in[r.irrep].l + 1, 2 * p.l3 + 1, P.in[r.irrep].mul % 32 == 0, r.R);
+    const auto key = std::make_tuple(2 * P.in[r.irrep].l + 1, 2 * p.l3 + 1, P.in[r.irrep].mul % 32 == 0);
     auto it = std::find(shapes.begin(), shapes.end(), key);
     shape_of[ri] = (int)(it - shapes.begin());
     if (it == shapes.end()) shapes.push_back(key);
@@ -113,26 +113,24 @@ static std::string gen_fwd_generic(const Plan& P, const std::vector<SliceLayout>
   const bool pk = K.packed;  // float2 accumulators of m3 pairs (fpath2)
   for (size_t k = 0; k < shapes.size(); ++k) {
     const int N1 = std::get<0>(shapes[k]), N3 = std::get<1>(shapes[k]);
-    const int NA = pk ? (N3 + 1) / 2 : N3;  // accumulators per channel block
+    const int NA = pk ? (N3 + 1) / 2 : N3;  // accumulators
     const std::string FT = pk ? "float2" : "float";
     const bool full = std::get<2>(shapes[k]);
-    const int R = std::get<3>(shapes[k]);
-    o << "// shape " << k << ": one path " << N1 << " x " << N3 << ", " << R << " channel(s) per lane"
-      << (pk ? ", packed" : "") << "\n"
+    o << "// shape " << k << ": one path " << N1 << " x " << N3 << ", one channel per lane" << (pk ? ", packed" : "")
+      << "\n"
       << "__device__ __noinline__ void fgen_" << k
       << "(const int* __restrict__ rowptr, int n_recv, float* __restrict__ out, int* __restrict__ err,\n"
          "    unsigned char* smem, int u0, int chs, int choff, int wst, int xst, int ooff, int mul, int* qp) {\n"
          "  const int lane = threadIdx.x & 31;\n"
          "  const u32 full0 = smem_u32(smem), empty0 = full0 + NSTAGE * 8;\n"
-         "  bool ok[" << R << "];\n"
-         "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) ok[r] = "
-      << (full ? "true" : "u0 + r * 32 + lane < mul") << ";\n"
+         "  const int u = u0 + lane;\n"
+         "  const bool ok = " << (full ? "true" : "u < mul") << ";\n"
          "  (void)mul;\n"
          "  int q = *qp;\n"
          "#pragma unroll 1\n  for (int i = RECV_FIRST; i < RECV_END; i += RECV_STEP) {\n"
          "  const int e0 = EDGE_LO(i), e1 = EDGE_HI(i);\n"
-         "  " << FT << " acc[" << R * NA << "];\n"
-         "#pragma unroll\n  for (int k = 0; k < " << R * NA << "; ++k) acc[k] = " << (pk ? "make_float2(0.f, 0.f)" : "0.f")
+         "  " << FT << " acc[" << NA << "];\n"
+         "#pragma unroll\n  for (int k = 0; k < " << NA << "; ++k) acc[k] = " << (pk ? "make_float2(0.f, 0.f)" : "0.f")
       << ";\n"
          "#pragma unroll 1\n  for (int eb = e0; eb < e1; eb += NB, ++q) {\n"
          "    const int s = q % NSTAGE;\n"
@@ -143,38 +141,29 @@ static std::string gen_fwd_generic(const Plan& P, const std::vector<SliceLayout>
          "    const float* sX = reinterpret_cast<const float*>(st + OFF_X) + xst;\n"
          "    const float* sC = reinterpret_cast<const float*>(st + OFF_CH) + choff;\n"
          "#pragma unroll 1\n    for (int b = 0; b < nb; ++b) {\n"
-         "      " << FT << " xv[" << R << "][" << N1 << "];\n      float w[" << R << "];\n"
-         "#pragma unroll\n      for (int r = 0; r < " << R << "; ++r) {\n"
-         "        const int u = u0 + r * 32 + lane;\n"
-         "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) "
-      << (pk ? "{ const float v = ok[r] ? sX[b * XS + u * " + std::to_string(N1) + " + m1] : 0.f; xv[r][m1] = make_float2(v, v); }"
-             : "xv[r][m1] = ok[r] ? sX[b * XS + u * " + std::to_string(N1) + " + m1] : 0.f;")
-      << "\n        w[r] = ok[r] ? sW[b * WS + u] : 0.f;\n      }\n";
+         "      " << FT << " xv[1][" << N1 << "];\n      float w[1];\n"
+         "#pragma unroll\n      for (int m1 = 0; m1 < " << N1 << "; ++m1) "
+      << (pk ? "{ const float v = ok ? sX[b * XS + u * " + std::to_string(N1) + " + m1] : 0.f; xv[0][m1] = make_float2(v, v); }"
+             : "xv[0][m1] = ok ? sX[b * XS + u * " + std::to_string(N1) + " + m1] : 0.f;")
+      << "\n      w[0] = ok ? sW[b * WS + u] : 0.f;\n";
     const std::string fp = pk ? "2<" : "<";
     if (K.tangent)
-      o << "      " << FT << " xtv[" << R << "][" << N1 << "];\n      float wt[" << R << "];\n"
+      o << "      " << FT << " xtv[1][" << N1 << "];\n      float wt[1];\n"
            "      const float* sXt = reinterpret_cast<const float*>(st + OFF_XT) + xst;\n"
            "      const float* sWt = reinterpret_cast<const float*>(st + OFF_WT) + wst;\n"
            "      const float* sCt = reinterpret_cast<const float*>(st + OFF_CHT) + choff;\n"
-           "#pragma unroll\n      for (int r = 0; r < " << R << "; ++r) {\n"
-           "        const int u = u0 + r * 32 + lane;\n"
-           "#pragma unroll\n        for (int m1 = 0; m1 < " << N1 << "; ++m1) "
-        << (pk ? "{ const float v = ok[r] ? sXt[b * XS + u * " + std::to_string(N1) + " + m1] : 0.f; xtv[r][m1] = make_float2(v, v); }"
-               : "xtv[r][m1] = ok[r] ? sXt[b * XS + u * " + std::to_string(N1) + " + m1] : 0.f;")
-        << "\n        wt[r] = ok[r] ? sWt[b * WS + u] : 0.f;\n      }\n"
-           "      fpath_tan" << fp << N1 << "," << N3 << "," << R << ",0," << R * NA
-        << ">(acc, sC + b * chs, sCt + b * chs, xv, xtv, w, wt);\n";
+           "#pragma unroll\n      for (int m1 = 0; m1 < " << N1 << "; ++m1) "
+        << (pk ? "{ const float v = ok ? sXt[b * XS + u * " + std::to_string(N1) + " + m1] : 0.f; xtv[0][m1] = make_float2(v, v); }"
+               : "xtv[0][m1] = ok ? sXt[b * XS + u * " + std::to_string(N1) + " + m1] : 0.f;")
+        << "\n      wt[0] = ok ? sWt[b * WS + u] : 0.f;\n"
+           "      fpath_tan" << fp << N1 << "," << N3 << ",1,0," << NA << ">(acc, sC + b * chs, sCt + b * chs, xv, xtv, w, wt);\n";
     else
-      o << "      fpath" << fp << N1 << "," << N3 << "," << R << ",0," << R * NA << ">(acc, sC + b * chs, xv, w);\n";
+      o << "      fpath" << fp << N1 << "," << N3 << ",1,0," << NA << ">(acc, sC + b * chs, xv, w);\n";
     o << "    }\n    __syncwarp();\n    if (lane == 0) mbar_arrive(empty0 + 8 * s);\n  }\n"
-         "#pragma unroll\n  for (int r = 0; r < " << R << "; ++r) if (ok[r]) {\n"
-         "    const int u = u0 + r * 32 + lane;\n"
-         "    float* orow = out + (size_t)i * DOUT + ooff;\n"
+         "  if (ok) {\n    float* orow = out + (size_t)i * DOUT + ooff;\n"
          "#pragma unroll\n    for (int m3 = 0; m3 < " << N3 << "; ++m3) "
       << (K.accumulate ? "red_add(&orow[u * " : "orow[u * ") << N3 << " + m3]" << (K.accumulate ? ", " : " = ")
-      << (pk ? "(m3 & 1) ? acc[r * " + std::to_string(NA) + " + (m3 >> 1)].y : acc[r * " + std::to_string(NA) + " + (m3 >> 1)].x"
-             : "acc[r * " + std::to_string(NA) + " + m3]")
-      << (K.accumulate ? ")" : "") << ";\n  }\n"
+      << (pk ? "(m3 & 1) ? acc[m3 >> 1].y : acc[m3 >> 1].x" : "acc[m3]") << (K.accumulate ? ")" : "") << ";\n  }\n"
          "  }\n  *qp = q;\n}\n";
   }
   gen_fwd_idle(o);
@@ -548,19 +537,14 @@ cgtp_status build_forward(Plan& P) {
   F.generic = wide && NR > 16;
   std::vector<FwdRole> roles;
   if (F.generic) {
-    // channel blocks of 32 per role (tuning override CGTP_FWD_GENERIC_R: 2
-    // blocks share each Chat row load)
-    int gR = 1;
-    if (const char* v = std::getenv("CGTP_FWD_GENERIC_R")) gR = std::max(1, std::min(2, std::atoi(v)));
     for (size_t k = 0; k < P.paths.size(); ++k) {
       const Path& p = P.paths[k];
       const int mul = P.in[p.irrep].mul;
-      for (int u0 = 0; u0 < mul;) {
+      for (int u0 = 0; u0 < mul; u0 += 32) {
         FwdRole r;
         r.irrep = p.irrep;
         r.u0 = u0;
-        r.R = mul - u0 >= 32 * gR ? gR : 1;
-        u0 += 32 * r.R;
+        r.R = 1;
         r.paths = {(int)k};
         r.cost = fwd_role_cost(P, r);
         roles.push_back(r);
