@@ -449,6 +449,19 @@ def run_cgtp(args, rank, world, local_rank):
     log(f"[rank {rank}] plan + workload {name}: N={N} E={E} ({wb.setup_s:.1f}s)")
     stream = wb.stream
     wb.warm(args.warmup)
+    if args.profile == "double_backward":  # for ncu: K double backwards (all three cotangents)
+        gen = torch.Generator(device=dev).manual_seed(3)
+        hx, hW, hY = (torch.randn(t.shape, device=dev, generator=gen) for t in (T["x"], T["W"], wb.Y))
+        grads = tuple(torch.empty_like(t) for t in (T["g"], T["x"], T["W"], wb.Y))
+        dws = torch.empty(max(plan.double_backward_workspace_size(N, N, E), 256), dtype=torch.uint8, device=dev)
+        plan.prepare_double_backward()
+        for _ in range(args.steps):
+            flush.zero_()
+            plan.double_backward(T["rowptr"], T["col"], T["rpt"], T["perm"], T["x"], wb.Y, T["W"], T["g"],
+                                 h_x=hx, h_W=hW, h_Y=hY, grads=grads, workspace=dws)
+        torch.cuda.synchronize()
+        plan.check_device_error()
+        return {"profile": name, "what": "double_backward", "steps": args.steps, "N": N, "E": E}
     if args.profile:  # for ncu: warm-up plus K plain steps, nothing else
         for _ in range(args.steps):
             flush.zero_()
@@ -841,8 +854,9 @@ def main():
                     help="seconds of oracle work for the cpu_baseline field (0 to skip)")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the per-workload figures of the five workloads")
-    ap.add_argument("--profile", action="store_true",
-                    help="warm-up + K steps only (no clock loop, e2e or CPU baseline), for ncu")
+    ap.add_argument("--profile", nargs="?", const="step", default=None, choices=["step", "double_backward"],
+                    help="warm-up + K steps only (no clock loop, e2e or CPU baseline), for ncu; "
+                         "'double_backward': K double backwards with all three cotangents instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
