@@ -560,7 +560,8 @@ cgtp_status build_forward(Plan& P) {
   }
   const int NR2 = (int)P.fwd_roles.size();
   if (F.generic) {
-    const int per = 8;
+    int per = 8;  // roles (consumer warps) per slice
+    if (const char* v = std::getenv("CGTP_FWD_GENERIC_WARPS")) per = std::max(1, std::min(16, std::atoi(v)));
     F.S = (NR2 + per - 1) / per;
     F.slice_roles.assign(F.S, {});
     for (int ri = 0; ri < NR2; ++ri) F.slice_roles[ri / per].push_back(ri);
