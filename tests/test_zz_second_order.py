@@ -59,9 +59,10 @@ def test_double_backward_forward_paths(hid, edge, fwd, dev, monkeypatch):
     _random_graph_case(plan, hid, edge, out, ("h_x", "h_W", "h_Y"), dev)
 
 
-def test_double_backward_first_call_chooses(dev):
+def test_double_backward_first_call_chooses(dev, monkeypatch):
     """With both ways of forming d grad_out built, the first call times them
     and keeps the faster; that call and the next give the same bits."""
+    monkeypatch.delenv("CGTP_DBWD_FWD", raising=False)  # the choice is the plan's
     hid, edge = "32x0e+17x1o+8x2e+33x3o", "1x0e+1x1o+1x2e+1x3o"
     out = _out_irreps(hid, edge)
     from equivariant_mlip_clebsch_b200 import cgtp as C
