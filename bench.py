@@ -38,9 +38,10 @@ from equivariant_mlip_clebsch_b200 import workloads as WL  # noqa: E402
 
 METRIC = "CGTP conv edges/s (fwd, fwd+bwd) on 1 B200; % of HBM/FP32 roofline"
 # the headline workload: the largest that fits one GPU (Table 1 Case 3 on
-# 6,144 atoms); the five workloads of PER_WORKLOAD are measured beside it
+# 6,144 atoms); the workloads of PER_WORKLOAD are measured beside it (the
+# five of the target, then Table 1 Cases 4-6)
 DEFAULT_CONFIG = "lmax3"
-PER_WORKLOAD = ("tiny", "lmax2", "lmax2_wide", "lmax3", "lmax6")
+PER_WORKLOAD = ("tiny", "lmax2", "lmax2_wide", "lmax3", "lmax6", "case4", "case5", "case6")
 L2_FLUSH_BYTES = 512 << 20
 
 
@@ -601,8 +602,9 @@ def run_cgtp(args, rank, world, local_rank):
                virial=virial, double_backward=double_backward, sparse=sparse,
                roofline=roof, fp32_peak=fp32, kernels=kernels, gpu_launches=int(gpu_launches), e2e=e2e,
                clocks=clocks_main)
-    # the five workloads of the target, each measured on its own (the headline
-    # workload's figures are taken again in the same way, for one table)
+    # the five workloads of the target and Table 1 Cases 4-6, each measured on
+    # its own (the headline workload's figures are taken again in the same
+    # way, for one table)
     if not args.no_per_workload:
         per = {}
         k = max(3, min(args.steps, 10))
