@@ -10,6 +10,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <mutex>
 
 #include "internal.hpp"
@@ -405,7 +406,8 @@ __global__ void __launch_bounds__(kFmaThreads) fma_peak_kernel(int64_t iters, fl
   sink[(int64_t)blockIdx.x * kFmaThreads + threadIdx.x] = s;
 }
 
-// The backward's closing reductions in one launch.
+// The backward's closing reductions in one launch (the block form; the warp
+// form, bwd_reduce_rows_kernel, below).
 //  blocks [0, n_send): dx[j][c] = sum over sender j's edges of m[perm_T[t]][c].
 //    Two groups of 128 threads take the even and the odd positions t0 + 2k of
 //    the sender's list, eight rows in flight each; the two partial sums are
@@ -480,6 +482,48 @@ __global__ void __launch_bounds__(kEpiThreads) bwd_reduce_kernel(
       __syncthreads();
     }
   }
+}
+
+// The same reductions with dx taken by warps (rows of a multiple of 4 floats):
+// warp w of blocks [0, dx_blocks) takes sender j = w / nchunk and the float4
+// columns [32 (w % nchunk), +32) of its row, reading the sender's message rows
+// in batches of eight predicated loads and adding them in list order (a lane
+// past the list adds zero), so the result is bitwise reproducible; blocks
+// from dx_blocks on sum the dY slice partials as above.
+__global__ void __launch_bounds__(kEpiThreads) bwd_reduce_rows_kernel(
+    int64_t n_send, int64_t w4, int64_t nchunk, int64_t dx_blocks, const int32_t* __restrict__ rowptr_T,
+    const int32_t* __restrict__ perm_T, const float4* __restrict__ m, float4* __restrict__ dx, int S, int64_t ny,
+    const float* __restrict__ parts, float* __restrict__ dy) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int64_t blk = blockIdx.x;
+  if (blk >= dx_blocks) {
+    const int64_t nblk = (int64_t)gridDim.x - dx_blocks;
+    for (int64_t k = (blk - dx_blocks) * kEpiThreads + threadIdx.x; k < ny; k += nblk * kEpiThreads) {
+      float acc = 0.f;
+      for (int q = 0; q < S; ++q) acc += parts[(int64_t)q * ny + k];
+      dy[k] = acc;
+    }
+    return;
+  }
+  const int64_t item = blk * (kEpiThreads / 32) + (threadIdx.x >> 5);
+  if (item >= n_send * nchunk) return;
+  const int64_t j = item / nchunk;
+  const int64_t c = (item % nchunk) * 32 + (threadIdx.x & 31);
+  if (c >= w4) return;
+  const int t0 = __ldg(rowptr_T + j), t1 = __ldg(rowptr_T + j + 1);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int t = t0; t < t1; t += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t + k < t1) v[k] = __ldcs(m + (int64_t)__ldg(perm_T + t + k) * w4 + c);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) add4(acc, v[k]);
+  }
+  dx[j * w4 + c] = acc;
 }
 
 }  // namespace
@@ -582,6 +626,27 @@ cudaError_t launch_bwd_reduce(int64_t n_send, int64_t width, const int32_t* rowp
   const int64_t nx = (dx && width > 0) ? n_send : 0;
   const int64_t ndy = (dy && S > 1 && ny > 0) ? std::min<int64_t>((ny + kEpiThreads - 1) / kEpiThreads, 148 * 4) : 0;
   if (nx + ndy == 0) return cudaSuccess;
+  // dx by warps when their items fill the GPU (at least 32 warps per SM;
+  // measured on B200: Lmax 3 108.9 -> 102.6 us, Lmax 2 wide 41.4 -> 33.6,
+  // Lmax 6 62.1 -> 59.8; with fewer items, Lmax 2 14.9 -> 16.8, the block
+  // form stays).  CGTP_REDUCE_ROWS=0/1 forces either form.
+  static const int force = [] {
+    const char* v = std::getenv("CGTP_REDUCE_ROWS");
+    return v && (*v == '0' || *v == '1') ? *v - '0' : -1;
+  }();
+  const int64_t w4 = width / 4, nchunk = (w4 + 31) / 32;
+  bool rows = false;
+  if (nx > 0 && width % 4 == 0) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    rows = force >= 0 ? force == 1 : nx * nchunk >= 32 * (int64_t)sms;
+  }
+  if (rows) {
+    const int64_t dx_blocks = (nx * nchunk + kEpiThreads / 32 - 1) / (kEpiThreads / 32);
+    return launch_pdl(bwd_reduce_rows_kernel, dim3((unsigned)(dx_blocks + ndy)), kEpiThreads, s, nx, w4, nchunk,
+                      dx_blocks, rowptr_T, perm_T, reinterpret_cast<const float4*>(m), reinterpret_cast<float4*>(dx),
+                      S, ndy ? ny : (int64_t)0, parts, dy);
+  }
   return launch_pdl(bwd_reduce_kernel, dim3((unsigned)(nx + ndy)), kEpiThreads, s, nx, width, rowptr_T, perm_T, m,
                     nx ? dx : nullptr, S, ndy ? ny : (int64_t)0, parts, dy);
 }
