@@ -381,16 +381,25 @@ cgtp_status cgtp_fma_peak(int64_t iters, float* sink, int64_t sink_floats, cgtp_
 cgtp_status cgtp_double_backward_workspace_size(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
                                                 size_t* bytes);
 
-/* With all three cotangents given, cgtp_double_backward runs two tangent
- * kernels instead of the calls above: the forward and the backward compiled
- * with every W, x and Y piece staged beside its direction (h_W, h_x, h_Y),
- * which give d/dt fwd(x + t h_x, Y + t h_Y, W + t h_W) = gg_out and
+/* With all three cotangents given, cgtp_double_backward replaces the calls
+ * above by one tangent backward, compiled with every W, x and Y piece staged
+ * beside its direction (h_W, h_x, h_Y), which gives
  * d/dt bwd(x + t h_x, Y + t h_Y, W + t h_W; grad_out) = (gx, gW, gY) in one
- * pass each (the same sums as above, every input read once).  They are
- * compiled on the plan's first such call; cgtp_plan_prepare_double_backward
- * compiles them ahead (call it before any stream capture).  *tangent (may be
- * NULL) receives 1 when they are available, 0 when the plan keeps the
- * composition (a tangent stage that does not fit shared memory, or
+ * pass, and forms gg_out = d/dt fwd(x + t h_x, Y + t h_Y, W + t h_W) either
+ * by the tangent forward (one pass, built the same way) or by one plain
+ * forward with h_x plus two passes of an accumulating forward with h_Y and
+ * h_W (the forward is trilinear).  Which of the two is faster depends on the
+ * plan: unless CGTP_DBWD_FWD=tangent|sum at plan creation fixes it, both are
+ * built, and the first such call made outside stream capture runs each once
+ * untimed, times each once, keeps the faster for the plan and runs it last,
+ * so that every call's gg_out comes from the kept form.  That first call
+ * therefore does three times the forward work and waits on the host for its
+ * timing events; under stream capture before that choice, the tangent
+ * forward runs.  The kernels are compiled on the plan's first such call;
+ * cgtp_plan_prepare_double_backward compiles them ahead (call it before any
+ * stream capture).  *tangent (may be NULL) receives 1 when they are
+ * available, 0 when the plan keeps the composition (a tangent backward whose
+ * stages do not fit shared memory at its roles' edge phases, or
  * CGTP_DBWD_COMPOSE set at the first call).  Errors: NULL, CUDA. */
 cgtp_status cgtp_plan_prepare_double_backward(cgtp_plan plan, int* tangent);
 cgtp_status cgtp_double_backward(cgtp_plan plan, int64_t n_recv, int64_t n_send, int64_t E,
